@@ -1,0 +1,331 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks one oracle function against a hand-written fixture, a library
+routine, a closed form, brute force on tiny inputs, or an invariant, so that a
+plausible slip (wrong nibble, wrong bias, dropped bias term, transposed
+operand, wrong tie rule) fails at least one of them.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import _cases as cs
+
+
+# ----------------------------------------------------------------- formats
+def test_e2m1_matches_fixture_table():
+    tab = cs.e2m1_table()
+    got = np.array([oracle.e2m1(c) for c in range(16)])
+    assert np.array_equal(got, tab)
+    assert np.array_equal(np.signbit(got), np.signbit(tab))
+
+
+def test_e8m0_bf16_exponent_field_fixture():
+    for code, bits, value, admitted in cs.read_golden("e8m0_bf16_field.txt"):
+        code = int(code)
+        bits = int(bits, 16)
+        assert bits == code << 7
+        f = synth.bf16_bits_to_f32(np.array([bits], dtype=np.uint16))[0]
+        assert float(f) == float(value)
+        ok = oracle.admit_scales("mxfp4", np.array([code], dtype=np.uint8)) < 0
+        assert ok == (admitted == "yes")
+        if ok:
+            assert oracle.e8m0(code) == float(value)
+
+
+def test_e8m0_all_codes_vs_ldexp():
+    for c in range(1, 255):
+        assert oracle.e8m0(c) == np.ldexp(1.0, c - 127)
+    bad = oracle.admit_scales("mxfp4", np.array([5, 0, 7, 255], dtype=np.uint8))
+    assert bad == 1
+
+
+def test_e4m3_all_codes_vs_torch():
+    torch = pytest.importorskip("torch")
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    # admission: NaN and negative block scales rejected, zero allowed
+    assert oracle.admit_scales("nvfp4", np.array([0, 0x38, 0x7E], dtype=np.uint8)) < 0
+    assert oracle.admit_scales("nvfp4", np.array([0x38, 0x7F], dtype=np.uint8)) == 1
+    assert oracle.admit_scales("nvfp4", np.array([0x38, 0xB8], dtype=np.uint8)) == 1
+
+
+def _one_row_layer(fmt, codes, scales, gscale=1.0):
+    K = codes.size * 2
+    z = np.zeros((1, 1, K // 2), dtype=np.uint8)
+    G = 32 if fmt == "mxfp4" else 16
+    c = [np.zeros((1, K, K // 2), np.uint8), np.zeros((1, K, K // 2), np.uint8),
+         np.zeros((1, K, K // 2), np.uint8)]
+    s = [np.full((1, K, K // G), 127 if fmt == "mxfp4" else 0x38, np.uint8) for _ in range(3)]
+    c[0][0, 0] = codes
+    s[0][0, 0] = scales
+    gl = np.full((1, 3), gscale, np.float32) if fmt == "nvfp4" else None
+    del z
+    return oracle.Layer(K, K, 1, 1, fmt, np.zeros((1, K), np.float32), None, c, s, gl)
+
+
+def test_mxfp4_block_fixture():
+    rows = {r[0]: r[1:] for r in cs.read_golden("mxfp4_block.txt")}
+    codes = np.array([int(b, 16) for b in rows["bytes"]], dtype=np.uint8)
+    want = np.array([float(v) for v in rows["values"]])
+    L = _one_row_layer("mxfp4", codes, np.array([int(rows["scale"][0])], np.uint8))
+    got = L.dequant(0, 0)[0]
+    assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want))
+
+
+def test_nvfp4_block_fixture():
+    rows = {r[0]: r[1:] for r in cs.read_golden("nvfp4_block.txt")}
+    codes = np.array([int(b, 16) for b in rows["bytes"]], dtype=np.uint8)
+    sc = np.array([int(b, 16) for b in rows["scales"]], dtype=np.uint8)
+    want = np.array([float(v) for v in rows["values"]])
+    L = _one_row_layer("nvfp4", codes, sc, float(rows["tensor"][0]))
+    got = L.dequant(0, 0)[0]
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_dequant_matches_numpy_decode(fmt):
+    wl = synth.custom_workload(128, 64, 3, 2, fmt=fmt)
+    lw = synth.make_layer(wl, seed=7)
+    L = oracle.Layer.from_weights(lw)
+    for m in range(3):
+        for e in range(3):
+            gs = 1.0 if lw.global_scale is None else float(lw.global_scale[e, m])
+            ref = cs.np_decode(lw.codes[m][e], lw.scales[m][e], fmt, gs)
+            assert np.array_equal(L.dequant(m, e), ref)
+
+
+# ----------------------------------------------------------------- routing
+def test_router_logits_vs_numpy_matmul():
+    wl = synth.custom_workload(256, 64, 16, 4, zipf_s=1.1)
+    lw = synth.make_layer(wl, seed=3)
+    L = oracle.Layer.from_weights(lw)
+    x = synth.make_tokens(wl, 37, seed=3)
+    lg, _, _ = L.route_all(x)
+    ref = (synth.bf16_bits_to_f32(x).astype(np.float64) @ lw.router_w.astype(np.float64).T
+           + lw.router_bias.astype(np.float64))
+    # both round an fp64 sum to fp32: at most one fp32 ulp apart (summation order)
+    ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(lg.astype(np.float64) - ref) <= ulp)
+
+
+def test_route_vs_argsort_and_full_softmax():
+    rng = np.random.default_rng(11)
+    E, k = 40, 7
+    for _ in range(200):
+        l = rng.standard_normal(E).astype(np.float32)
+        ids, g = oracle.route_row(l, k)
+        ref_ids = np.argsort(-l, kind="stable")[:k]
+        assert np.array_equal(ids, ref_ids)
+        p = np.exp(l.astype(np.float64) - l.max())
+        p /= p.sum()
+        ref_g = p[ref_ids] / p[ref_ids].sum()
+        assert np.allclose(g, ref_g, rtol=2e-7, atol=0)
+        assert abs(float(g.astype(np.float64).sum()) - 1.0) <= 4 * np.finfo(np.float32).eps
+
+
+def test_route_tie_goes_to_lower_index():
+    l = np.array([0.5, 2.0, 1.0, 2.0, 1.0, -3.0], dtype=np.float32)
+    ids, g = oracle.route_row(l, 4)
+    assert ids.tolist() == [1, 3, 2, 4]
+    assert g[0] == g[1] and g[2] == g[3]
+
+
+def test_permute_vs_stable_argsort():
+    rng = np.random.default_rng(5)
+    for T, k, E in [(1, 2, 8), (16, 2, 8), (33, 8, 64), (500, 6, 256)]:
+        ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+        counts, offsets, perm, inv = oracle.permute(ids, E)
+        flat = ids.reshape(-1)
+        assert np.array_equal(counts, np.bincount(flat, minlength=E))
+        assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts)
+        assert offsets[-1] == T * k
+        assert np.array_equal(perm, np.argsort(flat, kind="stable"))
+        assert np.array_equal(inv[perm], np.arange(T * k))
+        assert np.all(np.diff(flat[perm]) >= 0)
+
+
+# ----------------------------------------------------------------- expert FFN / layer
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_single_expert_is_dense_swiglu(fmt):
+    wl = synth.custom_workload(128, 64, 1, 1, fmt=fmt)
+    lw = synth.make_layer(wl, seed=21)
+    L = oracle.Layer.from_weights(lw)
+    x = synth.make_tokens(wl, 5, seed=21)
+    y, _, ids, g = L.forward(x)
+    assert np.all(ids == 0) and np.all(g == 1.0)
+    gs = (1, 1, 1) if lw.global_scale is None else lw.global_scale[0]
+    Wg = cs.np_decode(lw.codes[0][0], lw.scales[0][0], fmt, float(gs[0]))
+    Wu = cs.np_decode(lw.codes[1][0], lw.scales[1][0], fmt, float(gs[1]))
+    Wd = cs.np_decode(lw.codes[2][0], lw.scales[2][0], fmt, float(gs[2]))
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    a = (xf @ Wg.T).astype(np.float32).astype(np.float64)
+    u = (xf @ Wu.T).astype(np.float32).astype(np.float64)
+    h = (cs.np_silu(a) * u).astype(np.float32).astype(np.float64)
+    ref = h @ Wd.T
+    assert np.allclose(y, ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("shape", [
+    dict(hidden=64, inter=32, n_experts=4, top_k=2),
+    dict(hidden=64, inter=32, n_experts=4, top_k=2, fmt="nvfp4"),
+    dict(hidden=64, inter=32, n_experts=5, top_k=3, shared_inter=32),
+    dict(hidden=128, inter=64, n_experts=6, top_k=2, zipf_s=1.1),
+])
+def test_bruteforce_dense_tiny(shape):
+    wl = synth.custom_workload(**shape)
+    lw = synth.make_layer(wl, seed=13)
+    L = oracle.Layer.from_weights(lw)
+    x, _ = cs.tokens_with_margin(L, wl, 3, seed=13)
+    y, lg, ids, g = L.forward(x)
+    ry, rlg, rids, rg = cs.dense_layer(lw, x)
+    assert np.array_equal(ids, rids)
+    ulp = np.spacing(np.abs(rlg)).astype(np.float64)
+    assert np.all(np.abs(lg.astype(np.float64) - rlg) <= ulp)
+    assert np.allclose(g, rg, rtol=4e-7, atol=0)
+    assert np.allclose(y, ry, rtol=1e-6, atol=1e-6 * np.abs(ry).max())
+
+
+def test_bruteforce_dense_tiny_workload():
+    wl = synth.workload("tiny")
+    lw = synth.make_layer(wl)
+    L = oracle.Layer.from_weights(lw)
+    x, _ = cs.tokens_with_margin(L, wl, 16)
+    y, lg, ids, g = L.forward(x)
+    ry, rlg, rids, rg = cs.dense_layer(lw, x)
+    assert np.array_equal(ids, rids)
+    assert np.allclose(y, ry, rtol=1e-6, atol=1e-6 * np.abs(ry).max())
+    assert np.allclose(g.sum(axis=1), 1.0, atol=4 * np.finfo(np.float32).eps)
+
+
+def test_token_permutation_equivariance_and_subset():
+    wl = synth.custom_workload(128, 64, 8, 3, shared_inter=64)
+    lw = synth.make_layer(wl, seed=2)
+    L = oracle.Layer.from_weights(lw)
+    x = synth.make_tokens(wl, 9, seed=2)
+    y, lg, ids, g = L.forward(x)
+    pi = np.random.default_rng(0).permutation(9)
+    y2, lg2, ids2, g2 = L.forward(x[pi])
+    assert np.array_equal(y2, y[pi]) and np.array_equal(ids2, ids[pi]) and np.array_equal(g2, g[pi])
+    rows = np.array([4, 0, 8], dtype=np.int32)
+    y3, _, ids3, _ = L.forward(x, rows=rows)
+    assert np.array_equal(y3, y[rows]) and np.array_equal(ids3, ids[rows])
+
+
+def test_output_is_linear_in_down_projection_sign():
+    """Flipping the sign bit of every down-projection code negates the routed output."""
+    wl = synth.custom_workload(64, 32, 4, 2)
+    lw = synth.make_layer(wl, seed=4)
+    x = synth.make_tokens(wl, 4, seed=4)
+    y, *_ = oracle.Layer.from_weights(lw).forward(x)
+    lw.codes[2] = lw.codes[2] ^ np.uint8(0x88)
+    y2, *_ = oracle.Layer.from_weights(lw).forward(x)
+    assert np.array_equal(y2, -y)
+
+
+# ----------------------------------------------------------------- A4 quantisers
+def test_rne_e2m1_properties():
+    tab = cs.e2m1_table()
+    mags = tab[:8]
+    # exact values map to themselves
+    for c in range(16):
+        if c == 8:
+            continue
+        assert oracle.rne_e2m1(float(tab[c])) == c
+    # ties go to the even mantissa bit (codes 0, 2, 4, 6 are even)
+    ties = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for v, want in ties.items():
+        assert tab[oracle.rne_e2m1(v)] == want
+        assert tab[oracle.rne_e2m1(-v)] == -want
+    # saturation
+    assert tab[oracle.rne_e2m1(7.0)] == 6.0 and tab[oracle.rne_e2m1(1e30)] == 6.0
+    assert tab[oracle.rne_e2m1(-100.0)] == -6.0
+    # nearest: no representable value is strictly closer
+    rng = np.random.default_rng(1)
+    for v in rng.uniform(-7, 7, 2000).astype(np.float32):
+        q = tab[oracle.rne_e2m1(float(v))]
+        d = abs(abs(float(v)) - np.abs(mags))
+        assert abs(abs(float(v)) - abs(q)) <= d.min() + 0.0
+        assert np.sign(q) in (0.0, np.sign(v))
+
+
+def test_rn_e4m3_vs_torch():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(2)
+    v = np.concatenate([rng.uniform(0, 448, 3000), np.exp(rng.uniform(-14, 6, 3000)),
+                        [0.0, 448.0, 2.0 ** -9, 1.0625, 1.1875, 0.0009765625 * 1.5]]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.rn_e4m3(float(t)) for t in v], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_quant_mx_block_hand_built():
+    tab = cs.e2m1_table()
+    for n in (-3, 0, 5):
+        v = np.zeros(32, np.float32)
+        v[3] = 6.0 * 2.0 ** n
+        v[7] = -1.5 * 2.0 ** n
+        codes, sc = oracle.quant_mx_block(v)
+        assert sc == 127 + n
+        deq = tab[codes] * 2.0 ** (sc - 127)
+        assert np.array_equal(deq, v.astype(np.float64))
+        v2 = v.copy()
+        v2[3] = 8.0 * 2.0 ** n          # amax 8*2^n: exponent n+1, 8 -> 4
+        codes, sc = oracle.quant_mx_block(v2)
+        assert sc == 128 + n and tab[codes[3]] == 4.0
+        v3 = v.copy()
+        v3[3] = 7.0 * 2.0 ** n          # amax 7*2^n: exponent n, 7 saturates to 6
+        codes, sc = oracle.quant_mx_block(v3)
+        assert sc == 127 + n and tab[codes[3]] == 6.0
+    codes, sc = oracle.quant_mx_block(np.zeros(32, np.float32))
+    assert sc == 1 and np.all(tab[codes] == 0)
+
+
+def test_quant_nv_row_hand_built():
+    tab = cs.e2m1_table()
+    v = np.zeros(32, np.float32)
+    v[0] = 2688.0            # amax = 6*448: G = 1, scale 448
+    v[16] = 3.0              # block 1: scale RN(0.5) = 0.5, code 6
+    codes, sc, G = oracle.quant_nv_row(v)
+    assert G == 1.0
+    assert oracle.e4m3(int(sc[0])) == 448.0 and tab[codes[0]] == 6.0
+    assert oracle.e4m3(int(sc[1])) == 0.5 and tab[codes[16]] == 6.0
+    codes, sc, G = oracle.quant_nv_row(v * np.float32(4.0))
+    assert G == 4.0
+    codes, sc, G = oracle.quant_nv_row(v * np.float32(1.001))
+    assert G == 2.0
+    codes, sc, G = oracle.quant_nv_row(np.zeros(32, np.float32))
+    assert G == 1.0 and np.all(sc == 0) and np.all(codes == 0)
+
+
+def test_a4_mode_single_expert_matches_quantised_dense():
+    wl = synth.custom_workload(128, 64, 1, 1)
+    lw = synth.make_layer(wl, seed=8)
+    L = oracle.Layer.from_weights(lw, numerics="a4")
+    x = synth.make_tokens(wl, 3, seed=8)
+    y, *_ = L.forward(x)
+    tab = cs.e2m1_table()
+
+    def qdq(row):
+        out = np.empty(row.size)
+        for b in range(row.size // 32):
+            c, s = oracle.quant_mx_block(row[b * 32:(b + 1) * 32].astype(np.float32))
+            out[b * 32:(b + 1) * 32] = tab[c] * 2.0 ** (s - 127)
+        return out
+
+    Wg = cs.np_decode(lw.codes[0][0], lw.scales[0][0], "mxfp4")
+    Wu = cs.np_decode(lw.codes[1][0], lw.scales[1][0], "mxfp4")
+    Wd = cs.np_decode(lw.codes[2][0], lw.scales[2][0], "mxfp4")
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    for t in range(3):
+        xq = qdq(xf[t])
+        a = np.float32(Wg @ xq).astype(np.float64)
+        u = np.float32(Wu @ xq).astype(np.float64)
+        h = (cs.np_silu(a) * u).astype(np.float32)
+        ref = Wd @ qdq(h)
+        assert np.allclose(y[t], ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
