@@ -1,0 +1,781 @@
+// api.cu -- C ABI and host runtime of the MoE layer: admission, pinned expert
+// store in device layout, resident slots, staging ring for misses, forward
+// orchestration.
+//
+// Paging follows the pages' memory hierarchy: every expert pinned in host RAM,
+// a budget of hot experts resident on the GPU, the router and shared experts
+// always resident ("Strata, Explained", section 2; strata.amperor.ai, the
+// "budget ... resident experts/layer" option).  The device layout is packed
+// once, at create time, into the pinned store, so a miss costs one plain
+// cudaMemcpyAsync ("ro99/strata": a per-staging prepack lands on the
+// bottleneck term).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "moe_internal.h"
+
+using namespace moe;
+
+static thread_local std::string g_err;
+static int g_inject_create = 0;
+
+static moe_status_t fail(moe_status_t s, const std::string &msg) {
+  g_err = msg;
+  return s;
+}
+
+#define CUDA_TRY(call)                                                                   \
+  do {                                                                                   \
+    cudaError_t _e = (call);                                                             \
+    if (_e != cudaSuccess) {                                                             \
+      return fail(MOE_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(_e));     \
+    }                                                                                    \
+  } while (0)
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+BlobLayout moe::blob_layout(int H, int I, int fmt) {
+  BlobLayout L{};
+  L.fmt = fmt;
+  L.G = fmt == MOE_FMT_MXFP4 ? 32 : 16;
+  size_t off = 0;
+  for (int m = 0; m < 3; ++m) {
+    L.rows[m] = (m < 2) ? I : H;
+    L.K[m] = (m < 2) ? H : I;
+    L.codes[m] = off;
+    off = align256(off + (size_t)L.rows[m] * L.K[m] / 2);
+  }
+  for (int m = 0; m < 3; ++m) {
+    L.scales[m] = off;
+    off = align256(off + (size_t)L.rows[m] * L.K[m] / L.G);
+  }
+  if (fmt == MOE_FMT_MXFP4) {
+    for (int m = 0; m < 3; ++m) {
+      L.sref[m] = off;
+      off = align256(off + (size_t)L.rows[m]);
+    }
+    L.glob = 0;
+  } else {
+    for (int m = 0; m < 3; ++m) L.sref[m] = 0;
+    L.glob = off;
+    off = align256(off + 3 * sizeof(float));
+  }
+  L.bytes = off;
+  return L;
+}
+
+struct moe_layer {
+  moe_config_t cfg{};
+  BlobLayout L{};
+  int wf = 0;
+  int n_staging = 0;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_copied[2] = {}, ev_done[2] = {}, ev_counts = nullptr, ev_fwd_done = nullptr;
+  // device memory
+  std::vector<void *> dev;
+  float *router_w = nullptr, *router_b = nullptr;
+  uint16_t *shared_w[3] = {};
+  uint8_t *slots = nullptr, *staging = nullptr;
+  const uint8_t **ptr_resident = nullptr, **ptr_pass = nullptr;
+  float *logits = nullptr, *gates = nullptr;
+  int *ids = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr;
+  TileInfo *tiles = nullptr;
+  int *n_tiles = nullptr, *active = nullptr, *prow_token = nullptr, *prow_pair = nullptr;
+  uint16_t *xf16 = nullptr, *hbuf = nullptr, *sh_h = nullptr, *xin = nullptr;
+  float *xs = nullptr, *hscale = nullptr, *oprime = nullptr, *sh_s = nullptr, *yout = nullptr;
+  int *router_counter = nullptr;
+  // host
+  uint8_t *store = nullptr;          // pinned: E x blob bytes
+  int *h_counts = nullptr;           // pinned [E]
+  const uint8_t **h_ptr = nullptr;   // pinned [E]
+  std::vector<int> slot_of;
+  int n_resident = 0;
+  size_t max_prows = 0, max_tiles = 0;
+  moe_stats_t st{};
+  int inject = 0;
+  bool staging_used = false;
+  // tracing: CUDA event pairs per stage, read back by moe_profile_read
+  struct Pending {
+    int stage;
+    cudaEvent_t a, b;
+  };
+  bool prof = false;
+  std::vector<Pending> pend;
+  std::vector<cudaEvent_t> evpool;
+  moe_profile_t prof_acc{};
+};
+
+static cudaEvent_t take_event(moe_layer *L) {
+  if (!L->evpool.empty()) {
+    cudaEvent_t e = L->evpool.back();
+    L->evpool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+// Records an event pair around one stage of a forward when tracing is on, and
+// counts the stage's kernel launches.
+struct StageTimer {
+  moe_layer *L;
+  int stage;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  StageTimer(moe_layer *L_, int st, cudaStream_t s_) : L(L_), stage(st), s(s_) {
+    if (L->prof && (a = take_event(L))) cudaEventRecord(a, s);
+  }
+  void launched(int n) {
+    L->st.launches += n;
+    L->prof_acc.launches[stage] += n;
+  }
+  void end() {
+    if (!a) return;
+    cudaEvent_t b = take_event(L);
+    if (!b) {
+      L->evpool.push_back(a);
+      a = nullptr;
+      return;
+    }
+    cudaEventRecord(b, s);
+    L->pend.push_back({stage, a, b});
+    a = nullptr;
+  }
+};
+
+// ------------------------------------------------------------------ helpers
+static moe_status_t check_config(const moe_config_t *c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
+  if (c->hidden <= 0 || c->hidden % 256) return fail(MOE_ERR_INVALID_ARG, "hidden must be a positive multiple of 256");
+  if (c->inter <= 0 || c->inter % 128) return fail(MOE_ERR_INVALID_ARG, "inter must be a positive multiple of 128");
+  if (c->n_experts < 1 || c->n_experts > kMaxExperts) return fail(MOE_ERR_INVALID_ARG, "n_experts must be in 1..1024");
+  if (c->top_k < 1 || c->top_k > std::min(c->n_experts, kMaxTopK))
+    return fail(MOE_ERR_INVALID_ARG, "top_k must be in 1..min(n_experts, 32)");
+  if (c->shared_inter < 0 || c->shared_inter % 128) return fail(MOE_ERR_INVALID_ARG, "shared_inter must be 0 or a multiple of 128");
+  if (c->fmt != MOE_FMT_MXFP4 && c->fmt != MOE_FMT_NVFP4) return fail(MOE_ERR_INVALID_ARG, "fmt must be MXFP4 or NVFP4");
+  if (c->renormalize != 1) return fail(MOE_ERR_UNSUPPORTED, "only renormalised top-k gates are implemented (renormalize = 1)");
+  if (c->numerics != MOE_NUMERICS_EXACT && c->numerics != MOE_NUMERICS_A4)
+    return fail(MOE_ERR_INVALID_ARG, "numerics must be EXACT or A4");
+  if (c->numerics == MOE_NUMERICS_A4)
+    return fail(MOE_ERR_UNSUPPORTED, "A4 numerics is not available in this build");
+  if (c->n_slots < 0 || c->n_slots > c->n_experts) return fail(MOE_ERR_INVALID_ARG, "n_slots must be in 0..n_experts");
+  if (c->max_tokens < 1 || (int64_t)c->max_tokens * c->top_k > (1 << 30))
+    return fail(MOE_ERR_INVALID_ARG, "max_tokens must be >= 1 and max_tokens * top_k <= 2^30");
+  if (c->n_staging < 0 || c->n_staging > 2 * kPtrListMax) return fail(MOE_ERR_INVALID_ARG, "n_staging must be in 0..512");
+  if (c->n_slots < c->n_experts && c->n_staging == 1) return fail(MOE_ERR_INVALID_ARG, "n_staging must be >= 2 when n_slots < n_experts");
+  return MOE_OK;
+}
+
+static int default_staging(const moe_config_t *c) {
+  if (c->n_slots >= c->n_experts) return 0;
+  if (c->n_staging > 0) return c->n_staging;
+  return std::max(2, std::min(c->n_experts - c->n_slots, 64));
+}
+
+struct Sizes {
+  size_t P, max_prows, max_tiles;
+};
+static Sizes sizes_of(const moe_config_t *c) {
+  Sizes s;
+  s.P = (size_t)c->max_tokens * c->top_k;
+  const size_t act = std::min<size_t>(c->n_experts, s.P);
+  s.max_prows = s.P + 8 * act;
+  s.max_tiles = s.P / 8 + act + 1;
+  return s;
+}
+
+static size_t scratch_bytes(const moe_config_t *c) {
+  const Sizes z = sizes_of(c);
+  const size_t T = c->max_tokens, H = c->hidden, I = c->inter, E = c->n_experts, Is = c->shared_inter;
+  size_t b = 0;
+  b += align256(T * E * 4) + align256(z.P * 4) * 4 + align256(E * 4) + align256((E + 1) * 4);
+  b += align256(z.max_tiles * sizeof(TileInfo)) + 2 * align256(4) + 2 * align256(z.max_prows * 4);
+  b += align256(T * H * 2) + align256(T * (H / kChunk) * 4);
+  b += align256(z.max_prows * I * 2) + align256(z.max_prows * (I / kChunk) * 4);
+  b += align256(z.P * H * 4);
+  if (Is) b += align256(T * Is * 2) + align256(T * H * 4);
+  b += align256(((T + 3) / 4) * 4);
+  b += align256(T * H * 2) + align256(T * H * 4);
+  b += 2 * align256(E * sizeof(void *));
+  return b;
+}
+
+template <typename P>
+static moe_status_t dalloc(moe_layer *L, P **p, size_t bytes) {
+  if (g_inject_create == 2) {
+    g_inject_create = 0;
+    return fail(MOE_ERR_OOM, "injected device allocation failure");
+  }
+  void *q = nullptr;
+  cudaError_t e = cudaMalloc(&q, std::max<size_t>(bytes, 256));
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(MOE_ERR_OOM, std::string("cudaMalloc failed: ") + cudaGetErrorString(e));
+  }
+  L->dev.push_back(q);
+  *p = reinterpret_cast<P *>(q);
+  return MOE_OK;
+}
+
+#define ST_TRY(x)                 \
+  do {                            \
+    moe_status_t _s = (x);        \
+    if (_s != MOE_OK) return _s;  \
+  } while (0)
+
+static void free_layer(moe_layer *L) {
+  if (!L) return;
+  cudaSetDevice(L->cfg.device);
+  cudaDeviceSynchronize();
+  for (void *p : L->dev) cudaFree(p);
+  if (L->store) cudaFreeHost(L->store);
+  if (L->h_counts) cudaFreeHost(L->h_counts);
+  if (L->h_ptr) cudaFreeHost(L->h_ptr);
+  for (int i = 0; i < 2; ++i) {
+    if (L->ev_copied[i]) cudaEventDestroy(L->ev_copied[i]);
+    if (L->ev_done[i]) cudaEventDestroy(L->ev_done[i]);
+  }
+  if (L->ev_counts) cudaEventDestroy(L->ev_counts);
+  if (L->ev_fwd_done) cudaEventDestroy(L->ev_fwd_done);
+  for (auto &p : L->pend) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
+  for (auto e : L->evpool) cudaEventDestroy(e);
+  if (L->side) cudaStreamDestroy(L->side);
+  delete L;
+}
+
+// ------------------------------------------------------------------ C ABI
+extern "C" {
+
+const char *moe_last_error(void) { return g_err.c_str(); }
+
+moe_status_t moe_layer_plan(const moe_config_t *cfg, moe_plan_t *out) {
+  ST_TRY(check_config(cfg));
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  const BlobLayout L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt);
+  out->expert_bytes = L.bytes;
+  out->slot_bytes = (uint64_t)L.bytes * cfg->n_slots;
+  out->staging_bytes = (uint64_t)L.bytes * default_staging(cfg);
+  out->resident_bytes = (uint64_t)cfg->n_experts * cfg->hidden * 4 + cfg->n_experts * 4 +
+                        (uint64_t)3 * cfg->shared_inter * cfg->hidden * 2;
+  out->scratch_bytes = scratch_bytes(cfg);
+  out->pinned_bytes = (uint64_t)L.bytes * cfg->n_experts;
+  return MOE_OK;
+}
+
+moe_status_t moe_admit(const moe_config_t *cfg, const moe_weights_t *w) {
+  ST_TRY(check_config(cfg));
+  if (!w || !w->router_w) return fail(MOE_ERR_INVALID_ARG, "weights or router_w is NULL");
+  const BlobLayout L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt);
+  for (int m = 0; m < 3; ++m)
+    if (!w->codes[m] || !w->scales[m]) return fail(MOE_ERR_INVALID_ARG, "codes/scales table is NULL");
+  if (cfg->shared_inter > 0 && (!w->shared_w[0] || !w->shared_w[1] || !w->shared_w[2]))
+    return fail(MOE_ERR_INVALID_ARG, "shared expert weights are NULL");
+  if (cfg->fmt == MOE_FMT_NVFP4 && !w->global_scale)
+    return fail(MOE_ERR_INVALID_ARG, "NVFP4 needs global_scale [E,3]");
+  for (int e = 0; e < cfg->n_experts; ++e) {
+    for (int m = 0; m < 3; ++m) {
+      const uint8_t *s = w->scales[m][e];
+      if (!s || !w->codes[m][e]) return fail(MOE_ERR_INVALID_ARG, "NULL expert pointer");
+      const size_t n = (size_t)L.rows[m] * L.K[m] / L.G;
+      for (size_t i = 0; i < n; ++i) {
+        const unsigned c = s[i];
+        const bool bad = cfg->fmt == MOE_FMT_MXFP4 ? (c == 0u || c == 255u)
+                                                   : ((c & 0x7Fu) == 0x7Fu || (c & 0x80u));
+        if (bad) {
+          char buf[160];
+          snprintf(buf, sizeof buf, "scale admission failed: expert %d matrix %d index %zu code %u", e, m, i, c);
+          return fail(MOE_ERR_ADMISSION, buf);
+        }
+      }
+      if (cfg->fmt == MOE_FMT_NVFP4) {
+        const float gsc = w->global_scale[e * 3 + m];
+        if (!(gsc > 0.0f) || gsc == INFINITY) {
+          char buf[128];
+          snprintf(buf, sizeof buf, "scale admission failed: per-tensor scale of expert %d matrix %d", e, m);
+          return fail(MOE_ERR_ADMISSION, buf);
+        }
+      }
+    }
+  }
+  return MOE_OK;
+}
+
+static void pack_expert(const moe_config_t *cfg, const BlobLayout &L, const moe_weights_t *w, int e,
+                        uint8_t *dst) {
+  for (int m = 0; m < 3; ++m) {
+    const size_t ncode = (size_t)L.rows[m] * L.K[m] / 2;
+    const size_t nsc = (size_t)L.rows[m] * L.K[m] / L.G;
+    memcpy(dst + L.codes[m], w->codes[m][e], ncode);
+    memcpy(dst + L.scales[m], w->scales[m][e], nsc);
+    if (cfg->fmt == MOE_FMT_MXFP4) {
+      const int per = L.K[m] / L.G;
+      const uint8_t *s = w->scales[m][e];
+      for (int r = 0; r < L.rows[m]; ++r) {
+        uint8_t mx = 1;
+        for (int i = 0; i < per; ++i) mx = std::max(mx, s[(size_t)r * per + i]);
+        dst[L.sref[m] + r] = mx;
+      }
+    }
+  }
+  if (cfg->fmt == MOE_FMT_NVFP4) {
+    float g[3] = {w->global_scale[e * 3 + 0], w->global_scale[e * 3 + 1], w->global_scale[e * 3 + 2]};
+    memcpy(dst + L.glob, g, sizeof g);
+  }
+}
+
+moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, void *stream,
+                              moe_layer_t *out) {
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  ST_TRY(moe_admit(cfg, w));
+  CUDA_TRY(cudaSetDevice(cfg->device));
+  cudaStream_t s = (cudaStream_t)stream;
+  moe_layer *L = new moe_layer();
+  L->cfg = *cfg;
+  L->L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt);
+  L->wf = cfg->fmt == MOE_FMT_MXFP4 ? WF_MX : WF_NV;
+  L->n_staging = default_staging(cfg);
+  L->cfg.n_staging = L->n_staging;
+  const int E = cfg->n_experts, H = cfg->hidden, I = cfg->inter, Is = cfg->shared_inter;
+  const Sizes z = sizes_of(cfg);
+  L->max_prows = z.max_prows;
+  L->max_tiles = z.max_tiles;
+  const size_t T = cfg->max_tokens;
+  auto bail = [&](moe_status_t st) {
+    free_layer(L);
+    return st;
+  };
+#define C_TRY(x)                                \
+  do {                                          \
+    moe_status_t _s = (x);                      \
+    if (_s != MOE_OK) return bail(_s);          \
+  } while (0)
+#define C_CUDA(call)                                                                           \
+  do {                                                                                         \
+    cudaError_t _e = (call);                                                                   \
+    if (_e != cudaSuccess) {                                                                   \
+      return bail(fail(MOE_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(_e)));     \
+    }                                                                                          \
+  } while (0)
+
+  // pinned store in device layout
+  const size_t bytes = L->L.bytes;
+  if (cudaHostAlloc((void **)&L->store, bytes * E, cudaHostAllocDefault) != cudaSuccess) {
+    (void)cudaGetLastError();
+    L->store = nullptr;
+    return bail(fail(MOE_ERR_OOM, "pinned host store allocation failed"));
+  }
+  {
+    const int nth = std::max(1, std::min<int>(8, (int)std::thread::hardware_concurrency()));
+    std::vector<std::thread> th;
+    for (int t = 0; t < nth; ++t)
+      th.emplace_back([&, t] {
+        for (int e = t; e < E; e += nth) pack_expert(cfg, L->L, w, e, L->store + (size_t)e * bytes);
+      });
+    for (auto &x : th) x.join();
+  }
+  if (cudaHostAlloc((void **)&L->h_counts, sizeof(int) * E, cudaHostAllocDefault) != cudaSuccess ||
+      cudaHostAlloc((void **)&L->h_ptr, sizeof(void *) * E, cudaHostAllocDefault) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return bail(fail(MOE_ERR_OOM, "pinned host allocation failed"));
+  }
+
+  // device memory
+  C_TRY(dalloc(L, &L->router_w, (size_t)E * H * 4));
+  if (w->router_bias) C_TRY(dalloc(L, &L->router_b, (size_t)E * 4));
+  if (Is) for (int m = 0; m < 3; ++m) C_TRY(dalloc(L, &L->shared_w[m], (size_t)Is * H * 2));
+  if (cfg->n_slots) C_TRY(dalloc(L, &L->slots, bytes * cfg->n_slots));
+  if (L->n_staging) C_TRY(dalloc(L, &L->staging, bytes * L->n_staging));
+  C_TRY(dalloc(L, &L->ptr_resident, sizeof(void *) * E));
+  C_TRY(dalloc(L, &L->ptr_pass, sizeof(void *) * E));
+  C_TRY(dalloc(L, &L->logits, T * E * 4));
+  C_TRY(dalloc(L, &L->ids, z.P * 4));
+  C_TRY(dalloc(L, &L->gates, z.P * 4));
+  C_TRY(dalloc(L, &L->perm, z.P * 4));
+  C_TRY(dalloc(L, &L->inv, z.P * 4));
+  C_TRY(dalloc(L, &L->counts, (size_t)E * 4));
+  C_TRY(dalloc(L, &L->offsets, (size_t)(E + 1) * 4));
+  C_TRY(dalloc(L, &L->tiles, z.max_tiles * sizeof(TileInfo)));
+  C_TRY(dalloc(L, &L->n_tiles, 4));
+  C_TRY(dalloc(L, &L->active, 4));
+  C_TRY(dalloc(L, &L->prow_token, z.max_prows * 4));
+  C_TRY(dalloc(L, &L->prow_pair, z.max_prows * 4));
+  C_TRY(dalloc(L, &L->xf16, T * H * 2));
+  C_TRY(dalloc(L, &L->xs, T * (H / kChunk) * 4));
+  C_TRY(dalloc(L, &L->hbuf, z.max_prows * I * 2));
+  C_TRY(dalloc(L, &L->hscale, z.max_prows * (I / kChunk) * 4));
+  C_TRY(dalloc(L, &L->oprime, z.P * H * 4));
+  if (Is) {
+    C_TRY(dalloc(L, &L->sh_h, T * Is * 2));
+    C_TRY(dalloc(L, &L->sh_s, T * H * 4));
+  }
+  C_TRY(dalloc(L, &L->router_counter, ((T + 3) / 4) * 4));
+  C_TRY(dalloc(L, &L->xin, T * H * 2));
+  C_TRY(dalloc(L, &L->yout, T * H * 4));
+
+  C_CUDA(cudaMemsetAsync(L->router_counter, 0, ((T + 3) / 4) * 4, s));
+  C_CUDA(cudaMemsetAsync(L->ptr_resident, 0, sizeof(void *) * E, s));
+  C_CUDA(cudaMemsetAsync(L->ptr_pass, 0, sizeof(void *) * E, s));
+  C_CUDA(cudaMemcpyAsync(L->router_w, w->router_w, (size_t)E * H * 4, cudaMemcpyHostToDevice, s));
+  if (w->router_bias) C_CUDA(cudaMemcpyAsync(L->router_b, w->router_bias, (size_t)E * 4, cudaMemcpyHostToDevice, s));
+  if (Is)
+    for (int m = 0; m < 3; ++m)
+      C_CUDA(cudaMemcpyAsync(L->shared_w[m], w->shared_w[m], (size_t)Is * H * 2, cudaMemcpyHostToDevice, s));
+  C_CUDA(cudaStreamSynchronize(s));
+
+  C_CUDA(cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking));
+  for (int i = 0; i < 2; ++i) {
+    C_CUDA(cudaEventCreateWithFlags(&L->ev_copied[i], cudaEventDisableTiming));
+    C_CUDA(cudaEventCreateWithFlags(&L->ev_done[i], cudaEventDisableTiming));
+  }
+  C_CUDA(cudaEventCreateWithFlags(&L->ev_counts, cudaEventDisableTiming));
+  C_CUDA(cudaEventCreateWithFlags(&L->ev_fwd_done, cudaEventDisableTiming));
+  L->slot_of.assign(E, -1);
+  for (int e = 0; e < E; ++e) L->h_ptr[e] = nullptr;
+  L->st.expert_bytes = bytes;
+  L->st.pinned_bytes = bytes * E;
+  size_t dev_total = (size_t)E * H * 4 + (size_t)3 * Is * H * 2 + bytes * (cfg->n_slots + L->n_staging) +
+                     scratch_bytes(cfg);
+  L->st.device_bytes = dev_total;
+  *out = L;
+  return MOE_OK;
+#undef C_TRY
+#undef C_CUDA
+}
+
+moe_status_t moe_set_slot_table(moe_layer_t L, const int32_t *table, void *stream) {
+  if (!L || !table) return fail(MOE_ERR_INVALID_ARG, "layer or table is NULL");
+  const int E = L->cfg.n_experts, S = L->cfg.n_slots;
+  std::vector<int> used(S > 0 ? S : 1, -1);
+  int n = 0;
+  for (int e = 0; e < E; ++e) {
+    const int s = table[e];
+    if (s == -1) continue;
+    if (s < 0 || s >= S) {
+      char buf[96];
+      snprintf(buf, sizeof buf, "slot %d of expert %d is out of range [0, %d)", s, e, S);
+      return fail(MOE_ERR_SLOT_TABLE, buf);
+    }
+    if (used[s] >= 0) {
+      char buf[96];
+      snprintf(buf, sizeof buf, "slot %d given to experts %d and %d", s, used[s], e);
+      return fail(MOE_ERR_SLOT_TABLE, buf);
+    }
+    used[s] = e;
+    ++n;
+  }
+  if (n > S) return fail(MOE_ERR_SLOT_TABLE, "more resident experts than slots");
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  cudaStream_t st = (cudaStream_t)stream;
+  CUDA_TRY(cudaStreamSynchronize(st));
+  CUDA_TRY(cudaStreamSynchronize(L->side));
+  const size_t bytes = L->L.bytes;
+  for (int e = 0; e < E; ++e) {
+    const int s = table[e];
+    if (s >= 0 && L->slot_of[e] != s)
+      CUDA_TRY(cudaMemcpyAsync(L->slots + (size_t)s * bytes, L->store + (size_t)e * bytes, bytes,
+                               cudaMemcpyHostToDevice, st));
+    L->h_ptr[e] = s >= 0 ? L->slots + (size_t)s * bytes : nullptr;
+  }
+  CUDA_TRY(cudaMemcpyAsync(L->ptr_resident, L->h_ptr, sizeof(void *) * E, cudaMemcpyHostToDevice, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  for (int e = 0; e < E; ++e) L->slot_of[e] = table[e];
+  L->n_resident = n;
+  return MOE_OK;
+}
+
+static int pick_split(int est_ctas, int nck) {
+  int cs = 1;
+  while (cs < 8 && nck % (cs * 2) == 0 && est_ctas * cs < 2 * 148) cs *= 2;
+  return cs;
+}
+
+static moe_status_t run_experts(moe_layer *L, const uint8_t *const *ptrs, int nt, int grid_tiles,
+                                int cs_gu, int cs_dn, cudaStream_t s) {
+  const moe_config_t &c = L->cfg;
+  ExpertArgs a{};
+  a.expert_ptr = ptrs;
+  a.L = L->L;
+  a.tile_tokens = 8 * nt;
+  a.tiles = L->tiles;
+  a.n_tiles = L->n_tiles;
+  a.prow_token = L->prow_token;
+  a.prow_pair = L->prow_pair;
+  a.gates = L->gates;
+  // gate/up + SwiGLU
+  a.K = c.hidden;
+  a.rows = c.inter;
+  a.n_rowblocks = c.inter / 128;
+  a.k_split = cs_gu;
+  a.act = L->xf16;
+  a.act_scale = L->xs;
+  a.h_out = L->hbuf;
+  a.h_scale = L->hscale;
+  StageTimer t3(L, 3, s);
+  launch_expert(L->wf, MODE_GATEUP, nt, a, grid_tiles, s);
+  CUDA_TRY(cudaGetLastError());
+  t3.launched(1);
+  t3.end();
+  // down + gate scale -> O'
+  a.K = c.inter;
+  a.rows = c.hidden;
+  a.n_rowblocks = c.hidden / 256;
+  a.k_split = cs_dn;
+  a.act = L->hbuf;
+  a.act_scale = L->hscale;
+  a.o_out = L->oprime;
+  StageTimer t4(L, 4, s);
+  launch_expert(L->wf, MODE_DOWN, nt, a, grid_tiles, s);
+  CUDA_TRY(cudaGetLastError());
+  t4.launched(1);
+  t4.end();
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void *stream,
+                         const moe_routing_t *dbg) {
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  const moe_config_t &c = L->cfg;
+  if (T < 0 || T > c.max_tokens) return fail(MOE_ERR_INVALID_ARG, "T out of range [0, max_tokens]");
+  if (T == 0) return MOE_OK;
+  if (!x || !y) return fail(MOE_ERR_INVALID_ARG, "x or y is NULL");
+  CUDA_TRY(cudaSetDevice(c.device));
+  cudaStream_t s = (cudaStream_t)stream;
+  const int E = c.n_experts, k = c.top_k, H = c.hidden, I = c.inter, Is = c.shared_inter;
+  const int P = T * k;
+  const int act_est = std::min(E, P);
+  const int avg = (P + act_est - 1) / act_est;
+  const int nt = avg <= 8 ? 1 : (avg <= 16 ? 2 : 4);
+  const int ts = 8 * nt;
+  const int grid_tiles = P / ts + act_est + 1;
+
+  StageTimer t7(L, 7, s);
+  RouterArgs ra{};
+  ra.x = reinterpret_cast<const uint16_t *>(x);
+  ra.T = T; ra.H = H; ra.E = E; ra.k = k;
+  ra.w = L->router_w; ra.bias = L->router_b;
+  ra.logits = L->logits; ra.ids = L->ids; ra.gates = L->gates;
+  ra.xf16 = L->xf16; ra.xs = L->xs; ra.counter = L->router_counter;
+  StageTimer t0(L, 0, s);
+  launch_router(ra, s);
+  CUDA_TRY(cudaGetLastError());
+  t0.launched(1);
+  t0.end();
+
+  PermArgs pa{};
+  pa.ids = L->ids; pa.n_pairs = P; pa.E = E; pa.k = k; pa.tile_tokens = ts;
+  pa.counts = L->counts; pa.offsets = L->offsets; pa.perm = L->perm; pa.inv = L->inv;
+  pa.tiles = L->tiles; pa.n_tiles = L->n_tiles; pa.prow_token = L->prow_token;
+  pa.prow_pair = L->prow_pair; pa.active = L->active;
+  StageTimer t1(L, 1, s);
+  launch_permute(pa, s);
+  CUDA_TRY(cudaGetLastError());
+  t1.launched(1);
+  t1.end();
+
+  if (dbg) {
+    if (dbg->logits) CUDA_TRY(cudaMemcpyAsync(dbg->logits, L->logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->ids) CUDA_TRY(cudaMemcpyAsync(dbg->ids, L->ids, (size_t)P * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->gates) CUDA_TRY(cudaMemcpyAsync(dbg->gates, L->gates, (size_t)P * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->counts) CUDA_TRY(cudaMemcpyAsync(dbg->counts, L->counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->offsets) CUDA_TRY(cudaMemcpyAsync(dbg->offsets, L->offsets, (size_t)(E + 1) * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->perm) CUDA_TRY(cudaMemcpyAsync(dbg->perm, L->perm, (size_t)P * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->inv) CUDA_TRY(cudaMemcpyAsync(dbg->inv, L->inv, (size_t)P * 4, cudaMemcpyDeviceToDevice, s));
+  }
+
+  const bool resident = L->n_resident == E;
+  if (!resident) {
+    CUDA_TRY(cudaMemcpyAsync(L->h_counts, L->counts, (size_t)E * 4, cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaEventRecord(L->ev_counts, s));
+  }
+
+  // always-resident shared expert (runs while the host builds the miss list)
+  if (Is) {
+    StageTimer t2(L, 2, s);
+    const int snt = T <= 8 ? 1 : (T <= 16 ? 2 : 4);
+    const int stiles = (T + 8 * snt - 1) / (8 * snt);
+    ExpertArgs a{};
+    a.tile_tokens = 8 * snt;
+    a.T = T;
+    a.dense_w0 = L->shared_w[0];
+    a.dense_w1 = L->shared_w[1];
+    a.K = H; a.rows = Is; a.n_rowblocks = Is / 128;
+    a.k_split = pick_split(stiles * (Is / 128), H / 128);
+    a.act = reinterpret_cast<const uint16_t *>(x);
+    a.h_out = L->sh_h;
+    launch_expert(WF_BF16, MODE_GATEUP, snt, a, stiles, s);
+    CUDA_TRY(cudaGetLastError());
+    a.dense_w0 = L->shared_w[2];
+    a.dense_w1 = nullptr;
+    a.K = Is; a.rows = H; a.n_rowblocks = H / 256;
+    a.k_split = pick_split(stiles * (H / 256), Is / 128);
+    a.act = L->sh_h;
+    a.o_out = L->sh_s;
+    launch_expert(WF_BF16, MODE_DOWN, snt, a, stiles, s);
+    CUDA_TRY(cudaGetLastError());
+    t2.launched(2);
+    t2.end();
+  }
+
+  const int cs_gu = pick_split(act_est * (I / 128), H / 128);
+  const int cs_dn = pick_split(act_est * (H / 256), I / 128);
+  int waves = 0, misses_n = 0;
+  if (resident) {
+    ST_TRY(run_experts(L, L->ptr_resident, nt, grid_tiles, cs_gu, cs_dn, s));
+  } else {
+    CUDA_TRY(cudaEventSynchronize(L->ev_counts));
+    std::vector<int> misses;
+    int act = 0;
+    for (int e = 0; e < E; ++e) {
+      if (L->h_counts[e] > 0) {
+        ++act;
+        if (L->slot_of[e] < 0) misses.push_back(e);
+      }
+    }
+    L->st.last_active = act;
+    misses_n = (int)misses.size();
+    const int NS = L->n_staging;
+    if (misses.empty()) {
+      ST_TRY(run_experts(L, L->ptr_resident, nt, grid_tiles, cs_gu, cs_dn, s));
+    } else {
+      const bool one = misses_n <= NS;
+      const int wave_sz = one ? NS : NS / 2;
+      const int nw = (misses_n + wave_sz - 1) / wave_sz;
+      const size_t bytes = L->L.bytes;
+      if (L->inject == 1) {   // host-side failure injection: no copy is issued
+        L->inject = 0;
+        return fail(MOE_ERR_CUDA, "staging copy failed (injected)");
+      }
+      // the previous forward's kernels must be done with the staging ring
+      if (L->staging_used) CUDA_TRY(cudaStreamWaitEvent(L->side, L->ev_fwd_done, 0));
+      for (int w = 0; w < nw; ++w) {
+        const int half = one ? 0 : (w & 1);
+        const int base = one ? 0 : half * (NS / 2);
+        if (!one && w >= 2) CUDA_TRY(cudaStreamWaitEvent(L->side, L->ev_done[half], 0));
+        PtrUpdate u{};
+        u.E = E;
+        u.keep_resident = (w == 0);
+        const int b0 = w * wave_sz, b1 = std::min(misses_n, b0 + wave_sz);
+        for (int i = b0; i < b1; ++i) {
+          const int e = misses[i];
+          uint8_t *dst = L->staging + (size_t)(base + (i - b0)) * bytes;
+          CUDA_TRY(cudaMemcpyAsync(dst, L->store + (size_t)e * bytes, bytes, cudaMemcpyHostToDevice, L->side));
+          u.expert[u.n] = e;
+          u.ptr[u.n] = dst;
+          ++u.n;
+        }
+        CUDA_TRY(cudaEventRecord(L->ev_copied[half], L->side));
+        StageTimer t6(L, 6, s);
+        CUDA_TRY(cudaStreamWaitEvent(s, L->ev_copied[half], 0));
+        launch_ptr_update(u, L->ptr_resident, L->ptr_pass, s);
+        CUDA_TRY(cudaGetLastError());
+        t6.launched(1);
+        t6.end();
+        ST_TRY(run_experts(L, L->ptr_pass, nt, grid_tiles, cs_gu, cs_dn, s));
+        if (!one) CUDA_TRY(cudaEventRecord(L->ev_done[half], s));
+      }
+      CUDA_TRY(cudaEventRecord(L->ev_fwd_done, s));
+      L->staging_used = true;
+      waves = nw;
+      L->st.misses += misses_n;
+      L->st.bytes_staged += (uint64_t)misses_n * bytes;
+    }
+  }
+
+  CombineArgs ca{};
+  ca.oprime = L->oprime;
+  ca.shared = Is ? L->sh_s : nullptr;
+  ca.y = y;
+  ca.T = T; ca.H = H; ca.k = k;
+  StageTimer t5(L, 5, s);
+  launch_combine(ca, s);
+  CUDA_TRY(cudaGetLastError());
+  t5.launched(1);
+  t5.end();
+  t7.end();
+  if (L->prof) L->prof_acc.forwards += 1;
+
+  L->st.forwards += 1;
+  L->st.last_misses = misses_n;
+  L->st.last_waves = waves;
+  L->st.last_path = 0;
+  if (resident) L->st.last_active = -1;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward_host(moe_layer_t L, const uint16_t *x_host, int32_t T, float *y_host,
+                              void *stream) {
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  if (T < 0 || T > L->cfg.max_tokens) return fail(MOE_ERR_INVALID_ARG, "T out of range [0, max_tokens]");
+  if (T == 0) return MOE_OK;
+  if (!x_host || !y_host) return fail(MOE_ERR_INVALID_ARG, "x or y is NULL");
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t H = L->cfg.hidden;
+  CUDA_TRY(cudaMemcpyAsync(L->xin, x_host, (size_t)T * H * 2, cudaMemcpyHostToDevice, s));
+  ST_TRY(moe_forward(L, L->xin, T, L->yout, stream, nullptr));
+  CUDA_TRY(cudaMemcpyAsync(y_host, L->yout, (size_t)T * H * 4, cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  return MOE_OK;
+}
+
+moe_status_t moe_get_stats(moe_layer_t L, moe_stats_t *out) {
+  if (!L || !out) return fail(MOE_ERR_INVALID_ARG, "layer or out is NULL");
+  *out = L->st;
+  return MOE_OK;
+}
+
+static moe_status_t drain_profile(moe_layer *L) {
+  for (auto &p : L->pend) {
+    CUDA_TRY(cudaEventSynchronize(p.b));
+    float ms = 0.0f;
+    CUDA_TRY(cudaEventElapsedTime(&ms, p.a, p.b));
+    L->prof_acc.ms[p.stage] += ms;
+    L->evpool.push_back(p.a);
+    L->evpool.push_back(p.b);
+  }
+  L->pend.clear();
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_enable(moe_layer_t L, int32_t enable) {
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  ST_TRY(drain_profile(L));
+  L->prof_acc = moe_profile_t{};
+  L->prof = enable != 0;
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_read(moe_layer_t L, moe_profile_t *out) {
+  if (!L || !out) return fail(MOE_ERR_INVALID_ARG, "layer or out is NULL");
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  ST_TRY(drain_profile(L));
+  *out = L->prof_acc;
+  return MOE_OK;
+}
+
+void moe_destroy(moe_layer_t L) { free_layer(L); }
+
+moe_status_t moe_debug_inject(moe_layer_t L, int32_t what) {
+  if (what < 0 || what > 2) return fail(MOE_ERR_INVALID_ARG, "unknown injection");
+  if (what == 2 || (!L && what == 0)) {
+    g_inject_create = what;
+    return MOE_OK;
+  }
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  L->inject = what;
+  return MOE_OK;
+}
+
+}  // extern "C"

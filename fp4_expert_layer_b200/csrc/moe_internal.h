@@ -1,0 +1,130 @@
+// moe_internal.h -- internal interfaces of the sm_100a MoE layer library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe_layer.h"
+
+namespace moe {
+
+constexpr int kChunk = 128;        // K elements per activation-scale chunk / per mainloop step
+constexpr int kWarps = 8;          // warps per expert-kernel CTA
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+constexpr int kPermThreads = 512;
+constexpr int kPtrListMax = 256;   // expert pointers one table-update launch can carry
+
+// Device layout of one routed expert ("blob"): the checkpoint bytes of the three
+// matrices (codes unchanged, block scales unchanged) plus, for MXFP4, one byte
+// per row holding the row's largest E8M0 code (the row reference exponent the
+// decode kernels fold out of the f16 operand), or, for NVFP4, the three fp32
+// per-tensor scales.  Every piece starts on a 256-byte boundary.  The pinned
+// host store holds all E experts in exactly this layout, so a miss is one
+// contiguous host-to-device copy.
+struct BlobLayout {
+  size_t codes[3];
+  size_t scales[3];
+  size_t sref[3];     // MXFP4 only
+  size_t glob;        // NVFP4 only: float[3]
+  size_t bytes;
+  int rows[3];
+  int K[3];
+  int G;              // block size along K: 32 (MXFP4) or 16 (NVFP4)
+  int fmt;
+};
+
+BlobLayout blob_layout(int H, int I, int fmt);
+
+// One token tile of one expert: rows [prow0, prow0 + nrows) of the padded,
+// expert-sorted activation order; each expert's rows start on a multiple of 8.
+struct TileInfo {
+  int expert;
+  int prow0;
+  int nrows;
+  int sorted0;   // first row in the unpadded sorted order
+};
+
+// ------------------------------------------------------------------ routing
+struct RouterArgs {
+  const uint16_t *x;     // bf16 [T, H]
+  int T, H, E, k;
+  const float *w;        // [E, H]
+  const float *bias;     // [E] or null
+  float *logits;         // [T, E]
+  int *ids;              // [T, k]
+  float *gates;          // [T, k]
+  uint16_t *xf16;        // f16 [T, H], chunk-scaled
+  float *xs;             // [T, H/128] chunk multipliers
+  int *counter;          // [ceil(T/TT)] zero-initialised completion counters
+};
+void launch_router(const RouterArgs &a, cudaStream_t s);
+
+struct PermArgs {
+  const int *ids;        // [T*k]
+  int n_pairs, E, k, tile_tokens;
+  int *counts;           // [E]
+  int *offsets;          // [E+1]
+  int *perm;             // [n_pairs]
+  int *inv;              // [n_pairs]
+  TileInfo *tiles;       // [max tiles]
+  int *n_tiles;          // [1]
+  int *prow_token;       // [max prows]
+  int *prow_pair;        // [max prows]
+  int *active;           // [1] experts with >= 1 pair
+};
+void launch_permute(const PermArgs &a, cudaStream_t s);
+
+// ------------------------------------------------------------------ experts
+enum WeightFmt { WF_MX = 0, WF_NV = 1, WF_BF16 = 2 };
+enum ExpertMode { MODE_GATEUP = 0, MODE_DOWN = 1 };
+
+struct ExpertArgs {
+  // routed experts: blob pointer per expert (null = not in this pass)
+  const uint8_t *const *expert_ptr;
+  BlobLayout L;
+  // dense (shared expert) weights, bf16: m0 (and m1 for gate/up)
+  const uint16_t *dense_w0;
+  const uint16_t *dense_w1;
+  int K;                 // reduction length
+  int rows;              // output rows of one matrix (I, H or I_s)
+  int n_rowblocks;       // rows / rows-per-CTA
+  int k_split;           // cluster size along K
+  int tile_tokens;       // 8 * NT
+  // routed tiles
+  const TileInfo *tiles;
+  const int *n_tiles;
+  const int *prow_token; // padded row -> token (gate/up B rows) or -1
+  const int *prow_pair;  // padded row -> pair p or -1
+  const float *gates;    // [T*k]
+  int T;                 // dense path: number of tokens
+  // activations (B operand)
+  const uint16_t *act;   // f16 chunk-scaled (routed) or bf16 (dense), row stride K
+  const float *act_scale;// [rows][K/128] (routed only)
+  // outputs
+  uint16_t *h_out;       // gate/up: f16 chunk-scaled (routed) / bf16 (dense), row stride = rows
+  float *h_scale;        // routed gate/up: [prows][rows/128]
+  float *o_out;          // down: routed O'[pair][rows] or dense s[t][rows]
+};
+void launch_expert(int wf, int mode, int nt, const ExpertArgs &a, int grid_tiles, cudaStream_t s);
+
+struct CombineArgs {
+  const float *oprime;   // [T*k, H]
+  const float *shared;   // [T, H] or null
+  float *y;              // [T, H]
+  int T, H, k;
+};
+void launch_combine(const CombineArgs &a, cudaStream_t s);
+
+struct PtrUpdate {
+  int n;
+  int keep_resident;     // 1: start from the resident table, 0: start from all-null
+  int E;
+  int expert[kPtrListMax];
+  const uint8_t *ptr[kPtrListMax];
+};
+void launch_ptr_update(const PtrUpdate &u, const uint8_t *const *resident, const uint8_t **out,
+                       cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,304 @@
+// route.cu -- router GEMV/GEMM with fused softmax top-k, the token-to-expert
+// permutation, expert pointer-table updates and the ordered combine.
+//
+// Routing semantics (which function, how many experts, top-k) are what the
+// checkpoint declares and never change silently ("ro99/strata", rules list).
+// This library implements softmax routing with the top-k gates renormalised to
+// sum to one: ids are the k largest logits in descending order (lower expert
+// index first on ties) and g_j = exp(l_j - l_max) / sum_i exp(l_i - l_max)
+// over the chosen k, which equals softmax over all E renormalised to the k.
+#include <cooperative_groups.h>
+
+#include "device_utils.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+constexpr int kRouterTT = 4;      // tokens per router CTA
+constexpr int kRouterEB = 8;      // experts per router CTA (one per warp)
+
+// grid (ceil(T/TT), ceil(E/EB)), 256 threads, dynamic smem TT*H floats.
+// Each CTA computes logits for its TT tokens x EB experts; the CTA with
+// blockIdx.y == 0 also writes the chunk-scaled f16 copy of its tokens; the last
+// CTA of a token tile to finish (completion counter) runs top-k for the tile.
+__global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
+  extern __shared__ float xs_smem[];   // [TT][H]
+  __shared__ int is_last;
+  const int H = a.H, E = a.E;
+  const int t0 = blockIdx.x * kRouterTT;
+  const int nt = min(kRouterTT, a.T - t0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // x tile -> smem (fp32)
+  for (int i = threadIdx.x; i < nt * H / 2; i += blockDim.x) {
+    const int t = (2 * i) / H, h = (2 * i) % H;
+    uint32_t v = *reinterpret_cast<const uint32_t *>(a.x + (size_t)(t0 + t) * H + h);
+    xs_smem[t * H + h] = __uint_as_float(v << 16);
+    xs_smem[t * H + h + 1] = __uint_as_float(v & 0xFFFF0000u);
+  }
+  __syncthreads();
+
+  // logits: warp w -> expert e
+  const int e = blockIdx.y * kRouterEB + warp;
+  if (e < E) {
+    float acc[kRouterTT];
+#pragma unroll
+    for (int t = 0; t < kRouterTT; ++t) acc[t] = 0.0f;
+    const float *w = a.w + (size_t)e * H;
+    for (int h = lane * 4; h < H; h += 128) {
+      float4 wv = *reinterpret_cast<const float4 *>(w + h);
+#pragma unroll
+      for (int t = 0; t < kRouterTT; ++t) {
+        if (t < nt) {
+          const float4 xv = *reinterpret_cast<const float4 *>(xs_smem + t * H + h);
+          acc[t] = fmaf(wv.x, xv.x, acc[t]);
+          acc[t] = fmaf(wv.y, xv.y, acc[t]);
+          acc[t] = fmaf(wv.z, xv.z, acc[t]);
+          acc[t] = fmaf(wv.w, xv.w, acc[t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kRouterTT; ++t) {
+      float v = acc[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && t < nt) a.logits[(size_t)(t0 + t) * E + e] = v + (a.bias ? a.bias[e] : 0.0f);
+    }
+  }
+
+  // chunk-scaled f16 copy of x: warp per (token, 128-chunk)
+  if (blockIdx.y == 0) {
+    const int nck = H / kChunk;
+    for (int job = warp; job < nt * nck; job += kWarps) {
+      const int t = job / nck, c = job % nck;
+      const float4 v = *reinterpret_cast<const float4 *>(xs_smem + t * H + c * kChunk + lane * 4);
+      float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const int ce = chunk_exponent(m);
+      const float inv = pow2f(-ce);
+      uint2 out;
+      __half2 p0 = __floats2half2_rn(v.x * inv, v.y * inv);
+      __half2 p1 = __floats2half2_rn(v.z * inv, v.w * inv);
+      out.x = *reinterpret_cast<uint32_t *>(&p0);
+      out.y = *reinterpret_cast<uint32_t *>(&p1);
+      *reinterpret_cast<uint2 *>(a.xf16 + (size_t)(t0 + t) * H + c * kChunk + lane * 4) = out;
+      if (lane == 0) a.xs[(size_t)(t0 + t) * nck + c] = pow2f(ce);
+    }
+  }
+
+  // completion: the last CTA of this token tile runs top-k
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(&a.counter[blockIdx.x], 1);
+    is_last = (prev == (int)gridDim.y - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (threadIdx.x == 0) a.counter[blockIdx.x] = 0;
+
+  // top-k: warp per token; lane holds experts lane, lane+32, ...
+  const int k = a.k;
+  if (warp < nt) {
+    const int t = t0 + warp;
+    constexpr int kPer = kMaxExperts / 32;
+    float lv[kPer];
+    const float *lrow = a.logits + (size_t)t * E;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int ee = lane + 32 * i;
+      lv[i] = (ee < E) ? __ldcg(lrow + ee) : -INFINITY;
+    }
+    uint32_t taken = 0;   // bit i: lane's i-th expert already chosen
+    float lmax = 0.0f, den = 0.0f;
+    float my_l = 0.0f;    // lane j keeps the logit of choice j
+    int my_id = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int ee = lane + 32 * i;
+        if (ee < E && !((taken >> i) & 1u)) {
+          if (bi == 0x7fffffff || lv[i] > bv) { bv = lv[i]; bi = ee; }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (j == 0) lmax = bv;
+      if (lane == j) { my_l = bv; my_id = bi; }
+    }
+    const float ex = (lane < k) ? expf(my_l - lmax) : 0.0f;
+    // ordered sum over j = 0..k-1
+    for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, ex, j);
+    if (lane < k) {
+      a.ids[(size_t)t * k + lane] = my_id;
+      a.gates[(size_t)t * k + lane] = ex / den;
+    }
+  }
+}
+
+void launch_router(const RouterArgs &a, cudaStream_t s) {
+  dim3 grid((a.T + kRouterTT - 1) / kRouterTT, (a.E + kRouterEB - 1) / kRouterEB);
+  const size_t smem = (size_t)kRouterTT * a.H * sizeof(float);
+  if (smem > 48 * 1024) cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  router_kernel<<<grid, 256, smem, s>>>(a);
+}
+
+// ---------------------------------------------------------------------------
+// Permutation: stable counting sort of pair index p = t*k + j by expert.
+// Single CTA; pairs are processed in chunks of blockDim, ranks inside a chunk
+// from warp match + per-warp counts scanned in warp order, so the order of
+// equal experts is ascending p (stable).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermArgs a) {
+  extern __shared__ int psm[];
+  const int E = a.E;
+  constexpr int W = kPermThreads / 32;
+  int *cnt = psm;                 // [E]
+  int *cursor = cnt + E;          // [E]
+  int *poff = cursor + E;         // [E+1] padded offsets
+  int *toff = poff + E + 1;       // [E+1] tile offsets
+  int *wcnt = toff + E + 1;       // [W][E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int i = tid; i < E; i += blockDim.x) { cnt[i] = 0; cursor[i] = 0; }
+  for (int i = tid; i < W * E; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  for (int p = tid; p < a.n_pairs; p += blockDim.x) atomicAdd(&cnt[a.ids[p]], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int o = 0, po = 0, to = 0, act = 0;
+    for (int e = 0; e < E; ++e) {
+      const int c = cnt[e];
+      a.offsets[e] = o;
+      poff[e] = po;
+      toff[e] = to;
+      o += c;
+      po += (c + 7) & ~7;
+      to += (c + a.tile_tokens - 1) / a.tile_tokens;
+      act += c > 0;
+    }
+    a.offsets[E] = o;
+    poff[E] = po;
+    toff[E] = to;
+    *a.n_tiles = to;
+    *a.active = act;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int c = cnt[e];
+    a.counts[e] = c;
+    const int nt = (c + a.tile_tokens - 1) / a.tile_tokens;
+    for (int i = 0; i < nt; ++i) {
+      TileInfo ti;
+      ti.expert = e;
+      ti.prow0 = poff[e] + i * a.tile_tokens;
+      ti.nrows = min(a.tile_tokens, c - i * a.tile_tokens);
+      ti.sorted0 = a.offsets[e] + i * a.tile_tokens;
+      a.tiles[toff[e] + i] = ti;
+    }
+    for (int r = poff[e] + c; r < poff[e + 1]; ++r) { a.prow_token[r] = -1; a.prow_pair[r] = -1; }
+  }
+  __syncthreads();
+
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < a.n_pairs; base += blockDim.x) {
+    const int p = base + tid;
+    const bool valid = p < a.n_pairs;
+    const int e = valid ? a.ids[p] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    if (valid && rank == 0) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int run = cursor[ee];
+      for (int w = 0; w < W; ++w) {
+        const int c = wcnt[w * E + ee];
+        wcnt[w * E + ee] = run;
+        run += c;
+      }
+      cursor[ee] = run;
+    }
+    __syncthreads();
+    if (valid) {
+      const int local = wcnt[warp * E + e] + rank;
+      const int pos = a.offsets[e] + local;
+      const int prow = poff[e] + local;
+      a.perm[pos] = p;
+      a.inv[p] = pos;
+      a.prow_token[prow] = p / a.k;
+      a.prow_pair[prow] = p;
+    }
+    __syncthreads();
+    for (int i = tid; i < W * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+  }
+}
+
+void launch_permute(const PermArgs &a, cudaStream_t s) {
+  const int W = kPermThreads / 32;
+  const size_t smem = sizeof(int) * ((size_t)4 * a.E + 2 + (size_t)W * a.E);
+  if (smem > 48 * 1024) cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  permute_kernel<<<1, kPermThreads, smem, s>>>(a);
+}
+
+// ---------------------------------------------------------------------------
+// Expert pointer table for one pass: start from the resident table (or all
+// null) and overwrite the listed experts.
+// ---------------------------------------------------------------------------
+__global__ void ptr_update_kernel(const PtrUpdate u, const uint8_t *const *resident,
+                                  const uint8_t **out) {
+  for (int e = threadIdx.x; e < u.E; e += blockDim.x) out[e] = u.keep_resident ? resident[e] : nullptr;
+  __syncthreads();
+  for (int i = threadIdx.x; i < u.n; i += blockDim.x) out[u.expert[i]] = u.ptr[i];
+}
+
+void launch_ptr_update(const PtrUpdate &u, const uint8_t *const *resident, const uint8_t **out,
+                       cudaStream_t s) {
+  ptr_update_kernel<<<1, 256, 0, s>>>(u, resident, out);
+}
+
+// ---------------------------------------------------------------------------
+// Ordered combine: y[t] = sum_{j<k} O'[t*k + j] (in j order) + s[t].
+// ---------------------------------------------------------------------------
+__global__ void combine_kernel(const CombineArgs a) {
+  const int H4 = a.H / 4;
+  const size_t n = (size_t)a.T * H4;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t t = i / H4, c = i % H4;
+    const float4 *o = reinterpret_cast<const float4 *>(a.oprime) + t * a.k * H4 + c;
+    float4 acc = __ldcs(o);
+    for (int j = 1; j < a.k; ++j) {
+      const float4 v = __ldcs(o + (size_t)j * H4);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    if (a.shared) {
+      const float4 v = reinterpret_cast<const float4 *>(a.shared)[t * H4 + c];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    reinterpret_cast<float4 *>(a.y)[t * H4 + c] = acc;
+  }
+}
+
+void launch_combine(const CombineArgs &a, cudaStream_t s) {
+  const size_t n = (size_t)a.T * (a.H / 4);
+  int blocks = (int)((n + 255) / 256);
+  blocks = blocks > 148 * 8 ? 148 * 8 : blocks;
+  if (blocks < 1) blocks = 1;
+  combine_kernel<<<blocks, 256, 0, s>>>(a);
+}
+
+}  // namespace moe

@@ -1,0 +1,224 @@
+/*
+ * moe_layer.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts layer
+ * over 4-bit block-quantised experts.
+ *
+ * One layer forward:
+ *   router GEMM (fp32 logits) -> softmax top-k with renormalised gates ->
+ *   token-to-expert permutation -> SwiGLU expert FFN read straight from
+ *   MXFP4 / NVFP4 bytes -> gate-weighted combine (+ optional bf16 shared expert).
+ * Experts are addressed through a resident-slot table: a budget of experts
+ * lives in HBM slots, every expert lives in a library-owned pinned host
+ * store, and experts a forward needs that are not resident are copied from
+ * the pinned store with cudaMemcpyAsync on a side stream.
+ *
+ * Where each operation is defined (pages of the Strata reference set):
+ *  - expert formats: "ro99/strata", "MXFP4 is read as MXFP4" (two E2M1 codes
+ *    per byte, one E8M0 exponent per group of 32) and its model table
+ *    ("NVFP4 or MXFP4 experts");
+ *  - scale admission: "ro99/strata", "Scales are admitted, not clamped"
+ *    (E8M0 codes 0 and 255 fail admission at load);
+ *  - routing semantics, expert count and top-k come from the checkpoint and
+ *    never change silently; exact mode completes or fails ("ro99/strata",
+ *    list of rules under the introduction);
+ *  - the paging hierarchy (every expert pinned in host RAM, a budget of hot
+ *    experts on the GPU, shared experts always resident): "Strata, Explained",
+ *    section 2, and strata.amperor.ai ("budget ... resident experts/layer");
+ *  - paged output bit-identical to the resident model: strata.amperor.ai,
+ *    legend of the memory-fit list.
+ * The pages print no layer formula; the forms used (softmax routing,
+ * h = silu(gate) * up, low nibble = even element, groups along the input
+ * dimension) are the plainest readings and are listed in the design notes.
+ *
+ * Conventions for every call:
+ *  - Nothing throws across this ABI.  Every call returns a moe_status_t; on
+ *    failure moe_last_error() returns a thread-local description.
+ *  - "stream" is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  All device work of a call is ordered on that stream.
+ *  - Device pointers are CUDA device memory of the layer's device; host
+ *    pointers are ordinary (pageable or pinned) host memory.
+ */
+#ifndef MOE_LAYER_H
+#define MOE_LAYER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_layer *moe_layer_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* bad pointer, size, shape or enum value            */
+  MOE_ERR_ADMISSION = 2,   /* a block-scale code the format cannot represent   */
+  MOE_ERR_SLOT_TABLE = 3,  /* slot out of range, duplicate slot, over budget    */
+  MOE_ERR_OOM = 4,         /* device or pinned host allocation failed           */
+  MOE_ERR_CUDA = 5,        /* a CUDA runtime call failed (detail in last_error) */
+  MOE_ERR_UNSUPPORTED = 6  /* valid request this build does not implement       */
+} moe_status_t;
+
+typedef enum { MOE_FMT_MXFP4 = 0, MOE_FMT_NVFP4 = 1 } moe_fmt_t;
+
+/* EXACT (default): activations stay 16-bit, FP4 weights decode exactly, fp32
+ * accumulation.  A4 (opt-in): activations are quantised to the experts' own
+ * 4-bit format before each expert GEMM so the tcgen05 block-scaled FP4 MMA can
+ * run; never chosen silently. */
+typedef enum { MOE_NUMERICS_EXACT = 0, MOE_NUMERICS_A4 = 1 } moe_numerics_t;
+
+typedef struct {
+  int32_t hidden;       /* H; multiple of 256                                   */
+  int32_t inter;        /* I (routed expert intermediate); multiple of 128       */
+  int32_t n_experts;    /* E routed experts, 1..1024                            */
+  int32_t top_k;        /* k, 1..min(E, 32)                                     */
+  int32_t shared_inter; /* I_s of the always-on bf16 shared expert, 0 = none;   */
+                        /* multiple of 128                                      */
+  int32_t fmt;          /* moe_fmt_t                                            */
+  int32_t renormalize;  /* must be 1: top-k gates renormalised to sum to 1      */
+  int32_t numerics;     /* moe_numerics_t                                       */
+  int32_t n_slots;      /* S resident HBM slots, 0..E                           */
+  int32_t max_tokens;   /* largest T accepted by moe_forward, >= 1              */
+  int32_t n_staging;    /* staging buffers for non-resident experts; >= 2 when  */
+                        /* S < E (0 = library default)                          */
+  int32_t device;       /* CUDA device ordinal                                   */
+} moe_config_t;
+
+/* Layer weights in checkpoint layout (host memory; read only during create).
+ * Matrices are [out, in] row-major; E2M1 codes are packed two per byte with the
+ * even input index in the low nibble; block scales run along the input dim.
+ *   matrix 0 = gate [I, H], 1 = up [I, H], 2 = down [H, I]
+ *   codes[m][e]  : uint8 [rows, K/2]
+ *   scales[m][e] : MXFP4 E8M0 uint8 [rows, K/32]; NVFP4 E4M3 uint8 [rows, K/16]
+ *   global_scale : NVFP4 only, fp32 [E, 3] per-tensor scale; else NULL
+ *   shared_w[m]  : bf16 bit patterns, gate [I_s, H], up [I_s, H], down [H, I_s]
+ * The library copies everything during moe_layer_create; the caller may free
+ * these buffers when it returns. */
+typedef struct {
+  const float *router_w;            /* fp32 [E, H]                             */
+  const float *router_bias;         /* fp32 [E] added to the logits, or NULL   */
+  const uint8_t *const *codes[3];   /* codes[m] -> array of E host pointers    */
+  const uint8_t *const *scales[3];  /* scales[m] -> array of E host pointers   */
+  const float *global_scale;        /* fp32 [E, 3] or NULL                     */
+  const uint16_t *shared_w[3];      /* NULL when shared_inter == 0             */
+} moe_weights_t;
+
+/* Optional routing outputs of a forward (all device pointers, each may be
+ * NULL).  logits fp32 [T, E]; ids int32 [T, k] in descending-logit order (lower
+ * index first on ties); gates fp32 [T, k]; counts int32 [E]; offsets int32
+ * [E+1] (exclusive scan of counts); perm int32 [T*k]: sorted position -> pair
+ * index p = t*k + j (stable by expert, ties by ascending p); inv int32 [T*k]:
+ * p -> sorted position. */
+typedef struct {
+  float *logits;
+  int32_t *ids;
+  float *gates;
+  int32_t *counts;
+  int32_t *offsets;
+  int32_t *perm;
+  int32_t *inv;
+} moe_routing_t;
+
+typedef struct {
+  uint64_t forwards;       /* forwards run since create                         */
+  uint64_t misses;         /* expert copies from the pinned store, cumulative   */
+  uint64_t bytes_staged;   /* bytes copied host -> device for misses, cumulative */
+  int32_t last_misses;     /* misses of the last forward                        */
+  int32_t last_waves;      /* staging waves of the last forward (0 = resident)  */
+  int32_t last_active;     /* experts with at least one token, last forward     */
+  int32_t last_path;       /* 0 = decode kernels, 1 = tcgen05 grouped GEMM      */
+  uint64_t launches;       /* kernels this library launched, cumulative         */
+  uint64_t expert_bytes;   /* device-layout bytes of one routed expert          */
+  uint64_t device_bytes;   /* HBM held by the layer                             */
+  uint64_t pinned_bytes;   /* pinned host memory held by the layer              */
+} moe_stats_t;
+
+/* Memory plan of a configuration without allocating anything (the dry-run
+ * placement plan idea of "ro99/strata": --admission-only).  Validates the
+ * configuration. */
+typedef struct {
+  uint64_t expert_bytes;   /* one routed expert in device layout                */
+  uint64_t slot_bytes;     /* S resident slots                                  */
+  uint64_t staging_bytes;  /* staging ring                                      */
+  uint64_t resident_bytes; /* router + shared expert (always in HBM)            */
+  uint64_t scratch_bytes;  /* per-forward scratch sized by max_tokens           */
+  uint64_t pinned_bytes;   /* pinned host store of all E experts                */
+} moe_plan_t;
+
+moe_status_t moe_layer_plan(const moe_config_t *cfg, moe_plan_t *out);
+
+/* Check every block-scale code of the weights against the format (no
+ * allocation).  MXFP4: E8M0 codes 0 and 255 are rejected.  NVFP4: E4M3 NaN
+ * codes and negative scales are rejected, and the per-tensor scale must be
+ * finite and positive.  Returns MOE_ERR_ADMISSION with the expert, matrix and
+ * index in moe_last_error(). */
+moe_status_t moe_admit(const moe_config_t *cfg, const moe_weights_t *w);
+
+/* Create a layer on cfg->device: admits the scales, copies every routed expert
+ * into a pinned host store in device layout, uploads router and shared-expert
+ * weights to HBM, allocates S slots, the staging ring and scratch sized by
+ * max_tokens.  No expert is resident until moe_set_slot_table.  The stream
+ * orders the uploads; the call returns after they complete. */
+moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, void *stream,
+                              moe_layer_t *out);
+
+/* Set which experts are resident: slot_of_expert is host int32 [E], each entry
+ * a slot index in [0, S) or -1 (kept in host memory).  Rejects out-of-range
+ * slots, two experts on one slot and more than S resident experts with
+ * MOE_ERR_SLOT_TABLE (the previous table stays in force).  Copies newly
+ * resident experts into their slots on `stream`; later forwards on the same
+ * stream see the new table.  The table never changes inside moe_forward. */
+moe_status_t moe_set_slot_table(moe_layer_t layer, const int32_t *slot_of_expert, void *stream);
+
+/* Forward T tokens: x device bf16 [T, H] -> y device fp32 [T, H].
+ * 0 <= T <= max_tokens (T == 0 is a no-op).  x and y must not overlap.
+ * When every expert the forward needs is resident, the call only enqueues
+ * work on `stream` and returns.  Otherwise it waits for the routing counts
+ * (one small device-to-host copy), then copies the missing experts from the
+ * pinned store on the layer's side stream, overlapped with compute in waves
+ * of at most n_staging experts; it returns once all work is enqueued.
+ * dbg (may be NULL) receives the routing tensors of this forward. */
+moe_status_t moe_forward(moe_layer_t layer, const void *x, int32_t T, float *y, void *stream,
+                         const moe_routing_t *dbg);
+
+/* Same forward from and to HOST memory: copies x (host bf16 [T, H]) to a
+ * layer-owned device buffer, runs the forward and copies y back to host fp32
+ * [T, H].  Returns after y is in host memory. */
+moe_status_t moe_forward_host(moe_layer_t layer, const uint16_t *x_host, int32_t T,
+                              float *y_host, void *stream);
+
+moe_status_t moe_get_stats(moe_layer_t layer, moe_stats_t *out);
+
+/* Per-stage device timing (tracing).  While enabled, every forward records a
+ * CUDA event pair around each stage on the forward's stream; moe_profile_read
+ * waits for those events and returns the accumulated milliseconds and launch
+ * counts since the last enable.  Stages: 0 router + top-k, 1 permutation,
+ * 2 shared expert, 3 routed gate/up + SwiGLU, 4 routed down + gate scale,
+ * 5 combine, 6 waits on staging copies, 7 whole forward. */
+#define MOE_PROFILE_STAGES 8
+typedef struct {
+  uint64_t forwards;
+  double ms[MOE_PROFILE_STAGES];
+  uint64_t launches[MOE_PROFILE_STAGES];
+} moe_profile_t;
+
+moe_status_t moe_profile_enable(moe_layer_t layer, int32_t enable);
+moe_status_t moe_profile_read(moe_layer_t layer, moe_profile_t *out);
+
+/* Waits for the layer's work, then frees everything it holds.  NULL is a no-op. */
+void moe_destroy(moe_layer_t layer);
+
+/* Thread-local description of the last failure in this thread ("" if none). */
+const char *moe_last_error(void);
+
+/* Test hook for host-side failure injection (no GPU fault is ever caused):
+ * 1 = the next staging copy reports a failure, 2 = the next device allocation
+ * in moe_layer_create fails, 0 = off.  The forward must then return an error
+ * status and leave the CUDA context usable. */
+moe_status_t moe_debug_inject(moe_layer_t layer, int32_t what);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_LAYER_H */

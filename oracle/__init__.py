@@ -81,6 +81,8 @@ def lib():
         L.orc_route_row.restype = None
         L.orc_route_row.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]
         L.orc_max_threads.restype = C.c_int
+        L.orc_expert_rows.restype = None
+        L.orc_expert_rows.argtypes = [C.POINTER(_Layer), C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p]
         _lib = L
     return _lib
 
@@ -216,6 +218,15 @@ class Layer:
         g = np.zeros((T, self.k), dtype=np.float32)
         lib().orc_route_all(C.byref(self._s), _p(x), T, _p(lg), _p(ids), _p(g), threads)
         return lg, ids, g
+
+    def expert_rows(self, e: int, x_row_bits: np.ndarray, i0: int, n: int, o: np.ndarray = None):
+        """Timing sample: intermediate rows [i0, i0+n) of expert e on one token (EXACT)."""
+        xt = (np.asarray(x_row_bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+        xt = np.ascontiguousarray(xt, dtype=np.float64)
+        if o is None:
+            o = np.zeros(self.H, dtype=np.float64)
+        lib().orc_expert_rows(C.byref(self._s), e, xt.ctypes.data, i0, n, o.ctypes.data)
+        return o
 
     def dequant(self, m: int, e: int) -> np.ndarray:
         rows, K = (self.I, self.H) if m < 2 else (self.H, self.I)

@@ -335,6 +335,33 @@ void orc_expert_token(const orc_layer_t *L, int e, const double *xt, double *o) 
   free(row); free(xin); free(hin); free(h);
 }
 
+/* Timing sample for the benchmark's CPU leg (EXACT mode only): the formula of
+ * orc_expert_token restricted to intermediate rows [i0, i0+n): h_i for those
+ * rows and their terms Wd[r,i] * h_i added, in i order, into o[H]. */
+void orc_expert_rows(const orc_layer_t *L, int e, const double *xt, int i0, int n, double *o) {
+  const int H = L->H, I = L->I;
+  const int K = H > I ? H : I;
+  double *row = (double *)malloc(sizeof(double) * (size_t)K);
+  double *dcol = (double *)malloc(sizeof(double) * (size_t)I);
+  float *h = (float *)malloc(sizeof(float) * (size_t)n);
+  for (int i = i0; i < i0 + n; ++i) {
+    double a = 0.0, u = 0.0;
+    orc_dequant_row(L, 0, e, i, row);
+    for (int c = 0; c < H; ++c) a += row[c] * xt[c];
+    orc_dequant_row(L, 1, e, i, row);
+    for (int c = 0; c < H; ++c) u += row[c] * xt[c];
+    float af = (float)a, uf = (float)u;
+    h[i - i0] = (float)(silu((double)af) * (double)uf);
+  }
+  for (int r = 0; r < H; ++r) {
+    orc_dequant_row(L, 2, e, r, dcol);
+    double acc = o[r];
+    for (int i = i0; i < i0 + n; ++i) acc += dcol[i] * (double)h[i - i0];
+    o[r] = acc;
+  }
+  free(row); free(dcol); free(h);
+}
+
 /* Shared expert on one token: the same SwiGLU with bf16 weights, weight 1. */
 void orc_shared_token(const orc_layer_t *L, const double *xt, double *s) {
   const int H = L->H, Is = L->Is;

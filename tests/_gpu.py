@@ -1,0 +1,88 @@
+"""GPU-test helpers: build a layer through the C ABI, run it, compare with the oracle."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import synth
+from tests import _cases as cs
+
+
+def torch():
+    import torch as t
+    return t
+
+
+def library():
+    """The built CUDA library; a missing build is an error on a GPU machine, never a skip."""
+    import fp4_expert_layer_b200 as F
+    from fp4_expert_layer_b200 import build
+    build.build()
+    F.lib()
+    return F
+
+
+def make_layer(lw, n_slots=None, max_tokens=1, n_staging=0, table=None, numerics="exact"):
+    F = library()
+    wl = lw.wl
+    S = wl.n_experts if n_slots is None else n_slots
+    layer = F.MoELayer.from_weights(lw, n_slots=S, max_tokens=max_tokens, numerics=numerics,
+                                    n_staging=n_staging)
+    if table is None:
+        table = synth.slot_table(lw, S, policy="all" if S >= wl.n_experts else None)
+    layer.set_slot_table(table)
+    return layer
+
+
+def to_device(x_bits: np.ndarray):
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).cuda().view(t.bfloat16)
+
+
+def run(layer, x_bits):
+    t = torch()
+    y, r = layer.forward(to_device(x_bits), routing=True)
+    t.cuda.synchronize()
+    return y.cpu().numpy(), {k: v.cpu().numpy() for k, v in r.items()}
+
+
+def check_routing(r, lg, ids, gates, E, rows=None):
+    """Bit-exact ids / counts / offsets / perm / inv; logits within 1e-5; gates to fp32 rounding."""
+    T = r["ids"].shape[0]
+    sel = np.arange(T) if rows is None else np.asarray(rows)
+    assert np.array_equal(r["ids"][sel], ids), "expert ids differ from the oracle"
+    dl = np.abs(r["logits"][sel].astype(np.float64) - lg.astype(np.float64)).max()
+    assert dl <= 1e-5, f"router logits differ by {dl}"
+    dg = np.abs(r["gates"][sel].astype(np.float64) - gates.astype(np.float64)).max()
+    assert dg <= 2e-6, f"gates differ by {dg}"
+    if rows is None:
+        counts, offsets, perm, inv = oracle.permute(r["ids"], E)
+        assert np.array_equal(r["counts"], counts)
+        assert np.array_equal(r["offsets"], offsets)
+        assert np.array_equal(r["perm"], perm)
+        assert np.array_equal(r["inv"], inv)
+    return dl
+
+
+def check_output(y, ref):
+    tol = cs.output_tolerance(ref)
+    err = np.abs(y.astype(np.float64) - ref.astype(np.float64))
+    worst = float(err.max())
+    assert np.all(np.isfinite(y)), "non-finite output"
+    assert worst <= tol, f"max |gpu - oracle| = {worst} > {tol}"
+    return worst / max(float(np.abs(ref).max()), 1e-30)
+
+
+def check_routing_invariants(r, T, k, E):
+    """Routing tensors that hold at any size (used where the oracle would be too slow)."""
+    ids = r["ids"]
+    assert ids.min() >= 0 and ids.max() < E
+    assert all(len(set(row)) == k for row in ids.tolist())
+    lg = r["logits"]
+    sel = np.take_along_axis(lg, ids.astype(np.int64), axis=1)
+    assert np.all(np.diff(sel, axis=1) <= 0)
+    assert np.all(lg.max(axis=1) == sel[:, 0])
+    assert np.allclose(r["gates"].sum(axis=1), 1.0, atol=1e-6)
+    counts, offsets, perm, inv = oracle.permute(ids, E)
+    assert np.array_equal(r["counts"], counts) and np.array_equal(r["offsets"], offsets)
+    assert np.array_equal(r["perm"], perm) and np.array_equal(r["inv"], inv)

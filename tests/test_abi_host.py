@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI: no GPU needed, no compute call made."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def F():
+    import fp4_expert_layer_b200 as F
+    from fp4_expert_layer_b200 import build
+    build.build()
+    return F
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ \*]*?\b(moe_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(F):
+    decl = _declared_functions()
+    assert "moe_forward" in decl and "moe_layer_create" in decl
+    L = C.CDLL(F._lib.SO)
+    missing = [n for n in decl if not hasattr(L, n)]
+    assert not missing, missing
+    assert set(F._lib.EXPORTED) <= set(decl)
+
+
+def test_plan_sizes(F):
+    wl = synth.workload("olmoe_like")
+    cfg = F.make_config(wl.hidden, wl.inter, wl.n_experts, wl.top_k, max_tokens=32)
+    p = F.plan(cfg)
+    # codes + scales of one expert, plus one row-reference byte per row, 256-byte aligned pieces
+    assert p["expert_bytes"] >= wl.expert_bytes()
+    assert p["expert_bytes"] - wl.expert_bytes() < 3 * (wl.inter + wl.hidden) + 9 * 256
+    assert p["slot_bytes"] == 64 * p["expert_bytes"]
+    assert p["staging_bytes"] == 0
+    assert p["pinned_bytes"] == 64 * p["expert_bytes"]
+    wl4 = synth.workload("qwen3_8_flash_next_like")
+    cfg4 = F.make_config(wl4.hidden, wl4.inter, wl4.n_experts, wl4.top_k, wl4.shared_inter, "nvfp4",
+                         n_slots=46, max_tokens=8192)
+    p4 = F.plan(cfg4)
+    assert p4["staging_bytes"] == 64 * p4["expert_bytes"]
+    assert p4["expert_bytes"] >= wl4.expert_bytes()
+
+
+@pytest.mark.parametrize("bad, status", [
+    (dict(hidden=300), 1), (dict(inter=100), 1), (dict(n_experts=0), 1), (dict(top_k=0), 1),
+    (dict(top_k=9, n_experts=8), 1), (dict(shared_inter=64), 1), (dict(fmt=7), 1),
+    (dict(renormalize=0), 6), (dict(n_slots=65), 1), (dict(max_tokens=0), 1),
+    (dict(n_slots=10, n_staging=1), 1),
+])
+def test_config_validation(F, bad, status):
+    cfg = F.make_config(2048, 1024, 64, 8, max_tokens=8)
+    for k, v in bad.items():
+        setattr(cfg, k, v)
+    with pytest.raises(F.MoEError) as ei:
+        F.plan(cfg)
+    assert ei.value.status == status
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_admission_rejects_bad_scale_codes(F, fmt):
+    wl = synth.custom_workload(256, 128, 4, 2, fmt=fmt)
+    lw = synth.make_layer(wl, seed=1)
+    cfg = F.make_config(256, 128, 4, 2, fmt=fmt, max_tokens=4)
+    F.admit(cfg, F.weights_from_layer(lw))
+    bad_codes = [0, 255] if fmt == "mxfp4" else [0x7F, 0xFF, 0xB8]
+    for code in bad_codes:
+        lw2 = synth.make_layer(wl, seed=1)
+        lw2.scales[2][3, 5, 1] = code
+        with pytest.raises(F.MoEError) as ei:
+            F.admit(cfg, F.weights_from_layer(lw2))
+        assert ei.value.status == 2
+        assert "expert 3 matrix 2" in str(ei.value)
+    if fmt == "nvfp4":
+        lw3 = synth.make_layer(wl, seed=1)
+        lw3.global_scale[1, 0] = -1.0
+        with pytest.raises(F.MoEError):
+            F.admit(cfg, F.weights_from_layer(lw3))
+
+
+def test_a4_not_silently_substituted(F):
+    cfg = F.make_config(256, 128, 4, 2, numerics="a4", max_tokens=4)
+    try:
+        F.plan(cfg)
+    except F.MoEError as e:       # a build without the A4 path must refuse, never fall back
+        assert e.status == 6

@@ -329,3 +329,16 @@ def test_a4_mode_single_expert_matches_quantised_dense():
         h = (cs.np_silu(a) * u).astype(np.float32)
         ref = Wd @ qdq(h)
         assert np.allclose(y[t], ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
+
+
+def test_expert_rows_sample_sums_to_full_expert():
+    """The benchmark's row-range timing sample adds up to the full expert output."""
+    wl = synth.custom_workload(128, 64, 3, 1)
+    lw = synth.make_layer(wl, seed=6)
+    L = oracle.Layer.from_weights(lw)
+    x = synth.make_tokens(wl, 1, seed=6)
+    y, _, ids, g = L.forward(x)
+    o = np.zeros(128)
+    for i0 in range(0, 64, 16):
+        L.expert_rows(int(ids[0, 0]), x[0], i0, 16, o)
+    assert np.allclose(o.astype(np.float32), y[0], rtol=1e-6, atol=1e-6 * np.abs(y).max())
