@@ -25,7 +25,7 @@ def library():
 def make_layer(lw, n_slots=None, max_tokens=1, n_staging=0, table=None, numerics="exact"):
     F = library()
     wl = lw.wl
-    S = wl.n_experts if n_slots is None else n_slots
+    S = wl.n_slots if n_slots is None else n_slots
     layer = F.MoELayer.from_weights(lw, n_slots=S, max_tokens=max_tokens, numerics=numerics,
                                     n_staging=n_staging)
     if table is None:

@@ -114,6 +114,8 @@ def _paged_case(name, Ts, sample=8):
             rows = np.unique(np.concatenate([[0, T - 1], rng.integers(0, T, sample)]))
             y_ref, *_ = L.forward(x, rows=rows)
             G.check_output(yp[rows], y_ref)
+        assert paged.stats()["misses"] > 0, "the paged layer never staged an expert"
+        assert resident.stats()["misses"] == 0
     finally:
         for l in (paged, resident, few):
             l.close()
