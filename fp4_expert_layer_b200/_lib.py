@@ -23,7 +23,7 @@ NUMERICS = {"exact": 0, "a4": 1}
 
 EXPORTED = ["moe_layer_plan", "moe_admit", "moe_layer_create", "moe_set_slot_table", "moe_forward",
             "moe_forward_host", "moe_get_stats", "moe_destroy", "moe_last_error", "moe_debug_inject",
-            "moe_profile_enable", "moe_profile_read"]
+            "moe_profile_enable", "moe_profile_read", "moe_route_topk_noalloc"]
 
 
 class MoEError(RuntimeError):
@@ -95,6 +95,9 @@ def lib():
         L.moe_debug_inject.argtypes = [C.c_void_p, C.c_int32]
         L.moe_profile_enable.argtypes = [C.c_void_p, C.c_int32]
         L.moe_profile_read.argtypes = [C.c_void_p, C.POINTER(Profile)]
+        L.moe_route_topk_noalloc.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                                             C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
+                                             C.c_void_p]
         for n in EXPORTED:
             f = getattr(L, n)
             if n not in ("moe_destroy", "moe_last_error"):
@@ -155,6 +158,22 @@ def weights_from_layer(lw) -> _HostWeights:
 
 def admit(cfg: Config, hw: _HostWeights):
     check(lib().moe_admit(C.byref(cfg), C.byref(hw.w)))
+
+
+def route_topk_noalloc(x, router_w, router_bias, k, ids, gates, logits=None, stream=None):
+    """Routing alone through the entry point that allocates nothing (see moe_layer.h).
+
+    All arguments are caller-owned torch CUDA tensors: x bf16 [T, H], router_w fp32
+    [E, H], router_bias fp32 [E] or None, ids int32 [T, k], gates fp32 [T, k],
+    logits fp32 [T, E] or None.  For callers that must not allocate device memory
+    when they call in; the library uses its fixed device scratch instead.
+    """
+    T, H = x.shape
+    E = router_w.shape[0]
+    check(lib().moe_route_topk_noalloc(
+        x.data_ptr(), T, H, router_w.data_ptr(), None if router_bias is None else router_bias.data_ptr(),
+        E, k, ids.data_ptr(), gates.data_ptr(), None if logits is None else logits.data_ptr(),
+        _stream_ptr(stream)))
 
 
 def _stream_ptr(stream):

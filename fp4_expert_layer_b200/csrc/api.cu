@@ -30,6 +30,14 @@ static moe_status_t fail(moe_status_t s, const std::string &msg) {
   return s;
 }
 
+namespace moe {
+// Error text for entry points defined in other translation units.
+const char *set_error_text(const std::string &s) {
+  g_err = s;
+  return g_err.c_str();
+}
+}  // namespace moe
+
 #define CUDA_TRY(call)                                                                   \
   do {                                                                                   \
     cudaError_t _e = (call);                                                             \

@@ -205,6 +205,29 @@ typedef struct {
 moe_status_t moe_profile_enable(moe_layer_t layer, int32_t enable);
 moe_status_t moe_profile_read(moe_layer_t layer, moe_profile_t *out);
 
+/* Routing step alone, for callers that cannot allocate device memory when they
+ * call in (a serving loop that plans every byte of HBM once at start-up, or a
+ * latency-critical path that must not pay the device-wide synchronisation of
+ * cudaMalloc/cudaFree).  The pages have no counterpart of this entry point; it
+ * is a library convenience.  Computes, like moe_forward's routing, fp32 logits
+ * x * router_w^T (+ router_bias), the top-k expert ids in descending-logit
+ * order (lower index first on ties) and the softmax gates renormalised over
+ * the k.  Allocates nothing: its scratch (logits and completion counters) is a
+ * fixed file-scope device array of 4 MiB + 64 KiB that every GPU loading this
+ * library holds until exit.  Limits: T * E <= 2^20, T <= 65536, H a multiple of
+ * 4 and at most 14528, E <= 1024, k <= min(E, 32); larger requests return
+ * MOE_ERR_INVALID_ARG.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current, so make the
+ * first call before any stream capture.  All calls share the array and it
+ * keeps the last call's contents (the counters are cleared at every call);
+ * calls that overlap on the GPU race on it and must be serialised by the
+ * caller.  x: device bf16 [T, H]; router_w: device fp32 [E, H]; router_bias:
+ * device fp32 [E] or NULL; ids: device int32 [T, k]; gates: device fp32 [T, k];
+ * logits: device fp32 [T, E] or NULL (copied out of the scratch when given). */
+moe_status_t moe_route_topk_noalloc(const void *x, int32_t T, int32_t H, const float *router_w,
+                                    const float *router_bias, int32_t E, int32_t k, int32_t *ids,
+                                    float *gates, float *logits, void *stream);
+
 /* Waits for the layer's work, then frees everything it holds.  NULL is a no-op. */
 void moe_destroy(moe_layer_t layer);
 
