@@ -9,6 +9,8 @@
 // once, at create time, into the pinned store, so a miss costs one plain
 // cudaMemcpyAsync ("ro99/strata": a per-staging prepack lands on the
 // bottleneck term).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -91,17 +93,21 @@ struct moe_layer {
   uint16_t *shared_w[3] = {};
   uint8_t *slots = nullptr, *staging = nullptr;
   const uint8_t **ptr_resident = nullptr, **ptr_pass = nullptr;
+  int *loc_resident = nullptr, *loc_pass = nullptr;
+  CodeMaps maps{};
+  int *h_err = nullptr, *d_err = nullptr;   // mapped pinned error word (bounded device waits)
   float *logits = nullptr, *gates = nullptr;
   int *ids = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr;
   TileInfo *tiles = nullptr;
   int *n_tiles = nullptr, *active = nullptr, *prow_token = nullptr, *prow_pair = nullptr;
   uint16_t *xf16 = nullptr, *hbuf = nullptr, *sh_h = nullptr, *xin = nullptr;
   float *xs = nullptr, *hscale = nullptr, *oprime = nullptr, *sh_s = nullptr, *yout = nullptr;
-  int *router_counter = nullptr;
+  int *router_counter = nullptr, *tiles_done = nullptr, *comb_cnt = nullptr;
   // host
   uint8_t *store = nullptr;          // pinned: E x blob bytes
   int *h_counts = nullptr;           // pinned [E]
   const uint8_t **h_ptr = nullptr;   // pinned [E]
+  int *h_loc = nullptr;              // pinned [E]
   std::vector<int> slot_of;
   int n_resident = 0;
   size_t max_prows = 0, max_tiles = 0;
@@ -212,7 +218,7 @@ static size_t scratch_bytes(const moe_config_t *c) {
   b += align256(z.max_prows * I * 2) + align256(z.max_prows * (I / kChunk) * 4);
   b += align256(z.P * H * 4);
   if (Is) b += align256(T * Is * 2) + align256(T * H * 4);
-  b += align256(((T + 3) / 4) * 4);
+  b += align256(((T + 3) / 4) * 4) + align256(4) + align256(T * (H / 256) * 4);
   b += align256(T * H * 2) + align256(T * H * 4);
   b += 2 * align256(E * sizeof(void *));
   return b;
@@ -249,6 +255,8 @@ static void free_layer(moe_layer *L) {
   if (L->store) cudaFreeHost(L->store);
   if (L->h_counts) cudaFreeHost(L->h_counts);
   if (L->h_ptr) cudaFreeHost(L->h_ptr);
+  if (L->h_err) cudaFreeHost(L->h_err);
+  if (L->h_loc) cudaFreeHost(L->h_loc);
   for (int i = 0; i < 2; ++i) {
     if (L->ev_copied[i]) cudaEventDestroy(L->ev_copied[i]);
     if (L->ev_done[i]) cudaEventDestroy(L->ev_done[i]);
@@ -259,6 +267,40 @@ static void free_layer(moe_layer *L) {
   for (auto e : L->evpool) cudaEventDestroy(e);
   if (L->side) cudaStreamDestroy(L->side);
   delete L;
+}
+
+// ------------------------------------------------------------------ tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D map over the code bytes of matrix m of every blob in a region:
+// (K/2 bytes, rows, blob index), box 64 bytes x box_rows x 1, no swizzle.
+static moe_status_t make_code_map(CUtensorMap *map, const uint8_t *region, int nblobs, const BlobLayout &L, int m,
+                                  int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)(L.K[m] / 2), (cuuint64_t)L.rows[m], (cuuint64_t)nblobs};
+  cuuint64_t strides[2] = {(cuuint64_t)(L.K[m] / 2), (cuuint64_t)L.bytes};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void *)(region + L.codes[m]), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[96];
+    snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (%d) for matrix %d", (int)r, m);
+    return fail(MOE_ERR_CUDA, buf);
+  }
+  return MOE_OK;
 }
 
 // ------------------------------------------------------------------ C ABI
@@ -324,7 +366,13 @@ static void pack_expert(const moe_config_t *cfg, const BlobLayout &L, const moe_
     const size_t ncode = (size_t)L.rows[m] * L.K[m] / 2;
     const size_t nsc = (size_t)L.rows[m] * L.K[m] / L.G;
     memcpy(dst + L.codes[m], w->codes[m][e], ncode);
-    memcpy(dst + L.scales[m], w->scales[m][e], nsc);
+    {
+      const int nsf = L.K[m] / L.G;
+      const uint8_t *src = w->scales[m][e];
+      for (int r = 0; r < L.rows[m]; ++r)
+        for (int c = 0; c < nsf; ++c) dst[L.scales[m] + sf_offset(nsf, r, c)] = src[(size_t)r * nsf + c];
+    }
+    (void)nsc;
     if (cfg->fmt == MOE_FMT_MXFP4) {
       const int per = L.K[m] / L.G;
       const uint8_t *s = w->scales[m][e];
@@ -393,7 +441,9 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     for (auto &x : th) x.join();
   }
   if (cudaHostAlloc((void **)&L->h_counts, sizeof(int) * E, cudaHostAllocDefault) != cudaSuccess ||
-      cudaHostAlloc((void **)&L->h_ptr, sizeof(void *) * E, cudaHostAllocDefault) != cudaSuccess) {
+      cudaHostAlloc((void **)&L->h_ptr, sizeof(void *) * E, cudaHostAllocDefault) != cudaSuccess ||
+      cudaHostAlloc((void **)&L->h_loc, sizeof(int) * E, cudaHostAllocDefault) != cudaSuccess ||
+      cudaHostAlloc((void **)&L->h_err, sizeof(int), cudaHostAllocMapped) != cudaSuccess) {
     (void)cudaGetLastError();
     return bail(fail(MOE_ERR_OOM, "pinned host allocation failed"));
   }
@@ -406,6 +456,8 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   if (L->n_staging) C_TRY(dalloc(L, &L->staging, bytes * L->n_staging));
   C_TRY(dalloc(L, &L->ptr_resident, sizeof(void *) * E));
   C_TRY(dalloc(L, &L->ptr_pass, sizeof(void *) * E));
+  C_TRY(dalloc(L, &L->loc_resident, sizeof(int) * E));
+  C_TRY(dalloc(L, &L->loc_pass, sizeof(int) * E));
   C_TRY(dalloc(L, &L->logits, T * E * 4));
   C_TRY(dalloc(L, &L->ids, z.P * 4));
   C_TRY(dalloc(L, &L->gates, z.P * 4));
@@ -428,12 +480,25 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     C_TRY(dalloc(L, &L->sh_s, T * H * 4));
   }
   C_TRY(dalloc(L, &L->router_counter, ((T + 3) / 4) * 4));
+  C_TRY(dalloc(L, &L->tiles_done, 4));
+  C_TRY(dalloc(L, &L->comb_cnt, T * (H / 256) * 4));
   C_TRY(dalloc(L, &L->xin, T * H * 2));
   C_TRY(dalloc(L, &L->yout, T * H * 4));
 
   C_CUDA(cudaMemsetAsync(L->router_counter, 0, ((T + 3) / 4) * 4, s));
+  C_CUDA(cudaMemsetAsync(L->tiles_done, 0, 4, s));
+  C_CUDA(cudaMemsetAsync(L->comb_cnt, 0, T * (H / 256) * 4, s));
   C_CUDA(cudaMemsetAsync(L->ptr_resident, 0, sizeof(void *) * E, s));
   C_CUDA(cudaMemsetAsync(L->ptr_pass, 0, sizeof(void *) * E, s));
+  C_CUDA(cudaMemsetAsync(L->loc_resident, 0xFF, sizeof(int) * E, s));   // -1: absent
+  C_CUDA(cudaMemsetAsync(L->loc_pass, 0xFF, sizeof(int) * E, s));
+  *L->h_err = 0;
+  C_CUDA(cudaHostGetDevicePointer((void **)&L->d_err, L->h_err, 0));
+  for (int m = 0; m < 3; ++m) {
+    const int box_rows = m < 2 ? 128 : 256;
+    if (cfg->n_slots) C_TRY(make_code_map(&L->maps.slot[m], L->slots, cfg->n_slots, L->L, m, box_rows));
+    if (L->n_staging) C_TRY(make_code_map(&L->maps.stage[m], L->staging, L->n_staging, L->L, m, box_rows));
+  }
   C_CUDA(cudaMemcpyAsync(L->router_w, w->router_w, (size_t)E * H * 4, cudaMemcpyHostToDevice, s));
   if (w->router_bias) C_CUDA(cudaMemcpyAsync(L->router_b, w->router_bias, (size_t)E * 4, cudaMemcpyHostToDevice, s));
   if (Is)
@@ -494,8 +559,10 @@ moe_status_t moe_set_slot_table(moe_layer_t L, const int32_t *table, void *strea
       CUDA_TRY(cudaMemcpyAsync(L->slots + (size_t)s * bytes, L->store + (size_t)e * bytes, bytes,
                                cudaMemcpyHostToDevice, st));
     L->h_ptr[e] = s >= 0 ? L->slots + (size_t)s * bytes : nullptr;
+    L->h_loc[e] = s >= 0 ? s : kLocAbsent;
   }
   CUDA_TRY(cudaMemcpyAsync(L->ptr_resident, L->h_ptr, sizeof(void *) * E, cudaMemcpyHostToDevice, st));
+  CUDA_TRY(cudaMemcpyAsync(L->loc_resident, L->h_loc, sizeof(int) * E, cudaMemcpyHostToDevice, st));
   CUDA_TRY(cudaStreamSynchronize(st));
   for (int e = 0; e < E; ++e) L->slot_of[e] = table[e];
   L->n_resident = n;
@@ -508,11 +575,15 @@ static int pick_split(int est_ctas, int nck) {
   return cs;
 }
 
-static moe_status_t run_experts(moe_layer *L, const uint8_t *const *ptrs, int nt, int grid_tiles,
-                                int cs_gu, int cs_dn, cudaStream_t s) {
+static moe_status_t run_experts(moe_layer *L, const int *locs, int nt, int grid_tiles, int cs_gu, int cs_dn,
+                                float *y, cudaStream_t s) {
   const moe_config_t &c = L->cfg;
-  ExpertArgs a{};
-  a.expert_ptr = ptrs;
+  TmaExpertArgs a{};
+  a.maps = L->maps;
+  a.loc = locs;
+  a.slots = L->slots;
+  a.staging = L->staging;
+  a.blob_bytes = L->L.bytes;
   a.L = L->L;
   a.tile_tokens = 8 * nt;
   a.tiles = L->tiles;
@@ -520,6 +591,11 @@ static moe_status_t run_experts(moe_layer *L, const uint8_t *const *ptrs, int nt
   a.prow_token = L->prow_token;
   a.prow_pair = L->prow_pair;
   a.gates = L->gates;
+  a.err = L->d_err;
+  a.y = y;
+  a.shared = c.shared_inter ? L->sh_s : nullptr;
+  a.comb_cnt = L->comb_cnt;
+  a.top_k = c.top_k;
   // gate/up + SwiGLU
   a.K = c.hidden;
   a.rows = c.inter;
@@ -530,7 +606,7 @@ static moe_status_t run_experts(moe_layer *L, const uint8_t *const *ptrs, int nt
   a.h_out = L->hbuf;
   a.h_scale = L->hscale;
   StageTimer t3(L, 3, s);
-  launch_expert(L->wf, MODE_GATEUP, nt, a, grid_tiles, s);
+  launch_expert_tma(L->wf, MODE_GATEUP, nt, a, grid_tiles, s);
   CUDA_TRY(cudaGetLastError());
   t3.launched(1);
   t3.end();
@@ -543,7 +619,7 @@ static moe_status_t run_experts(moe_layer *L, const uint8_t *const *ptrs, int nt
   a.act_scale = L->hscale;
   a.o_out = L->oprime;
   StageTimer t4(L, 4, s);
-  launch_expert(L->wf, MODE_DOWN, nt, a, grid_tiles, s);
+  launch_expert_tma(L->wf, MODE_DOWN, nt, a, grid_tiles, s);
   CUDA_TRY(cudaGetLastError());
   t4.launched(1);
   t4.end();
@@ -557,6 +633,13 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   if (T < 0 || T > c.max_tokens) return fail(MOE_ERR_INVALID_ARG, "T out of range [0, max_tokens]");
   if (T == 0) return MOE_OK;
   if (!x || !y) return fail(MOE_ERR_INVALID_ARG, "x or y is NULL");
+  if (*(volatile int *)L->h_err != 0) {
+    char buf[128];
+    snprintf(buf, sizeof buf, "a device-side wait of an earlier forward gave up (code %d); outputs of that "
+             "forward are invalid", *(volatile int *)L->h_err);
+    *(volatile int *)L->h_err = 0;
+    return fail(MOE_ERR_CUDA, buf);
+  }
   CUDA_TRY(cudaSetDevice(c.device));
   cudaStream_t s = (cudaStream_t)stream;
   const int E = c.n_experts, k = c.top_k, H = c.hidden, I = c.inter, Is = c.shared_inter;
@@ -574,22 +657,28 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   ra.w = L->router_w; ra.bias = L->router_b;
   ra.logits = L->logits; ra.ids = L->ids; ra.gates = L->gates;
   ra.xf16 = L->xf16; ra.xs = L->xs; ra.counter = L->router_counter;
-  StageTimer t0(L, 0, s);
-  launch_router(ra, s);
-  CUDA_TRY(cudaGetLastError());
-  t0.launched(1);
-  t0.end();
-
   PermArgs pa{};
   pa.ids = L->ids; pa.n_pairs = P; pa.E = E; pa.k = k; pa.tile_tokens = ts;
   pa.counts = L->counts; pa.offsets = L->offsets; pa.perm = L->perm; pa.inv = L->inv;
   pa.tiles = L->tiles; pa.n_tiles = L->n_tiles; pa.prow_token = L->prow_token;
   pa.prow_pair = L->prow_pair; pa.active = L->active;
-  StageTimer t1(L, 1, s);
-  launch_permute(pa, s);
+  // decode-sized batches: the router's last CTA also runs the permutation
+  const bool fuse_perm = P <= 2048;
+  ra.fuse_perm = fuse_perm ? 1 : 0;
+  ra.tiles_done = L->tiles_done;
+  ra.perm = pa;
+  StageTimer t0(L, 0, s);
+  launch_router(ra, s);
   CUDA_TRY(cudaGetLastError());
-  t1.launched(1);
-  t1.end();
+  t0.launched(1);
+  t0.end();
+  if (!fuse_perm) {
+    StageTimer t1(L, 1, s);
+    launch_permute(pa, s);
+    CUDA_TRY(cudaGetLastError());
+    t1.launched(1);
+    t1.end();
+  }
 
   if (dbg) {
     if (dbg->logits) CUDA_TRY(cudaMemcpyAsync(dbg->logits, L->logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
@@ -639,7 +728,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   const int cs_dn = pick_split(act_est * (H / 256), I / 128);
   int waves = 0, misses_n = 0;
   if (resident) {
-    ST_TRY(run_experts(L, L->ptr_resident, nt, grid_tiles, cs_gu, cs_dn, s));
+    ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
   } else {
     CUDA_TRY(cudaEventSynchronize(L->ev_counts));
     std::vector<int> misses;
@@ -654,7 +743,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     misses_n = (int)misses.size();
     const int NS = L->n_staging;
     if (misses.empty()) {
-      ST_TRY(run_experts(L, L->ptr_resident, nt, grid_tiles, cs_gu, cs_dn, s));
+      ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
     } else {
       const bool one = misses_n <= NS;
       const int wave_sz = one ? NS : NS / 2;
@@ -670,7 +759,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
         const int half = one ? 0 : (w & 1);
         const int base = one ? 0 : half * (NS / 2);
         if (!one && w >= 2) CUDA_TRY(cudaStreamWaitEvent(L->side, L->ev_done[half], 0));
-        PtrUpdate u{};
+        LocUpdate u{};
         u.E = E;
         u.keep_resident = (w == 0);
         const int b0 = w * wave_sz, b1 = std::min(misses_n, b0 + wave_sz);
@@ -679,17 +768,17 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
           uint8_t *dst = L->staging + (size_t)(base + (i - b0)) * bytes;
           CUDA_TRY(cudaMemcpyAsync(dst, L->store + (size_t)e * bytes, bytes, cudaMemcpyHostToDevice, L->side));
           u.expert[u.n] = e;
-          u.ptr[u.n] = dst;
+          u.loc[u.n] = loc_staging(base + (i - b0));
           ++u.n;
         }
         CUDA_TRY(cudaEventRecord(L->ev_copied[half], L->side));
         StageTimer t6(L, 6, s);
         CUDA_TRY(cudaStreamWaitEvent(s, L->ev_copied[half], 0));
-        launch_ptr_update(u, L->ptr_resident, L->ptr_pass, s);
+        launch_loc_update(u, L->loc_resident, L->loc_pass, s);
         CUDA_TRY(cudaGetLastError());
         t6.launched(1);
         t6.end();
-        ST_TRY(run_experts(L, L->ptr_pass, nt, grid_tiles, cs_gu, cs_dn, s));
+        ST_TRY(run_experts(L, L->loc_pass, nt, grid_tiles, cs_gu, cs_dn, y, s));
         if (!one) CUDA_TRY(cudaEventRecord(L->ev_done[half], s));
       }
       CUDA_TRY(cudaEventRecord(L->ev_fwd_done, s));
@@ -700,16 +789,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     }
   }
 
-  CombineArgs ca{};
-  ca.oprime = L->oprime;
-  ca.shared = Is ? L->sh_s : nullptr;
-  ca.y = y;
-  ca.T = T; ca.H = H; ca.k = k;
-  StageTimer t5(L, 5, s);
-  launch_combine(ca, s);
-  CUDA_TRY(cudaGetLastError());
-  t5.launched(1);
-  t5.end();
+  // the ordered combine runs inside the routed down pass (last arrival per token)
   t7.end();
   if (L->prof) L->prof_acc.forwards += 1;
 

@@ -414,18 +414,12 @@ static cudaError_t launch_nt(int nt, const ExpertArgs &a, int grid_tiles, cudaSt
   }
 }
 
+// Only the dense bf16 (shared expert) path is instantiated here; routed FP4
+// experts run in the TMA-fed kernels of expert_tma.cu.
 void launch_expert(int wf, int mode, int nt, const ExpertArgs &a, int grid_tiles, cudaStream_t s) {
-  if (grid_tiles <= 0) return;
-  if (wf == WF_MX) {
-    if (mode == MODE_GATEUP) launch_nt<WF_MX, MODE_GATEUP>(nt, a, grid_tiles, s);
-    else launch_nt<WF_MX, MODE_DOWN>(nt, a, grid_tiles, s);
-  } else if (wf == WF_NV) {
-    if (mode == MODE_GATEUP) launch_nt<WF_NV, MODE_GATEUP>(nt, a, grid_tiles, s);
-    else launch_nt<WF_NV, MODE_DOWN>(nt, a, grid_tiles, s);
-  } else {
-    if (mode == MODE_GATEUP) launch_nt<WF_BF16, MODE_GATEUP>(nt, a, grid_tiles, s);
-    else launch_nt<WF_BF16, MODE_DOWN>(nt, a, grid_tiles, s);
-  }
+  if (grid_tiles <= 0 || wf != WF_BF16) return;
+  if (mode == MODE_GATEUP) launch_nt<WF_BF16, MODE_GATEUP>(nt, a, grid_tiles, s);
+  else launch_nt<WF_BF16, MODE_DOWN>(nt, a, grid_tiles, s);
 }
 
 }  // namespace moe

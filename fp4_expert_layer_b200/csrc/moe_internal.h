@@ -1,6 +1,7 @@
 // moe_internal.h -- internal interfaces of the sm_100a MoE layer library.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -16,8 +17,10 @@ constexpr int kMaxTopK = 32;
 constexpr int kPermThreads = 512;
 constexpr int kPtrListMax = 256;   // expert pointers one table-update launch can carry
 
-// Device layout of one routed expert ("blob"): the checkpoint bytes of the three
-// matrices (codes unchanged, block scales unchanged) plus, for MXFP4, one byte
+// Device layout of one routed expert ("blob"): the checkpoint code bytes of the
+// three matrices unchanged, the block scales rearranged into 512-byte blocks of
+// 128 rows x 4 scale columns (the scale-factor block the sm_100 block-scaled MMA
+// reads through tcgen05.cp; see sf_offset), plus, for MXFP4, one byte
 // per row holding the row's largest E8M0 code (the row reference exponent the
 // decode kernels fold out of the f16 operand), or, for NVFP4, the three fp32
 // per-tensor scales.  Every piece starts on a 256-byte boundary.  The pinned
@@ -37,6 +40,20 @@ struct BlobLayout {
 
 BlobLayout blob_layout(int H, int I, int fmt);
 
+// Byte offset of scale (row r, scale column col) inside a matrix's scale area
+// with nsf scale columns per row: blocks of 128 rows x 4 columns (512 bytes),
+// ordered row-block-major; inside a block, row r sits at 16*(r%32) + 4*((r%128)/32)
+// and its 4 columns are consecutive bytes.
+__host__ __device__ inline size_t sf_offset(int nsf, int r, int col) {
+  return ((size_t)(r >> 7) * (size_t)(nsf >> 2) + (size_t)(col >> 2)) * 512u + 16u * (r & 31) +
+         4u * ((r & 127) >> 5) + (col & 3);
+}
+
+// Where an expert's blob lives for one pass: >= 0 resident slot, <= -2 staging
+// buffer (-2 - index), -1 not available in this pass.
+constexpr int kLocAbsent = -1;
+__host__ __device__ inline int loc_staging(int i) { return -2 - i; }
+
 // One token tile of one expert: rows [prow0, prow0 + nrows) of the padded,
 // expert-sorted activation order; each expert's rows start on a multiple of 8.
 struct TileInfo {
@@ -47,20 +64,6 @@ struct TileInfo {
 };
 
 // ------------------------------------------------------------------ routing
-struct RouterArgs {
-  const uint16_t *x;     // bf16 [T, H]
-  int T, H, E, k;
-  const float *w;        // [E, H]
-  const float *bias;     // [E] or null
-  float *logits;         // [T, E]
-  int *ids;              // [T, k]
-  float *gates;          // [T, k]
-  uint16_t *xf16;        // f16 [T, H], chunk-scaled
-  float *xs;             // [T, H/128] chunk multipliers
-  int *counter;          // [ceil(T/TT)] zero-initialised completion counters
-};
-void launch_router(const RouterArgs &a, cudaStream_t s);
-
 struct PermArgs {
   const int *ids;        // [T*k]
   int n_pairs, E, k, tile_tokens;
@@ -74,6 +77,23 @@ struct PermArgs {
   int *prow_pair;        // [max prows]
   int *active;           // [1] experts with >= 1 pair
 };
+struct RouterArgs {
+  const uint16_t *x;     // bf16 [T, H]
+  int T, H, E, k;
+  const float *w;        // [E, H]
+  const float *bias;     // [E] or null
+  float *logits;         // [T, E]
+  int *ids;              // [T, k]
+  float *gates;          // [T, k]
+  uint16_t *xf16;        // f16 [T, H], chunk-scaled
+  float *xs;             // [T, H/128] chunk multipliers
+  int *counter;          // [ceil(T/TT)] zero-initialised completion counters
+  int fuse_perm;         // 1: the last token tile also runs the permutation
+  int *tiles_done;       // [1] zero-initialised second-level counter
+  PermArgs perm;         // permutation arguments (fuse_perm only)
+};
+void launch_router(const RouterArgs &a, cudaStream_t s);
+
 void launch_permute(const PermArgs &a, cudaStream_t s);
 
 // ------------------------------------------------------------------ experts
@@ -126,5 +146,50 @@ struct PtrUpdate {
 };
 void launch_ptr_update(const PtrUpdate &u, const uint8_t *const *resident, const uint8_t **out,
                        cudaStream_t s);
+
+// ------------------------------------------------------------------ TMA-fed routed experts
+struct LocUpdate {
+  int n;
+  int keep_resident;
+  int E;
+  int expert[kPtrListMax];
+  int loc[kPtrListMax];
+};
+void launch_loc_update(const LocUpdate &u, const int *resident, int *out, cudaStream_t s);
+
+// Tensor maps over the code bytes of one matrix for every blob of a region
+// (3-D: K/2 bytes, rows, blob index), box = 64 bytes x (128 or 256) rows.
+struct CodeMaps {
+  CUtensorMap slot[3];
+  CUtensorMap stage[3];
+};
+
+struct TmaExpertArgs {
+  CodeMaps maps;
+  const int *loc;          // [E]
+  const uint8_t *slots;    // slot pool base
+  const uint8_t *staging;  // staging ring base
+  size_t blob_bytes;
+  BlobLayout L;
+  int K, rows, n_rowblocks, k_split, tile_tokens;
+  const TileInfo *tiles;
+  const int *n_tiles;
+  const int *prow_token;
+  const int *prow_pair;
+  const float *gates;
+  const uint16_t *act;
+  const float *act_scale;
+  uint16_t *h_out;
+  float *h_scale;
+  float *o_out;
+  int *err;                // device-visible error word (bounded waits)
+  // fused ordered combine (down pass): the last of a token's k contributions to
+  // a 256-row block writes y = sum_j O'[t*k + j] (j order) + shared[t]
+  float *y;
+  const float *shared;     // [T, H] or null
+  int *comb_cnt;           // [max_tokens, H/256] zero-initialised arrival counters
+  int top_k;
+};
+void launch_expert_tma(int wf, int mode, int nt, const TmaExpertArgs &a, int grid_tiles, cudaStream_t s);
 
 }  // namespace moe

@@ -9,6 +9,8 @@
 // over the chosen k, which equals softmax over all E renormalised to the k.
 #include <cooperative_groups.h>
 
+#include <algorithm>
+
 #include "device_utils.cuh"
 #include "moe_internal.h"
 
@@ -17,12 +19,149 @@ namespace moe {
 constexpr int kRouterTT = 4;      // tokens per router CTA
 constexpr int kRouterEB = 8;      // experts per router CTA (one per warp)
 
-// grid (ceil(T/TT), ceil(E/EB)), 256 threads, dynamic smem TT*H floats.
-// Each CTA computes logits for its TT tokens x EB experts; the CTA with
-// blockIdx.y == 0 also writes the chunk-scaled f16 copy of its tokens; the last
-// CTA of a token tile to finish (completion counter) runs top-k for the tile.
+// ---------------------------------------------------------------------------
+// Permutation: stable counting sort of pair index p = t*k + j by expert, as a
+// block-level routine (NTH threads, `sm` = shared scratch of
+// (5E + 3 + (NTH/32)*E) ints).  Counts by shared-memory atomics, offsets /
+// padded offsets / tile offsets by one block scan, then pairs are placed in
+// chunks of NTH: ranks inside a chunk come from warp match plus per-warp counts
+// scanned in warp order, so equal experts keep ascending p (stable).
+// ---------------------------------------------------------------------------
+template <int NTH>
+__device__ void permute_block(const PermArgs &a, int *sm) {
+  constexpr int W = NTH / 32;
+  __shared__ int4 wsum[W];
+  const int E = a.E;
+  int *cnt = sm;                  // [E]
+  int *cursor = cnt + E;          // [E]
+  int *off = cursor + E;          // [E+1]
+  int *poff = off + E + 1;        // [E+1] padded (multiple of 8) offsets
+  int *toff = poff + E + 1;       // [E+1] tile offsets
+  int *wcnt = toff + E + 1;       // [W][E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int i = tid; i < E; i += NTH) { cnt[i] = 0; cursor[i] = 0; }
+  for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;
+  __syncthreads();
+  for (int p = tid; p < a.n_pairs; p += NTH) atomicAdd(&cnt[__ldcg(a.ids + p)], 1);
+  __syncthreads();
+
+  // block exclusive scan of (count, padded count, tiles, active) over experts
+  const int per = (E + NTH - 1) / NTH;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+  int4 v = make_int4(0, 0, 0, 0);
+  for (int e = e0; e < e1; ++e) {
+    const int c = cnt[e];
+    v.x += c;
+    v.y += (c + 7) & ~7;
+    v.z += (c + a.tile_tokens - 1) / a.tile_tokens;
+    v.w += c > 0;
+  }
+  int4 inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int4 t;
+    t.x = __shfl_up_sync(0xffffffffu, inc.x, o);
+    t.y = __shfl_up_sync(0xffffffffu, inc.y, o);
+    t.z = __shfl_up_sync(0xffffffffu, inc.z, o);
+    t.w = __shfl_up_sync(0xffffffffu, inc.w, o);
+    if (lane >= o) { inc.x += t.x; inc.y += t.y; inc.z += t.z; inc.w += t.w; }
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int4 w = lane < W ? wsum[lane] : make_int4(0, 0, 0, 0);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int4 t;
+      t.x = __shfl_up_sync(0xffffffffu, w.x, o);
+      t.y = __shfl_up_sync(0xffffffffu, w.y, o);
+      t.z = __shfl_up_sync(0xffffffffu, w.z, o);
+      t.w = __shfl_up_sync(0xffffffffu, w.w, o);
+      if (lane >= o) { w.x += t.x; w.y += t.y; w.z += t.z; w.w += t.w; }
+    }
+    if (lane < W) wsum[lane] = w;
+  }
+  __syncthreads();
+  {
+    const int4 pre = warp > 0 ? wsum[warp - 1] : make_int4(0, 0, 0, 0);
+    int o = pre.x + inc.x - v.x, po = pre.y + inc.y - v.y, to = pre.z + inc.z - v.z;
+    for (int e = e0; e < e1; ++e) {
+      const int c = cnt[e];
+      off[e] = o; poff[e] = po; toff[e] = to;
+      o += c;
+      po += (c + 7) & ~7;
+      to += (c + a.tile_tokens - 1) / a.tile_tokens;
+    }
+    if (tid == NTH - 1) {
+      const int4 tot = wsum[W - 1];
+      off[E] = tot.x; poff[E] = tot.y; toff[E] = tot.z;
+      *a.n_tiles = tot.z;
+      *a.active = tot.w;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e <= E; e += NTH) a.offsets[e] = off[e];
+  for (int e = tid; e < E; e += NTH) {
+    const int c = cnt[e];
+    a.counts[e] = c;
+    const int nt = (c + a.tile_tokens - 1) / a.tile_tokens;
+    for (int i = 0; i < nt; ++i) {
+      TileInfo ti;
+      ti.expert = e;
+      ti.prow0 = poff[e] + i * a.tile_tokens;
+      ti.nrows = min(a.tile_tokens, c - i * a.tile_tokens);
+      ti.sorted0 = off[e] + i * a.tile_tokens;
+      a.tiles[toff[e] + i] = ti;
+    }
+    for (int r = poff[e] + c; r < poff[e + 1]; ++r) { a.prow_token[r] = -1; a.prow_pair[r] = -1; }
+  }
+
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < a.n_pairs; base += NTH) {
+    const int p = base + tid;
+    const bool valid = p < a.n_pairs;
+    const int e = valid ? __ldcg(a.ids + p) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    if (valid && rank == 0) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += NTH) {
+      int run = cursor[ee];
+      for (int w = 0; w < W; ++w) {
+        const int c = wcnt[w * E + ee];
+        wcnt[w * E + ee] = run;
+        run += c;
+      }
+      cursor[ee] = run;
+    }
+    __syncthreads();
+    if (valid) {
+      const int local = wcnt[warp * E + e] + rank;
+      const int pos = off[e] + local;
+      const int prow = poff[e] + local;
+      a.perm[pos] = p;
+      a.inv[p] = pos;
+      a.prow_token[prow] = p / a.k;
+      a.prow_pair[prow] = p;
+    }
+    __syncthreads();
+    for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;
+    __syncthreads();
+  }
+}
+
+__host__ __device__ inline size_t perm_smem_ints(int E, int nth) { return (size_t)5 * E + 3 + (size_t)(nth / 32) * E; }
+
+// grid (ceil(T/TT), ceil(E/EB)), 256 threads.  Each CTA computes logits for
+// its TT tokens x EB experts; the CTA with blockIdx.y == 0 also writes the
+// chunk-scaled f16 copy of its tokens; the last CTA of a token tile to finish
+// (completion counter) runs top-k for the tile; with fuse_perm, the last of
+// those (second counter) runs the permutation for the whole batch.
+// KPER = experts per lane in the top-k scan (E <= 32 * KPER).
+template <int KPER>
 __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
-  extern __shared__ float xs_smem[];   // [TT][H]
+  extern __shared__ float xs_smem[];   // [TT][H], reused by the fused permutation
   __shared__ int is_last;
   const int H = a.H, E = a.E;
   const int t0 = blockIdx.x * kRouterTT;
@@ -45,16 +184,28 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
 #pragma unroll
     for (int t = 0; t < kRouterTT; ++t) acc[t] = 0.0f;
     const float *w = a.w + (size_t)e * H;
-    for (int h = lane * 4; h < H; h += 128) {
-      float4 wv = *reinterpret_cast<const float4 *>(w + h);
+    // 8 independent 16-byte loads in flight per lane before any use
+    for (int h0 = lane * 4; h0 < H; h0 += 128 * 8) {
+      float4 wv[8];
 #pragma unroll
-      for (int t = 0; t < kRouterTT; ++t) {
-        if (t < nt) {
-          const float4 xv = *reinterpret_cast<const float4 *>(xs_smem + t * H + h);
-          acc[t] = fmaf(wv.x, xv.x, acc[t]);
-          acc[t] = fmaf(wv.y, xv.y, acc[t]);
-          acc[t] = fmaf(wv.z, xv.z, acc[t]);
-          acc[t] = fmaf(wv.w, xv.w, acc[t]);
+      for (int u = 0; u < 8; ++u) {
+        const int h = h0 + u * 128;
+        wv[u] = h < H ? __ldg(reinterpret_cast<const float4 *>(w + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int h = h0 + u * 128;
+        if (h < H) {
+#pragma unroll
+          for (int t = 0; t < kRouterTT; ++t) {
+            if (t < nt) {
+              const float4 xv = *reinterpret_cast<const float4 *>(xs_smem + t * H + h);
+              acc[t] = fmaf(wv[u].x, xv.x, acc[t]);
+              acc[t] = fmaf(wv[u].y, xv.y, acc[t]);
+              acc[t] = fmaf(wv[u].z, xv.z, acc[t]);
+              acc[t] = fmaf(wv[u].w, xv.w, acc[t]);
+            }
+          }
         }
       }
     }
@@ -104,11 +255,10 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
   const int k = a.k;
   if (warp < nt) {
     const int t = t0 + warp;
-    constexpr int kPer = kMaxExperts / 32;
-    float lv[kPer];
+    float lv[KPER];
     const float *lrow = a.logits + (size_t)t * E;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
+    for (int i = 0; i < KPER; ++i) {
       const int ee = lane + 32 * i;
       lv[i] = (ee < E) ? __ldcg(lrow + ee) : -INFINITY;
     }
@@ -120,7 +270,7 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
+      for (int i = 0; i < KPER; ++i) {
         const int ee = lane + 32 * i;
         if (ee < E && !((taken >> i) & 1u)) {
           if (bi == 0x7fffffff || lv[i] > bv) { bv = lv[i]; bi = ee; }
@@ -147,109 +297,43 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
       a.gates[(size_t)t * k + lane] = ex / den;
     }
   }
+  if (!a.fuse_perm) return;
+
+  // the last token tile to finish top-k runs the permutation
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(a.tiles_done, 1) == (int)gridDim.x - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (threadIdx.x == 0) *a.tiles_done = 0;
+  permute_block<256>(a.perm, reinterpret_cast<int *>(xs_smem));
+}
+
+template <int KPER>
+static void launch_router_k(const RouterArgs &a, cudaStream_t s) {
+  dim3 grid((a.T + kRouterTT - 1) / kRouterTT, (a.E + kRouterEB - 1) / kRouterEB);
+  size_t smem = (size_t)kRouterTT * a.H * sizeof(float);
+  if (a.fuse_perm) smem = std::max(smem, perm_smem_ints(a.E, 256) * sizeof(int));
+  if (smem > 48 * 1024) cudaFuncSetAttribute(router_kernel<KPER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  router_kernel<KPER><<<grid, 256, smem, s>>>(a);
 }
 
 void launch_router(const RouterArgs &a, cudaStream_t s) {
-  dim3 grid((a.T + kRouterTT - 1) / kRouterTT, (a.E + kRouterEB - 1) / kRouterEB);
-  const size_t smem = (size_t)kRouterTT * a.H * sizeof(float);
-  if (smem > 48 * 1024) cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  router_kernel<<<grid, 256, smem, s>>>(a);
+  if (a.E <= 64) launch_router_k<2>(a, s);
+  else if (a.E <= 128) launch_router_k<4>(a, s);
+  else if (a.E <= 256) launch_router_k<8>(a, s);
+  else if (a.E <= 512) launch_router_k<16>(a, s);
+  else launch_router_k<32>(a, s);
 }
 
-// ---------------------------------------------------------------------------
-// Permutation: stable counting sort of pair index p = t*k + j by expert.
-// Single CTA; pairs are processed in chunks of blockDim, ranks inside a chunk
-// from warp match + per-warp counts scanned in warp order, so the order of
-// equal experts is ascending p (stable).
-// ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const PermArgs a) {
   extern __shared__ int psm[];
-  const int E = a.E;
-  constexpr int W = kPermThreads / 32;
-  int *cnt = psm;                 // [E]
-  int *cursor = cnt + E;          // [E]
-  int *poff = cursor + E;         // [E+1] padded offsets
-  int *toff = poff + E + 1;       // [E+1] tile offsets
-  int *wcnt = toff + E + 1;       // [W][E]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  for (int i = tid; i < E; i += blockDim.x) { cnt[i] = 0; cursor[i] = 0; }
-  for (int i = tid; i < W * E; i += blockDim.x) wcnt[i] = 0;
-  __syncthreads();
-  for (int p = tid; p < a.n_pairs; p += blockDim.x) atomicAdd(&cnt[a.ids[p]], 1);
-  __syncthreads();
-  if (tid == 0) {
-    int o = 0, po = 0, to = 0, act = 0;
-    for (int e = 0; e < E; ++e) {
-      const int c = cnt[e];
-      a.offsets[e] = o;
-      poff[e] = po;
-      toff[e] = to;
-      o += c;
-      po += (c + 7) & ~7;
-      to += (c + a.tile_tokens - 1) / a.tile_tokens;
-      act += c > 0;
-    }
-    a.offsets[E] = o;
-    poff[E] = po;
-    toff[E] = to;
-    *a.n_tiles = to;
-    *a.active = act;
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) {
-    const int c = cnt[e];
-    a.counts[e] = c;
-    const int nt = (c + a.tile_tokens - 1) / a.tile_tokens;
-    for (int i = 0; i < nt; ++i) {
-      TileInfo ti;
-      ti.expert = e;
-      ti.prow0 = poff[e] + i * a.tile_tokens;
-      ti.nrows = min(a.tile_tokens, c - i * a.tile_tokens);
-      ti.sorted0 = a.offsets[e] + i * a.tile_tokens;
-      a.tiles[toff[e] + i] = ti;
-    }
-    for (int r = poff[e] + c; r < poff[e + 1]; ++r) { a.prow_token[r] = -1; a.prow_pair[r] = -1; }
-  }
-  __syncthreads();
-
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < a.n_pairs; base += blockDim.x) {
-    const int p = base + tid;
-    const bool valid = p < a.n_pairs;
-    const int e = valid ? a.ids[p] : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & lt_mask);
-    if (valid && rank == 0) wcnt[warp * E + e] = __popc(peers);
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += blockDim.x) {
-      int run = cursor[ee];
-      for (int w = 0; w < W; ++w) {
-        const int c = wcnt[w * E + ee];
-        wcnt[w * E + ee] = run;
-        run += c;
-      }
-      cursor[ee] = run;
-    }
-    __syncthreads();
-    if (valid) {
-      const int local = wcnt[warp * E + e] + rank;
-      const int pos = a.offsets[e] + local;
-      const int prow = poff[e] + local;
-      a.perm[pos] = p;
-      a.inv[p] = pos;
-      a.prow_token[prow] = p / a.k;
-      a.prow_pair[prow] = p;
-    }
-    __syncthreads();
-    for (int i = tid; i < W * E; i += blockDim.x) wcnt[i] = 0;
-    __syncthreads();
-  }
+  permute_block<kPermThreads>(a, psm);
 }
 
 void launch_permute(const PermArgs &a, cudaStream_t s) {
-  const int W = kPermThreads / 32;
-  const size_t smem = sizeof(int) * ((size_t)4 * a.E + 2 + (size_t)W * a.E);
+  const size_t smem = sizeof(int) * perm_smem_ints(a.E, kPermThreads);
   if (smem > 48 * 1024) cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   permute_kernel<<<1, kPermThreads, smem, s>>>(a);
 }
