@@ -23,7 +23,7 @@ NUMERICS = {"exact": 0, "a4": 1}
 
 EXPORTED = ["moe_layer_plan", "moe_admit", "moe_layer_create", "moe_set_slot_table", "moe_forward",
             "moe_forward_host", "moe_get_stats", "moe_destroy", "moe_last_error", "moe_debug_inject",
-            "moe_profile_enable", "moe_profile_read", "moe_route_topk_noalloc"]
+            "moe_profile_enable", "moe_profile_read", "moe_route_topk_noalloc", "moe_debug_read"]
 
 
 class MoEError(RuntimeError):
@@ -56,7 +56,7 @@ class Stats(C.Structure):
         ("last_misses", C.c_int32), ("last_waves", C.c_int32), ("last_active", C.c_int32),
         ("last_path", C.c_int32), ("launches", C.c_uint64), ("expert_bytes", C.c_uint64),
         ("device_bytes", C.c_uint64),
-        ("pinned_bytes", C.c_uint64),
+        ("pinned_bytes", C.c_uint64), ("device_error", C.c_int32),
     ]
 
 
@@ -95,6 +95,7 @@ def lib():
         L.moe_debug_inject.argtypes = [C.c_void_p, C.c_int32]
         L.moe_profile_enable.argtypes = [C.c_void_p, C.c_int32]
         L.moe_profile_read.argtypes = [C.c_void_p, C.POINTER(Profile)]
+        L.moe_debug_read.argtypes = [C.c_void_p, C.c_int32, C.c_void_p, C.c_uint64]
         L.moe_route_topk_noalloc.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
                                              C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
                                              C.c_void_p]
@@ -257,6 +258,12 @@ class MoELayer:
         return {"forwards": p.forwards,
                 "ms": {n: p.ms[i] for i, n in enumerate(PROFILE_STAGES)},
                 "launches": {n: p.launches[i] for i, n in enumerate(PROFILE_STAGES)}}
+
+    def debug_read(self, which: int, dtype, count: int) -> np.ndarray:
+        """Test hook: copy an internal buffer of the last forward to host."""
+        out = np.empty(count, dtype=dtype)
+        check(lib().moe_debug_read(self.handle, which, out.ctypes.data, out.nbytes))
+        return out
 
     def inject(self, what: int):
         check(lib().moe_debug_inject(self.handle, what))

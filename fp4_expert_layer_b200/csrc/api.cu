@@ -103,6 +103,13 @@ struct moe_layer {
   uint16_t *xf16 = nullptr, *hbuf = nullptr, *sh_h = nullptr, *xin = nullptr;
   float *xs = nullptr, *hscale = nullptr, *oprime = nullptr, *sh_s = nullptr, *yout = nullptr;
   int *router_counter = nullptr, *tiles_done = nullptr, *comb_cnt = nullptr;
+  // A4 (activation FP4) path
+  bool a4 = false;
+  size_t a4_rows = 0;
+  A4Maps a4maps{};
+  uint8_t *xq = nullptr, *xsf = nullptr, *hq = nullptr, *hsf = nullptr;
+  float *xG = nullptr, *hG = nullptr, *h32 = nullptr;
+  int *n_prows = nullptr;
   // host
   uint8_t *store = nullptr;          // pinned: E x blob bytes
   int *h_counts = nullptr;           // pinned [E]
@@ -180,8 +187,6 @@ static moe_status_t check_config(const moe_config_t *c) {
   if (c->renormalize != 1) return fail(MOE_ERR_UNSUPPORTED, "only renormalised top-k gates are implemented (renormalize = 1)");
   if (c->numerics != MOE_NUMERICS_EXACT && c->numerics != MOE_NUMERICS_A4)
     return fail(MOE_ERR_INVALID_ARG, "numerics must be EXACT or A4");
-  if (c->numerics == MOE_NUMERICS_A4)
-    return fail(MOE_ERR_UNSUPPORTED, "A4 numerics is not available in this build");
   if (c->n_slots < 0 || c->n_slots > c->n_experts) return fail(MOE_ERR_INVALID_ARG, "n_slots must be in 0..n_experts");
   if (c->max_tokens < 1 || (int64_t)c->max_tokens * c->top_k > (1 << 30))
     return fail(MOE_ERR_INVALID_ARG, "max_tokens must be >= 1 and max_tokens * top_k <= 2^30");
@@ -197,7 +202,7 @@ static int default_staging(const moe_config_t *c) {
 }
 
 struct Sizes {
-  size_t P, max_prows, max_tiles;
+  size_t P, max_prows, max_tiles, a4_rows;
 };
 static Sizes sizes_of(const moe_config_t *c) {
   Sizes s;
@@ -205,7 +210,18 @@ static Sizes sizes_of(const moe_config_t *c) {
   const size_t act = std::min<size_t>(c->n_experts, s.P);
   s.max_prows = s.P + 8 * act;
   s.max_tiles = s.P / 8 + act + 1;
+  s.a4_rows = s.P + 128 * act + 128;     // padded to 128 rows per expert, + one tile of slack
   return s;
+}
+
+static size_t a4_scratch_bytes(const moe_config_t *c) {
+  if (c->numerics != MOE_NUMERICS_A4) return 0;
+  const Sizes z = sizes_of(c);
+  const size_t H = c->hidden, I = c->inter, G = c->fmt == MOE_FMT_MXFP4 ? 32 : 16;
+  size_t b = align256(z.a4_rows * H / 2) + align256(z.a4_rows * H / G) + align256(z.a4_rows * 4);
+  b += align256(z.a4_rows * I * 4) + align256(z.a4_rows * I / 2) + align256(z.a4_rows * I / G) + align256(z.a4_rows * 4);
+  b += align256(z.P * H * 4) + align256(4);
+  return b;
 }
 
 static size_t scratch_bytes(const moe_config_t *c) {
@@ -303,6 +319,37 @@ static moe_status_t make_code_map(CUtensorMap *map, const uint8_t *region, int n
   return MOE_OK;
 }
 
+// A4 weight map: (K/2 bytes, rows, blob index), box 128 bytes x 128 rows, 128-byte swizzle.
+static moe_status_t make_a4_weight_map(CUtensorMap *map, const uint8_t *region, int nblobs, const BlobLayout &L,
+                                       int m) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)(L.K[m] / 2), (cuuint64_t)L.rows[m], (cuuint64_t)nblobs};
+  cuuint64_t strides[2] = {(cuuint64_t)(L.K[m] / 2), (cuuint64_t)L.bytes};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void *)(region + L.codes[m]), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an A4 weight map");
+  return MOE_OK;
+}
+
+// A4 activation map: (row bytes, rows), box 128 bytes x 128 rows, 128-byte swizzle.
+static moe_status_t make_a4_act_map(CUtensorMap *map, const uint8_t *base, size_t row_bytes, size_t rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void *)base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an A4 activation map");
+  return MOE_OK;
+}
+
 // ------------------------------------------------------------------ C ABI
 extern "C" {
 
@@ -317,7 +364,7 @@ moe_status_t moe_layer_plan(const moe_config_t *cfg, moe_plan_t *out) {
   out->staging_bytes = (uint64_t)L.bytes * default_staging(cfg);
   out->resident_bytes = (uint64_t)cfg->n_experts * cfg->hidden * 4 + cfg->n_experts * 4 +
                         (uint64_t)3 * cfg->shared_inter * cfg->hidden * 2;
-  out->scratch_bytes = scratch_bytes(cfg);
+  out->scratch_bytes = scratch_bytes(cfg) + a4_scratch_bytes(cfg);
   out->pinned_bytes = (uint64_t)L.bytes * cfg->n_experts;
   return MOE_OK;
 }
@@ -468,8 +515,9 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   C_TRY(dalloc(L, &L->tiles, z.max_tiles * sizeof(TileInfo)));
   C_TRY(dalloc(L, &L->n_tiles, 4));
   C_TRY(dalloc(L, &L->active, 4));
-  C_TRY(dalloc(L, &L->prow_token, z.max_prows * 4));
-  C_TRY(dalloc(L, &L->prow_pair, z.max_prows * 4));
+  const size_t prow_cap = cfg->numerics == MOE_NUMERICS_A4 ? std::max(z.max_prows, z.a4_rows) : z.max_prows;
+  C_TRY(dalloc(L, &L->prow_token, prow_cap * 4));
+  C_TRY(dalloc(L, &L->prow_pair, prow_cap * 4));
   C_TRY(dalloc(L, &L->xf16, T * H * 2));
   C_TRY(dalloc(L, &L->xs, T * (H / kChunk) * 4));
   C_TRY(dalloc(L, &L->hbuf, z.max_prows * I * 2));
@@ -483,6 +531,21 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   C_TRY(dalloc(L, &L->tiles_done, 4));
   C_TRY(dalloc(L, &L->comb_cnt, T * (H / 256) * 4));
   C_TRY(dalloc(L, &L->xin, T * H * 2));
+  L->a4 = cfg->numerics == MOE_NUMERICS_A4;
+  if (L->a4) {
+    const size_t R = z.a4_rows, G = L->L.G;
+    L->a4_rows = R;
+    C_TRY(dalloc(L, &L->xq, R * H / 2));
+    C_TRY(dalloc(L, &L->xsf, R * H / G));
+    C_TRY(dalloc(L, &L->xG, R * 4));
+    C_TRY(dalloc(L, &L->h32, R * I * 4));
+    C_TRY(dalloc(L, &L->hq, R * I / 2));
+    C_TRY(dalloc(L, &L->hsf, R * I / G));
+    C_TRY(dalloc(L, &L->hG, R * 4));
+    C_TRY(dalloc(L, &L->n_prows, 4));
+    C_TRY(make_a4_act_map(&L->a4maps.act[0], L->xq, H / 2, R));
+    C_TRY(make_a4_act_map(&L->a4maps.act[1], L->hq, I / 2, R));
+  }
   C_TRY(dalloc(L, &L->yout, T * H * 4));
 
   C_CUDA(cudaMemsetAsync(L->router_counter, 0, ((T + 3) / 4) * 4, s));
@@ -498,6 +561,8 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     const int box_rows = m < 2 ? 128 : 256;
     if (cfg->n_slots) C_TRY(make_code_map(&L->maps.slot[m], L->slots, cfg->n_slots, L->L, m, box_rows));
     if (L->n_staging) C_TRY(make_code_map(&L->maps.stage[m], L->staging, L->n_staging, L->L, m, box_rows));
+    if (L->a4 && cfg->n_slots) C_TRY(make_a4_weight_map(&L->a4maps.w[0][m], L->slots, cfg->n_slots, L->L, m));
+    if (L->a4 && L->n_staging) C_TRY(make_a4_weight_map(&L->a4maps.w[1][m], L->staging, L->n_staging, L->L, m));
   }
   C_CUDA(cudaMemcpyAsync(L->router_w, w->router_w, (size_t)E * H * 4, cudaMemcpyHostToDevice, s));
   if (w->router_bias) C_CUDA(cudaMemcpyAsync(L->router_b, w->router_bias, (size_t)E * 4, cudaMemcpyHostToDevice, s));
@@ -518,7 +583,7 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   L->st.expert_bytes = bytes;
   L->st.pinned_bytes = bytes * E;
   size_t dev_total = (size_t)E * H * 4 + (size_t)3 * Is * H * 2 + bytes * (cfg->n_slots + L->n_staging) +
-                     scratch_bytes(cfg);
+                     scratch_bytes(cfg) + a4_scratch_bytes(cfg);
   L->st.device_bytes = dev_total;
   *out = L;
   return MOE_OK;
@@ -626,6 +691,63 @@ static moe_status_t run_experts(moe_layer *L, const int *locs, int nt, int grid_
   return MOE_OK;
 }
 
+// A4 pass over the experts present in `locs`: tcgen05 gate/up + SwiGLU -> h fp32,
+// quantise h rows of these experts, tcgen05 down + gate -> O'.
+static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles, cudaStream_t s) {
+  const moe_config_t &c = L->cfg;
+  A4GemmArgs g{};
+  g.maps = L->a4maps;
+  g.loc = locs;
+  g.slots = L->slots;
+  g.staging = L->staging;
+  g.blob_bytes = L->L.bytes;
+  g.L = L->L;
+  g.tiles = L->tiles;
+  g.n_tiles = L->n_tiles;
+  g.prow_pair = L->prow_pair;
+  g.gates = L->gates;
+  g.err = L->d_err;
+  g.act_map = 0;
+  g.K = c.hidden;
+  g.rows = c.inter;
+  g.n_rowblocks = c.inter / 128;
+  g.bsf = L->xsf;
+  g.bG = L->xG;
+  g.h_out = L->h32;
+  StageTimer t3(L, 3, s);
+  launch_gemm_a4(L->wf, MODE_GATEUP, g, grid_tiles, s);
+  CUDA_TRY(cudaGetLastError());
+  QuantArgs q{};
+  q.max_rows = (int)L->a4_rows;
+  q.n_rows = L->n_prows;
+  q.K = c.inter;
+  q.fmt = c.fmt;
+  q.src_f32 = L->h32;
+  q.row_pair = L->prow_pair;
+  q.loc = locs;
+  q.ids = L->ids;
+  q.codes = L->hq;
+  q.sf = L->hsf;
+  q.G = L->hG;
+  launch_quant(q, s);
+  CUDA_TRY(cudaGetLastError());
+  t3.launched(2);
+  t3.end();
+  g.act_map = 1;
+  g.K = c.inter;
+  g.rows = c.hidden;
+  g.n_rowblocks = c.hidden / 128;
+  g.bsf = L->hsf;
+  g.bG = L->hG;
+  g.o_out = L->oprime;
+  StageTimer t4(L, 4, s);
+  launch_gemm_a4(L->wf, MODE_DOWN, g, grid_tiles, s);
+  CUDA_TRY(cudaGetLastError());
+  t4.launched(1);
+  t4.end();
+  return MOE_OK;
+}
+
 moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void *stream,
                          const moe_routing_t *dbg) {
   if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
@@ -647,7 +769,8 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   const int act_est = std::min(E, P);
   const int avg = (P + act_est - 1) / act_est;
   const int nt = avg <= 8 ? 1 : (avg <= 16 ? 2 : 4);
-  const int ts = 8 * nt;
+  const bool a4 = L->a4;
+  const int ts = a4 ? 128 : 8 * nt;
   const int grid_tiles = P / ts + act_est + 1;
 
   StageTimer t7(L, 7, s);
@@ -662,6 +785,8 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   pa.counts = L->counts; pa.offsets = L->offsets; pa.perm = L->perm; pa.inv = L->inv;
   pa.tiles = L->tiles; pa.n_tiles = L->n_tiles; pa.prow_token = L->prow_token;
   pa.prow_pair = L->prow_pair; pa.active = L->active;
+  pa.pad = a4 ? 128 : 8;
+  pa.n_prows = a4 ? L->n_prows : nullptr;
   // decode-sized batches: the router's last CTA also runs the permutation
   const bool fuse_perm = P <= 2048;
   ra.fuse_perm = fuse_perm ? 1 : 0;
@@ -724,11 +849,29 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     t2.end();
   }
 
+  if (a4) {
+    QuantArgs q{};
+    q.max_rows = (int)L->a4_rows;
+    q.n_rows = L->n_prows;
+    q.K = H;
+    q.fmt = c.fmt;
+    q.src_bf16 = reinterpret_cast<const uint16_t *>(x);
+    q.row_token = L->prow_token;
+    q.codes = L->xq;
+    q.sf = L->xsf;
+    q.G = L->xG;
+    StageTimer tq(L, 1, s);
+    launch_quant(q, s);
+    CUDA_TRY(cudaGetLastError());
+    tq.launched(1);
+    tq.end();
+  }
   const int cs_gu = pick_split(act_est * (I / 128), H / 128);
   const int cs_dn = pick_split(act_est * (H / 256), I / 128);
   int waves = 0, misses_n = 0;
   if (resident) {
-    ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
+    if (a4) ST_TRY(run_experts_a4(L, L->loc_resident, grid_tiles, s));
+    else ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
   } else {
     CUDA_TRY(cudaEventSynchronize(L->ev_counts));
     std::vector<int> misses;
@@ -743,7 +886,8 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     misses_n = (int)misses.size();
     const int NS = L->n_staging;
     if (misses.empty()) {
-      ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
+      if (a4) ST_TRY(run_experts_a4(L, L->loc_resident, grid_tiles, s));
+      else ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
     } else {
       const bool one = misses_n <= NS;
       const int wave_sz = one ? NS : NS / 2;
@@ -778,7 +922,8 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
         CUDA_TRY(cudaGetLastError());
         t6.launched(1);
         t6.end();
-        ST_TRY(run_experts(L, L->loc_pass, nt, grid_tiles, cs_gu, cs_dn, y, s));
+        if (a4) ST_TRY(run_experts_a4(L, L->loc_pass, grid_tiles, s));
+        else ST_TRY(run_experts(L, L->loc_pass, nt, grid_tiles, cs_gu, cs_dn, y, s));
         if (!one) CUDA_TRY(cudaEventRecord(L->ev_done[half], s));
       }
       CUDA_TRY(cudaEventRecord(L->ev_fwd_done, s));
@@ -789,14 +934,27 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     }
   }
 
-  // the ordered combine runs inside the routed down pass (last arrival per token)
+  // EXACT: the ordered combine runs inside the routed down pass (last arrival
+  // per token); A4: a separate ordered combine.
+  if (a4) {
+    CombineArgs ca{};
+    ca.oprime = L->oprime;
+    ca.shared = Is ? L->sh_s : nullptr;
+    ca.y = y;
+    ca.T = T; ca.H = H; ca.k = k;
+    StageTimer t5(L, 5, s);
+    launch_combine(ca, s);
+    CUDA_TRY(cudaGetLastError());
+    t5.launched(1);
+    t5.end();
+  }
   t7.end();
   if (L->prof) L->prof_acc.forwards += 1;
 
   L->st.forwards += 1;
   L->st.last_misses = misses_n;
   L->st.last_waves = waves;
-  L->st.last_path = 0;
+  L->st.last_path = a4 ? 1 : 0;
   if (resident) L->st.last_active = -1;
   return MOE_OK;
 }
@@ -820,6 +978,7 @@ moe_status_t moe_forward_host(moe_layer_t L, const uint16_t *x_host, int32_t T, 
 moe_status_t moe_get_stats(moe_layer_t L, moe_stats_t *out) {
   if (!L || !out) return fail(MOE_ERR_INVALID_ARG, "layer or out is NULL");
   *out = L->st;
+  out->device_error = L->h_err ? *(volatile int *)L->h_err : 0;
   return MOE_OK;
 }
 
@@ -850,6 +1009,28 @@ moe_status_t moe_profile_read(moe_layer_t L, moe_profile_t *out) {
   CUDA_TRY(cudaSetDevice(L->cfg.device));
   ST_TRY(drain_profile(L));
   *out = L->prof_acc;
+  return MOE_OK;
+}
+
+moe_status_t moe_debug_read(moe_layer_t L, int32_t which, void *dst, uint64_t bytes) {
+  if (!L || !dst) return fail(MOE_ERR_INVALID_ARG, "layer or dst is NULL");
+  const void *src = nullptr;
+  switch (which) {
+    case 1: src = L->xq; break;
+    case 2: src = L->xsf; break;
+    case 3: src = L->h32; break;
+    case 4: src = L->hq; break;
+    case 5: src = L->hsf; break;
+    case 6: src = L->n_prows; break;
+    case 7: src = L->prow_token; break;
+    case 8: src = L->prow_pair; break;
+    case 11: src = L->oprime; break;
+    default: break;
+  }
+  if (!src) return fail(MOE_ERR_INVALID_ARG, "unknown or absent debug buffer");
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost));
   return MOE_OK;
 }
 

@@ -76,6 +76,8 @@ struct PermArgs {
   int *prow_token;       // [max prows]
   int *prow_pair;        // [max prows]
   int *active;           // [1] experts with >= 1 pair
+  int pad;               // row padding granularity per expert (8 or 128)
+  int *n_prows;          // [1] total padded rows (may be null)
 };
 struct RouterArgs {
   const uint16_t *x;     // bf16 [T, H]
@@ -191,5 +193,50 @@ struct TmaExpertArgs {
   int top_k;
 };
 void launch_expert_tma(int wf, int mode, int nt, const TmaExpertArgs &a, int grid_tiles, cudaStream_t s);
+
+// ------------------------------------------------------------------ A4 (activation FP4) path
+// Quantise rows to the experts' 4-bit format: codes [rows, K/2], scale blocks
+// laid out like the weights' (sf_offset over rows), NVFP4 per-row tensor scale.
+struct QuantArgs {
+  int max_rows;
+  const int *n_rows;         // device: rows to produce (padded count)
+  int K, fmt;
+  const uint16_t *src_bf16;  // x [T, K] gathered by row_token (x path), or null
+  const int *row_token;      // padded row -> token (-1 = pad)
+  const float *src_f32;      // h [rows, K] (h path), or null
+  const int *row_pair;       // padded row -> pair (-1 = pad), h path
+  const int *loc;            // h path: only rows whose expert is present in this pass
+  const int *ids;            // [T*k] pair -> expert
+  uint8_t *codes;
+  uint8_t *sf;
+  float *G;                  // NVFP4: per-row tensor scale
+};
+void launch_quant(const QuantArgs &q, cudaStream_t s);
+
+struct A4Maps {
+  CUtensorMap w[2][3];       // [slot | staging][matrix]: code bytes, box 128 B x 128 rows, 128-byte swizzle
+  CUtensorMap act[2];        // [x | h]: quantised activation rows, box 128 B x 128 rows, 128-byte swizzle
+};
+
+struct A4GemmArgs {
+  A4Maps maps;
+  int act_map;               // 0 = x (gate/up), 1 = h (down)
+  const int *loc;
+  const uint8_t *slots;
+  const uint8_t *staging;
+  size_t blob_bytes;
+  BlobLayout L;
+  int K, rows, n_rowblocks;
+  const TileInfo *tiles;
+  const int *n_tiles;
+  const uint8_t *bsf;        // activation scale blocks
+  const float *bG;           // NVFP4 activation per-row scale (null for MXFP4)
+  float *h_out;              // gate/up: h fp32 [rows of activations, I]
+  float *o_out;              // down: O' [pairs, H]
+  const int *prow_pair;
+  const float *gates;
+  int *err;
+};
+void launch_gemm_a4(int wf, int mode, const A4GemmArgs &a, int grid_tiles, cudaStream_t s);
 
 }  // namespace moe

@@ -53,7 +53,7 @@ __device__ void permute_block(const PermArgs &a, int *sm) {
   for (int e = e0; e < e1; ++e) {
     const int c = cnt[e];
     v.x += c;
-    v.y += (c + 7) & ~7;
+    v.y += (c + a.pad - 1) / a.pad * a.pad;
     v.z += (c + a.tile_tokens - 1) / a.tile_tokens;
     v.w += c > 0;
   }
@@ -90,7 +90,7 @@ __device__ void permute_block(const PermArgs &a, int *sm) {
       const int c = cnt[e];
       off[e] = o; poff[e] = po; toff[e] = to;
       o += c;
-      po += (c + 7) & ~7;
+      po += (c + a.pad - 1) / a.pad * a.pad;
       to += (c + a.tile_tokens - 1) / a.tile_tokens;
     }
     if (tid == NTH - 1) {
@@ -98,6 +98,7 @@ __device__ void permute_block(const PermArgs &a, int *sm) {
       off[E] = tot.x; poff[E] = tot.y; toff[E] = tot.z;
       *a.n_tiles = tot.z;
       *a.active = tot.w;
+      if (a.n_prows) *a.n_prows = tot.y;
     }
   }
   __syncthreads();

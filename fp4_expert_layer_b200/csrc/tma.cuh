@@ -5,9 +5,16 @@
 
 namespace moe {
 
-// Upper bound on polls of one mbarrier phase before a kernel gives up, records
-// an error and continues (so that no wait can run forever).
-constexpr uint32_t kWaitLimit = 1u << 22;
+// A wait gives up after this much GPU wall time (or at once when another wait
+// has already recorded an error), records an error code and lets the kernel run
+// to completion, so that no wait can run forever.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -42,12 +49,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for phase `parity` of a barrier.  Returns false (and records
-// `code` in *err) when the limit is reached.
+// `code` in *err) when the limit is reached or another wait already failed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *err, int code) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-  if (err) atomicExch(err, code);
-  return false;
+    if ((i & 255u) == 0) {
+      if (err && *(volatile int *)err != 0) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        if (err) atomicExch(err, code);
+        return false;
+      }
+    }
+  }
 }
 
 // 3-D tiled TMA load of one box into this CTA's shared memory.

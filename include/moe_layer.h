@@ -131,6 +131,9 @@ typedef struct {
   uint64_t expert_bytes;   /* device-layout bytes of one routed expert          */
   uint64_t device_bytes;   /* HBM held by the layer                             */
   uint64_t pinned_bytes;   /* pinned host memory held by the layer              */
+  int32_t device_error;    /* nonzero: a device-side wait gave up (code of the  */
+                           /* first one); the next moe_forward reports and      */
+                           /* clears it                                         */
 } moe_stats_t;
 
 /* Memory plan of a configuration without allocating anything (the dry-run
@@ -239,6 +242,13 @@ const char *moe_last_error(void);
  * in moe_layer_create fails, 0 = off.  The forward must then return an error
  * status and leave the CUDA context usable. */
 moe_status_t moe_debug_inject(moe_layer_t layer, int32_t what);
+
+/* Test hook: synchronously copy up to `bytes` of an internal device buffer of
+ * the last forward into host memory.  which: 1 quantised x codes, 2 x scale
+ * blocks, 3 h (fp32, A4 path), 4 quantised h codes, 5 h scale blocks, 6 padded
+ * row count, 7 padded row -> token, 8 padded row -> pair, 11 O' (fp32).
+ * Returns MOE_ERR_INVALID_ARG for an unknown or absent buffer. */
+moe_status_t moe_debug_read(moe_layer_t layer, int32_t which, void *dst_host, uint64_t bytes);
 
 #ifdef __cplusplus
 }

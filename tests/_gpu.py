@@ -43,6 +43,7 @@ def run(layer, x_bits):
     t = torch()
     y, r = layer.forward(to_device(x_bits), routing=True)
     t.cuda.synchronize()
+    assert layer.stats()["device_error"] == 0, "a device-side wait gave up"
     return y.cpu().numpy(), {k: v.cpu().numpy() for k, v in r.items()}
 
 
