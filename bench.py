@@ -49,6 +49,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="olmoe_like", choices=sorted(synth.WORKLOADS))
     p.add_argument("--tokens", type=int, default=32)
+    p.add_argument("--numerics", default="exact", choices=["exact", "a4"])
     p.add_argument("--slots", default="workload", choices=["workload", "all"],
                    help="resident budget: the workload's own, or every expert resident")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline sample budget")
@@ -62,8 +63,9 @@ def peaks():
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 # ------------------------------------------------------------------ clocks
@@ -137,7 +139,7 @@ def layer_bytes(wl, n_active, T):
 
 def traffic_record(kernel_src):
     """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
-    path = os.path.join(ROOT, "profiles", "gateup_olmoe_like_T32_traffic.json")
+    path = os.path.join(ROOT, "profiles", "expert_tma_gateup_olmoe_like_T32_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -148,21 +150,28 @@ def traffic_record(kernel_src):
 
 
 # ------------------------------------------------------------------ CPU (oracle) legs
-def cpu_baseline(lw, x_bits, budget_s):
-    """The oracle as it stands, all host threads, full forwards of the benchmark batch."""
+def cpu_baseline(lw, x_bits, budget_s, numerics="exact"):
+    """The oracle as it stands, all host threads, forwards over consecutive
+    slices of the benchmark batch (the whole batch when it is small) until the
+    time budget is spent."""
     import oracle
-    L = oracle.Layer.from_weights(lw)
+    L = oracle.Layer.from_weights(lw, numerics=numerics)
     threads = oracle.max_threads()
     T = x_bits.shape[0]
-    n, t0 = 0, time.perf_counter()
+    chunk = T if T <= 64 else max(2 * threads, 16)
+    n, i, t0 = 0, 0, time.perf_counter()
     while True:
-        L.forward(x_bits, threads=threads)
-        n += 1
+        c = min(chunk, T - i)
+        L.forward(x_bits[i:i + c], threads=threads)
+        n += c
+        i = (i + c) % T
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return {"value": n * T / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} full forwards of the {T}-token batch ({n * T} tokens, {el:.1f} s)"}
+    what = (f"full forwards of the {T}-token batch" if chunk == T
+            else f"forwards of consecutive {chunk}-token slices of the {T}-token batch")
+    return {"value": n / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{what} ({n} tokens, {el:.1f} s, {numerics} numerics)"}
 
 
 def reference_arm(args, wl, lw, world):
@@ -250,7 +259,7 @@ def main():
     T = args.tokens
     lw = synth.make_layer(wl)
     S = wl.n_experts if args.slots == "all" else wl.n_slots
-    layer = F.MoELayer.from_weights(lw, n_slots=S, max_tokens=T)
+    layer = F.MoELayer.from_weights(lw, n_slots=S, max_tokens=T, numerics=args.numerics)
     layer.set_slot_table(synth.slot_table(lw, S))
     x_bits = synth.make_tokens(wl, T, stream=rank)
     x = torch.from_numpy(x_bits.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -275,7 +284,6 @@ def main():
     launches0 = layer.stats()["launches"]
     clocks.start()
     time.sleep(0.3)
-    layer.profile_enable(True)
     barrier()
     torch.cuda.synchronize()
     w0 = time.perf_counter()
@@ -288,9 +296,16 @@ def main():
     barrier()
     wall = time.perf_counter() - w0
     clk = clocks.stop()
+    launches = layer.stats()["launches"] - launches0
+    # per-stage device times: a separate pass of the same loop with the
+    # library's stage event pairs on, so that they do not touch the timed steps
+    layer.profile_enable(True)
+    for i in range(min(K, 200)):
+        flush.zero_()
+        layer.forward_ptr(x.data_ptr(), T, y.data_ptr(), sp)
+    torch.cuda.synchronize()
     prof = layer.profile_read()
     layer.profile_enable(False)
-    launches = layer.stats()["launches"] - launches0
     dev_ms = sum(a.elapsed_time(b) for a, b in zip(ev0, ev1))
 
     # e2e through the public host-buffer call: H2D of x, forward, D2H of y
@@ -321,29 +336,43 @@ def main():
     dev_ms_max, e2e_ms_max = float(vals[0]), float(vals[1])
 
     if rank == 0:
-        hbm_peak, bf16_peak, peak_src = peaks()
+        hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
         ms_step = dev_ms_max / K
         value = world * T * K / (dev_ms_max / 1e3)
         g_ms = prof["ms"]["gateup"] / max(1, prof["launches"]["gateup"])
-        g_bytes = gateup_bytes(wl, n_active, T)
-        achieved = g_bytes / (g_ms / 1e3) / 1e9
-        traffic = traffic_record(os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert.cu"))
+        if args.numerics == "a4":
+            # tcgen05 gate/up GEMM: FP4 FLOPs of the real (unpadded) token rows
+            g_flops = 4.0 * T * wl.top_k * wl.hidden * wl.inter
+            achieved = g_flops / (g_ms / 1e3) / 1e12
+            # the GEMM runs back to back for seconds inside the step loop: sustained figure
+            fp4_peak = 4.0 * bf16_sus
+            roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                    "frac": achieved / fp4_peak, "traffic": None,
+                    "kernel": "gemm_a4_kernel gate/up+SwiGLU (tcgen05 block-scaled FP4)",
+                    "peak_source": f"{peak_src} bf16_tflops_sustained x 4 (nominal FP4/BF16 dense ratio)",
+                    "algorithmic_flops_per_launch": g_flops, "kernel_ms": g_ms,
+                    "hbm_gbs_of_same_launch": gateup_bytes(wl, n_active, T) / (g_ms / 1e3) / 1e9}
+        else:
+            g_bytes = gateup_bytes(wl, n_active, T)
+            achieved = g_bytes / (g_ms / 1e3) / 1e9
+            traffic = traffic_record(os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert_tma.cu"))
+            roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "traffic": traffic,
+                    "kernel": "expert_tma_kernel gate/up+SwiGLU (routed)",
+                    "peak_source": f"{peak_src} hbm_gbs",
+                    "algorithmic_bytes_per_launch": g_bytes, "kernel_ms": g_ms}
         stage_ms = {k: v / max(1, prof["forwards"]) for k, v in prof["ms"].items()}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16xfp4->f32",
+            "vs_baseline": None, "dtype": "f16xfp4->f32" if args.numerics == "exact" else "fp4xfp4->f32",
             "data": "synthetic (seeded; random-init weights of the workload's shape)",
             "config": {"workload": wl.name, "tokens": T, "hidden": wl.hidden, "inter": wl.inter,
                        "n_experts": wl.n_experts, "top_k": wl.top_k, "fmt": wl.fmt,
-                       "shared_inter": wl.shared_inter, "resident_slots": S, "numerics": "exact",
+                       "shared_inter": wl.shared_inter, "resident_slots": S, "numerics": args.numerics,
                        "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before every step",
                        "active_experts": n_active},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": traffic,
-                         "kernel": "expert_kernel gate/up+SwiGLU (routed)",
-                         "peak_source": f"{peak_src} hbm_gbs",
-                         "algorithmic_bytes_per_launch": g_bytes, "kernel_ms": g_ms},
+            "roofline": roof,
             "layer_roofline": {"bytes_per_step": layer_bytes(wl, n_active, T),
                                "hbm_frac": layer_bytes(wl, n_active, T) / (ms_step / 1e3) / 1e9 / hbm_peak},
             "stage_ms": stage_ms,
@@ -355,7 +384,7 @@ def main():
             line["e2e"] = {"value": world * T * e2e[1] / (e2e_ms_max / 1e3), "unit": "tokens/s",
                            "h2d_bytes_per_step": T * wl.hidden * 2, "d2h_bytes_per_step": T * wl.hidden * 4}
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(lw, x_bits, args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(lw, x_bits, args.cpu_seconds, args.numerics)
         print(json.dumps(line), flush=True)
 
     layer.close()

@@ -60,11 +60,12 @@ class Stats(C.Structure):
     ]
 
 
-PROFILE_STAGES = ["router", "permute", "shared", "gateup", "down", "combine", "staging_wait", "forward"]
+PROFILE_STAGES = ["router", "permute", "shared", "gateup", "down", "combine", "staging_wait", "forward",
+                  "quantise", "unused"]
 
 
 class Profile(C.Structure):
-    _fields_ = [("forwards", C.c_uint64), ("ms", C.c_double * 8), ("launches", C.c_uint64 * 8)]
+    _fields_ = [("forwards", C.c_uint64), ("ms", C.c_double * 10), ("launches", C.c_uint64 * 10)]
 
 
 class Plan(C.Structure):

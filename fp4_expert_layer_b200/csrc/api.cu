@@ -50,9 +50,10 @@ const char *set_error_text(const std::string &s) {
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-BlobLayout moe::blob_layout(int H, int I, int fmt) {
+BlobLayout moe::blob_layout(int H, int I, int fmt, int tiled) {
   BlobLayout L{};
   L.fmt = fmt;
+  L.tiled = tiled;
   L.G = fmt == MOE_FMT_MXFP4 ? 32 : 16;
   size_t off = 0;
   for (int m = 0; m < 3; ++m) {
@@ -110,6 +111,12 @@ struct moe_layer {
   uint8_t *xq = nullptr, *xsf = nullptr, *hq = nullptr, *hsf = nullptr;
   float *xG = nullptr, *hG = nullptr, *h32 = nullptr;
   int *n_prows = nullptr;
+  // EXACT numerics of MXFP4 experts on the tensor core (E4M3 activation pieces)
+  bool tc = false;
+  int n_sms = 148;
+  size_t tc_rows = 0;
+  TcMaps tcmaps{};
+  uint8_t *txq = nullptr, *txsf = nullptr, *thq = nullptr, *thsf = nullptr;
   // host
   uint8_t *store = nullptr;          // pinned: E x blob bytes
   int *h_counts = nullptr;           // pinned [E]
@@ -202,7 +209,7 @@ static int default_staging(const moe_config_t *c) {
 }
 
 struct Sizes {
-  size_t P, max_prows, max_tiles, a4_rows;
+  size_t P, max_prows, max_tiles, a4_rows, tc_tiles;
 };
 static Sizes sizes_of(const moe_config_t *c) {
   Sizes s;
@@ -211,6 +218,9 @@ static Sizes sizes_of(const moe_config_t *c) {
   s.max_prows = s.P + 8 * act;
   s.max_tiles = s.P / 8 + act + 1;
   s.a4_rows = s.P + 128 * act + 128;     // padded to 128 rows per expert, + one tile of slack
+  // tensor-core EXACT path: tiles of 16 tokens only while P <= 12 * active experts
+  // (then at most 1.75 x act tiles), else tiles of 64 tokens
+  s.tc_tiles = std::max(s.P / 64 + act, (7 * act) / 4 + 1) + 2;
   return s;
 }
 
@@ -224,6 +234,17 @@ static size_t a4_scratch_bytes(const moe_config_t *c) {
   return b;
 }
 
+static bool uses_tc(const moe_config_t *c) {
+  return c->numerics == MOE_NUMERICS_EXACT && c->fmt == MOE_FMT_MXFP4;
+}
+
+static size_t tc_scratch_bytes(const moe_config_t *c) {
+  if (!uses_tc(c)) return 0;
+  const Sizes z = sizes_of(c);
+  const size_t R = z.tc_tiles * kTcSlotRows, H = c->hidden, I = c->inter;
+  return align256(R * H) + align256(R * H / 32) + align256(R * I) + align256(R * I / 32);
+}
+
 static size_t scratch_bytes(const moe_config_t *c) {
   const Sizes z = sizes_of(c);
   const size_t T = c->max_tokens, H = c->hidden, I = c->inter, E = c->n_experts, Is = c->shared_inter;
@@ -234,7 +255,7 @@ static size_t scratch_bytes(const moe_config_t *c) {
   b += align256(z.max_prows * I * 2) + align256(z.max_prows * (I / kChunk) * 4);
   b += align256(z.P * H * 4);
   if (Is) b += align256(T * Is * 2) + align256(T * H * 4);
-  b += align256(((T + 3) / 4) * 4) + align256(4) + align256(T * (H / 256) * 4);
+  b += align256(((T + 3) / 4) * 4) + align256(4) + align256(T * (H / 128) * 4);
   b += align256(T * H * 2) + align256(T * H * 4);
   b += 2 * align256(E * sizeof(void *));
   return b;
@@ -350,6 +371,32 @@ static moe_status_t make_a4_act_map(CUtensorMap *map, const uint8_t *base, size_
   return MOE_OK;
 }
 
+// Tensor-core EXACT weight map over a tiled code region: 4-D (128 elements,
+// 256 rows of 64 bytes, chunk, blob), box 128 x 256 x 1 x 1 = one contiguous
+// 16 KB chunk, unpacked by the TMA to one byte per element (8 code bytes + 8
+// empty bytes per 16 elements, the shared-memory form the f8f6f4 MMA kinds
+// read), 128-byte swizzle.
+static moe_status_t make_tc_weight_map(CUtensorMap *map, const uint8_t *region, int nblobs, const BlobLayout &L,
+                                       bool gate_up) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const int H = L.K[0], I = L.rows[0];
+  const size_t nchunks = gate_up ? (size_t)(I / 128) * (H / 128) : (size_t)(H / 256) * (I / 128);
+  cuuint64_t dims[4] = {128, 256, (cuuint64_t)nchunks, (cuuint64_t)nblobs};
+  cuuint64_t strides[3] = {64, (cuuint64_t)kTcChunk, (cuuint64_t)L.bytes};
+  cuuint32_t box[4] = {128, 256, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, (void *)(region + L.codes[gate_up ? 0 : 2]), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[96];
+    snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (%d) for a tiled weight map", (int)r);
+    return fail(MOE_ERR_CUDA, buf);
+  }
+  return MOE_OK;
+}
+
 // ------------------------------------------------------------------ C ABI
 extern "C" {
 
@@ -358,13 +405,13 @@ const char *moe_last_error(void) { return g_err.c_str(); }
 moe_status_t moe_layer_plan(const moe_config_t *cfg, moe_plan_t *out) {
   ST_TRY(check_config(cfg));
   if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
-  const BlobLayout L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt);
+  const BlobLayout L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt, uses_tc(cfg));
   out->expert_bytes = L.bytes;
   out->slot_bytes = (uint64_t)L.bytes * cfg->n_slots;
   out->staging_bytes = (uint64_t)L.bytes * default_staging(cfg);
   out->resident_bytes = (uint64_t)cfg->n_experts * cfg->hidden * 4 + cfg->n_experts * 4 +
                         (uint64_t)3 * cfg->shared_inter * cfg->hidden * 2;
-  out->scratch_bytes = scratch_bytes(cfg) + a4_scratch_bytes(cfg);
+  out->scratch_bytes = scratch_bytes(cfg) + a4_scratch_bytes(cfg) + tc_scratch_bytes(cfg);
   out->pinned_bytes = (uint64_t)L.bytes * cfg->n_experts;
   return MOE_OK;
 }
@@ -372,7 +419,7 @@ moe_status_t moe_layer_plan(const moe_config_t *cfg, moe_plan_t *out) {
 moe_status_t moe_admit(const moe_config_t *cfg, const moe_weights_t *w) {
   ST_TRY(check_config(cfg));
   if (!w || !w->router_w) return fail(MOE_ERR_INVALID_ARG, "weights or router_w is NULL");
-  const BlobLayout L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt);
+  const BlobLayout L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt, 0);
   for (int m = 0; m < 3; ++m)
     if (!w->codes[m] || !w->scales[m]) return fail(MOE_ERR_INVALID_ARG, "codes/scales table is NULL");
   if (cfg->shared_inter > 0 && (!w->shared_w[0] || !w->shared_w[1] || !w->shared_w[2]))
@@ -407,8 +454,45 @@ moe_status_t moe_admit(const moe_config_t *cfg, const moe_weights_t *w) {
   return MOE_OK;
 }
 
+// Tile-major codes and scales (layout tiled = 1).
+static void pack_expert_tiled(const BlobLayout &L, const moe_weights_t *w, int e, uint8_t *dst) {
+  const int H = L.K[0], I = L.rows[0];
+  const int ns_gu = H / 128, ns_dn = I / 128;
+  // gate / up: chunk (rb, slab) = [gate 128 rows][up 128 rows] x 64 bytes
+  for (int rb = 0; rb < I / 128; ++rb)
+    for (int slab = 0; slab < ns_gu; ++slab)
+      for (int mat = 0; mat < 2; ++mat) {
+        const size_t chunk = (size_t)rb * ns_gu + slab;
+        uint8_t *cd = dst + L.codes[0] + chunk * kTcChunk + (size_t)mat * (kTcChunk / 2);
+        uint8_t *sd = dst + L.scales[0] + chunk * kTcSfChunk + (size_t)mat * 512;
+        const uint8_t *cs = w->codes[mat][e], *ss = w->scales[mat][e];
+        for (int r = 0; r < 128; ++r) {
+          const size_t row = (size_t)rb * 128 + r;
+          memcpy(cd + r * 64, cs + row * (H / 2) + (size_t)slab * 64, 64);
+          for (int c = 0; c < 4; ++c) sd[sf_offset(4, r, c)] = ss[row * (H / 32) + slab * 4 + c];
+        }
+      }
+  // down: chunk (rb, slab) = 256 rows x 64 bytes; scale halves rows 0..127, 128..255
+  for (int rb = 0; rb < H / 256; ++rb)
+    for (int slab = 0; slab < ns_dn; ++slab) {
+      const size_t chunk = (size_t)rb * ns_dn + slab;
+      uint8_t *cd = dst + L.codes[2] + chunk * kTcChunk;
+      uint8_t *sd = dst + L.scales[2] + chunk * kTcSfChunk;
+      const uint8_t *cs = w->codes[2][e], *ss = w->scales[2][e];
+      for (int r = 0; r < 256; ++r) {
+        const size_t row = (size_t)rb * 256 + r;
+        memcpy(cd + r * 64, cs + row * (I / 2) + (size_t)slab * 64, 64);
+        for (int c = 0; c < 4; ++c) sd[(r / 128) * 512 + sf_offset(4, r % 128, c)] = ss[row * (I / 32) + slab * 4 + c];
+      }
+    }
+}
+
 static void pack_expert(const moe_config_t *cfg, const BlobLayout &L, const moe_weights_t *w, int e,
                         uint8_t *dst) {
+  if (L.tiled) {
+    pack_expert_tiled(L, w, e, dst);
+    return;
+  }
   for (int m = 0; m < 3; ++m) {
     const size_t ncode = (size_t)L.rows[m] * L.K[m] / 2;
     const size_t nsc = (size_t)L.rows[m] * L.K[m] / L.G;
@@ -445,7 +529,7 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   cudaStream_t s = (cudaStream_t)stream;
   moe_layer *L = new moe_layer();
   L->cfg = *cfg;
-  L->L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt);
+  L->L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt, uses_tc(cfg));
   L->wf = cfg->fmt == MOE_FMT_MXFP4 ? WF_MX : WF_NV;
   L->n_staging = default_staging(cfg);
   L->cfg.n_staging = L->n_staging;
@@ -529,7 +613,7 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   }
   C_TRY(dalloc(L, &L->router_counter, ((T + 3) / 4) * 4));
   C_TRY(dalloc(L, &L->tiles_done, 4));
-  C_TRY(dalloc(L, &L->comb_cnt, T * (H / 256) * 4));
+  C_TRY(dalloc(L, &L->comb_cnt, T * (H / 128) * 4));
   C_TRY(dalloc(L, &L->xin, T * H * 2));
   L->a4 = cfg->numerics == MOE_NUMERICS_A4;
   if (L->a4) {
@@ -546,11 +630,29 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     C_TRY(make_a4_act_map(&L->a4maps.act[0], L->xq, H / 2, R));
     C_TRY(make_a4_act_map(&L->a4maps.act[1], L->hq, I / 2, R));
   }
+  L->tc = uses_tc(cfg);
+  {
+    int nsm = 0;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, cfg->device) == cudaSuccess && nsm > 0)
+      L->n_sms = nsm;
+  }
+  if (L->tc) {
+    const size_t R = z.tc_tiles * kTcSlotRows;
+    L->tc_rows = R;
+    C_TRY(dalloc(L, &L->txq, R * H));
+    C_TRY(dalloc(L, &L->txsf, R * H / 32));
+    C_TRY(dalloc(L, &L->thq, R * I));
+    C_TRY(dalloc(L, &L->thsf, R * I / 32));
+    C_CUDA(cudaMemsetAsync(L->txq, 0, R * H, s));
+    C_CUDA(cudaMemsetAsync(L->txsf, 127, R * H / 32, s));
+    C_CUDA(cudaMemsetAsync(L->thq, 0, R * I, s));
+    C_CUDA(cudaMemsetAsync(L->thsf, 127, R * I / 32, s));
+  }
   C_TRY(dalloc(L, &L->yout, T * H * 4));
 
   C_CUDA(cudaMemsetAsync(L->router_counter, 0, ((T + 3) / 4) * 4, s));
   C_CUDA(cudaMemsetAsync(L->tiles_done, 0, 4, s));
-  C_CUDA(cudaMemsetAsync(L->comb_cnt, 0, T * (H / 256) * 4, s));
+  C_CUDA(cudaMemsetAsync(L->comb_cnt, 0, T * (H / 128) * 4, s));
   C_CUDA(cudaMemsetAsync(L->ptr_resident, 0, sizeof(void *) * E, s));
   C_CUDA(cudaMemsetAsync(L->ptr_pass, 0, sizeof(void *) * E, s));
   C_CUDA(cudaMemsetAsync(L->loc_resident, 0xFF, sizeof(int) * E, s));   // -1: absent
@@ -563,6 +665,12 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     if (L->n_staging) C_TRY(make_code_map(&L->maps.stage[m], L->staging, L->n_staging, L->L, m, box_rows));
     if (L->a4 && cfg->n_slots) C_TRY(make_a4_weight_map(&L->a4maps.w[0][m], L->slots, cfg->n_slots, L->L, m));
     if (L->a4 && L->n_staging) C_TRY(make_a4_weight_map(&L->a4maps.w[1][m], L->staging, L->n_staging, L->L, m));
+  }
+  if (L->tc) {
+    for (int g = 0; g < 2; ++g) {
+      if (cfg->n_slots) C_TRY(make_tc_weight_map(&L->tcmaps.w[0][g], L->slots, cfg->n_slots, L->L, g == 0));
+      if (L->n_staging) C_TRY(make_tc_weight_map(&L->tcmaps.w[1][g], L->staging, L->n_staging, L->L, g == 0));
+    }
   }
   C_CUDA(cudaMemcpyAsync(L->router_w, w->router_w, (size_t)E * H * 4, cudaMemcpyHostToDevice, s));
   if (w->router_bias) C_CUDA(cudaMemcpyAsync(L->router_b, w->router_bias, (size_t)E * 4, cudaMemcpyHostToDevice, s));
@@ -583,7 +691,7 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   L->st.expert_bytes = bytes;
   L->st.pinned_bytes = bytes * E;
   size_t dev_total = (size_t)E * H * 4 + (size_t)3 * Is * H * 2 + bytes * (cfg->n_slots + L->n_staging) +
-                     scratch_bytes(cfg) + a4_scratch_bytes(cfg);
+                     scratch_bytes(cfg) + a4_scratch_bytes(cfg) + tc_scratch_bytes(cfg);
   L->st.device_bytes = dev_total;
   *out = L;
   return MOE_OK;
@@ -691,6 +799,55 @@ static moe_status_t run_experts(moe_layer *L, const int *locs, int nt, int grid_
   return MOE_OK;
 }
 
+// Tensor-core EXACT pass over the experts present in `locs`: gate/up + SwiGLU
+// -> h pieces, down + gate -> O' and the ordered combine into y.
+static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int grid_tiles, float *y,
+                                   cudaStream_t s) {
+  const moe_config_t &c = L->cfg;
+  TcArgs a{};
+  a.maps = L->tcmaps;
+  a.loc = locs;
+  a.slots = L->slots;
+  a.staging = L->staging;
+  a.blob_bytes = L->L.bytes;
+  a.L = L->L;
+  a.tiles = L->tiles;
+  a.n_tiles = L->n_tiles;
+  a.prow_pair = L->prow_pair;
+  a.gates = L->gates;
+  a.err = L->d_err;
+  a.hq = L->thq;
+  a.hsf = L->thsf;
+  a.o_out = L->oprime;
+  a.y = y;
+  a.shared = c.shared_inter ? L->sh_s : nullptr;
+  a.comb_cnt = L->comb_cnt;
+  a.top_k = c.top_k;
+  a.act = L->txq;
+  a.K = c.hidden;
+  a.rows = c.inter;
+  a.n_rowblocks = c.inter / 128;
+  a.bsf = L->txsf;
+  a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
+  StageTimer t3(L, 3, s);
+  launch_expert_tc(MODE_GATEUP, nbox, a, grid_tiles, s);
+  CUDA_TRY(cudaGetLastError());
+  t3.launched(1);
+  t3.end();
+  a.act = L->thq;
+  a.K = c.inter;
+  a.rows = c.hidden;
+  a.n_rowblocks = c.hidden / 256;
+  a.bsf = L->thsf;
+  a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
+  StageTimer t4(L, 4, s);
+  launch_expert_tc(MODE_DOWN, nbox, a, grid_tiles, s);
+  CUDA_TRY(cudaGetLastError());
+  t4.launched(1);
+  t4.end();
+  return MOE_OK;
+}
+
 // A4 pass over the experts present in `locs`: tcgen05 gate/up + SwiGLU -> h fp32,
 // quantise h rows of these experts, tcgen05 down + gate -> O'.
 static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles, cudaStream_t s) {
@@ -717,6 +874,9 @@ static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles
   StageTimer t3(L, 3, s);
   launch_gemm_a4(L->wf, MODE_GATEUP, g, grid_tiles, s);
   CUDA_TRY(cudaGetLastError());
+  t3.launched(1);
+  t3.end();
+  StageTimer t8(L, 8, s);
   QuantArgs q{};
   q.max_rows = (int)L->a4_rows;
   q.n_rows = L->n_prows;
@@ -731,8 +891,8 @@ static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles
   q.G = L->hG;
   launch_quant(q, s);
   CUDA_TRY(cudaGetLastError());
-  t3.launched(2);
-  t3.end();
+  t8.launched(1);
+  t8.end();
   g.act_map = 1;
   g.K = c.inter;
   g.rows = c.hidden;
@@ -770,7 +930,11 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   const int avg = (P + act_est - 1) / act_est;
   const int nt = avg <= 8 ? 1 : (avg <= 16 ? 2 : 4);
   const bool a4 = L->a4;
-  const int ts = a4 ? 128 : 8 * nt;
+  const bool tc = L->tc;
+  // tensor-core EXACT: 16-token tiles (32 piece rows) while the batch is
+  // decode-sized, else 64-token tiles (128 piece rows)
+  const int nbox = (tc && P <= 12 * act_est) ? 32 : 128;
+  const int ts = a4 ? 128 : (tc ? nbox / 2 : 8 * nt);
   const int grid_tiles = P / ts + act_est + 1;
 
   StageTimer t7(L, 7, s);
@@ -779,7 +943,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   ra.T = T; ra.H = H; ra.E = E; ra.k = k;
   ra.w = L->router_w; ra.bias = L->router_b;
   ra.logits = L->logits; ra.ids = L->ids; ra.gates = L->gates;
-  ra.xf16 = L->xf16; ra.xs = L->xs; ra.counter = L->router_counter;
+  ra.xf16 = tc ? nullptr : L->xf16; ra.xs = L->xs; ra.counter = L->router_counter;
   PermArgs pa{};
   pa.ids = L->ids; pa.n_pairs = P; pa.E = E; pa.k = k; pa.tile_tokens = ts;
   pa.counts = L->counts; pa.offsets = L->offsets; pa.perm = L->perm; pa.inv = L->inv;
@@ -860,8 +1024,25 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     q.codes = L->xq;
     q.sf = L->xsf;
     q.G = L->xG;
-    StageTimer tq(L, 1, s);
+    StageTimer tq(L, 8, s);
     launch_quant(q, s);
+    CUDA_TRY(cudaGetLastError());
+    tq.launched(1);
+    tq.end();
+  }
+  if (tc) {
+    TcQuantArgs q{};
+    q.x = reinterpret_cast<const uint16_t *>(x);
+    q.H = H;
+    q.tiles = L->tiles;
+    q.n_tiles = L->n_tiles;
+    q.max_tiles = grid_tiles;
+    q.tile_tokens = ts;
+    q.prow_token = L->prow_token;
+    q.xq = L->txq;
+    q.xsf = L->txsf;
+    StageTimer tq(L, 8, s);
+    launch_tc_quant_x(q, s);
     CUDA_TRY(cudaGetLastError());
     tq.launched(1);
     tq.end();
@@ -871,6 +1052,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   int waves = 0, misses_n = 0;
   if (resident) {
     if (a4) ST_TRY(run_experts_a4(L, L->loc_resident, grid_tiles, s));
+    else if (tc) ST_TRY(run_experts_tc(L, L->loc_resident, nbox, grid_tiles, y, s));
     else ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
   } else {
     CUDA_TRY(cudaEventSynchronize(L->ev_counts));
@@ -887,6 +1069,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     const int NS = L->n_staging;
     if (misses.empty()) {
       if (a4) ST_TRY(run_experts_a4(L, L->loc_resident, grid_tiles, s));
+      else if (tc) ST_TRY(run_experts_tc(L, L->loc_resident, nbox, grid_tiles, y, s));
       else ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
     } else {
       const bool one = misses_n <= NS;
@@ -923,6 +1106,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
         t6.launched(1);
         t6.end();
         if (a4) ST_TRY(run_experts_a4(L, L->loc_pass, grid_tiles, s));
+        else if (tc) ST_TRY(run_experts_tc(L, L->loc_pass, nbox, grid_tiles, y, s));
         else ST_TRY(run_experts(L, L->loc_pass, nt, grid_tiles, cs_gu, cs_dn, y, s));
         if (!one) CUDA_TRY(cudaEventRecord(L->ev_done[half], s));
       }
@@ -954,7 +1138,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   L->st.forwards += 1;
   L->st.last_misses = misses_n;
   L->st.last_waves = waves;
-  L->st.last_path = a4 ? 1 : 0;
+  L->st.last_path = a4 ? 1 : (tc ? 2 : 0);
   if (resident) L->st.last_active = -1;
   return MOE_OK;
 }
@@ -1025,6 +1209,12 @@ moe_status_t moe_debug_read(moe_layer_t L, int32_t which, void *dst, uint64_t by
     case 7: src = L->prow_token; break;
     case 8: src = L->prow_pair; break;
     case 11: src = L->oprime; break;
+    case 12: src = L->txq; break;
+    case 13: src = L->txsf; break;
+    case 14: src = L->thq; break;
+    case 15: src = L->thsf; break;
+    case 16: src = L->tiles; break;
+    case 17: src = L->n_tiles; break;
     default: break;
   }
   if (!src) return fail(MOE_ERR_INVALID_ARG, "unknown or absent debug buffer");

@@ -1,0 +1,512 @@
+// expert_tc.cu -- EXACT numerics for MXFP4 experts on the tcgen05 tensor core.
+//
+// The pages' engines decode E2M1 to BF16 in registers and multiply with
+// mma.sync ("ro99/strata", description of the SM86 kernel).  On sm_100a the
+// tensor core can take E2M1 weights with their E8M0 block scales directly
+// (tcgen05.mma kind::mxf8f6f4, block32), but only against an 8-bit (or
+// narrower) second operand.  A bf16 activation v is therefore written as two
+// E4M3 "pieces" with their own UE8M0 block scales,
+//     v = 2^e1 * q1 + 2^e2 * q2,
+// q1 = RN_E4M3(v * 2^-e1) with e1 = floor(log2(max|v| of the 32-block)) - 7,
+// q2 = RN_E4M3(r * 2^-e2) for the remainder r.  A bf16 value has 8
+// significant bits and E4M3 holds 4, so q1 keeps the top four bits and the
+// remainder (at most four bits) is exact in q2: the split is exact for every
+// block element within 13 binades of the block maximum (smaller ones are
+// rounded at 2^-9 of the piece scale).  Both pieces are rows of the B operand
+// (N = 2 x tokens); the epilogue adds the two columns of each token, so one
+// MMA pass over the weight tile computes the exact products accumulated in
+// fp32.  The weights' own scales are the A scale factors, unchanged.
+//
+// The same split is applied to h = silu(a) * u (fp32) in the gate/up
+// epilogue: there the two pieces keep about nine significant bits, the
+// precision of a bf16 h.
+//
+// Kernels:
+//  * tc_quant_x_kernel: gathers each tile's token rows of x (expert-sorted
+//    order) and writes the two E4M3 pieces and their scale-factor blocks;
+//  * expert_tc_kernel<GATEUP|DOWN, NBOX>: one CTA per (tile, 128 weight rows);
+//    a producer warp streams 128x128 weight tiles (TMA unpacks the E2M1 codes
+//    to one byte per element), the matching 128-element slab of the tile's
+//    activation pieces and both scale-factor blocks into a ring of stages;
+//    one thread issues the MMAs (M = 128, N = 2 x tokens, K = 32 each) into
+//    TMEM; four warps read the accumulators back.  Gate/up stages alternate
+//    gate and up tiles of the same K slab (two accumulators) and the epilogue
+//    computes SwiGLU and the pieces of h; down scales by the gate, writes O'
+//    and the last arrival per (token, row block) sums the token's k rows in
+//    fixed order (plus the shared expert) into y.
+//  All mbarrier waits are bounded (error word, then the kernel runs out).
+#include "device_utils.cuh"
+#include "moe_internal.h"
+#include "tcgen05.cuh"
+#include "tma.cuh"
+
+namespace moe {
+
+namespace {
+
+// warp 0: weight TMA; warp 1: TMEM allocation and MMA issue; warps 2..5:
+// epilogue; warps 6..7: activation pieces and scale factors by cp.async (the
+// LSU path), so that the per-SM TMA unit carries only the weight stream
+constexpr int kTcThreads = 256;
+constexpr int kTcLoaders = 64;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the barrier's expected count includes these arrivals).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+
+__device__ __forceinline__ int floor_log2_pos(float v) {   // v > 0 finite; subnormals give -127
+  const int ex = (int)((__float_as_uint(v) >> 23) & 0xFF);
+  return ex == 0 ? -127 : ex - 127;
+}
+
+__device__ __forceinline__ float exp2_int(int e) {          // 2^e for e in [-126, 127]
+  return __int_as_float((e + 127) << 23);
+}
+
+// Two E4M3 codes: `lo` in bits 0..7, `hi` in bits 8..15.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)(code & 0xFFu));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Block exponents of the split.  e1 from the block maximum of |v|; e2
+// (absolute) from the maximum of the remainders, in the units of 2^e1.
+__device__ __forceinline__ int split_e1(float amax) {
+  return amax > 0.0f ? max(-127, floor_log2_pos(amax) - 7) : 0;
+}
+__device__ __forceinline__ int split_e2rel(float rmax, int e1) {
+  if (!(rmax > 0.0f)) return 0;
+  int e = floor_log2_pos(rmax) - 7;
+  e = max(e, -120);
+  return max(e, -127 - e1);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// x pieces: one warp per (tile, token of the tile); lane handles 32-blocks
+// lane, lane + 32, ...
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) tc_quant_x_kernel(const TcQuantArgs q) {
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int tile = gw / q.tile_tokens, j = gw % q.tile_tokens;
+  if (tile >= q.max_tiles || tile >= *q.n_tiles) return;
+  const TileInfo ti = q.tiles[tile];
+  if (j >= ti.nrows) return;
+  const int token = q.prow_token[ti.prow0 + j];
+  const int H = q.H, nsf = H / 32;
+  const size_t row0 = (size_t)tile * kTcSlotRows + 2 * j;
+  const uint16_t *xr = q.x + (size_t)token * H;
+  const bool vec = ((reinterpret_cast<uintptr_t>(xr) & 15u) == 0);
+  for (int b = lane; b < nsf; b += 32) {
+    float v[32];
+    if (vec) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(xr + b * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 u = __ldg(src + i);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          v[8 * i + 2 * c] = __uint_as_float(w[c] << 16);
+          v[8 * i + 2 * c + 1] = __uint_as_float(w[c] & 0xFFFF0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = bf16_bits_to_float(xr[b * 32 + i]);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int e1 = split_e1(amax);
+    const float inv1 = exp2_int(-e1);
+    uint32_t c1[8];
+    float rmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float w0 = v[2 * i] * inv1, w1 = v[2 * i + 1] * inv1;
+      const uint32_t pr = e4m3x2(w0, w1);
+      const float r0 = w0 - e4m3_value(pr), r1 = w1 - e4m3_value(pr >> 8);
+      v[2 * i] = r0;
+      v[2 * i + 1] = r1;
+      rmax = fmaxf(rmax, fmaxf(fabsf(r0), fabsf(r1)));
+      if (i & 1) c1[i >> 1] |= pr << 16;
+      else c1[i >> 1] = pr;
+    }
+    const int e2r = split_e2rel(rmax, e1);
+    const float inv2 = exp2_int(-e2r);
+    uint32_t c2[8];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t pr = e4m3x2(v[2 * i] * inv2, v[2 * i + 1] * inv2);
+      if (i & 1) c2[i >> 1] |= pr << 16;
+      else c2[i >> 1] = pr;
+    }
+    uint4 *d1 = reinterpret_cast<uint4 *>(q.xq + row0 * H + b * 32);
+    uint4 *d2 = reinterpret_cast<uint4 *>(q.xq + (row0 + 1) * H + b * 32);
+    d1[0] = make_uint4(c1[0], c1[1], c1[2], c1[3]);
+    d1[1] = make_uint4(c1[4], c1[5], c1[6], c1[7]);
+    d2[0] = make_uint4(c2[0], c2[1], c2[2], c2[3]);
+    d2[1] = make_uint4(c2[4], c2[5], c2[6], c2[7]);
+    q.xsf[sf_offset(nsf, (int)row0, b)] = (uint8_t)(e1 + 127);
+    q.xsf[sf_offset(nsf, (int)row0 + 1, b)] = (uint8_t)(e1 + e2r + 127);
+  }
+}
+
+void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s) {
+  const long warps = (long)q.max_tiles * q.tile_tokens;
+  const int blocks = (int)((warps + 7) / 8);
+  if (blocks > 0) tc_quant_x_kernel<<<blocks, 256, 0, s>>>(q);
+}
+
+// ---------------------------------------------------------------------------
+// Expert pass on the tensor core, persistent.  A work item is (tile, 256
+// weight rows): gate/up = 128 gate rows + the same 128 up rows (one 4-D TMA
+// box), down = 256 output rows (one 3-D box); each half has its own
+// accumulator.  Items are taken round-robin by the CTAs; the stage ring runs
+// across items, and the accumulators are double-buffered (NBOX = 32) so the
+// epilogue of one item overlaps the main loop of the next.
+// ---------------------------------------------------------------------------
+namespace {
+template <int NBOX>
+struct TcGeom {
+  static constexpr int STAGES = NBOX <= 32 ? 5 : 4;
+  static constexpr int A_BYTES = 2 * 128 * 128;      // two 128 x 128 tiles, E2M1 unpacked to bytes
+  static constexpr int A_TX = 2 * 128 * 128 / 2;     // bytes the TMA moves for them (packed)
+  static constexpr int B_OFF = A_BYTES;
+  static constexpr int B_BYTES = NBOX * 128;         // NBOX piece rows x 128 E4M3
+  static constexpr int SF_OFF = B_OFF + B_BYTES;     // SFA half 0, SFA half 1, SFB: 512 B each
+  static constexpr int STAGE = ((SF_OFF + 3 * 512) + 1023) / 1024 * 1024;
+  static constexpr int NBUF = NBOX <= 32 ? 2 : 1;    // accumulator buffers
+  static constexpr int SF_COL0 = NBUF * 2 * NBOX;    // TMEM: accumulators first
+  static constexpr int COLS_NEEDED = SF_COL0 + 12 * STAGES;
+  static constexpr int TMEM_COLS = COLS_NEEDED <= 128 ? 128 : (COLS_NEEDED <= 256 ? 256 : 512);
+  static_assert(COLS_NEEDED <= 512, "TMEM budget");
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024;
+};
+}  // namespace
+
+template <int MODE, int NBOX>
+__global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_constant__ TcArgs a) {
+  using Geo = TcGeom<NBOX>;
+  constexpr int S = Geo::STAGES;
+  constexpr int NBUF = Geo::NBUF;
+  extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[S];    // weights landed (TMA)
+  __shared__ __align__(8) uint64_t bfull_bar[S];   // activation pieces + scale factors landed (cp.async)
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ __align__(8) uint64_t accf_bar[NBUF];
+  __shared__ __align__(8) uint64_t acce_bar[NBUF];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int last_tok[NBOX / 2];
+
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = a.K;
+  const int nslab = K / 128;
+  const int nsf = K / 32;
+  const int n_tiles = *a.n_tiles;
+  const int ipt = a.n_rowblocks;                      // items per tile
+  const int n_items = n_tiles * ipt;
+  const int region_map = (MODE == MODE_GATEUP) ? 0 : 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&bfull_bar[s]), kTcLoaders);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(smem_u32(&accf_bar[b]), 1);
+      mbar_init(smem_u32(&acce_bar[b]), 4);           // one arrival per epilogue warp
+    }
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_base_s), Geo::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+
+  if (warp == 0) {
+    // ---------------- producer
+    if (lane == 0) {
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      bool failed = false;
+      for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
+        const int tile = item / ipt, rb = item % ipt;
+        const TileInfo ti = a.tiles[tile];
+        const int loc = a.loc[ti.expert];
+        if (loc == kLocAbsent) continue;
+        const bool in_slot = loc >= 0;
+        const int bidx = in_slot ? loc : (-2 - loc);
+        const int region = in_slot ? 0 : 1;
+        const CUtensorMap *wm = &a.maps.w[region][region_map];
+        for (int slab = 0; slab < nslab; ++slab) {
+          if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 32)) { failed = true; break; }
+          const uint32_t bar = smem_u32(&full_bar[s]);
+          const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+          mbar_arrive_expect_tx(bar, (uint32_t)Geo::A_TX);
+          tma_load_4d(st, wm, bar, 0, 0, rb * nslab + slab, bidx);   // one contiguous 16 KB chunk
+          ++issued;
+          if (++s == S) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (failed) {
+        // let the copies already issued land before the CTA exits
+        int s2 = 0;
+        uint32_t ph2 = 0;
+        for (int i = 0; i < issued; ++i) {
+          if (i >= issued - S) mbar_drain(smem_u32(&full_bar[s2]), ph2);
+          if (++s2 == S) { s2 = 0; ph2 ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one lane)
+    if (lane == 0) {
+      int s = 0, n = 0;
+      uint32_t ph = 0;
+      bool failed = false;
+      for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
+        const int tile = item / ipt;
+        const TileInfo ti = a.tiles[tile];
+        if (a.loc[ti.expert] == kLocAbsent) continue;
+        const int N = max(16, (2 * ti.nrows + 15) & ~15);    // piece rows rounded up to 16
+        const int buf = n % NBUF;
+        // the epilogue must have drained this accumulator buffer
+        if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 34)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX);
+        for (int slab = 0; slab < nslab; ++slab) {
+          if (!mbar_wait(smem_u32(&full_bar[s]), ph, a.err, 31) ||
+              !mbar_wait(smem_u32(&bfull_bar[s]), ph, a.err, 36)) {
+            failed = true;
+            break;
+          }
+          fence_proxy_async();                               // cp.async data -> tensor-core reads
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+          const uint32_t sf = tmem + (uint32_t)(Geo::SF_COL0 + 12 * s);
+          tc_cp_sf_block(sf, st + Geo::SF_OFF);
+          tc_cp_sf_block(sf + 4, st + Geo::SF_OFF + 512);
+          tc_cp_sf_block(sf + 8, st + Geo::SF_OFF + 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {                  // K = 32 per MMA
+            const uint64_t bdesc = umma_desc(st + Geo::B_OFF + 32 * kk, 16, 1024, 2);
+            const uint32_t idesc = idesc_f8f6f4_block(128, N, kFmtE2M1_f8f6f4, kFmtE4M3, (uint32_t)kk, (uint32_t)kk);
+            const uint32_t sfb = (sf + 8) | ((uint32_t)kk << 30);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t adesc = umma_desc(st + h * 16384 + 32 * kk, 16, 1024, 2);
+              umma_mxf8f6f4(acc + (uint32_t)(h * NBOX), adesc, bdesc, idesc, (sf + 4 * h) | ((uint32_t)kk << 30),
+                            sfb, (slab > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(smem_u32(&empty_bar[s]));                // stage free once these MMAs finish
+          if (++s == S) { s = 0; ph ^= 1u; }
+        }
+        tc_commit(smem_u32(&accf_bar[buf]));                 // this item's accumulators complete
+        ++n;
+      }
+    }
+  } else if (warp >= 6) {
+    // ---------------- loaders: the tile's activation-piece rows of this K slab
+    // (written with the 128-byte swizzle the MMA descriptor expects) and the
+    // three scale-factor blocks, by 16-byte cp.async
+    const int lt = threadIdx.x - 192;
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    bool failed = false;
+    for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
+      const int tile = item / ipt, rb = item % ipt;
+      const TileInfo ti = a.tiles[tile];
+      const int loc = a.loc[ti.expert];
+      if (loc == kLocAbsent) continue;
+      const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
+      const int act_row0 = tile * kTcSlotRows;
+      // scale blocks of the chunk's two halves (1 KB per chunk), and of the activation rows
+      const uint8_t *sfa = blob + a.L.scales[MODE == MODE_GATEUP ? 0 : 2] + (size_t)rb * nslab * kTcSfChunk;
+      const uint8_t *sfb = a.bsf + sf_offset(nsf, act_row0, 0);
+      const uint8_t *act = a.act + (size_t)act_row0 * K;
+      const int nb = 8 * max(16, (2 * ti.nrows + 15) & ~15);   // 16-byte chunks of the piece rows read
+      for (int slab = 0; slab < nslab; ++slab) {
+        if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 35)) { failed = true; break; }
+        const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+        for (int c = lt; c < nb + 96; c += kTcLoaders) {
+          if (c < nb) {
+            const int r = c >> 3, q = c & 7;
+            cp_async16(st + Geo::B_OFF + r * 128 + ((q ^ (r & 7)) << 4), act + (size_t)r * K + slab * 128 + q * 16);
+          } else {
+            const int cc = c - nb;
+            const uint8_t *src = cc < 64 ? sfa + (size_t)slab * kTcSfChunk + cc * 16
+                                         : sfb + (size_t)slab * 512 + (cc - 64) * 16;
+            cp_async16(st + Geo::SF_OFF + cc * 16, src);
+          }
+        }
+        cp_async_arrive(smem_u32(&bfull_bar[s]));
+        ++issued;
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+    }
+    cp_async_wait_all();
+  } else {
+    // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+    const int quad = warp & 3;
+    const int et = threadIdx.x - 64;                         // 0..127 (warps 2..5)
+    int n = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int tile = item / ipt, rb = item % ipt;
+      const TileInfo ti = a.tiles[tile];
+      if (a.loc[ti.expert] == kLocAbsent) continue;
+      const int ntok = ti.nrows;
+      const int act_row0 = tile * kTcSlotRows;
+      const int buf = n % NBUF;
+      ok = mbar_wait(smem_u32(&accf_bar[buf]), (n / NBUF) & 1, a.err, 33);
+      ok = named_bar_and(1, 128, ok);                        // one decision for all four warps
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX) + ((uint32_t)(32 * quad) << 16);
+      if constexpr (MODE == MODE_GATEUP) {
+        const int I = a.rows, nsf_h = I / 32;
+        const int r = rb * 128 + 32 * quad + lane;           // h column
+        for (int c0 = 0; c0 < 2 * ntok; c0 += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(acc + (uint32_t)c0, g);
+          tmem_ld32(acc + (uint32_t)(NBOX + c0), u);
+          tmem_ld_wait();
+          if (!ok) continue;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = c0 / 2 + jj;
+            if (j >= ntok) continue;                         // warp-uniform
+            const float av = __uint_as_float(g[2 * jj]) + __uint_as_float(g[2 * jj + 1]);
+            const float uv = __uint_as_float(u[2 * jj]) + __uint_as_float(u[2 * jj + 1]);
+            const float h = silu_f(av) * uv;
+            float amax = fabsf(h);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const int e1 = split_e1(amax);
+            const float w = h * exp2_int(-e1);
+            const uint32_t c1 = e4m3x2(w, 0.0f) & 0xFFu;
+            const float rr = w - e4m3_value(c1);
+            float rmax = fabsf(rr);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, o));
+            const int e2r = split_e2rel(rmax, e1);
+            const uint32_t c2 = e4m3x2(rr * exp2_int(-e2r), 0.0f) & 0xFFu;
+            const size_t row = (size_t)act_row0 + 2 * j;
+            a.hq[row * I + r] = (uint8_t)c1;
+            a.hq[(row + 1) * I + r] = (uint8_t)c2;
+            if (lane == 0) {
+              a.hsf[sf_offset(nsf_h, (int)row, r / 32)] = (uint8_t)(e1 + 127);
+              a.hsf[sf_offset(nsf_h, (int)row + 1, r / 32)] = (uint8_t)(e1 + e2r + 127);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&acce_bar[buf]));
+      } else {
+        const int H = a.rows;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int r = rb * 256 + hh * 128 + 32 * quad + lane;   // output row
+          for (int c0 = 0; c0 < 2 * ntok; c0 += 32) {
+            uint32_t d[32];
+            tmem_ld32(acc + (uint32_t)(hh * NBOX + c0), d);
+            tmem_ld_wait();
+            if (!ok) continue;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = c0 / 2 + jj;
+              if (j >= ntok) continue;
+              const int p = a.prow_pair[ti.prow0 + j];
+              a.o_out[(size_t)p * H + r] =
+                  (__uint_as_float(d[2 * jj]) + __uint_as_float(d[2 * jj + 1])) * a.gates[p];
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&acce_bar[buf]));
+        // ordered combine by the last arrival of each token on these 256 rows
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (et < ntok) {
+          int t = -1;
+          if (ok) {
+            const int p = a.prow_pair[ti.prow0 + et];
+            const int tok = p / a.top_k;
+            if (atomicAdd(&a.comb_cnt[(size_t)tok * ipt + rb], 1) == a.top_k - 1) t = tok;
+          }
+          last_tok[et] = t;
+        }
+        named_bar_sync(1, 128);
+        __threadfence();
+        for (int j = 0; j < ntok; ++j) {
+          const int t = last_tok[j];
+          if (t < 0) continue;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = rb * 256 + hh * 128 + et;
+            const float *o = a.o_out + (size_t)t * a.top_k * H + r;
+            float v = __ldcg(o);
+            for (int q = 1; q < a.top_k; ++q) v += __ldcg(o + (size_t)q * H);
+            if (a.shared) v += __ldcg(a.shared + (size_t)t * H + r);
+            a.y[(size_t)t * H + r] = v;
+          }
+          if (et == 0) a.comb_cnt[(size_t)t * ipt + rb] = 0;
+        }
+        named_bar_sync(1, 128);                              // last_tok is reused by the next item
+      }
+      ++n;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Geo::TMEM_COLS);
+  }
+}
+
+template <int MODE, int NBOX>
+static void launch_tc_one(const TcArgs &a, cudaStream_t s) {
+  using Geo = TcGeom<NBOX>;
+  auto fn = expert_tc_kernel<MODE, NBOX>;
+  cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::SMEM);
+  fn<<<a.grid, kTcThreads, Geo::SMEM, s>>>(a);
+}
+
+void launch_expert_tc(int mode, int nbox, const TcArgs &a, int grid_tiles, cudaStream_t s) {
+  if (grid_tiles <= 0 || a.grid <= 0) return;
+  if (nbox <= 32) {
+    if (mode == MODE_GATEUP) launch_tc_one<MODE_GATEUP, 32>(a, s);
+    else launch_tc_one<MODE_DOWN, 32>(a, s);
+  } else {
+    if (mode == MODE_GATEUP) launch_tc_one<MODE_GATEUP, 128>(a, s);
+    else launch_tc_one<MODE_DOWN, 128>(a, s);
+  }
+}
+
+}  // namespace moe

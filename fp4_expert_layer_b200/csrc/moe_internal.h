@@ -36,9 +36,21 @@ struct BlobLayout {
   int K[3];
   int G;              // block size along K: 32 (MXFP4) or 16 (NVFP4)
   int fmt;
+  int tiled;          // 1: tile-major codes and scales (tensor-core EXACT layers), see below
 };
 
-BlobLayout blob_layout(int H, int I, int fmt);
+// tiled = 0: codes in checkpoint order ([rows, K/2] per matrix), scales in
+// 512-byte blocks (sf_offset).  tiled = 1 (MXFP4 layers on the tensor-core
+// EXACT path): every 16 KB chunk of codes the kernels stream is contiguous --
+//   gate/up, chunk rb * (H/128) + slab: gate rows rb*128 .. +127 then up rows
+//     rb*128 .. +127, 64 bytes (128 elements, K slab `slab`) each;
+//   down, chunk rb * (I/128) + slab: rows rb*256 .. +255, 64 bytes each;
+// and the scale blocks of a chunk (gate, up / rows 0..127, 128..255 of the
+// chunk) are one contiguous 1 KB at the same chunk index.  codes[0] / scales[0]
+// start the gate/up regions, codes[2] / scales[2] the down regions.
+BlobLayout blob_layout(int H, int I, int fmt, int tiled);
+constexpr int kTcChunk = 16384;      // code bytes of one tiled chunk
+constexpr int kTcSfChunk = 1024;     // scale bytes of one tiled chunk
 
 // Byte offset of scale (row r, scale column col) inside a matrix's scale area
 // with nsf scale columns per row: blocks of 128 rows x 4 columns (512 bytes),
@@ -238,5 +250,65 @@ struct A4GemmArgs {
   int *err;
 };
 void launch_gemm_a4(int wf, int mode, const A4GemmArgs &a, int grid_tiles, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// EXACT numerics on the tensor core (MXFP4 experts): the weights stay E2M1
+// with their E8M0 block scales; each activation row (x before gate/up, h
+// before down) is written as two E4M3 rows ("pieces") with one UE8M0 scale per
+// 32 elements each, v = s1 * q1 + s2 * q2, so that kind::mxf8f6f4 MMAs of the
+// E2M1 weights against both pieces sum to the product with the activation.
+// For a bf16 value the two pieces are exact; for the fp32 h they keep about
+// nine significant bits.  Activation rows live in per-tile slots of
+// kTcSlotRows rows: row kTcSlotRows * tile + 2 * j + piece for the tile's j-th
+// pair, so that every tile starts a 128-row scale-factor block.
+constexpr int kTcSlotRows = 128;
+
+struct TcMaps {
+  // [slot | staging][0 = gate and up together (4-D: K, rows, matrix, blob; box 128 x 128 x 2 x 1),
+  //                  1 = down (3-D: K, rows, blob; box 128 x 256 x 1)]: E2M1 codes unpacked by the
+  // TMA to one byte per element, 128-byte swizzle
+  CUtensorMap w[2][2];
+};
+
+struct TcQuantArgs {
+  const uint16_t *x;         // [T, H] bf16
+  int H;
+  const TileInfo *tiles;
+  const int *n_tiles;
+  int max_tiles, tile_tokens;
+  const int *prow_token;
+  uint8_t *xq;               // [max_tiles * kTcSlotRows, H] E4M3 pieces
+  uint8_t *xsf;              // scale-factor blocks of xq (UE8M0, per 32)
+};
+void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s);
+
+struct TcArgs {
+  TcMaps maps;
+  const int *loc;
+  const uint8_t *slots;
+  const uint8_t *staging;
+  size_t blob_bytes;
+  BlobLayout L;
+  int K, rows, n_rowblocks;  // reduction length, weight rows of the pass, rows / 128
+  const TileInfo *tiles;
+  const int *n_tiles;
+  const uint8_t *act;        // activation pieces [slot rows, K] E4M3 (x for gate/up, h for down)
+  const uint8_t *bsf;        // activation scale-factor blocks
+  // gate/up: h pieces for the down pass
+  uint8_t *hq, *hsf;
+  // down: O', then the ordered combine into y by the last arrival per (token, row block)
+  const int *prow_pair;
+  const float *gates;
+  float *o_out, *y;
+  const float *shared;
+  int *comb_cnt;
+  int top_k;
+  int *err;
+  int grid;                  // persistent CTAs
+};
+// nbox: activation rows per tile (2 x tile tokens): 32 or 128.  The kernel is
+// persistent: `a.grid` CTAs walk the work items (tile, 256 weight rows)
+// round-robin.
+void launch_expert_tc(int mode, int nbox, const TcArgs &a, int grid_tiles, cudaStream_t s);
 
 }  // namespace moe

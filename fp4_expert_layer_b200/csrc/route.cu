@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
   }
 
   // chunk-scaled f16 copy of x: warp per (token, 128-chunk)
-  if (blockIdx.y == 0) {
+  if (blockIdx.y == 0 && a.xf16) {
     const int nck = H / kChunk;
     for (int job = warp; job < nt * nck; job += kWarps) {
       const int t = job / nck, c = job % nck;

@@ -126,7 +126,9 @@ typedef struct {
   int32_t last_misses;     /* misses of the last forward                        */
   int32_t last_waves;      /* staging waves of the last forward (0 = resident)  */
   int32_t last_active;     /* experts with at least one token, last forward     */
-  int32_t last_path;       /* 0 = decode kernels, 1 = tcgen05 grouped GEMM      */
+  int32_t last_path;       /* 0 = register-decode kernels (EXACT), 1 = A4      */
+                           /* tcgen05 FP4 x FP4, 2 = EXACT on tcgen05 (MXFP4    */
+                           /* weights x E4M3 activation pieces)                 */
   uint64_t launches;       /* kernels this library launched, cumulative         */
   uint64_t expert_bytes;   /* device-layout bytes of one routed expert          */
   uint64_t device_bytes;   /* HBM held by the layer                             */
@@ -197,8 +199,9 @@ moe_status_t moe_get_stats(moe_layer_t layer, moe_stats_t *out);
  * waits for those events and returns the accumulated milliseconds and launch
  * counts since the last enable.  Stages: 0 router + top-k, 1 permutation,
  * 2 shared expert, 3 routed gate/up + SwiGLU, 4 routed down + gate scale,
- * 5 combine, 6 waits on staging copies, 7 whole forward. */
-#define MOE_PROFILE_STAGES 8
+ * 5 combine, 6 waits on staging copies, 7 whole forward, 8 A4 activation
+ * quantisation, 9 unused. */
+#define MOE_PROFILE_STAGES 10
 typedef struct {
   uint64_t forwards;
   double ms[MOE_PROFILE_STAGES];
@@ -246,7 +249,10 @@ moe_status_t moe_debug_inject(moe_layer_t layer, int32_t what);
 /* Test hook: synchronously copy up to `bytes` of an internal device buffer of
  * the last forward into host memory.  which: 1 quantised x codes, 2 x scale
  * blocks, 3 h (fp32, A4 path), 4 quantised h codes, 5 h scale blocks, 6 padded
- * row count, 7 padded row -> token, 8 padded row -> pair, 11 O' (fp32).
+ * row count, 7 padded row -> token, 8 padded row -> pair, 11 O' (fp32);
+ * tensor-core EXACT path: 12 x pieces (E4M3, 128-row slot per tile), 13 their
+ * scale blocks, 14 h pieces, 15 their scale blocks, 16 tile list, 17 tile
+ * count.
  * Returns MOE_ERR_INVALID_ARG for an unknown or absent buffer. */
 moe_status_t moe_debug_read(moe_layer_t layer, int32_t which, void *dst_host, uint64_t bytes);
 

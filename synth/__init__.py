@@ -85,6 +85,9 @@ WORKLOADS = {
         Workload("qwen3_30b_a3b_like", 2, 2048, 768, 128, 8, 0, "mxfp4", 1.1, (1, 16), 2048, 64, "hottest"),
         Workload("deepseek_v4_flash_like", 3, 4096, 2048, 256, 6, 2048, "mxfp4", None, (1, 64), 4096, 64, "random"),
         Workload("qwen3_8_flash_next_like", 4, 4096, 1024, 512, 10, 1024, "nvfp4", 1.1, (1, 4), 8192, 46, "hottest"),
+        # supplementary compute-bound probe: DeepSeek-V4-Flash-like expert shapes, 16 resident
+        # experts, 8192 tokens top-2 (about 1024 rows per expert)
+        Workload("fp4_peak_probe", 5, 4096, 2048, 16, 2, 0, "mxfp4", None, (1,), 8192, 16, "all"),
     ]
 }
 
