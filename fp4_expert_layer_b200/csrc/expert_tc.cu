@@ -49,6 +49,11 @@ namespace {
 // LSU path), so that the per-SM TMA unit carries only the weight stream
 constexpr int kTcThreads = 256;
 constexpr int kTcLoaders = 64;
+constexpr int kTcMeta = 64;       // work items per CTA whose descriptors are cached in shared memory
+
+// Programmatic dependent launch: wait until the preceding kernel on the stream
+// has completed and its memory is visible (a no-op for a normal launch).
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -102,6 +107,7 @@ __device__ __forceinline__ int split_e2rel(float rmax, int e1) {
 // lane, lane + 32, ...
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) tc_quant_x_kernel(const TcQuantArgs q) {
+  wait_prior_grid();
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int tile = gw / q.tile_tokens, j = gw % q.tile_tokens;
   if (tile >= q.max_tiles || tile >= *q.n_tiles) return;
@@ -168,10 +174,29 @@ __global__ void __launch_bounds__(256) tc_quant_x_kernel(const TcQuantArgs q) {
   }
 }
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// before its predecessor on the stream has finished; it waits with
+// griddepcontrol.wait before reading the predecessor's results.
+template <typename... Args>
+static void launch_dependent(void (*fn)(Args...), int grid, int block, size_t smem, cudaStream_t s,
+                             const Args &...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, fn, args...);
+}
+
 void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s) {
   const long warps = (long)q.max_tiles * q.tile_tokens;
   const int blocks = (int)((warps + 7) / 8);
-  if (blocks > 0) tc_quant_x_kernel<<<blocks, 256, 0, s>>>(q);
+  if (blocks > 0) launch_dependent(tc_quant_x_kernel, blocks, 256, 0, s, q);
 }
 
 // ---------------------------------------------------------------------------
@@ -214,15 +239,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
   __shared__ uint32_t tmem_base_s;
   __shared__ int last_tok[NBOX / 2];
+  // this CTA's first kTcMeta work items: tile descriptor and expert location,
+  // loaded once in parallel so that no role waits on dependent global loads
+  // at an item boundary
+  __shared__ TileInfo meta_ti[kTcMeta];
+  __shared__ int meta_loc[kTcMeta];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = a.K;
   const int nslab = K / 128;
   const int nsf = K / 32;
-  const int n_tiles = *a.n_tiles;
   const int ipt = a.n_rowblocks;                      // items per tile
-  const int n_items = n_tiles * ipt;
   const int region_map = (MODE == MODE_GATEUP) ? 0 : 1;
 
   if (threadIdx.x == 0) {
@@ -241,10 +269,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     tmem_alloc(smem_u32(&tmem_base_s), Geo::TMEM_COLS);
     tmem_relinquish();
   }
+  // everything above overlaps the previous kernel; the tile list is its output
+  wait_prior_grid();
+  const int n_items = *a.n_tiles * ipt;
+  if (warp == 0) {
+    for (int j = lane; j < kTcMeta; j += 32) {
+      const int item = blockIdx.x + j * gridDim.x;
+      if (item >= n_items) break;
+      const TileInfo ti = a.tiles[item / ipt];
+      meta_ti[j] = ti;
+      meta_loc[j] = a.loc[ti.expert];
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  // work item j of this CTA (item = blockIdx.x + j * gridDim.x)
+  auto item_tile = [&](int j, int item) -> TileInfo { return j < kTcMeta ? meta_ti[j] : a.tiles[item / ipt]; };
+  auto item_loc = [&](int j, const TileInfo &ti) -> int { return j < kTcMeta ? meta_loc[j] : a.loc[ti.expert]; };
 
   if (warp == 0) {
     // ---------------- producer
@@ -252,10 +295,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool failed = false;
-      for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
-        const int tile = item / ipt, rb = item % ipt;
-        const TileInfo ti = a.tiles[tile];
-        const int loc = a.loc[ti.expert];
+      for (int item = blockIdx.x, j = 0; item < n_items && !failed; item += gridDim.x, ++j) {
+        const int rb = item % ipt;
+        const TileInfo ti = item_tile(j, item);
+        const int loc = item_loc(j, ti);
         if (loc == kLocAbsent) continue;
         const bool in_slot = loc >= 0;
         const int bidx = in_slot ? loc : (-2 - loc);
@@ -287,10 +330,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       int s = 0, n = 0;
       uint32_t ph = 0;
       bool failed = false;
-      for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
-        const int tile = item / ipt;
-        const TileInfo ti = a.tiles[tile];
-        if (a.loc[ti.expert] == kLocAbsent) continue;
+      for (int item = blockIdx.x, j = 0; item < n_items && !failed; item += gridDim.x, ++j) {
+        const TileInfo ti = item_tile(j, item);
+        if (item_loc(j, ti) == kLocAbsent) continue;
         const int N = max(16, (2 * ti.nrows + 15) & ~15);    // piece rows rounded up to 16
         const int buf = n % NBUF;
         // the epilogue must have drained this accumulator buffer
@@ -337,10 +379,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     int s = 0, issued = 0;
     uint32_t ph = 0;
     bool failed = false;
-    for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
+    for (int item = blockIdx.x, j = 0; item < n_items && !failed; item += gridDim.x, ++j) {
       const int tile = item / ipt, rb = item % ipt;
-      const TileInfo ti = a.tiles[tile];
-      const int loc = a.loc[ti.expert];
+      const TileInfo ti = item_tile(j, item);
+      const int loc = item_loc(j, ti);
       if (loc == kLocAbsent) continue;
       const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
       const int act_row0 = tile * kTcSlotRows;
@@ -375,10 +417,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     const int et = threadIdx.x - 64;                         // 0..127 (warps 2..5)
     int n = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    for (int item = blockIdx.x, j = 0; item < n_items && ok; item += gridDim.x, ++j) {
       const int tile = item / ipt, rb = item % ipt;
-      const TileInfo ti = a.tiles[tile];
-      if (a.loc[ti.expert] == kLocAbsent) continue;
+      const TileInfo ti = item_tile(j, item);
+      if (item_loc(j, ti) == kLocAbsent) continue;
       const int ntok = ti.nrows;
       const int act_row0 = tile * kTcSlotRows;
       const int buf = n % NBUF;
@@ -495,7 +537,7 @@ static void launch_tc_one(const TcArgs &a, cudaStream_t s) {
   using Geo = TcGeom<NBOX>;
   auto fn = expert_tc_kernel<MODE, NBOX>;
   cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::SMEM);
-  fn<<<a.grid, kTcThreads, Geo::SMEM, s>>>(a);
+  launch_dependent(fn, a.grid, kTcThreads, Geo::SMEM, s, a);
 }
 
 void launch_expert_tc(int mode, int nbox, const TcArgs &a, int grid_tiles, cudaStream_t s) {
