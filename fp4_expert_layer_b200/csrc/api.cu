@@ -819,10 +819,6 @@ static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int 
   a.hq = L->thq;
   a.hsf = L->thsf;
   a.o_out = L->oprime;
-  a.y = y;
-  a.shared = c.shared_inter ? L->sh_s : nullptr;
-  a.comb_cnt = L->comb_cnt;
-  a.top_k = c.top_k;
   a.act = L->txq;
   a.K = c.hidden;
   a.rows = c.inter;
@@ -1118,9 +1114,10 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     }
   }
 
-  // EXACT: the ordered combine runs inside the routed down pass (last arrival
-  // per token); A4: a separate ordered combine.
-  if (a4) {
+  // register-decode EXACT kernels: the ordered combine runs inside the routed
+  // down pass (last arrival per token); tensor-core EXACT and A4: a separate
+  // ordered combine after the last pass.
+  if (a4 || tc) {
     CombineArgs ca{};
     ca.oprime = L->oprime;
     ca.shared = Is ? L->sh_s : nullptr;

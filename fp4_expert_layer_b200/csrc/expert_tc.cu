@@ -31,12 +31,13 @@
 //    one thread issues the MMAs (M = 128, N = 2 x tokens, K = 32 each) into
 //    TMEM; four warps read the accumulators back.  Gate/up stages alternate
 //    gate and up tiles of the same K slab (two accumulators) and the epilogue
-//    computes SwiGLU and the pieces of h; down scales by the gate, writes O'
-//    and the last arrival per (token, row block) sums the token's k rows in
-//    fixed order (plus the shared expert) into y.
+//    computes SwiGLU and the pieces of h; down scales by the gate and writes
+//    O' (the ordered combine into y is a separate kernel).
 //  All mbarrier waits are bounded (error word, then the kernel runs out).
 #include "device_utils.cuh"
 #include "moe_internal.h"
+#include "launch.cuh"
+#include "pieces.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
 
@@ -51,10 +52,6 @@ constexpr int kTcThreads = 256;
 constexpr int kTcLoaders = 64;
 constexpr int kTcMeta = 64;       // work items per CTA whose descriptors are cached in shared memory
 
-// Programmatic dependent launch: wait until the preceding kernel on the stream
-// has completed and its memory is visible (a no-op for a normal launch).
-__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -67,39 +64,6 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 
-__device__ __forceinline__ int floor_log2_pos(float v) {   // v > 0 finite; subnormals give -127
-  const int ex = (int)((__float_as_uint(v) >> 23) & 0xFF);
-  return ex == 0 ? -127 : ex - 127;
-}
-
-__device__ __forceinline__ float exp2_int(int e) {          // 2^e for e in [-126, 127]
-  return __int_as_float((e + 127) << 23);
-}
-
-// Two E4M3 codes: `lo` in bits 0..7, `hi` in bits 8..15.
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ float e4m3_value(uint32_t code) {
-  const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)(code & 0xFFu));
-  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-}
-
-// Block exponents of the split.  e1 from the block maximum of |v|; e2
-// (absolute) from the maximum of the remainders, in the units of 2^e1.
-__device__ __forceinline__ int split_e1(float amax) {
-  return amax > 0.0f ? max(-127, floor_log2_pos(amax) - 7) : 0;
-}
-__device__ __forceinline__ int split_e2rel(float rmax, int e1) {
-  if (!(rmax > 0.0f)) return 0;
-  int e = floor_log2_pos(rmax) - 7;
-  e = max(e, -120);
-  return max(e, -127 - e1);
-}
-
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -108,89 +72,10 @@ __device__ __forceinline__ int split_e2rel(float rmax, int e1) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) tc_quant_x_kernel(const TcQuantArgs q) {
   wait_prior_grid();
-  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int tile = gw / q.tile_tokens, j = gw % q.tile_tokens;
   if (tile >= q.max_tiles || tile >= *q.n_tiles) return;
-  const TileInfo ti = q.tiles[tile];
-  if (j >= ti.nrows) return;
-  const int token = q.prow_token[ti.prow0 + j];
-  const int H = q.H, nsf = H / 32;
-  const size_t row0 = (size_t)tile * kTcSlotRows + 2 * j;
-  const uint16_t *xr = q.x + (size_t)token * H;
-  const bool vec = ((reinterpret_cast<uintptr_t>(xr) & 15u) == 0);
-  for (int b = lane; b < nsf; b += 32) {
-    float v[32];
-    if (vec) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(xr + b * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 u = __ldg(src + i);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          v[8 * i + 2 * c] = __uint_as_float(w[c] << 16);
-          v[8 * i + 2 * c + 1] = __uint_as_float(w[c] & 0xFFFF0000u);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = bf16_bits_to_float(xr[b * 32 + i]);
-    }
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    const int e1 = split_e1(amax);
-    const float inv1 = exp2_int(-e1);
-    uint32_t c1[8];
-    float rmax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float w0 = v[2 * i] * inv1, w1 = v[2 * i + 1] * inv1;
-      const uint32_t pr = e4m3x2(w0, w1);
-      const float r0 = w0 - e4m3_value(pr), r1 = w1 - e4m3_value(pr >> 8);
-      v[2 * i] = r0;
-      v[2 * i + 1] = r1;
-      rmax = fmaxf(rmax, fmaxf(fabsf(r0), fabsf(r1)));
-      if (i & 1) c1[i >> 1] |= pr << 16;
-      else c1[i >> 1] = pr;
-    }
-    const int e2r = split_e2rel(rmax, e1);
-    const float inv2 = exp2_int(-e2r);
-    uint32_t c2[8];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t pr = e4m3x2(v[2 * i] * inv2, v[2 * i + 1] * inv2);
-      if (i & 1) c2[i >> 1] |= pr << 16;
-      else c2[i >> 1] = pr;
-    }
-    uint4 *d1 = reinterpret_cast<uint4 *>(q.xq + row0 * H + b * 32);
-    uint4 *d2 = reinterpret_cast<uint4 *>(q.xq + (row0 + 1) * H + b * 32);
-    d1[0] = make_uint4(c1[0], c1[1], c1[2], c1[3]);
-    d1[1] = make_uint4(c1[4], c1[5], c1[6], c1[7]);
-    d2[0] = make_uint4(c2[0], c2[1], c2[2], c2[3]);
-    d2[1] = make_uint4(c2[4], c2[5], c2[6], c2[7]);
-    q.xsf[sf_offset(nsf, (int)row0, b)] = (uint8_t)(e1 + 127);
-    q.xsf[sf_offset(nsf, (int)row0 + 1, b)] = (uint8_t)(e1 + e2r + 127);
-  }
-}
-
-// Launch with programmatic stream serialisation: the kernel may be scheduled
-// before its predecessor on the stream has finished; it waits with
-// griddepcontrol.wait before reading the predecessor's results.
-template <typename... Args>
-static void launch_dependent(void (*fn)(Args...), int grid, int block, size_t smem, cudaStream_t s,
-                             const Args &...args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3((unsigned)block);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, fn, args...);
+  tc_quant_x_row(q, tile, j);
 }
 
 void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s) {
@@ -238,7 +123,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   __shared__ __align__(8) uint64_t accf_bar[NBUF];
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
   __shared__ uint32_t tmem_base_s;
-  __shared__ int last_tok[NBOX / 2];
   // this CTA's first kTcMeta work items: tile descriptor and expert location,
   // loaded once in parallel so that no role waits on dependent global loads
   // at an item boundary
@@ -414,7 +298,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   } else {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
     const int quad = warp & 3;
-    const int et = threadIdx.x - 64;                         // 0..127 (warps 2..5)
     int n = 0;
     bool ok = true;
     for (int item = blockIdx.x, j = 0; item < n_items && ok; item += gridDim.x, ++j) {
@@ -490,35 +373,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&acce_bar[buf]));
-        // ordered combine by the last arrival of each token on these 256 rows
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (et < ntok) {
-          int t = -1;
-          if (ok) {
-            const int p = a.prow_pair[ti.prow0 + et];
-            const int tok = p / a.top_k;
-            if (atomicAdd(&a.comb_cnt[(size_t)tok * ipt + rb], 1) == a.top_k - 1) t = tok;
-          }
-          last_tok[et] = t;
-        }
-        named_bar_sync(1, 128);
-        __threadfence();
-        for (int j = 0; j < ntok; ++j) {
-          const int t = last_tok[j];
-          if (t < 0) continue;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int r = rb * 256 + hh * 128 + et;
-            const float *o = a.o_out + (size_t)t * a.top_k * H + r;
-            float v = __ldcg(o);
-            for (int q = 1; q < a.top_k; ++q) v += __ldcg(o + (size_t)q * H);
-            if (a.shared) v += __ldcg(a.shared + (size_t)t * H + r);
-            a.y[(size_t)t * H + r] = v;
-          }
-          if (et == 0) a.comb_cnt[(size_t)t * ipt + rb] = 0;
-        }
-        named_bar_sync(1, 128);                              // last_tok is reused by the next item
       }
       ++n;
     }

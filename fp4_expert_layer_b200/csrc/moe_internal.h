@@ -296,13 +296,10 @@ struct TcArgs {
   const uint8_t *bsf;        // activation scale-factor blocks
   // gate/up: h pieces for the down pass
   uint8_t *hq, *hsf;
-  // down: O', then the ordered combine into y by the last arrival per (token, row block)
+  // down: O'[pair, H] = gate * (W_down . h)
   const int *prow_pair;
   const float *gates;
-  float *o_out, *y;
-  const float *shared;
-  int *comb_cnt;
-  int top_k;
+  float *o_out;
   int *err;
   int grid;                  // persistent CTAs
 };

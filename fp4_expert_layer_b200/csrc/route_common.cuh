@@ -1,0 +1,200 @@
+// route_common.cuh -- block-level pieces of the routing step shared by the
+// router kernels: warp top-k with renormalised gates, and the stable
+// token-to-expert permutation.
+#pragma once
+
+#include "device_utils.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+template <bool IDS_GLOBAL>
+__device__ __forceinline__ int load_id(const int *ids, int p) {
+  if constexpr (IDS_GLOBAL) return __ldcg(ids + p);
+  else return ids[p];
+}
+
+// Top-k of one token by one warp: lane holds the logits of experts lane,
+// lane + 32, ... in lv (-inf past E).  Ids in descending-logit order, lower
+// index first on ties; gates g_j = exp(l_j - l_max) / sum_i exp(l_i - l_max)
+// over the k chosen, summed in j order.  Writes ids / gates (k entries each)
+// and, if ids_s is not null, the ids to shared memory too.
+template <int KPER>
+__device__ __forceinline__ void topk_warp(const float (&lv)[KPER], int E, int k, int *ids, float *gates,
+                                          int *ids_s) {
+  const int lane = threadIdx.x & 31;
+  uint32_t taken = 0;   // bit i: lane's i-th expert already chosen
+  float lmax = 0.0f, den = 0.0f;
+  float my_l = 0.0f;    // lane j keeps the logit of choice j
+  int my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < KPER; ++i) {
+      const int ee = lane + 32 * i;
+      if (ee < E && !((taken >> i) & 1u)) {
+        if (bi == 0x7fffffff || lv[i] > bv) { bv = lv[i]; bi = ee; }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (j == 0) lmax = bv;
+    if (lane == j) { my_l = bv; my_id = bi; }
+  }
+  const float ex = (lane < k) ? expf(my_l - lmax) : 0.0f;
+  // ordered sum over j = 0..k-1
+  for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, ex, j);
+  if (lane < k) {
+    ids[lane] = my_id;
+    gates[lane] = ex / den;
+    if (ids_s) ids_s[lane] = my_id;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Permutation: stable counting sort of pair index p = t*k + j by expert, as a
+// block-level routine (NTH threads, `sm` = shared scratch of
+// (5E + 3 + (NTH/32)*E) ints).  Counts by shared-memory atomics, offsets /
+// padded offsets / tile offsets by one block scan, then pairs are placed in
+// chunks of NTH: ranks inside a chunk come from warp match plus per-warp counts
+// scanned in warp order, so equal experts keep ascending p (stable).  The
+// expert ids are read from global memory (IDS_GLOBAL, another CTA wrote them)
+// or from this CTA's shared memory.
+// ---------------------------------------------------------------------------
+template <int NTH, bool IDS_GLOBAL>
+__device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
+  constexpr int W = NTH / 32;
+  __shared__ int4 wsum[W];
+  const int E = a.E;
+  int *cnt = sm;                  // [E]
+  int *cursor = cnt + E;          // [E]
+  int *off = cursor + E;          // [E+1]
+  int *poff = off + E + 1;        // [E+1] padded (multiple of 8) offsets
+  int *toff = poff + E + 1;       // [E+1] tile offsets
+  int *wcnt = toff + E + 1;       // [W][E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int i = tid; i < E; i += NTH) { cnt[i] = 0; cursor[i] = 0; }
+  for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;
+  __syncthreads();
+  for (int p = tid; p < a.n_pairs; p += NTH) atomicAdd(&cnt[load_id<IDS_GLOBAL>(ids, p)], 1);
+  __syncthreads();
+
+  // block exclusive scan of (count, padded count, tiles, active) over experts
+  const int per = (E + NTH - 1) / NTH;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+  int4 v = make_int4(0, 0, 0, 0);
+  for (int e = e0; e < e1; ++e) {
+    const int c = cnt[e];
+    v.x += c;
+    v.y += (c + a.pad - 1) / a.pad * a.pad;
+    v.z += (c + a.tile_tokens - 1) / a.tile_tokens;
+    v.w += c > 0;
+  }
+  int4 inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int4 t;
+    t.x = __shfl_up_sync(0xffffffffu, inc.x, o);
+    t.y = __shfl_up_sync(0xffffffffu, inc.y, o);
+    t.z = __shfl_up_sync(0xffffffffu, inc.z, o);
+    t.w = __shfl_up_sync(0xffffffffu, inc.w, o);
+    if (lane >= o) { inc.x += t.x; inc.y += t.y; inc.z += t.z; inc.w += t.w; }
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int4 w = lane < W ? wsum[lane] : make_int4(0, 0, 0, 0);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int4 t;
+      t.x = __shfl_up_sync(0xffffffffu, w.x, o);
+      t.y = __shfl_up_sync(0xffffffffu, w.y, o);
+      t.z = __shfl_up_sync(0xffffffffu, w.z, o);
+      t.w = __shfl_up_sync(0xffffffffu, w.w, o);
+      if (lane >= o) { w.x += t.x; w.y += t.y; w.z += t.z; w.w += t.w; }
+    }
+    if (lane < W) wsum[lane] = w;
+  }
+  __syncthreads();
+  {
+    const int4 pre = warp > 0 ? wsum[warp - 1] : make_int4(0, 0, 0, 0);
+    int o = pre.x + inc.x - v.x, po = pre.y + inc.y - v.y, to = pre.z + inc.z - v.z;
+    for (int e = e0; e < e1; ++e) {
+      const int c = cnt[e];
+      off[e] = o; poff[e] = po; toff[e] = to;
+      o += c;
+      po += (c + a.pad - 1) / a.pad * a.pad;
+      to += (c + a.tile_tokens - 1) / a.tile_tokens;
+    }
+    if (tid == NTH - 1) {
+      const int4 tot = wsum[W - 1];
+      off[E] = tot.x; poff[E] = tot.y; toff[E] = tot.z;
+      *a.n_tiles = tot.z;
+      *a.active = tot.w;
+      if (a.n_prows) *a.n_prows = tot.y;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e <= E; e += NTH) a.offsets[e] = off[e];
+  for (int e = tid; e < E; e += NTH) {
+    const int c = cnt[e];
+    a.counts[e] = c;
+    const int nt = (c + a.tile_tokens - 1) / a.tile_tokens;
+    for (int i = 0; i < nt; ++i) {
+      TileInfo ti;
+      ti.expert = e;
+      ti.prow0 = poff[e] + i * a.tile_tokens;
+      ti.nrows = min(a.tile_tokens, c - i * a.tile_tokens);
+      ti.sorted0 = off[e] + i * a.tile_tokens;
+      a.tiles[toff[e] + i] = ti;
+    }
+    for (int r = poff[e] + c; r < poff[e + 1]; ++r) { a.prow_token[r] = -1; a.prow_pair[r] = -1; }
+  }
+
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < a.n_pairs; base += NTH) {
+    const int p = base + tid;
+    const bool valid = p < a.n_pairs;
+    const int e = valid ? load_id<IDS_GLOBAL>(ids, p) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & lt_mask);
+    if (valid && rank == 0) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += NTH) {
+      int run = cursor[ee];
+      for (int w = 0; w < W; ++w) {
+        const int c = wcnt[w * E + ee];
+        wcnt[w * E + ee] = run;
+        run += c;
+      }
+      cursor[ee] = run;
+    }
+    __syncthreads();
+    if (valid) {
+      const int local = wcnt[warp * E + e] + rank;
+      const int pos = off[e] + local;
+      const int prow = poff[e] + local;
+      a.perm[pos] = p;
+      a.inv[p] = pos;
+      a.prow_token[prow] = p / a.k;
+      a.prow_pair[prow] = p;
+    }
+    __syncthreads();
+    for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;
+    __syncthreads();
+  }
+}
+
+__host__ __device__ inline size_t perm_smem_ints(int E, int nth) { return (size_t)5 * E + 3 + (size_t)(nth / 32) * E; }
+
+}  // namespace moe
