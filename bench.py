@@ -137,16 +137,23 @@ def layer_bytes(wl, n_active, T):
     return b
 
 
-def traffic_record(kernel_src):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
-    path = os.path.join(ROOT, "profiles", "expert_tma_gateup_olmoe_like_T32_traffic.json")
+def traffic_record(summary, kernel_src):
+    """DRAM bytes per launch from a committed ncu summary (profiles/<summary>), if it
+    was taken on the kernel source as it is now (its sha256 is recorded there)."""
+    path = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(path):
         return None
+    rec = {}
     with open(path) as f:
-        rec = json.load(f)
+        for line in f:
+            if ":" in line and line.lstrip().startswith(("dram_bytes_per_launch", "kernel_source_sha256")):
+                k, v = line.split(":", 1)
+                rec[k.strip(" -*`")] = v.strip(" `\n")
     with open(kernel_src, "rb") as f:
         h = hashlib.sha256(f.read()).hexdigest()
-    return rec.get("dram_bytes_per_launch") if rec.get("kernel_sha256") == h else None
+    if rec.get("kernel_source_sha256") != h or "dram_bytes_per_launch" not in rec:
+        return None
+    return float(rec["dram_bytes_per_launch"])
 
 
 # ------------------------------------------------------------------ CPU (oracle) legs
@@ -342,7 +349,8 @@ def main():
         g_ms = prof["ms"]["gateup"] / max(1, prof["launches"]["gateup"])
         if args.numerics == "a4":
             # tcgen05 gate/up GEMM: FP4 FLOPs of the real (unpadded) token rows
-            g_flops = 4.0 * T * wl.top_k * wl.hidden * wl.inter
+            waves = max(1.0, prof["launches"]["gateup"] / max(1, prof["forwards"]))
+            g_flops = 4.0 * T * wl.top_k * wl.hidden * wl.inter / waves
             achieved = g_flops / (g_ms / 1e3) / 1e12
             # the GEMM runs back to back for seconds inside the step loop: sustained figure
             fp4_peak = 4.0 * bf16_sus
@@ -353,12 +361,19 @@ def main():
                     "algorithmic_flops_per_launch": g_flops, "kernel_ms": g_ms,
                     "hbm_gbs_of_same_launch": gateup_bytes(wl, n_active, T) / (g_ms / 1e3) / 1e9}
         else:
-            g_bytes = gateup_bytes(wl, n_active, T)
+            # paged runs launch the pass once per staging wave: bytes per launch
+            waves = max(1.0, prof["launches"]["gateup"] / max(1, prof["forwards"]))
+            g_bytes = gateup_bytes(wl, n_active, T) / waves
             achieved = g_bytes / (g_ms / 1e3) / 1e9
-            traffic = traffic_record(os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert_tma.cu"))
+            tc = wl.fmt == "mxfp4"
+            src = os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert_tc.cu" if tc else "expert_tma.cu")
+            traffic = None
+            if tc and wl.name == "olmoe_like" and T == 32 and S == wl.n_experts:
+                traffic = traffic_record("expert_tc_gateup_olmoe_like_T32.md", src)
             roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                     "frac": achieved / hbm_peak, "traffic": traffic,
-                    "kernel": "expert_tma_kernel gate/up+SwiGLU (routed)",
+                    "kernel": ("expert_tc_kernel gate/up+SwiGLU (tcgen05, E2M1 weights x E4M3 activation pieces)"
+                               if tc else "expert_tma_kernel gate/up+SwiGLU (register decode, mma.sync)"),
                     "peak_source": f"{peak_src} hbm_gbs",
                     "algorithmic_bytes_per_launch": g_bytes, "kernel_ms": g_ms}
         stage_ms = {k: v / max(1, prof["forwards"]) for k, v in prof["ms"].items()}

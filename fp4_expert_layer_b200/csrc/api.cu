@@ -218,9 +218,9 @@ static Sizes sizes_of(const moe_config_t *c) {
   s.max_prows = s.P + 8 * act;
   s.max_tiles = s.P / 8 + act + 1;
   s.a4_rows = s.P + 128 * act + 128;     // padded to 128 rows per expert, + one tile of slack
-  // tensor-core EXACT path: tiles of 16 tokens only while P <= 12 * active experts
-  // (then at most 1.75 x act tiles), else tiles of 64 tokens
-  s.tc_tiles = std::max(s.P / 64 + act, (7 * act) / 4 + 1) + 2;
+  // tensor-core EXACT path: tiles of 8 tokens only while P <= 12 * active experts
+  // (then at most 2.5 x act tiles), else tiles of 64 tokens
+  s.tc_tiles = std::max(s.P / 64 + act, (5 * act) / 2 + 1) + 2;
   return s;
 }
 
@@ -927,9 +927,9 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   const int nt = avg <= 8 ? 1 : (avg <= 16 ? 2 : 4);
   const bool a4 = L->a4;
   const bool tc = L->tc;
-  // tensor-core EXACT: 16-token tiles (32 piece rows) while the batch is
-  // decode-sized, else 64-token tiles (128 piece rows)
-  const int nbox = (tc && P <= 12 * act_est) ? 32 : 128;
+  // tensor-core EXACT: 8-token tiles (16 piece rows, 6 stages in flight) while
+  // the batch is decode-sized, else 64-token tiles (128 piece rows)
+  const int nbox = (tc && P <= 12 * act_est) ? 16 : 128;
   const int ts = a4 ? 128 : (tc ? nbox / 2 : 8 * nt);
   const int grid_tiles = P / ts + act_est + 1;
 

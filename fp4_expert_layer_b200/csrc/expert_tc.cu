@@ -95,7 +95,7 @@ void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s) {
 namespace {
 template <int NBOX>
 struct TcGeom {
-  static constexpr int STAGES = NBOX <= 32 ? 5 : 4;
+  static constexpr int STAGES = NBOX <= 16 ? 6 : (NBOX <= 32 ? 5 : 4);
   static constexpr int A_BYTES = 2 * 128 * 128;      // two 128 x 128 tiles, E2M1 unpacked to bytes
   static constexpr int A_TX = 2 * 128 * 128 / 2;     // bytes the TMA moves for them (packed)
   static constexpr int B_OFF = A_BYTES;
@@ -128,6 +128,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   // at an item boundary
   __shared__ TileInfo meta_ti[kTcMeta];
   __shared__ int meta_loc[kTcMeta];
+  // down epilogue: pair index and gate of each token of the current item
+  __shared__ int tok_pair[NBOX / 2];
+  __shared__ float tok_gate[NBOX / 2];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,7 +310,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       const int ntok = ti.nrows;
       const int act_row0 = tile * kTcSlotRows;
       const int buf = n % NBUF;
+      const int et = threadIdx.x - 64;                       // 0..127 over warps 2..5
+      // down: load the item's pair indices and gates while its MMAs run
+      int my_pair = 0;
+      float my_gate = 0.0f;
+      if (MODE == MODE_DOWN && et < ntok) {
+        my_pair = __ldg(a.prow_pair + ti.prow0 + et);
+        my_gate = __ldg(a.gates + my_pair);
+      }
       ok = mbar_wait(smem_u32(&accf_bar[buf]), (n / NBUF) & 1, a.err, 33);
+      if (MODE == MODE_DOWN && et < ntok) {
+        tok_pair[et] = my_pair;
+        tok_gate[et] = my_gate;
+      }
       ok = named_bar_and(1, 128, ok);                        // one decision for all four warps
       tc_fence_after();
       const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX) + ((uint32_t)(32 * quad) << 16);
@@ -320,31 +335,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
           tmem_ld32(acc + (uint32_t)(NBOX + c0), u);
           tmem_ld_wait();
           if (!ok) continue;
+          // 16 tokens at a time: the warp reductions of different tokens are
+          // independent, so their shuffles overlap (columns past the tile's
+          // tokens hold no data and are never stored)
+          float w[16], am[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const float av = __uint_as_float(g[2 * jj]) + __uint_as_float(g[2 * jj + 1]);
+            const float uv = __uint_as_float(u[2 * jj]) + __uint_as_float(u[2 * jj + 1]);
+            w[jj] = silu_f(av) * uv;
+            am[jj] = fabsf(w[jj]);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) am[jj] = fmaxf(am[jj], __shfl_xor_sync(0xffffffffu, am[jj], o));
+          int e1[16];
+          uint32_t c1[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            e1[jj] = split_e1(am[jj]);
+            const float v = w[jj] * exp2_int(-e1[jj]);
+            c1[jj] = e4m3x2(v, 0.0f) & 0xFFu;
+            w[jj] = v - e4m3_value(c1[jj]);                   // remainder in units of 2^e1
+            am[jj] = fabsf(w[jj]);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) am[jj] = fmaxf(am[jj], __shfl_xor_sync(0xffffffffu, am[jj], o));
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int j = c0 / 2 + jj;
             if (j >= ntok) continue;                         // warp-uniform
-            const float av = __uint_as_float(g[2 * jj]) + __uint_as_float(g[2 * jj + 1]);
-            const float uv = __uint_as_float(u[2 * jj]) + __uint_as_float(u[2 * jj + 1]);
-            const float h = silu_f(av) * uv;
-            float amax = fabsf(h);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            const int e1 = split_e1(amax);
-            const float w = h * exp2_int(-e1);
-            const uint32_t c1 = e4m3x2(w, 0.0f) & 0xFFu;
-            const float rr = w - e4m3_value(c1);
-            float rmax = fabsf(rr);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, o));
-            const int e2r = split_e2rel(rmax, e1);
-            const uint32_t c2 = e4m3x2(rr * exp2_int(-e2r), 0.0f) & 0xFFu;
+            const int e2r = split_e2rel(am[jj], e1[jj]);
+            const uint32_t c2 = e4m3x2(w[jj] * exp2_int(-e2r), 0.0f) & 0xFFu;
             const size_t row = (size_t)act_row0 + 2 * j;
-            a.hq[row * I + r] = (uint8_t)c1;
+            a.hq[row * I + r] = (uint8_t)c1[jj];
             a.hq[(row + 1) * I + r] = (uint8_t)c2;
             if (lane == 0) {
-              a.hsf[sf_offset(nsf_h, (int)row, r / 32)] = (uint8_t)(e1 + 127);
-              a.hsf[sf_offset(nsf_h, (int)row + 1, r / 32)] = (uint8_t)(e1 + e2r + 127);
+              a.hsf[sf_offset(nsf_h, (int)row, r / 32)] = (uint8_t)(e1[jj] + 127);
+              a.hsf[sf_offset(nsf_h, (int)row + 1, r / 32)] = (uint8_t)(e1[jj] + e2r + 127);
             }
           }
         }
@@ -364,15 +395,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
             for (int jj = 0; jj < 16; ++jj) {
               const int j = c0 / 2 + jj;
               if (j >= ntok) continue;
-              const int p = a.prow_pair[ti.prow0 + j];
-              a.o_out[(size_t)p * H + r] =
-                  (__uint_as_float(d[2 * jj]) + __uint_as_float(d[2 * jj + 1])) * a.gates[p];
+              a.o_out[(size_t)tok_pair[j] * H + r] =
+                  (__uint_as_float(d[2 * jj]) + __uint_as_float(d[2 * jj + 1])) * tok_gate[j];
             }
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&acce_bar[buf]));
+        named_bar_sync(1, 128);                              // tok_pair / tok_gate are rewritten next item
       }
       ++n;
     }
@@ -396,7 +427,10 @@ static void launch_tc_one(const TcArgs &a, cudaStream_t s) {
 
 void launch_expert_tc(int mode, int nbox, const TcArgs &a, int grid_tiles, cudaStream_t s) {
   if (grid_tiles <= 0 || a.grid <= 0) return;
-  if (nbox <= 32) {
+  if (nbox <= 16) {
+    if (mode == MODE_GATEUP) launch_tc_one<MODE_GATEUP, 16>(a, s);
+    else launch_tc_one<MODE_DOWN, 16>(a, s);
+  } else if (nbox <= 32) {
     if (mode == MODE_GATEUP) launch_tc_one<MODE_GATEUP, 32>(a, s);
     else launch_tc_one<MODE_DOWN, 32>(a, s);
   } else {

@@ -61,7 +61,7 @@ def test_tile_list_covers_every_pair_once():
         k = wl.top_k
         counts = np.bincount(r["ids"].ravel(), minlength=wl.n_experts)
         assert tiles[:, 2].sum() == 32 * k
-        assert np.all(tiles[:, 2] >= 1) and np.all(tiles[:, 2] <= 16)
+        assert np.all(tiles[:, 2] >= 1) and np.all(tiles[:, 2] <= 8)
         for e in range(wl.n_experts):
             assert tiles[tiles[:, 0] == e, 2].sum() == counts[e]
         prow_pair = layer.debug_read(8, np.int32, int(tiles[:, 1].max() + 16))
@@ -168,6 +168,6 @@ def test_large_tiles_vs_oracle(T):
         G.check_routing(r, lg, ids, g, wl.n_experts)
         G.check_output(y, y_ref)
         tiles = _tiles(layer)
-        assert tiles[:, 2].max() > 16 and tiles[:, 2].max() <= 64
+        assert tiles[:, 2].max() > 8 and tiles[:, 2].max() <= 64
     finally:
         layer.close()
