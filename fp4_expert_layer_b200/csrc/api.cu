@@ -102,6 +102,9 @@ struct moe_layer {
   TileInfo *tiles = nullptr;
   int *n_tiles = nullptr, *active = nullptr, *prow_token = nullptr, *prow_pair = nullptr;
   uint16_t *xf16 = nullptr, *hbuf = nullptr, *sh_h = nullptr, *xin = nullptr;
+  // shared expert on the tensor core (prefill): bf16 weight maps and the h map
+  CUtensorMap sh_map[3];
+  CUtensorMap sh_hmap;
   float *xs = nullptr, *hscale = nullptr, *oprime = nullptr, *sh_s = nullptr, *yout = nullptr;
   int *router_counter = nullptr, *tiles_done = nullptr, *comb_cnt = nullptr;
   // A4 (activation FP4) path
@@ -397,6 +400,25 @@ static moe_status_t make_tc_weight_map(CUtensorMap *map, const uint8_t *region, 
   return MOE_OK;
 }
 
+// bf16 row-major [rows, K] map, box 64 elements (128 B) x 128 rows, 128-byte swizzle.
+static moe_status_t make_bf16_map(CUtensorMap *map, const void *base, size_t K, size_t rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K * 2)};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a bf16 map");
+  return MOE_OK;
+}
+
+// Tokens from which the shared expert runs on the tensor core (below that the
+// register kernels, which split K over a cluster, keep more SMs busy).
+constexpr int kDenseTcMinTokens = 256;
+
 // ------------------------------------------------------------------ C ABI
 extern "C" {
 
@@ -614,6 +636,12 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   C_TRY(dalloc(L, &L->router_counter, ((T + 3) / 4) * 4));
   C_TRY(dalloc(L, &L->tiles_done, 4));
   C_TRY(dalloc(L, &L->comb_cnt, T * (H / 128) * 4));
+  if (Is) {
+    C_TRY(make_bf16_map(&L->sh_map[0], L->shared_w[0], H, Is));
+    C_TRY(make_bf16_map(&L->sh_map[1], L->shared_w[1], H, Is));
+    C_TRY(make_bf16_map(&L->sh_map[2], L->shared_w[2], Is, H));
+    C_TRY(make_bf16_map(&L->sh_hmap, L->sh_h, Is, T));
+  }
   C_TRY(dalloc(L, &L->xin, T * H * 2));
   L->a4 = cfg->numerics == MOE_NUMERICS_A4;
   if (L->a4) {
@@ -982,7 +1010,29 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   }
 
   // always-resident shared expert (runs while the host builds the miss list)
-  if (Is) {
+  const bool dense_tc = Is && T >= kDenseTcMinTokens && (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
+  if (dense_tc) {
+    StageTimer t2(L, 2, s);
+    DenseTcArgs d{};
+    d.wmap[0] = L->sh_map[0];
+    d.wmap[1] = L->sh_map[1];
+    ST_TRY(make_bf16_map(&d.xmap, x, H, T));
+    d.T = T; d.K = H; d.rows = Is; d.n_rowblocks = Is / 128;
+    d.grid = std::min(((T + 127) / 128) * d.n_rowblocks, L->n_sms);
+    d.h_out = L->sh_h;
+    d.err = L->d_err;
+    launch_dense_tc(MODE_GATEUP, d, s);
+    CUDA_TRY(cudaGetLastError());
+    d.wmap[0] = L->sh_map[2];
+    d.xmap = L->sh_hmap;
+    d.K = Is; d.rows = H; d.n_rowblocks = H / 256;
+    d.grid = std::min(((T + 127) / 128) * d.n_rowblocks, L->n_sms);
+    d.s_out = L->sh_s;
+    launch_dense_tc(MODE_DOWN, d, s);
+    CUDA_TRY(cudaGetLastError());
+    t2.launched(2);
+    t2.end();
+  } else if (Is) {
     StageTimer t2(L, 2, s);
     const int snt = T <= 8 ? 1 : (T <= 16 ? 2 : 4);
     const int stiles = (T + 8 * snt - 1) / (8 * snt);

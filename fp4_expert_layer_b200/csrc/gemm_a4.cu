@@ -52,6 +52,11 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
   __shared__ __align__(8) uint64_t empty_bar[kGStages];
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t tmem_base_s;
+  // epilogue: per-column activation scale, pair index and gate of the tile,
+  // loaded once (the output stores would otherwise order every such load)
+  __shared__ float col_bs[128];
+  __shared__ int col_pair[128];
+  __shared__ float col_gate[128];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -155,6 +160,18 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
   } else if (warp >= 4) {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
     const int quad = warp & 3;
+    {
+      const int c = threadIdx.x - 128;                               // 0..127 over warps 4..7
+      if (c < nrows) {
+        col_bs[c] = (WF == WF_NV) ? __ldg(a.bG + prow0 + c) : 1.0f;
+        if constexpr (MODE == MODE_DOWN) {
+          const int p = __ldg(a.prow_pair + prow0 + c);
+          col_pair[c] = p;
+          col_gate[c] = __ldg(a.gates + p);
+        }
+      }
+      named_bar_sync(1, 128);
+    }
     mbar_wait(smem_u32(&acc_bar), 0, a.err, 13);
     tc_fence_after();
     const int r_local = 32 * quad + lane;
@@ -177,14 +194,13 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
         const int col = 32 * cb + jj;
         if (col >= nrows) continue;
         const int prow = prow0 + col;
-        const float bs = (WF == WF_NV) ? a.bG[prow] : 1.0f;
+        const float bs = col_bs[col];
         if constexpr (MODE == MODE_GATEUP) {
           const float av = __uint_as_float(d0[jj]) * (wsc[0] * bs);
           const float uv = __uint_as_float(d1[jj]) * (wsc[1] * bs);
           a.h_out[(size_t)prow * a.rows + row] = silu_f(av) * uv;
         } else {
-          const int p = a.prow_pair[prow];
-          a.o_out[(size_t)p * a.rows + row] = __uint_as_float(d0[jj]) * (wsc[0] * bs) * a.gates[p];
+          a.o_out[(size_t)col_pair[col] * a.rows + row] = __uint_as_float(d0[jj]) * (wsc[0] * bs) * col_gate[col];
         }
       }
     }

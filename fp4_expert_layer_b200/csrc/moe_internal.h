@@ -282,6 +282,17 @@ struct TcQuantArgs {
 };
 void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s);
 
+// Shared expert (bf16) on the tensor core for prefill-sized batches.
+struct DenseTcArgs {
+  CUtensorMap wmap[2];       // gate/up: gate [I_s, H], up [I_s, H]; down: [H, I_s] (bf16, box 64 x 128)
+  CUtensorMap xmap;          // activations bf16 [rows >= T, K], box 64 x 128
+  int T, K, rows, n_rowblocks, grid;
+  uint16_t *h_out;           // gate/up: bf16 [T, I_s]
+  float *s_out;              // down: fp32 [T, H]
+  int *err;
+};
+void launch_dense_tc(int mode, const DenseTcArgs &a, cudaStream_t s);
+
 struct TcArgs {
   TcMaps maps;
   const int *loc;
