@@ -146,9 +146,10 @@ def traffic_record(summary, kernel_src):
     rec = {}
     with open(path) as f:
         for line in f:
-            if ":" in line and line.lstrip().startswith(("dram_bytes_per_launch", "kernel_source_sha256")):
+            line = line.strip().lstrip("-* `")
+            if ":" in line and line.startswith(("dram_bytes_per_launch", "kernel_source_sha256")):
                 k, v = line.split(":", 1)
-                rec[k.strip(" -*`")] = v.strip(" `\n")
+                rec[k.strip()] = v.strip(" `")
     with open(kernel_src, "rb") as f:
         h = hashlib.sha256(f.read()).hexdigest()
     if rec.get("kernel_source_sha256") != h or "dram_bytes_per_launch" not in rec:
