@@ -91,6 +91,7 @@ struct moe_layer {
   // device memory
   std::vector<void *> dev;
   float *router_w = nullptr, *router_b = nullptr;
+  float *router_parts = nullptr;     // split-K partial logits of the prefill router GEMM
   uint16_t *shared_w[3] = {};
   uint8_t *slots = nullptr, *staging = nullptr;
   const uint8_t **ptr_resident = nullptr, **ptr_pass = nullptr;
@@ -261,6 +262,7 @@ static size_t scratch_bytes(const moe_config_t *c) {
   b += align256(((T + 3) / 4) * 4) + align256(4) + align256(T * (H / 128) * 4);
   b += align256(T * H * 2) + align256(T * H * 4);
   b += 2 * align256(E * sizeof(void *));
+  if (T >= 256) b += align256((size_t)(4 << 20) * 4);     // split-K partial logits (prefill router)
   return b;
 }
 
@@ -418,6 +420,7 @@ static moe_status_t make_bf16_map(CUtensorMap *map, const void *base, size_t K, 
 // Tokens from which the shared expert runs on the tensor core (below that the
 // register kernels, which split K over a cluster, keep more SMs busy).
 constexpr int kDenseTcMinTokens = 256;
+constexpr size_t kRouterPartFloats = (size_t)4 << 20;   // 16 MiB of split-K partial logits
 
 // ------------------------------------------------------------------ C ABI
 extern "C" {
@@ -636,6 +639,7 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   C_TRY(dalloc(L, &L->router_counter, ((T + 3) / 4) * 4));
   C_TRY(dalloc(L, &L->tiles_done, 4));
   C_TRY(dalloc(L, &L->comb_cnt, T * (H / 128) * 4));
+  if (T >= (size_t)kDenseTcMinTokens) C_TRY(dalloc(L, &L->router_parts, kRouterPartFloats * 4));
   if (Is) {
     C_TRY(make_bf16_map(&L->sh_map[0], L->shared_w[0], H, Is));
     C_TRY(make_bf16_map(&L->sh_map[1], L->shared_w[1], H, Is));
@@ -980,12 +984,25 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   ra.fuse_perm = fuse_perm ? 1 : 0;
   ra.tiles_done = L->tiles_done;
   ra.perm = pa;
+  // prefill-sized batches: logits by a tiled GEMM, then top-k and the
+  // permutation as their own kernels (the register-decode kernels of NVFP4
+  // EXACT layers need the router's f16 copy of x, so they keep the router)
+  const bool big_batch = T >= kDenseTcMinTokens && (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
+  const bool router_gemm = big_batch && (tc || a4);
   StageTimer t0(L, 0, s);
-  launch_router(ra, s);
+  if (router_gemm) {
+    const int sp = router_gemm_splits(T, H, E, kRouterPartFloats);
+    launch_router_gemm(ra.x, L->router_w, L->router_b, T, H, E, L->logits, L->router_parts, sp, s);
+    CUDA_TRY(cudaGetLastError());
+    launch_topk(L->logits, L->router_parts, sp, L->router_b, T, E, k, L->ids, L->gates, s);
+    t0.launched(1);
+  } else {
+    launch_router(ra, s);
+  }
   CUDA_TRY(cudaGetLastError());
   t0.launched(1);
   t0.end();
-  if (!fuse_perm) {
+  if (!fuse_perm || router_gemm) {
     StageTimer t1(L, 1, s);
     launch_permute(pa, s);
     CUDA_TRY(cudaGetLastError());
@@ -1010,7 +1027,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   }
 
   // always-resident shared expert (runs while the host builds the miss list)
-  const bool dense_tc = Is && T >= kDenseTcMinTokens && (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
+  const bool dense_tc = Is && big_batch;
   if (dense_tc) {
     StageTimer t2(L, 2, s);
     DenseTcArgs d{};

@@ -110,6 +110,16 @@ void launch_router(const RouterArgs &a, cudaStream_t s);
 
 void launch_permute(const PermArgs &a, cudaStream_t s);
 
+// Prefill-sized batches: router logits by a register-tiled fp32 GEMM
+// (x 16-byte aligned, H a multiple of 32), then top-k from the logits.
+// splits > 1: partial logits of K ranges into parts [splits, T, E], assembled
+// (in split order, + bias) by the top-k kernel.
+int router_gemm_splits(int T, int H, int E, size_t part_floats);
+void launch_router_gemm(const uint16_t *x, const float *w, const float *bias, int T, int H, int E, float *logits,
+                        float *parts, int splits, cudaStream_t s);
+void launch_topk(float *logits, const float *parts, int splits, const float *bias, int T, int E, int k, int *ids,
+                 float *gates, cudaStream_t s);
+
 // ------------------------------------------------------------------ experts
 enum WeightFmt { WF_MX = 0, WF_NV = 1, WF_BF16 = 2 };
 enum ExpertMode { MODE_GATEUP = 0, MODE_DOWN = 1 };

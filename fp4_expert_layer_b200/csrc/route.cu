@@ -213,6 +213,171 @@ __global__ void combine_kernel(const CombineArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Router logits for prefill-sized batches: a register-tiled fp32 GEMM on the
+// CUDA cores.  CTA tile 128 tokens x 64 experts, K in chunks of 32 staged in
+// shared memory (x converted from bf16, both operands transposed to [k][.]),
+// each thread 8 tokens x 4 experts.  Each chunk's 32 products are summed into
+// a chunk partial that is then added to the running sum (two-level summation:
+// the fp32 rounding of H = 4096 sequential additions would otherwise approach
+// the 1e-5 the logits are held to).  With few tiles (small T or E) the K range
+// is split over gridDim.z CTAs that write partial logits to a workspace; the
+// top-k kernel adds the parts in split order (deterministic, no atomics).
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kRgT = 128, kRgE = 64, kRgK = 32;
+}
+
+__global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__restrict__ x, const float *__restrict__ w,
+                                                          const float *__restrict__ bias, int T, int H, int E,
+                                                          float *__restrict__ logits, float *__restrict__ parts) {
+  __shared__ __align__(16) float xs[2][kRgK][kRgT];
+  __shared__ __align__(16) float ws[2][kRgK][kRgE];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;               // experts 4*tx.., tokens 8*ty..
+  const int t0 = blockIdx.x * kRgT, e0 = blockIdx.y * kRgE;
+  const int nsplit = gridDim.z;
+  const int ck0 = (int)((long)(H / kRgK) * blockIdx.z / nsplit);
+  const int ck1 = (int)((long)(H / kRgK) * (blockIdx.z + 1) / nsplit);
+  const int nck = ck1 - ck0;
+  // loader roles: x: token tid/2, 16 elements from (tid%2)*16; w: expert tid/4, 8 from (tid%4)*8
+  const int lt = tid >> 1, lk = (tid & 1) * 16;
+  const int le = tid >> 2, lkw = (tid & 3) * 8;
+  const bool xok = t0 + lt < T, wok = e0 + le < E;
+  const uint16_t *xrow = x + (size_t)(t0 + lt) * H + lk;
+  const float *wrow = w + (size_t)(e0 + le) * H + lkw;
+  uint4 xr0, xr1;
+  float4 wr0, wr1;
+  auto fetch = [&](int c) {
+    const int k0 = (ck0 + c) * kRgK;
+    if (xok) {
+      xr0 = __ldg(reinterpret_cast<const uint4 *>(xrow + k0));
+      xr1 = __ldg(reinterpret_cast<const uint4 *>(xrow + k0 + 8));
+    } else {
+      xr0 = xr1 = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (wok) {
+      wr0 = __ldg(reinterpret_cast<const float4 *>(wrow + k0));
+      wr1 = __ldg(reinterpret_cast<const float4 *>(wrow + k0 + 4));
+    } else {
+      wr0 = wr1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto stash = [&](int b) {
+    const uint32_t xv[8] = {xr0.x, xr0.y, xr0.z, xr0.w, xr1.x, xr1.y, xr1.z, xr1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      xs[b][lk + 2 * i][lt] = __uint_as_float(xv[i] << 16);
+      xs[b][lk + 2 * i + 1][lt] = __uint_as_float(xv[i] & 0xFFFF0000u);
+    }
+    const float wv[8] = {wr0.x, wr0.y, wr0.z, wr0.w, wr1.x, wr1.y, wr1.z, wr1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ws[b][lkw + i][le] = wv[i];
+  };
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  for (int c = 0; c < nck; ++c) {
+    const int b = c & 1;
+    if (c + 1 < nck) fetch(c + 1);
+    float part[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.0f;
+#pragma unroll 8
+    for (int k = 0; k < kRgK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&xs[b][k][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&xs[b][k][ty * 8 + 4]);
+      const float4 bw = *reinterpret_cast<const float4 *>(&ws[b][k][tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
+    if (c + 1 < nck) stash(b ^ 1);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + ty * 8 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e >= E) continue;
+      if (nsplit == 1) logits[(size_t)t * E + e] = acc[i][j] + (bias ? bias[e] : 0.0f);
+      else parts[((size_t)blockIdx.z * T + t) * E + e] = acc[i][j];
+    }
+  }
+}
+
+int router_gemm_splits(int T, int H, int E, size_t part_floats) {
+  const int tiles = ((T + kRgT - 1) / kRgT) * ((E + kRgE - 1) / kRgE);
+  int sp = 1;
+  while (sp < 8 && tiles * sp < 2 * 148 && (H / kRgK) / (sp * 2) >= 4 &&
+         (size_t)(sp * 2) * T * E <= part_floats)
+    sp *= 2;
+  return sp;
+}
+
+void launch_router_gemm(const uint16_t *x, const float *w, const float *bias, int T, int H, int E, float *logits,
+                        float *parts, int splits, cudaStream_t s) {
+  dim3 grid((T + kRgT - 1) / kRgT, (E + kRgE - 1) / kRgE, splits);
+  router_gemm_kernel<<<grid, 256, 0, s>>>(x, w, bias, T, H, E, logits, parts);
+}
+
+// Top-k of tokens whose logits are in memory: warp per token.
+// With splits > 1 the logits are first assembled from the K parts (in split
+// order, plus the bias) and written out.
+template <int KPER>
+__global__ void __launch_bounds__(256) topk_kernel(float *logits, const float *parts, int splits,
+                                                   const float *bias, int T, int E, int k, int *ids,
+                                                   float *gates) {
+  wait_prior_grid();
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= T) return;
+  float lv[KPER];
+  float *lrow = logits + (size_t)t * E;
+#pragma unroll
+  for (int i = 0; i < KPER; ++i) {
+    const int ee = lane + 32 * i;
+    if (ee >= E) {
+      lv[i] = -INFINITY;
+    } else if (splits > 1) {
+      float v = __ldcg(parts + (size_t)t * E + ee);
+      for (int sp = 1; sp < splits; ++sp) v += __ldcg(parts + ((size_t)sp * T + t) * E + ee);
+      v += bias ? bias[ee] : 0.0f;
+      lrow[ee] = v;
+      lv[i] = v;
+    } else {
+      lv[i] = __ldcg(lrow + ee);
+    }
+  }
+  topk_warp<KPER>(lv, E, k, ids + (size_t)t * k, gates + (size_t)t * k, nullptr);
+}
+
+void launch_topk(float *logits, const float *parts, int splits, const float *bias, int T, int E, int k, int *ids,
+                 float *gates, cudaStream_t s) {
+  const int blocks = (T + 7) / 8;
+  if (E <= 64) launch_dependent(topk_kernel<2>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
+  else if (E <= 128) launch_dependent(topk_kernel<4>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
+  else if (E <= 256) launch_dependent(topk_kernel<8>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
+  else if (E <= 512) launch_dependent(topk_kernel<16>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
+  else launch_dependent(topk_kernel<32>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
+}
+
 void launch_combine(const CombineArgs &a, cudaStream_t s) {
   const size_t n = (size_t)a.T * (a.H / 4);
   int blocks = (int)((n + 255) / 256);
