@@ -223,8 +223,8 @@ static Sizes sizes_of(const moe_config_t *c) {
   s.max_tiles = s.P / 8 + act + 1;
   s.a4_rows = s.P + 128 * act + 128;     // padded to 128 rows per expert, + one tile of slack
   // tensor-core EXACT path: tiles of 8 tokens only while P <= 12 * active experts
-  // (then at most 2.5 x act tiles), else tiles of 64 tokens
-  s.tc_tiles = std::max(s.P / 64 + act, (5 * act) / 2 + 1) + 2;
+  // (then at most 2.5 x act tiles), else tiles of 56 tokens
+  s.tc_tiles = std::max(s.P / 56 + act, (5 * act) / 2 + 1) + 2;
   return s;
 }
 
@@ -857,6 +857,7 @@ static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int 
   a.n_rowblocks = c.inter / 128;
   a.bsf = L->txsf;
   a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
+  a.early = locs == L->loc_resident ? 1 : 0;
   StageTimer t3(L, 3, s);
   launch_expert_tc(MODE_GATEUP, nbox, a, grid_tiles, s);
   CUDA_TRY(cudaGetLastError());
@@ -868,6 +869,10 @@ static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int 
   a.n_rowblocks = c.hidden / 256;
   a.bsf = L->thsf;
   a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
+  // the down pass starts its weight stream before the gate/up pass ends only
+  // with decode-sized tiles (there the gate/up CTAs end at different times);
+  // with prefill tiles this measured several times slower
+  a.early = (a.early && nbox <= 16) ? 1 : 0;
   StageTimer t4(L, 4, s);
   launch_expert_tc(MODE_DOWN, nbox, a, grid_tiles, s);
   CUDA_TRY(cudaGetLastError());
@@ -960,8 +965,9 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   const bool a4 = L->a4;
   const bool tc = L->tc;
   // tensor-core EXACT: 8-token tiles (16 piece rows, 6 stages in flight) while
-  // the batch is decode-sized, else 64-token tiles (128 piece rows)
-  const int nbox = (tc && P <= 12 * act_est) ? 16 : 128;
+  // the batch is decode-sized, else 56-token tiles (112 piece rows, two
+  // accumulator buffers so that the epilogue overlaps the next item's MMAs)
+  const int nbox = (tc && P <= 12 * act_est) ? 16 : 112;
   const int ts = a4 ? 128 : (tc ? nbox / 2 : 8 * nt);
   const int grid_tiles = P / ts + act_est + 1;
 

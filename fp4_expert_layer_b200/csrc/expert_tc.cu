@@ -24,7 +24,8 @@
 // Kernels:
 //  * tc_quant_x_kernel: gathers each tile's token rows of x (expert-sorted
 //    order) and writes the two E4M3 pieces and their scale-factor blocks;
-//  * expert_tc_kernel<GATEUP|DOWN, NBOX>: one CTA per (tile, 128 weight rows);
+//  * expert_tc_kernel<GATEUP|DOWN, NBOX>: persistent, work items (tile, 256
+//    weight rows), NBOX piece rows per tile;
 //    a producer warp streams 128x128 weight tiles (TMA unpacks the E2M1 codes
 //    to one byte per element), the matching 128-element slab of the tile's
 //    activation pieces and both scale-factor blocks into a ring of stages;
@@ -62,6 +63,11 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// tile descriptor read from L2 (written by another kernel)
+__device__ __forceinline__ TileInfo load_tile(const TileInfo *p) {
+  const int4 v = __ldcg(reinterpret_cast<const int4 *>(p));
+  return TileInfo{v.x, v.y, v.z, v.w};
+}
 
 
 }  // namespace
@@ -72,6 +78,7 @@ __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) tc_quant_x_kernel(const TcQuantArgs q) {
   wait_prior_grid();
+  if (threadIdx.x == 0) trigger_dependents();          // the expert pass may start its weight stream
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int tile = gw / q.tile_tokens, j = gw % q.tile_tokens;
   if (tile >= q.max_tiles || tile >= *q.n_tiles) return;
@@ -88,9 +95,12 @@ void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s) {
 // Expert pass on the tensor core, persistent.  A work item is (tile, 256
 // weight rows): gate/up = 128 gate rows + the same 128 up rows (one 4-D TMA
 // box), down = 256 output rows (one 3-D box); each half has its own
-// accumulator.  Items are taken round-robin by the CTAs; the stage ring runs
-// across items, and the accumulators are double-buffered (NBOX = 32) so the
-// epilogue of one item overlaps the main loop of the next.
+// accumulator.  Items are taken round-robin by the CTAs (concurrent CTAs then
+// work on neighbouring items: tiles of one expert share its weights in L2);
+// the stage ring runs across items, and the accumulators are double-buffered
+// (8-token tiles with six stages, 56-token tiles with four: 2 x 2 x 112
+// accumulator columns plus 12 scale columns per stage fill the 512 TMEM
+// columns) so the epilogue of one item overlaps the main loop of the next.
 // ---------------------------------------------------------------------------
 namespace {
 template <int NBOX>
@@ -102,7 +112,8 @@ struct TcGeom {
   static constexpr int B_BYTES = NBOX * 128;         // NBOX piece rows x 128 E4M3
   static constexpr int SF_OFF = B_OFF + B_BYTES;     // SFA half 0, SFA half 1, SFB: 512 B each
   static constexpr int STAGE = ((SF_OFF + 3 * 512) + 1023) / 1024 * 1024;
-  static constexpr int NBUF = NBOX <= 32 ? 2 : 1;    // accumulator buffers
+  // accumulator buffers: two whenever they fit in TMEM beside the scale columns
+  static constexpr int NBUF = (2 * 2 * NBOX + 12 * STAGES <= 512) ? 2 : 1;
   static constexpr int SF_COL0 = NBUF * 2 * NBOX;    // TMEM: accumulators first
   static constexpr int COLS_NEEDED = SF_COL0 + 12 * STAGES;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 128 ? 128 : (COLS_NEEDED <= 256 ? 256 : 512);
@@ -156,25 +167,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     tmem_alloc(smem_u32(&tmem_base_s), Geo::TMEM_COLS);
     tmem_relinquish();
   }
-  // everything above overlaps the previous kernel; the tile list is its output
-  wait_prior_grid();
-  const int n_items = *a.n_tiles * ipt;
+  // Everything above overlaps the previous kernel.  With `early`, the tile
+  // list and expert locations (written by the routing step, which finished
+  // before the previous kernel let this one launch) are read now and the
+  // producer streams weights at once; every other role waits for the previous
+  // kernel below, before it reads activations.
+  if (!a.early) wait_prior_grid();
+  const int n_items = __ldcg(a.n_tiles) * ipt;
   if (warp == 0) {
     for (int j = lane; j < kTcMeta; j += 32) {
       const int item = blockIdx.x + j * gridDim.x;
       if (item >= n_items) break;
-      const TileInfo ti = a.tiles[item / ipt];
+      const TileInfo ti = load_tile(a.tiles + item / ipt);
       meta_ti[j] = ti;
-      meta_loc[j] = a.loc[ti.expert];
+      meta_loc[j] = __ldcg(a.loc + ti.expert);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (a.early && warp != 0) wait_prior_grid();
+  // the down pass (persistent, one CTA per SM: it lands on SMs as this grid's
+  // CTAs exit) may start its own weight stream now; after the down pass the
+  // combine kernel is launched as usual, when this grid exits (its many
+  // waiting blocks would share the SMs with this pass)
+  if (MODE == MODE_GATEUP && threadIdx.x == 64) trigger_dependents();   // after this thread's wait
   const uint32_t tmem = tmem_base_s;
   // work item j of this CTA (item = blockIdx.x + j * gridDim.x)
-  auto item_tile = [&](int j, int item) -> TileInfo { return j < kTcMeta ? meta_ti[j] : a.tiles[item / ipt]; };
-  auto item_loc = [&](int j, const TileInfo &ti) -> int { return j < kTcMeta ? meta_loc[j] : a.loc[ti.expert]; };
+  auto item_tile = [&](int j, int item) -> TileInfo { return j < kTcMeta ? meta_ti[j] : load_tile(a.tiles + item / ipt); };
+  auto item_loc = [&](int j, const TileInfo &ti) -> int { return j < kTcMeta ? meta_loc[j] : __ldcg(a.loc + ti.expert); };
 
   if (warp == 0) {
     // ---------------- producer
@@ -434,8 +455,8 @@ void launch_expert_tc(int mode, int nbox, const TcArgs &a, int grid_tiles, cudaS
     if (mode == MODE_GATEUP) launch_tc_one<MODE_GATEUP, 32>(a, s);
     else launch_tc_one<MODE_DOWN, 32>(a, s);
   } else {
-    if (mode == MODE_GATEUP) launch_tc_one<MODE_GATEUP, 128>(a, s);
-    else launch_tc_one<MODE_DOWN, 128>(a, s);
+    if (mode == MODE_GATEUP) launch_tc_one<MODE_GATEUP, 112>(a, s);
+    else launch_tc_one<MODE_DOWN, 112>(a, s);
   }
 }
 

@@ -11,6 +11,12 @@ namespace moe {
 // has completed and its memory is visible (a no-op for a normal launch).
 __device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Let the next kernel on the stream (launched programmatically) be scheduled
+// now rather than when this CTA exits.  Called after this CTA's own
+// wait_prior_grid, so a kernel that starts early can rely on every kernel
+// before this one having finished and flushed its results.
+__device__ __forceinline__ void trigger_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Launch with programmatic stream serialisation: the kernel may be scheduled
 // before its predecessor on the stream has finished; it waits with
 // griddepcontrol.wait before reading the predecessor's results.

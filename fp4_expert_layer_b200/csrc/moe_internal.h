@@ -68,7 +68,7 @@ __host__ __device__ inline int loc_staging(int i) { return -2 - i; }
 
 // One token tile of one expert: rows [prow0, prow0 + nrows) of the padded,
 // expert-sorted activation order; each expert's rows start on a multiple of 8.
-struct TileInfo {
+struct alignas(16) TileInfo {
   int expert;
   int prow0;
   int nrows;
@@ -323,8 +323,13 @@ struct TcArgs {
   float *o_out;
   int *err;
   int grid;                  // persistent CTAs
+  // 1: the tile list and `loc` were written two or more kernels back on the
+  // stream, so the weight stream may start before this kernel waits for its
+  // predecessor (the resident path; not the staged waves, whose location
+  // table is written by the kernel right before)
+  int early;
 };
-// nbox: activation rows per tile (2 x tile tokens): 32 or 128.  The kernel is
+// nbox: activation rows per tile (2 x tile tokens): 16 or 112.  The kernel is
 // persistent: `a.grid` CTAs walk the work items (tile, 256 weight rows)
 // round-robin.
 void launch_expert_tc(int mode, int nbox, const TcArgs &a, int grid_tiles, cudaStream_t s);

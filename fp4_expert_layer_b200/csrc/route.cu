@@ -36,6 +36,15 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
   const int t0 = blockIdx.x * kRouterTT;
   const int nt = min(kRouterTT, a.T - t0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.y * kRouterEB + warp;
+  const float *w = a.w + (size_t)min(e, E - 1) * H;
+  // the first 8 weight vectors of this lane are in flight while x is staged
+  float4 wv[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int h = lane * 4 + u * 128;
+    wv[u] = h < H ? __ldg(reinterpret_cast<const float4 *>(w + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 
   // x tile -> smem (fp32)
   for (int i = threadIdx.x; i < nt * H / 2; i += blockDim.x) {
@@ -47,19 +56,18 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
   __syncthreads();
 
   // logits: warp w -> expert e
-  const int e = blockIdx.y * kRouterEB + warp;
   if (e < E) {
     float acc[kRouterTT];
 #pragma unroll
     for (int t = 0; t < kRouterTT; ++t) acc[t] = 0.0f;
-    const float *w = a.w + (size_t)e * H;
     // 8 independent 16-byte loads in flight per lane before any use
     for (int h0 = lane * 4; h0 < H; h0 += 128 * 8) {
-      float4 wv[8];
+      if (h0 != lane * 4) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int h = h0 + u * 128;
-        wv[u] = h < H ? __ldg(reinterpret_cast<const float4 *>(w + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < 8; ++u) {
+          const int h = h0 + u * 128;
+          wv[u] = h < H ? __ldg(reinterpret_cast<const float4 *>(w + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
