@@ -55,6 +55,7 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
     return p.parse_args()
 
 
@@ -338,10 +339,37 @@ def main():
         e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e0, e1))
         e2e = [e2e_ms, Ke]
 
-    vals = torch.tensor([dev_ms, e2e[0] if e2e else 0.0], dtype=torch.float64, device=dev)
+    # CUDA-graph replay of the same forward (all-resident layers): the same
+    # launch chain without the CPU cost of each launch; L2 flushed as above
+    graph_ms = 0.0
+    if S == wl.n_experts and not args.no_graph:
+        gs = torch.cuda.Stream(dev)
+        yg = torch.empty_like(y)
+        gph = layer.capture_graph(x.data_ptr(), T, yg.data_ptr(), gs.cuda_stream)
+        with torch.cuda.stream(gs):
+            for _ in range(args.warmup):
+                flush.zero_()
+                gph.launch(gs.cuda_stream)
+        gs.synchronize()
+        g0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        g1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(gs):
+            for i in range(K):
+                flush.zero_()
+                g0[i].record(gs)
+                gph.launch(gs.cuda_stream)
+                g1[i].record(gs)
+        gs.synchronize()
+        barrier()
+        graph_ms = sum(a.elapsed_time(b) for a, b in zip(g0, g1))
+        gph.close()
+
+    vals = torch.tensor([dev_ms, e2e[0] if e2e else 0.0, graph_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    dev_ms_max, e2e_ms_max = float(vals[0]), float(vals[1])
+    dev_ms_max, e2e_ms_max, graph_ms_max = float(vals[0]), float(vals[1]), float(vals[2])
 
     if rank == 0:
         hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
@@ -399,6 +427,10 @@ def main():
         if e2e:
             line["e2e"] = {"value": world * T * e2e[1] / (e2e_ms_max / 1e3), "unit": "tokens/s",
                            "h2d_bytes_per_step": T * wl.hidden * 2, "d2h_bytes_per_step": T * wl.hidden * 4}
+        if graph_ms_max > 0:
+            line["graph"] = {"value": world * T * K / (graph_ms_max / 1e3), "unit": "tokens/s",
+                             "ms_per_step": graph_ms_max / K,
+                             "how": "moe_graph_capture of this forward, replayed K times (L2 flushed before each)"}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(lw, x_bits, args.cpu_seconds, args.numerics)
         print(json.dumps(line), flush=True)

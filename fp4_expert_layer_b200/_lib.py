@@ -23,7 +23,8 @@ NUMERICS = {"exact": 0, "a4": 1}
 
 EXPORTED = ["moe_layer_plan", "moe_admit", "moe_layer_create", "moe_set_slot_table", "moe_forward",
             "moe_forward_host", "moe_get_stats", "moe_destroy", "moe_last_error", "moe_debug_inject",
-            "moe_profile_enable", "moe_profile_read", "moe_route_topk_noalloc", "moe_debug_read"]
+            "moe_profile_enable", "moe_profile_read", "moe_route_topk_noalloc", "moe_debug_read",
+            "moe_graph_capture", "moe_graph_launch", "moe_graph_destroy"]
 
 
 class MoEError(RuntimeError):
@@ -90,6 +91,10 @@ def lib():
         L.moe_forward.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.POINTER(Routing)]
         L.moe_forward_host.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]
         L.moe_get_stats.argtypes = [C.c_void_p, C.POINTER(Stats)]
+        L.moe_graph_capture.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p,
+                                        C.POINTER(C.c_void_p)]
+        L.moe_graph_launch.argtypes = [C.c_void_p, C.c_void_p]
+        L.moe_graph_destroy.argtypes = [C.c_void_p]
         L.moe_destroy.argtypes = [C.c_void_p]
         L.moe_destroy.restype = None
         L.moe_last_error.restype = C.c_char_p
@@ -185,6 +190,21 @@ def _stream_ptr(stream):
     return getattr(stream, "cuda_stream", stream)
 
 
+class Graph:
+    """A captured forward (moe_graph_t): launch() replays it; close() before the layer's."""
+
+    def __init__(self, handle):
+        self.handle = handle
+
+    def launch(self, stream_ptr: int):
+        check(lib().moe_graph_launch(self.handle, stream_ptr))
+
+    def close(self):
+        if self.handle:
+            lib().moe_graph_destroy(self.handle)
+            self.handle = None
+
+
 class MoELayer:
     """One layer on one GPU.  ``forward`` takes and returns torch CUDA tensors."""
 
@@ -244,6 +264,12 @@ class MoELayer:
 
     def forward_host_ptr(self, x_ptr: int, T: int, y_ptr: int, stream_ptr: int):
         check(lib().moe_forward_host(self.handle, x_ptr, T, y_ptr, stream_ptr))
+
+    def capture_graph(self, x_ptr: int, T: int, y_ptr: int, stream_ptr: int) -> "Graph":
+        """CUDA graph of one all-resident forward for these fixed buffers."""
+        h = C.c_void_p()
+        check(lib().moe_graph_capture(self.handle, x_ptr, T, y_ptr, stream_ptr, C.byref(h)))
+        return Graph(h.value)
 
     def stats(self) -> dict:
         s = Stats()

@@ -128,6 +128,7 @@ struct moe_layer {
   int *h_loc = nullptr;              // pinned [E]
   std::vector<int> slot_of;
   int n_resident = 0;
+  uint64_t table_version = 0;        // bumped by every moe_set_slot_table
   size_t max_prows = 0, max_tiles = 0;
   moe_stats_t st{};
   int inject = 0;
@@ -771,6 +772,7 @@ moe_status_t moe_set_slot_table(moe_layer_t L, const int32_t *table, void *strea
   CUDA_TRY(cudaStreamSynchronize(st));
   for (int e = 0; e < E; ++e) L->slot_of[e] = table[e];
   L->n_resident = n;
+  L->table_version += 1;
   return MOE_OK;
 }
 
@@ -1226,6 +1228,97 @@ moe_status_t moe_forward_host(moe_layer_t L, const uint16_t *x_host, int32_t T, 
   ST_TRY(moe_forward(L, L->xin, T, L->yout, stream, nullptr));
   CUDA_TRY(cudaMemcpyAsync(y_host, L->yout, (size_t)T * H * 4, cudaMemcpyDeviceToHost, s));
   CUDA_TRY(cudaStreamSynchronize(s));
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-graph capture of one all-resident forward (fixed x, T, y).  The
+// resident forward only enqueues kernels (no host synchronisation), so it can
+// be captured as it is; a replay runs the same launch chain without the
+// per-kernel CPU launch cost.
+// ---------------------------------------------------------------------------
+struct moe_graph {
+  moe_layer *L = nullptr;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  uint64_t table_version = 0;
+  uint64_t launches = 0;             // library kernels per replay
+};
+
+moe_status_t moe_graph_capture(moe_layer_t L, const void *x, int32_t T, float *y, void *stream,
+                               moe_graph_t *out) {
+  if (!L || !out) return fail(MOE_ERR_INVALID_ARG, "layer or out is NULL");
+  *out = nullptr;
+  if (T < 1 || T > L->cfg.max_tokens) return fail(MOE_ERR_INVALID_ARG, "T out of range [1, max_tokens]");
+  if (!x || !y) return fail(MOE_ERR_INVALID_ARG, "x or y is NULL");
+  if (!stream) return fail(MOE_ERR_INVALID_ARG, "graph capture needs a created (non-default) stream");
+  if (L->n_resident != L->cfg.n_experts)
+    return fail(MOE_ERR_INVALID_ARG, "graph capture needs every expert resident (a staged forward reads the "
+                                     "routing counts on the host)");
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  cudaStream_t s = (cudaStream_t)stream;
+  const bool prof = L->prof;
+  const moe_stats_t st0 = L->st;
+  L->prof = false;
+  CUDA_TRY(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
+  const moe_status_t r = moe_forward(L, x, T, y, stream, nullptr);
+  cudaGraph_t g = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(s, &g);
+  L->prof = prof;
+  const uint64_t launches = L->st.launches - st0.launches;
+  L->st = st0;                                   // nothing ran yet
+  if (r != MOE_OK) {
+    if (g) cudaGraphDestroy(g);
+    (void)cudaGetLastError();
+    return r;
+  }
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, std::string("graph capture failed: ") + cudaGetErrorString(e));
+  cudaGraphExec_t ex = nullptr;
+  const cudaError_t ei = cudaGraphInstantiate(&ex, g, 0);
+  if (ei != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return fail(MOE_ERR_CUDA, std::string("graph instantiation failed: ") + cudaGetErrorString(ei));
+  }
+  moe_graph *G = new (std::nothrow) moe_graph;
+  if (!G) {
+    cudaGraphExecDestroy(ex);
+    cudaGraphDestroy(g);
+    return fail(MOE_ERR_OOM, "graph handle allocation failed");
+  }
+  G->L = L;
+  G->graph = g;
+  G->exec = ex;
+  G->table_version = L->table_version;
+  G->launches = launches;
+  *out = G;
+  return MOE_OK;
+}
+
+moe_status_t moe_graph_launch(moe_graph_t G, void *stream) {
+  if (!G || !G->L) return fail(MOE_ERR_INVALID_ARG, "graph is NULL");
+  moe_layer *L = G->L;
+  if (L->table_version != G->table_version)
+    return fail(MOE_ERR_INVALID_ARG, "the slot table changed since the graph was captured");
+  if (*(volatile int *)L->h_err != 0) {
+    char buf[128];
+    snprintf(buf, sizeof buf, "a device-side wait of an earlier forward gave up (code %d); outputs of that "
+             "forward are invalid", *(volatile int *)L->h_err);
+    *(volatile int *)L->h_err = 0;
+    return fail(MOE_ERR_CUDA, buf);
+  }
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  CUDA_TRY(cudaGraphLaunch(G->exec, (cudaStream_t)stream));
+  L->st.forwards += 1;
+  L->st.launches += G->launches;
+  return MOE_OK;
+}
+
+moe_status_t moe_graph_destroy(moe_graph_t G) {
+  if (!G) return MOE_OK;
+  if (G->L) cudaSetDevice(G->L->cfg.device);
+  if (G->exec) cudaGraphExecDestroy(G->exec);
+  if (G->graph) cudaGraphDestroy(G->graph);
+  delete G;
   return MOE_OK;
 }
 

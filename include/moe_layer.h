@@ -192,6 +192,22 @@ moe_status_t moe_forward(moe_layer_t layer, const void *x, int32_t T, float *y, 
 moe_status_t moe_forward_host(moe_layer_t layer, const uint16_t *x_host, int32_t T,
                               float *y_host, void *stream);
 
+/* CUDA graph of one forward (launch overhead of a decode step).
+ * moe_graph_capture records the forward of T tokens from x (device bf16
+ * [T, H]) into y (device fp32 [T, H]) on `stream` (a created stream, not the
+ * legacy default stream) into a CUDA graph without running it; each
+ * moe_graph_launch replays it on `stream`, reading the x and writing the y
+ * given at capture.  Requires every expert resident (the staged path waits for
+ * the routing counts on the host): otherwise MOE_ERR_INVALID_ARG.  A launch
+ * after moe_set_slot_table has changed the table returns MOE_ERR_INVALID_ARG.
+ * The graph belongs to the caller: moe_graph_destroy before moe_destroy of its
+ * layer.  Replays count in moe_stats_t (forwards, launches). */
+typedef struct moe_graph *moe_graph_t;
+moe_status_t moe_graph_capture(moe_layer_t layer, const void *x, int32_t T, float *y, void *stream,
+                               moe_graph_t *out);
+moe_status_t moe_graph_launch(moe_graph_t graph, void *stream);
+moe_status_t moe_graph_destroy(moe_graph_t graph);
+
 moe_status_t moe_get_stats(moe_layer_t layer, moe_stats_t *out);
 
 /* Per-stage device timing (tracing).  While enabled, every forward records a
