@@ -121,6 +121,8 @@ struct moe_layer {
   size_t tc_rows = 0;
   TcMaps tcmaps{};
   uint8_t *txq = nullptr, *txsf = nullptr, *thq = nullptr, *thsf = nullptr;
+  int *tc_work = nullptr;            // [kWorkCtrs] item counters of the expert passes
+  int *tile_done = nullptr;          // [tc tiles] gate/up items finished per tile (decode hand-over)
   // host
   uint8_t *store = nullptr;          // pinned: E x blob bytes
   int *h_counts = nullptr;           // pinned [E]
@@ -247,7 +249,8 @@ static size_t tc_scratch_bytes(const moe_config_t *c) {
   if (!uses_tc(c)) return 0;
   const Sizes z = sizes_of(c);
   const size_t R = z.tc_tiles * kTcSlotRows, H = c->hidden, I = c->inter;
-  return align256(R * H) + align256(R * H / 32) + align256(R * I) + align256(R * I / 32);
+  return align256(R * H) + align256(R * H / 32) + align256(R * I) + align256(R * I / 32) +
+         align256(kWorkCtrs * sizeof(int)) + align256(z.tc_tiles * sizeof(int));
 }
 
 static size_t scratch_bytes(const moe_config_t *c) {
@@ -680,6 +683,10 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     C_CUDA(cudaMemsetAsync(L->txsf, 127, R * H / 32, s));
     C_CUDA(cudaMemsetAsync(L->thq, 0, R * I, s));
     C_CUDA(cudaMemsetAsync(L->thsf, 127, R * I / 32, s));
+    C_TRY(dalloc(L, &L->tc_work, kWorkCtrs * sizeof(int)));
+    C_CUDA(cudaMemsetAsync(L->tc_work, 0, kWorkCtrs * sizeof(int), s));
+    C_TRY(dalloc(L, &L->tile_done, z.tc_tiles * sizeof(int)));
+    C_CUDA(cudaMemsetAsync(L->tile_done, 0, z.tc_tiles * sizeof(int), s));
   }
   C_TRY(dalloc(L, &L->yout, T * H * 4));
 
@@ -858,8 +865,13 @@ static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int 
   a.rows = c.inter;
   a.n_rowblocks = c.inter / 128;
   a.bsf = L->txsf;
+  a.work_ctr = L->tc_work;
   a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
   a.early = locs == L->loc_resident ? 1 : 0;
+  // decode tiles, all resident: the down pass takes each tile's h as soon as
+  // the gate/up items of that tile are done (counters zeroed by the routing step)
+  a.tile_done = (a.early && nbox <= 16) ? L->tile_done : nullptr;
+  a.tile_target = c.inter / 128;
   StageTimer t3(L, 3, s);
   launch_expert_tc(MODE_GATEUP, nbox, a, grid_tiles, s);
   CUDA_TRY(cudaGetLastError());
@@ -870,6 +882,7 @@ static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int 
   a.rows = c.hidden;
   a.n_rowblocks = c.hidden / 256;
   a.bsf = L->thsf;
+  a.work_ctr = L->tc_work + 1;
   a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
   // the down pass starts its weight stream before the gate/up pass ends only
   // with decode-sized tiles (there the gate/up CTAs end at different times);
@@ -987,6 +1000,8 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   pa.prow_pair = L->prow_pair; pa.active = L->active;
   pa.pad = a4 ? 128 : 8;
   pa.n_prows = a4 ? L->n_prows : nullptr;
+  pa.work_ctr = tc ? L->tc_work : nullptr;
+  pa.tile_done = tc ? L->tile_done : nullptr;
   // decode-sized batches: the router's last CTA also runs the permutation
   const bool fuse_perm = P <= 2048;
   ra.fuse_perm = fuse_perm ? 1 : 0;
@@ -1159,6 +1174,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
         if (!one && w >= 2) CUDA_TRY(cudaStreamWaitEvent(L->side, L->ev_done[half], 0));
         LocUpdate u{};
         u.E = E;
+        u.work_ctr = tc ? L->tc_work : nullptr;
         u.keep_resident = (w == 0);
         const int b0 = w * wave_sz, b1 = std::min(misses_n, b0 + wave_sz);
         for (int i = b0; i < b1; ++i) {

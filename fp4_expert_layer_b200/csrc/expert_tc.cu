@@ -51,7 +51,8 @@ namespace {
 // LSU path), so that the per-SM TMA unit carries only the weight stream
 constexpr int kTcThreads = 256;
 constexpr int kTcLoaders = 64;
-constexpr int kTcMeta = 64;       // work items per CTA whose descriptors are cached in shared memory
+constexpr int kSched = 8;         // work items handed from the producer to the other roles in flight
+constexpr int kSchedReaders = 7;  // arrivals that free a hand-over slot: MMA lane, 2 loader warps, 4 epilogue warps
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -134,11 +135,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   __shared__ __align__(8) uint64_t accf_bar[NBUF];
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
   __shared__ uint32_t tmem_base_s;
-  // this CTA's first kTcMeta work items: tile descriptor and expert location,
-  // loaded once in parallel so that no role waits on dependent global loads
-  // at an item boundary
-  __shared__ TileInfo meta_ti[kTcMeta];
-  __shared__ int meta_loc[kTcMeta];
+  // Work items are taken from the pass's counter (atomicAdd, in index order)
+  // by the producer, which loads each item's tile descriptor and expert
+  // location and hands all three to the other roles through this ring (-1 =
+  // no more items).  A CTA that starts early or runs faster takes more items.
+  __shared__ __align__(8) uint64_t sched_full[kSched];
+  __shared__ __align__(8) uint64_t sched_empty[kSched];
+  __shared__ int sched_item[kSched];
+  __shared__ TileInfo sched_ti[kSched];
+  __shared__ int sched_loc[kSched];
   // down epilogue: pair index and gate of each token of the current item
   __shared__ int tok_pair[NBOX / 2];
   __shared__ float tok_gate[NBOX / 2];
@@ -161,6 +166,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       mbar_init(smem_u32(&accf_bar[b]), 1);
       mbar_init(smem_u32(&acce_bar[b]), 4);           // one arrival per epilogue warp
     }
+    for (int q = 0; q < kSched; ++q) {
+      mbar_init(smem_u32(&sched_full[q]), 1);
+      mbar_init(smem_u32(&sched_empty[q]), kSchedReaders);
+    }
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -168,59 +177,93 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     tmem_relinquish();
   }
   // Everything above overlaps the previous kernel.  With `early`, the tile
-  // list and expert locations (written by the routing step, which finished
-  // before the previous kernel let this one launch) are read now and the
-  // producer streams weights at once; every other role waits for the previous
-  // kernel below, before it reads activations.
+  // list, the expert locations and the item counter (written by the routing
+  // step, which finished before the previous kernel let this one launch) are
+  // read now and the producer streams weights at once; every other role waits
+  // for the previous kernel below, before it reads activations.
   if (!a.early) wait_prior_grid();
   const int n_items = __ldcg(a.n_tiles) * ipt;
-  if (warp == 0) {
-    for (int j = lane; j < kTcMeta; j += 32) {
-      const int item = blockIdx.x + j * gridDim.x;
-      if (item >= n_items) break;
-      const TileInfo ti = load_tile(a.tiles + item / ipt);
-      meta_ti[j] = ti;
-      meta_loc[j] = __ldcg(a.loc + ti.expert);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (a.early && warp != 0) wait_prior_grid();
+  // (a down pass with per-tile hand-over never waits for the whole gate/up
+  // grid: its loaders wait for each tile's count instead)
+  const bool per_tile = MODE == MODE_DOWN && a.tile_done != nullptr;
+  if (a.early && warp != 0 && !per_tile) wait_prior_grid();
   // the down pass (persistent, one CTA per SM: it lands on SMs as this grid's
   // CTAs exit) may start its own weight stream now; after the down pass the
   // combine kernel is launched as usual, when this grid exits (its many
   // waiting blocks would share the SMs with this pass)
   if (MODE == MODE_GATEUP && threadIdx.x == 64) trigger_dependents();   // after this thread's wait
   const uint32_t tmem = tmem_base_s;
-  // work item j of this CTA (item = blockIdx.x + j * gridDim.x)
-  auto item_tile = [&](int j, int item) -> TileInfo { return j < kTcMeta ? meta_ti[j] : load_tile(a.tiles + item / ipt); };
-  auto item_loc = [&](int j, const TileInfo &ti) -> int { return j < kTcMeta ? meta_loc[j] : __ldcg(a.loc + ti.expert); };
 
   if (warp == 0) {
     // ---------------- producer
     if (lane == 0) {
       int s = 0, issued = 0;
       uint32_t ph = 0;
+      int q = 0;
+      uint32_t qph = 0;
       bool failed = false;
-      for (int item = blockIdx.x, j = 0; item < n_items && !failed; item += gridDim.x, ++j) {
-        const int rb = item % ipt;
-        const TileInfo ti = item_tile(j, item);
-        const int loc = item_loc(j, ti);
-        if (loc == kLocAbsent) continue;
-        const bool in_slot = loc >= 0;
-        const int bidx = in_slot ? loc : (-2 - loc);
-        const int region = in_slot ? 0 : 1;
-        const CUtensorMap *wm = &a.maps.w[region][region_map];
-        for (int slab = 0; slab < nslab; ++slab) {
-          if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 32)) { failed = true; break; }
-          const uint32_t bar = smem_u32(&full_bar[s]);
-          const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
-          mbar_arrive_expect_tx(bar, (uint32_t)Geo::A_TX);
-          tma_load_4d(st, wm, bar, 0, 0, rb * nslab + slab, bidx);   // one contiguous 16 KB chunk
-          ++issued;
-          if (++s == S) { s = 0; ph ^= 1u; }
+      int item = atomicAdd(a.work_ctr, 1);
+      TileInfo ti{};
+      int loc = kLocAbsent;
+      if (item < n_items) {
+        ti = load_tile(a.tiles + item / ipt);
+        loc = __ldcg(a.loc + ti.expert);
+      }
+      for (int j = 0; !failed; ++j) {
+        // hand item j (or the end) to the other roles
+        if (j >= kSched && !mbar_wait(smem_u32(&sched_empty[q]), qph ^ 1u, a.err, 38)) { failed = true; break; }
+        const bool done = item >= n_items;
+        sched_item[q] = done ? -1 : item;
+        sched_ti[q] = ti;
+        sched_loc[q] = loc;
+        mbar_arrive(smem_u32(&sched_full[q]));               // release: the slot is written
+        if (++q == kSched) { q = 0; qph ^= 1u; }
+        if (done) break;
+        // the next item's index is fetched at this item's first slab and its
+        // descriptor loaded a few slabs later, both hidden behind the stream
+        int nxt = -1;
+        TileInfo nti{};
+        int nloc = kLocAbsent;
+        bool have_next = false;
+        if (loc != kLocAbsent) {
+          const int rb = item % ipt;
+          const bool in_slot = loc >= 0;
+          const int bidx = in_slot ? loc : (-2 - loc);
+          const int region = in_slot ? 0 : 1;
+          const CUtensorMap *wm = &a.maps.w[region][region_map];
+          const int slab_meta = min(2, nslab - 1);
+          for (int slab = 0; slab < nslab; ++slab) {
+            if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 32)) { failed = true; break; }
+            const uint32_t bar = smem_u32(&full_bar[s]);
+            const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+            mbar_arrive_expect_tx(bar, (uint32_t)Geo::A_TX);
+            tma_load_4d(st, wm, bar, 0, 0, rb * nslab + slab, bidx);   // one contiguous 16 KB chunk
+            ++issued;
+            if (++s == S) { s = 0; ph ^= 1u; }
+            if (slab == 0) nxt = atomicAdd(a.work_ctr, 1);
+            if (slab == slab_meta) {
+              if (nxt < n_items) {
+                nti = load_tile(a.tiles + nxt / ipt);
+                nloc = __ldcg(a.loc + nti.expert);
+              }
+              have_next = true;
+            }
+          }
         }
+        if (failed) break;
+        if (!have_next) {
+          if (nxt < 0) nxt = atomicAdd(a.work_ctr, 1);
+          if (nxt < n_items) {
+            nti = load_tile(a.tiles + nxt / ipt);
+            nloc = __ldcg(a.loc + nti.expert);
+          }
+        }
+        item = nxt;
+        ti = nti;
+        loc = nloc;
       }
       if (failed) {
         // let the copies already issued land before the CTA exits
@@ -237,10 +280,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     if (lane == 0) {
       int s = 0, n = 0;
       uint32_t ph = 0;
+      int q = 0;
+      uint32_t qph = 0;
       bool failed = false;
-      for (int item = blockIdx.x, j = 0; item < n_items && !failed; item += gridDim.x, ++j) {
-        const TileInfo ti = item_tile(j, item);
-        if (item_loc(j, ti) == kLocAbsent) continue;
+      while (!failed) {
+        if (!mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 39)) break;
+        const int item = sched_item[q];
+        const TileInfo ti = sched_ti[q];
+        const int loc = sched_loc[q];
+        mbar_arrive(smem_u32(&sched_empty[q]));
+        if (++q == kSched) { q = 0; qph ^= 1u; }
+        if (item < 0) break;
+        if (loc == kLocAbsent) continue;
         const int N = max(16, (2 * ti.nrows + 15) & ~15);    // piece rows rounded up to 16
         const int buf = n % NBUF;
         // the epilogue must have drained this accumulator buffer
@@ -286,12 +337,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     const int lt = threadIdx.x - 192;
     int s = 0, issued = 0;
     uint32_t ph = 0;
+    int q = 0;
+    uint32_t qph = 0;
     bool failed = false;
-    for (int item = blockIdx.x, j = 0; item < n_items && !failed; item += gridDim.x, ++j) {
-      const int tile = item / ipt, rb = item % ipt;
-      const TileInfo ti = item_tile(j, item);
-      const int loc = item_loc(j, ti);
+    while (!failed) {
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 40) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;                                       // warp-uniform
+      __syncwarp();
+      const int item = sched_item[q];
+      const TileInfo ti = sched_ti[q];
+      const int loc = sched_loc[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+      if (++q == kSched) { q = 0; qph ^= 1u; }
+      if (item < 0) break;
       if (loc == kLocAbsent) continue;
+      const int tile = item / ipt, rb = item % ipt;
       const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
       const int act_row0 = tile * kTcSlotRows;
       // scale blocks of the chunk's two halves (1 KB per chunk), and of the activation rows
@@ -299,6 +362,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       const uint8_t *sfb = a.bsf + sf_offset(nsf, act_row0, 0);
       const uint8_t *act = a.act + (size_t)act_row0 * K;
       const int nb = 8 * max(16, (2 * ti.nrows + 15) & ~15);   // 16-byte chunks of the piece rows read
+      if (per_tile) {
+        // this tile's h pieces are complete once every gate/up item of it is
+        int okt = 1;
+        if (lane == 0) okt = flag_wait(a.tile_done + tile, a.tile_target, a.err, 42) ? 1 : 0;
+        okt = __shfl_sync(0xffffffffu, okt, 0);
+        if (!okt) { failed = true; break; }                  // warp-uniform
+      }
       for (int slab = 0; slab < nslab; ++slab) {
         if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 35)) { failed = true; break; }
         const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
@@ -324,10 +394,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     const int quad = warp & 3;
     int n = 0;
     bool ok = true;
-    for (int item = blockIdx.x, j = 0; item < n_items && ok; item += gridDim.x, ++j) {
+    int q = 0;
+    uint32_t qph = 0;
+    while (ok) {
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 41) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      __syncwarp();
+      const int item = okw ? sched_item[q] : -1;
+      const TileInfo ti = sched_ti[q];
+      const int loc = sched_loc[q];
+      __syncwarp();
+      if (okw && lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+      if (++q == kSched) { q = 0; qph ^= 1u; }
+      // the four warps stop together (each takes every named barrier below)
+      if (!named_bar_and(1, 128, okw != 0 && item >= 0)) break;
+      if (loc == kLocAbsent) continue;
       const int tile = item / ipt, rb = item % ipt;
-      const TileInfo ti = item_tile(j, item);
-      if (item_loc(j, ti) == kLocAbsent) continue;
       const int ntok = ti.nrows;
       const int act_row0 = tile * kTcSlotRows;
       const int buf = n % NBUF;
@@ -403,6 +486,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&acce_bar[buf]));
+        if (a.tile_done) {
+          __threadfence();                                   // this thread's h pieces and scales are out
+          named_bar_sync(1, 128);
+          if (et == 0 && ok) atomicAdd(a.tile_done + tile, 1);
+        }
       } else {
         const int H = a.rows;
         for (int hh = 0; hh < 2; ++hh) {

@@ -467,6 +467,7 @@ void launch_expert_tma(int wf, int mode, int nt, const TmaExpertArgs &a, int gri
 // absent) and overwrite the listed experts.
 __global__ void loc_update_kernel(const LocUpdate u, const int *resident, int *out) {
   for (int e = threadIdx.x; e < u.E; e += blockDim.x) out[e] = u.keep_resident ? resident[e] : kLocAbsent;
+  if (u.work_ctr && (int)threadIdx.x < kWorkCtrs) u.work_ctr[threadIdx.x] = 0;
   __syncthreads();
   for (int i = threadIdx.x; i < u.n; i += blockDim.x) out[u.expert[i]] = u.loc[i];
 }

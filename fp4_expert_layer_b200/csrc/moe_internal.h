@@ -68,6 +68,11 @@ __host__ __device__ inline int loc_staging(int i) { return -2 - i; }
 
 // One token tile of one expert: rows [prow0, prow0 + nrows) of the padded,
 // expert-sorted activation order; each expert's rows start on a multiple of 8.
+// Item counters of the tensor-core expert passes ([0] gate/up, [1] down): the
+// CTAs take work items in index order by atomicAdd; the kernel that writes the
+// tile list (or the staged wave's location update) zeroes them.
+constexpr int kWorkCtrs = 2;
+
 struct alignas(16) TileInfo {
   int expert;
   int prow0;
@@ -90,6 +95,8 @@ struct PermArgs {
   int *active;           // [1] experts with >= 1 pair
   int pad;               // row padding granularity per expert (8 or 128)
   int *n_prows;          // [1] total padded rows (may be null)
+  int *work_ctr;         // [kWorkCtrs] zeroed here (may be null): item counters of the expert passes
+  int *tile_done;        // [tiles] zeroed here (may be null): gate/up items finished per tile
 };
 struct RouterArgs {
   const uint16_t *x;     // bf16 [T, H]
@@ -176,6 +183,7 @@ struct LocUpdate {
   int n;
   int keep_resident;
   int E;
+  int *work_ctr;         // [kWorkCtrs] zeroed for the wave's expert passes (may be null)
   int expert[kPtrListMax];
   int loc[kPtrListMax];
 };
@@ -321,6 +329,13 @@ struct TcArgs {
   const int *prow_pair;
   const float *gates;
   float *o_out;
+  int *work_ctr;             // item counter of this pass, zero at launch (set two or more kernels back)
+  // Per-tile hand-over from the gate/up pass to the down pass (decode, all
+  // resident; null otherwise): gate/up adds 1 per finished item of a tile, the
+  // down pass reads a tile's h once its count reaches tile_target (I / 128)
+  // instead of waiting for the whole gate/up grid
+  int *tile_done;
+  int tile_target;
   int *err;
   int grid;                  // persistent CTAs
   // 1: the tile list and `loc` were written two or more kernels back on the

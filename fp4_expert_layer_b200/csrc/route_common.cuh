@@ -84,6 +84,7 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   for (int i = tid; i < E; i += NTH) { cnt[i] = 0; cursor[i] = 0; }
+  if (a.work_ctr && tid < kWorkCtrs) a.work_ctr[tid] = 0;
   for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;
   __syncthreads();
   for (int p = tid; p < a.n_pairs; p += NTH) atomicAdd(&cnt[load_id<IDS_GLOBAL>(ids, p)], 1);
@@ -145,6 +146,8 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
     }
   }
   __syncthreads();
+  if (a.tile_done)
+    for (int t = tid; t < toff[E]; t += NTH) a.tile_done[t] = 0;
   for (int e = tid; e <= E; e += NTH) a.offsets[e] = off[e];
   for (int e = tid; e < E; e += NTH) {
     const int c = cnt[e];

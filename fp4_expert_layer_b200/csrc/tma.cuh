@@ -65,6 +65,30 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *er
   }
 }
 
+// Counters between kernels: the writer fences its data, then bumps the
+// counter; the reader acquires it before reading the data.
+__device__ __forceinline__ int flag_acquire(const int *f) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
+// Bounded wait until *f == v; false (and `code` in *err) past the limit or
+// once another wait has failed.
+__device__ __forceinline__ bool flag_wait(const int *f, int v, int *err, int code) {
+  if (flag_acquire(f) == v) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (flag_acquire(f) == v) return true;
+    if ((i & 63u) == 0) {
+      if (err && *(volatile int *)err != 0) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        if (err) atomicExch(err, code);
+        return false;
+      }
+    }
+  }
+}
+
 // 3-D tiled TMA load of one box into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint32_t bar, int c0, int c1,
                                             int c2) {
