@@ -919,28 +919,38 @@ static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles
   g.bsf = L->xsf;
   g.bG = L->xG;
   g.h_out = L->h32;
+  // MXFP4: the gate/up epilogue quantises h itself (its block scale is local
+  // to 32 columns of one token); NVFP4's per-row tensor scale needs the whole
+  // row first, so there h goes through fp32 and the quantiser
+  const bool fuse_hq = c.fmt == MOE_FMT_MXFP4;
+  g.hq_out = fuse_hq ? L->hq : nullptr;
+  g.hsf_out = fuse_hq ? L->hsf : nullptr;
   StageTimer t3(L, 3, s);
   launch_gemm_a4(L->wf, MODE_GATEUP, g, grid_tiles, s);
   CUDA_TRY(cudaGetLastError());
   t3.launched(1);
   t3.end();
-  StageTimer t8(L, 8, s);
-  QuantArgs q{};
-  q.max_rows = (int)L->a4_rows;
-  q.n_rows = L->n_prows;
-  q.K = c.inter;
-  q.fmt = c.fmt;
-  q.src_f32 = L->h32;
-  q.row_pair = L->prow_pair;
-  q.loc = locs;
-  q.ids = L->ids;
-  q.codes = L->hq;
-  q.sf = L->hsf;
-  q.G = L->hG;
-  launch_quant(q, s);
-  CUDA_TRY(cudaGetLastError());
-  t8.launched(1);
-  t8.end();
+  if (!fuse_hq) {
+    StageTimer t8(L, 8, s);
+    QuantArgs q{};
+    q.max_rows = (int)L->a4_rows;
+    q.n_rows = L->n_prows;
+    q.K = c.inter;
+    q.fmt = c.fmt;
+    q.src_f32 = L->h32;
+    q.row_pair = L->prow_pair;
+    q.loc = locs;
+    q.ids = L->ids;
+    q.codes = L->hq;
+    q.sf = L->hsf;
+    q.G = L->hG;
+    launch_quant(q, s);
+    CUDA_TRY(cudaGetLastError());
+    t8.launched(1);
+    t8.end();
+  }
+  g.hq_out = nullptr;
+  g.hsf_out = nullptr;
   g.act_map = 1;
   g.K = c.inter;
   g.rows = c.hidden;

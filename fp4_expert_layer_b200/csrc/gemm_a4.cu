@@ -27,6 +27,17 @@ namespace moe {
 
 namespace {
 constexpr int kGStages = 4;
+
+// Two E2M1 codes (round to nearest even, saturating): `lo` in bits 0..3.
+__device__ __forceinline__ uint32_t e2m1x2_pack(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
+      "cvt.u32.u8 %0, b;\n\t}"
+      : "=r"(r)
+      : "f"(lo), "f"(hi));
+  return r;
+}
 constexpr int kTileBytes = 128 * 128;   // 128 rows x 128 bytes (256 FP4 per row)
 constexpr int kGThreads = 256;
 }  // namespace
@@ -57,6 +68,10 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
   __shared__ float col_bs[128];
   __shared__ int col_pair[128];
   __shared__ float col_gate[128];
+  // MXFP4 gate/up with h quantised in the epilogue: per epilogue warp, the
+  // codes and block scales of 32 tokens before they go out
+  __shared__ __align__(16) uint8_t hq_stage[4][32][16];
+  __shared__ uint8_t sf_stage[4][32];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -184,7 +199,55 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
         wsc[j] = reinterpret_cast<const float *>(blob + a.L.glob)[m];
       }
     }
-    for (int cb = 0; cb < 4; ++cb) {
+    bool quantised = false;
+    if constexpr (WF == WF_MX && MODE == MODE_GATEUP) {
+      if (a.hq_out) {
+        quantised = true;
+        // h quantised here for the down pass (MXFP4 rule of the activation
+        // quantiser: per 32 consecutive h columns of a token, E8M0 exponent
+        // clamp(floor(log2 amax) - 2 + 127, 1, 254), codes RNE E2M1 of
+        // h * 2^(127 - e), saturating).  A warp holds 32 consecutive columns
+        // (one block) of each token; 32 tokens at a time so that the block
+        // maxima of different tokens reduce in parallel.
+        const int I = a.rows;
+        const int blk = (rb * 128 + 32 * quad) / 32;
+        uint8_t(*qs)[16] = hq_stage[quad];                       // [token][16 code bytes] of this warp
+        for (int cb = 0; cb < 4; ++cb) {
+          if (32 * cb >= nrows) break;                           // warp-uniform
+          uint32_t d0[32], d1[32];
+          tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * cb, d0);
+          tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 128 + 32 * cb, d1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            const float h = silu_f(__uint_as_float(d0[jj])) * __uint_as_float(d1[jj]);
+            // block maximum of |h| over the warp's 32 columns (non-negative
+            // floats order like their bit patterns)
+            const uint32_t am = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h)));
+            int code = 1;
+            if (am != 0u) {
+              const int ex = (int)((am >> 23) & 0xFF);
+              code = min(254, max(1, (ex == 0 ? -127 : ex - 127) - 2 + 127));
+            }
+            const float v = h * __int_as_float((254 - code) << 23);   // h * 2^(127 - code)
+            const float vn = __shfl_down_sync(0xffffffffu, v, 1);
+            if ((lane & 1) == 0) qs[jj][lane >> 1] = (uint8_t)(e2m1x2_pack(v, vn) & 0xFFu);
+            if (lane == 0) sf_stage[quad][jj] = (uint8_t)code;
+          }
+          __syncwarp();
+          // lane j writes token j of the chunk: 16 code bytes and one scale
+          const int col = 32 * cb + lane;
+          if (col < nrows) {
+            const size_t prow = (size_t)(prow0 + col);
+            *reinterpret_cast<uint4 *>(a.hq_out + prow * (I / 2) + (rb * 128 + 32 * quad) / 2) =
+                *reinterpret_cast<const uint4 *>(qs[lane]);
+            a.hsf_out[sf_offset(I / 32, (int)prow, blk)] = sf_stage[quad][lane];
+          }
+          __syncwarp();
+        }
+      }
+    }
+    for (int cb = 0; cb < 4 && !quantised; ++cb) {
       uint32_t d0[32], d1[32];
       tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * cb, d0);
       if constexpr (NMAT == 2) tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 128 + 32 * cb, d1);

@@ -262,6 +262,10 @@ struct A4GemmArgs {
   const uint8_t *bsf;        // activation scale blocks
   const float *bG;           // NVFP4 activation per-row scale (null for MXFP4)
   float *h_out;              // gate/up: h fp32 [rows of activations, I]
+  // gate/up, MXFP4 only (may be null): h quantised in the epilogue instead,
+  // E2M1 codes [rows, I/2] and E8M0 block scales (sf_offset layout, I/32 per row)
+  uint8_t *hq_out;
+  uint8_t *hsf_out;
   float *o_out;              // down: O' [pairs, H]
   const int *prow_pair;
   const float *gates;
