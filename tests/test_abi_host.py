@@ -98,3 +98,17 @@ def test_a4_not_silently_substituted(F):
         F.plan(cfg)
     except F.MoEError as e:       # a build without the A4 path must refuse, never fall back
         assert e.status == 6
+
+
+def test_null_handles_are_refused_without_touching_the_gpu(F):
+    """Entry points check their arguments before any CUDA call: a NULL layer or
+    graph returns MOE_ERR_INVALID_ARG (destroy of NULL is a no-op)."""
+    L = F.lib()
+    out = C.c_void_p(123)
+    assert L.moe_graph_capture(None, None, 1, None, None, C.byref(out)) == 1
+    assert L.moe_graph_launch(None, None) == 1
+    assert L.moe_graph_destroy(None) == 0
+    assert L.moe_forward(None, None, 1, None, None, None) == 1
+    assert L.moe_forward_host(None, None, 1, None, None) == 1
+    assert L.moe_set_slot_table(None, None, None) == 1
+    assert b"NULL" in L.moe_last_error()
