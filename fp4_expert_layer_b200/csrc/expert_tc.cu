@@ -96,9 +96,10 @@ void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s) {
 // Expert pass on the tensor core, persistent.  A work item is (tile, 256
 // weight rows): gate/up = 128 gate rows + the same 128 up rows (one 4-D TMA
 // box), down = 256 output rows (one 3-D box); each half has its own
-// accumulator.  Items are taken round-robin by the CTAs (concurrent CTAs then
-// work on neighbouring items: tiles of one expert share its weights in L2);
-// the stage ring runs across items, and the accumulators are double-buffered
+// accumulator.  CTAs take items from the pass's counter in index order
+// (concurrent CTAs then work on neighbouring items: tiles of one expert share
+// its weights in L2; a CTA that starts early takes more); the stage ring runs
+// across items, and the accumulators are double-buffered
 // (8-token tiles with six stages, 56-token tiles with four: 2 x 2 x 112
 // accumulator columns plus 12 scale columns per stage fill the 512 TMEM
 // columns) so the epilogue of one item overlaps the main loop of the next.

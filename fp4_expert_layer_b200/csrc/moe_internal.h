@@ -349,8 +349,8 @@ struct TcArgs {
   int early;
 };
 // nbox: activation rows per tile (2 x tile tokens): 16 or 112.  The kernel is
-// persistent: `a.grid` CTAs walk the work items (tile, 256 weight rows)
-// round-robin.
+// persistent: `a.grid` CTAs take the work items (tile, 256 weight rows) from
+// `a.work_ctr` in index order.
 void launch_expert_tc(int mode, int nbox, const TcArgs &a, int grid_tiles, cudaStream_t s);
 
 }  // namespace moe
