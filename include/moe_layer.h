@@ -264,7 +264,8 @@ moe_status_t moe_debug_inject(moe_layer_t layer, int32_t what);
 
 /* Test hook: synchronously copy up to `bytes` of an internal device buffer of
  * the last forward into host memory.  which: 1 quantised x codes, 2 x scale
- * blocks, 3 h (fp32, A4 path), 4 quantised h codes, 5 h scale blocks, 6 padded
+ * blocks, 3 h (fp32, A4 path of NVFP4 layers; MXFP4 layers quantise h in the
+ * gate/up epilogue and never write it), 4 quantised h codes, 5 h scale blocks, 6 padded
  * row count, 7 padded row -> token, 8 padded row -> pair, 11 O' (fp32);
  * tensor-core EXACT path: 12 x pieces (E4M3, 128-row slot per tile), 13 their
  * scale blocks, 14 h pieces, 15 their scale blocks, 16 tile list, 17 tile
