@@ -183,6 +183,21 @@ def cpu_baseline(lw, x_bits, budget_s, numerics="exact"):
             "sample": f"{what} ({n} tokens, {el:.1f} s, {numerics} numerics)"}
 
 
+def max_over_ranks(vals, world):
+    """Element-wise maximum of this rank's timings over all ranks, returned on
+    every rank: the job is as slow as its slowest replica."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    return vals
+
+
+def whole_job_tokens_per_s(world, tokens_per_rank, steps, max_ms):
+    """Tokens of all ranks (independent replicas, one batch each per step)
+    over the slowest rank's time for `steps` steps."""
+    return world * tokens_per_rank * steps / (max_ms / 1e3)
+
+
 def reference_arm(args, wl, lw, world):
     """--impl reference: the oracle timed on host cores, each step a bounded sample."""
     import oracle
@@ -367,14 +382,13 @@ def main():
         gph.close()
 
     vals = torch.tensor([dev_ms, e2e[0] if e2e else 0.0, graph_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    vals = max_over_ranks(vals, world)
     dev_ms_max, e2e_ms_max, graph_ms_max = float(vals[0]), float(vals[1]), float(vals[2])
 
     if rank == 0:
         hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
         ms_step = dev_ms_max / K
-        value = world * T * K / (dev_ms_max / 1e3)
+        value = whole_job_tokens_per_s(world, T, K, dev_ms_max)
         g_ms = prof["ms"]["gateup"] / max(1, prof["launches"]["gateup"])
         if args.numerics == "a4":
             # tcgen05 gate/up GEMM: FP4 FLOPs of the real (unpadded) token rows
@@ -425,10 +439,10 @@ def main():
             "clocks": clk,
         }
         if e2e:
-            line["e2e"] = {"value": world * T * e2e[1] / (e2e_ms_max / 1e3), "unit": "tokens/s",
+            line["e2e"] = {"value": whole_job_tokens_per_s(world, T, e2e[1], e2e_ms_max), "unit": "tokens/s",
                            "h2d_bytes_per_step": T * wl.hidden * 2, "d2h_bytes_per_step": T * wl.hidden * 4}
         if graph_ms_max > 0:
-            line["graph"] = {"value": world * T * K / (graph_ms_max / 1e3), "unit": "tokens/s",
+            line["graph"] = {"value": whole_job_tokens_per_s(world, T, K, graph_ms_max), "unit": "tokens/s",
                              "ms_per_step": graph_ms_max / K,
                              "how": "moe_graph_capture of this forward, replayed K times (L2 flushed before each)"}
         if world == 1 and not args.no_cpu_baseline:
