@@ -1,0 +1,72 @@
+"""Host-side pieces of bench.py that decide what a bench line reports: the
+algorithmic byte counts behind the roofline, the committed ncu traffic record
+(used only while the kernel source is unchanged), and the clock record that
+rejects throttled runs.  No GPU needed."""
+import os
+import sys
+
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_gateup_bytes_counts_codes_scales_x_and_h():
+    wl = synth.workload("olmoe_like")          # H 2048, I 1024, k 8, MXFP4 (group 32)
+    per_expert = 2 * 1024 * 2048 // 2 + 2 * 1024 * 2048 // 32   # codes + E8M0 scales of gate and up
+    want = 64 * per_expert + 32 * 2048 * 2 + 32 * 8 * 1024 * 2
+    assert bench.gateup_bytes(wl, 64, 32) == want == 143261696
+
+
+def test_layer_bytes_adds_router_shared_expert_and_io():
+    wl = synth.workload("deepseek_v4_flash_like")
+    got = bench.layer_bytes(wl, 10, 4)
+    want = (10 * wl.expert_bytes() + wl.n_experts * wl.hidden * 4 + 4 * wl.hidden * 6
+            + 3 * wl.shared_inter * wl.hidden * 2)
+    assert got == want
+
+
+def test_traffic_record_only_for_the_profiled_source(tmp_path):
+    src = os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert_tc.cu")
+    rec = bench.traffic_record("expert_tc_gateup_olmoe_like_T32.md", src)
+    assert rec is not None and rec > 1e8
+    other = tmp_path / "k.cu"
+    other.write_bytes(open(src, "rb").read() + b"\n// changed\n")
+    assert bench.traffic_record("expert_tc_gateup_olmoe_like_T32.md", str(other)) is None
+    assert bench.traffic_record("no_such_summary.md", src) is None
+
+
+class _FakeSmi:
+    def __init__(self, out):
+        self.out = out
+
+    def terminate(self):
+        pass
+
+    def communicate(self, timeout=None):
+        return self.out, ""
+
+
+@pytest.mark.parametrize("rows,reasons", [
+    (["0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active"] * 3, []),
+    (["0, 1965, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+      "0, 1830, 1965, 999.0, 0x4, Not Active, Not Active, Not Active, Active"], ["sw_power_cap"]),
+    (["0, 1200, 1965, 600.0, 0x8, Active, Not Active, Not Active, Not Active"], ["hw_slowdown"]),
+])
+def test_clock_record_reports_median_and_throttle_reasons(rows, reasons):
+    cs = bench.ClockSampler(None)
+    cs.proc = _FakeSmi("\n".join(rows + ["garbage line"]) + "\n")
+    rec = cs.stop()
+    assert rec["samples"] == len(rows)
+    assert rec["reasons"] == reasons
+    assert rec["sm_max_mhz"] == 1965.0
+    sm = sorted(float(r.split(",")[1]) for r in rows)
+    assert rec["sm_mhz"] == (sm[len(sm) // 2] if len(sm) % 2 else (sm[len(sm) // 2 - 1] + sm[len(sm) // 2]) / 2)
+
+
+def test_clock_record_without_nvidia_smi():
+    rec = bench.ClockSampler(None).stop()
+    assert rec["samples"] == 0 and rec["reasons"] == ["nvidia-smi unavailable"]
