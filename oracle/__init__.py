@@ -68,6 +68,8 @@ def lib():
         L.orc_quant_mx_block.argtypes = [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]
         L.orc_quant_nv_row.restype = None
         L.orc_quant_nv_row.argtypes = [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]
+        L.orc_a4_qdq_row.restype = None
+        L.orc_a4_qdq_row.argtypes = [C.c_int, C.c_void_p, C.c_int, C.c_void_p]
         L.orc_dequant_row.restype = None
         L.orc_dequant_row.argtypes = [C.POINTER(_Layer), C.c_int, C.c_int, C.c_int, C.c_void_p]
         L.orc_permute.restype = None
@@ -132,6 +134,14 @@ def quant_nv_row(v: np.ndarray):
     G = np.zeros(1, dtype=np.float32)
     lib().orc_quant_nv_row(_p(v), v.size, _p(codes), _p(sc), _p(G))
     return codes, sc, float(G[0])
+
+
+def a4_qdq_row(fmt: str, v: np.ndarray) -> np.ndarray:
+    """The A4 activation rule of the format applied to one row: quantise, then decode (fp64)."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.zeros(v.size, dtype=np.float64)
+    lib().orc_a4_qdq_row(FMT[fmt], _p(v), v.size, _p(out))
+    return out
 
 
 def permute(ids: np.ndarray, n_experts: int):

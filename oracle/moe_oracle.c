@@ -217,8 +217,10 @@ void orc_quant_nv_row(const float *v, int K, uint8_t *codes, uint8_t *scales, fl
   }
 }
 
-/* Quantise-dequantise one activation row per the A4 rule of the layer's format. */
-static void a4_row(int fmt, const float *v, int K, double *out) {
+/* Quantise-dequantise one activation row per the A4 rule of the layer's format:
+ * MXFP4 out[i] = e2m1(code_i) * 2^(scale_{i/32} - 127); NVFP4
+ * out[i] = e2m1(code_i) * e4m3(scale_{i/16}) * G (per-row G, rule above). */
+void orc_a4_qdq_row(int fmt, const float *v, int K, double *out) {
   uint8_t *codes = (uint8_t *)malloc((size_t)K);
   if (fmt == ORC_FMT_MXFP4) {
     uint8_t sc;
@@ -310,7 +312,7 @@ void orc_expert_token(const orc_layer_t *L, int e, const double *xt, double *o) 
   if (L->numerics == ORC_A4) {
     float *xf = (float *)malloc(sizeof(float) * (size_t)H);
     for (int c = 0; c < H; ++c) xf[c] = (float)xt[c];
-    a4_row(L->fmt, xf, H, xin);
+    orc_a4_qdq_row(L->fmt, xf, H, xin);
     free(xf);
   } else {
     memcpy(xin, xt, sizeof(double) * (size_t)H);
@@ -324,7 +326,7 @@ void orc_expert_token(const orc_layer_t *L, int e, const double *xt, double *o) 
     float af = (float)a, uf = (float)u;
     h[i] = (float)(silu((double)af) * (double)uf);
   }
-  if (L->numerics == ORC_A4) a4_row(L->fmt, h, I, hin);
+  if (L->numerics == ORC_A4) orc_a4_qdq_row(L->fmt, h, I, hin);
   else for (int i = 0; i < I; ++i) hin[i] = (double)h[i];
   for (int r = 0; r < H; ++r) {
     double acc = 0.0;

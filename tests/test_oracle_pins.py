@@ -331,6 +331,87 @@ def test_a4_mode_single_expert_matches_quantised_dense():
         assert np.allclose(y[t], ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
 
 
+def _np_e4m3(codes):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn) \
+        .to(torch.float64).numpy()
+
+
+def test_a4_qdq_row_nvfp4_hand_built():
+    """NVFP4 activation rule on a hand-worked row: per-row G != 1, two different
+    block scales, a tie broken to the even code.  Worked by hand:
+      amax_row = 168 -> G = 2^ceil(log2(168 / 2688)) = 2^-4;
+      block 0: amax 168 -> scale RN_E4M3(168/6/G) = 448; 168 -> code 6, 14 -> 0.5;
+      block 1: amax 3 -> scale RN_E4M3(3/6/G) = 8; 3 -> 6, 1 -> 2, 1.25 -> 2.5,
+               a tie between 2 and 3 broken to the even code 2."""
+    v = np.zeros(32, np.float32)
+    v[0], v[1], v[16], v[17], v[18] = 168.0, 14.0, 3.0, 1.0, 1.25
+    codes, sc, G = oracle.quant_nv_row(v)
+    assert G == 2.0 ** -4
+    assert oracle.e4m3(int(sc[0])) == 448.0 and oracle.e4m3(int(sc[1])) == 8.0
+    out = oracle.a4_qdq_row("nvfp4", v)
+    want = np.zeros(32)
+    want[0], want[1], want[16], want[17], want[18] = 168.0, 14.0, 3.0, 1.0, 1.0
+    assert np.array_equal(out, want)
+
+
+def test_a4_qdq_row_mxfp4_hand_built():
+    """MXFP4 activation rule on a hand-worked row of two 32-blocks with
+    different shared exponents: block 0 amax 6 -> 2^0 (codes exact: 6, 0.5);
+    block 1 amax 0.75 -> 2^(floor(log2 .75) - 2) = 2^-3: 0.75 -> 6 * 2^-3,
+    0.3 -> 2.4 -> 2 -> 0.25."""
+    v = np.zeros(64, np.float32)
+    v[0], v[1], v[32], v[33] = 6.0, 0.5, 0.75, 0.3
+    out = oracle.a4_qdq_row("mxfp4", v)
+    want = np.zeros(64)
+    want[0], want[1], want[32], want[33] = 6.0, 0.5, 0.75, 0.25
+    assert np.array_equal(out, want)
+
+
+def test_a4_qdq_row_nvfp4_recomposes_from_its_pieces():
+    """The recomposition e2m1(code) * e4m3(scale[i // 16]) * G, written with numpy
+    from the pieces quant_nv_row returns, on rows whose 16-blocks all differ."""
+    tab = cs.e2m1_table()
+    rng = np.random.default_rng(12)
+    for K in (64, 256):
+        v = (rng.standard_normal(K) * np.repeat(2.0 ** rng.integers(-6, 6, K // 16), 16)).astype(np.float32)
+        codes, sc, G = oracle.quant_nv_row(v)
+        assert G != 1.0 and len(set(sc.tolist())) > 1
+        ref = tab[codes] * np.repeat(_np_e4m3(sc), 16) * G
+        assert np.array_equal(oracle.a4_qdq_row("nvfp4", v), ref)
+
+
+def test_a4_mode_single_expert_matches_quantised_dense_nvfp4():
+    """E = k = 1 NVFP4 layer in A4 numerics against numpy: x and h quantised by the
+    NVFP4 activation rule (codes, per-16 E4M3 scales and per-row G from
+    quant_nv_row, recomposed here as e2m1 * e4m3(scale[i // 16]) * G), weights
+    decoded independently (e2m1 * e4m3 * per-tensor scale)."""
+    wl = synth.custom_workload(128, 64, 1, 1, fmt="nvfp4")
+    lw = synth.make_layer(wl, seed=8)
+    L = oracle.Layer.from_weights(lw, numerics="a4")
+    x = synth.make_tokens(wl, 3, seed=8)
+    y, *_ = L.forward(x)
+    tab = cs.e2m1_table()
+
+    def qdq(row):
+        codes, sc, G = oracle.quant_nv_row(np.asarray(row, np.float32))
+        assert G != 1.0
+        return tab[codes] * np.repeat(_np_e4m3(sc), 16) * G
+
+    gs = lw.global_scale[0].astype(np.float64)
+    Wg = cs.np_decode(lw.codes[0][0], lw.scales[0][0], "nvfp4", gs[0])
+    Wu = cs.np_decode(lw.codes[1][0], lw.scales[1][0], "nvfp4", gs[1])
+    Wd = cs.np_decode(lw.codes[2][0], lw.scales[2][0], "nvfp4", gs[2])
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    for t in range(3):
+        xq = qdq(xf[t])
+        a = np.float32(Wg @ xq).astype(np.float64)
+        u = np.float32(Wu @ xq).astype(np.float64)
+        h = (cs.np_silu(a) * u).astype(np.float32)
+        ref = Wd @ qdq(h)
+        assert np.allclose(y[t], ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
+
+
 def test_expert_rows_sample_sums_to_full_expert():
     """The benchmark's row-range timing sample adds up to the full expert output."""
     wl = synth.custom_workload(128, 64, 3, 1)
