@@ -1,9 +1,12 @@
-// expert_tma.cu -- routed expert FFN kernels fed by TMA, for decode-sized batches.
+// expert_tma.cu -- routed NVFP4 expert FFN kernels fed by TMA, for decode-sized batches.
 //
-// Same arithmetic as the register-fed kernel (weights = mma A operand, E2M1
-// pairs decoded to f16x2, group scale folded into f16, tokens = B operand, fp32
-// accumulation, per-chunk activation multipliers).
-// but the weight stream is decoupled from registers: one producer warp issues
+// Weights are the mma.sync A operand: E2M1 pairs are decoded to f16x2 in
+// registers by the hardware conversion and multiplied by their group's E4M3
+// scale in f16 (an E2M1 value times an E4M3 value is exact in f16); the
+// per-tensor fp32 scale is applied after the K loop.  The tokens of one
+// expert are the B operand, as f16 rows with one power-of-two multiplier per
+// 128-element chunk, and the tensor core accumulates each chunk in fp32.
+// The weight stream is decoupled from registers: one producer warp issues
 // TMA tile loads of the code bytes (64 bytes x 128 or 256 rows per 128-element
 // K chunk) and bulk copies of the matching 512-byte scale-factor blocks into a
 // 4-stage shared-memory ring guarded by mbarriers; eight consumer warps decode
@@ -32,10 +35,10 @@ constexpr int kConsumers = 8;                       // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;     // + producer warp
 constexpr int kABytes = 16384;                      // code bytes per stage (256 rows x 64 B)
 
-template <int WF>
+// Scale bytes per stage: two 128-row groups x two 512-byte E4M3 blocks (a
+// 128-element K chunk holds 8 NVFP4 groups of 16).
 struct StageGeom {
-  // scale bytes per stage: two 128-row groups x (1 block for MXFP4 | 2 blocks for NVFP4)
-  static constexpr int kSfPerGroup = (WF == WF_MX) ? 512 : 1024;
+  static constexpr int kSfPerGroup = 1024;
   static constexpr int kSfBytes = 2 * kSfPerGroup;
   static constexpr int kStageBytes = kABytes + kSfBytes;
 };
@@ -50,9 +53,9 @@ __device__ __forceinline__ uint32_t comp(const uint4 &v) {
 
 }  // namespace
 
-template <int WF, int MODE, int NT>
+template <int MODE, int NT>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(const __grid_constant__ TmaExpertArgs a) {
-  using Geo = StageGeom<WF>;
+  using Geo = StageGeom;
   constexpr int RPW = (MODE == MODE_GATEUP) ? 16 : 32;
   constexpr int RPC = RPW * kConsumers;                     // 128 (gate/up) or 256 (down) rows
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
   if (warp == kConsumers) {
     // ================= producer: one lane issues every copy
     if (lane == 0) {
-      const int nsf = K / (WF == WF_MX ? 32 : 16);
+      const int nsf = K / 16;
       for (int it = 0; it < n_iter; ++it) {
         const int s = it % kStages;
         if (it >= kStages && !mbar_wait(smem_u32(&empty_bar[s]), ((it / kStages) - 1) & 1, a.err, 2)) break;
@@ -117,8 +120,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
         const uint32_t bar = smem_u32(&full_bar[s]);
         const uint32_t dst = smem_u32(smem + (size_t)s * Geo::kStageBytes);
         mbar_arrive_expect_tx(bar, Geo::kStageBytes);
-        // scale columns covered by this chunk: MXFP4 4 columns (one block), NVFP4 8 (two blocks)
-        const int col0 = (WF == WF_MX) ? 4 * c : 8 * c;
+        // scale columns covered by this chunk: 8 (two 512-byte blocks)
+        const int col0 = 8 * c;
         if constexpr (MODE == MODE_GATEUP) {
           tma_load_3d(dst, &maps[0], bar, c * 64, rb * 128, bidx);
           tma_load_3d(dst + 8192, &maps[1], bar, c * 64, rb * 128, bidx);
@@ -142,16 +145,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
         const int m = (MODE == MODE_GATEUP) ? j : 2;
         const int local = (MODE == MODE_GATEUP) ? (warp * 16 + g + 8 * i) : (warp * 32 + 16 * j + g + 8 * i);
         mrow[j][i] = rb * RPC + local;
-        if constexpr (WF == WF_MX) rowf[j][i] = pow2f((int)blob[a.L.sref[m] + mrow[j][i]] - 127);
-        else rowf[j][i] = reinterpret_cast<const float *>(blob + a.L.glob)[m];
-      }
-    int sref[2][2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int m = (MODE == MODE_GATEUP) ? j : 2;
-        sref[j][i] = (WF == WF_MX) ? (int)blob[a.L.sref[m] + mrow[j][i]] : 0;
+        rowf[j][i] = reinterpret_cast<const float *>(blob + a.L.glob)[m];   // per-tensor fp32 scale
       }
 
     // B rows (token rows of n-tile nt, row g) and C columns (2q, 2q+1)
@@ -184,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
         const int grp = (MODE == MODE_GATEUP) ? j : (local >> 7);                 // 128-row scale group
         const int rr = local & 127;
         const uint32_t base = grp * Geo::kSfPerGroup + 16 * (rr & 31) + 4 * (rr >> 5);
-        sf_off[j][i] = kABytes + base + ((WF == WF_MX) ? q : ((q >> 1) * 512 + 2 * (q & 1)));
+        sf_off[j][i] = kABytes + base + (q >> 1) * 512 + 2 * (q & 1);
       }
 
     // B operand of chunk c: 32 sixteen-bit values of token row g, physical 32q..32q+31.
@@ -234,15 +228,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           wv[j][i] = lds128(st + a_off[j][i]);
-          if constexpr (WF == WF_MX) {
-            const int sc = smem[(size_t)s * Geo::kStageBytes + sf_off[j][i]];
-            mul[j][i][0] = mul[j][i][1] = f16x2_pow2(sc - sref[j][i]);
-          } else {
-            const uint16_t s2 = *reinterpret_cast<const uint16_t *>(smem + (size_t)s * Geo::kStageBytes + sf_off[j][i]);
-            const uint32_t h2 = e4m3x2_to_f16x2(s2);
-            mul[j][i][0] = dup_lo16(h2);
-            mul[j][i][1] = dup_hi16(h2);
-          }
+          const uint16_t s2 = *reinterpret_cast<const uint16_t *>(smem + (size_t)s * Geo::kStageBytes + sf_off[j][i]);
+          const uint32_t h2 = e4m3x2_to_f16x2(s2);
+          mul[j][i][0] = dup_lo16(h2);
+          mul[j][i][1] = dup_hi16(h2);
         }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty_bar[s]));
@@ -263,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
       e2m1x8_to_f16x2(comp<W>(wv[j][1]), f[j][1]);                                      \
     }                                                                                   \
     _Pragma("unroll") for (int sub = 0; sub < 2; ++sub) {                               \
-      constexpr int ms = (WF == WF_NV && W >= 2) ? 1 : 0;                               \
+      constexpr int ms = (W >= 2) ? 1 : 0;                                              \
       uint32_t A[2][4];                                                                 \
       _Pragma("unroll") for (int j = 0; j < 2; ++j) {                                   \
         A[j][0] = hmul2_u32(f[j][0][2 * sub], mul[j][0][ms]);                           \
@@ -417,13 +406,13 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
   }
 }
 
-template <int WF, int MODE, int NT>
+template <int MODE, int NT>
 static void launch_tma_one(const TmaExpertArgs &a, int grid_tiles, cudaStream_t s) {
-  using Geo = StageGeom<WF>;
+  using Geo = StageGeom;
   const int CS = a.k_split;
   const size_t red = CS > 1 ? (size_t)2 * NT * 4 * 256 * sizeof(float) : 0;
   const size_t smem = (size_t)kStages * Geo::kStageBytes + red + 1024;
-  auto fn = expert_tma_kernel<WF, MODE, NT>;
+  auto fn = expert_tma_kernel<MODE, NT>;
   cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(grid_tiles * a.n_rowblocks * CS));
@@ -443,24 +432,22 @@ static void launch_tma_one(const TmaExpertArgs &a, int grid_tiles, cudaStream_t 
   cudaLaunchKernelEx(&cfg, fn, a);
 }
 
-template <int WF, int MODE>
+template <int MODE>
 static void launch_tma_nt(int nt, const TmaExpertArgs &a, int grid_tiles, cudaStream_t s) {
   switch (nt) {
-    case 1: launch_tma_one<WF, MODE, 1>(a, grid_tiles, s); break;
-    case 2: launch_tma_one<WF, MODE, 2>(a, grid_tiles, s); break;
-    default: launch_tma_one<WF, MODE, 4>(a, grid_tiles, s); break;
+    case 1: launch_tma_one<MODE, 1>(a, grid_tiles, s); break;
+    case 2: launch_tma_one<MODE, 2>(a, grid_tiles, s); break;
+    default: launch_tma_one<MODE, 4>(a, grid_tiles, s); break;
   }
 }
 
 void launch_expert_tma(int wf, int mode, int nt, const TmaExpertArgs &a, int grid_tiles, cudaStream_t s) {
   if (grid_tiles <= 0) return;
-  if (wf == WF_MX) {
-    if (mode == MODE_GATEUP) launch_tma_nt<WF_MX, MODE_GATEUP>(nt, a, grid_tiles, s);
-    else launch_tma_nt<WF_MX, MODE_DOWN>(nt, a, grid_tiles, s);
-  } else {
-    if (mode == MODE_GATEUP) launch_tma_nt<WF_NV, MODE_GATEUP>(nt, a, grid_tiles, s);
-    else launch_tma_nt<WF_NV, MODE_DOWN>(nt, a, grid_tiles, s);
-  }
+  // NVFP4 experts only: MXFP4 experts in EXACT numerics run on the tensor core
+  // (expert_tc.cu)
+  if (wf != WF_NV) return;
+  if (mode == MODE_GATEUP) launch_tma_nt<MODE_GATEUP>(nt, a, grid_tiles, s);
+  else launch_tma_nt<MODE_DOWN>(nt, a, grid_tiles, s);
 }
 
 // Expert location table for one pass: start from the resident table (or all

@@ -24,6 +24,7 @@
 
 #include "device_utils.cuh"
 #include "moe_internal.h"
+#include "route_common.cuh"
 
 namespace moe {
 const char *set_error_text(const std::string &s);   // defined in api.cu
@@ -103,34 +104,8 @@ __global__ void __launch_bounds__(256) route_static_kernel(const StaticRouteArgs
     const int ee = lane + 32 * i;
     lv[i] = (ee < E) ? __ldcg(a.logits + (size_t)t * E + ee) : -INFINITY;
   }
-  uint32_t taken = 0;
-  float lmax = 0.f, my_l = 0.f;
-  int my_id = 0;
-  for (int j = 0; j < a.k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int ee = lane + 32 * i;
-      if (ee < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || lv[i] > bv)) { bv = lv[i]; bi = ee; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; }
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (j == 0) lmax = bv;
-    if (lane == j) { my_l = bv; my_id = bi; }
-  }
-  const float ex = (lane < a.k) ? expf(my_l - lmax) : 0.0f;
-  float den = 0.0f;
-  for (int j = 0; j < a.k; ++j) den += __shfl_sync(0xffffffffu, ex, j);
-  if (lane < a.k) {
-    a.ids[(size_t)t * a.k + lane] = my_id;
-    a.gates[(size_t)t * a.k + lane] = ex / den;
-  }
+  // the same warp top-k and gate arithmetic as moe_forward's routing step
+  moe::topk_warp<kPer>(lv, E, a.k, a.ids + (size_t)t * a.k, a.gates + (size_t)t * a.k, nullptr);
 }
 
 std::mutex g_setup_mu;
@@ -157,6 +132,22 @@ moe_status_t scratch_for_current_device(unsigned char **out) {
   return MOE_OK;
 }
 
+// Largest dynamic shared memory the routing kernel may use on the current
+// device: the per-block opt-in limit less the kernel's static shared memory.
+moe_status_t shared_limit_for_current_device(size_t *out) {
+  int dev = 0, optin = 0;
+  cudaFuncAttributes fa{};
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, route_static_kernel);
+  if (e != cudaSuccess) {
+    moe::set_error_text(std::string("moe_route_topk_noalloc: ") + cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  *out = (size_t)optin > fa.sharedSizeBytes ? (size_t)optin - fa.sharedSizeBytes : 0;
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" moe_status_t moe_route_topk_noalloc(const void *x, int32_t T, int32_t H, const float *router_w,
@@ -176,14 +167,25 @@ extern "C" moe_status_t moe_route_topk_noalloc(const void *x, int32_t T, int32_t
                         "split the batch or use moe_forward");
     return MOE_ERR_INVALID_ARG;
   }
-  const size_t smem = (size_t)kTT * H * sizeof(float);
-  if (smem > 227 * 1024) {
-    moe::set_error_text("moe_route_topk_noalloc: H too large for the shared-memory token tile (H <= 14528)");
+  if (reinterpret_cast<uintptr_t>(router_w) & 15u) {
+    moe::set_error_text("moe_route_topk_noalloc: router_w must be 16-byte aligned (its rows are read as float4)");
     return MOE_ERR_INVALID_ARG;
   }
   unsigned char *scratch = nullptr;
   moe_status_t st = scratch_for_current_device(&scratch);
   if (st != MOE_OK) return st;
+  // the kernel's token tile (kTT rows of x in fp32) plus its static shared
+  // memory must fit the per-block limit of the device
+  const size_t smem = (size_t)kTT * H * sizeof(float);
+  size_t smem_limit = 0;
+  st = shared_limit_for_current_device(&smem_limit);
+  if (st != MOE_OK) return st;
+  if (smem > smem_limit) {
+    const size_t hmax = (smem_limit / (kTT * sizeof(float))) & ~(size_t)3;
+    moe::set_error_text("moe_route_topk_noalloc: H too large for the shared-memory token tile (H <= " +
+                        std::to_string(hmax) + " on this device)");
+    return MOE_ERR_INVALID_ARG;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int tiles = (T + kTT - 1) / kTT;
   int *counter = reinterpret_cast<int *>(scratch + kCounterOff);

@@ -237,8 +237,11 @@ moe_status_t moe_profile_read(moe_layer_t layer, moe_profile_t *out);
  * the k.  Allocates nothing: its scratch (logits and completion counters) is a
  * fixed file-scope device array of 4 MiB + 64 KiB that every GPU loading this
  * library holds until exit.  Limits: T * E <= 2^20, T <= 65536, H a multiple of
- * 4 and at most 14528, E <= 1024, k <= min(E, 32); larger requests return
- * MOE_ERR_INVALID_ARG.  The first call on each device looks up the array's
+ * 4 whose 4-token fp32 tile (16 * H bytes) fits the device's per-block shared
+ * memory with the kernel's own (H <= 14524 on a B200, 227 KiB per block),
+ * E <= 1024, k <= min(E, 32); router_w must be 16-byte aligned (its rows are
+ * read as float4); anything else returns MOE_ERR_INVALID_ARG and launches
+ * nothing.  The first call on each device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current, so make the
  * first call before any stream capture.  All calls share the array and it
  * keeps the last call's contents (the counters are cleared at every call);
