@@ -44,7 +44,10 @@ class _Layer(C.Structure):
         ("router_w", C.c_void_p), ("router_bias", C.c_void_p),
         ("codes", C.c_void_p * 3), ("scales", C.c_void_p * 3),
         ("global_scale", C.c_void_p), ("shared_w", C.c_void_p * 3),
+        ("scoring", C.c_int), ("renorm", C.c_int), ("n_sinks", C.c_int), ("shared_gate_w", C.c_void_p),
     ]
+
+SCORING = {"softmax": 0, "sigmoid": 1}
 
 
 def lib():
@@ -82,6 +85,8 @@ def lib():
                                     C.c_void_p, C.c_int]
         L.orc_route_row.restype = None
         L.orc_route_row.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]
+        L.orc_route_row_v.restype = None
+        L.orc_route_row_v.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p]
         L.orc_max_threads.restype = C.c_int
         L.orc_expert_rows.restype = None
         L.orc_expert_rows.argtypes = [C.POINTER(_Layer), C.c_int, C.c_void_p, C.c_int, C.c_int, C.c_void_p]
@@ -155,11 +160,12 @@ def permute(ids: np.ndarray, n_experts: int):
     return counts, offsets, perm, inv
 
 
-def route_row(logits_row: np.ndarray, k: int):
+def route_row(logits_row: np.ndarray, k: int, scoring: str = "softmax", renorm: bool = True):
+    """Top-k ids and gates of one row of target logits (all targets, sinks included)."""
     l = np.ascontiguousarray(logits_row, dtype=np.float32)
     ids = np.zeros(k, dtype=np.int32)
     g = np.zeros(k, dtype=np.float32)
-    lib().orc_route_row(_p(l), l.size, k, _p(ids), _p(g))
+    lib().orc_route_row_v(_p(l), l.size, k, SCORING[scoring], 1 if renorm else 0, _p(ids), _p(g))
     return ids, g
 
 
@@ -168,10 +174,14 @@ class Layer:
 
     ``codes[m]``/``scales[m]`` are uint8 arrays [E, rows, K/2] / [E, rows, K/G]
     for m = gate, up, down; ``shared_w`` three bf16-bit uint16 matrices or None.
+    Router variants: ``router_w`` / ``router_bias`` cover the E experts and then
+    ``n_sinks`` sink targets; ``scoring`` "softmax" | "sigmoid"; ``renorm``;
+    ``shared_gate_w`` fp32 [H] or None.
     """
 
     def __init__(self, hidden, inter, n_experts, top_k, fmt, router_w, router_bias, codes, scales,
-                 global_scale=None, shared_w=None, numerics="exact"):
+                 global_scale=None, shared_w=None, numerics="exact", scoring="softmax", renorm=True,
+                 n_sinks=0, shared_gate_w=None):
         self._keep = []
 
         def keep(a, dt):
@@ -196,22 +206,28 @@ class Layer:
             s.scales[m] = _p(keep(scales[m], np.uint8))
             s.shared_w[m] = None if shared_w is None else _p(keep(shared_w[m], np.uint16))
         s.global_scale = _p(keep(global_scale, np.float32))
+        s.scoring = SCORING[scoring]
+        s.renorm = 1 if renorm else 0
+        s.n_sinks = n_sinks
+        s.shared_gate_w = _p(keep(shared_gate_w, np.float32))
+        self.n_targets = n_experts + n_sinks
         self._s = s
 
     @classmethod
     def from_weights(cls, lw, numerics="exact"):
         wl = lw.wl
         return cls(wl.hidden, wl.inter, wl.n_experts, wl.top_k, wl.fmt, lw.router_w, lw.router_bias,
-                   lw.codes, lw.scales, lw.global_scale, lw.shared_w, numerics)
+                   lw.codes, lw.scales, lw.global_scale, lw.shared_w, numerics, wl.scoring, wl.renormalize,
+                   wl.n_sinks, lw.shared_gate_w)
 
     def forward(self, x_bits: np.ndarray, rows=None, threads: int = 0):
-        """y [n,H] fp32, logits [n,E], ids [n,k], gates [n,k] for the listed token rows."""
+        """y [n,H] fp32, logits [n, E + n_sinks], ids [n,k], gates [n,k] for the listed token rows."""
         x = np.ascontiguousarray(x_bits, dtype=np.uint16)
         T = x.shape[0]
         r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
         n = T if r is None else r.size
         y = np.zeros((n, self.H), dtype=np.float32)
-        lg = np.zeros((n, self.E), dtype=np.float32)
+        lg = np.zeros((n, self.n_targets), dtype=np.float32)
         ids = np.zeros((n, self.k), dtype=np.int32)
         g = np.zeros((n, self.k), dtype=np.float32)
         rc = lib().orc_forward(C.byref(self._s), _p(x), T, _p(r), 0 if r is None else r.size,
@@ -223,7 +239,7 @@ class Layer:
     def route_all(self, x_bits: np.ndarray, threads: int = 0):
         x = np.ascontiguousarray(x_bits, dtype=np.uint16)
         T = x.shape[0]
-        lg = np.zeros((T, self.E), dtype=np.float32)
+        lg = np.zeros((T, self.n_targets), dtype=np.float32)
         ids = np.zeros((T, self.k), dtype=np.int32)
         g = np.zeros((T, self.k), dtype=np.float32)
         lib().orc_route_all(C.byref(self._s), _p(x), T, _p(lg), _p(ids), _p(g), threads)

@@ -46,17 +46,32 @@
 #define ORC_FMT_NVFP4 1
 #define ORC_EXACT 0
 #define ORC_A4 1
+#define ORC_SOFTMAX 0
+#define ORC_SIGMOID 1
 
+/* Router variants (what a checkpoint may declare; "ro99/strata", rules list:
+ * routing, expert count and top-k come from the checkpoint, and its model
+ * table: "256 experts + 2 sinks", "256 experts + 1 shared").  The routing
+ * targets are the E experts followed by n_sinks sink targets: a sink takes part
+ * in scoring, top-k and renormalisation like an expert but has no FFN, so
+ * choosing it contributes nothing to y.  scoring: softmax over all targets, or
+ * an independent sigmoid per target; renorm: the k chosen scores divided by
+ * their sum, or used as they are.  shared_gate_w (optional): the shared expert
+ * is scaled by sigmoid(x . shared_gate_w) instead of weight 1. */
 typedef struct {
   int H, I, E, k, Is;
   int fmt;                       /* ORC_FMT_* */
   int numerics;                  /* ORC_EXACT or ORC_A4 */
-  const float *router_w;         /* [E, H] */
-  const float *router_bias;      /* [E] or NULL */
+  const float *router_w;         /* [E + n_sinks, H] */
+  const float *router_bias;      /* [E + n_sinks] or NULL */
   const uint8_t *codes[3];       /* [E, rows, K/2]: gate [I,H], up [I,H], down [H,I] */
   const uint8_t *scales[3];      /* [E, rows, K/G] */
   const float *global_scale;     /* [E, 3] (NVFP4) or NULL */
   const uint16_t *shared_w[3];   /* bf16: [Is,H], [Is,H], [H,Is]; NULL if Is == 0 */
+  int scoring;                   /* ORC_SOFTMAX or ORC_SIGMOID */
+  int renorm;                    /* 1: chosen scores renormalised to sum to 1 */
+  int n_sinks;                   /* sink targets after the E experts */
+  const float *shared_gate_w;    /* [H] or NULL */
 } orc_layer_t;
 
 /* ------------------------------------------------------------------------ */
@@ -241,8 +256,9 @@ void orc_a4_qdq_row(int fmt, const float *v, int K, double *out) {
 /* ------------------------------------------------------------------------ */
 /* O2: router logits   l[t,e] = fp32( sum_h x[t,h] * W_r[e,h] + b[e] )      */
 /* ------------------------------------------------------------------------ */
+/* The logits of all E + n_sinks routing targets (experts first, then sinks). */
 void orc_router_logits_row(const orc_layer_t *L, const uint16_t *xt, float *lt) {
-  for (int e = 0; e < L->E; ++e) {
+  for (int e = 0; e < L->E + L->n_sinks; ++e) {
     double acc = 0.0;
     const float *w = L->router_w + (size_t)e * L->H;
     for (int h = 0; h < L->H; ++h) acc += orc_bf16(xt[h]) * (double)w[h];
@@ -251,25 +267,53 @@ void orc_router_logits_row(const orc_layer_t *L, const uint16_t *xt, float *lt) 
   }
 }
 
+/* Shared-expert gate logit fp32( sum_h x[t,h] * w_sg[h] ) (0 without a gate). */
+float orc_shared_gate_logit(const orc_layer_t *L, const uint16_t *xt) {
+  if (!L->shared_gate_w) return 0.0f;
+  double acc = 0.0;
+  for (int h = 0; h < L->H; ++h) acc += orc_bf16(xt[h]) * (double)L->shared_gate_w[h];
+  return (float)acc;
+}
+
 /* ------------------------------------------------------------------------ */
-/* O3: routing.  ids = the k experts of largest logit, in descending order,   */
-/* the lower index first on ties; gates = softmax over all E renormalised to  */
-/* the chosen k, i.e. exp(l_j - l_max) / sum_{i in top-k} exp(l_i - l_max).   */
+/* O3: routing over n targets.  ids = the k targets of largest logit, in     */
+/* descending order, the lower index first on ties (both scorings are        */
+/* monotone in the logit, so the order is the logits' order).  Scores, fp64: */
+/*   softmax: s_j = exp(l_j - l_max) / sum_{all n targets} exp(l_e - l_max)  */
+/*   sigmoid: s_j = 1 / (1 + exp(-l_j))                                      */
+/* gates = s_j / sum_{i in top-k} s_i when renormalised, else s_j; rounded   */
+/* to fp32.  (Softmax renormalised equals exp(l_j - l_max) over the chosen   */
+/* k's sum.)                                                                 */
 /* ------------------------------------------------------------------------ */
-void orc_route_row(const float *lt, int E, int k, int32_t *ids, float *gates) {
-  char *taken = (char *)calloc((size_t)E, 1);
+void orc_route_row_v(const float *lt, int n, int k, int scoring, int renorm, int32_t *ids, float *gates) {
+  char *taken = (char *)calloc((size_t)n, 1);
   for (int j = 0; j < k; ++j) {
     int best = -1;
-    for (int e = 0; e < E; ++e)
+    for (int e = 0; e < n; ++e)
       if (!taken[e] && (best < 0 || lt[e] > lt[best])) best = e;
     taken[best] = 1;
     ids[j] = best;
   }
   free(taken);
-  double lmax = (double)lt[ids[0]];
+  double s[64];
+  const double lmax = (double)lt[ids[0]];
+  double all = 0.0;
+  if (scoring == ORC_SOFTMAX && !renorm)
+    for (int e = 0; e < n; ++e) all += exp((double)lt[e] - lmax);
+  for (int j = 0; j < k; ++j) {
+    const double l = (double)lt[ids[j]];
+    if (scoring == ORC_SOFTMAX) s[j] = renorm ? exp(l - lmax) : exp(l - lmax) / all;
+    else s[j] = 1.0 / (1.0 + exp(-l));
+  }
   double den = 0.0;
-  for (int j = 0; j < k; ++j) den += exp((double)lt[ids[j]] - lmax);
-  for (int j = 0; j < k; ++j) gates[j] = (float)(exp((double)lt[ids[j]] - lmax) / den);
+  for (int j = 0; j < k; ++j) den += s[j];
+  for (int j = 0; j < k; ++j) gates[j] = (float)(renorm ? s[j] / den : s[j]);
+}
+
+/* The default routing: softmax over all E renormalised to the chosen k,
+ * i.e. exp(l_j - l_max) / sum_{i in top-k} exp(l_i - l_max). */
+void orc_route_row(const float *lt, int E, int k, int32_t *ids, float *gates) {
+  orc_route_row_v(lt, E, k, ORC_SOFTMAX, 1, ids, gates);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -387,14 +431,16 @@ void orc_shared_token(const orc_layer_t *L, const double *xt, double *s) {
 
 /* ------------------------------------------------------------------------ */
 /* O6: the layer.  For every listed token t:                                  */
-/*   y[t] = fp32( sum_{j<k} g_j * o_{ids_j}(x_t)  + s(x_t) )                 */
-/* the routed terms added in j order, then the shared expert.                 */
+/*   y[t] = fp32( sum_{j<k, ids_j < E} g_j * o_{ids_j}(x_t)  + gs * s(x_t) ) */
+/* the routed terms added in j order (a chosen sink adds nothing), then the   */
+/* shared expert, with gs = 1, or sigmoid(shared-gate logit) (fp64) when the  */
+/* layer has a shared-expert gate.                                            */
 /* rows: token indices to evaluate (NULL = all T); outputs are per listed row.*/
-/* logits [n,E], ids [n,k], gates [n,k] may be NULL.                          */
+/* logits [n, E + n_sinks], ids [n,k], gates [n,k] may be NULL.               */
 /* ------------------------------------------------------------------------ */
 int orc_forward(const orc_layer_t *L, const uint16_t *x, int T, const int32_t *rows, int n_rows,
                 float *y, float *logits, int32_t *ids, float *gates, int n_threads) {
-  const int H = L->H, E = L->E, k = L->k;
+  const int H = L->H, E = L->E + L->n_sinks, k = L->k;
   const int n = rows ? n_rows : T;
   if (L->Is > 0 && !L->shared_w[0]) return -1;
 #ifdef _OPENMP
@@ -416,14 +462,16 @@ int orc_forward(const orc_layer_t *L, const uint16_t *x, int T, const int32_t *r
     double *acc = (double *)calloc((size_t)H, sizeof(double));
     for (int c = 0; c < H; ++c) xt[c] = orc_bf16(xt16[c]);
     orc_router_logits_row(L, xt16, lt);
-    orc_route_row(lt, E, k, it, gt);
+    orc_route_row_v(lt, E, k, L->scoring, L->renorm, it, gt);
     for (int j = 0; j < k; ++j) {
+      if (it[j] >= L->E) continue;                 /* a sink: no FFN */
       orc_expert_token(L, it[j], xt, o);
       for (int c = 0; c < H; ++c) acc[c] += (double)gt[j] * o[c];
     }
     if (L->Is > 0) {
+      const double gs = L->shared_gate_w ? 1.0 / (1.0 + exp(-(double)orc_shared_gate_logit(L, xt16))) : 1.0;
       orc_shared_token(L, xt, o);
-      for (int c = 0; c < H; ++c) acc[c] += o[c];
+      for (int c = 0; c < H; ++c) acc[c] += gs * o[c];
     }
     for (int c = 0; c < H; ++c) y[(size_t)r * H + c] = (float)acc[c];
     if (logits) memcpy(logits + (size_t)r * E, lt, sizeof(float) * (size_t)E);
@@ -442,11 +490,12 @@ void orc_route_all(const orc_layer_t *L, const uint16_t *x, int T, float *logits
 #else
   (void)n_threads;
 #endif
+  const int n = L->E + L->n_sinks;
 #pragma omp parallel for schedule(static)
   for (int t = 0; t < T; ++t) {
-    orc_router_logits_row(L, x + (size_t)t * L->H, logits + (size_t)t * L->E);
-    orc_route_row(logits + (size_t)t * L->E, L->E, L->k, ids + (size_t)t * L->k,
-                  gates + (size_t)t * L->k);
+    orc_router_logits_row(L, x + (size_t)t * L->H, logits + (size_t)t * n);
+    orc_route_row_v(logits + (size_t)t * n, n, L->k, L->scoring, L->renorm, ids + (size_t)t * L->k,
+                    gates + (size_t)t * L->k);
   }
 }
 

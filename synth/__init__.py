@@ -56,6 +56,16 @@ class Workload:
     prefill_tokens: Optional[int]
     n_slots: int          # resident budget S
     slot_policy: str      # "all" | "hottest" | "random"
+    # router variants a checkpoint may declare (defaults: softmax, renormalised,
+    # no sinks, shared expert with weight 1)
+    scoring: str = "softmax"       # "softmax" | "sigmoid"
+    renormalize: bool = True
+    n_sinks: int = 0               # sink targets after the experts (no FFN)
+    shared_gate: bool = False      # shared expert scaled by sigmoid(x . w_sg)
+
+    @property
+    def n_targets(self) -> int:
+        return self.n_experts + self.n_sinks
 
     @property
     def group(self) -> int:
@@ -97,11 +107,12 @@ def workload(name: str) -> Workload:
 
 
 def custom_workload(hidden, inter, n_experts, top_k, shared_inter=0, fmt="mxfp4",
-                    zipf_s=None, n_slots=None, name="custom", index=99) -> Workload:
+                    zipf_s=None, n_slots=None, name="custom", index=99, scoring="softmax",
+                    renormalize=True, n_sinks=0, shared_gate=False) -> Workload:
     """A workload of arbitrary (small) shape, for tests."""
     return Workload(name, index, hidden, inter, n_experts, top_k, shared_inter, fmt,
                     zipf_s, (1,), None, n_experts if n_slots is None else n_slots,
-                    "all" if n_slots is None else "hottest")
+                    "all" if n_slots is None else "hottest", scoring, renormalize, n_sinks, shared_gate)
 
 
 # ----------------------------------------------------------------------------
@@ -126,13 +137,14 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 @dataclasses.dataclass
 class LayerWeights:
     wl: Workload
-    router_w: np.ndarray                  # fp32 [E, H]
-    router_bias: Optional[np.ndarray]     # fp32 [E] or None
-    zipf_rank: Optional[np.ndarray]       # int64 [E], 1 = most popular (None without skew)
+    router_w: np.ndarray                  # fp32 [E + n_sinks, H]
+    router_bias: Optional[np.ndarray]     # fp32 [E + n_sinks] or None
+    zipf_rank: Optional[np.ndarray]       # int64 [E + n_sinks], 1 = most popular (None without skew)
     codes: list                           # 3 x uint8 [E, rows, K/2]
     scales: list                          # 3 x uint8 [E, rows, K/G]
     global_scale: Optional[np.ndarray]    # fp32 [E, 3] (NVFP4) or None
     shared_w: Optional[list]              # 3 x uint16 bf16 bits: [Is,H], [Is,H], [H,Is]
+    shared_gate_w: Optional[np.ndarray] = None   # fp32 [H] (shared-expert gate) or None
 
 
 def _streams(seed: int, n: int):
@@ -140,7 +152,7 @@ def _streams(seed: int, n: int):
 
 
 # substream slots
-_S_X, _S_ROUTER, _S_BIAS, _S_EXPERTS, _S_SHARED, _S_RESAMPLE, _S_SLOTS = range(7)
+_S_X, _S_ROUTER, _S_BIAS, _S_EXPERTS, _S_SHARED, _S_RESAMPLE, _S_SLOTS, _S_SGATE = range(8)
 
 
 def _seed(wl: Workload, seed: Optional[int]) -> int:
@@ -154,21 +166,24 @@ def make_layer(wl: Workload, seed: Optional[int] = None, experts: Optional[int] 
     values (uniform random bytes); E8M0 block exponents uniform in [118, 124];
     NVFP4 block scales are E4M3 codes with exponent field uniform in [7, 12] and
     any mantissa (values 1..60) and a per-tensor fp32 scale of 2^-9; shared
-    expert weights N(0, 0.02^2) rounded to bf16; Zipf(s) skew as a per-expert
-    router bias -s*ln(rank) with ranks a seeded permutation of 1..E.
+    expert weights N(0, 0.02^2) rounded to bf16; Zipf(s) skew as a per-target
+    router bias -s*ln(rank) with ranks a seeded permutation of 1..E + n_sinks;
+    sink targets get router rows like experts and no expert weights; the
+    shared-expert gate vector (shared_gate) is N(0, 0.02^2) fp32.
     ``experts`` limits how many experts get distinct draws (the rest repeat
     them); only tests of host logic use it.
     """
-    ss = _streams(_seed(wl, seed), 7)
+    ss = _streams(_seed(wl, seed), 8)
     E, H = wl.n_experts, wl.hidden
+    NT = wl.n_targets                      # experts, then sink targets (router rows only)
     rng_r = np.random.Generator(np.random.PCG64(ss[_S_ROUTER]))
-    router_w = (rng_r.standard_normal((E, H), dtype=np.float32) * np.float32(0.02)).astype(np.float32)
+    router_w = (rng_r.standard_normal((NT, H), dtype=np.float32) * np.float32(0.02)).astype(np.float32)
 
     router_bias = None
     rank = None
     if wl.zipf_s is not None:
         rng_b = np.random.Generator(np.random.PCG64(ss[_S_BIAS]))
-        rank = rng_b.permutation(E) + 1
+        rank = rng_b.permutation(NT) + 1
         router_bias = (-wl.zipf_s * np.log(rank.astype(np.float64))).astype(np.float32)
 
     G = wl.group
@@ -208,7 +223,11 @@ def make_layer(wl: Workload, seed: Optional[int] = None, experts: Optional[int] 
             f32_to_bf16_bits(rng_s.standard_normal((Is, H), dtype=np.float32) * np.float32(0.02)),
             f32_to_bf16_bits(rng_s.standard_normal((H, Is), dtype=np.float32) * np.float32(0.02)),
         ]
-    return LayerWeights(wl, router_w, router_bias, rank, codes, scales, global_scale, shared_w)
+    shared_gate_w = None
+    if wl.shared_gate:
+        rng_g = np.random.Generator(np.random.PCG64(ss[_S_SGATE]))
+        shared_gate_w = (rng_g.standard_normal(H, dtype=np.float32) * np.float32(0.02)).astype(np.float32)
+    return LayerWeights(wl, router_w, router_bias, rank, codes, scales, global_scale, shared_w, shared_gate_w)
 
 
 def make_tokens(wl: Workload, T: int, seed: Optional[int] = None, stream: int = 0) -> np.ndarray:
@@ -250,7 +269,7 @@ def slot_table(lw: LayerWeights, n_slots: Optional[int] = None, seed: Optional[i
             table[:S] = np.arange(S, dtype=np.int32)
         return table
     if policy == "hottest" and lw.zipf_rank is not None:
-        order = np.argsort(lw.zipf_rank, kind="stable")
+        order = np.argsort(lw.zipf_rank[:E], kind="stable")      # experts only (sinks hold no weights)
     else:
         ss = _streams(_seed(wl, seed), 7)[_S_SLOTS]
         order = np.random.Generator(np.random.PCG64(ss)).permutation(E)

@@ -79,8 +79,12 @@ def np_silu(a):
 def dense_layer(lw, x_bits, ids_from=None):
     """Dense evaluation: every expert on every token, gate 0 outside the top-k.
 
-    Routing: numpy stable argsort on the negated fp32 logits (lower index first on
-    ties); gates: full softmax over all E, then renormalised over the chosen k.
+    Routing: numpy stable argsort on the negated fp32 logits of all targets
+    (experts, then sinks; lower index first on ties); scores: full softmax over
+    all targets, or an elementwise sigmoid; gates: the chosen scores, divided by
+    their sum when the layer renormalises.  A chosen sink keeps its gate but has
+    no FFN; the shared expert is scaled by sigmoid(fp32(x . w_sg)) when the
+    layer has a shared-expert gate.
     """
     wl = lw.wl
     E, k = wl.n_experts, wl.top_k
@@ -91,11 +95,14 @@ def dense_layer(lw, x_bits, ids_from=None):
     logits32 = logits.astype(np.float32)
     ids = np.argsort(-logits32, axis=1, kind="stable")[:, :k] if ids_from is None else ids_from
     l64 = logits32.astype(np.float64)
-    p = np.exp(l64 - l64.max(axis=1, keepdims=True))
-    p = p / p.sum(axis=1, keepdims=True)
+    if wl.scoring == "softmax":
+        p = np.exp(l64 - l64.max(axis=1, keepdims=True))
+        p = p / p.sum(axis=1, keepdims=True)
+    else:
+        p = 1.0 / (1.0 + np.exp(-l64))
     sel = np.take_along_axis(p, ids, axis=1)
-    gates = (sel / sel.sum(axis=1, keepdims=True)).astype(np.float32)
-    G = np.zeros((x.shape[0], E), dtype=np.float64)
+    gates = (sel / sel.sum(axis=1, keepdims=True) if wl.renormalize else sel).astype(np.float32)
+    G = np.zeros((x.shape[0], wl.n_targets), dtype=np.float64)
     np.put_along_axis(G, ids, gates.astype(np.float64), axis=1)
     y = np.zeros((x.shape[0], wl.hidden), dtype=np.float64)
     for e in range(E):
@@ -112,7 +119,11 @@ def dense_layer(lw, x_bits, ids_from=None):
         a = (x @ Wsg.T).astype(np.float32).astype(np.float64)
         u = (x @ Wsu.T).astype(np.float32).astype(np.float64)
         h = (np_silu(a) * u).astype(np.float32).astype(np.float64)
-        y += h @ Wsd.T
+        gs = 1.0
+        if lw.shared_gate_w is not None:
+            sg = (x @ lw.shared_gate_w.astype(np.float64)).astype(np.float32).astype(np.float64)
+            gs = (1.0 / (1.0 + np.exp(-sg)))[:, None]
+        y += gs * (h @ Wsd.T)
     return y.astype(np.float32), logits32, ids.astype(np.int32), gates
 
 

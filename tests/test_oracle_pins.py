@@ -129,6 +129,60 @@ def test_route_vs_argsort_and_full_softmax():
         assert abs(float(g.astype(np.float64).sum()) - 1.0) <= 4 * np.finfo(np.float32).eps
 
 
+@pytest.mark.parametrize("scoring, renorm", [("softmax", False), ("sigmoid", True), ("sigmoid", False)])
+def test_route_variants_vs_numpy(scoring, renorm):
+    """Selection is by logit (both scorings are monotone); scores are the full
+    softmax over all targets or the elementwise logistic; gates are the chosen
+    scores, renormalised over the k when asked."""
+    rng = np.random.default_rng(12)
+    n, k = 40, 6
+    for _ in range(200):
+        l = (3 * rng.standard_normal(n)).astype(np.float32)
+        ids, g = oracle.route_row(l, k, scoring, renorm)
+        ref_ids = np.argsort(-l, kind="stable")[:k]
+        assert np.array_equal(ids, ref_ids)
+        l64 = l.astype(np.float64)
+        if scoring == "softmax":
+            p = np.exp(l64 - l64.max())
+            p /= p.sum()
+        else:
+            p = 1.0 / (1.0 + np.exp(-l64))
+        sel = p[ref_ids]
+        ref_g = sel / sel.sum() if renorm else sel
+        assert np.allclose(g, ref_g, rtol=2e-7, atol=0)
+        if renorm:
+            assert abs(float(g.astype(np.float64).sum()) - 1.0) <= 4 * np.finfo(np.float32).eps
+        elif scoring == "softmax":
+            assert float(g.astype(np.float64).sum()) < 1.0 + 1e-6
+
+
+def test_sigmoid_gate_closed_form():
+    """logistic(0) = 1/2 and logistic(ln 3) = 3/4 exactly representable."""
+    ids, g = oracle.route_row(np.array([0.0, np.log(3.0), -50.0], np.float32), 2, "sigmoid", False)
+    assert ids.tolist() == [1, 0]
+    assert g[1] == np.float32(0.5) and abs(float(g[0]) - 0.75) <= 1e-7
+
+
+def test_sink_choice_contributes_nothing():
+    """A layer whose sink target always wins (a large bias) equals the same
+    layer without the sink with its remaining k - 1 experts' gates scaled by
+    their share: y = sum over chosen experts only; the sink's gate is lost."""
+    wl = synth.custom_workload(64, 32, 4, 3, n_sinks=1)
+    lw = synth.make_layer(wl, seed=21)
+    lw.router_bias = np.zeros(5, np.float32)
+    lw.router_bias[4] = 100.0                       # the sink is always chosen first
+    L = oracle.Layer.from_weights(lw)
+    x = synth.make_tokens(wl, 4, seed=21)
+    y, lg, ids, g = L.forward(x)
+    assert np.all(ids[:, 0] == 4)
+    assert np.all(g[:, 0] > 0.999)                  # nearly all mass on the sink
+    ry, _, rids, _ = cs.dense_layer(lw, x)
+    assert np.array_equal(ids, rids)
+    assert np.allclose(y, ry, rtol=1e-6, atol=1e-6 * np.abs(ry).max())
+    assert np.abs(y).max() < 1e-2 * np.abs(cs.dense_layer(
+        synth.make_layer(synth.custom_workload(64, 32, 4, 2), seed=21), x)[0]).max()
+
+
 def test_route_tie_goes_to_lower_index():
     l = np.array([0.5, 2.0, 1.0, 2.0, 1.0, -3.0], dtype=np.float32)
     ids, g = oracle.route_row(l, 4)
@@ -176,6 +230,13 @@ def test_single_expert_is_dense_swiglu(fmt):
     dict(hidden=64, inter=32, n_experts=4, top_k=2, fmt="nvfp4"),
     dict(hidden=64, inter=32, n_experts=5, top_k=3, shared_inter=32),
     dict(hidden=128, inter=64, n_experts=6, top_k=2, zipf_s=1.1),
+    # router variants: sigmoid scoring, no renormalisation, sink targets,
+    # sigmoid-gated shared expert
+    dict(hidden=64, inter=32, n_experts=6, top_k=2, scoring="sigmoid"),
+    dict(hidden=64, inter=32, n_experts=6, top_k=3, renormalize=False),
+    dict(hidden=64, inter=32, n_experts=4, top_k=3, n_sinks=2),
+    dict(hidden=128, inter=64, n_experts=5, top_k=3, shared_inter=32, shared_gate=True, n_sinks=2,
+         scoring="sigmoid", renormalize=False, zipf_s=1.1, fmt="nvfp4"),
 ])
 def test_bruteforce_dense_tiny(shape):
     wl = synth.custom_workload(**shape)
