@@ -1,13 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of one sparse MoE layer forward over FP4 experts on B200.
 
-Metric: MoE-layer tokens/s.  Default workload: the OLMoE-like layer (hidden
-2048, expert intermediate 1024, 64 MXFP4 experts, top-8, all resident) at a
-decode batch of 32 tokens.  A step is one full layer forward (router, top-k,
-permutation, expert gate/up + SwiGLU, down + gate scale, combine) of one batch.
+Metric: MoE-layer tokens/s.  Default workload (the largest single-GPU layer):
+the Qwen3.8-Flash-Next-like layer (hidden 4096, expert intermediate 1024, 512
+NVFP4 experts, top-10 plus one bf16 shared expert, Zipf-skewed routing) at a
+prefill of 8192 tokens with its own resident budget of 46 of 512 experts
+(hottest first), the rest copied from pinned host memory, EXACT numerics.  A
+step is one full layer forward (router, top-k, permutation, misses staged from
+host memory, expert gate/up + SwiGLU, down + gate scale, shared expert,
+combine) of one batch.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload NAME --tokens T]
   python bench.py --impl reference ...   # the CPU oracle arm (rank 0 only)
+
+Besides the headline line, the same run measures (unless --no-legs):
+  * the binding roof tau = max(t_HBM, t_PCIe, t_TC) + serial, with the pinned
+    host-to-device bandwidth measured in this process;
+  * the same layer all resident (the prefill kernels' own roofline);
+  * the OLMoE-like decode step (32 tokens, HBM roofline of the gate/up pass);
+  * the compute-bound A4 probe (FP4 tensor-pipe fraction of the FP4 GEMM).
 
 Multi-GPU: one process per GPU (torchrun), each rank an independent replica on
 its own batch (the layer has no exchange step), so value = all tokens / max
@@ -17,7 +28,8 @@ Timing: per step, L2 is flushed (a 256 MiB write) outside the timed events,
 then CUDA events on the launching stream bracket the forward; the timed region
 is bracketed by a barrier and device synchronisation and the result is the
 maximum over ranks.  Stage timing (CUDA events recorded by the library around
-each kernel) gives the live duration of the dominant kernel for the roofline.
+each kernel, in a separate pass) gives the live duration of the dominant
+kernel for the roofline.
 """
 from __future__ import annotations
 
@@ -39,16 +51,18 @@ import synth  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
 METRIC = "MoE-layer tokens/s on 1 B200; % HBM roofline (decode), % FP4 peak (prefill)"
+DEFAULT_WORKLOAD = "qwen3_8_flash_next_like"
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
-    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="olmoe_like", choices=sorted(synth.WORKLOADS))
-    p.add_argument("--tokens", type=int, default=32)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--tokens", type=int, default=None,
+                   help="batch size (default: the workload's prefill size, else its largest decode batch)")
     p.add_argument("--numerics", default="exact", choices=["exact", "a4"])
     p.add_argument("--slots", default="workload", choices=["workload", "all"],
                    help="resident budget: the workload's own, or every expert resident")
@@ -56,7 +70,12 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
-    return p.parse_args()
+    p.add_argument("--no-legs", action="store_true", help="skip the resident / decode / FP4-probe legs")
+    a = p.parse_args(argv)
+    if a.tokens is None:
+        wl = synth.workload(a.workload)
+        a.tokens = wl.prefill_tokens or max(wl.decode_tokens)
+    return a
 
 
 def peaks():
@@ -124,7 +143,7 @@ def pci_index(torch, dev):
 # ------------------------------------------------------------------ work model
 def gateup_bytes(wl, n_active, T):
     """Algorithmic HBM bytes of one routed gate/up launch: the gate and up codes and
-    block scales of every active expert, the f16 activations read once, and h written."""
+    block scales of every active expert, the activations read once, and h written."""
     per_expert = 2 * wl.inter * wl.hidden * (0.5 + 1.0 / wl.group)
     return n_active * per_expert + T * wl.hidden * 2 + T * wl.top_k * wl.inter * 2
 
@@ -136,6 +155,37 @@ def layer_bytes(wl, n_active, T):
     if wl.shared_inter:
         b += 3 * wl.shared_inter * wl.hidden * 2
     return b
+
+
+def routed_flops(wl, T):
+    """Multiply-add FLOPs of the routed experts (gate, up and down) for T tokens."""
+    return 6.0 * T * wl.top_k * wl.hidden * wl.inter
+
+
+def gateup_flops(wl, T):
+    return 4.0 * T * wl.top_k * wl.hidden * wl.inter
+
+
+def shared_flops(wl, T):
+    return 6.0 * T * wl.hidden * wl.shared_inter
+
+
+def binding_roof(wl, T, n_active, miss_bytes, h2d_gbs, hbm_gbs, tensor_tflops, serial_ms, step_ms):
+    """tau = max(t_HBM, t_PCIe, t_TC) + serial (the routing step and the combine,
+    which no other stage can overlap), and the achieved fraction tau / step.
+
+    t_HBM: algorithmic HBM bytes / measured copy bandwidth; t_PCIe: bytes of the
+    experts staged from pinned host memory / measured pinned H2D bandwidth; t_TC:
+    routed + shared FLOPs at `tensor_tflops` (the rate of the MMA kind the path
+    uses)."""
+    t_hbm = layer_bytes(wl, n_active, T) / (hbm_gbs * 1e9) * 1e3
+    t_pcie = miss_bytes / (h2d_gbs * 1e9) * 1e3 if h2d_gbs else 0.0
+    t_tc = (routed_flops(wl, T) + shared_flops(wl, T)) / (tensor_tflops * 1e12) * 1e3
+    terms = {"t_hbm_ms": t_hbm, "t_pcie_ms": t_pcie, "t_tc_ms": t_tc}
+    bind = max(terms, key=terms.get)
+    tau = terms[bind] + serial_ms
+    return {"tau_ms": tau, **terms, "serial_ms": serial_ms, "binding": bind[2:-3],
+            "step_ms": step_ms, "frac_of_tau": tau / step_ms if step_ms > 0 else None}
 
 
 def traffic_record(summary, kernel_src):
@@ -246,6 +296,129 @@ def reference_arm(args, wl, lw, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+def pinned_h2d_gbs(torch, dev, nbytes=512 << 20, reps=5):
+    """Pinned host -> device bandwidth of one large cudaMemcpyAsync (the copy the
+    staging of a missed expert issues), median over `reps`, CUDA events."""
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dst.copy_(src, non_blocking=True)
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        out.append(nbytes / (a.elapsed_time(b) / 1e3) / 1e9)
+    del src, dst
+    return statistics.median(out)
+
+
+def time_steps(torch, layer, x, y, T, K, W, flush, stream):
+    """W untimed warm-up forwards, then K forwards each bracketed by CUDA events
+    on the launching stream (L2 flushed before each); returns the summed device
+    ms and the library's stage profile from a separate pass."""
+    sp = stream.cuda_stream
+    for _ in range(W):
+        flush.zero_()
+        layer.forward_ptr(x.data_ptr(), T, y.data_ptr(), sp)
+    torch.cuda.synchronize()
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        ev0[i].record(stream)
+        layer.forward_ptr(x.data_ptr(), T, y.data_ptr(), sp)
+        ev1[i].record(stream)
+    torch.cuda.synchronize()
+    dev_ms = sum(a.elapsed_time(b) for a, b in zip(ev0, ev1))
+    return dev_ms
+
+
+def stage_profile(torch, layer, x, y, T, n, flush, stream):
+    layer.profile_enable(True)
+    for _ in range(n):
+        flush.zero_()
+        layer.forward_ptr(x.data_ptr(), T, y.data_ptr(), stream.cuda_stream)
+    torch.cuda.synchronize()
+    prof = layer.profile_read()
+    layer.profile_enable(False)
+    return prof
+
+
+def per_step(prof, stage):
+    return prof["ms"][stage] / max(1, prof["forwards"])
+
+
+def gateup_roofline(wl, T, n_active, prof, hbm_peak, bf16_sus, numerics, peak_src, traffic=None):
+    """Roofline of the routed gate/up pass (the dominant kernel): summed over the
+    pass's launches in a step (one per staging wave when experts are paged)."""
+    g_ms = per_step(prof, "gateup")
+    launches = prof["launches"]["gateup"] / max(1, prof["forwards"])
+    if numerics == "a4":
+        flops = gateup_flops(wl, T)
+        peak = 4.0 * bf16_sus
+        ach = flops / (g_ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": traffic, "kernel": "gemm_a4_kernel gate/up+SwiGLU (tcgen05 block-scaled FP4)",
+                "peak_source": f"{peak_src} bf16_tflops_sustained x 4 (nominal FP4/BF16 dense ratio)",
+                "algorithmic_flops_per_step": flops, "kernel_ms_per_step": g_ms, "launches_per_step": launches,
+                "hbm_gbs_of_same_pass": gateup_bytes(wl, n_active, T) / (g_ms / 1e3) / 1e9}
+    prefill_nv = wl.fmt == "nvfp4" and T * wl.top_k > 12 * min(wl.n_experts, T * wl.top_k)
+    if prefill_nv:
+        flops = gateup_flops(wl, T)
+        ach = flops / (g_ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": bf16_sus, "unit": "TFLOP/s", "frac": ach / bf16_sus,
+                "traffic": traffic,
+                "kernel": "expert_dq_kernel gate/up+SwiGLU (tcgen05 kind::f16, NVFP4 decoded to bf16 in shared memory)",
+                "peak_source": f"{peak_src} bf16_tflops_sustained (the MMA kind this path runs)",
+                "algorithmic_flops_per_step": flops, "kernel_ms_per_step": g_ms, "launches_per_step": launches,
+                "hbm_gbs_of_same_pass": gateup_bytes(wl, n_active, T) / (g_ms / 1e3) / 1e9}
+    b = gateup_bytes(wl, n_active, T)
+    ach = b / (g_ms / 1e3) / 1e9
+    tc = wl.fmt == "mxfp4"
+    return {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+            "traffic": traffic,
+            "kernel": ("expert_tc_kernel gate/up+SwiGLU (tcgen05, E2M1 weights x E4M3 activation pieces)"
+                       if tc else "expert_tma_kernel gate/up+SwiGLU (register decode, mma.sync)"),
+            "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_step": b, "kernel_ms_per_step": g_ms,
+            "launches_per_step": launches}
+
+
+def short_leg(torch, F, dev, flush, stream, name, T, numerics, K, W, peaks_t, slots="all"):
+    """One extra measurement on another workload / budget: tokens/s, step time
+    and the gate/up pass's roofline."""
+    hbm_peak, _, bf16_sus, src = peaks_t
+    wl = synth.workload(name)
+    lw = synth.make_layer(wl)
+    S = wl.n_experts if slots == "all" else wl.n_slots
+    layer = F.MoELayer.from_weights(lw, n_slots=S, max_tokens=T, numerics=numerics)
+    try:
+        layer.set_slot_table(synth.slot_table(lw, S))
+        xb = synth.make_tokens(wl, T)
+        x = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((T, wl.hidden), dtype=torch.float32, device=dev)
+        _, r = layer.forward(x, routing=True)
+        torch.cuda.synchronize()
+        n_active = int((r["counts"] > 0).sum().item())
+        ms = time_steps(torch, layer, x, y, T, K, W, flush, stream) / K
+        prof = stage_profile(torch, layer, x, y, T, min(K, 50), flush, stream)
+        traffic = None
+        if name == "olmoe_like" and T == 32:
+            traffic = traffic_record("expert_tc_gateup_olmoe_like_T32.md",
+                                     os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert_tc.cu"))
+        roof = gateup_roofline(wl, T, n_active, prof, hbm_peak, bf16_sus, numerics, src, traffic)
+        return {"workload": name, "tokens": T, "numerics": numerics, "resident_slots": S,
+                "value": T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": K,
+                "active_experts": n_active, "roofline": roof,
+                "layer_hbm_frac": layer_bytes(wl, n_active, T) / (ms / 1e3) / 1e9 / hbm_peak,
+                "stage_ms": {k: per_step(prof, k) for k in prof["ms"]}}
+    finally:
+        layer.close()
+
+
 def main():
     args = parse()
     wl = synth.workload(args.workload)
@@ -291,10 +464,13 @@ def main():
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    h2d_gbs = pinned_h2d_gbs(torch, dev)
 
     _, r = layer.forward(x, routing=True)
     torch.cuda.synchronize()
     n_active = int((r["counts"] > 0).sum().item())
+    misses = int(layer.stats()["last_misses"])
+    expert_bytes = int(layer.stats()["expert_bytes"])
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -321,24 +497,18 @@ def main():
     wall = time.perf_counter() - w0
     clk = clocks.stop()
     launches = layer.stats()["launches"] - launches0
+    dev_ms = sum(a.elapsed_time(b) for a, b in zip(ev0, ev1))
     # per-stage device times: a separate pass of the same loop with the
     # library's stage event pairs on, so that they do not touch the timed steps
-    layer.profile_enable(True)
-    for i in range(min(K, 200)):
-        flush.zero_()
-        layer.forward_ptr(x.data_ptr(), T, y.data_ptr(), sp)
-    torch.cuda.synchronize()
-    prof = layer.profile_read()
-    layer.profile_enable(False)
-    dev_ms = sum(a.elapsed_time(b) for a, b in zip(ev0, ev1))
+    prof = stage_profile(torch, layer, x, y, T, min(K, 50), flush, stream)
 
     # e2e through the public host-buffer call: H2D of x, forward, D2H of y
     e2e = None
     if not args.no_e2e:
         xh = torch.from_numpy(x_bits.view(np.int16)).pin_memory()
         yh = torch.empty((T, wl.hidden), dtype=torch.float32).pin_memory()
-        Ke = max(10, K // 4)
-        for _ in range(5):
+        Ke = max(5, K // 4)
+        for _ in range(2):
             layer.forward_host_ptr(xh.data_ptr(), T, yh.data_ptr(), sp)
         e0 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
         e1 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
@@ -380,50 +550,47 @@ def main():
         barrier()
         graph_ms = sum(a.elapsed_time(b) for a, b in zip(g0, g1))
         gph.close()
+    layer.close()
 
     vals = torch.tensor([dev_ms, e2e[0] if e2e else 0.0, graph_ms], dtype=torch.float64, device=dev)
     vals = max_over_ranks(vals, world)
     dev_ms_max, e2e_ms_max, graph_ms_max = float(vals[0]), float(vals[1]), float(vals[2])
 
+    # extra legs (every rank runs them, so that the collective sequence stays the same)
+    pk = peaks()
+    legs = {}
+    if not args.no_legs and world == 1:
+        if S < wl.n_experts:
+            legs["resident_leg"] = short_leg(torch, F, dev, flush, stream, wl.name, T, args.numerics,
+                                             max(5, K // 2), 2, pk)
+        legs["decode_leg"] = short_leg(torch, F, dev, flush, stream, "olmoe_like", 32, "exact", 500, 20, pk)
+        legs["fp4_leg"] = short_leg(torch, F, dev, flush, stream, "fp4_peak_probe", 8192, "a4", 20, 3, pk)
+
     if rank == 0:
-        hbm_peak, bf16_peak, bf16_sus, peak_src = peaks()
+        hbm_peak, bf16_peak, bf16_sus, peak_src = pk
         ms_step = dev_ms_max / K
         value = whole_job_tokens_per_s(world, T, K, dev_ms_max)
-        g_ms = prof["ms"]["gateup"] / max(1, prof["launches"]["gateup"])
-        if args.numerics == "a4":
-            # tcgen05 gate/up GEMM: FP4 FLOPs of the real (unpadded) token rows
-            waves = max(1.0, prof["launches"]["gateup"] / max(1, prof["forwards"]))
-            g_flops = 4.0 * T * wl.top_k * wl.hidden * wl.inter / waves
-            achieved = g_flops / (g_ms / 1e3) / 1e12
-            # the GEMM runs back to back for seconds inside the step loop: sustained figure
-            fp4_peak = 4.0 * bf16_sus
-            roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
-                    "frac": achieved / fp4_peak, "traffic": None,
-                    "kernel": "gemm_a4_kernel gate/up+SwiGLU (tcgen05 block-scaled FP4)",
-                    "peak_source": f"{peak_src} bf16_tflops_sustained x 4 (nominal FP4/BF16 dense ratio)",
-                    "algorithmic_flops_per_launch": g_flops, "kernel_ms": g_ms,
-                    "hbm_gbs_of_same_launch": gateup_bytes(wl, n_active, T) / (g_ms / 1e3) / 1e9}
-        else:
-            # paged runs launch the pass once per staging wave: bytes per launch
-            waves = max(1.0, prof["launches"]["gateup"] / max(1, prof["forwards"]))
-            g_bytes = gateup_bytes(wl, n_active, T) / waves
-            achieved = g_bytes / (g_ms / 1e3) / 1e9
-            tc = wl.fmt == "mxfp4"
-            src = os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert_tc.cu" if tc else "expert_tma.cu")
-            traffic = None
-            if tc and wl.name == "olmoe_like" and T == 32 and S == wl.n_experts:
-                traffic = traffic_record("expert_tc_gateup_olmoe_like_T32.md", src)
-            roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved / hbm_peak, "traffic": traffic,
-                    "kernel": ("expert_tc_kernel gate/up+SwiGLU (tcgen05, E2M1 weights x E4M3 activation pieces)"
-                               if tc else "expert_tma_kernel gate/up+SwiGLU (register decode, mma.sync)"),
-                    "peak_source": f"{peak_src} hbm_gbs",
-                    "algorithmic_bytes_per_launch": g_bytes, "kernel_ms": g_ms}
-        stage_ms = {k: v / max(1, prof["forwards"]) for k, v in prof["ms"].items()}
+        roof = gateup_roofline(wl, T, n_active, prof, hbm_peak, bf16_sus, args.numerics, peak_src)
+        serial = per_step(prof, "router") + per_step(prof, "permute") + per_step(prof, "combine")
+        # A4: FP4 x FP4; EXACT: 4-bit weights times 16-bit activations run at the
+        # bf16 rate (NVFP4: kind::f16) or as two 8-bit pieces at twice it (MXFP4)
+        tensor_rate = 4.0 * bf16_sus if args.numerics == "a4" else bf16_sus
+        roof["tau"] = binding_roof(wl, T, n_active, misses * expert_bytes, h2d_gbs, hbm_peak, tensor_rate,
+                                   serial, ms_step)
+        roof["tau"].update({"pinned_h2d_gbs_measured": h2d_gbs, "misses_per_step": misses,
+                            "staged_bytes_per_step": misses * expert_bytes,
+                            "tensor_rate_tflops": tensor_rate,
+                            "tensor_rate_note": ("FP4 x FP4 at 4 x measured sustained bf16" if args.numerics == "a4"
+                                                 else "EXACT numerics multiply 4-bit weights with 16-bit "
+                                                      "activations: bf16 / 8-bit-piece tensor rate (measured "
+                                                      "sustained bf16)"),
+                            "serial_stages": "router + top-k + permutation, ordered combine"})
+        stage_ms = {k: per_step(prof, k) for k in prof["ms"]}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16xfp4->f32" if args.numerics == "exact" else "fp4xfp4->f32",
+            "vs_baseline": None, "dtype": ("bf16xfp4->f32" if wl.fmt == "nvfp4" else "e4m3x2xfp4->f32")
+            if args.numerics == "exact" else "fp4xfp4->f32",
             "data": "synthetic (seeded; random-init weights of the workload's shape)",
             "config": {"workload": wl.name, "tokens": T, "hidden": wl.hidden, "inter": wl.inter,
                        "n_experts": wl.n_experts, "top_k": wl.top_k, "fmt": wl.fmt,
@@ -445,11 +612,11 @@ def main():
             line["graph"] = {"value": whole_job_tokens_per_s(world, T, K, graph_ms_max), "unit": "tokens/s",
                              "ms_per_step": graph_ms_max / K,
                              "how": "moe_graph_capture of this forward, replayed K times (L2 flushed before each)"}
+        line.update(legs)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(lw, x_bits, args.cpu_seconds, args.numerics)
         print(json.dumps(line), flush=True)
 
-    layer.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

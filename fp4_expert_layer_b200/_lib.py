@@ -18,13 +18,16 @@ SO = os.path.join(HERE, "libfp4moe.so")
 MOE_OK = 0
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ADMISSION", 3: "MOE_ERR_SLOT_TABLE",
           4: "MOE_ERR_OOM", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_UNSUPPORTED"}
-FMT = {"mxfp4": 0, "nvfp4": 1}
+FMT = {"mxfp4": 0, "nvfp4": 1, "int4g128": 2, "fp8b128": 3}
 NUMERICS = {"exact": 0, "a4": 1}
+SCORING = {"softmax": 0, "sigmoid": 1}
+OUT_DTYPE = {"f32": 0, "bf16": 1}
 
 EXPORTED = ["moe_layer_plan", "moe_admit", "moe_layer_create", "moe_set_slot_table", "moe_forward",
             "moe_forward_host", "moe_get_stats", "moe_destroy", "moe_last_error", "moe_debug_inject",
             "moe_profile_enable", "moe_profile_read", "moe_route_topk_noalloc", "moe_debug_read",
-            "moe_graph_capture", "moe_graph_launch", "moe_graph_destroy"]
+            "moe_graph_capture", "moe_graph_launch", "moe_graph_destroy", "moe_set_policy", "moe_prefetch"]
+POLICY = {"static": 0, "none": 1, "cache": 2, "hybrid": 3}
 
 
 class MoEError(RuntimeError):
@@ -36,7 +39,7 @@ class MoEError(RuntimeError):
 class Config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in (
         "hidden", "inter", "n_experts", "top_k", "shared_inter", "fmt", "renormalize", "numerics",
-        "n_slots", "max_tokens", "n_staging", "device")]
+        "n_slots", "max_tokens", "n_staging", "device", "scoring", "n_sinks", "shared_gate", "out_dtype")]
 
 
 class Weights(C.Structure):
@@ -44,6 +47,7 @@ class Weights(C.Structure):
         ("router_w", C.c_void_p), ("router_bias", C.c_void_p),
         ("codes", C.c_void_p * 3), ("scales", C.c_void_p * 3),
         ("global_scale", C.c_void_p), ("shared_w", C.c_void_p * 3),
+        ("shared_gate_w", C.c_void_p),
     ]
 
 
@@ -58,6 +62,7 @@ class Stats(C.Structure):
         ("last_path", C.c_int32), ("launches", C.c_uint64), ("expert_bytes", C.c_uint64),
         ("device_bytes", C.c_uint64),
         ("pinned_bytes", C.c_uint64), ("device_error", C.c_int32),
+        ("policy", C.c_int32), ("admitted", C.c_uint64), ("prefetched", C.c_uint64),
     ]
 
 
@@ -88,6 +93,8 @@ def lib():
         L.moe_admit.argtypes = [C.POINTER(Config), C.POINTER(Weights)]
         L.moe_layer_create.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.c_void_p, C.POINTER(C.c_void_p)]
         L.moe_set_slot_table.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p]
+        L.moe_set_policy.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p]
+        L.moe_prefetch.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p]
         L.moe_forward.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.POINTER(Routing)]
         L.moe_forward_host.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]
         L.moe_get_stats.argtypes = [C.c_void_p, C.POINTER(Stats)]
@@ -119,9 +126,11 @@ def check(status):
 
 
 def make_config(hidden, inter, n_experts, top_k, shared_inter=0, fmt="mxfp4", numerics="exact",
-                n_slots=None, max_tokens=1, n_staging=0, device=0) -> Config:
-    return Config(hidden, inter, n_experts, top_k, shared_inter, FMT[fmt], 1, NUMERICS[numerics],
-                  n_experts if n_slots is None else n_slots, max_tokens, n_staging, device)
+                n_slots=None, max_tokens=1, n_staging=0, device=0, scoring="softmax", renormalize=True,
+                n_sinks=0, shared_gate=False, out_dtype="f32") -> Config:
+    return Config(hidden, inter, n_experts, top_k, shared_inter, FMT[fmt], 1 if renormalize else 0,
+                  NUMERICS[numerics], n_experts if n_slots is None else n_slots, max_tokens, n_staging, device,
+                  SCORING[scoring], n_sinks, 1 if shared_gate else 0, OUT_DTYPE[out_dtype])
 
 
 def plan(cfg: Config) -> dict:
@@ -133,7 +142,7 @@ def plan(cfg: Config) -> dict:
 class _HostWeights:
     """Keeps the numpy arrays alive and exposes them as a moe_weights_t."""
 
-    def __init__(self, router_w, router_bias, codes, scales, global_scale, shared_w):
+    def __init__(self, router_w, router_bias, codes, scales, global_scale, shared_w, shared_gate_w=None):
         self.keep = []
         w = Weights()
 
@@ -146,8 +155,11 @@ class _HostWeights:
         w.router_bias = None if router_bias is None else arr(router_bias, np.float32).ctypes.data
         for m in range(3):
             cm = arr(codes[m], np.uint8)
-            sm = arr(scales[m], np.uint8)
             E = cm.shape[0]
+            # scales go in as their bytes: uint8 codes, bf16 bits (uint16) or fp32, by format
+            sm = np.ascontiguousarray(scales[m])
+            sm = sm.view(np.uint8).reshape(E, -1)
+            self.keep.append(sm)
             cp = (C.c_void_p * E)(*[cm[e].ctypes.data for e in range(E)])
             sp = (C.c_void_p * E)(*[sm[e].ctypes.data for e in range(E)])
             self.keep += [cp, sp]
@@ -156,11 +168,13 @@ class _HostWeights:
         w.global_scale = None if global_scale is None else arr(global_scale, np.float32).ctypes.data
         for m in range(3):
             w.shared_w[m] = None if shared_w is None else arr(shared_w[m], np.uint16).ctypes.data
+        w.shared_gate_w = None if shared_gate_w is None else arr(shared_gate_w, np.float32).ctypes.data
         self.w = w
 
 
 def weights_from_layer(lw) -> _HostWeights:
-    return _HostWeights(lw.router_w, lw.router_bias, lw.codes, lw.scales, lw.global_scale, lw.shared_w)
+    return _HostWeights(lw.router_w, lw.router_bias, lw.codes, lw.scales, lw.global_scale, lw.shared_w,
+                        getattr(lw, "shared_gate_w", None))
 
 
 def admit(cfg: Config, hw: _HostWeights):
@@ -215,15 +229,33 @@ class MoELayer:
 
     @classmethod
     def from_weights(cls, lw, n_slots=None, max_tokens=1, numerics="exact", n_staging=0, device=0,
-                     stream=None):
+                     stream=None, out_dtype="f32"):
+        """The routing semantics (scoring, renormalisation, sinks, shared-expert
+        gate) are the layer's own, as its workload declares them."""
         wl = lw.wl
         cfg = make_config(wl.hidden, wl.inter, wl.n_experts, wl.top_k, wl.shared_inter, wl.fmt, numerics,
-                          wl.n_experts if n_slots is None else n_slots, max_tokens, n_staging, device)
+                          wl.n_experts if n_slots is None else n_slots, max_tokens, n_staging, device,
+                          getattr(wl, "scoring", "softmax"), getattr(wl, "renormalize", True),
+                          getattr(wl, "n_sinks", 0), getattr(wl, "shared_gate", False), out_dtype)
         return cls(cfg, weights_from_layer(lw), stream)
+
+    @property
+    def out_torch_dtype(self):
+        import torch
+        return torch.bfloat16 if self.cfg.out_dtype == OUT_DTYPE["bf16"] else torch.float32
 
     def set_slot_table(self, table, stream=None):
         t = np.ascontiguousarray(table, dtype=np.int32)
         check(lib().moe_set_slot_table(self.handle, t.ctypes.data, _stream_ptr(stream)))
+
+    def set_policy(self, policy: str, n_pinned: int = 0, stream=None):
+        """Residency policy: "static" (the caller's table), "none", "cache" or "hybrid"."""
+        check(lib().moe_set_policy(self.handle, POLICY[policy], n_pinned, _stream_ptr(stream)))
+
+    def prefetch(self, experts, stream=None):
+        """Copy predicted experts into evictable slots ahead of a forward (cache / hybrid)."""
+        e = np.ascontiguousarray(experts, dtype=np.int32).reshape(-1)
+        check(lib().moe_prefetch(self.handle, e.ctypes.data if e.size else None, e.size, _stream_ptr(stream)))
 
     def forward(self, x, y=None, routing: bool = False, stream=None):
         import torch
@@ -231,11 +263,12 @@ class MoELayer:
         H = self.cfg.hidden
         assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[1] == H
         if y is None:
-            y = torch.empty((T, H), dtype=torch.float32, device=x.device)
+            y = torch.empty((T, H), dtype=self.out_torch_dtype, device=x.device)
+        assert y.dtype == self.out_torch_dtype and y.is_contiguous()
         r = None
         rp = None
         if routing:
-            E, k = self.cfg.n_experts, self.cfg.top_k
+            E, k = self.cfg.n_experts + self.cfg.n_sinks, self.cfg.top_k   # routing targets
             dev = x.device
             r = {
                 "logits": torch.empty((T, E), dtype=torch.float32, device=dev),
@@ -258,7 +291,8 @@ class MoELayer:
         x = np.ascontiguousarray(x_host, dtype=np.uint16)
         T = x.shape[0]
         if y_host is None:
-            y_host = np.empty((T, self.cfg.hidden), dtype=np.float32)
+            bf16 = self.cfg.out_dtype == OUT_DTYPE["bf16"]
+            y_host = np.empty((T, self.cfg.hidden), dtype=np.uint16 if bf16 else np.float32)
         check(lib().moe_forward_host(self.handle, x.ctypes.data, T, y_host.ctypes.data, _stream_ptr(stream)))
         return y_host
 

@@ -54,26 +54,30 @@ BlobLayout moe::blob_layout(int H, int I, int fmt, int tiled) {
   BlobLayout L{};
   L.fmt = fmt;
   L.tiled = tiled;
-  L.G = fmt == MOE_FMT_MXFP4 ? 32 : 16;
+  L.G = fmt == MOE_FMT_MXFP4 ? 32 : (fmt == MOE_FMT_NVFP4 ? 16 : 128);
   size_t off = 0;
   for (int m = 0; m < 3; ++m) {
     L.rows[m] = (m < 2) ? I : H;
     L.K[m] = (m < 2) ? H : I;
     L.codes[m] = off;
-    off = align256(off + (size_t)L.rows[m] * L.K[m] / 2);
+    const size_t cb = fmt == MOE_FMT_FP8B128 ? (size_t)L.rows[m] * L.K[m] : (size_t)L.rows[m] * L.K[m] / 2;
+    off = align256(off + cb);
   }
   for (int m = 0; m < 3; ++m) {
     L.scales[m] = off;
-    off = align256(off + (size_t)L.rows[m] * L.K[m] / L.G);
+    size_t sb = (size_t)L.rows[m] * L.K[m] / L.G;                                  // one byte per block
+    if (fmt == MOE_FMT_INT4G128) sb *= 2;                                           // bf16 per row and group
+    if (fmt == MOE_FMT_FP8B128) sb = (size_t)(L.rows[m] / 128) * (L.K[m] / 128) * 4;  // fp32 per 128 x 128
+    off = align256(off + sb);
   }
+  for (int m = 0; m < 3; ++m) L.sref[m] = 0;
+  L.glob = 0;
   if (fmt == MOE_FMT_MXFP4) {
     for (int m = 0; m < 3; ++m) {
       L.sref[m] = off;
       off = align256(off + (size_t)L.rows[m]);
     }
-    L.glob = 0;
-  } else {
-    for (int m = 0; m < 3; ++m) L.sref[m] = 0;
+  } else if (fmt == MOE_FMT_NVFP4) {
     L.glob = off;
     off = align256(off + 3 * sizeof(float));
   }
@@ -123,6 +127,11 @@ struct moe_layer {
   uint8_t *txq = nullptr, *txsf = nullptr, *thq = nullptr, *thsf = nullptr;
   int *tc_work = nullptr;            // [kWorkCtrs] item counters of the expert passes
   int *tile_done = nullptr;          // [tc tiles] gate/up items finished per tile (decode hand-over)
+  // EXACT numerics of NVFP4 experts at prefill sizes on the tensor core
+  // (weights decoded to bf16 in shared memory)
+  bool nv = false;
+  DqMaps dqmaps{};
+  int *dq_work = nullptr;            // [kWorkCtrs] item counters of the two passes
   // host
   uint8_t *store = nullptr;          // pinned: E x blob bytes
   int *h_counts = nullptr;           // pinned [E]
@@ -130,8 +139,17 @@ struct moe_layer {
   int *h_loc = nullptr;              // pinned [E]
   std::vector<int> slot_of;
   int n_resident = 0;
-  uint64_t table_version = 0;        // bumped by every moe_set_slot_table
+  uint64_t table_version = 0;        // bumped by every change of the slot table
   size_t max_prows = 0, max_tiles = 0;
+  // library-managed residency (moe_set_policy): the slot holding each
+  // expert changes only between forwards, by admission of staged misses
+  // (cache / hybrid) or by moe_prefetch
+  int policy = MOE_POLICY_STATIC;
+  int n_pinned = 0;                  // hybrid: slots [0, n_pinned) are never evicted
+  std::vector<int> expert_of_slot;   // [S] expert in each slot, -1 = empty
+  std::vector<uint64_t> last_use;    // [E] forward index of each expert's last use
+  cudaEvent_t ev_prefetch = nullptr; // prefetch copies done (side stream)
+  bool prefetch_pending = false;
   moe_stats_t st{};
   int inject = 0;
   bool staging_used = false;
@@ -194,13 +212,24 @@ static moe_status_t check_config(const moe_config_t *c) {
   if (c->hidden <= 0 || c->hidden % 256) return fail(MOE_ERR_INVALID_ARG, "hidden must be a positive multiple of 256");
   if (c->inter <= 0 || c->inter % 128) return fail(MOE_ERR_INVALID_ARG, "inter must be a positive multiple of 128");
   if (c->n_experts < 1 || c->n_experts > kMaxExperts) return fail(MOE_ERR_INVALID_ARG, "n_experts must be in 1..1024");
-  if (c->top_k < 1 || c->top_k > std::min(c->n_experts, kMaxTopK))
-    return fail(MOE_ERR_INVALID_ARG, "top_k must be in 1..min(n_experts, 32)");
+  if (c->n_sinks < 0 || c->shared_gate < 0 || c->shared_gate > 1 ||
+      c->n_experts + c->n_sinks + c->shared_gate > kMaxExperts)
+    return fail(MOE_ERR_INVALID_ARG, "need n_sinks >= 0, shared_gate 0 or 1, n_experts + n_sinks + shared_gate <= 1024");
+  if (c->top_k < 1 || c->top_k > std::min(c->n_experts + c->n_sinks, kMaxTopK))
+    return fail(MOE_ERR_INVALID_ARG, "top_k must be in 1..min(n_experts + n_sinks, 32)");
   if (c->shared_inter < 0 || c->shared_inter % 128) return fail(MOE_ERR_INVALID_ARG, "shared_inter must be 0 or a multiple of 128");
-  if (c->fmt != MOE_FMT_MXFP4 && c->fmt != MOE_FMT_NVFP4) return fail(MOE_ERR_INVALID_ARG, "fmt must be MXFP4 or NVFP4");
-  if (c->renormalize != 1) return fail(MOE_ERR_UNSUPPORTED, "only renormalised top-k gates are implemented (renormalize = 1)");
+  if (c->shared_gate && c->shared_inter == 0) return fail(MOE_ERR_INVALID_ARG, "shared_gate needs a shared expert");
+  if (c->fmt < MOE_FMT_MXFP4 || c->fmt > MOE_FMT_FP8B128)
+    return fail(MOE_ERR_INVALID_ARG, "fmt must be MXFP4, NVFP4, INT4G128 or FP8B128");
+  if (c->renormalize != 0 && c->renormalize != 1) return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
+  if (c->scoring != MOE_SCORING_SOFTMAX && c->scoring != MOE_SCORING_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "scoring must be SOFTMAX or SIGMOID");
+  if (c->out_dtype != MOE_OUT_F32 && c->out_dtype != MOE_OUT_BF16) return fail(MOE_ERR_INVALID_ARG, "out_dtype must be F32 or BF16");
   if (c->numerics != MOE_NUMERICS_EXACT && c->numerics != MOE_NUMERICS_A4)
     return fail(MOE_ERR_INVALID_ARG, "numerics must be EXACT or A4");
+  if (c->numerics == MOE_NUMERICS_A4 && c->fmt != MOE_FMT_MXFP4 && c->fmt != MOE_FMT_NVFP4)
+    return fail(MOE_ERR_UNSUPPORTED, "A4 numerics quantises activations to the experts' FP4 format: "
+                                     "MXFP4 and NVFP4 layers only");
   if (c->n_slots < 0 || c->n_slots > c->n_experts) return fail(MOE_ERR_INVALID_ARG, "n_slots must be in 0..n_experts");
   if (c->max_tokens < 1 || (int64_t)c->max_tokens * c->top_k > (1 << 30))
     return fail(MOE_ERR_INVALID_ARG, "max_tokens must be >= 1 and max_tokens * top_k <= 2^30");
@@ -214,6 +243,11 @@ static int default_staging(const moe_config_t *c) {
   if (c->n_staging > 0) return c->n_staging;
   return std::max(2, std::min(c->n_experts - c->n_slots, 64));
 }
+
+// Routing targets (experts, then sinks) and router logit rows (targets, then
+// the shared-expert gate row when the layer has one).
+static int n_targets(const moe_config_t *c) { return c->n_experts + c->n_sinks; }
+static int n_logit_rows(const moe_config_t *c) { return n_targets(c) + c->shared_gate; }
 
 struct Sizes {
   size_t P, max_prows, max_tiles, a4_rows, tc_tiles;
@@ -245,7 +279,18 @@ static bool uses_tc(const moe_config_t *c) {
   return c->numerics == MOE_NUMERICS_EXACT && c->fmt == MOE_FMT_MXFP4;
 }
 
+// NVFP4 layers in EXACT numerics: prefill-sized batches run the tensor-core
+// kernels that decode weights to bf16 in shared memory (decode-sized batches
+// keep the register-decode kernels); both read the same blob layout.
+static bool uses_dq(const moe_config_t *c) {
+  return c->numerics == MOE_NUMERICS_EXACT && c->fmt != MOE_FMT_MXFP4;
+}
+// INT4 group-128 and FP8 block-128 experts run only on the dequantising
+// tensor-core kernels (every batch size)
+static bool dq_only(const moe_config_t *c) { return c->fmt == MOE_FMT_INT4G128 || c->fmt == MOE_FMT_FP8B128; }
+
 static size_t tc_scratch_bytes(const moe_config_t *c) {
+  if (uses_dq(c)) return align256(kWorkCtrs * sizeof(int));
   if (!uses_tc(c)) return 0;
   const Sizes z = sizes_of(c);
   const size_t R = z.tc_tiles * kTcSlotRows, H = c->hidden, I = c->inter;
@@ -257,7 +302,8 @@ static size_t scratch_bytes(const moe_config_t *c) {
   const Sizes z = sizes_of(c);
   const size_t T = c->max_tokens, H = c->hidden, I = c->inter, E = c->n_experts, Is = c->shared_inter;
   size_t b = 0;
-  b += align256(T * E * 4) + align256(z.P * 4) * 4 + align256(E * 4) + align256((E + 1) * 4);
+  const size_t NT = n_targets(c), NR = n_logit_rows(c);
+  b += align256(T * NR * 4) + align256(z.P * 4) * 4 + align256(NT * 4) + align256((NT + 1) * 4);
   b += align256(z.max_tiles * sizeof(TileInfo)) + 2 * align256(4) + 2 * align256(z.max_prows * 4);
   b += align256(T * H * 2) + align256(T * (H / kChunk) * 4);
   b += align256(z.max_prows * I * 2) + align256(z.max_prows * (I / kChunk) * 4);
@@ -309,6 +355,7 @@ static void free_layer(moe_layer *L) {
   }
   if (L->ev_counts) cudaEventDestroy(L->ev_counts);
   if (L->ev_fwd_done) cudaEventDestroy(L->ev_fwd_done);
+  if (L->ev_prefetch) cudaEventDestroy(L->ev_prefetch);
   for (auto &p : L->pend) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
   for (auto e : L->evpool) cudaEventDestroy(e);
   if (L->side) cudaStreamDestroy(L->side);
@@ -329,14 +376,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 3-D map over the code bytes of matrix m of every blob in a region:
-// (K/2 bytes, rows, blob index), box 64 bytes x box_rows x 1, no swizzle.
+// (K/2 bytes, rows, blob index), box box_bytes x box_rows x 1, no swizzle.
 static moe_status_t make_code_map(CUtensorMap *map, const uint8_t *region, int nblobs, const BlobLayout &L, int m,
-                                  int box_rows) {
+                                  int box_rows, int box_bytes = 64) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  cuuint64_t dims[3] = {(cuuint64_t)(L.K[m] / 2), (cuuint64_t)L.rows[m], (cuuint64_t)nblobs};
-  cuuint64_t strides[2] = {(cuuint64_t)(L.K[m] / 2), (cuuint64_t)L.bytes};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  const cuuint64_t row_bytes = L.fmt == MOE_FMT_FP8B128 ? (cuuint64_t)L.K[m] : (cuuint64_t)(L.K[m] / 2);
+  cuuint64_t dims[3] = {row_bytes, (cuuint64_t)L.rows[m], (cuuint64_t)nblobs};
+  cuuint64_t strides[2] = {row_bytes, (cuuint64_t)L.bytes};
+  cuuint32_t box[3] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, (void *)(region + L.codes[m]), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -426,6 +474,66 @@ static moe_status_t make_bf16_map(CUtensorMap *map, const void *base, size_t K, 
 constexpr int kDenseTcMinTokens = 256;
 constexpr size_t kRouterPartFloats = (size_t)4 << 20;   // 16 MiB of split-K partial logits
 
+// ------------------------------------------------------------------ residency policies
+// Slots a CACHE / HYBRID layer may overwrite now: not pinned, and either empty
+// or holding an expert that `busy` does not mark; empty first, then least
+// recently used (ties: lower slot).
+static std::vector<int> evictable_slots(const moe_layer *L, const std::vector<char> &busy) {
+  std::vector<int> cand;
+  const int S = L->cfg.n_slots;
+  const int first = L->policy == MOE_POLICY_HYBRID ? L->n_pinned : 0;
+  for (int v = first; v < S; ++v) {
+    const int u = L->expert_of_slot[v];
+    if (u < 0 || !busy[u]) cand.push_back(v);
+  }
+  std::stable_sort(cand.begin(), cand.end(), [&](int a, int b) {
+    const int ua = L->expert_of_slot[a], ub = L->expert_of_slot[b];
+    const uint64_t ka = ua < 0 ? 0 : L->last_use[ua] + 1, kb = ub < 0 ? 0 : L->last_use[ub] + 1;
+    return ka < kb;
+  });
+  return cand;
+}
+
+// Admission plan of one staged forward (CACHE / HYBRID): slot for each miss
+// (index into `misses`) or -1.  Misses with more tokens are admitted first;
+// only slots whose expert this forward does not use are taken.
+static std::vector<int> plan_admission(const moe_layer *L, const std::vector<int> &misses) {
+  std::vector<int> slot(misses.size(), -1);
+  if (L->policy != MOE_POLICY_CACHE && L->policy != MOE_POLICY_HYBRID) return slot;
+  const int E = L->cfg.n_experts;
+  std::vector<char> busy(E, 0);
+  for (int e = 0; e < E; ++e) busy[e] = L->h_counts[e] > 0;
+  const std::vector<int> cand = evictable_slots(L, busy);
+  std::vector<int> order(misses.size());
+  for (size_t i = 0; i < order.size(); ++i) order[i] = (int)i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int a, int b) { return L->h_counts[misses[a]] > L->h_counts[misses[b]]; });
+  for (size_t i = 0; i < order.size() && i < cand.size(); ++i) slot[order[i]] = cand[i];
+  return slot;
+}
+
+// Bring the device copies of the slot table up to date with the host's
+// (slot_of), ordered on `s` behind the work already queued there.  The sources
+// are pageable, so the call returns once they have been read.
+static moe_status_t push_table(moe_layer *L, cudaStream_t s) {
+  const int E = L->cfg.n_experts;
+  const size_t bytes = L->L.bytes;
+  std::vector<int> loc(E);
+  std::vector<const uint8_t *> ptr(E);
+  int n = 0;
+  for (int e = 0; e < E; ++e) {
+    const int v = L->slot_of[e];
+    loc[e] = v >= 0 ? v : kLocAbsent;
+    ptr[e] = v >= 0 ? L->slots + (size_t)v * bytes : nullptr;
+    n += v >= 0;
+  }
+  CUDA_TRY(cudaMemcpyAsync(L->loc_resident, loc.data(), sizeof(int) * E, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaMemcpyAsync(L->ptr_resident, ptr.data(), sizeof(void *) * E, cudaMemcpyHostToDevice, s));
+  L->n_resident = n;
+  L->table_version += 1;
+  return MOE_OK;
+}
+
 // ------------------------------------------------------------------ C ABI
 extern "C" {
 
@@ -438,7 +546,7 @@ moe_status_t moe_layer_plan(const moe_config_t *cfg, moe_plan_t *out) {
   out->expert_bytes = L.bytes;
   out->slot_bytes = (uint64_t)L.bytes * cfg->n_slots;
   out->staging_bytes = (uint64_t)L.bytes * default_staging(cfg);
-  out->resident_bytes = (uint64_t)cfg->n_experts * cfg->hidden * 4 + cfg->n_experts * 4 +
+  out->resident_bytes = (uint64_t)n_logit_rows(cfg) * cfg->hidden * 4 + n_logit_rows(cfg) * 4 +
                         (uint64_t)3 * cfg->shared_inter * cfg->hidden * 2;
   out->scratch_bytes = scratch_bytes(cfg) + a4_scratch_bytes(cfg) + tc_scratch_bytes(cfg);
   out->pinned_bytes = (uint64_t)L.bytes * cfg->n_experts;
@@ -455,10 +563,47 @@ moe_status_t moe_admit(const moe_config_t *cfg, const moe_weights_t *w) {
     return fail(MOE_ERR_INVALID_ARG, "shared expert weights are NULL");
   if (cfg->fmt == MOE_FMT_NVFP4 && !w->global_scale)
     return fail(MOE_ERR_INVALID_ARG, "NVFP4 needs global_scale [E,3]");
+  if (cfg->shared_gate && !w->shared_gate_w)
+    return fail(MOE_ERR_INVALID_ARG, "shared_gate needs shared_gate_w [H]");
   for (int e = 0; e < cfg->n_experts; ++e) {
     for (int m = 0; m < 3; ++m) {
       const uint8_t *s = w->scales[m][e];
       if (!s || !w->codes[m][e]) return fail(MOE_ERR_INVALID_ARG, "NULL expert pointer");
+      if (cfg->fmt == MOE_FMT_INT4G128 || cfg->fmt == MOE_FMT_FP8B128) {
+        // INT4: bf16 scales [rows, K/128], NaN / infinity rejected; FP8: fp32
+        // inverse scales [rows/128, K/128] must be finite and positive, and an
+        // E4M3 NaN code (S.1111.111) in the weights is rejected
+        const bool i4 = cfg->fmt == MOE_FMT_INT4G128;
+        const size_t n = i4 ? (size_t)L.rows[m] * (L.K[m] / 128) : (size_t)(L.rows[m] / 128) * (L.K[m] / 128);
+        for (size_t i = 0; i < n; ++i) {
+          bool bad;
+          if (i4) {
+            uint16_t b;
+            memcpy(&b, s + 2 * i, 2);
+            bad = (b & 0x7F80u) == 0x7F80u;
+          } else {
+            float f;
+            memcpy(&f, s + 4 * i, 4);
+            bad = !(f > 0.0f) || f == INFINITY;
+          }
+          if (bad) {
+            char buf[160];
+            snprintf(buf, sizeof buf, "scale admission failed: expert %d matrix %d index %zu", e, m, i);
+            return fail(MOE_ERR_ADMISSION, buf);
+          }
+        }
+        if (!i4) {
+          const uint8_t *q = w->codes[m][e];
+          const size_t nq = (size_t)L.rows[m] * L.K[m];
+          for (size_t i = 0; i < nq; ++i)
+            if ((q[i] & 0x7Fu) == 0x7Fu) {
+              char buf[160];
+              snprintf(buf, sizeof buf, "weight admission failed: E4M3 NaN code in expert %d matrix %d index %zu", e, m, i);
+              return fail(MOE_ERR_ADMISSION, buf);
+            }
+        }
+        continue;
+      }
       const size_t n = (size_t)L.rows[m] * L.K[m] / L.G;
       for (size_t i = 0; i < n; ++i) {
         const unsigned c = s[i];
@@ -522,6 +667,27 @@ static void pack_expert(const moe_config_t *cfg, const BlobLayout &L, const moe_
     pack_expert_tiled(L, w, e, dst);
     return;
   }
+  if (cfg->fmt == MOE_FMT_INT4G128 || cfg->fmt == MOE_FMT_FP8B128) {
+    for (int m = 0; m < 3; ++m) {
+      const int rows = L.rows[m], K = L.K[m];
+      if (cfg->fmt == MOE_FMT_FP8B128) {
+        // codes and the [rows/128, K/128] fp32 block scales as they are
+        memcpy(dst + L.codes[m], w->codes[m][e], (size_t)rows * K);
+        memcpy(dst + L.scales[m], w->scales[m][e], (size_t)(rows / 128) * (K / 128) * 4);
+      } else {
+        // codes as they are; the bf16 scales of each (128-row block, K group)
+        // contiguous (256 bytes), so that one slab's scales are one copy
+        memcpy(dst + L.codes[m], w->codes[m][e], (size_t)rows * K / 2);
+        const int ng = K / 128;
+        const uint8_t *src = w->scales[m][e];
+        for (int r = 0; r < rows; ++r)
+          for (int g = 0; g < ng; ++g)
+            memcpy(dst + L.scales[m] + ((size_t)(r / 128) * ng + g) * 256 + (r % 128) * 2,
+                   src + ((size_t)r * ng + g) * 2, 2);
+      }
+    }
+    return;
+  }
   for (int m = 0; m < 3; ++m) {
     const size_t ncode = (size_t)L.rows[m] * L.K[m] / 2;
     const size_t nsc = (size_t)L.rows[m] * L.K[m] / L.G;
@@ -559,7 +725,7 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   moe_layer *L = new moe_layer();
   L->cfg = *cfg;
   L->L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt, uses_tc(cfg));
-  L->wf = cfg->fmt == MOE_FMT_MXFP4 ? WF_MX : WF_NV;
+  L->wf = cfg->fmt == MOE_FMT_MXFP4 ? WF_MX : (cfg->fmt == MOE_FMT_NVFP4 ? WF_NV : -1);
   L->n_staging = default_staging(cfg);
   L->cfg.n_staging = L->n_staging;
   const int E = cfg->n_experts, H = cfg->hidden, I = cfg->inter, Is = cfg->shared_inter;
@@ -609,8 +775,10 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   }
 
   // device memory
-  C_TRY(dalloc(L, &L->router_w, (size_t)E * H * 4));
-  if (w->router_bias) C_TRY(dalloc(L, &L->router_b, (size_t)E * 4));
+  // router rows: the E experts, the sinks, then the shared-expert gate row
+  const int NT = n_targets(cfg), NR = n_logit_rows(cfg);
+  C_TRY(dalloc(L, &L->router_w, (size_t)NR * H * 4));
+  if (w->router_bias) C_TRY(dalloc(L, &L->router_b, (size_t)NR * 4));
   if (Is) for (int m = 0; m < 3; ++m) C_TRY(dalloc(L, &L->shared_w[m], (size_t)Is * H * 2));
   if (cfg->n_slots) C_TRY(dalloc(L, &L->slots, bytes * cfg->n_slots));
   if (L->n_staging) C_TRY(dalloc(L, &L->staging, bytes * L->n_staging));
@@ -618,13 +786,13 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   C_TRY(dalloc(L, &L->ptr_pass, sizeof(void *) * E));
   C_TRY(dalloc(L, &L->loc_resident, sizeof(int) * E));
   C_TRY(dalloc(L, &L->loc_pass, sizeof(int) * E));
-  C_TRY(dalloc(L, &L->logits, T * E * 4));
+  C_TRY(dalloc(L, &L->logits, T * NR * 4));
   C_TRY(dalloc(L, &L->ids, z.P * 4));
   C_TRY(dalloc(L, &L->gates, z.P * 4));
   C_TRY(dalloc(L, &L->perm, z.P * 4));
   C_TRY(dalloc(L, &L->inv, z.P * 4));
-  C_TRY(dalloc(L, &L->counts, (size_t)E * 4));
-  C_TRY(dalloc(L, &L->offsets, (size_t)(E + 1) * 4));
+  C_TRY(dalloc(L, &L->counts, (size_t)NT * 4));
+  C_TRY(dalloc(L, &L->offsets, (size_t)(NT + 1) * 4));
   C_TRY(dalloc(L, &L->tiles, z.max_tiles * sizeof(TileInfo)));
   C_TRY(dalloc(L, &L->n_tiles, 4));
   C_TRY(dalloc(L, &L->active, 4));
@@ -688,6 +856,11 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     C_TRY(dalloc(L, &L->tile_done, z.tc_tiles * sizeof(int)));
     C_CUDA(cudaMemsetAsync(L->tile_done, 0, z.tc_tiles * sizeof(int), s));
   }
+  L->nv = uses_dq(cfg);
+  if (L->nv) {
+    C_TRY(dalloc(L, &L->dq_work, kWorkCtrs * sizeof(int)));
+    C_CUDA(cudaMemsetAsync(L->dq_work, 0, kWorkCtrs * sizeof(int), s));
+  }
   C_TRY(dalloc(L, &L->yout, T * H * 4));
 
   C_CUDA(cudaMemsetAsync(L->router_counter, 0, ((T + 3) / 4) * 4, s));
@@ -705,6 +878,12 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     if (L->n_staging) C_TRY(make_code_map(&L->maps.stage[m], L->staging, L->n_staging, L->L, m, box_rows));
     if (L->a4 && cfg->n_slots) C_TRY(make_a4_weight_map(&L->a4maps.w[0][m], L->slots, cfg->n_slots, L->L, m));
     if (L->a4 && L->n_staging) C_TRY(make_a4_weight_map(&L->a4maps.w[1][m], L->staging, L->n_staging, L->L, m));
+    // dequantising kernels: one 64-element K slab per box (32 bytes of nibbles, or 64 FP8 bytes)
+    const int dq_box = cfg->fmt == MOE_FMT_FP8B128 ? 64 : 32;
+    if (L->nv && cfg->n_slots)
+      C_TRY(make_code_map(&L->dqmaps.slot[m], L->slots, cfg->n_slots, L->L, m, box_rows, dq_box));
+    if (L->nv && L->n_staging)
+      C_TRY(make_code_map(&L->dqmaps.stage[m], L->staging, L->n_staging, L->L, m, box_rows, dq_box));
   }
   if (L->tc) {
     for (int g = 0; g < 2; ++g) {
@@ -712,8 +891,13 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
       if (L->n_staging) C_TRY(make_tc_weight_map(&L->tcmaps.w[1][g], L->staging, L->n_staging, L->L, g == 0));
     }
   }
-  C_CUDA(cudaMemcpyAsync(L->router_w, w->router_w, (size_t)E * H * 4, cudaMemcpyHostToDevice, s));
-  if (w->router_bias) C_CUDA(cudaMemcpyAsync(L->router_b, w->router_bias, (size_t)E * 4, cudaMemcpyHostToDevice, s));
+  C_CUDA(cudaMemcpyAsync(L->router_w, w->router_w, (size_t)NT * H * 4, cudaMemcpyHostToDevice, s));
+  if (cfg->shared_gate)
+    C_CUDA(cudaMemcpyAsync(L->router_w + (size_t)NT * H, w->shared_gate_w, (size_t)H * 4, cudaMemcpyHostToDevice, s));
+  if (w->router_bias) {
+    C_CUDA(cudaMemcpyAsync(L->router_b, w->router_bias, (size_t)NT * 4, cudaMemcpyHostToDevice, s));
+    if (cfg->shared_gate) C_CUDA(cudaMemsetAsync(L->router_b + NT, 0, sizeof(float), s));   // the gate row has no bias
+  }
   if (Is)
     for (int m = 0; m < 3; ++m)
       C_CUDA(cudaMemcpyAsync(L->shared_w[m], w->shared_w[m], (size_t)Is * H * 2, cudaMemcpyHostToDevice, s));
@@ -726,11 +910,14 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   }
   C_CUDA(cudaEventCreateWithFlags(&L->ev_counts, cudaEventDisableTiming));
   C_CUDA(cudaEventCreateWithFlags(&L->ev_fwd_done, cudaEventDisableTiming));
+  C_CUDA(cudaEventCreateWithFlags(&L->ev_prefetch, cudaEventDisableTiming));
   L->slot_of.assign(E, -1);
+  L->expert_of_slot.assign(cfg->n_slots, -1);
+  L->last_use.assign(E, 0);
   for (int e = 0; e < E; ++e) L->h_ptr[e] = nullptr;
   L->st.expert_bytes = bytes;
   L->st.pinned_bytes = bytes * E;
-  size_t dev_total = (size_t)E * H * 4 + (size_t)3 * Is * H * 2 + bytes * (cfg->n_slots + L->n_staging) +
+  size_t dev_total = (size_t)NR * H * 4 + (size_t)3 * Is * H * 2 + bytes * (cfg->n_slots + L->n_staging) +
                      scratch_bytes(cfg) + a4_scratch_bytes(cfg) + tc_scratch_bytes(cfg);
   L->st.device_bytes = dev_total;
   *out = L;
@@ -778,6 +965,9 @@ moe_status_t moe_set_slot_table(moe_layer_t L, const int32_t *table, void *strea
   CUDA_TRY(cudaMemcpyAsync(L->loc_resident, L->h_loc, sizeof(int) * E, cudaMemcpyHostToDevice, st));
   CUDA_TRY(cudaStreamSynchronize(st));
   for (int e = 0; e < E; ++e) L->slot_of[e] = table[e];
+  std::fill(L->expert_of_slot.begin(), L->expert_of_slot.end(), -1);
+  for (int e = 0; e < E; ++e)
+    if (table[e] >= 0) L->expert_of_slot[table[e]] = e;
   L->n_resident = n;
   L->table_version += 1;
   return MOE_OK;
@@ -842,8 +1032,7 @@ static moe_status_t run_experts(moe_layer *L, const int *locs, int nt, int grid_
 
 // Tensor-core EXACT pass over the experts present in `locs`: gate/up + SwiGLU
 // -> h pieces, down + gate -> O' and the ordered combine into y.
-static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int grid_tiles, float *y,
-                                   cudaStream_t s) {
+static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int grid_tiles, cudaStream_t s) {
   const moe_config_t &c = L->cfg;
   TcArgs a{};
   a.maps = L->tcmaps;
@@ -890,6 +1079,53 @@ static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int 
   a.early = (a.early && nbox <= 16) ? 1 : 0;
   StageTimer t4(L, 4, s);
   launch_expert_tc(MODE_DOWN, nbox, a, grid_tiles, s);
+  CUDA_TRY(cudaGetLastError());
+  t4.launched(1);
+  t4.end();
+  return MOE_OK;
+}
+
+// NVFP4 EXACT pass on the tensor core over the experts present in `locs`
+// (tiles of nb tokens): gate/up + SwiGLU -> h (bf16, padded-row order), then
+// down + gate -> O'; the ordered combine follows after the last pass.
+static moe_status_t run_experts_dq(moe_layer *L, const int *locs, const void *x, int nb, int grid_tiles,
+                                   cudaStream_t s) {
+  const moe_config_t &c = L->cfg;
+  DqArgs a{};
+  a.maps = L->dqmaps;
+  a.loc = locs;
+  a.slots = L->slots;
+  a.staging = L->staging;
+  a.blob_bytes = L->L.bytes;
+  a.L = L->L;
+  a.tiles = L->tiles;
+  a.n_tiles = L->n_tiles;
+  a.prow_token = L->prow_token;
+  a.prow_pair = L->prow_pair;
+  a.gates = L->gates;
+  a.err = L->d_err;
+  a.K = c.hidden;
+  a.rows = c.inter;
+  a.n_rowblocks = c.inter / 128;
+  a.act = reinterpret_cast<const uint16_t *>(x);
+  a.h_out = L->hbuf;
+  a.work_ctr = L->dq_work;
+  a.wfmt = c.fmt == MOE_FMT_INT4G128 ? DQ_I4 : (c.fmt == MOE_FMT_FP8B128 ? DQ_F8 : DQ_NV);
+  a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
+  StageTimer t3(L, 3, s);
+  launch_expert_dq(MODE_GATEUP, nb, a, s);
+  CUDA_TRY(cudaGetLastError());
+  t3.launched(1);
+  t3.end();
+  a.K = c.inter;
+  a.rows = c.hidden;
+  a.n_rowblocks = c.hidden / 256;
+  a.act = L->hbuf;
+  a.o_out = L->oprime;
+  a.work_ctr = L->dq_work + 1;
+  a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
+  StageTimer t4(L, 4, s);
+  launch_expert_dq(MODE_DOWN, nb, a, s);
   CUDA_TRY(cudaGetLastError());
   t4.launched(1);
   t4.end();
@@ -966,7 +1202,7 @@ static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles
   return MOE_OK;
 }
 
-moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void *stream,
+moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void *stream,
                          const moe_routing_t *dbg) {
   if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
   const moe_config_t &c = L->cfg;
@@ -993,24 +1229,39 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   // the batch is decode-sized, else 56-token tiles (112 piece rows, two
   // accumulator buffers so that the epilogue overlaps the next item's MMAs)
   const int nbox = (tc && P <= 12 * act_est) ? 16 : 112;
-  const int ts = a4 ? 128 : (tc ? nbox / 2 : 8 * nt);
+  // NVFP4 EXACT: prefill-sized batches (x 16-byte aligned for the 16-byte
+  // activation copies) on the tensor core with tiles of 64 or 128 tokens;
+  // decode-sized batches on the register-decode kernels
+  const bool x16 = (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
+  if (dq_only(&c) && !x16) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned for INT4 / FP8 experts");
+  const bool dq = L->nv && (dq_only(&c) || P > 12 * act_est) && x16;
+  const int nb_dq = avg >= 96 ? 128 : 64;
+  const int ts = a4 ? 128 : (tc ? nbox / 2 : (dq ? nb_dq : 8 * nt));
   const int grid_tiles = P / ts + act_est + 1;
+  // routing targets (experts, then sinks) and logit rows (+ the shared-expert gate)
+  const int NT = n_targets(&c), NR = n_logit_rows(&c);
+  // the register-decode kernels fuse the ordered combine into their down pass
+  // for fp32 outputs of layers without sinks or a shared-expert gate; every
+  // other case runs the combine kernel after the last pass
+  const bool sep_combine = a4 || tc || dq || c.n_sinks > 0 || c.shared_gate || c.out_dtype == MOE_OUT_BF16;
+  float *y_fused = sep_combine ? nullptr : static_cast<float *>(y);
 
   StageTimer t7(L, 7, s);
   RouterArgs ra{};
   ra.x = reinterpret_cast<const uint16_t *>(x);
-  ra.T = T; ra.H = H; ra.E = E; ra.k = k;
+  ra.T = T; ra.H = H; ra.E = NR; ra.k = k;
+  ra.E_t = NT; ra.scoring = c.scoring; ra.renorm = c.renormalize;
   ra.w = L->router_w; ra.bias = L->router_b;
   ra.logits = L->logits; ra.ids = L->ids; ra.gates = L->gates;
   ra.xf16 = tc ? nullptr : L->xf16; ra.xs = L->xs; ra.counter = L->router_counter;
   PermArgs pa{};
-  pa.ids = L->ids; pa.n_pairs = P; pa.E = E; pa.k = k; pa.tile_tokens = ts;
+  pa.ids = L->ids; pa.n_pairs = P; pa.E = NT; pa.n_real = E; pa.k = k; pa.tile_tokens = ts;
   pa.counts = L->counts; pa.offsets = L->offsets; pa.perm = L->perm; pa.inv = L->inv;
   pa.tiles = L->tiles; pa.n_tiles = L->n_tiles; pa.prow_token = L->prow_token;
   pa.prow_pair = L->prow_pair; pa.active = L->active;
   pa.pad = a4 ? 128 : 8;
   pa.n_prows = a4 ? L->n_prows : nullptr;
-  pa.work_ctr = tc ? L->tc_work : nullptr;
+  pa.work_ctr = tc ? L->tc_work : (dq ? L->dq_work : nullptr);
   pa.tile_done = tc ? L->tile_done : nullptr;
   // decode-sized batches: the router's last CTA also runs the permutation
   const bool fuse_perm = P <= 2048;
@@ -1021,13 +1272,14 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   // permutation as their own kernels (the register-decode kernels of NVFP4
   // EXACT layers need the router's f16 copy of x, so they keep the router)
   const bool big_batch = T >= kDenseTcMinTokens && (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
-  const bool router_gemm = big_batch && (tc || a4);
+  const bool router_gemm = big_batch && (tc || a4 || dq);
   StageTimer t0(L, 0, s);
   if (router_gemm) {
-    const int sp = router_gemm_splits(T, H, E, kRouterPartFloats);
-    launch_router_gemm(ra.x, L->router_w, L->router_b, T, H, E, L->logits, L->router_parts, sp, s);
+    const int sp = router_gemm_splits(T, H, NR, kRouterPartFloats);
+    launch_router_gemm(ra.x, L->router_w, L->router_b, T, H, NR, L->logits, L->router_parts, sp, s);
     CUDA_TRY(cudaGetLastError());
-    launch_topk(L->logits, L->router_parts, sp, L->router_b, T, E, k, L->ids, L->gates, s);
+    launch_topk(L->logits, L->router_parts, sp, L->router_b, T, NR, NT, k, c.scoring, c.renormalize, L->ids,
+                L->gates, s);
     t0.launched(1);
   } else {
     launch_router(ra, s);
@@ -1044,16 +1296,25 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   }
 
   if (dbg) {
-    if (dbg->logits) CUDA_TRY(cudaMemcpyAsync(dbg->logits, L->logits, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s));
+    // logits of the NT routing targets (the rows' stride is NR)
+    if (dbg->logits)
+      CUDA_TRY(cudaMemcpy2DAsync(dbg->logits, (size_t)NT * 4, L->logits, (size_t)NR * 4, (size_t)NT * 4, T,
+                                 cudaMemcpyDeviceToDevice, s));
     if (dbg->ids) CUDA_TRY(cudaMemcpyAsync(dbg->ids, L->ids, (size_t)P * 4, cudaMemcpyDeviceToDevice, s));
     if (dbg->gates) CUDA_TRY(cudaMemcpyAsync(dbg->gates, L->gates, (size_t)P * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->counts) CUDA_TRY(cudaMemcpyAsync(dbg->counts, L->counts, (size_t)E * 4, cudaMemcpyDeviceToDevice, s));
-    if (dbg->offsets) CUDA_TRY(cudaMemcpyAsync(dbg->offsets, L->offsets, (size_t)(E + 1) * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->counts) CUDA_TRY(cudaMemcpyAsync(dbg->counts, L->counts, (size_t)NT * 4, cudaMemcpyDeviceToDevice, s));
+    if (dbg->offsets)
+      CUDA_TRY(cudaMemcpyAsync(dbg->offsets, L->offsets, (size_t)(NT + 1) * 4, cudaMemcpyDeviceToDevice, s));
     if (dbg->perm) CUDA_TRY(cudaMemcpyAsync(dbg->perm, L->perm, (size_t)P * 4, cudaMemcpyDeviceToDevice, s));
     if (dbg->inv) CUDA_TRY(cudaMemcpyAsync(dbg->inv, L->inv, (size_t)P * 4, cudaMemcpyDeviceToDevice, s));
   }
 
   const bool resident = L->n_resident == E;
+  // slots filled by moe_prefetch: the expert passes wait for those copies
+  if (L->prefetch_pending) {
+    CUDA_TRY(cudaStreamWaitEvent(s, L->ev_prefetch, 0));
+    L->prefetch_pending = false;
+  }
   if (!resident) {
     CUDA_TRY(cudaMemcpyAsync(L->h_counts, L->counts, (size_t)E * 4, cudaMemcpyDeviceToHost, s));
     CUDA_TRY(cudaEventRecord(L->ev_counts, s));
@@ -1146,10 +1407,12 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
   const int cs_gu = pick_split(act_est * (I / 128), H / 128);
   const int cs_dn = pick_split(act_est * (H / 256), I / 128);
   int waves = 0, misses_n = 0;
+  bool admit_table_pending = false;
   if (resident) {
     if (a4) ST_TRY(run_experts_a4(L, L->loc_resident, grid_tiles, s));
-    else if (tc) ST_TRY(run_experts_tc(L, L->loc_resident, nbox, grid_tiles, y, s));
-    else ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
+    else if (tc) ST_TRY(run_experts_tc(L, L->loc_resident, nbox, grid_tiles, s));
+    else if (dq) ST_TRY(run_experts_dq(L, L->loc_resident, x, nb_dq, grid_tiles, s));
+    else ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y_fused, s));
   } else {
     CUDA_TRY(cudaEventSynchronize(L->ev_counts));
     std::vector<int> misses;
@@ -1163,10 +1426,16 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
     L->st.last_active = act;
     misses_n = (int)misses.size();
     const int NS = L->n_staging;
+    const uint64_t fwd_index = L->st.forwards + 1;
+    for (int e = 0; e < E; ++e)
+      if (L->h_counts[e] > 0) L->last_use[e] = fwd_index;
+    // CACHE / HYBRID: which misses this forward admits, and into which slots
+    const std::vector<int> admit_slot = plan_admission(L, misses);
     if (misses.empty()) {
       if (a4) ST_TRY(run_experts_a4(L, L->loc_resident, grid_tiles, s));
-      else if (tc) ST_TRY(run_experts_tc(L, L->loc_resident, nbox, grid_tiles, y, s));
-      else ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y, s));
+      else if (tc) ST_TRY(run_experts_tc(L, L->loc_resident, nbox, grid_tiles, s));
+      else if (dq) ST_TRY(run_experts_dq(L, L->loc_resident, x, nb_dq, grid_tiles, s));
+      else ST_TRY(run_experts(L, L->loc_resident, nt, grid_tiles, cs_gu, cs_dn, y_fused, s));
     } else {
       const bool one = misses_n <= NS;
       const int wave_sz = one ? NS : NS / 2;
@@ -1184,7 +1453,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
         if (!one && w >= 2) CUDA_TRY(cudaStreamWaitEvent(L->side, L->ev_done[half], 0));
         LocUpdate u{};
         u.E = E;
-        u.work_ctr = tc ? L->tc_work : nullptr;
+        u.work_ctr = tc ? L->tc_work : (dq ? L->dq_work : nullptr);
         u.keep_resident = (w == 0);
         const int b0 = w * wave_sz, b1 = std::min(misses_n, b0 + wave_sz);
         for (int i = b0; i < b1; ++i) {
@@ -1203,8 +1472,17 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
         t6.launched(1);
         t6.end();
         if (a4) ST_TRY(run_experts_a4(L, L->loc_pass, grid_tiles, s));
-        else if (tc) ST_TRY(run_experts_tc(L, L->loc_pass, nbox, grid_tiles, y, s));
-        else ST_TRY(run_experts(L, L->loc_pass, nt, grid_tiles, cs_gu, cs_dn, y, s));
+        else if (tc) ST_TRY(run_experts_tc(L, L->loc_pass, nbox, grid_tiles, s));
+        else if (dq) ST_TRY(run_experts_dq(L, L->loc_pass, x, nb_dq, grid_tiles, s));
+        else ST_TRY(run_experts(L, L->loc_pass, nt, grid_tiles, cs_gu, cs_dn, y_fused, s));
+        // admissions: the staged copy of an admitted miss goes into its slot
+        // while the staging buffer still holds it (a slot whose expert this
+        // forward does not use, so no kernel of this forward reads it)
+        for (int i = b0; i < b1; ++i)
+          if (admit_slot[i] >= 0)
+            CUDA_TRY(cudaMemcpyAsync(L->slots + (size_t)admit_slot[i] * bytes,
+                                     L->staging + (size_t)(base + (i - b0)) * bytes, bytes,
+                                     cudaMemcpyDeviceToDevice, s));
         if (!one) CUDA_TRY(cudaEventRecord(L->ev_done[half], s));
       }
       CUDA_TRY(cudaEventRecord(L->ev_fwd_done, s));
@@ -1212,36 +1490,58 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, float *y, void
       waves = nw;
       L->st.misses += misses_n;
       L->st.bytes_staged += (uint64_t)misses_n * bytes;
+      // the admitted experts are resident from the next forward on: the new
+      // table reaches the device behind this forward's kernels on the stream
+      int admitted = 0;
+      for (int i = 0; i < misses_n; ++i) {
+        const int v = admit_slot[i];
+        if (v < 0) continue;
+        const int old = L->expert_of_slot[v];
+        if (old >= 0) L->slot_of[old] = -1;
+        L->slot_of[misses[i]] = v;
+        L->expert_of_slot[v] = misses[i];
+        ++admitted;
+      }
+      if (admitted) {
+        L->st.admitted += admitted;
+        admit_table_pending = true;
+      }
     }
   }
 
-  // register-decode EXACT kernels: the ordered combine runs inside the routed
-  // down pass (last arrival per token); tensor-core EXACT and A4: a separate
-  // ordered combine after the last pass.
-  if (a4 || tc) {
+  // the ordered combine: inside the register-decode down pass (last arrival
+  // per token) when y_fused is set, else this kernel after the last pass
+  if (sep_combine) {
     CombineArgs ca{};
     ca.oprime = L->oprime;
     ca.shared = Is ? L->sh_s : nullptr;
     ca.y = y;
     ca.T = T; ca.H = H; ca.k = k;
+    ca.out_bf16 = c.out_dtype == MOE_OUT_BF16 ? 1 : 0;
+    ca.ids = c.n_sinks > 0 ? L->ids : nullptr;
+    ca.n_real = E;
+    ca.sg_logits = c.shared_gate ? L->logits : nullptr;
+    ca.ld = NR;
+    ca.sg_col = NT;
     StageTimer t5(L, 5, s);
     launch_combine(ca, s);
     CUDA_TRY(cudaGetLastError());
     t5.launched(1);
     t5.end();
   }
+  if (admit_table_pending) ST_TRY(push_table(L, s));
   t7.end();
   if (L->prof) L->prof_acc.forwards += 1;
 
   L->st.forwards += 1;
   L->st.last_misses = misses_n;
   L->st.last_waves = waves;
-  L->st.last_path = a4 ? 1 : (tc ? 2 : 0);
+  L->st.last_path = a4 ? 1 : (tc ? 2 : (dq ? 3 : 0));
   if (resident) L->st.last_active = -1;
   return MOE_OK;
 }
 
-moe_status_t moe_forward_host(moe_layer_t L, const uint16_t *x_host, int32_t T, float *y_host,
+moe_status_t moe_forward_host(moe_layer_t L, const uint16_t *x_host, int32_t T, void *y_host,
                               void *stream) {
   if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
   if (T < 0 || T > L->cfg.max_tokens) return fail(MOE_ERR_INVALID_ARG, "T out of range [0, max_tokens]");
@@ -1252,7 +1552,8 @@ moe_status_t moe_forward_host(moe_layer_t L, const uint16_t *x_host, int32_t T, 
   const size_t H = L->cfg.hidden;
   CUDA_TRY(cudaMemcpyAsync(L->xin, x_host, (size_t)T * H * 2, cudaMemcpyHostToDevice, s));
   ST_TRY(moe_forward(L, L->xin, T, L->yout, stream, nullptr));
-  CUDA_TRY(cudaMemcpyAsync(y_host, L->yout, (size_t)T * H * 4, cudaMemcpyDeviceToHost, s));
+  const size_t ybytes = L->cfg.out_dtype == MOE_OUT_BF16 ? 2 : 4;
+  CUDA_TRY(cudaMemcpyAsync(y_host, L->yout, (size_t)T * H * ybytes, cudaMemcpyDeviceToHost, s));
   CUDA_TRY(cudaStreamSynchronize(s));
   return MOE_OK;
 }
@@ -1271,7 +1572,7 @@ struct moe_graph {
   uint64_t launches = 0;             // library kernels per replay
 };
 
-moe_status_t moe_graph_capture(moe_layer_t L, const void *x, int32_t T, float *y, void *stream,
+moe_status_t moe_graph_capture(moe_layer_t L, const void *x, int32_t T, void *y, void *stream,
                                moe_graph_t *out) {
   if (!L || !out) return fail(MOE_ERR_INVALID_ARG, "layer or out is NULL");
   *out = nullptr;
@@ -1345,6 +1646,69 @@ moe_status_t moe_graph_destroy(moe_graph_t G) {
   if (G->exec) cudaGraphExecDestroy(G->exec);
   if (G->graph) cudaGraphDestroy(G->graph);
   delete G;
+  return MOE_OK;
+}
+
+moe_status_t moe_set_policy(moe_layer_t L, int32_t policy, int32_t n_pinned, void *stream) {
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  if (policy < MOE_POLICY_STATIC || policy > MOE_POLICY_HYBRID) return fail(MOE_ERR_INVALID_ARG, "unknown policy");
+  const int S = L->cfg.n_slots;
+  if (policy == MOE_POLICY_HYBRID && (n_pinned < 0 || n_pinned > S))
+    return fail(MOE_ERR_INVALID_ARG, "n_pinned must be in 0..n_slots");
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  cudaStream_t st = (cudaStream_t)stream;
+  CUDA_TRY(cudaStreamSynchronize(st));
+  CUDA_TRY(cudaStreamSynchronize(L->side));
+  if (policy == MOE_POLICY_NONE) {
+    std::vector<int32_t> none(L->cfg.n_experts, -1);
+    ST_TRY(moe_set_slot_table(L, none.data(), stream));
+  }
+  L->policy = policy;
+  L->n_pinned = policy == MOE_POLICY_HYBRID ? n_pinned : 0;
+  L->st.policy = policy;
+  return MOE_OK;
+}
+
+moe_status_t moe_prefetch(moe_layer_t L, const int32_t *experts, int32_t n, void *stream) {
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  if (L->policy != MOE_POLICY_CACHE && L->policy != MOE_POLICY_HYBRID)
+    return fail(MOE_ERR_INVALID_ARG, "moe_prefetch needs the CACHE or HYBRID policy");
+  if (n < 0 || (n > 0 && !experts)) return fail(MOE_ERR_INVALID_ARG, "bad expert list");
+  const int E = L->cfg.n_experts;
+  for (int i = 0; i < n; ++i)
+    if (experts[i] < 0 || experts[i] >= E) return fail(MOE_ERR_INVALID_ARG, "expert id out of range");
+  if (n == 0) return MOE_OK;
+  CUDA_TRY(cudaSetDevice(L->cfg.device));
+  cudaStream_t st = (cudaStream_t)stream;
+  // listed experts are not evicted for one another
+  std::vector<char> busy(E, 0);
+  for (int i = 0; i < n; ++i) busy[experts[i]] = 1;
+  const std::vector<int> cand = evictable_slots(L, busy);
+  // the copies start after the work queued on `stream` (a forward in flight
+  // may still read the slots they overwrite) and run on the side stream
+  CUDA_TRY(cudaEventRecord(L->ev_prefetch, st));
+  CUDA_TRY(cudaStreamWaitEvent(L->side, L->ev_prefetch, 0));
+  const size_t bytes = L->L.bytes;
+  size_t c = 0;
+  int copied = 0;
+  for (int i = 0; i < n && c < cand.size(); ++i) {
+    const int e = experts[i];
+    if (L->slot_of[e] >= 0) continue;                // resident already (or listed twice)
+    const int v = cand[c++];
+    CUDA_TRY(cudaMemcpyAsync(L->slots + (size_t)v * bytes, L->store + (size_t)e * bytes, bytes,
+                             cudaMemcpyHostToDevice, L->side));
+    const int old = L->expert_of_slot[v];
+    if (old >= 0) L->slot_of[old] = -1;
+    L->slot_of[e] = v;
+    L->expert_of_slot[v] = e;
+    ++copied;
+  }
+  if (copied) {
+    ST_TRY(push_table(L, L->side));
+    CUDA_TRY(cudaEventRecord(L->ev_prefetch, L->side));
+    L->prefetch_pending = true;
+    L->st.prefetched += copied;
+  }
   return MOE_OK;
 }
 

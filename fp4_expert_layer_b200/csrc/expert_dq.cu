@@ -1,0 +1,625 @@
+// expert_dq.cu -- EXACT numerics for NVFP4 experts on the tcgen05 tensor core at
+// prefill-sized batches.
+//
+// The pages' engines decode E2M1 to BF16 in registers for mma.sync
+// ("ro99/strata", description of the SM86 kernel).  On sm_100a the
+// block-scaled MMA kinds cannot take an NVFP4 weight against a 16-bit
+// activation: kind::mxf4nvf4 (the one that reads E4M3 block scales) wants
+// FP4 on both sides, and kind::mxf8f6f4 takes only UE8M0 per-32 scales.  So
+// each weight tile is decoded ONCE per token tile into shared memory as bf16
+// and multiplied with tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM):
+//   * an E2M1 value (at most 2 significant bits) times its E4M3 block scale
+//     (4 significant bits, 2^-9 .. 448) has at most 6 significant bits and lies
+//     in [2^-10, 2688]: exact in f16 and in bf16;
+//   * the per-tensor fp32 scale G multiplies the fp32 accumulator in the
+//     epilogue;
+//   * the gate/up activations are the bf16 x rows themselves (exact), the down
+//     activations are h = silu(G_g a) * (G_u u) rounded to bf16.
+// The decode cost of a weight tile is shared by the up to NB tokens of a tile.
+//
+// Kernel expert_dq_kernel<MODE, NB>: persistent, one CTA per SM, work items
+// (tile of up to NB tokens, 256 weight rows: 128 gate + the same 128 up rows,
+// or 256 down rows) taken from a counter in index order.  Roles:
+//   warp 0       producer: per 64-element K slab, one TMA box of the packed
+//                codes (32 bytes x 128 or 256 rows) per matrix and the
+//                512-byte E4M3 scale-factor blocks by bulk copy, into a ring
+//                of raw stages;
+//   warp 1       MMA issuer (one lane): M = 128, N = tokens rounded up to 16,
+//                K = 16, two accumulators (gate and up, or the two 128-row
+//                halves of down) per item, double-buffered across items;
+//   warps 2..5   epilogue: TMEM -> SwiGLU -> h (bf16, padded-row order), or
+//                G_d * gate * acc -> O' (fp32, pair order);
+//   warps 6..9   decoders: raw stage -> bf16 weight tile in the 128-byte
+//                swizzled K-major layout the MMA descriptor reads;
+//   warps 10..11 activation loaders: the tile's bf16 rows of this K slab by
+//                16-byte cp.async (x rows gathered through the padded-row ->
+//                token map for gate/up; h rows for down).
+// Every mbarrier wait is bounded (error word, then the kernel runs out).
+#include "device_utils.cuh"
+#include "launch.cuh"
+#include "moe_internal.h"
+#include "tcgen05.cuh"
+#include "tma.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kDqThreads = 384;
+constexpr int kDqDecoders = 128;   // warps 6..9
+constexpr int kDqLoaders = 64;     // warps 10..11
+constexpr int kDqSched = 8;
+// arrivals that free a hand-over slot: MMA lane, 4 epilogue warps, 4 decoder warps, 2 loader warps
+constexpr int kDqSchedReaders = 11;
+// Raw stage of one 64-element K slab of 256 weight rows, per weight format:
+//   DQ_NV  NVFP4: codes 256 rows x 32 bytes, then two 512-byte E4M3 scale blocks
+//          (rows 0..127, 128..255; 4 scales per row);
+//   DQ_I4  INT4 group-128: codes 256 rows x 32 bytes, then two 256-byte bf16
+//          scale blocks (one scale per row: the group of 128 holding the slab);
+//   DQ_F8  FP8 E4M3 block-128: codes 256 rows x 64 bytes (the fp32 block
+//          scales, one per 128 rows, are read from the blob by the decoders).
+template <int F>
+struct DqRaw;
+template <>
+struct DqRaw<DQ_NV> {
+  static constexpr int BYTES = 256 * 32 + 2 * 512;
+};
+template <>
+struct DqRaw<DQ_I4> {
+  static constexpr int BYTES = 256 * 32 + 2 * 256;
+};
+template <>
+struct DqRaw<DQ_F8> {
+  static constexpr int BYTES = 256 * 64;
+};
+
+template <int NB, int F>
+struct DqGeom {
+  static constexpr int A_BYTES = 2 * 128 * 128;           // two 128-row x 64-element bf16 tiles
+  static constexpr int B_OFF = A_BYTES;
+  static constexpr int B_BYTES = NB * 128;                 // NB token rows x 64 bf16
+  static constexpr int OP_STAGE = A_BYTES + B_BYTES;       // multiple of 1024
+  static constexpr int OP_STAGES = NB >= 128 ? 3 : 4;
+  static constexpr int RAW_OFF = OP_STAGES * OP_STAGE;
+  static constexpr int RAW_BYTES = DqRaw<F>::BYTES;
+  // raw stages in what is left of 227 KB (1 KB alignment slack, 4 KB for the static part)
+  static constexpr int RAW_FIT = (227 * 1024 - 1024 - 4096 - RAW_OFF) / RAW_BYTES;
+  static constexpr int RAW_STAGES = RAW_FIT < 8 ? RAW_FIT : 8;
+  static constexpr int NBUF = 2;
+  static constexpr int COLS = NBUF * 2 * NB;
+  static constexpr int TMEM_COLS = COLS <= 128 ? 128 : (COLS <= 256 ? 256 : 512);
+  static constexpr size_t SMEM = (size_t)RAW_OFF + (size_t)RAW_STAGES * RAW_BYTES + 1024;
+  static_assert(OP_STAGE % 1024 == 0, "operand stages must keep the 1024-byte swizzle alignment");
+  static_assert(RAW_BYTES % 512 == 0, "raw stages keep 128-byte TMA destinations");
+  static_assert(RAW_STAGES >= 3, "raw ring depth");
+  static_assert(COLS <= 512, "TMEM budget");
+  static_assert(SMEM <= 227 * 1024, "shared-memory budget");
+};
+
+// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, K-major.
+__device__ __forceinline__ uint32_t idesc_bf16_dq(int M, int N) {
+  uint32_t d = 0;
+  d |= 1u << 4;    // C: F32
+  d |= 1u << 7;    // A: BF16
+  d |= 1u << 10;   // B: BF16
+  d |= (uint32_t)(N >> 3) << 17;
+  d |= (uint32_t)(M >> 4) << 24;
+  return d;
+}
+
+__device__ __forceinline__ void umma_bf16_dq(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void cp_async16_dq(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_dq(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_dq() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ TileInfo load_tile_dq(const TileInfo *p) {
+  const int4 v = __ldcg(reinterpret_cast<const int4 *>(p));
+  return TileInfo{v.x, v.y, v.z, v.w};
+}
+
+// f16x2 -> bf16x2 for values exactly representable in bf16 (no rounding happens).
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
+  const float lo = __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
+  const float hi = __half2float(__ushort_as_half((unsigned short)(h >> 16)));
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Eight E2M1 codes (one 32-bit word, element 2i in the low nibble of byte i)
+// times one E4M3 scale (f16x2 with the scale in both halves) -> eight bf16.
+__device__ __forceinline__ uint4 decode8(uint32_t w, uint32_t sc2) {
+  uint32_t f[4];
+  e2m1x8_to_f16x2(w, f);
+  uint4 o;
+  o.x = f16x2_to_bf16x2(hmul2_u32(f[0], sc2));
+  o.y = f16x2_to_bf16x2(hmul2_u32(f[1], sc2));
+  o.z = f16x2_to_bf16x2(hmul2_u32(f[2], sc2));
+  o.w = f16x2_to_bf16x2(hmul2_u32(f[3], sc2));
+  return o;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// Eight INT4 codes (two's complement nibbles, element 2i in the low nibble of
+// byte i) times one bf16 scale (both halves of sc2) -> eight bf16, each the
+// product q * s rounded to nearest even.  q + 8 (0..15) is placed in the
+// mantissa of bf16 128.0 (0x4300), so that the bf16 value is 136 + q exactly;
+// one fma removes the 136 (exact), the next multiplies by the scale (one
+// rounding).
+__device__ __forceinline__ uint4 decode8_int4(uint32_t w, uint32_t sc2) {
+  const uint32_t x = w ^ 0x88888888u;                      // q + 8 per nibble
+  const uint32_t one2 = 0x3F803F80u, m136 = 0xC308C308u, nzero = 0x80008000u;   // 1.0, -136.0, -0.0
+  uint32_t o[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t byte = (x >> (8 * b)) & 0xFFu;
+    const uint32_t bits = 0x43004300u | (byte & 0xFu) | ((byte >> 4) << 16);
+    const uint32_t q2 = bf16x2_fma(bits, one2, m136);
+    o[b] = bf16x2_fma(q2, sc2, nzero);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Eight E4M3 codes (two 32-bit words, element i in byte i) times an fp32
+// block scale -> eight bf16: each code is exact in f16 and in fp32, the
+// product is rounded to fp32 and then to bf16 (nearest even).
+__device__ __forceinline__ uint4 decode8_fp8(uint32_t w0, uint32_t w1, float s) {
+  const uint32_t ws[2] = {w0, w1};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)((ws[i >> 1] >> (16 * (i & 1))) & 0xFFFFu));
+    const float lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))) * s;
+    const float hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16))) * s;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[i]) : "f"(hi), "f"(lo));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+}  // namespace
+
+template <int MODE, int NB, int F>
+__global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_constant__ DqArgs a) {
+  using Geo = DqGeom<NB, F>;
+  constexpr int kRawBytes = Geo::RAW_BYTES;
+  constexpr int SO = Geo::OP_STAGES;
+  constexpr int SR = Geo::RAW_STAGES;
+  constexpr int NBUF = Geo::NBUF;
+  extern __shared__ __align__(1024) uint8_t dq_smem_raw[];
+  __shared__ __align__(8) uint64_t raw_full[SR];    // packed codes + scales landed (TMA / bulk)
+  __shared__ __align__(8) uint64_t raw_empty[SR];   // decoders done with a raw stage
+  __shared__ __align__(8) uint64_t op_full[SO];     // bf16 weights decoded + activation rows landed
+  __shared__ __align__(8) uint64_t op_empty[SO];    // MMAs done with an operand stage
+  __shared__ __align__(8) uint64_t accf_bar[NBUF];
+  __shared__ __align__(8) uint64_t acce_bar[NBUF];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ __align__(8) uint64_t sched_full[kDqSched];
+  __shared__ __align__(8) uint64_t sched_empty[kDqSched];
+  __shared__ int sched_item[kDqSched];
+  __shared__ TileInfo sched_ti[kDqSched];
+  __shared__ int sched_loc[kDqSched];
+  __shared__ int tok_pair[NB];
+  __shared__ float tok_gate[NB];
+
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dq_smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = a.K;
+  const int nslab = K / 64;
+  const int ipt = a.n_rowblocks;
+  const int nsf = K / 16;                              // E4M3 scale columns per weight row
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SR; ++s) {
+      mbar_init(smem_u32(&raw_full[s]), 1);
+      mbar_init(smem_u32(&raw_empty[s]), kDqDecoders / 32);
+    }
+    for (int s = 0; s < SO; ++s) {
+      mbar_init(smem_u32(&op_full[s]), kDqLoaders + kDqDecoders / 32);
+      mbar_init(smem_u32(&op_empty[s]), 1);
+    }
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(smem_u32(&accf_bar[b]), 1);
+      mbar_init(smem_u32(&acce_bar[b]), 4);
+    }
+    for (int q = 0; q < kDqSched; ++q) {
+      mbar_init(smem_u32(&sched_full[q]), 1);
+      mbar_init(smem_u32(&sched_empty[q]), kDqSchedReaders);
+    }
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_base_s), Geo::TMEM_COLS);
+    tmem_relinquish();
+  }
+  wait_prior_grid();                                   // routing, h and locations come from earlier kernels
+  const int n_items = __ldcg(a.n_tiles) * ipt;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+
+  if (warp == 0) {
+    // ---------------- producer (one lane): work items and the raw weight stream
+    if (lane == 0) {
+      int r = 0, issued = 0;
+      uint32_t ph = 0;
+      int q = 0;
+      uint32_t qph = 0;
+      bool failed = false;
+      for (int j = 0; !failed; ++j) {
+        const int item = atomicAdd(a.work_ctr, 1);
+        TileInfo ti{};
+        int loc = kLocAbsent;
+        if (item < n_items) {
+          ti = load_tile_dq(a.tiles + item / ipt);
+          loc = __ldcg(a.loc + ti.expert);
+        }
+        if (j >= kDqSched && !mbar_wait(smem_u32(&sched_empty[q]), qph ^ 1u, a.err, 58)) { failed = true; break; }
+        const bool done = item >= n_items;
+        sched_item[q] = done ? -1 : item;
+        sched_ti[q] = ti;
+        sched_loc[q] = loc;
+        mbar_arrive(smem_u32(&sched_full[q]));
+        if (++q == kDqSched) { q = 0; qph ^= 1u; }
+        if (done) break;
+        if (loc == kLocAbsent) continue;
+        const int rb = item % ipt;
+        const bool in_slot = loc >= 0;
+        const int bidx = in_slot ? loc : (-2 - loc);
+        const uint8_t *blob = (in_slot ? a.slots : a.staging) + (size_t)bidx * a.blob_bytes;
+        const CUtensorMap *maps = in_slot ? a.maps.slot : a.maps.stage;
+        for (int slab = 0; slab < nslab; ++slab) {
+          if (issued >= SR && !mbar_wait(smem_u32(&raw_empty[r]), ph ^ 1u, a.err, 52)) { failed = true; break; }
+          const uint32_t bar = smem_u32(&raw_full[r]);
+          const uint32_t st = smem_u32(smem + Geo::RAW_OFF + (size_t)r * kRawBytes);
+          mbar_arrive_expect_tx(bar, (uint32_t)kRawBytes);
+          // codes of the slab (TMA boxes of 32 bytes = 64 nibbles, or 64
+          // bytes = 64 E4M3), then the scales the decoders need
+          constexpr int cw = F == DQ_F8 ? 64 : 32;              // code bytes per row per slab
+          if constexpr (MODE == MODE_GATEUP) {
+            tma_load_3d(st, &maps[0], bar, slab * cw, rb * 128, bidx);
+            tma_load_3d(st + 128 * cw, &maps[1], bar, slab * cw, rb * 128, bidx);
+          } else {
+            tma_load_3d(st, &maps[2], bar, slab * cw, rb * 256, bidx);
+          }
+          if constexpr (F == DQ_NV) {
+            const int m0 = MODE == MODE_GATEUP ? 0 : 2, m1 = MODE == MODE_GATEUP ? 1 : 2;
+            const int r0 = MODE == MODE_GATEUP ? rb * 128 : rb * 256;
+            const int r1 = MODE == MODE_GATEUP ? rb * 128 : rb * 256 + 128;
+            bulk_load(st + 8192, blob + a.L.scales[m0] + sf_offset(nsf, r0, slab * 4), 512, bar);
+            bulk_load(st + 8704, blob + a.L.scales[m1] + sf_offset(nsf, r1, slab * 4), 512, bar);
+          } else if constexpr (F == DQ_I4) {
+            // 256-byte blocks of 128 rows' bf16 scales per group of 128 along K
+            const int m0 = MODE == MODE_GATEUP ? 0 : 2, m1 = MODE == MODE_GATEUP ? 1 : 2;
+            const int b0 = MODE == MODE_GATEUP ? rb : 2 * rb, b1 = MODE == MODE_GATEUP ? rb : 2 * rb + 1;
+            const int ng = K / 128;
+            bulk_load(st + 8192, blob + a.L.scales[m0] + ((size_t)b0 * ng + slab / 2) * 256, 256, bar);
+            bulk_load(st + 8448, blob + a.L.scales[m1] + ((size_t)b1 * ng + slab / 2) * 256, 256, bar);
+          }
+          ++issued;
+          if (++r == SR) { r = 0; ph ^= 1u; }
+        }
+      }
+      if (failed) {
+        // let the copies already issued land before the CTA exits
+        int r2 = 0;
+        uint32_t ph2 = 0;
+        for (int i = 0; i < issued; ++i) {
+          if (i >= issued - SR) mbar_drain(smem_u32(&raw_full[r2]), ph2);
+          if (++r2 == SR) { r2 = 0; ph2 ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one lane)
+    if (lane == 0) {
+      int s = 0, n = 0;
+      uint32_t ph = 0;
+      int q = 0;
+      uint32_t qph = 0;
+      while (true) {
+        if (!mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 59)) break;
+        const int item = sched_item[q];
+        const TileInfo ti = sched_ti[q];
+        const int loc = sched_loc[q];
+        mbar_arrive(smem_u32(&sched_empty[q]));
+        if (++q == kDqSched) { q = 0; qph ^= 1u; }
+        if (item < 0) break;
+        if (loc == kLocAbsent) continue;
+        const int N = max(16, (ti.nrows + 15) & ~15);
+        const int buf = n % NBUF;
+        if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 54)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(buf * 2 * NB);
+        const uint32_t idesc = idesc_bf16_dq(128, N);
+        bool failed = false;
+        for (int slab = 0; slab < nslab; ++slab) {
+          if (!mbar_wait(smem_u32(&op_full[s]), ph, a.err, 51)) { failed = true; break; }
+          fence_proxy_async_dq();
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {                   // K = 16 per MMA
+            const uint64_t bdesc = umma_desc(st + Geo::B_OFF + 32 * kk, 16, 1024, 2);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t adesc = umma_desc(st + h * 16384 + 32 * kk, 16, 1024, 2);
+              umma_bf16_dq(acc + (uint32_t)(h * NB), adesc, bdesc, idesc, (slab > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(smem_u32(&op_empty[s]));                 // stage free once these MMAs finish
+          if (++s == SO) { s = 0; ph ^= 1u; }
+        }
+        if (failed) break;
+        tc_commit(smem_u32(&accf_bar[buf]));
+        ++n;
+      }
+    }
+  } else if (warp >= 6 && warp < 10) {
+    // ---------------- decoders: raw codes + E4M3 scales -> bf16 weight tile
+    const int d = threadIdx.x - 192;                         // 0..127: rows d and d + 128 of the 256
+    int r = 0, s = 0, n_slabs = 0;
+    uint32_t rph = 0, sph = 0;
+    int q = 0;
+    uint32_t qph = 0;
+    bool failed = false;
+    while (!failed) {
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 60) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      __syncwarp();
+      const int item = sched_item[q];
+      const int loc = sched_loc[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+      if (++q == kDqSched) { q = 0; qph ^= 1u; }
+      if (item < 0) break;
+      if (loc == kLocAbsent) continue;
+      for (int slab = 0; slab < nslab; ++slab) {
+        int ok = 1;
+        if (lane == 0) {
+          ok = mbar_wait(smem_u32(&raw_full[r]), rph, a.err, 53) ? 1 : 0;
+          if (ok && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 55) ? 1 : 0;
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { failed = true; break; }
+        const uint8_t *raw = smem + Geo::RAW_OFF + (size_t)r * kRawBytes;
+        const uint32_t ast = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int row = d + 128 * hh;                      // row of the 256 in the raw stage
+          const int rr = row & 127;
+          const uint32_t rowa = ast + hh * 16384 + rr * 128;
+          if constexpr (F == DQ_F8) {
+            // the fp32 scale of this row's 128 x 128 block, from the blob
+            const int m = MODE == MODE_GATEUP ? hh : 2;
+            const int rbk = MODE == MODE_GATEUP ? item % ipt : 2 * (item % ipt) + hh;
+            const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
+            const float bs = __ldg(reinterpret_cast<const float *>(blob + a.L.scales[m]) + (size_t)rbk * (K / 128) + slab / 2);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const uint4 cv = *reinterpret_cast<const uint4 *>(raw + row * 64 + c4 * 16);
+              sts128(rowa + (((2 * c4) ^ (rr & 7)) << 4), decode8_fp8(cv.x, cv.y, bs));
+              sts128(rowa + (((2 * c4 + 1) ^ (rr & 7)) << 4), decode8_fp8(cv.z, cv.w, bs));
+            }
+          } else {
+            const uint4 c0 = *reinterpret_cast<const uint4 *>(raw + row * 32);
+            const uint4 c1 = *reinterpret_cast<const uint4 *>(raw + row * 32 + 16);
+            const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            if constexpr (F == DQ_NV) {
+              const uint32_t sf4 =
+                  *reinterpret_cast<const uint32_t *>(raw + 8192 + hh * 512 + 16 * (rr & 31) + 4 * (rr >> 5));
+              const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(sf4 & 0xFFFFu));
+              const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(sf4 >> 16));
+              const uint32_t sc[4] = {dup_lo16(s01), dup_hi16(s01), dup_lo16(s23), dup_hi16(s23)};
+#pragma unroll
+              for (int c = 0; c < 8; ++c) sts128(rowa + ((c ^ (rr & 7)) << 4), decode8(w[c], sc[c >> 1]));
+            } else {
+              const uint32_t sb = *reinterpret_cast<const uint16_t *>(raw + 8192 + hh * 256 + rr * 2);
+              const uint32_t sc2 = sb | (sb << 16);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) sts128(rowa + ((c ^ (rr & 7)) << 4), decode8_int4(w[c], sc2));
+            }
+          }
+        }
+        fence_proxy_async_dq();                              // generic-proxy writes -> tensor-core reads
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&raw_empty[r]));
+          mbar_arrive(smem_u32(&op_full[s]));
+        }
+        ++n_slabs;
+        if (++r == SR) { r = 0; rph ^= 1u; }
+        if (++s == SO) { s = 0; sph ^= 1u; }
+      }
+    }
+  } else if (warp >= 10) {
+    // ---------------- activation loaders: the tile's bf16 rows of this K slab
+    const int lt = threadIdx.x - 320;                        // 0..63
+    int s = 0, n_slabs = 0;
+    uint32_t sph = 0;
+    int q = 0;
+    uint32_t qph = 0;
+    bool failed = false;
+    while (!failed) {
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 61) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      __syncwarp();
+      const int item = sched_item[q];
+      const TileInfo ti = sched_ti[q];
+      const int loc = sched_loc[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+      if (++q == kDqSched) { q = 0; qph ^= 1u; }
+      if (item < 0) break;
+      if (loc == kLocAbsent) continue;
+      const int N = max(16, (ti.nrows + 15) & ~15);
+      // this thread's rows: j = lt / 8 + 8 i; 16-byte chunk lt % 8 of each
+      const int cq = lt & 7;
+      for (int slab = 0; slab < nslab; ++slab) {
+        int ok = 1;
+        if (lane == 0 && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 56) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { failed = true; break; }
+        const uint32_t bst = smem_u32(smem + (size_t)s * Geo::OP_STAGE + Geo::B_OFF);
+        for (int j = lt >> 3; j < N; j += kDqLoaders / 8) {
+          if (j >= ti.nrows) continue;                       // pad columns: never stored by the epilogue
+          const uint16_t *src;
+          if constexpr (MODE == MODE_GATEUP) {
+            const int tok = __ldg(a.prow_token + ti.prow0 + j);
+            src = a.act + (size_t)tok * K;
+          } else {
+            src = a.act + (size_t)(ti.prow0 + j) * K;
+          }
+          cp_async16_dq(bst + j * 128 + ((cq ^ (j & 7)) << 4), src + slab * 64 + cq * 8);
+        }
+        cp_async_arrive_dq(smem_u32(&op_full[s]));
+        ++n_slabs;
+        if (++s == SO) { s = 0; sph ^= 1u; }
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else {
+    // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+    const int quad = warp & 3;
+    int n = 0;
+    bool ok = true;
+    int q = 0;
+    uint32_t qph = 0;
+    while (ok) {
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 62) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      __syncwarp();
+      const int item = okw ? sched_item[q] : -1;
+      const TileInfo ti = sched_ti[q];
+      const int loc = sched_loc[q];
+      __syncwarp();
+      if (okw && lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+      if (++q == kDqSched) { q = 0; qph ^= 1u; }
+      if (!named_bar_and(1, 128, okw != 0 && item >= 0)) break;
+      if (loc == kLocAbsent) continue;
+      const int rb = item % ipt;
+      const int ntok = ti.nrows;
+      const int buf = n % NBUF;
+      const int et = threadIdx.x - 64;                       // 0..127 over warps 2..5
+      const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
+      // NVFP4: the per-tensor fp32 scales of gate, up and down; other formats carry none
+      const float one3[3] = {1.0f, 1.0f, 1.0f};
+      const float *gsc = F == DQ_NV ? reinterpret_cast<const float *>(blob + a.L.glob) : one3;
+      int my_pair = 0;
+      float my_gate = 0.0f;
+      if (MODE == MODE_DOWN && et < ntok) {
+        my_pair = __ldg(a.prow_pair + ti.prow0 + et);
+        my_gate = __ldg(a.gates + my_pair);
+      }
+      ok = mbar_wait(smem_u32(&accf_bar[buf]), (n / NBUF) & 1, a.err, 57);
+      if (MODE == MODE_DOWN && et < ntok) {
+        tok_pair[et] = my_pair;
+        tok_gate[et] = my_gate;
+      }
+      ok = named_bar_and(1, 128, ok);
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(buf * 2 * NB) + ((uint32_t)(32 * quad) << 16);
+      if constexpr (MODE == MODE_GATEUP) {
+        const float gg = gsc[0], gu = gsc[1];
+        const int I = a.rows;
+        const int rcol = rb * 128 + 32 * quad + lane;        // h column
+        for (int c0 = 0; c0 < ntok; c0 += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(acc + (uint32_t)c0, g);
+          tmem_ld32(acc + (uint32_t)(NB + c0), u);
+          tmem_ld_wait();
+          if (!ok) continue;
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            const int j = c0 + jj;
+            if (j >= ntok) continue;                         // warp-uniform
+            const float av = __uint_as_float(g[jj]) * gg;
+            const float uv = __uint_as_float(u[jj]) * gu;
+            a.h_out[(size_t)(ti.prow0 + j) * I + rcol] = bf16_bits(silu_f(av) * uv);
+          }
+        }
+      } else {
+        const float gd = gsc[2];
+        const int H = a.rows;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int orow = rb * 256 + hh * 128 + 32 * quad + lane;
+          for (int c0 = 0; c0 < ntok; c0 += 32) {
+            uint32_t dv[32];
+            tmem_ld32(acc + (uint32_t)(hh * NB + c0), dv);
+            tmem_ld_wait();
+            if (!ok) continue;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+              const int j = c0 + jj;
+              if (j >= ntok) continue;
+              a.o_out[(size_t)tok_pair[j] * H + orow] = __uint_as_float(dv[jj]) * gd * tok_gate[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acce_bar[buf]));
+      named_bar_sync(1, 128);                                // tok_pair / tok_gate are rewritten next item
+      ++n;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Geo::TMEM_COLS);
+  }
+}
+
+template <int MODE, int NB, int F>
+static void launch_dq_one(const DqArgs &a, cudaStream_t s) {
+  using Geo = DqGeom<NB, F>;
+  auto fn = expert_dq_kernel<MODE, NB, F>;
+  cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::SMEM);
+  launch_dependent(fn, a.grid, kDqThreads, Geo::SMEM, s, a);
+}
+
+template <int F>
+static void launch_dq_fmt(int mode, int nb, const DqArgs &a, cudaStream_t s) {
+  if (nb <= 64) {
+    if (mode == MODE_GATEUP) launch_dq_one<MODE_GATEUP, 64, F>(a, s);
+    else launch_dq_one<MODE_DOWN, 64, F>(a, s);
+  } else {
+    if (mode == MODE_GATEUP) launch_dq_one<MODE_GATEUP, 128, F>(a, s);
+    else launch_dq_one<MODE_DOWN, 128, F>(a, s);
+  }
+}
+
+void launch_expert_dq(int mode, int nb, const DqArgs &a, cudaStream_t s) {
+  if (a.grid <= 0) return;
+  if (a.wfmt == DQ_I4) launch_dq_fmt<DQ_I4>(mode, nb, a, s);
+  else if (a.wfmt == DQ_F8) launch_dq_fmt<DQ_F8>(mode, nb, a, s);
+  else launch_dq_fmt<DQ_NV>(mode, nb, a, s);
+}
+
+}  // namespace moe

@@ -373,6 +373,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
           a.o_out[(size_t)p * a.rows + mrow[j][x >> 1]] = acc[j][nt][x] * rowf[j][x >> 1] * gp;
       }
     // ordered combine by the last arrival of each token on this row block
+    // (y null: the combine kernel runs after this pass instead)
+    if (a.y == nullptr) return;
     __threadfence();
     named_bar_sync(1, kConsumers * 32);
     if (threadIdx.x < 8 * NT) {

@@ -83,7 +83,8 @@ struct alignas(16) TileInfo {
 // ------------------------------------------------------------------ routing
 struct PermArgs {
   const int *ids;        // [T*k]
-  int n_pairs, E, k, tile_tokens;
+  int n_pairs, E, k, tile_tokens;   // E: routing targets (experts, then sinks)
+  int n_real;            // experts with an FFN; targets >= n_real are sinks (no rows, no tiles)
   int *counts;           // [E]
   int *offsets;          // [E+1]
   int *perm;             // [n_pairs]
@@ -100,7 +101,9 @@ struct PermArgs {
 };
 struct RouterArgs {
   const uint16_t *x;     // bf16 [T, H]
-  int T, H, E, k;
+  int T, H, E, k;        // E: logit rows (targets, then the shared-expert gate row if any)
+  int E_t;               // routing targets (experts, then sinks) among the E rows
+  int scoring, renorm;   // 0 softmax / 1 sigmoid; 1: chosen scores renormalised
   const float *w;        // [E, H]
   const float *bias;     // [E] or null
   float *logits;         // [T, E]
@@ -124,8 +127,10 @@ void launch_permute(const PermArgs &a, cudaStream_t s);
 int router_gemm_splits(int T, int H, int E, size_t part_floats);
 void launch_router_gemm(const uint16_t *x, const float *w, const float *bias, int T, int H, int E, float *logits,
                         float *parts, int splits, cudaStream_t s);
-void launch_topk(float *logits, const float *parts, int splits, const float *bias, int T, int E, int k, int *ids,
-                 float *gates, cudaStream_t s);
+// E: logit rows (row stride); E_t: routing targets among them (top-k runs over
+// the first E_t); scoring / renorm as in RouterArgs.
+void launch_topk(float *logits, const float *parts, int splits, const float *bias, int T, int E, int E_t, int k,
+                 int scoring, int renorm, int *ids, float *gates, cudaStream_t s);
 
 // ------------------------------------------------------------------ experts
 enum WeightFmt { WF_MX = 0, WF_NV = 1, WF_BF16 = 2 };
@@ -163,8 +168,17 @@ void launch_expert(int wf, int mode, int nt, const ExpertArgs &a, int grid_tiles
 struct CombineArgs {
   const float *oprime;   // [T*k, H]
   const float *shared;   // [T, H] or null
-  float *y;              // [T, H]
+  void *y;               // [T, H]: fp32, or bf16 when out_bf16
   int T, H, k;
+  int out_bf16;
+  // sink targets: slots whose id is >= n_real add nothing (their O' rows are
+  // never written); ids may be null when the layer has no sinks
+  const int *ids;        // [T*k]
+  int n_real;
+  // sigmoid-gated shared expert: s is scaled by sigmoid(logits[t * ld + sg_col])
+  // (null: weight 1)
+  const float *sg_logits;
+  int ld, sg_col;
 };
 void launch_combine(const CombineArgs &a, cudaStream_t s);
 
@@ -352,5 +366,45 @@ struct TcArgs {
 // persistent: `a.grid` CTAs take the work items (tile, 256 weight rows) from
 // `a.work_ctr` in index order.
 void launch_expert_tc(int mode, int nbox, const TcArgs &a, int grid_tiles, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// EXACT numerics for NVFP4 experts at prefill-sized batches (expert_dq.cu):
+// each 64-element K slab of a weight tile is decoded once per token tile into
+// shared memory as bf16 (E2M1 x E4M3 is exact in bf16) and multiplied with
+// tcgen05 kind::f16 against bf16 activation rows; the per-tensor scale is
+// applied in the epilogue.  h is written as bf16 in padded-row order.
+struct DqMaps {
+  // code bytes of matrix m of every blob in a region, 3-D (K/2 bytes, rows,
+  // blob), box 32 bytes x (128 rows: gate / up | 256 rows: down) x 1
+  CUtensorMap slot[3];
+  CUtensorMap stage[3];
+};
+
+// weight formats of the dequantise-to-shared kernels
+enum DqFmt { DQ_NV = 0, DQ_I4 = 1, DQ_F8 = 2 };
+
+struct DqArgs {
+  DqMaps maps;
+  int wfmt;                  // DqFmt
+  const int *loc;
+  const uint8_t *slots;
+  const uint8_t *staging;
+  size_t blob_bytes;
+  BlobLayout L;
+  int K, rows, n_rowblocks;  // reduction length, weight rows of the pass, items per tile
+  const TileInfo *tiles;
+  const int *n_tiles;
+  const int *prow_token;     // gate/up: padded row -> token
+  const int *prow_pair;      // down: padded row -> pair
+  const float *gates;
+  const uint16_t *act;       // gate/up: x bf16 [T, H]; down: h bf16 [padded rows, I]
+  uint16_t *h_out;           // gate/up: h bf16 [padded rows, I]
+  float *o_out;              // down: O' [pairs, H]
+  int *work_ctr;             // item counter of this pass, zero at launch
+  int *err;
+  int grid;                  // persistent CTAs
+};
+// nb: tokens per tile (64 or 128)
+void launch_expert_dq(int mode, int nb, const DqArgs &a, cudaStream_t s);
 
 }  // namespace moe

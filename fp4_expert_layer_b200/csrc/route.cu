@@ -136,9 +136,10 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
 #pragma unroll
     for (int i = 0; i < KPER; ++i) {
       const int ee = lane + 32 * i;
-      lv[i] = (ee < E) ? __ldcg(lrow + ee) : -INFINITY;
+      lv[i] = (ee < a.E_t) ? __ldcg(lrow + ee) : -INFINITY;
     }
-    topk_warp<KPER>(lv, E, a.k, a.ids + (size_t)t * a.k, a.gates + (size_t)t * a.k, nullptr);
+    topk_warp<KPER>(lv, a.E_t, a.k, a.ids + (size_t)t * a.k, a.gates + (size_t)t * a.k, nullptr, a.scoring,
+                    a.renorm);
   }
   if (!a.fuse_perm) return;
 
@@ -163,10 +164,10 @@ static void launch_router_k(const RouterArgs &a, cudaStream_t s) {
 }
 
 void launch_router(const RouterArgs &a, cudaStream_t s) {
-  if (a.E <= 64) launch_router_k<2>(a, s);
-  else if (a.E <= 128) launch_router_k<4>(a, s);
-  else if (a.E <= 256) launch_router_k<8>(a, s);
-  else if (a.E <= 512) launch_router_k<16>(a, s);
+  if (a.E_t <= 64) launch_router_k<2>(a, s);
+  else if (a.E_t <= 128) launch_router_k<4>(a, s);
+  else if (a.E_t <= 256) launch_router_k<8>(a, s);
+  else if (a.E_t <= 512) launch_router_k<16>(a, s);
   else launch_router_k<32>(a, s);
 }
 
@@ -198,7 +199,8 @@ void launch_ptr_update(const PtrUpdate &u, const uint8_t *const *resident, const
 }
 
 // ---------------------------------------------------------------------------
-// Ordered combine: y[t] = sum_{j<k} O'[t*k + j] (in j order) + s[t].
+// Ordered combine: y[t] = sum_{j<k, ids_j an expert} O'[t*k + j] (in j order)
+// + gs[t] * s[t], gs = 1 or sigmoid(shared-gate logit); y fp32 or bf16 (RN).
 // ---------------------------------------------------------------------------
 __global__ void combine_kernel(const CombineArgs a) {
   wait_prior_grid();
@@ -208,16 +210,28 @@ __global__ void combine_kernel(const CombineArgs a) {
        i += (size_t)gridDim.x * blockDim.x) {
     const size_t t = i / H4, c = i % H4;
     const float4 *o = reinterpret_cast<const float4 *>(a.oprime) + t * a.k * H4 + c;
-    float4 acc = __ldcs(o);
-    for (int j = 1; j < a.k; ++j) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);       // 0 + v == v: the first term is exact
+    for (int j = 0; j < a.k; ++j) {
+      if (a.ids && __ldg(a.ids + t * a.k + j) >= a.n_real) continue;   // a sink: no FFN
       const float4 v = __ldcs(o + (size_t)j * H4);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
     if (a.shared) {
-      const float4 v = reinterpret_cast<const float4 *>(a.shared)[t * H4 + c];
+      float4 v = reinterpret_cast<const float4 *>(a.shared)[t * H4 + c];
+      if (a.sg_logits) {
+        const float gs = 1.0f / (1.0f + expf(-__ldg(a.sg_logits + t * a.ld + a.sg_col)));
+        v.x *= gs; v.y *= gs; v.z *= gs; v.w *= gs;
+      }
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
-    reinterpret_cast<float4 *>(a.y)[t * H4 + c] = acc;
+    if (a.out_bf16) {
+      uint2 b;
+      b.x = (uint32_t)bf16_bits(acc.x) | ((uint32_t)bf16_bits(acc.y) << 16);
+      b.y = (uint32_t)bf16_bits(acc.z) | ((uint32_t)bf16_bits(acc.w) << 16);
+      reinterpret_cast<uint2 *>(a.y)[t * H4 + c] = b;
+    } else {
+      reinterpret_cast<float4 *>(a.y)[t * H4 + c] = acc;
+    }
   }
 }
 
@@ -351,39 +365,41 @@ void launch_router_gemm(const uint16_t *x, const float *w, const float *bias, in
 // order, plus the bias) and written out.
 template <int KPER>
 __global__ void __launch_bounds__(256) topk_kernel(float *logits, const float *parts, int splits,
-                                                   const float *bias, int T, int E, int k, int *ids,
-                                                   float *gates) {
+                                                   const float *bias, int T, int E, int E_t, int k, int scoring,
+                                                   int renorm, int *ids, float *gates) {
   wait_prior_grid();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (t >= T) return;
-  float lv[KPER];
   float *lrow = logits + (size_t)t * E;
-#pragma unroll
-  for (int i = 0; i < KPER; ++i) {
-    const int ee = lane + 32 * i;
-    if (ee >= E) {
-      lv[i] = -INFINITY;
-    } else if (splits > 1) {
+  if (splits > 1) {
+    // every logit row of the token (targets and a shared-expert gate row)
+    for (int ee = lane; ee < E; ee += 32) {
       float v = __ldcg(parts + (size_t)t * E + ee);
       for (int sp = 1; sp < splits; ++sp) v += __ldcg(parts + ((size_t)sp * T + t) * E + ee);
       v += bias ? bias[ee] : 0.0f;
       lrow[ee] = v;
-      lv[i] = v;
-    } else {
-      lv[i] = __ldcg(lrow + ee);
     }
+    __syncwarp();
   }
-  topk_warp<KPER>(lv, E, k, ids + (size_t)t * k, gates + (size_t)t * k, nullptr);
+  float lv[KPER];
+#pragma unroll
+  for (int i = 0; i < KPER; ++i) {
+    const int ee = lane + 32 * i;
+    lv[i] = ee < E_t ? __ldcg(lrow + ee) : -INFINITY;
+  }
+  topk_warp<KPER>(lv, E_t, k, ids + (size_t)t * k, gates + (size_t)t * k, nullptr, scoring, renorm);
 }
 
-void launch_topk(float *logits, const float *parts, int splits, const float *bias, int T, int E, int k, int *ids,
-                 float *gates, cudaStream_t s) {
+void launch_topk(float *logits, const float *parts, int splits, const float *bias, int T, int E, int E_t, int k,
+                 int scoring, int renorm, int *ids, float *gates, cudaStream_t s) {
   const int blocks = (T + 7) / 8;
-  if (E <= 64) launch_dependent(topk_kernel<2>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
-  else if (E <= 128) launch_dependent(topk_kernel<4>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
-  else if (E <= 256) launch_dependent(topk_kernel<8>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
-  else if (E <= 512) launch_dependent(topk_kernel<16>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
-  else launch_dependent(topk_kernel<32>, blocks, 256, 0, s, logits, parts, splits, bias, T, E, k, ids, gates);
+#define MOE_TOPK_ARGS logits, parts, splits, bias, T, E, E_t, k, scoring, renorm, ids, gates
+  if (E_t <= 64) launch_dependent(topk_kernel<2>, blocks, 256, 0, s, MOE_TOPK_ARGS);
+  else if (E_t <= 128) launch_dependent(topk_kernel<4>, blocks, 256, 0, s, MOE_TOPK_ARGS);
+  else if (E_t <= 256) launch_dependent(topk_kernel<8>, blocks, 256, 0, s, MOE_TOPK_ARGS);
+  else if (E_t <= 512) launch_dependent(topk_kernel<16>, blocks, 256, 0, s, MOE_TOPK_ARGS);
+  else launch_dependent(topk_kernel<32>, blocks, 256, 0, s, MOE_TOPK_ARGS);
+#undef MOE_TOPK_ARGS
 }
 
 void launch_combine(const CombineArgs &a, cudaStream_t s) {

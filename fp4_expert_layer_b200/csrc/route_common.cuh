@@ -14,14 +14,18 @@ __device__ __forceinline__ int load_id(const int *ids, int p) {
   else return ids[p];
 }
 
-// Top-k of one token by one warp: lane holds the logits of experts lane,
-// lane + 32, ... in lv (-inf past E).  Ids in descending-logit order, lower
-// index first on ties; gates g_j = exp(l_j - l_max) / sum_i exp(l_i - l_max)
-// over the k chosen, summed in j order.  Writes ids / gates (k entries each)
-// and, if ids_s is not null, the ids to shared memory too.
+// Top-k of one token by one warp: lane holds the logits of targets lane,
+// lane + 32, ... in lv (-inf past E; E counts experts and sink targets).  Ids
+// in descending-logit order, lower index first on ties (both scorings are
+// monotone in the logit).  Scores: softmax s_j = exp(l_j - l_max) / sum over
+// all E targets, or sigmoid s_j = 1 / (1 + exp(-l_j)); gates = s_j / sum of
+// the k chosen s (summed in j order) when renorm, else s_j.  Softmax with
+// renormalisation is computed as exp(l_j - l_max) over the chosen k's sum.
+// Writes ids / gates (k entries each) and, if ids_s is not null, the ids to
+// shared memory too.
 template <int KPER>
 __device__ __forceinline__ void topk_warp(const float (&lv)[KPER], int E, int k, int *ids, float *gates,
-                                          int *ids_s) {
+                                          int *ids_s, int scoring = 0, int renorm = 1) {
   const int lane = threadIdx.x & 31;
   uint32_t taken = 0;   // bit i: lane's i-th expert already chosen
   float lmax = 0.0f, den = 0.0f;
@@ -50,12 +54,29 @@ __device__ __forceinline__ void topk_warp(const float (&lv)[KPER], int E, int k,
     if (j == 0) lmax = bv;
     if (lane == j) { my_l = bv; my_id = bi; }
   }
-  const float ex = (lane < k) ? expf(my_l - lmax) : 0.0f;
-  // ordered sum over j = 0..k-1
-  for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, ex, j);
+  float ex;
+  if (scoring == 0) {
+    ex = (lane < k) ? expf(my_l - lmax) : 0.0f;
+    if (!renorm) {
+      // softmax over every target: this lane's terms, then a butterfly sum
+      float all = 0.0f;
+#pragma unroll
+      for (int i = 0; i < KPER; ++i)
+        if (lane + 32 * i < E) all += expf(lv[i] - lmax);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) all += __shfl_xor_sync(0xffffffffu, all, o);
+      ex = ex / all;
+    }
+  } else {
+    ex = (lane < k) ? 1.0f / (1.0f + expf(-my_l)) : 0.0f;
+  }
+  if (renorm) {
+    // ordered sum over j = 0..k-1
+    for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, ex, j);
+  }
   if (lane < k) {
     ids[lane] = my_id;
-    gates[lane] = ex / den;
+    gates[lane] = renorm ? ex / den : ex;
     if (ids_s) ids_s[lane] = my_id;
   }
 }
@@ -90,16 +111,18 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
   for (int p = tid; p < a.n_pairs; p += NTH) atomicAdd(&cnt[load_id<IDS_GLOBAL>(ids, p)], 1);
   __syncthreads();
 
-  // block exclusive scan of (count, padded count, tiles, active) over experts
+  // block exclusive scan of (count, padded count, tiles, active) over targets;
+  // sink targets (e >= n_real) have counts and offsets but no rows or tiles
   const int per = (E + NTH - 1) / NTH;
   const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
   int4 v = make_int4(0, 0, 0, 0);
   for (int e = e0; e < e1; ++e) {
     const int c = cnt[e];
+    const int cr = e < a.n_real ? c : 0;
     v.x += c;
-    v.y += (c + a.pad - 1) / a.pad * a.pad;
-    v.z += (c + a.tile_tokens - 1) / a.tile_tokens;
-    v.w += c > 0;
+    v.y += (cr + a.pad - 1) / a.pad * a.pad;
+    v.z += (cr + a.tile_tokens - 1) / a.tile_tokens;
+    v.w += cr > 0;
   }
   int4 inc = v;
 #pragma unroll
@@ -132,10 +155,11 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
     int o = pre.x + inc.x - v.x, po = pre.y + inc.y - v.y, to = pre.z + inc.z - v.z;
     for (int e = e0; e < e1; ++e) {
       const int c = cnt[e];
+      const int cr = e < a.n_real ? c : 0;
       off[e] = o; poff[e] = po; toff[e] = to;
       o += c;
-      po += (c + a.pad - 1) / a.pad * a.pad;
-      to += (c + a.tile_tokens - 1) / a.tile_tokens;
+      po += (cr + a.pad - 1) / a.pad * a.pad;
+      to += (cr + a.tile_tokens - 1) / a.tile_tokens;
     }
     if (tid == NTH - 1) {
       const int4 tot = wsum[W - 1];
@@ -152,6 +176,7 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
   for (int e = tid; e < E; e += NTH) {
     const int c = cnt[e];
     a.counts[e] = c;
+    if (e >= a.n_real) continue;                   // a sink: no rows, no tiles
     const int nt = (c + a.tile_tokens - 1) / a.tile_tokens;
     for (int i = 0; i < nt; ++i) {
       TileInfo ti;
@@ -186,11 +211,13 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
     if (valid) {
       const int local = wcnt[warp * E + e] + rank;
       const int pos = off[e] + local;
-      const int prow = poff[e] + local;
       a.perm[pos] = p;
       a.inv[p] = pos;
-      a.prow_token[prow] = p / a.k;
-      a.prow_pair[prow] = p;
+      if (e < a.n_real) {
+        const int prow = poff[e] + local;
+        a.prow_token[prow] = p / a.k;
+        a.prow_pair[prow] = p;
+      }
     }
     __syncthreads();
     for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;

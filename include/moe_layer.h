@@ -59,7 +59,18 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 6  /* valid request this build does not implement       */
 } moe_status_t;
 
-typedef enum { MOE_FMT_MXFP4 = 0, MOE_FMT_NVFP4 = 1 } moe_fmt_t;
+/* Expert weight formats ("ro99/strata", model table: "NVFP4 or MXFP4
+ * experts", "INT4 group-128, W4A16", "FP8 E4M3 block-128 with F32 inverse
+ * scales"; never below four bits):
+ *   MXFP4     E2M1 codes, two per byte, one E8M0 exponent per 32 along K;
+ *   NVFP4     E2M1 codes, one E4M3 scale per 16 along K, one fp32 scale per
+ *             matrix;
+ *   INT4G128  signed 4-bit integers (two's complement, -8..7), two per byte,
+ *             one bf16 scale per 128 along K; w = q * s;
+ *   FP8B128   one E4M3 byte per weight, one fp32 inverse scale per block of
+ *             128 rows x 128 columns; w = q * s.
+ * In every format the even input index is the low nibble / first byte. */
+typedef enum { MOE_FMT_MXFP4 = 0, MOE_FMT_NVFP4 = 1, MOE_FMT_INT4G128 = 2, MOE_FMT_FP8B128 = 3 } moe_fmt_t;
 
 /* EXACT (default): activations stay 16-bit, FP4 weights decode exactly, fp32
  * accumulation.  A4 (opt-in): activations are quantised to the experts' own
@@ -67,21 +78,43 @@ typedef enum { MOE_FMT_MXFP4 = 0, MOE_FMT_NVFP4 = 1 } moe_fmt_t;
  * run; never chosen silently. */
 typedef enum { MOE_NUMERICS_EXACT = 0, MOE_NUMERICS_A4 = 1 } moe_numerics_t;
 
+/* Router scoring: softmax over every routing target, or an independent
+ * logistic per target (ids are the k largest logits either way). */
+typedef enum { MOE_SCORING_SOFTMAX = 0, MOE_SCORING_SIGMOID = 1 } moe_scoring_t;
+
+typedef enum { MOE_OUT_F32 = 0, MOE_OUT_BF16 = 1 } moe_out_dtype_t;
+
+/* The routing semantics are what the checkpoint declares ("ro99/strata",
+ * rules list: precision, routing, expert count and top-k come from the
+ * checkpoint and never change silently): scoring, renormalisation, sink
+ * targets (its model table has "256 experts + 2 sinks") and a sigmoid gate on
+ * the shared expert are configuration, never chosen by the library.
+ * Routing targets are the E experts followed by n_sinks sinks; a sink is
+ * scored and chosen like an expert but has no FFN: choosing it adds nothing to
+ * y (its gate share is not given to the other experts unless renormalisation
+ * already did). */
 typedef struct {
   int32_t hidden;       /* H; multiple of 256                                   */
   int32_t inter;        /* I (routed expert intermediate); multiple of 128       */
   int32_t n_experts;    /* E routed experts, 1..1024                            */
-  int32_t top_k;        /* k, 1..min(E, 32)                                     */
+  int32_t top_k;        /* k, 1..min(E + n_sinks, 32)                           */
   int32_t shared_inter; /* I_s of the always-on bf16 shared expert, 0 = none;   */
                         /* multiple of 128                                      */
   int32_t fmt;          /* moe_fmt_t                                            */
-  int32_t renormalize;  /* must be 1: top-k gates renormalised to sum to 1      */
+  int32_t renormalize;  /* 1: the k chosen scores are divided by their sum;     */
+                        /* 0: they are used as they are                         */
   int32_t numerics;     /* moe_numerics_t                                       */
   int32_t n_slots;      /* S resident HBM slots, 0..E                           */
   int32_t max_tokens;   /* largest T accepted by moe_forward, >= 1              */
   int32_t n_staging;    /* staging buffers for non-resident experts; >= 2 when  */
                         /* S < E (0 = library default)                          */
   int32_t device;       /* CUDA device ordinal                                   */
+  int32_t scoring;      /* moe_scoring_t                                        */
+  int32_t n_sinks;      /* sink targets after the experts, >= 0;                */
+                        /* E + n_sinks + shared_gate <= 1024                    */
+  int32_t shared_gate;  /* 1: the shared expert is scaled by                    */
+                        /* sigmoid(x . shared_gate_w) (needs shared_inter > 0)  */
+  int32_t out_dtype;    /* moe_out_dtype_t of y                                 */
 } moe_config_t;
 
 /* Layer weights in checkpoint layout (host memory; read only during create).
@@ -95,19 +128,22 @@ typedef struct {
  * The library copies everything during moe_layer_create; the caller may free
  * these buffers when it returns. */
 typedef struct {
-  const float *router_w;            /* fp32 [E, H]                             */
-  const float *router_bias;         /* fp32 [E] added to the logits, or NULL   */
+  const float *router_w;            /* fp32 [E + n_sinks, H]                   */
+  const float *router_bias;         /* fp32 [E + n_sinks] added to the logits, */
+                                    /* or NULL                                 */
   const uint8_t *const *codes[3];   /* codes[m] -> array of E host pointers    */
   const uint8_t *const *scales[3];  /* scales[m] -> array of E host pointers   */
   const float *global_scale;        /* fp32 [E, 3] or NULL                     */
   const uint16_t *shared_w[3];      /* NULL when shared_inter == 0             */
+  const float *shared_gate_w;       /* fp32 [H] when shared_gate, else NULL    */
 } moe_weights_t;
 
 /* Optional routing outputs of a forward (all device pointers, each may be
- * NULL).  logits fp32 [T, E]; ids int32 [T, k] in descending-logit order (lower
- * index first on ties); gates fp32 [T, k]; counts int32 [E]; offsets int32
- * [E+1] (exclusive scan of counts); perm int32 [T*k]: sorted position -> pair
- * index p = t*k + j (stable by expert, ties by ascending p); inv int32 [T*k]:
+ * NULL).  With NT = E + n_sinks routing targets: logits fp32 [T, NT]; ids
+ * int32 [T, k] in descending-logit order (lower index first on ties; ids >= E
+ * are sinks); gates fp32 [T, k]; counts int32 [NT]; offsets int32 [NT+1]
+ * (exclusive scan of counts); perm int32 [T*k]: sorted position -> pair index
+ * p = t*k + j (stable by target, ties by ascending p); inv int32 [T*k]:
  * p -> sorted position. */
 typedef struct {
   float *logits;
@@ -128,7 +164,9 @@ typedef struct {
   int32_t last_active;     /* experts with at least one token, last forward     */
   int32_t last_path;       /* 0 = register-decode kernels (EXACT), 1 = A4      */
                            /* tcgen05 FP4 x FP4, 2 = EXACT on tcgen05 (MXFP4    */
-                           /* weights x E4M3 activation pieces)                 */
+                           /* weights x E4M3 activation pieces), 3 = EXACT on   */
+                           /* tcgen05 (NVFP4 weights decoded to bf16 in shared  */
+                           /* memory x bf16 activations)                        */
   uint64_t launches;       /* kernels this library launched, cumulative         */
   uint64_t expert_bytes;   /* device-layout bytes of one routed expert          */
   uint64_t device_bytes;   /* HBM held by the layer                             */
@@ -136,6 +174,9 @@ typedef struct {
   int32_t device_error;    /* nonzero: a device-side wait gave up (code of the  */
                            /* first one); the next moe_forward reports and      */
                            /* clears it                                         */
+  int32_t policy;          /* moe_policy_t in force                             */
+  uint64_t admitted;       /* staged experts admitted into slots, cumulative    */
+  uint64_t prefetched;     /* experts copied into slots by moe_prefetch         */
 } moe_stats_t;
 
 /* Memory plan of a configuration without allocating anything (the dry-run
@@ -175,7 +216,41 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
  * stream see the new table.  The table never changes inside moe_forward. */
 moe_status_t moe_set_slot_table(moe_layer_t layer, const int32_t *slot_of_expert, void *stream);
 
-/* Forward T tokens: x device bf16 [T, H] -> y device fp32 [T, H].
+/* Who decides which experts are resident (the routing/paging policies
+ * none | warm | cache | hybrid of strata.amperor.ai; "Strata, Explained",
+ * section 2: an adaptive VRAM cache over every expert pinned in RAM):
+ *   STATIC  the caller's slot table, changed only by moe_set_slot_table (a
+ *           hottest-first table set once is the "warm" policy); the default;
+ *   NONE    no expert is resident: the table is cleared and every expert a
+ *           forward needs is staged;
+ *   CACHE   the library manages the slots as a cache: after each forward
+ *           that staged experts, missed experts are admitted into slots whose
+ *           expert that forward did not use (empty slots first, then least
+ *           recently used), by a device-to-device copy from the staging
+ *           buffer right after the wave that used it; the new table holds for
+ *           the next forward;
+ *   HYBRID  CACHE on slots [n_pinned, S); the experts in slots [0, n_pinned)
+ *           at the time of the call are pinned (a warm fill plus a cache).
+ * The current table is the cache's starting content.  Residency never changes
+ * what a forward computes: output is bit-identical under every policy.
+ * n_pinned is used by HYBRID only (0..S).  Returns after the stream's queued
+ * work completes. */
+typedef enum { MOE_POLICY_STATIC = 0, MOE_POLICY_NONE = 1, MOE_POLICY_CACHE = 2, MOE_POLICY_HYBRID = 3 } moe_policy_t;
+moe_status_t moe_set_policy(moe_layer_t layer, int32_t policy, int32_t n_pinned, void *stream);
+
+/* Prefetch under CACHE or HYBRID: copies the listed experts (host int32
+ * [n], a predictor's guess for a coming forward) that are not resident into
+ * evictable slots (empty first, then least recently used; experts listed in
+ * the same call are not evicted for one another), from the pinned store on the
+ * layer's side stream after the work already queued on `stream`; the next
+ * forward waits for these copies before its expert passes.  A predictor only
+ * reorders work ("ro99/strata", rules list): what the next forward computes
+ * does not change.  Experts beyond the evictable slots are skipped.  Other
+ * policies: MOE_ERR_INVALID_ARG. */
+moe_status_t moe_prefetch(moe_layer_t layer, const int32_t *experts, int32_t n, void *stream);
+
+/* Forward T tokens: x device bf16 [T, H] -> y device [T, H], fp32 or bf16
+ * (rounded to nearest even) as the config's out_dtype says.
  * 0 <= T <= max_tokens (T == 0 is a no-op).  x and y must not overlap.
  * When every expert the forward needs is resident, the call only enqueues
  * work on `stream` and returns.  Otherwise it waits for the routing counts
@@ -183,18 +258,18 @@ moe_status_t moe_set_slot_table(moe_layer_t layer, const int32_t *slot_of_expert
  * pinned store on the layer's side stream, overlapped with compute in waves
  * of at most n_staging experts; it returns once all work is enqueued.
  * dbg (may be NULL) receives the routing tensors of this forward. */
-moe_status_t moe_forward(moe_layer_t layer, const void *x, int32_t T, float *y, void *stream,
+moe_status_t moe_forward(moe_layer_t layer, const void *x, int32_t T, void *y, void *stream,
                          const moe_routing_t *dbg);
 
 /* Same forward from and to HOST memory: copies x (host bf16 [T, H]) to a
- * layer-owned device buffer, runs the forward and copies y back to host fp32
- * [T, H].  Returns after y is in host memory. */
+ * layer-owned device buffer, runs the forward and copies y back to host
+ * [T, H] (fp32 or bf16 per out_dtype).  Returns after y is in host memory. */
 moe_status_t moe_forward_host(moe_layer_t layer, const uint16_t *x_host, int32_t T,
-                              float *y_host, void *stream);
+                              void *y_host, void *stream);
 
 /* CUDA graph of one forward (launch overhead of a decode step).
  * moe_graph_capture records the forward of T tokens from x (device bf16
- * [T, H]) into y (device fp32 [T, H]) on `stream` (a created stream, not the
+ * [T, H]) into y (device [T, H], out_dtype) on `stream` (a created stream, not the
  * legacy default stream) into a CUDA graph without running it; each
  * moe_graph_launch replays it on `stream`, reading the x and writing the y
  * given at capture.  Requires every expert resident (the staged path waits for
@@ -203,7 +278,7 @@ moe_status_t moe_forward_host(moe_layer_t layer, const uint16_t *x_host, int32_t
  * The graph belongs to the caller: moe_graph_destroy before moe_destroy of its
  * layer.  Replays count in moe_stats_t (forwards, launches). */
 typedef struct moe_graph *moe_graph_t;
-moe_status_t moe_graph_capture(moe_layer_t layer, const void *x, int32_t T, float *y, void *stream,
+moe_status_t moe_graph_capture(moe_layer_t layer, const void *x, int32_t T, void *y, void *stream,
                                moe_graph_t *out);
 moe_status_t moe_graph_launch(moe_graph_t graph, void *stream);
 moe_status_t moe_graph_destroy(moe_graph_t graph);

@@ -21,7 +21,7 @@ _SO = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-FMT = {"mxfp4": 0, "nvfp4": 1}
+FMT = {"mxfp4": 0, "nvfp4": 1, "int4g128": 2, "fp8b128": 3}
 NUMERICS = {"exact": 0, "a4": 1}
 
 
@@ -67,6 +67,10 @@ def lib():
         L.orc_rn_e4m3.argtypes = [C.c_float]
         L.orc_admit_scales.restype = C.c_long
         L.orc_admit_scales.argtypes = [C.c_int, C.c_void_p, C.c_long]
+        L.orc_admit_fp8_codes.restype = C.c_long
+        L.orc_admit_fp8_codes.argtypes = [C.c_void_p, C.c_long]
+        L.orc_int4.restype = C.c_double
+        L.orc_int4.argtypes = [C.c_uint]
         L.orc_quant_mx_block.restype = None
         L.orc_quant_mx_block.argtypes = [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]
         L.orc_quant_nv_row.restype = None
@@ -120,8 +124,19 @@ def rn_e4m3(t: float) -> int:
 
 
 def admit_scales(fmt: str, s: np.ndarray) -> int:
-    s = np.ascontiguousarray(s, dtype=np.uint8)
-    return lib().orc_admit_scales(FMT[fmt], _p(s), s.size)
+    """Index of the first scale the format rejects, or -1 (s holds the format's
+    scale values: uint8 codes, bf16 bits as uint16, or fp32)."""
+    s = np.ascontiguousarray(s)
+    return lib().orc_admit_scales(FMT[fmt], _p(s.view(np.uint8)), s.size)
+
+
+def admit_fp8_codes(q: np.ndarray) -> int:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    return lib().orc_admit_fp8_codes(_p(q), q.size)
+
+
+def int4(nibble: int) -> float:
+    return lib().orc_int4(nibble)
 
 
 def quant_mx_block(v: np.ndarray):
@@ -203,7 +218,8 @@ class Layer:
         s.router_bias = _p(keep(router_bias, np.float32))
         for m in range(3):
             s.codes[m] = _p(keep(codes[m], np.uint8))
-            s.scales[m] = _p(keep(scales[m], np.uint8))
+            # scales are passed as their bytes (uint8 codes, bf16 bits or fp32 by format)
+            s.scales[m] = _p(keep(np.ascontiguousarray(scales[m]).view(np.uint8), np.uint8))
             s.shared_w[m] = None if shared_w is None else _p(keep(shared_w[m], np.uint16))
         s.global_scale = _p(keep(global_scale, np.float32))
         s.scoring = SCORING[scoring]

@@ -44,6 +44,18 @@
 
 #define ORC_FMT_MXFP4 0
 #define ORC_FMT_NVFP4 1
+/* Other expert formats of at least four bits that checkpoints ship
+ * ("ro99/strata", model table: "INT4 group-128, W4A16" and "FP8 E4M3
+ * block-128 with F32 inverse scales"):
+ *  INT4G128: codes [rows, K/2], two signed 4-bit integers per byte (even
+ *            element in the low nibble, two's complement, -8..7), one bf16
+ *            scale per row and group of 128 along K: scales [rows, K/128]
+ *            (uint16 bf16 bits); w = q * scale;
+ *  FP8B128:  codes [rows, K], one E4M3 byte per weight, one fp32 inverse
+ *            scale per block of 128 rows x 128 columns: scales [rows/128,
+ *            K/128] (fp32); w = e4m3(q) * scale. */
+#define ORC_FMT_INT4G128 2
+#define ORC_FMT_FP8B128 3
 #define ORC_EXACT 0
 #define ORC_A4 1
 #define ORC_SOFTMAX 0
@@ -110,9 +122,23 @@ double orc_bf16(uint16_t b) {
 
 /* Admission: index of the first rejected scale code, or -1.
  * MXFP4: E8M0 codes 0 and 255 are rejected.  NVFP4: E4M3 NaN codes and codes
- * with the sign bit set are rejected (a block scale is a magnitude). */
+ * with the sign bit set are rejected (a block scale is a magnitude).  INT4G128
+ * (bf16 scales, n = number of scales): NaN and infinite scales are rejected.
+ * FP8B128 (fp32 scales): NaN, infinite, zero and negative scales. */
 long orc_admit_scales(int fmt, const uint8_t *s, long n) {
   for (long i = 0; i < n; ++i) {
+    if (fmt == ORC_FMT_INT4G128) {
+      uint16_t b;
+      memcpy(&b, s + 2 * i, 2);
+      if ((b & 0x7F80u) == 0x7F80u) return i;
+      continue;
+    }
+    if (fmt == ORC_FMT_FP8B128) {
+      float f;
+      memcpy(&f, s + 4 * i, 4);
+      if (!(f > 0.0f) || isinf(f)) return i;
+      continue;
+    }
     unsigned c = s[i];
     if (fmt == ORC_FMT_MXFP4) {
       if (c == 0u || c == 255u) return i;
@@ -123,6 +149,13 @@ long orc_admit_scales(int fmt, const uint8_t *s, long n) {
   return -1;
 }
 
+/* FP8B128 weights: E4M3 NaN codes (S.1111.111) are rejected; index or -1. */
+long orc_admit_fp8_codes(const uint8_t *q, long n) {
+  for (long i = 0; i < n; ++i)
+    if ((q[i] & 0x7Fu) == 0x7Fu) return i;
+  return -1;
+}
+
 static void mat_shape(const orc_layer_t *L, int m, int *rows, int *K) {
   if (m == 2) { *rows = L->H; *K = L->I; }
   else { *rows = L->I; *K = L->H; }
@@ -130,10 +163,35 @@ static void mat_shape(const orc_layer_t *L, int m, int *rows, int *K) {
 
 static int group_of(const orc_layer_t *L) { return L->fmt == ORC_FMT_MXFP4 ? 32 : 16; }
 
+/* INT4: a nibble as a two's complement integer in -8..7. */
+double orc_int4(unsigned nib) { return (double)((int)(nib & 15u) - ((nib & 8u) ? 16 : 0)); }
+
 /* Decode row r of matrix m of expert e into out[K] (fp64, exact). */
 void orc_dequant_row(const orc_layer_t *L, int m, int e, int r, double *out) {
   int rows, K;
   mat_shape(L, m, &rows, &K);
+  if (L->fmt == ORC_FMT_INT4G128) {
+    const uint8_t *codes = L->codes[m] + ((size_t)e * rows + r) * (size_t)(K / 2);
+    const uint8_t *sc = L->scales[m] + ((size_t)e * rows + r) * (size_t)(K / 128) * 2;
+    for (int c = 0; c < K; ++c) {
+      uint8_t byte = codes[c / 2];
+      unsigned nib = (c % 2 == 0) ? (byte & 15u) : (byte >> 4);
+      uint16_t sb;
+      memcpy(&sb, sc + 2 * (c / 128), 2);
+      out[c] = orc_int4(nib) * orc_bf16(sb);
+    }
+    return;
+  }
+  if (L->fmt == ORC_FMT_FP8B128) {
+    const uint8_t *codes = L->codes[m] + ((size_t)e * rows + r) * (size_t)K;
+    const uint8_t *sc = L->scales[m] + ((size_t)e * (rows / 128) + r / 128) * (size_t)(K / 128) * 4;
+    for (int c = 0; c < K; ++c) {
+      float s;
+      memcpy(&s, sc + 4 * (c / 128), 4);
+      out[c] = orc_e4m3(codes[c]) * (double)s;
+    }
+    return;
+  }
   const int G = group_of(L);
   const uint8_t *codes = L->codes[m] + ((size_t)e * rows + r) * (size_t)(K / 2);
   const uint8_t *sc = L->scales[m] + ((size_t)e * rows + r) * (size_t)(K / G);

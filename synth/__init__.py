@@ -69,19 +69,35 @@ class Workload:
 
     @property
     def group(self) -> int:
-        return 32 if self.fmt == "mxfp4" else 16
+        """Weights per block scale along K (FP8 block-128: 128 x 128 blocks)."""
+        return {"mxfp4": 32, "nvfp4": 16, "int4g128": 128, "fp8b128": 128}[self.fmt]
 
     def shape(self, m: int):
         """(rows, K) of matrix m."""
         H, I = self.hidden, self.inter
         return (I, H) if m in (GATE, UP) else (H, I)
 
+    def code_shape(self, m: int):
+        """(rows, bytes per row) of matrix m's codes."""
+        r, k = self.shape(m)
+        return (r, k) if self.fmt == "fp8b128" else (r, k // 2)
+
+    def scale_shape(self, m: int):
+        r, k = self.shape(m)
+        return (r // 128, k // 128) if self.fmt == "fp8b128" else (r, k // self.group)
+
+    @property
+    def scale_dtype(self):
+        return {"mxfp4": np.uint8, "nvfp4": np.uint8, "int4g128": np.uint16, "fp8b128": np.float32}[self.fmt]
+
     def expert_bytes(self) -> int:
         """Checkpoint bytes of one routed expert (codes + block scales [+ fp32 per-tensor])."""
         n = 0
+        item = np.dtype(self.scale_dtype).itemsize
         for m in range(3):
-            r, k = self.shape(m)
-            n += r * k // 2 + r * k // self.group
+            cr, cb = self.code_shape(m)
+            sr, sc = self.scale_shape(m)
+            n += cr * cb + sr * sc * item
         if self.fmt == "nvfp4":
             n += 3 * 4
         return n
@@ -186,12 +202,10 @@ def make_layer(wl: Workload, seed: Optional[int] = None, experts: Optional[int] 
         rank = rng_b.permutation(NT) + 1
         router_bias = (-wl.zipf_s * np.log(rank.astype(np.float64))).astype(np.float32)
 
-    G = wl.group
     codes, scales = [], []
     for m in range(3):
-        r, k = wl.shape(m)
-        codes.append(np.empty((E, r, k // 2), dtype=np.uint8))
-        scales.append(np.empty((E, r, k // G), dtype=np.uint8))
+        codes.append(np.empty((E,) + wl.code_shape(m), dtype=np.uint8))
+        scales.append(np.empty((E,) + wl.scale_shape(m), dtype=wl.scale_dtype))
     expert_ss = ss[_S_EXPERTS].spawn(E)
     n_distinct = E if experts is None else min(E, experts)
     for e in range(E):
@@ -202,14 +216,26 @@ def make_layer(wl: Workload, seed: Optional[int] = None, experts: Optional[int] 
             continue
         rng_e = np.random.Generator(np.random.PCG64(expert_ss[e]))
         for m in range(3):
-            r, k = wl.shape(m)
-            codes[m][e] = np.frombuffer(rng_e.bytes(r * k // 2), dtype=np.uint8).reshape(r, k // 2)
+            cr, cb = wl.code_shape(m)
+            ssh = wl.scale_shape(m)
+            codes[m][e] = np.frombuffer(rng_e.bytes(cr * cb), dtype=np.uint8).reshape(cr, cb)
             if wl.fmt == "mxfp4":
-                scales[m][e] = rng_e.integers(118, 125, size=(r, k // G), dtype=np.uint8)
-            else:
-                ex = rng_e.integers(7, 13, size=(r, k // G), dtype=np.uint8)
-                mant = rng_e.integers(0, 8, size=(r, k // G), dtype=np.uint8)
+                scales[m][e] = rng_e.integers(118, 125, size=ssh, dtype=np.uint8)
+            elif wl.fmt == "nvfp4":
+                ex = rng_e.integers(7, 13, size=ssh, dtype=np.uint8)
+                mant = rng_e.integers(0, 8, size=ssh, dtype=np.uint8)
                 scales[m][e] = (ex << 3) | mant
+            elif wl.fmt == "int4g128":
+                # bf16 scales 2^u * [1, 2), u in -9..-5 (|w| up to 8 * 2^-4)
+                v = np.ldexp(1.0 + rng_e.random(ssh), rng_e.integers(-9, -4, size=ssh)).astype(np.float32)
+                scales[m][e] = f32_to_bf16_bits(v)
+            else:
+                # FP8 E4M3 weights over every finite code (NaN codes S.1111.111
+                # redrawn as +-448), fp32 inverse scales 2^u * [1, 2), u in -14..-10
+                q = codes[m][e]
+                nan = (q & 0x7F) == 0x7F
+                q[nan] = q[nan] & 0xFE
+                scales[m][e] = np.ldexp(1.0 + rng_e.random(ssh), rng_e.integers(-14, -9, size=ssh)).astype(np.float32)
     global_scale = None
     if wl.fmt == "nvfp4":
         global_scale = np.full((E, 3), 2.0 ** -9, dtype=np.float32)

@@ -56,9 +56,25 @@ def tokens_with_margin(orc_layer, wl, T, seed=None, stream=0, margin=1e-3, max_r
     raise RuntimeError("could not draw tokens with the requested top-k margin")
 
 
+def int4_table():
+    """16 code values from the hand-written fixture."""
+    return np.array([float(v) for _, v in read_golden("int4_values.txt")], dtype=np.float64)
+
+
+def _torch_e4m3(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).view(torch.float8_e4m3fn) \
+        .to(torch.float64).numpy()
+
+
 def np_decode(codes: np.ndarray, scales: np.ndarray, fmt: str, gscale: float = 1.0) -> np.ndarray:
-    """Independent numpy decode of one [rows, K/2] code matrix with its scales."""
-    tab = e2m1_table()
+    """Independent numpy decode of one code matrix ([rows, K/2] nibbles, or
+    [rows, K] bytes for FP8) with its scales."""
+    if fmt == "fp8b128":
+        q = _torch_e4m3(codes)
+        s = np.repeat(np.repeat(scales.astype(np.float64), 128, axis=0), 128, axis=1)
+        return q * s
+    tab = int4_table() if fmt == "int4g128" else e2m1_table()
     lo = codes & 0x0F
     hi = codes >> 4
     q = np.empty((codes.shape[0], codes.shape[1] * 2), dtype=np.float64)
@@ -67,8 +83,10 @@ def np_decode(codes: np.ndarray, scales: np.ndarray, fmt: str, gscale: float = 1
     if fmt == "mxfp4":
         s = np.ldexp(1.0, scales.astype(np.int64) - 127)
         return q * np.repeat(s, 32, axis=1)
-    import torch
-    s = torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    if fmt == "int4g128":
+        s = synth.bf16_bits_to_f32(scales).astype(np.float64)
+        return q * np.repeat(s, 128, axis=1)
+    s = _torch_e4m3(scales)
     return q * np.repeat(s, 16, axis=1) * gscale
 
 

@@ -87,3 +87,38 @@ def check_routing_invariants(r, T, k, E):
     counts, offsets, perm, inv = oracle.permute(ids, E)
     assert np.array_equal(r["counts"], counts) and np.array_equal(r["offsets"], offsets)
     assert np.array_equal(r["perm"], perm) and np.array_equal(r["inv"], inv)
+
+
+
+def tile_list(layer):
+    """The last forward's tile list: rows (expert, first padded row, rows, first sorted position)."""
+    n = int(layer.debug_read(17, np.int32, 1)[0])
+    return layer.debug_read(16, np.int32, 4 * n).reshape(n, 4)
+
+
+def boundary_rows(layer, r, k, rng=None, extra=0, max_tiles=6):
+    """Token rows that exercise the tile scheduler of the last forward: the first
+    and last row of every tile of the hottest expert (at most max_tiles of them),
+    of the coldest active expert's tile, and of a few ragged tails (tiles
+    shorter than the longest tile, the last one of an expert that has several),
+    token 0 and the last token, plus `extra` random tokens."""
+    tiles = tile_list(layer)
+    perm = np.asarray(r["perm"])
+    counts = np.asarray(r["counts"])
+    T = np.asarray(r["ids"]).shape[0]
+    active = np.nonzero(counts > 0)[0]
+    hot = int(np.argmax(counts))
+    cold = int(active[np.argmin(counts[active])])
+    pick = list(np.nonzero(tiles[:, 0] == hot)[0][:max_tiles]) + list(np.nonzero(tiles[:, 0] == cold)[0][:1])
+    longest = int(tiles[:, 2].max())
+    multi = np.nonzero(np.bincount(tiles[:, 0], minlength=counts.size) > 1)[0]
+    tails = [i for i in range(len(tiles)) if tiles[i, 2] < longest and tiles[i, 0] in multi]
+    pick += tails[:: max(1, len(tails) // 3)][:3]
+    pos = set()
+    for i in pick:
+        _, _, n, s0 = (int(v) for v in tiles[i])
+        pos.update({s0, s0 + n - 1})
+    rows = {int(perm[p]) // k for p in pos} | {0, T - 1}
+    if extra and rng is not None:
+        rows |= set(int(v) for v in rng.integers(0, T, extra))
+    return np.array(sorted(rows), dtype=np.int32)

@@ -59,8 +59,10 @@ def test_plan_sizes(F):
 @pytest.mark.parametrize("bad, status", [
     (dict(hidden=300), 1), (dict(inter=100), 1), (dict(n_experts=0), 1), (dict(top_k=0), 1),
     (dict(top_k=9, n_experts=8), 1), (dict(shared_inter=64), 1), (dict(fmt=7), 1),
-    (dict(renormalize=0), 6), (dict(n_slots=65), 1), (dict(max_tokens=0), 1),
-    (dict(n_slots=10, n_staging=1), 1),
+    (dict(renormalize=2), 1), (dict(n_slots=65), 1), (dict(max_tokens=0), 1),
+    (dict(n_slots=10, n_staging=1), 1), (dict(scoring=2), 1), (dict(n_sinks=-1), 1),
+    (dict(n_sinks=961), 1), (dict(shared_gate=1), 1), (dict(out_dtype=2), 1),
+    (dict(top_k=11, n_experts=8, n_sinks=2), 1),
 ])
 def test_config_validation(F, bad, status):
     cfg = F.make_config(2048, 1024, 64, 8, max_tokens=8)
@@ -69,6 +71,33 @@ def test_config_validation(F, bad, status):
     with pytest.raises(F.MoEError) as ei:
         F.plan(cfg)
     assert ei.value.status == status
+
+
+@pytest.mark.parametrize("variant", [
+    dict(renormalize=0), dict(scoring=1), dict(scoring=1, renormalize=0), dict(n_sinks=2, top_k=10),
+    dict(n_sinks=960), dict(shared_inter=256, shared_gate=1), dict(out_dtype=1),
+])
+def test_router_variants_and_output_dtype_are_valid_configurations(F, variant):
+    """Routing semantics a checkpoint declares are configuration: each of these
+    plans without error, and sink targets and a shared-expert gate row add
+    router rows to the resident bytes."""
+    cfg = F.make_config(2048, 1024, 64, 8, max_tokens=8)
+    base = F.plan(cfg)["resident_bytes"]
+    for k, v in variant.items():
+        setattr(cfg, k, v)
+    p = F.plan(cfg)
+    extra_rows = variant.get("n_sinks", 0) + variant.get("shared_gate", 0)
+    extra_shared = 3 * variant.get("shared_inter", 0) * 2048 * 2
+    assert p["resident_bytes"] == base + extra_rows * (2048 * 4 + 4) + extra_shared
+
+
+def test_shared_gate_needs_its_weights(F):
+    wl = synth.custom_workload(256, 128, 4, 2, shared_inter=128)
+    lw = synth.make_layer(wl, seed=1)
+    cfg = F.make_config(256, 128, 4, 2, shared_inter=128, max_tokens=4, shared_gate=True)
+    with pytest.raises(F.MoEError) as ei:
+        F.admit(cfg, F.weights_from_layer(lw))
+    assert ei.value.status == 1 and "shared_gate_w" in str(ei.value)
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
@@ -90,6 +119,42 @@ def test_admission_rejects_bad_scale_codes(F, fmt):
         lw3.global_scale[1, 0] = -1.0
         with pytest.raises(F.MoEError):
             F.admit(cfg, F.weights_from_layer(lw3))
+
+
+@pytest.mark.parametrize("fmt", ["int4g128", "fp8b128"])
+def test_admission_of_other_formats(F, fmt):
+    """INT4: non-finite bf16 scales are rejected; FP8: non-positive or
+    non-finite fp32 scales and E4M3 NaN weights are rejected; A4 numerics is
+    refused for both (it quantises activations to an FP4 format)."""
+    wl = synth.custom_workload(256, 128, 4, 2, fmt=fmt)
+    lw = synth.make_layer(wl, seed=2)
+    cfg = F.make_config(256, 128, 4, 2, fmt=fmt, max_tokens=4)
+    F.admit(cfg, F.weights_from_layer(lw))
+    bad = synth.make_layer(wl, seed=2)
+    if fmt == "int4g128":
+        bad.scales[1][3, 5, 0] = 0x7FC0          # NaN bf16
+    else:
+        bad.scales[1][3, 0, 1] = -0.5
+    with pytest.raises(F.MoEError) as ei:
+        F.admit(cfg, F.weights_from_layer(bad))
+    assert ei.value.status == 2 and "expert 3 matrix 1" in str(ei.value)
+    if fmt == "fp8b128":
+        bad = synth.make_layer(wl, seed=2)
+        bad.codes[0][1, 2, 3] = 0x7F
+        with pytest.raises(F.MoEError) as ei:
+            F.admit(cfg, F.weights_from_layer(bad))
+        assert ei.value.status == 2 and "NaN" in str(ei.value)
+    cfg_a4 = F.make_config(256, 128, 4, 2, fmt=fmt, numerics="a4", max_tokens=4)
+    with pytest.raises(F.MoEError) as ei:
+        F.plan(cfg_a4)
+    assert ei.value.status == 6
+
+
+@pytest.mark.parametrize("fmt", ["int4g128", "fp8b128"])
+def test_plan_sizes_of_other_formats(F, fmt):
+    wl = synth.custom_workload(2048, 1024, 8, 2, fmt=fmt)
+    p = F.plan(F.make_config(2048, 1024, 8, 2, fmt=fmt, max_tokens=4))
+    assert wl.expert_bytes() <= p["expert_bytes"] < wl.expert_bytes() + 6 * 256
 
 
 def test_a4_not_silently_substituted(F):

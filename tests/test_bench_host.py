@@ -70,3 +70,29 @@ def test_clock_record_reports_median_and_throttle_reasons(rows, reasons):
 def test_clock_record_without_nvidia_smi():
     rec = bench.ClockSampler(None).stop()
     assert rec["samples"] == 0 and rec["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_binding_roof_takes_the_slowest_resource_plus_serial_stages():
+    wl = synth.workload("qwen3_8_flash_next_like")
+    T, act = 8192, 500
+    miss = 450 * 7077900
+    r = bench.binding_roof(wl, T, act, miss, 50.0, 6500.0, 1400.0, 1.5, 80.0)
+    assert r["binding"] == "pcie"
+    assert r["t_pcie_ms"] == pytest.approx(miss / 50e9 * 1e3)
+    assert r["t_hbm_ms"] == pytest.approx(bench.layer_bytes(wl, act, T) / 6500e9 * 1e3)
+    flops = 6.0 * T * 10 * 4096 * 1024 + 6.0 * T * 4096 * 1024
+    assert r["t_tc_ms"] == pytest.approx(flops / 1400e12 * 1e3)
+    assert r["tau_ms"] == pytest.approx(r["t_pcie_ms"] + 1.5)
+    assert r["frac_of_tau"] == pytest.approx(r["tau_ms"] / 80.0)
+    # all resident: nothing staged, the tensor work binds
+    r = bench.binding_roof(wl, T, act, 0, 50.0, 6500.0, 1400.0, 1.5, 3.0)
+    assert r["binding"] == "tc" and r["t_pcie_ms"] == 0.0
+
+
+def test_default_workload_is_the_largest_single_gpu_layer():
+    a = bench.parse([])
+    wl = synth.workload(a.workload)
+    assert a.workload == "qwen3_8_flash_next_like" and a.tokens == wl.prefill_tokens == 8192
+    assert a.slots == "workload" and a.numerics == "exact" and a.warmup >= 3
+    sizes = {n: w.n_experts * w.expert_bytes() for n, w in synth.WORKLOADS.items()}
+    assert max(sizes, key=sizes.get) == a.workload

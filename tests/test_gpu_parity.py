@@ -111,7 +111,9 @@ def _paged_case(name, Ts, sample=8):
             assert st["last_misses"] >= 0
             lg, ids, g = L.route_all(x)
             G.check_routing(rp, lg, ids, g, wl.n_experts)
-            rows = np.unique(np.concatenate([[0, T - 1], rng.integers(0, T, sample)]))
+            # tile-scheduler classes (hottest / coldest expert, tile boundaries,
+            # ragged tails) plus random rows
+            rows = G.boundary_rows(resident, rr, wl.top_k, rng=rng, extra=sample)
             y_ref, *_ = L.forward(x, rows=rows)
             G.check_output(yp[rows], y_ref)
         assert paged.stats()["misses"] > 0, "the paged layer never staged an expert"

@@ -1,0 +1,117 @@
+"""Library-managed residency (moe_set_policy / moe_prefetch): an adaptive cache
+of experts in HBM slots over the pinned store.  Whatever the policy, a forward
+computes the same thing: every output here is compared bit for bit with the
+all-resident layer's output for the same tokens.
+"""
+import numpy as np
+import pytest
+
+import synth
+from tests import _gpu as G
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pair():
+    wl = synth.custom_workload(512, 256, 16, 2, shared_inter=128, zipf_s=1.1, n_slots=4)
+    lw = synth.make_layer(wl, seed=51)
+    resident = G.make_layer(lw, n_slots=wl.n_experts, max_tokens=64)
+    yield wl, lw, resident
+    resident.close()
+
+
+def _batches(wl, n, T, seed):
+    return [synth.make_tokens(wl, T, seed=seed, stream=i) for i in range(n)]
+
+
+@pytest.mark.parametrize("fmt_T", [("mxfp4", 2), ("mxfp4", 48)])
+def test_cache_policy_admits_misses_and_keeps_outputs(pair, fmt_T):
+    wl, lw, resident = pair
+    _, T = fmt_T
+    layer = G.make_layer(lw, n_slots=4, max_tokens=64, n_staging=2)
+    try:
+        layer.set_policy("cache")
+        assert layer.stats()["policy"] == 2
+        x = synth.make_tokens(wl, T, seed=7)
+        y0, r0 = G.run(layer, x)
+        yr, _ = G.run(resident, x)
+        assert np.array_equal(y0, yr)
+        first_misses = layer.stats()["last_misses"]
+        assert first_misses > 0 and layer.stats()["admitted"] > 0
+        # the same batch again: the admitted experts now hit
+        y1, _ = G.run(layer, x)
+        assert np.array_equal(y1, yr)
+        assert layer.stats()["last_misses"] < first_misses
+        # a stream of different batches: outputs stay identical to the resident layer
+        for xb in _batches(wl, 5, T, 9):
+            yb, _ = G.run(layer, xb)
+            yrb, _ = G.run(resident, xb)
+            assert np.array_equal(yb, yrb)
+    finally:
+        layer.close()
+
+
+def test_hybrid_policy_never_evicts_pinned_slots(pair):
+    wl, lw, resident = pair
+    layer = G.make_layer(lw, n_slots=4, max_tokens=64, n_staging=2)
+    try:
+        table = synth.slot_table(lw, 4)                 # hottest first: slots 0..3
+        pinned = {int(e) for e in np.nonzero((table >= 0) & (table < 2))[0]}
+        layer.set_policy("hybrid", n_pinned=2)
+        for xb in _batches(wl, 6, 16, 13):
+            yb, _ = G.run(layer, xb)
+            yrb, _ = G.run(resident, xb)
+            assert np.array_equal(yb, yrb)
+        assert layer.stats()["admitted"] > 0
+        # a pinned expert is still resident: a batch routed only to pinned experts has no misses
+        # (checked through the routing of the resident layer on a probe batch)
+        probe = synth.make_tokens(wl, 8, seed=77)
+        _, rr = G.run(resident, probe)
+        need = set(np.unique(rr["ids"]).tolist())
+        G.run(layer, probe)
+        missed = layer.stats()["last_misses"]
+        assert missed <= len(need - pinned)
+    finally:
+        layer.close()
+
+
+def test_none_policy_stages_everything(pair):
+    wl, lw, resident = pair
+    layer = G.make_layer(lw, n_slots=4, max_tokens=64, n_staging=2)
+    try:
+        layer.set_policy("none")
+        x = synth.make_tokens(wl, 8, seed=5)
+        y, r = G.run(layer, x)
+        yr, _ = G.run(resident, x)
+        assert np.array_equal(y, yr)
+        assert layer.stats()["last_misses"] == len(np.unique(r["ids"]))
+        assert layer.stats()["admitted"] == 0
+    finally:
+        layer.close()
+
+
+def test_prefetch_of_predicted_experts_removes_misses(pair):
+    """A perfect predictor (the resident layer's routing of the next batch):
+    after moe_prefetch the next forward stages nothing, and its output is
+    unchanged; prefetch outside the cache policies is refused."""
+    F = G.library()
+    wl, lw, resident = pair
+    layer = G.make_layer(lw, n_slots=4, max_tokens=64, n_staging=2)
+    try:
+        x = synth.make_tokens(wl, 2, seed=21)
+        with pytest.raises(F.MoEError) as ei:
+            layer.prefetch([0, 1])
+        assert ei.value.status == 1
+        layer.set_policy("cache")
+        _, rr = G.run(resident, x)
+        need = np.unique(rr["ids"])
+        assert need.size <= 4
+        layer.prefetch(need)
+        y, _ = G.run(layer, x)
+        yr, _ = G.run(resident, x)
+        assert np.array_equal(y, yr)
+        assert layer.stats()["last_misses"] == 0
+        assert layer.stats()["prefetched"] > 0
+    finally:
+        layer.close()

@@ -183,6 +183,67 @@ def test_sink_choice_contributes_nothing():
         synth.make_layer(synth.custom_workload(64, 32, 4, 2), seed=21), x)[0]).max()
 
 
+def test_int4_matches_fixture_table():
+    tab = cs.int4_table()
+    assert [oracle.int4(c) for c in range(16)] == tab.tolist()
+
+
+def test_int4g128_row_hand_built():
+    """One row of 256 weights: group 0 scale 2^-3, group 1 scale 1.5 (bf16
+    0x3FC0); codes 7 and 8 (= -8) at the group edges."""
+    wl = synth.custom_workload(256, 128, 1, 1, fmt="int4g128")
+    lw = synth.make_layer(wl, seed=1)
+    lw.codes[0][0, 0, :] = 0
+    lw.codes[0][0, 0, 0] = 0x87          # element 0 -> 7, element 1 -> -8
+    lw.codes[0][0, 0, 63] = 0x10         # element 126 -> 0, element 127 -> 1
+    lw.codes[0][0, 0, 64] = 0x0F         # element 128 -> -1, element 129 -> 0
+    lw.scales[0][0, 0, :] = [0x3E00, 0x3FC0]   # bf16 0.125, 1.5
+    L = oracle.Layer.from_weights(lw)
+    row = L.dequant(0, 0)[0]
+    want = np.zeros(256)
+    want[0], want[1], want[127], want[128] = 7 * 0.125, -8 * 0.125, 0.125, -1.5
+    assert np.array_equal(row, want)
+
+
+def test_fp8b128_blocks_hand_built():
+    """Down matrix [256, 128]: rows 0..127 use block scale 0.5, rows 128..255
+    scale 3.0; E4M3 codes 0x38 (1.0), 0xC0 (-2.0), 0x7E (448)."""
+    wl = synth.custom_workload(256, 128, 1, 1, fmt="fp8b128")
+    lw = synth.make_layer(wl, seed=1)
+    lw.codes[2][0] = 0
+    lw.codes[2][0, 0, 0] = 0x38
+    lw.codes[2][0, 127, 5] = 0xC0
+    lw.codes[2][0, 128, 127] = 0x7E
+    lw.scales[2][0] = np.array([[0.5], [3.0]], np.float32)
+    W = oracle.Layer.from_weights(lw).dequant(2, 0)
+    want = np.zeros((256, 128))
+    want[0, 0], want[127, 5], want[128, 127] = 0.5, -1.0, 1344.0
+    assert np.array_equal(W, want)
+
+
+@pytest.mark.parametrize("fmt", ["int4g128", "fp8b128"])
+def test_other_formats_dequant_matches_numpy(fmt):
+    wl = synth.custom_workload(256, 128, 2, 1, fmt=fmt)
+    lw = synth.make_layer(wl, seed=6)
+    L = oracle.Layer.from_weights(lw)
+    for m in range(3):
+        for e in range(2):
+            ref = cs.np_decode(lw.codes[m][e], lw.scales[m][e], fmt)
+            assert np.array_equal(L.dequant(m, e), ref)
+
+
+def test_other_formats_admission():
+    s = np.array([0x3F80, 0x7F80, 0x0000, 0xFFC1], np.uint16)        # 1.0, +inf, 0, NaN
+    assert oracle.admit_scales("int4g128", s) == 1
+    assert oracle.admit_scales("int4g128", s[[0, 2]]) == -1          # a zero bf16 scale is admitted
+    f = np.array([1.0, 2.0 ** -20, 0.0, -1.0], np.float32)
+    assert oracle.admit_scales("fp8b128", f) == 2
+    assert oracle.admit_scales("fp8b128", f[:2]) == -1
+    assert oracle.admit_scales("fp8b128", np.array([np.inf], np.float32)) == 0
+    assert oracle.admit_fp8_codes(np.array([0x00, 0x7E, 0xFE, 0xFF], np.uint8)) == 3
+    assert oracle.admit_fp8_codes(np.array([0x7F], np.uint8)) == 0
+
+
 def test_route_tie_goes_to_lower_index():
     l = np.array([0.5, 2.0, 1.0, 2.0, 1.0, -3.0], dtype=np.float32)
     ids, g = oracle.route_row(l, 4)
@@ -237,6 +298,9 @@ def test_single_expert_is_dense_swiglu(fmt):
     dict(hidden=64, inter=32, n_experts=4, top_k=3, n_sinks=2),
     dict(hidden=128, inter=64, n_experts=5, top_k=3, shared_inter=32, shared_gate=True, n_sinks=2,
          scoring="sigmoid", renormalize=False, zipf_s=1.1, fmt="nvfp4"),
+    # other expert formats: INT4 group-128 (bf16 scales), FP8 E4M3 block-128 (fp32 scales)
+    dict(hidden=256, inter=128, n_experts=4, top_k=2, fmt="int4g128"),
+    dict(hidden=256, inter=128, n_experts=4, top_k=2, fmt="fp8b128", shared_inter=128),
 ])
 def test_bruteforce_dense_tiny(shape):
     wl = synth.custom_workload(**shape)
