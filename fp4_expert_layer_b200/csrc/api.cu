@@ -98,7 +98,6 @@ struct moe_layer {
   float *router_parts = nullptr;     // split-K partial logits of the prefill router GEMM
   uint16_t *shared_w[3] = {};
   uint8_t *slots = nullptr, *staging = nullptr;
-  const uint8_t **ptr_resident = nullptr, **ptr_pass = nullptr;
   int *loc_resident = nullptr, *loc_pass = nullptr;
   CodeMaps maps{};
   int *h_err = nullptr, *d_err = nullptr;   // mapped pinned error word (bounded device waits)
@@ -135,7 +134,6 @@ struct moe_layer {
   // host
   uint8_t *store = nullptr;          // pinned: E x blob bytes
   int *h_counts = nullptr;           // pinned [E]
-  const uint8_t **h_ptr = nullptr;   // pinned [E]
   int *h_loc = nullptr;              // pinned [E]
   std::vector<int> slot_of;
   int n_resident = 0;
@@ -300,7 +298,7 @@ static size_t tc_scratch_bytes(const moe_config_t *c) {
 
 static size_t scratch_bytes(const moe_config_t *c) {
   const Sizes z = sizes_of(c);
-  const size_t T = c->max_tokens, H = c->hidden, I = c->inter, E = c->n_experts, Is = c->shared_inter;
+  const size_t T = c->max_tokens, H = c->hidden, I = c->inter, Is = c->shared_inter;
   size_t b = 0;
   const size_t NT = n_targets(c), NR = n_logit_rows(c);
   b += align256(T * NR * 4) + align256(z.P * 4) * 4 + align256(NT * 4) + align256((NT + 1) * 4);
@@ -311,8 +309,7 @@ static size_t scratch_bytes(const moe_config_t *c) {
   if (Is) b += align256(T * Is * 2) + align256(T * H * 4);
   b += align256(((T + 3) / 4) * 4) + align256(4) + align256(T * (H / 128) * 4);
   b += align256(T * H * 2) + align256(T * H * 4);
-  b += 2 * align256(E * sizeof(void *));
-  if (T >= 256) b += align256((size_t)(4 << 20) * 4);     // split-K partial logits (prefill router)
+    if (T >= 256) b += align256((size_t)(4 << 20) * 4);     // split-K partial logits (prefill router)
   return b;
 }
 
@@ -346,7 +343,6 @@ static void free_layer(moe_layer *L) {
   for (void *p : L->dev) cudaFree(p);
   if (L->store) cudaFreeHost(L->store);
   if (L->h_counts) cudaFreeHost(L->h_counts);
-  if (L->h_ptr) cudaFreeHost(L->h_ptr);
   if (L->h_err) cudaFreeHost(L->h_err);
   if (L->h_loc) cudaFreeHost(L->h_loc);
   for (int i = 0; i < 2; ++i) {
@@ -454,13 +450,13 @@ static moe_status_t make_tc_weight_map(CUtensorMap *map, const uint8_t *region, 
   return MOE_OK;
 }
 
-// bf16 row-major [rows, K] map, box 64 elements (128 B) x 128 rows, 128-byte swizzle.
-static moe_status_t make_bf16_map(CUtensorMap *map, const void *base, size_t K, size_t rows) {
+// bf16 row-major [rows, K] map, box 64 elements (128 B) x box_rows rows, 128-byte swizzle.
+static moe_status_t make_bf16_map(CUtensorMap *map, const void *base, size_t K, size_t rows, int box_rows = 128) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(K * 2)};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -517,18 +513,14 @@ static std::vector<int> plan_admission(const moe_layer *L, const std::vector<int
 // are pageable, so the call returns once they have been read.
 static moe_status_t push_table(moe_layer *L, cudaStream_t s) {
   const int E = L->cfg.n_experts;
-  const size_t bytes = L->L.bytes;
   std::vector<int> loc(E);
-  std::vector<const uint8_t *> ptr(E);
   int n = 0;
   for (int e = 0; e < E; ++e) {
     const int v = L->slot_of[e];
     loc[e] = v >= 0 ? v : kLocAbsent;
-    ptr[e] = v >= 0 ? L->slots + (size_t)v * bytes : nullptr;
     n += v >= 0;
   }
   CUDA_TRY(cudaMemcpyAsync(L->loc_resident, loc.data(), sizeof(int) * E, cudaMemcpyHostToDevice, s));
-  CUDA_TRY(cudaMemcpyAsync(L->ptr_resident, ptr.data(), sizeof(void *) * E, cudaMemcpyHostToDevice, s));
   L->n_resident = n;
   L->table_version += 1;
   return MOE_OK;
@@ -767,7 +759,6 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     for (auto &x : th) x.join();
   }
   if (cudaHostAlloc((void **)&L->h_counts, sizeof(int) * E, cudaHostAllocDefault) != cudaSuccess ||
-      cudaHostAlloc((void **)&L->h_ptr, sizeof(void *) * E, cudaHostAllocDefault) != cudaSuccess ||
       cudaHostAlloc((void **)&L->h_loc, sizeof(int) * E, cudaHostAllocDefault) != cudaSuccess ||
       cudaHostAlloc((void **)&L->h_err, sizeof(int), cudaHostAllocMapped) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -782,8 +773,6 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   if (Is) for (int m = 0; m < 3; ++m) C_TRY(dalloc(L, &L->shared_w[m], (size_t)Is * H * 2));
   if (cfg->n_slots) C_TRY(dalloc(L, &L->slots, bytes * cfg->n_slots));
   if (L->n_staging) C_TRY(dalloc(L, &L->staging, bytes * L->n_staging));
-  C_TRY(dalloc(L, &L->ptr_resident, sizeof(void *) * E));
-  C_TRY(dalloc(L, &L->ptr_pass, sizeof(void *) * E));
   C_TRY(dalloc(L, &L->loc_resident, sizeof(int) * E));
   C_TRY(dalloc(L, &L->loc_pass, sizeof(int) * E));
   C_TRY(dalloc(L, &L->logits, T * NR * 4));
@@ -866,8 +855,6 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   C_CUDA(cudaMemsetAsync(L->router_counter, 0, ((T + 3) / 4) * 4, s));
   C_CUDA(cudaMemsetAsync(L->tiles_done, 0, 4, s));
   C_CUDA(cudaMemsetAsync(L->comb_cnt, 0, T * (H / 128) * 4, s));
-  C_CUDA(cudaMemsetAsync(L->ptr_resident, 0, sizeof(void *) * E, s));
-  C_CUDA(cudaMemsetAsync(L->ptr_pass, 0, sizeof(void *) * E, s));
   C_CUDA(cudaMemsetAsync(L->loc_resident, 0xFF, sizeof(int) * E, s));   // -1: absent
   C_CUDA(cudaMemsetAsync(L->loc_pass, 0xFF, sizeof(int) * E, s));
   *L->h_err = 0;
@@ -914,7 +901,6 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   L->slot_of.assign(E, -1);
   L->expert_of_slot.assign(cfg->n_slots, -1);
   L->last_use.assign(E, 0);
-  for (int e = 0; e < E; ++e) L->h_ptr[e] = nullptr;
   L->st.expert_bytes = bytes;
   L->st.pinned_bytes = bytes * E;
   size_t dev_total = (size_t)NR * H * 4 + (size_t)3 * Is * H * 2 + bytes * (cfg->n_slots + L->n_staging) +
@@ -958,10 +944,8 @@ moe_status_t moe_set_slot_table(moe_layer_t L, const int32_t *table, void *strea
     if (s >= 0 && L->slot_of[e] != s)
       CUDA_TRY(cudaMemcpyAsync(L->slots + (size_t)s * bytes, L->store + (size_t)e * bytes, bytes,
                                cudaMemcpyHostToDevice, st));
-    L->h_ptr[e] = s >= 0 ? L->slots + (size_t)s * bytes : nullptr;
     L->h_loc[e] = s >= 0 ? s : kLocAbsent;
   }
-  CUDA_TRY(cudaMemcpyAsync(L->ptr_resident, L->h_ptr, sizeof(void *) * E, cudaMemcpyHostToDevice, st));
   CUDA_TRY(cudaMemcpyAsync(L->loc_resident, L->h_loc, sizeof(int) * E, cudaMemcpyHostToDevice, st));
   CUDA_TRY(cudaStreamSynchronize(st));
   for (int e = 0; e < E; ++e) L->slot_of[e] = table[e];
@@ -1320,52 +1304,47 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     CUDA_TRY(cudaEventRecord(L->ev_counts, s));
   }
 
-  // always-resident shared expert (runs while the host builds the miss list)
-  const bool dense_tc = Is && big_batch;
-  if (dense_tc) {
+  // always-resident shared expert (runs while the host builds the miss list),
+  // bf16 on the tensor core: decode-sized batches (T <= 128) split K over a
+  // thread-block cluster per row block, larger ones run persistent tiles of
+  // 128 tokens.  Its operands are read by TMA, which needs x 16-byte aligned:
+  // an unaligned x is first copied to the layer's own buffer.
+  if (Is) {
     StageTimer t2(L, 2, s);
+    const void *xs = x;
+    if (!x16) {
+      CUDA_TRY(cudaMemcpyAsync(L->xin, x, (size_t)T * H * 2, cudaMemcpyDeviceToDevice, s));
+      xs = L->xin;
+    }
     DenseTcArgs d{};
     d.wmap[0] = L->sh_map[0];
     d.wmap[1] = L->sh_map[1];
-    ST_TRY(make_bf16_map(&d.xmap, x, H, T));
     d.T = T; d.K = H; d.rows = Is; d.n_rowblocks = Is / 128;
-    d.grid = std::min(((T + 127) / 128) * d.n_rowblocks, L->n_sms);
     d.h_out = L->sh_h;
-    d.err = L->d_err;
-    launch_dense_tc(MODE_GATEUP, d, s);
-    CUDA_TRY(cudaGetLastError());
-    d.wmap[0] = L->sh_map[2];
-    d.xmap = L->sh_hmap;
-    d.K = Is; d.rows = H; d.n_rowblocks = H / 256;
-    d.grid = std::min(((T + 127) / 128) * d.n_rowblocks, L->n_sms);
     d.s_out = L->sh_s;
-    launch_dense_tc(MODE_DOWN, d, s);
-    CUDA_TRY(cudaGetLastError());
-    t2.launched(2);
-    t2.end();
-  } else if (Is) {
-    StageTimer t2(L, 2, s);
-    const int snt = T <= 8 ? 1 : (T <= 16 ? 2 : 4);
-    const int stiles = (T + 8 * snt - 1) / (8 * snt);
-    ExpertArgs a{};
-    a.tile_tokens = 8 * snt;
-    a.T = T;
-    a.dense_w0 = L->shared_w[0];
-    a.dense_w1 = L->shared_w[1];
-    a.K = H; a.rows = Is; a.n_rowblocks = Is / 128;
-    a.k_split = pick_split(stiles * (Is / 128), H / 128);
-    a.act = reinterpret_cast<const uint16_t *>(x);
-    a.h_out = L->sh_h;
-    launch_expert(WF_BF16, MODE_GATEUP, snt, a, stiles, s);
-    CUDA_TRY(cudaGetLastError());
-    a.dense_w0 = L->shared_w[2];
-    a.dense_w1 = nullptr;
-    a.K = Is; a.rows = H; a.n_rowblocks = H / 256;
-    a.k_split = pick_split(stiles * (H / 256), Is / 128);
-    a.act = L->sh_h;
-    a.o_out = L->sh_s;
-    launch_expert(WF_BF16, MODE_DOWN, snt, a, stiles, s);
-    CUDA_TRY(cudaGetLastError());
+    d.err = L->d_err;
+    if (T <= 128) {
+      const int np = dense_splitk_rows(T);
+      ST_TRY(make_bf16_map(&d.xmap, xs, H, T, np));
+      launch_dense_splitk(MODE_GATEUP, d, dense_splitk_ways(d.n_rowblocks, H, L->n_sms), s);
+      CUDA_TRY(cudaGetLastError());
+      d.wmap[0] = L->sh_map[2];
+      ST_TRY(make_bf16_map(&d.xmap, L->sh_h, Is, T, np));
+      d.K = Is; d.rows = H; d.n_rowblocks = H / 256;
+      launch_dense_splitk(MODE_DOWN, d, dense_splitk_ways(d.n_rowblocks, Is, L->n_sms), s);
+      CUDA_TRY(cudaGetLastError());
+    } else {
+      ST_TRY(make_bf16_map(&d.xmap, xs, H, T));
+      d.grid = std::min(((T + 127) / 128) * d.n_rowblocks, L->n_sms);
+      launch_dense_tc(MODE_GATEUP, d, s);
+      CUDA_TRY(cudaGetLastError());
+      d.wmap[0] = L->sh_map[2];
+      d.xmap = L->sh_hmap;
+      d.K = Is; d.rows = H; d.n_rowblocks = H / 256;
+      d.grid = std::min(((T + 127) / 128) * d.n_rowblocks, L->n_sms);
+      launch_dense_tc(MODE_DOWN, d, s);
+      CUDA_TRY(cudaGetLastError());
+    }
     t2.launched(2);
     t2.end();
   }

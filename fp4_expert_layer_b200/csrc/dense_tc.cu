@@ -12,11 +12,15 @@
 // 2..5 read the double-buffered accumulators back: gate/up writes h (bf16
 // [T, I_s]), down writes s (fp32 [T, H]) for the ordered combine.
 // All mbarrier waits are bounded.
+#include <cooperative_groups.h>
+
 #include "device_utils.cuh"
 #include "launch.cuh"
 #include "moe_internal.h"
 #include "tcgen05.cuh"
 #include "tma.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace moe {
 
@@ -242,6 +246,217 @@ void launch_dense_tc(int mode, const DenseTcArgs &a, cudaStream_t s) {
   if (a.grid <= 0) return;
   if (mode == MODE_GATEUP) launch_dense_one<MODE_GATEUP, 128>(a, s);
   else launch_dense_one<MODE_DOWN, 128>(a, s);
+}
+
+// ---------------------------------------------------------------------------
+// Decode-sized batches (T <= 128): the weight stream is what costs, and one
+// CTA per row block would leave most SMs idle, so K is split over a
+// thread-block cluster of S CTAs.  CTA ks of the cluster for row block rb
+// accumulates its 128 gate + 128 up rows (or 256 down rows) over the K slabs
+// [ks * nslab / S, (ks + 1) * nslab / S) for all T tokens at once (N = T
+// rounded up to 16; TMA zero-fills the rows past T), copies the partial
+// accumulators to its shared memory, and the cluster sums them in rank order
+// through distributed shared memory (the same order every run, so the result
+// does not depend on timing), each CTA finishing 128 / S of the rows.
+// Roles: warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 epilogue.
+// ---------------------------------------------------------------------------
+namespace {
+template <int NP>
+struct SplitGeom {
+  static constexpr int STAGES = NP <= 32 ? 6 : (NP <= 64 ? 5 : 4);
+  static constexpr int A_BYTES = 2 * 128 * 128;   // two 128-row x 64-element bf16 tiles
+  static constexpr int B_OFF = A_BYTES;
+  static constexpr int B_BYTES = NP * 128;
+  static constexpr int STAGE = (A_BYTES + B_BYTES + 1023) / 1024 * 1024;
+  static constexpr int COLS = 2 * NP;
+  static constexpr int TMEM_COLS = COLS <= 32 ? 32 : (COLS <= 64 ? 64 : (COLS <= 128 ? 128 : 256));
+  static constexpr int RED_BYTES = 2 * 128 * NP * 4;   // partial accumulators, fp32
+  static constexpr size_t SMEM = (size_t)(STAGES * STAGE > RED_BYTES ? STAGES * STAGE : RED_BYTES) + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared-memory budget");
+};
+}  // namespace
+
+template <int MODE, int NP>
+__global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __grid_constant__ DenseTcArgs a) {
+  using Geo = SplitGeom<NP>;
+  constexpr int SN = Geo::STAGES;
+  extern __shared__ __align__(1024) uint8_t sk_smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[SN];
+  __shared__ __align__(8) uint64_t empty_bar[SN];
+  __shared__ __align__(8) uint64_t accf_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int ok_s;
+
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sk_smem_raw) + 1023) & ~uintptr_t(1023));
+  float *red = reinterpret_cast<float *>(smem);       // [2][128][NP], over the stages once they are consumed
+  cg::cluster_group cluster = cg::this_cluster();
+  const int S = (int)cluster.num_blocks();
+  const int ks = (int)cluster.block_rank();
+  const int rb = blockIdx.x / S;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nslab = a.K / 64;
+  const int s0 = ks * nslab / S, s1 = (ks + 1) * nslab / S;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SN; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    mbar_init(smem_u32(&accf_bar), 1);
+    mbar_fence_init();
+    ok_s = 1;
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_base_s), Geo::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  wait_prior_grid();                                   // x / h come from earlier kernels
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      bool failed = false;
+      for (int slab = s0; slab < s1; ++slab) {
+        if (issued >= SN && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 46)) { failed = true; break; }
+        const uint32_t bar = smem_u32(&full_bar[s]);
+        const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+        mbar_arrive_expect_tx(bar, (uint32_t)(Geo::A_BYTES + Geo::B_BYTES));
+        if constexpr (MODE == MODE_GATEUP) {
+          tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 128);
+          tma_load_2d(st + 16384, &a.wmap[1], bar, slab * 64, rb * 128);
+        } else {
+          tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 256);
+          tma_load_2d(st + 16384, &a.wmap[0], bar, slab * 64, rb * 256 + 128);
+        }
+        tma_load_2d(st + Geo::B_OFF, &a.xmap, bar, slab * 64, 0);
+        ++issued;
+        if (++s == SN) { s = 0; ph ^= 1u; }
+      }
+      if (failed) {
+        int s2 = 0;
+        uint32_t ph2 = 0;
+        for (int i = 0; i < issued; ++i) {
+          if (i >= issued - SN) mbar_drain(smem_u32(&full_bar[s2]), ph2);
+          if (++s2 == SN) { s2 = 0; ph2 ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool failed = false;
+      const uint32_t idesc = idesc_bf16(128, NP);
+      for (int slab = s0; slab < s1; ++slab) {
+        if (!mbar_wait(smem_u32(&full_bar[s]), ph, a.err, 47)) { failed = true; break; }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bdesc = umma_desc(st + Geo::B_OFF + 32 * kk, 16, 1024, 2);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint64_t adesc = umma_desc(st + h * 16384 + 32 * kk, 16, 1024, 2);
+            umma_bf16(tmem + (uint32_t)(h * NP), adesc, bdesc, idesc, (slab > s0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(smem_u32(&empty_bar[s]));
+        if (++s == SN) { s = 0; ph ^= 1u; }
+      }
+      // completes once every MMA above has (or at once, with none issued)
+      tc_commit(smem_u32(&accf_bar));
+      if (failed) ok_s = 0;
+    }
+  } else {
+    // epilogue warps: partial accumulators -> shared memory (rows 32*quad + lane)
+    const int quad = warp & 3;
+    const bool ok = mbar_wait(smem_u32(&accf_bar), 0, a.err, 48);
+    tc_fence_after();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = 32 * quad + lane;
+#pragma unroll
+      for (int c0 = 0; c0 < NP; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + (uint32_t)(h * NP + c0) + ((uint32_t)(32 * quad) << 16), v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) red[(h * 128 + row) * NP + c0 + j] = ok ? __uint_as_float(v[j]) : 0.0f;
+      }
+    }
+    if (!ok) ok_s = 0;
+  }
+  tc_fence_before();
+  cluster.sync();                                      // every rank's partials are in its shared memory
+  // this rank finishes rows [ks * 128 / S, (ks + 1) * 128 / S) of both halves,
+  // summing the ranks' partials in rank order
+  const int rows = 128 / S, r0 = ks * rows;
+  for (int i = threadIdx.x; i < rows * NP; i += blockDim.x) {
+    const int r = r0 + i / NP, c = i % NP;
+    float v0 = 0.0f, v1 = 0.0f;
+    for (int q = 0; q < S; ++q) {
+      const float *rr = cluster.map_shared_rank(red, q);
+      v0 += rr[(0 * 128 + r) * NP + c];
+      v1 += rr[(1 * 128 + r) * NP + c];
+    }
+    if (c >= a.T) continue;
+    if constexpr (MODE == MODE_GATEUP) {
+      a.h_out[(size_t)c * a.rows + rb * 128 + r] = bf16_bits(silu_f(v0) * v1);
+    } else {
+      a.s_out[(size_t)c * a.rows + rb * 256 + r] = v0;
+      a.s_out[(size_t)c * a.rows + rb * 256 + 128 + r] = v1;
+    }
+  }
+  cluster.sync();                                      // no rank leaves while others read its partials
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Geo::TMEM_COLS);
+  }
+}
+
+template <int MODE, int NP>
+static void launch_splitk_one(const DenseTcArgs &a, int S, cudaStream_t s) {
+  using Geo = SplitGeom<NP>;
+  auto fn = dense_splitk_kernel<MODE, NP>;
+  cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::SMEM);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.n_rowblocks * S));
+  cfg.blockDim = dim3(kDenseThreads);
+  cfg.dynamicSmemBytes = Geo::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaLaunchKernelEx(&cfg, fn, a);
+}
+
+int dense_splitk_ways(int n_rowblocks, int K, int n_sms) {
+  int S = 1;
+  while (S < 8 && n_rowblocks * S * 2 <= n_sms && (K / 64) >= S * 2 * 2) S *= 2;
+  return S;
+}
+
+void launch_dense_splitk(int mode, const DenseTcArgs &a, int S, cudaStream_t s) {
+  const int np = dense_splitk_rows(a.T);
+#define MOE_SPLITK(NP)                                              \
+  if (mode == MODE_GATEUP) launch_splitk_one<MODE_GATEUP, NP>(a, S, s); \
+  else launch_splitk_one<MODE_DOWN, NP>(a, S, s);
+  if (np == 16) { MOE_SPLITK(16) }
+  else if (np == 32) { MOE_SPLITK(32) }
+  else if (np == 64) { MOE_SPLITK(64) }
+  else { MOE_SPLITK(128) }
+#undef MOE_SPLITK
 }
 
 }  // namespace moe

@@ -15,7 +15,7 @@ constexpr int kWarps = 8;          // warps per expert-kernel CTA
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kPermThreads = 512;
-constexpr int kPtrListMax = 256;   // expert pointers one table-update launch can carry
+constexpr int kPtrListMax = 256;   // experts one location-table update launch can carry
 
 // Device layout of one routed expert ("blob"): the checkpoint code bytes of the
 // three matrices unchanged, the block scales rearranged into 512-byte blocks of
@@ -133,37 +133,8 @@ void launch_topk(float *logits, const float *parts, int splits, const float *bia
                  int scoring, int renorm, int *ids, float *gates, cudaStream_t s);
 
 // ------------------------------------------------------------------ experts
-enum WeightFmt { WF_MX = 0, WF_NV = 1, WF_BF16 = 2 };
+enum WeightFmt { WF_MX = 0, WF_NV = 1 };
 enum ExpertMode { MODE_GATEUP = 0, MODE_DOWN = 1 };
-
-struct ExpertArgs {
-  // routed experts: blob pointer per expert (null = not in this pass)
-  const uint8_t *const *expert_ptr;
-  BlobLayout L;
-  // dense (shared expert) weights, bf16: m0 (and m1 for gate/up)
-  const uint16_t *dense_w0;
-  const uint16_t *dense_w1;
-  int K;                 // reduction length
-  int rows;              // output rows of one matrix (I, H or I_s)
-  int n_rowblocks;       // rows / rows-per-CTA
-  int k_split;           // cluster size along K
-  int tile_tokens;       // 8 * NT
-  // routed tiles
-  const TileInfo *tiles;
-  const int *n_tiles;
-  const int *prow_token; // padded row -> token (gate/up B rows) or -1
-  const int *prow_pair;  // padded row -> pair p or -1
-  const float *gates;    // [T*k]
-  int T;                 // dense path: number of tokens
-  // activations (B operand)
-  const uint16_t *act;   // f16 chunk-scaled (routed) or bf16 (dense), row stride K
-  const float *act_scale;// [rows][K/128] (routed only)
-  // outputs
-  uint16_t *h_out;       // gate/up: f16 chunk-scaled (routed) / bf16 (dense), row stride = rows
-  float *h_scale;        // routed gate/up: [prows][rows/128]
-  float *o_out;          // down: routed O'[pair][rows] or dense s[t][rows]
-};
-void launch_expert(int wf, int mode, int nt, const ExpertArgs &a, int grid_tiles, cudaStream_t s);
 
 struct CombineArgs {
   const float *oprime;   // [T*k, H]
@@ -182,15 +153,6 @@ struct CombineArgs {
 };
 void launch_combine(const CombineArgs &a, cudaStream_t s);
 
-struct PtrUpdate {
-  int n;
-  int keep_resident;     // 1: start from the resident table, 0: start from all-null
-  int E;
-  int expert[kPtrListMax];
-  const uint8_t *ptr[kPtrListMax];
-};
-void launch_ptr_update(const PtrUpdate &u, const uint8_t *const *resident, const uint8_t **out,
-                       cudaStream_t s);
 
 // ------------------------------------------------------------------ TMA-fed routed experts
 struct LocUpdate {
@@ -328,6 +290,11 @@ struct DenseTcArgs {
   int *err;
 };
 void launch_dense_tc(int mode, const DenseTcArgs &a, cudaStream_t s);
+// Decode-sized batches (T <= 128): K split over a cluster of S CTAs per row
+// block (xmap's box is 64 x NP rows, NP = T rounded up to 16, 32, 64 or 128).
+int dense_splitk_ways(int n_rowblocks, int K, int n_sms);
+void launch_dense_splitk(int mode, const DenseTcArgs &a, int S, cudaStream_t s);
+inline int dense_splitk_rows(int T) { return T <= 16 ? 16 : (T <= 32 ? 32 : (T <= 64 ? 64 : 128)); }
 
 struct TcArgs {
   TcMaps maps;

@@ -183,22 +183,6 @@ void launch_permute(const PermArgs &a, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// Expert pointer table for one pass: start from the resident table (or all
-// null) and overwrite the listed experts.
-// ---------------------------------------------------------------------------
-__global__ void ptr_update_kernel(const PtrUpdate u, const uint8_t *const *resident,
-                                  const uint8_t **out) {
-  for (int e = threadIdx.x; e < u.E; e += blockDim.x) out[e] = u.keep_resident ? resident[e] : nullptr;
-  __syncthreads();
-  for (int i = threadIdx.x; i < u.n; i += blockDim.x) out[u.expert[i]] = u.ptr[i];
-}
-
-void launch_ptr_update(const PtrUpdate &u, const uint8_t *const *resident, const uint8_t **out,
-                       cudaStream_t s) {
-  ptr_update_kernel<<<1, 256, 0, s>>>(u, resident, out);
-}
-
-// ---------------------------------------------------------------------------
 // Ordered combine: y[t] = sum_{j<k, ids_j an expert} O'[t*k + j] (in j order)
 // + gs[t] * s[t], gs = 1 or sigmoid(shared-gate logit); y fp32 or bf16 (RN).
 // ---------------------------------------------------------------------------

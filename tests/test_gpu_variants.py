@@ -50,7 +50,7 @@ def test_router_variant_parity(variant, fmt, numerics, T):
         y, r = G.run(layer, x)
         G.check_routing(r, lg, ids, g, wl.n_targets)
         G.check_output(y, y_ref)
-        if wl.n_sinks:
+        if wl.n_sinks and T >= 16:        # (a few tokens may all pass the sinks by)
             assert (ids >= wl.n_experts).any(), "no token chose a sink"
     finally:
         layer.close()
