@@ -191,7 +191,7 @@ def binding_roof(wl, T, n_active, miss_bytes, h2d_gbs, hbm_gbs, tensor_tflops, s
 def traffic_record(summary, kernel_src):
     """DRAM bytes per launch from a committed ncu summary (profiles/<summary>), if it
     was taken on the kernel source as it is now (its sha256 is recorded there)."""
-    path = os.path.join(ROOT, "profiles", summary)
+    path = summary if os.path.isabs(summary) else os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(path):
         return None
     rec = {}

@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_tc_kernel(const __grid
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ __align__(8) uint64_t accf_bar[NBUF];
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
+  __shared__ __align__(8) uint64_t quiesce_bar;   // all MMAs of the CTA done (before TMEM is freed)
   __shared__ uint32_t tmem_base_s;
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dn_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -91,6 +92,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_tc_kernel(const __grid
       mbar_init(smem_u32(&accf_bar[b]), 1);
       mbar_init(smem_u32(&acce_bar[b]), 4);
     }
+    mbar_init(smem_u32(&quiesce_bar), 1);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -171,6 +173,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_tc_kernel(const __grid
         tc_commit(smem_u32(&accf_bar[buf]));
         ++n;
       }
+      // every MMA issued above has completed before the CTA frees TMEM and
+      // leaves (also after a wait gave up and the loop was left early)
+      tc_commit(smem_u32(&quiesce_bar));
+      mbar_drain(smem_u32(&quiesce_bar), 0);
     }
   } else {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
@@ -368,8 +374,11 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
         tc_commit(smem_u32(&empty_bar[s]));
         if (++s == SN) { s = 0; ph ^= 1u; }
       }
-      // completes once every MMA above has (or at once, with none issued)
+      // completes once every MMA above has (or at once, with none issued);
+      // this lane also waits for it, so that no MMA is still running when the
+      // cluster's final barrier lets the CTA free TMEM and leave
       tc_commit(smem_u32(&accf_bar));
+      mbar_drain(smem_u32(&accf_bar), 0);
       if (failed) ok_s = 0;
     }
   } else {

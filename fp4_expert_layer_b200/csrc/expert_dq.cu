@@ -210,6 +210,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
   __shared__ __align__(8) uint64_t op_empty[SO];    // MMAs done with an operand stage
   __shared__ __align__(8) uint64_t accf_bar[NBUF];
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
+  __shared__ __align__(8) uint64_t quiesce_bar;     // all MMAs of the CTA done (before TMEM is freed)
   __shared__ uint32_t tmem_base_s;
   __shared__ __align__(8) uint64_t sched_full[kDqSched];
   __shared__ __align__(8) uint64_t sched_empty[kDqSched];
@@ -243,6 +244,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       mbar_init(smem_u32(&sched_full[q]), 1);
       mbar_init(smem_u32(&sched_empty[q]), kDqSchedReaders);
     }
+    mbar_init(smem_u32(&quiesce_bar), 1);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -372,6 +374,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         tc_commit(smem_u32(&accf_bar[buf]));
         ++n;
       }
+      // every MMA issued above has completed before the CTA frees TMEM and
+      // leaves (also after a wait gave up and the loop was left early)
+      tc_commit(smem_u32(&quiesce_bar));
+      mbar_drain(smem_u32(&quiesce_bar), 0);
     }
   } else if (warp >= 6 && warp < 10) {
     // ---------------- decoders: raw codes + E4M3 scales -> bf16 weight tile

@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ __align__(8) uint64_t accf_bar[NBUF];
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
+  __shared__ __align__(8) uint64_t quiesce_bar;   // all MMAs of the CTA done (before TMEM is freed)
   __shared__ uint32_t tmem_base_s;
   // Work items are taken from the pass's counter (atomicAdd, in index order)
   // by the producer, which loads each item's tile descriptor and expert
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       mbar_init(smem_u32(&sched_full[q]), 1);
       mbar_init(smem_u32(&sched_empty[q]), kSchedReaders);
     }
+    mbar_init(smem_u32(&quiesce_bar), 1);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -330,6 +332,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
         tc_commit(smem_u32(&accf_bar[buf]));                 // this item's accumulators complete
         ++n;
       }
+      // every MMA issued above has completed before the CTA frees TMEM and
+      // leaves (also after a wait gave up and the loop was left early)
+      tc_commit(smem_u32(&quiesce_bar));
+      mbar_drain(smem_u32(&quiesce_bar), 0);
     }
   } else if (warp >= 6) {
     // ---------------- loaders: the tile's activation-piece rows of this K slab

@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
         if (++s == kGStages) { s = 0; ph ^= 1u; }
       }
       tc_commit(smem_u32(&acc_bar));                               // accumulators complete
+      // this lane waits for them too: no MMA may still run when the CTA frees
+      // TMEM and leaves, even if the epilogue's wait gave up
+      mbar_drain(smem_u32(&acc_bar), 0);
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31

@@ -30,13 +30,18 @@ def test_layer_bytes_adds_router_shared_expert_and_io():
 
 
 def test_traffic_record_only_for_the_profiled_source(tmp_path):
-    src = os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert_tc.cu")
-    rec = bench.traffic_record("expert_tc_gateup_olmoe_like_T32.md", src)
-    assert rec is not None and rec > 1e8
-    other = tmp_path / "k.cu"
-    other.write_bytes(open(src, "rb").read() + b"\n// changed\n")
-    assert bench.traffic_record("expert_tc_gateup_olmoe_like_T32.md", str(other)) is None
-    assert bench.traffic_record("no_such_summary.md", src) is None
+    """A summary's DRAM bytes count only while the kernel source it was taken
+    on is unchanged (its sha256 is recorded in the summary)."""
+    import hashlib
+    src = tmp_path / "k.cu"
+    src.write_bytes(b"// kernel source\n")
+    h = hashlib.sha256(src.read_bytes()).hexdigest()
+    summ = tmp_path / "summary.md"
+    summ.write_text(f"- dram_bytes_per_launch: 149500000\n- kernel_source_sha256: `{h}`\n")
+    assert bench.traffic_record(str(summ), str(src)) == 149500000.0
+    src.write_bytes(b"// kernel source\n// changed\n")
+    assert bench.traffic_record(str(summ), str(src)) is None
+    assert bench.traffic_record(str(tmp_path / "no_such_summary.md"), str(src)) is None
 
 
 class _FakeSmi:

@@ -74,3 +74,28 @@ def test_a4_close_to_exact_mode():
     assert rel < 0.5, rel
     e.close()
     a.close()
+
+
+@pytest.mark.parametrize("name", ["deepseek_v4_flash_like", "qwen3_8_flash_next_like"])
+def test_a4_full_size_prefill_all_resident(name):
+    """A4 at the prefill sizes the measurements quote (DeepSeek-V4-Flash-like
+    4096 tokens, MXFP4; Qwen3.8-Flash-Next-like 8192 tokens, NVFP4), every
+    expert resident: routing bit-exact against the oracle for every token,
+    outputs against the oracle's A4 mode on the rows of the hottest and
+    coldest experts' tiles, tile boundaries and ragged tails."""
+    wl = synth.workload(name)
+    lw = synth.make_layer(wl)
+    L = oracle.Layer.from_weights(lw, numerics="a4")
+    T = wl.prefill_tokens
+    x, _ = cs.tokens_with_margin(L, wl, T, stream=T)
+    layer = G.make_layer(lw, n_slots=wl.n_experts, max_tokens=T, numerics="a4")
+    try:
+        y, r = G.run(layer, x)
+        assert layer.stats()["last_path"] == 1
+        lg, ids, g = L.route_all(x)
+        G.check_routing(r, lg, ids, g, wl.n_experts)
+        rows = G.boundary_rows(layer, r, wl.top_k, rng=np.random.default_rng(9), extra=3)
+        y_ref, *_ = L.forward(x, rows=rows)
+        G.check_output(y[rows], y_ref)
+    finally:
+        layer.close()
