@@ -1200,6 +1200,13 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     *(volatile int *)L->h_err = 0;
     return fail(MOE_ERR_CUDA, buf);
   }
+  if (L->inject == 3) {
+    // test hook: the device error word is set before this forward's kernels
+    // run, so that every bounded wait of theirs that has to wait gives up
+    // at once (the path a wait takes when its time limit passes)
+    L->inject = 0;
+    *(volatile int *)L->h_err = 99;
+  }
   CUDA_TRY(cudaSetDevice(c.device));
   cudaStream_t s = (cudaStream_t)stream;
   const int E = c.n_experts, k = c.top_k, H = c.hidden, I = c.inter, Is = c.shared_inter;
@@ -1759,7 +1766,7 @@ moe_status_t moe_debug_read(moe_layer_t L, int32_t which, void *dst, uint64_t by
 void moe_destroy(moe_layer_t L) { free_layer(L); }
 
 moe_status_t moe_debug_inject(moe_layer_t L, int32_t what) {
-  if (what < 0 || what > 2) return fail(MOE_ERR_INVALID_ARG, "unknown injection");
+  if (what < 0 || what > 3) return fail(MOE_ERR_INVALID_ARG, "unknown injection");
   if (what == 2 || (!L && what == 0)) {
     g_inject_create = what;
     return MOE_OK;

@@ -130,7 +130,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_tc_kernel(const __grid
           if (++s == S) { s = 0; ph ^= 1u; }
         }
       }
-      if (failed) {
+      {
+        // the last copies issued have landed before the CTA exits: at once on
+        // a normal run (their consumers waited for them), and also when a
+        // consumer gave up waiting
         int s2 = 0;
         uint32_t ph2 = 0;
         for (int i = 0; i < issued; ++i) {
@@ -343,7 +346,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
         ++issued;
         if (++s == SN) { s = 0; ph ^= 1u; }
       }
-      if (failed) {
+      {
+        // the last copies issued have landed before the CTA exits: at once on
+        // a normal run (their consumers waited for them), and also when a
+        // consumer gave up waiting
         int s2 = 0;
         uint32_t ph2 = 0;
         for (int i = 0; i < issued; ++i) {

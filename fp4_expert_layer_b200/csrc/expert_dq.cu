@@ -320,8 +320,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
           if (++r == SR) { r = 0; ph ^= 1u; }
         }
       }
-      if (failed) {
-        // let the copies already issued land before the CTA exits
+      {
+        // the last copies issued have landed before the CTA exits: at once on
+        // a normal run (their consumers waited for them), and also when a
+        // consumer gave up waiting
         int r2 = 0;
         uint32_t ph2 = 0;
         for (int i = 0; i < issued; ++i) {

@@ -113,9 +113,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
     // ================= producer: one lane issues every copy
     if (lane == 0) {
       const int nsf = K / 16;
+      int issued = 0;
       for (int it = 0; it < n_iter; ++it) {
         const int s = it % kStages;
         if (it >= kStages && !mbar_wait(smem_u32(&empty_bar[s]), ((it / kStages) - 1) & 1, a.err, 2)) break;
+        issued = it + 1;
         const int c = c_begin + it;
         const uint32_t bar = smem_u32(&full_bar[s]);
         const uint32_t dst = smem_u32(smem + (size_t)s * Geo::kStageBytes);
@@ -135,6 +137,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
                       blob + a.L.scales[2] + sf_offset(nsf, rb * 256 + 128 * j, col0), Geo::kSfPerGroup, bar);
         }
       }
+      // the last copies issued have landed before the CTA exits: at once on a
+      // normal run (the consumers waited for them), and also when a wait gave up
+      for (int i = max(0, issued - kStages); i < issued; ++i)
+        mbar_drain(smem_u32(&full_bar[i % kStages]), (i / kStages) & 1);
     }
   } else {
     // ================= consumers

@@ -111,10 +111,11 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
   if (warp == 0) {
     // ---------------- producer
     if (lane == 0) {
-      int s = 0;
+      int s = 0, issued = 0;
       uint32_t ph = 0;
       for (int it = 0; it < nk; ++it) {
         if (it >= kGStages && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 12)) break;
+        ++issued;
         const uint32_t bar = smem_u32(&full_bar[s]);
         const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
         // a half stage (last 128 K elements) carries half the scale blocks; the
@@ -132,6 +133,14 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
         tma_load_2d(st + Geo::B_OFF, &a.maps.act[a.act_map], bar, it * 128, prow0);
         bulk_load(st + Geo::SF_OFF + NMAT * Geo::SF_BYTES, a.bsf + sf_offset(nsf, prow0, col0), (uint32_t)sfb, bar);
         if (++s == kGStages) { s = 0; ph ^= 1u; }
+      }
+      // the last copies issued have landed before the CTA exits: at once on a
+      // normal run (the MMA lane waited for them), and also when a wait gave up
+      int s2 = 0;
+      uint32_t ph2 = 0;
+      for (int i = 0; i < issued; ++i) {
+        if (i >= issued - kGStages) mbar_drain(smem_u32(&full_bar[s2]), ph2);
+        if (++s2 == kGStages) { s2 = 0; ph2 ^= 1u; }
       }
     }
   } else if (warp == 1) {

@@ -336,8 +336,12 @@ const char *moe_last_error(void);
 
 /* Test hook for host-side failure injection (no GPU fault is ever caused):
  * 1 = the next staging copy reports a failure, 2 = the next device allocation
- * in moe_layer_create fails, 0 = off.  The forward must then return an error
- * status and leave the CUDA context usable. */
+ * in moe_layer_create fails, 3 = the next forward's device error word is set
+ * from the host before its kernels run, so that every bounded device wait of
+ * that forward which has to wait gives up (the path a wait takes when its time
+ * limit passes; the outputs of that forward are invalid and the following
+ * moe_forward reports MOE_ERR_CUDA), 0 = off.  The forward must then return an
+ * error status and leave the CUDA context usable. */
 moe_status_t moe_debug_inject(moe_layer_t layer, int32_t what);
 
 /* Test hook: synchronously copy up to `bytes` of an internal device buffer of

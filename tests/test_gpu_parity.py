@@ -208,3 +208,40 @@ def test_injected_allocation_failure_at_create():
     y, _ = G.run(layer, x)
     assert np.all(np.isfinite(y))
     layer.close()
+
+
+@pytest.mark.parametrize("fmt, numerics, T", [("mxfp4", "exact", 8), ("mxfp4", "exact", 300),
+                                              ("nvfp4", "exact", 3), ("nvfp4", "exact", 300),
+                                              ("mxfp4", "a4", 130)])
+def test_bounded_waits_give_up_and_the_context_recovers(fmt, numerics, T):
+    """The device error word is set before a forward's kernels run (test hook
+    3), so every bounded wait of theirs that has to wait gives up at once: the
+    kernels run out without hanging (well under their 2 s time limit), the next
+    forward reports MOE_ERR_CUDA and clears the word, and the forward after
+    that is bit-identical to a clean one.  Shapes cover the MXFP4 tensor-core
+    path (8- and 56-token tiles), the NVFP4 register and tensor-core paths,
+    both shared-expert kernels, and A4."""
+    import time
+    t = G.torch()
+    F = G.library()
+    wl = synth.custom_workload(512, 256, 8, 2, shared_inter=256, fmt=fmt)
+    lw = synth.make_layer(wl, seed=71)
+    x = synth.make_tokens(wl, T, seed=71)
+    layer = G.make_layer(lw, n_slots=wl.n_experts, max_tokens=T, numerics=numerics)
+    try:
+        y0, _ = G.run(layer, x)
+        xd = G.to_device(x)
+        layer.inject(3)
+        t0 = time.perf_counter()
+        layer.forward(xd)
+        t.cuda.synchronize()
+        assert time.perf_counter() - t0 < 1.5, "a wait ran to its time limit"
+        assert layer.stats()["device_error"] != 0
+        with pytest.raises(F.MoEError) as ei:
+            layer.forward(xd)
+        assert ei.value.status == 5
+        assert layer.stats()["device_error"] == 0
+        y1, _ = G.run(layer, x)
+        assert np.array_equal(y0, y1)
+    finally:
+        layer.close()
