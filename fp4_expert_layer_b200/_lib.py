@@ -13,7 +13,8 @@ import os
 import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SO = os.path.join(HERE, "libfp4moe.so")
+# FP4MOE_CHECKED=1 loads the build with the device bounds checks compiled in
+SO = os.path.join(HERE, "libfp4moe_checked.so" if os.environ.get("FP4MOE_CHECKED") == "1" else "libfp4moe.so")
 
 MOE_OK = 0
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_ADMISSION", 3: "MOE_ERR_SLOT_TABLE",

@@ -131,6 +131,7 @@ struct moe_layer {
   bool nv = false;
   DqMaps dqmaps{};
   int *dq_work = nullptr;            // [kWorkCtrs] item counters of the two passes
+  int cur_T = 0;                     // tokens of the forward being enqueued
   // host
   uint8_t *store = nullptr;          // pinned: E x blob bytes
   int *h_counts = nullptr;           // pinned [E]
@@ -957,6 +958,20 @@ moe_status_t moe_set_slot_table(moe_layer_t L, const int32_t *table, void *strea
   return MOE_OK;
 }
 
+// Index ranges of the forward being enqueued, for the device bounds checks of
+// the checked build.
+static DevBounds dev_bounds(const moe_layer *L) {
+  DevBounds b;
+  b.n_experts = L->cfg.n_experts;
+  b.n_targets = n_targets(&L->cfg);
+  b.n_slots = L->cfg.n_slots;
+  b.n_staging = L->n_staging;
+  b.n_tokens = L->cur_T;
+  b.n_pairs = L->cur_T * L->cfg.top_k;
+  b.err = L->d_err;
+  return b;
+}
+
 static int pick_split(int est_ctas, int nck) {
   int cs = 1;
   while (cs < 8 && nck % (cs * 2) == 0 && est_ctas * cs < 2 * 148) cs *= 2;
@@ -967,6 +982,7 @@ static moe_status_t run_experts(moe_layer *L, const int *locs, int nt, int grid_
                                 float *y, cudaStream_t s) {
   const moe_config_t &c = L->cfg;
   TmaExpertArgs a{};
+  a.db = dev_bounds(L);
   a.maps = L->maps;
   a.loc = locs;
   a.slots = L->slots;
@@ -1019,6 +1035,7 @@ static moe_status_t run_experts(moe_layer *L, const int *locs, int nt, int grid_
 static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int grid_tiles, cudaStream_t s) {
   const moe_config_t &c = L->cfg;
   TcArgs a{};
+  a.db = dev_bounds(L);
   a.maps = L->tcmaps;
   a.loc = locs;
   a.slots = L->slots;
@@ -1076,6 +1093,7 @@ static moe_status_t run_experts_dq(moe_layer *L, const int *locs, const void *x,
                                    cudaStream_t s) {
   const moe_config_t &c = L->cfg;
   DqArgs a{};
+  a.db = dev_bounds(L);
   a.maps = L->dqmaps;
   a.loc = locs;
   a.slots = L->slots;
@@ -1121,6 +1139,7 @@ static moe_status_t run_experts_dq(moe_layer *L, const int *locs, const void *x,
 static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles, cudaStream_t s) {
   const moe_config_t &c = L->cfg;
   A4GemmArgs g{};
+  g.db = dev_bounds(L);
   g.maps = L->a4maps;
   g.loc = locs;
   g.slots = L->slots;
@@ -1153,6 +1172,7 @@ static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles
   if (!fuse_hq) {
     StageTimer t8(L, 8, s);
     QuantArgs q{};
+    q.db = dev_bounds(L);
     q.max_rows = (int)L->a4_rows;
     q.n_rows = L->n_prows;
     q.K = c.inter;
@@ -1211,6 +1231,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   cudaStream_t s = (cudaStream_t)stream;
   const int E = c.n_experts, k = c.top_k, H = c.hidden, I = c.inter, Is = c.shared_inter;
   const int P = T * k;
+  L->cur_T = T;
   const int act_est = std::min(E, P);
   const int avg = (P + act_est - 1) / act_est;
   const int nt = avg <= 8 ? 1 : (avg <= 16 ? 2 : 4);
@@ -1246,6 +1267,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   ra.logits = L->logits; ra.ids = L->ids; ra.gates = L->gates;
   ra.xf16 = tc ? nullptr : L->xf16; ra.xs = L->xs; ra.counter = L->router_counter;
   PermArgs pa{};
+  pa.db = dev_bounds(L);
   pa.ids = L->ids; pa.n_pairs = P; pa.E = NT; pa.n_real = E; pa.k = k; pa.tile_tokens = ts;
   pa.counts = L->counts; pa.offsets = L->offsets; pa.perm = L->perm; pa.inv = L->inv;
   pa.tiles = L->tiles; pa.n_tiles = L->n_tiles; pa.prow_token = L->prow_token;
@@ -1358,6 +1380,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
 
   if (a4) {
     QuantArgs q{};
+    q.db = dev_bounds(L);
     q.max_rows = (int)L->a4_rows;
     q.n_rows = L->n_prows;
     q.K = H;
@@ -1375,6 +1398,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   }
   if (tc) {
     TcQuantArgs q{};
+    q.db = dev_bounds(L);
     q.x = reinterpret_cast<const uint16_t *>(x);
     q.H = H;
     q.tiles = L->tiles;

@@ -35,6 +35,7 @@
 //                16-byte cp.async (x rows gathered through the padded-row ->
 //                token map for gate/up; h rows for down).
 // Every mbarrier wait is bounded (error word, then the kernel runs out).
+#include "checks.cuh"
 #include "device_utils.cuh"
 #include "launch.cuh"
 #include "moe_internal.h"
@@ -272,7 +273,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         int loc = kLocAbsent;
         if (item < n_items) {
           ti = load_tile_dq(a.tiles + item / ipt);
-          loc = __ldcg(a.loc + ti.expert);
+          loc = load_loc(a.loc, ti.expert, a.db);
         }
         if (j >= kDqSched && !mbar_wait(smem_u32(&sched_empty[q]), qph ^ 1u, a.err, 58)) { failed = true; break; }
         const bool done = item >= n_items;
@@ -495,7 +496,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
           if (j >= ti.nrows) continue;                       // pad columns: never stored by the epilogue
           const uint16_t *src;
           if constexpr (MODE == MODE_GATEUP) {
-            const int tok = __ldg(a.prow_token + ti.prow0 + j);
+            const int tok = checked_index(__ldg(a.prow_token + ti.prow0 + j), 0, a.db.n_tokens, 0, a.db.err, kChkToken);
             src = a.act + (size_t)tok * K;
           } else {
             src = a.act + (size_t)(ti.prow0 + j) * K;
@@ -539,7 +540,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       int my_pair = 0;
       float my_gate = 0.0f;
       if (MODE == MODE_DOWN && et < ntok) {
-        my_pair = __ldg(a.prow_pair + ti.prow0 + et);
+        my_pair = checked_index(__ldg(a.prow_pair + ti.prow0 + et), 0, a.db.n_pairs, 0, a.db.err, kChkPair);
         my_gate = __ldg(a.gates + my_pair);
       }
       ok = mbar_wait(smem_u32(&accf_bar[buf]), (n / NBUF) & 1, a.err, 57);

@@ -35,6 +35,7 @@
 //    computes SwiGLU and the pieces of h; down scales by the gate and writes
 //    O' (the ordered combine into y is a separate kernel).
 //  All mbarrier waits are bounded (error word, then the kernel runs out).
+#include "checks.cuh"
 #include "device_utils.cuh"
 #include "moe_internal.h"
 #include "launch.cuh"
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       int loc = kLocAbsent;
       if (item < n_items) {
         ti = load_tile(a.tiles + item / ipt);
-        loc = __ldcg(a.loc + ti.expert);
+        loc = load_loc(a.loc, ti.expert, a.db);
       }
       for (int j = 0; !failed; ++j) {
         // hand item j (or the end) to the other roles
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
             if (slab == slab_meta) {
               if (nxt < n_items) {
                 nti = load_tile(a.tiles + nxt / ipt);
-                nloc = __ldcg(a.loc + nti.expert);
+                nloc = load_loc(a.loc, nti.expert, a.db);
               }
               have_next = true;
             }
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
           if (nxt < 0) nxt = atomicAdd(a.work_ctr, 1);
           if (nxt < n_items) {
             nti = load_tile(a.tiles + nxt / ipt);
-            nloc = __ldcg(a.loc + nti.expert);
+            nloc = load_loc(a.loc, nti.expert, a.db);
           }
         }
         item = nxt;
@@ -428,7 +429,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       int my_pair = 0;
       float my_gate = 0.0f;
       if (MODE == MODE_DOWN && et < ntok) {
-        my_pair = __ldg(a.prow_pair + ti.prow0 + et);
+        my_pair = checked_index(__ldg(a.prow_pair + ti.prow0 + et), 0, a.db.n_pairs, 0, a.db.err, kChkPair);
         my_gate = __ldg(a.gates + my_pair);
       }
       ok = mbar_wait(smem_u32(&accf_bar[buf]), (n / NBUF) & 1, a.err, 33);

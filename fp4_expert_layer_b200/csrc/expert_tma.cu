@@ -20,6 +20,7 @@
 // data, so the kernel always terminates and the host reports the failure.
 #include <cooperative_groups.h>
 
+#include "checks.cuh"
 #include "device_utils.cuh"
 #include "moe_internal.h"
 #include "tma.cuh"
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
   // ---- task (uniform over the CTA and its cluster)
   if (tile >= *a.n_tiles) return;
   const TileInfo ti = a.tiles[tile];
-  const int loc = a.loc[ti.expert];
+  const int loc = load_loc(a.loc, ti.expert, a.db);
   if (loc == kLocAbsent) return;
   const int prow0 = ti.prow0, nrows = ti.nrows;
   const bool in_slot = loc >= 0;
@@ -161,13 +162,19 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
     for (int nt = 0; nt < NT; ++nt) {
       const int lb = nt * 8 + g;
       int arow = -1;
-      if (lb < nrows) arow = (MODE == MODE_GATEUP) ? a.prow_token[prow0 + lb] : prow0 + lb;
+      if (lb < nrows)
+        arow = (MODE == MODE_GATEUP)
+                   ? checked_index(a.prow_token[prow0 + lb], 0, a.db.n_tokens, 0, a.db.err, kChkToken)
+                   : prow0 + lb;
       bptr[nt] = (arow >= 0) ? a.act + (size_t)arow * K + q * 32 : nullptr;
 #pragma unroll
       for (int cb = 0; cb < 2; ++cb) {
         const int lc = nt * 8 + 2 * q + cb;
         int r = -1;
-        if (lc < nrows) r = (MODE == MODE_GATEUP) ? a.prow_token[prow0 + lc] : prow0 + lc;
+        if (lc < nrows)
+          r = (MODE == MODE_GATEUP)
+                  ? checked_index(a.prow_token[prow0 + lc], 0, a.db.n_tokens, 0, a.db.err, kChkToken)
+                  : prow0 + lc;
         crow[nt][cb] = r;
       }
     }
@@ -372,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
       for (int x = 0; x < 4; ++x) {
         const int col = nt * 8 + 2 * q + (x & 1);
         if (col >= nrows) continue;
-        const int p = a.prow_pair[prow0 + col];
+        const int p = checked_index(a.prow_pair[prow0 + col], 0, a.db.n_pairs, 0, a.db.err, kChkPair);
         const float gp = a.gates[p];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
@@ -387,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
       const int col = threadIdx.x;
       int t = -1;
       if (col < nrows) {
-        const int p = a.prow_pair[prow0 + col];
+        const int p = checked_index(a.prow_pair[prow0 + col], 0, a.db.n_pairs, 0, a.db.err, kChkPair);
         const int tok = p / a.top_k;
         if (atomicAdd(&a.comb_cnt[(size_t)tok * a.n_rowblocks + rb], 1) == a.top_k - 1) t = tok;
       }

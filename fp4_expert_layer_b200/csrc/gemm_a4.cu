@@ -18,6 +18,7 @@
 //
 // TMEM columns: accumulators at 0 and 128 (128 fp32 columns each), scale
 // factors of stage s at 256 + s * (4 per block).
+#include "checks.cuh"
 #include "device_utils.cuh"
 #include "moe_internal.h"
 #include "tcgen05.cuh"
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
   const int tile = blockIdx.x / a.n_rowblocks;
   if (tile >= *a.n_tiles) return;
   const TileInfo ti = a.tiles[tile];
-  const int loc = a.loc[ti.expert];
+  const int loc = load_loc(a.loc, ti.expert, a.db);
   if (loc == kLocAbsent) return;
   const int prow0 = ti.prow0, nrows = ti.nrows;
   const bool in_slot = loc >= 0;
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
       if (c < nrows) {
         col_bs[c] = (WF == WF_NV) ? __ldg(a.bG + prow0 + c) : 1.0f;
         if constexpr (MODE == MODE_DOWN) {
-          const int p = __ldg(a.prow_pair + prow0 + c);
+          const int p = checked_index(__ldg(a.prow_pair + prow0 + c), 0, a.db.n_pairs, 0, a.db.err, kChkPair);
           col_pair[c] = p;
           col_gate[c] = __ldg(a.gates + p);
         }

@@ -80,6 +80,17 @@ struct alignas(16) TileInfo {
   int sorted0;   // first row in the unpadded sorted order
 };
 
+// Ranges of the indices the kernels take from device data (a routing target,
+// a location-table entry, a padded row's token or pair), for the device bounds
+// checks of the checked build (checks.cuh); the normal build ignores them.
+struct DevBounds {
+  int n_experts;           // location-table entries (routed experts)
+  int n_targets;           // routing targets (experts, then sinks)
+  int n_slots, n_staging;  // blobs in the slot pool and in the staging ring
+  int n_tokens, n_pairs;   // tokens of this forward, and T * k
+  int *err;                // the layer's error word
+};
+
 // ------------------------------------------------------------------ routing
 struct PermArgs {
   const int *ids;        // [T*k]
@@ -98,6 +109,7 @@ struct PermArgs {
   int *n_prows;          // [1] total padded rows (may be null)
   int *work_ctr;         // [kWorkCtrs] zeroed here (may be null): item counters of the expert passes
   int *tile_done;        // [tiles] zeroed here (may be null): gate/up items finished per tile
+  DevBounds db;           // device bounds checks (checked build)
 };
 struct RouterArgs {
   const uint16_t *x;     // bf16 [T, H]
@@ -197,6 +209,7 @@ struct TmaExpertArgs {
   const float *shared;     // [T, H] or null
   int *comb_cnt;           // [max_tokens, H/256] zero-initialised arrival counters
   int top_k;
+  DevBounds db;           // device bounds checks (checked build)
 };
 void launch_expert_tma(int wf, int mode, int nt, const TmaExpertArgs &a, int grid_tiles, cudaStream_t s);
 
@@ -216,6 +229,7 @@ struct QuantArgs {
   uint8_t *codes;
   uint8_t *sf;
   float *G;                  // NVFP4: per-row tensor scale
+  DevBounds db;           // device bounds checks (checked build)
 };
 void launch_quant(const QuantArgs &q, cudaStream_t s);
 
@@ -246,6 +260,7 @@ struct A4GemmArgs {
   const int *prow_pair;
   const float *gates;
   int *err;
+  DevBounds db;           // device bounds checks (checked build)
 };
 void launch_gemm_a4(int wf, int mode, const A4GemmArgs &a, int grid_tiles, cudaStream_t s);
 
@@ -277,6 +292,7 @@ struct TcQuantArgs {
   const int *prow_token;
   uint8_t *xq;               // [max_tiles * kTcSlotRows, H] E4M3 pieces
   uint8_t *xsf;              // scale-factor blocks of xq (UE8M0, per 32)
+  DevBounds db;           // device bounds checks (checked build)
 };
 void launch_tc_quant_x(const TcQuantArgs &q, cudaStream_t s);
 
@@ -328,6 +344,7 @@ struct TcArgs {
   // predecessor (the resident path; not the staged waves, whose location
   // table is written by the kernel right before)
   int early;
+  DevBounds db;           // device bounds checks (checked build)
 };
 // nbox: activation rows per tile (2 x tile tokens): 16 or 112.  The kernel is
 // persistent: `a.grid` CTAs take the work items (tile, 256 weight rows) from
@@ -370,6 +387,7 @@ struct DqArgs {
   int *work_ctr;             // item counter of this pass, zero at launch
   int *err;
   int grid;                  // persistent CTAs
+  DevBounds db;           // device bounds checks (checked build)
 };
 // nb: tokens per tile (64 or 128)
 void launch_expert_dq(int mode, int nb, const DqArgs &a, cudaStream_t s);

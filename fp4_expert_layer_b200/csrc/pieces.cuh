@@ -3,6 +3,7 @@
 // e1 = floor(log2(max|v|)) - 7 and e2 from the largest remainder, q = RN_E4M3.
 #pragma once
 
+#include "checks.cuh"
 #include "device_utils.cuh"
 #include "moe_internal.h"
 
@@ -49,7 +50,8 @@ __device__ __forceinline__ void tc_quant_x_slot(const TcQuantArgs &q, size_t row
 __device__ __forceinline__ void tc_quant_x_row(const TcQuantArgs &q, int tile, int j) {
   const TileInfo ti = q.tiles[tile];
   if (j >= ti.nrows) return;
-  tc_quant_x_slot(q, (size_t)tile * kTcSlotRows + 2 * j, q.prow_token[ti.prow0 + j]);
+  tc_quant_x_slot(q, (size_t)tile * kTcSlotRows + 2 * j,
+                  checked_index(q.prow_token[ti.prow0 + j], 0, q.db.n_tokens, 0, q.db.err, kChkToken));
 }
 
 // Pieces of token `token` into activation rows row0 (first piece) and row0 + 1.

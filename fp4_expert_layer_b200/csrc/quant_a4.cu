@@ -16,6 +16,7 @@
 //
 // One warp per padded row; rows past the padded count exit, pad rows are
 // written as zero codes.
+#include "checks.cuh"
 #include "device_utils.cuh"
 #include "moe_internal.h"
 
@@ -58,11 +59,12 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const QuantArgs q) {
   const int K = q.K;
   int src = -1;
   if (q.src_bf16) {
-    src = q.row_token[row];
+    src = checked_index(q.row_token[row], -1, q.db.n_tokens, -1, q.db.err, kChkToken);
   } else {
-    const int p = q.row_pair[row];
+    const int p = checked_index(q.row_pair[row], -1, q.db.n_pairs, -1, q.db.err, kChkPair);
     if (p >= 0) {
-      if (q.loc && q.loc[q.ids[p]] == kLocAbsent) return;   // expert not in this pass: its h is not ready
+      // expert not in this pass: its h is not ready
+      if (q.loc && load_loc(q.loc, q.ids[p], q.db) == kLocAbsent) return;
       src = row;
     }
   }

@@ -3,6 +3,7 @@
 // token-to-expert permutation.
 #pragma once
 
+#include "checks.cuh"
 #include "device_utils.cuh"
 #include "moe_internal.h"
 
@@ -108,7 +109,10 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
   if (a.work_ctr && tid < kWorkCtrs) a.work_ctr[tid] = 0;
   for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;
   __syncthreads();
-  for (int p = tid; p < a.n_pairs; p += NTH) atomicAdd(&cnt[load_id<IDS_GLOBAL>(ids, p)], 1);
+  for (int p = tid; p < a.n_pairs; p += NTH) {
+    const int e = load_id<IDS_GLOBAL>(ids, p);
+    if (dcheck(e >= 0 && e < E, a.db.err, kChkTarget)) atomicAdd(&cnt[e], 1);
+  }
   __syncthreads();
 
   // block exclusive scan of (count, padded count, tiles, active) over targets;
@@ -192,8 +196,9 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int base = 0; base < a.n_pairs; base += NTH) {
     const int p = base + tid;
-    const bool valid = p < a.n_pairs;
-    const int e = valid ? load_id<IDS_GLOBAL>(ids, p) : -1;
+    int e = p < a.n_pairs ? load_id<IDS_GLOBAL>(ids, p) : -1;
+    if (kCheckedBuild && (e < 0 || e >= E)) e = -1;   // recorded by the count above
+    const bool valid = e >= 0;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & lt_mask);
     if (valid && rank == 0) wcnt[warp * E + e] = __popc(peers);

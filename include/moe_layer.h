@@ -171,8 +171,12 @@ typedef struct {
   uint64_t expert_bytes;   /* device-layout bytes of one routed expert          */
   uint64_t device_bytes;   /* HBM held by the layer                             */
   uint64_t pinned_bytes;   /* pinned host memory held by the layer              */
-  int32_t device_error;    /* nonzero: a device-side wait gave up (code of the  */
-                           /* first one); the next moe_forward reports and      */
+  int32_t device_error;    /* nonzero: a device-side wait gave up (code 1..99   */
+                           /* of the first one) or, in the bounds-checked build */
+                           /* (libfp4moe_checked.so, -DMOE_DEBUG_CHECKS), an     */
+                           /* index read from device data was out of range      */
+                           /* (201 target, 202/203 location table, 204 token,   */
+                           /* 205 pair); the next moe_forward reports and       */
                            /* clears it                                         */
   int32_t policy;          /* moe_policy_t in force                             */
   uint64_t admitted;       /* staged experts admitted into slots, cumulative    */

@@ -17,7 +17,7 @@ def library():
     """The built CUDA library; a missing build is an error on a GPU machine, never a skip."""
     import fp4_expert_layer_b200 as F
     from fp4_expert_layer_b200 import build
-    build.build()
+    build.build(checked=F._lib.SO.endswith("_checked.so"))
     F.lib()
     return F
 

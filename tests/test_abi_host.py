@@ -38,6 +38,16 @@ def test_library_exports_every_declared_symbol(F):
     assert set(F._lib.EXPORTED) <= set(decl)
 
 
+def test_checked_library_builds_and_exports_every_declared_symbol(F):
+    from fp4_expert_layer_b200 import build
+    so = build.build(checked=True)
+    assert so.endswith("libfp4moe_checked.so")
+    assert "-DMOE_DEBUG_CHECKS" not in build.nvcc_cmd("x")
+    L = C.CDLL(so)
+    missing = [n for n in _declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
 def test_plan_sizes(F):
     wl = synth.workload("olmoe_like")
     cfg = F.make_config(wl.hidden, wl.inter, wl.n_experts, wl.top_k, max_tokens=32)
