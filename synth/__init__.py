@@ -281,8 +281,9 @@ def slot_table(lw: LayerWeights, n_slots: Optional[int] = None, seed: Optional[i
     """Resident-slot table: int32 [E], slot index or -1 (expert kept in host memory).
 
     "all": every expert resident (slot = expert index); "hottest": the S experts
-    with the lowest Zipf rank (a static warm fill); "random": a seeded random
-    subset of S experts.
+    with the lowest Zipf rank (a static warm fill); "coldest": the S experts with
+    the highest Zipf rank (a cold start: most routed pairs miss); "random": a
+    seeded random subset of S experts.
     """
     wl = lw.wl
     E = wl.n_experts
@@ -294,8 +295,10 @@ def slot_table(lw: LayerWeights, n_slots: Optional[int] = None, seed: Optional[i
         if S < E:
             table[:S] = np.arange(S, dtype=np.int32)
         return table
-    if policy == "hottest" and lw.zipf_rank is not None:
+    if policy in ("hottest", "coldest") and lw.zipf_rank is not None:
         order = np.argsort(lw.zipf_rank[:E], kind="stable")      # experts only (sinks hold no weights)
+        if policy == "coldest":
+            order = order[::-1]
     else:
         ss = _streams(_seed(wl, seed), 7)[_S_SLOTS]
         order = np.random.Generator(np.random.PCG64(ss)).permutation(E)

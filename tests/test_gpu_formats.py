@@ -50,7 +50,9 @@ def test_format_paged_equals_resident(fmt):
     lw = synth.make_layer(wl, seed=62)
     T = 64
     x = synth.make_tokens(wl, T, seed=62)
-    paged = G.make_layer(lw, n_slots=4, max_tokens=T, n_staging=2)
+    # the coldest experts resident: most pairs miss, so the forward runs several waves
+    paged = G.make_layer(lw, n_slots=4, max_tokens=T, n_staging=2,
+                         table=synth.slot_table(lw, 4, policy="coldest"))
     resident = G.make_layer(lw, n_slots=wl.n_experts, max_tokens=T)
     try:
         yp, _ = G.run(paged, x)

@@ -21,6 +21,12 @@ def pair():
     resident.close()
 
 
+def _cold_layer(lw):
+    """4 slots holding the coldest experts (a cold start: the hot experts all
+    miss at first), two staging buffers."""
+    return G.make_layer(lw, n_slots=4, max_tokens=64, n_staging=2, table=synth.slot_table(lw, 4, policy="coldest"))
+
+
 def _batches(wl, n, T, seed):
     return [synth.make_tokens(wl, T, seed=seed, stream=i) for i in range(n)]
 
@@ -29,7 +35,7 @@ def _batches(wl, n, T, seed):
 def test_cache_policy_admits_misses_and_keeps_outputs(pair, fmt_T):
     wl, lw, resident = pair
     _, T = fmt_T
-    layer = G.make_layer(lw, n_slots=4, max_tokens=64, n_staging=2)
+    layer = _cold_layer(lw)
     try:
         layer.set_policy("cache")
         assert layer.stats()["policy"] == 2
@@ -97,7 +103,7 @@ def test_prefetch_of_predicted_experts_removes_misses(pair):
     unchanged; prefetch outside the cache policies is refused."""
     F = G.library()
     wl, lw, resident = pair
-    layer = G.make_layer(lw, n_slots=4, max_tokens=64, n_staging=2)
+    layer = _cold_layer(lw)
     try:
         x = synth.make_tokens(wl, 2, seed=21)
         with pytest.raises(F.MoEError) as ei:
