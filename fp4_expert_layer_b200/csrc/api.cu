@@ -118,6 +118,7 @@ struct moe_layer {
   uint8_t *xq = nullptr, *xsf = nullptr, *hq = nullptr, *hsf = nullptr;
   float *xG = nullptr, *hG = nullptr, *h32 = nullptr;
   int *n_prows = nullptr;
+  int *a4_work = nullptr;            // [kWorkCtrs] item counters of the two A4 passes
   // EXACT numerics of MXFP4 experts on the tensor core (E4M3 activation pieces)
   bool tc = false;
   int n_sms = 148;
@@ -270,12 +271,18 @@ static size_t a4_scratch_bytes(const moe_config_t *c) {
   const size_t H = c->hidden, I = c->inter, G = c->fmt == MOE_FMT_MXFP4 ? 32 : 16;
   size_t b = align256(z.a4_rows * H / 2) + align256(z.a4_rows * H / G) + align256(z.a4_rows * 4);
   b += align256(z.a4_rows * I * 4) + align256(z.a4_rows * I / 2) + align256(z.a4_rows * I / G) + align256(z.a4_rows * 4);
-  b += align256(z.P * H * 4) + align256(4);
+  b += align256(z.P * H * 4) + align256(4) + align256(kWorkCtrs * sizeof(int));
   return b;
 }
 
 static bool uses_tc(const moe_config_t *c) {
   return c->numerics == MOE_NUMERICS_EXACT && c->fmt == MOE_FMT_MXFP4;
+}
+
+// Blob layout of a layer's experts: tile-major for the tensor-core EXACT path,
+// gate/up interleaved per 64 rows for A4, checkpoint order otherwise.
+static int blob_tiling(const moe_config_t *c) {
+  return uses_tc(c) ? 1 : (c->numerics == MOE_NUMERICS_A4 ? 2 : 0);
 }
 
 // NVFP4 layers in EXACT numerics: prefill-sized batches run the tensor-core
@@ -399,7 +406,9 @@ static moe_status_t make_a4_weight_map(CUtensorMap *map, const uint8_t *region, 
                                        int m) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  cuuint64_t dims[3] = {(cuuint64_t)(L.K[m] / 2), (cuuint64_t)L.rows[m], (cuuint64_t)nblobs};
+  // gate/up of the interleaved layout: one matrix of 2I rows from codes[0]
+  const cuuint64_t rows = (L.tiled == 2 && m == 0) ? (cuuint64_t)(2 * L.rows[0]) : (cuuint64_t)L.rows[m];
+  cuuint64_t dims[3] = {(cuuint64_t)(L.K[m] / 2), rows, (cuuint64_t)nblobs};
   cuuint64_t strides[2] = {(cuuint64_t)(L.K[m] / 2), (cuuint64_t)L.bytes};
   cuuint32_t box[3] = {128, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
@@ -535,7 +544,7 @@ const char *moe_last_error(void) { return g_err.c_str(); }
 moe_status_t moe_layer_plan(const moe_config_t *cfg, moe_plan_t *out) {
   ST_TRY(check_config(cfg));
   if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
-  const BlobLayout L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt, uses_tc(cfg));
+  const BlobLayout L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt, blob_tiling(cfg));
   out->expert_bytes = L.bytes;
   out->slot_bytes = (uint64_t)L.bytes * cfg->n_slots;
   out->staging_bytes = (uint64_t)L.bytes * default_staging(cfg);
@@ -654,9 +663,16 @@ static void pack_expert_tiled(const BlobLayout &L, const moe_weights_t *w, int e
     }
 }
 
+// Row c of the interleaved gate/up matrix (layout tiled = 2): matrix (c / 64) % 2
+// (0 gate, 1 up), row (c / 128) * 64 + c % 64 of it.
+static void a4_gu_source(int c, int *mat, int *row) {
+  *mat = (c >> 6) & 1;
+  *row = (c >> 7) * 64 + (c & 63);
+}
+
 static void pack_expert(const moe_config_t *cfg, const BlobLayout &L, const moe_weights_t *w, int e,
                         uint8_t *dst) {
-  if (L.tiled) {
+  if (L.tiled == 1) {
     pack_expert_tiled(L, w, e, dst);
     return;
   }
@@ -681,7 +697,18 @@ static void pack_expert(const moe_config_t *cfg, const BlobLayout &L, const moe_
     }
     return;
   }
-  for (int m = 0; m < 3; ++m) {
+  if (L.tiled == 2) {
+    // gate and up interleaved per 64 rows into one matrix of 2I rows
+    const int H = L.K[0], I = L.rows[0], nsf = H / L.G;
+    for (int c = 0; c < 2 * I; ++c) {
+      int mat, row;
+      a4_gu_source(c, &mat, &row);
+      memcpy(dst + L.codes[0] + (size_t)c * (H / 2), w->codes[mat][e] + (size_t)row * (H / 2), (size_t)H / 2);
+      const uint8_t *src = w->scales[mat][e] + (size_t)row * nsf;
+      for (int col = 0; col < nsf; ++col) dst[L.scales[0] + sf_offset(nsf, c, col)] = src[col];
+    }
+  }
+  for (int m = L.tiled == 2 ? 2 : 0; m < 3; ++m) {
     const size_t ncode = (size_t)L.rows[m] * L.K[m] / 2;
     const size_t nsc = (size_t)L.rows[m] * L.K[m] / L.G;
     memcpy(dst + L.codes[m], w->codes[m][e], ncode);
@@ -717,7 +744,7 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   cudaStream_t s = (cudaStream_t)stream;
   moe_layer *L = new moe_layer();
   L->cfg = *cfg;
-  L->L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt, uses_tc(cfg));
+  L->L = blob_layout(cfg->hidden, cfg->inter, cfg->fmt, blob_tiling(cfg));
   L->wf = cfg->fmt == MOE_FMT_MXFP4 ? WF_MX : (cfg->fmt == MOE_FMT_NVFP4 ? WF_NV : -1);
   L->n_staging = default_staging(cfg);
   L->cfg.n_staging = L->n_staging;
@@ -821,6 +848,8 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     C_TRY(dalloc(L, &L->hsf, R * I / G));
     C_TRY(dalloc(L, &L->hG, R * 4));
     C_TRY(dalloc(L, &L->n_prows, 4));
+    C_TRY(dalloc(L, &L->a4_work, kWorkCtrs * sizeof(int)));
+    C_CUDA(cudaMemsetAsync(L->a4_work, 0, kWorkCtrs * sizeof(int), s));
     C_TRY(make_a4_act_map(&L->a4maps.act[0], L->xq, H / 2, R));
     C_TRY(make_a4_act_map(&L->a4maps.act[1], L->hq, I / 2, R));
   }
@@ -864,8 +893,11 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     const int box_rows = m < 2 ? 128 : 256;
     if (cfg->n_slots) C_TRY(make_code_map(&L->maps.slot[m], L->slots, cfg->n_slots, L->L, m, box_rows));
     if (L->n_staging) C_TRY(make_code_map(&L->maps.stage[m], L->staging, L->n_staging, L->L, m, box_rows));
-    if (L->a4 && cfg->n_slots) C_TRY(make_a4_weight_map(&L->a4maps.w[0][m], L->slots, cfg->n_slots, L->L, m));
-    if (L->a4 && L->n_staging) C_TRY(make_a4_weight_map(&L->a4maps.w[1][m], L->staging, L->n_staging, L->L, m));
+    // A4: gate and up are one interleaved matrix of 2I rows (map 0); down is map 2
+    if (L->a4 && m != 1 && cfg->n_slots)
+      C_TRY(make_a4_weight_map(&L->a4maps.w[0][m], L->slots, cfg->n_slots, L->L, m));
+    if (L->a4 && m != 1 && L->n_staging)
+      C_TRY(make_a4_weight_map(&L->a4maps.w[1][m], L->staging, L->n_staging, L->L, m));
     // dequantising kernels: one 64-element K slab per box (32 bytes of nibbles, or 64 FP8 bytes)
     const int dq_box = cfg->fmt == MOE_FMT_FP8B128 ? 64 : 32;
     if (L->nv && cfg->n_slots)
@@ -1154,7 +1186,9 @@ static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles
   g.act_map = 0;
   g.K = c.hidden;
   g.rows = c.inter;
-  g.n_rowblocks = c.inter / 128;
+  g.n_rowblocks = c.inter / 64;                 // 64 h columns (gate + up rows) per item
+  g.work_ctr = L->a4_work;
+  g.grid = std::min(grid_tiles * g.n_rowblocks, L->n_sms);
   g.bsf = L->xsf;
   g.bG = L->xG;
   g.h_out = L->h32;
@@ -1165,7 +1199,7 @@ static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles
   g.hq_out = fuse_hq ? L->hq : nullptr;
   g.hsf_out = fuse_hq ? L->hsf : nullptr;
   StageTimer t3(L, 3, s);
-  launch_gemm_a4(L->wf, MODE_GATEUP, g, grid_tiles, s);
+  launch_gemm_a4(L->wf, MODE_GATEUP, g, s);
   CUDA_TRY(cudaGetLastError());
   t3.launched(1);
   t3.end();
@@ -1195,11 +1229,13 @@ static moe_status_t run_experts_a4(moe_layer *L, const int *locs, int grid_tiles
   g.K = c.inter;
   g.rows = c.hidden;
   g.n_rowblocks = c.hidden / 128;
+  g.work_ctr = L->a4_work + 1;
+  g.grid = std::min(grid_tiles * g.n_rowblocks, L->n_sms);
   g.bsf = L->hsf;
   g.bG = L->hG;
   g.o_out = L->oprime;
   StageTimer t4(L, 4, s);
-  launch_gemm_a4(L->wf, MODE_DOWN, g, grid_tiles, s);
+  launch_gemm_a4(L->wf, MODE_DOWN, g, s);
   CUDA_TRY(cudaGetLastError());
   t4.launched(1);
   t4.end();
@@ -1274,7 +1310,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   pa.prow_pair = L->prow_pair; pa.active = L->active;
   pa.pad = a4 ? 128 : 8;
   pa.n_prows = a4 ? L->n_prows : nullptr;
-  pa.work_ctr = tc ? L->tc_work : (dq ? L->dq_work : nullptr);
+  pa.work_ctr = tc ? L->tc_work : (dq ? L->dq_work : (a4 ? L->a4_work : nullptr));
   pa.tile_done = tc ? L->tile_done : nullptr;
   // decode-sized batches: the router's last CTA also runs the permutation
   const bool fuse_perm = P <= 2048;
@@ -1463,7 +1499,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
         if (!one && w >= 2) CUDA_TRY(cudaStreamWaitEvent(L->side, L->ev_done[half], 0));
         LocUpdate u{};
         u.E = E;
-        u.work_ctr = tc ? L->tc_work : (dq ? L->dq_work : nullptr);
+        u.work_ctr = tc ? L->tc_work : (dq ? L->dq_work : (a4 ? L->a4_work : nullptr));
         u.keep_resident = (w == 0);
         const int b0 = w * wave_sz, b1 = std::min(misses_n, b0 + wave_sz);
         for (int i = b0; i < b1; ++i) {

@@ -17,6 +17,14 @@
 //     activations are h = silu(G_g a) * (G_u u) rounded to bf16.
 // The decode cost of a weight tile is shared by the up to NB tokens of a tile.
 //
+// The decoded weight tile is the MMA's A operand in TMEM (tcgen05.st by the
+// decoders, one lane per weight row), not in shared memory: a bf16 tile
+// written to and read back from shared memory would cost 64 KB of
+// shared-memory traffic per 64-wide K slab of 256 rows on top of the MMAs'
+// own reads of the activations, more than the 128 bytes per clock shared
+// memory serves; from TMEM only the activation tile (B) and the packed raw
+// codes pass through shared memory.
+//
 // Kernel expert_dq_kernel<MODE, NB>: persistent, one CTA per SM, work items
 // (tile of up to NB tokens, 256 weight rows: 128 gate + the same 128 up rows,
 // or 256 down rows) taken from a counter in index order.  Roles:
@@ -25,15 +33,21 @@
 //                512-byte E4M3 scale-factor blocks by bulk copy, into a ring
 //                of raw stages;
 //   warp 1       MMA issuer (one lane): M = 128, N = tokens rounded up to 16,
-//                K = 16, two accumulators (gate and up, or the two 128-row
-//                halves of down) per item, double-buffered across items;
+//                K = 16, A from TMEM, B from shared memory, two accumulators
+//                (gate and up, or the two 128-row halves of down) per item;
 //   warps 2..5   epilogue: TMEM -> SwiGLU -> h (bf16, padded-row order), or
 //                G_d * gate * acc -> O' (fp32, pair order);
-//   warps 6..9   decoders: raw stage -> bf16 weight tile in the 128-byte
-//                swizzled K-major layout the MMA descriptor reads;
-//   warps 10..11 activation loaders: the tile's bf16 rows of this K slab by
+//   warps 6..13  decoders: raw stage -> bf16 weight rows in TMEM, warp w the
+//                rows of TMEM lane quadrant w % 4 of the first (w < 10) or
+//                second 128 rows (NVFP4: one hardware E2M1 -> f16x2
+//                conversion per two codes, then integer bit moves and one
+//                bf16 multiply by the scale);
+//   warps 14..15 activation loaders: the tile's bf16 rows of this K slab by
 //                16-byte cp.async (x rows gathered through the padded-row ->
-//                token map for gate/up; h rows for down).
+//                token map for gate/up; h rows for down), 128-byte swizzled
+//                K-major as the B descriptor reads them.
+// TMEM: accumulators (2 x NB columns per buffer; two buffers when NB = 64),
+// then 4 A stages of 64 columns (32 per 128-row half: 64 bf16 of a row).
 // Every mbarrier wait is bounded (error word, then the kernel runs out).
 #include "checks.cuh"
 #include "device_utils.cuh"
@@ -46,12 +60,12 @@ namespace moe {
 
 namespace {
 
-constexpr int kDqThreads = 384;
-constexpr int kDqDecoders = 128;   // warps 6..9
-constexpr int kDqLoaders = 64;     // warps 10..11
+constexpr int kDqThreads = 512;
+constexpr int kDqDecoders = 256;   // warps 6..13
+constexpr int kDqLoaders = 64;     // warps 14..15
 constexpr int kDqSched = 8;
-// arrivals that free a hand-over slot: MMA lane, 4 epilogue warps, 4 decoder warps, 2 loader warps
-constexpr int kDqSchedReaders = 11;
+// arrivals that free a hand-over slot: MMA lane, 4 epilogue warps, 8 decoder warps, 2 loader warps
+constexpr int kDqSchedReaders = 15;
 // Raw stage of one 64-element K slab of 256 weight rows, per weight format:
 //   DQ_NV  NVFP4: codes 256 rows x 32 bytes, then two 512-byte E4M3 scale blocks
 //          (rows 0..127, 128..255; 4 scales per row);
@@ -76,24 +90,24 @@ struct DqRaw<DQ_F8> {
 
 template <int NB, int F>
 struct DqGeom {
-  static constexpr int A_BYTES = 2 * 128 * 128;           // two 128-row x 64-element bf16 tiles
-  static constexpr int B_OFF = A_BYTES;
   static constexpr int B_BYTES = NB * 128;                 // NB token rows x 64 bf16
-  static constexpr int OP_STAGE = A_BYTES + B_BYTES;       // multiple of 1024
-  static constexpr int OP_STAGES = NB >= 128 ? 3 : 4;
+  static constexpr int OP_STAGE = B_BYTES;                 // multiple of 1024
+  static constexpr int OP_STAGES = 4;
+  static constexpr int A_COLS = 64;                        // TMEM columns of one stage's A (2 halves x 32)
+  static constexpr int ACC_COLS = 2 * NB;                  // gate + up (or the two down halves)
+  static constexpr int NBUF = (512 - OP_STAGES * A_COLS) / ACC_COLS >= 2 ? 2 : 1;
+  static constexpr int A_TMEM = NBUF * ACC_COLS;           // first A column
+  static constexpr int TMEM_COLS = 512;
   static constexpr int RAW_OFF = OP_STAGES * OP_STAGE;
   static constexpr int RAW_BYTES = DqRaw<F>::BYTES;
   // raw stages in what is left of 227 KB (1 KB alignment slack, 4 KB for the static part)
   static constexpr int RAW_FIT = (227 * 1024 - 1024 - 4096 - RAW_OFF) / RAW_BYTES;
-  static constexpr int RAW_STAGES = RAW_FIT < 8 ? RAW_FIT : 8;
-  static constexpr int NBUF = 2;
-  static constexpr int COLS = NBUF * 2 * NB;
-  static constexpr int TMEM_COLS = COLS <= 128 ? 128 : (COLS <= 256 ? 256 : 512);
+  static constexpr int RAW_STAGES = RAW_FIT < 12 ? RAW_FIT : 12;
   static constexpr size_t SMEM = (size_t)RAW_OFF + (size_t)RAW_STAGES * RAW_BYTES + 1024;
   static_assert(OP_STAGE % 1024 == 0, "operand stages must keep the 1024-byte swizzle alignment");
   static_assert(RAW_BYTES % 512 == 0, "raw stages keep 128-byte TMA destinations");
   static_assert(RAW_STAGES >= 3, "raw ring depth");
-  static_assert(COLS <= 512, "TMEM budget");
+  static_assert(A_TMEM + OP_STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared-memory budget");
 };
 
@@ -108,13 +122,15 @@ __device__ __forceinline__ uint32_t idesc_bf16_dq(int M, int N) {
   return d;
 }
 
-__device__ __forceinline__ void umma_bf16_dq(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+// D (TMEM) += A (TMEM: lane = row, two bf16 per column, lower K in the low
+// half) x B (shared memory, descriptor).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -131,32 +147,47 @@ __device__ __forceinline__ TileInfo load_tile_dq(const TileInfo *p) {
   return TileInfo{v.x, v.y, v.z, v.w};
 }
 
-// f16x2 -> bf16x2 for values exactly representable in bf16 (no rounding happens).
-__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
-  const float lo = __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
-  const float hi = __half2float(__ushort_as_half((unsigned short)(h >> 16)));
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// Eight E2M1 codes (one 32-bit word, element 2i in the low nibble of byte i)
-// times one E4M3 scale (f16x2 with the scale in both halves) -> eight bf16.
-__device__ __forceinline__ uint4 decode8(uint32_t w, uint32_t sc2) {
-  uint32_t f[4];
-  e2m1x8_to_f16x2(w, f);
-  uint4 o;
-  o.x = f16x2_to_bf16x2(hmul2_u32(f[0], sc2));
-  o.y = f16x2_to_bf16x2(hmul2_u32(f[1], sc2));
-  o.z = f16x2_to_bf16x2(hmul2_u32(f[2], sc2));
-  o.w = f16x2_to_bf16x2(hmul2_u32(f[3], sc2));
-  return o;
-}
-
 __device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t r;
   asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
+}
+
+// f16x2 -> bf16x2 of the same two values times 2^-112, for values whose f16
+// significand has its low three bits zero (E2M1 values, E4M3 values): the
+// 5-bit exponent and the top 7 mantissa bits move down by three bit positions
+// into the bf16 fields, so the bf16 exponent field equals the f16 one (a bias
+// difference of 127 - 15 = 112); zeros and f16 subnormals map the same way.
+// Integer operations only, where a conversion through fp32 would take three
+// conversions per pair.
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2_m112(uint32_t h) {
+  return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
+}
+
+constexpr uint32_t kBf16x2Pow112 = 0x77807780u;   // 2^112 in both halves
+constexpr uint32_t kBf16x2NegZero = 0x80008000u;
+
+// Two E4M3 block scales (low byte first) -> bf16x2 of scale * 2^112, exact
+// (scales lie in [2^-9, 448]; the result in [2^103, 2^121]).
+__device__ __forceinline__ uint32_t nv_scale2_p112(uint16_t two_codes) {
+  const uint32_t t = f16x2_to_bf16x2_m112(e4m3x2_to_f16x2(two_codes));   // scale * 2^-112
+  return bf16x2_fma(bf16x2_fma(t, kBf16x2Pow112, kBf16x2NegZero), kBf16x2Pow112, kBf16x2NegZero);
+}
+
+// Eight E2M1 codes (one 32-bit word, element 2i in the low nibble of byte i)
+// times one E4M3 scale -> eight bf16.  sc2: bf16x2 of scale * 2^112 in both
+// halves.  Each code becomes v * 2^-112 in bf16 and one bf16 multiply by
+// scale * 2^112 gives v * scale exactly (at most 6 significant bits, in
+// [2^-10, 2688]).
+__device__ __forceinline__ uint4 decode8(uint32_t w, uint32_t sc2) {
+  uint32_t f[4];
+  e2m1x8_to_f16x2(w, f);
+  uint4 o;
+  o.x = bf16x2_fma(f16x2_to_bf16x2_m112(f[0]), sc2, kBf16x2NegZero);
+  o.y = bf16x2_fma(f16x2_to_bf16x2_m112(f[1]), sc2, kBf16x2NegZero);
+  o.z = bf16x2_fma(f16x2_to_bf16x2_m112(f[2]), sc2, kBf16x2NegZero);
+  o.w = bf16x2_fma(f16x2_to_bf16x2_m112(f[3]), sc2, kBf16x2NegZero);
+  return o;
 }
 
 // Eight INT4 codes (two's complement nibbles, element 2i in the low nibble of
@@ -353,7 +384,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         const int buf = n % NBUF;
         if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 54)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * 2 * NB);
+        const uint32_t acc = tmem + (uint32_t)(buf * Geo::ACC_COLS);
         const uint32_t idesc = idesc_bf16_dq(128, N);
         bool failed = false;
         for (int slab = 0; slab < nslab; ++slab) {
@@ -361,14 +392,14 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
           fence_proxy_async_dq();
           tc_fence_after();
           const uint32_t st = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
+          const uint32_t at = tmem + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {                   // K = 16 per MMA
-            const uint64_t bdesc = umma_desc(st + Geo::B_OFF + 32 * kk, 16, 1024, 2);
+          for (int kk = 0; kk < 4; ++kk) {                   // K = 16 per MMA (8 TMEM columns of A)
+            const uint64_t bdesc = umma_desc(st + 32 * kk, 16, 1024, 2);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint64_t adesc = umma_desc(st + h * 16384 + 32 * kk, 16, 1024, 2);
-              umma_bf16_dq(acc + (uint32_t)(h * NB), adesc, bdesc, idesc, (slab > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int h = 0; h < 2; ++h)
+              umma_bf16_ts(acc + (uint32_t)(h * NB), at + (uint32_t)(h * 32 + 8 * kk), bdesc, idesc,
+                           (slab > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(smem_u32(&op_empty[s]));                 // stage free once these MMAs finish
           if (++s == SO) { s = 0; ph ^= 1u; }
@@ -382,9 +413,12 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       tc_commit(smem_u32(&quiesce_bar));
       mbar_drain(smem_u32(&quiesce_bar), 0);
     }
-  } else if (warp >= 6 && warp < 10) {
-    // ---------------- decoders: raw codes + E4M3 scales -> bf16 weight tile
-    const int d = threadIdx.x - 192;                         // 0..127: rows d and d + 128 of the 256
+  } else if (warp >= 6 && warp < 14) {
+    // ---------------- decoders: raw codes + scales -> bf16 weight rows in TMEM
+    const int quad = warp & 3;                               // TMEM lane quadrant of this warp
+    const int hh = warp >= 10 ? 1 : 0;                       // first or second 128 rows of the 256
+    const int rr = 32 * quad + lane;                         // row within the 128-row half
+    const int row = 128 * hh + rr;                           // row of the 256 in the raw stage
     int r = 0, s = 0, n_slabs = 0;
     uint32_t rph = 0, sph = 0;
     int q = 0;
@@ -403,67 +437,95 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       if (++q == kDqSched) { q = 0; qph ^= 1u; }
       if (item < 0) break;
       if (loc == kLocAbsent) continue;
-      for (int slab = 0; slab < nslab; ++slab) {
-        int ok = 1;
-        if (lane == 0) {
-          ok = mbar_wait(smem_u32(&raw_full[r]), rph, a.err, 53) ? 1 : 0;
-          if (ok && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 55) ? 1 : 0;
+      if constexpr (F == DQ_F8) {
+        // base of this row's fp32 block scales (one per 128 K) in the blob
+        const int m = MODE == MODE_GATEUP ? hh : 2;
+        const int rbk = MODE == MODE_GATEUP ? item % ipt : 2 * (item % ipt) + hh;
+        const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
+        const float *bsp = reinterpret_cast<const float *>(blob + a.L.scales[m]) + (size_t)rbk * (K / 128);
+        for (int slab = 0; slab < nslab; ++slab) {
+          int ok = 1;
+          if (lane == 0) {
+            ok = mbar_wait(smem_u32(&raw_full[r]), rph, a.err, 53) ? 1 : 0;
+            if (ok && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 55) ? 1 : 0;
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) { failed = true; break; }
+          tc_fence_after();
+          const uint8_t *raw = smem + Geo::RAW_OFF + (size_t)r * kRawBytes;
+          const float sblk = __ldg(bsp + slab / 2);
+          uint32_t v[32];
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint4 cv = *reinterpret_cast<const uint4 *>(raw + row * 64 + c4 * 16);
+            const uint4 o0 = decode8_fp8(cv.x, cv.y, sblk), o1 = decode8_fp8(cv.z, cv.w, sblk);
+            v[8 * c4 + 0] = o0.x; v[8 * c4 + 1] = o0.y; v[8 * c4 + 2] = o0.z; v[8 * c4 + 3] = o0.w;
+            v[8 * c4 + 4] = o1.x; v[8 * c4 + 5] = o1.y; v[8 * c4 + 6] = o1.z; v[8 * c4 + 7] = o1.w;
+          }
+          tmem_st32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS + 32 * hh), v);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(&raw_empty[r]));
+            mbar_arrive(smem_u32(&op_full[s]));
+          }
+          ++n_slabs;
+          if (++r == SR) { r = 0; rph ^= 1u; }
+          if (++s == SO) { s = 0; sph ^= 1u; }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) { failed = true; break; }
-        const uint8_t *raw = smem + Geo::RAW_OFF + (size_t)r * kRawBytes;
-        const uint32_t ast = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
+      } else {
+        for (int slab = 0; slab < nslab; ++slab) {
+          int ok = 1;
+          if (lane == 0) {
+            ok = mbar_wait(smem_u32(&raw_full[r]), rph, a.err, 53) ? 1 : 0;
+            if (ok && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 55) ? 1 : 0;
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) { failed = true; break; }
+          tc_fence_after();
+          const uint8_t *raw = smem + Geo::RAW_OFF + (size_t)r * kRawBytes;
+          const uint4 c0 = *reinterpret_cast<const uint4 *>(raw + row * 32);
+          const uint4 c1 = *reinterpret_cast<const uint4 *>(raw + row * 32 + 16);
+          const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          uint32_t v[32];
+          if constexpr (F == DQ_NV) {
+            const uint32_t sf4 =
+                *reinterpret_cast<const uint32_t *>(raw + 8192 + hh * 512 + 16 * (rr & 31) + 4 * (rr >> 5));
+            const uint32_t s01 = nv_scale2_p112((uint16_t)(sf4 & 0xFFFFu));
+            const uint32_t s23 = nv_scale2_p112((uint16_t)(sf4 >> 16));
+            const uint32_t sc[4] = {dup_lo16(s01), dup_hi16(s01), dup_lo16(s23), dup_hi16(s23)};
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int row = d + 128 * hh;                      // row of the 256 in the raw stage
-          const int rr = row & 127;
-          const uint32_t rowa = ast + hh * 16384 + rr * 128;
-          if constexpr (F == DQ_F8) {
-            // the fp32 scale of this row's 128 x 128 block, from the blob
-            const int m = MODE == MODE_GATEUP ? hh : 2;
-            const int rbk = MODE == MODE_GATEUP ? item % ipt : 2 * (item % ipt) + hh;
-            const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
-            const float bs = __ldg(reinterpret_cast<const float *>(blob + a.L.scales[m]) + (size_t)rbk * (K / 128) + slab / 2);
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const uint4 cv = *reinterpret_cast<const uint4 *>(raw + row * 64 + c4 * 16);
-              sts128(rowa + (((2 * c4) ^ (rr & 7)) << 4), decode8_fp8(cv.x, cv.y, bs));
-              sts128(rowa + (((2 * c4 + 1) ^ (rr & 7)) << 4), decode8_fp8(cv.z, cv.w, bs));
+            for (int c = 0; c < 8; ++c) {
+              const uint4 o = decode8(w[c], sc[c >> 1]);
+              v[4 * c + 0] = o.x; v[4 * c + 1] = o.y; v[4 * c + 2] = o.z; v[4 * c + 3] = o.w;
             }
           } else {
-            const uint4 c0 = *reinterpret_cast<const uint4 *>(raw + row * 32);
-            const uint4 c1 = *reinterpret_cast<const uint4 *>(raw + row * 32 + 16);
-            const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            if constexpr (F == DQ_NV) {
-              const uint32_t sf4 =
-                  *reinterpret_cast<const uint32_t *>(raw + 8192 + hh * 512 + 16 * (rr & 31) + 4 * (rr >> 5));
-              const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(sf4 & 0xFFFFu));
-              const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(sf4 >> 16));
-              const uint32_t sc[4] = {dup_lo16(s01), dup_hi16(s01), dup_lo16(s23), dup_hi16(s23)};
+            const uint32_t sb = *reinterpret_cast<const uint16_t *>(raw + 8192 + hh * 256 + rr * 2);
+            const uint32_t sc2 = sb | (sb << 16);
 #pragma unroll
-              for (int c = 0; c < 8; ++c) sts128(rowa + ((c ^ (rr & 7)) << 4), decode8(w[c], sc[c >> 1]));
-            } else {
-              const uint32_t sb = *reinterpret_cast<const uint16_t *>(raw + 8192 + hh * 256 + rr * 2);
-              const uint32_t sc2 = sb | (sb << 16);
-#pragma unroll
-              for (int c = 0; c < 8; ++c) sts128(rowa + ((c ^ (rr & 7)) << 4), decode8_int4(w[c], sc2));
+            for (int c = 0; c < 8; ++c) {
+              const uint4 o = decode8_int4(w[c], sc2);
+              v[4 * c + 0] = o.x; v[4 * c + 1] = o.y; v[4 * c + 2] = o.z; v[4 * c + 3] = o.w;
             }
           }
+          tmem_st32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS + 32 * hh), v);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(&raw_empty[r]));
+            mbar_arrive(smem_u32(&op_full[s]));
+          }
+          ++n_slabs;
+          if (++r == SR) { r = 0; rph ^= 1u; }
+          if (++s == SO) { s = 0; sph ^= 1u; }
         }
-        fence_proxy_async_dq();                              // generic-proxy writes -> tensor-core reads
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(smem_u32(&raw_empty[r]));
-          mbar_arrive(smem_u32(&op_full[s]));
-        }
-        ++n_slabs;
-        if (++r == SR) { r = 0; rph ^= 1u; }
-        if (++s == SO) { s = 0; sph ^= 1u; }
       }
     }
-  } else if (warp >= 10) {
+  } else if (warp >= 14) {
     // ---------------- activation loaders: the tile's bf16 rows of this K slab
-    const int lt = threadIdx.x - 320;                        // 0..63
+    const int lt = threadIdx.x - 448;                        // 0..63
     int s = 0, n_slabs = 0;
     uint32_t sph = 0;
     int q = 0;
@@ -483,25 +545,37 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       if (++q == kDqSched) { q = 0; qph ^= 1u; }
       if (item < 0) break;
       if (loc == kLocAbsent) continue;
-      const int N = max(16, (ti.nrows + 15) & ~15);
-      // this thread's rows: j = lt / 8 + 8 i; 16-byte chunk lt % 8 of each
+      // this thread's rows: j = lt / 8 + 8 i, 16-byte chunk lt % 8 of each;
+      // their element offsets are looked up once per item (one round of
+      // independent loads), not per slab; rows past the tile's tokens are
+      // pad columns the epilogue never stores and are not copied
+      constexpr int RPT = NB / (kDqLoaders / 8);
       const int cq = lt & 7;
+      uint32_t roff[RPT];
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int j = (lt >> 3) + (kDqLoaders / 8) * i;
+        roff[i] = 0xFFFFFFFFu;
+        if (j < ti.nrows) {
+          if constexpr (MODE == MODE_GATEUP) {
+            const int tok = checked_index(__ldg(a.prow_token + ti.prow0 + j), 0, a.db.n_tokens, 0, a.db.err, kChkToken);
+            roff[i] = (uint32_t)tok * (uint32_t)K;
+          } else {
+            roff[i] = (uint32_t)(ti.prow0 + j) * (uint32_t)K;
+          }
+        }
+      }
       for (int slab = 0; slab < nslab; ++slab) {
         int ok = 1;
         if (lane == 0 && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 56) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { failed = true; break; }
-        const uint32_t bst = smem_u32(smem + (size_t)s * Geo::OP_STAGE + Geo::B_OFF);
-        for (int j = lt >> 3; j < N; j += kDqLoaders / 8) {
-          if (j >= ti.nrows) continue;                       // pad columns: never stored by the epilogue
-          const uint16_t *src;
-          if constexpr (MODE == MODE_GATEUP) {
-            const int tok = checked_index(__ldg(a.prow_token + ti.prow0 + j), 0, a.db.n_tokens, 0, a.db.err, kChkToken);
-            src = a.act + (size_t)tok * K;
-          } else {
-            src = a.act + (size_t)(ti.prow0 + j) * K;
-          }
-          cp_async16_dq(bst + j * 128 + ((cq ^ (j & 7)) << 4), src + slab * 64 + cq * 8);
+        const uint32_t bst = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+          const int j = (lt >> 3) + (kDqLoaders / 8) * i;
+          if (roff[i] != 0xFFFFFFFFu)
+            cp_async16_dq(bst + j * 128 + ((cq ^ (j & 7)) << 4), a.act + roff[i] + slab * 64 + cq * 8);
         }
         cp_async_arrive_dq(smem_u32(&op_full[s]));
         ++n_slabs;

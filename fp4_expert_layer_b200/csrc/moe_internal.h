@@ -36,7 +36,8 @@ struct BlobLayout {
   int K[3];
   int G;              // block size along K: 32 (MXFP4) or 16 (NVFP4)
   int fmt;
-  int tiled;          // 1: tile-major codes and scales (tensor-core EXACT layers), see below
+  int tiled;          // 1: tile-major codes and scales (tensor-core EXACT layers);
+                      // 2: gate and up interleaved per 64 rows (A4 layers); see below
 };
 
 // tiled = 0: codes in checkpoint order ([rows, K/2] per matrix), scales in
@@ -48,6 +49,11 @@ struct BlobLayout {
 // and the scale blocks of a chunk (gate, up / rows 0..127, 128..255 of the
 // chunk) are one contiguous 1 KB at the same chunk index.  codes[0] / scales[0]
 // start the gate/up regions, codes[2] / scales[2] the down regions.
+// tiled = 2 (A4 layers): gate and up form one matrix of 2I rows from codes[0]
+// / scales[0] (the two regions are adjacent), row c holding gate row
+// (c / 128) * 64 + c % 64 when (c / 64) is even, else that up row; codes in
+// checkpoint row format, scales in 512-byte blocks (sf_offset over the 2I
+// rows); down as in tiled = 0.
 BlobLayout blob_layout(int H, int I, int fmt, int tiled);
 constexpr int kTcChunk = 16384;      // code bytes of one tiled chunk
 constexpr int kTcSfChunk = 1024;     // scale bytes of one tiled chunk
@@ -234,7 +240,10 @@ struct QuantArgs {
 void launch_quant(const QuantArgs &q, cudaStream_t s);
 
 struct A4Maps {
-  CUtensorMap w[2][3];       // [slot | staging][matrix]: code bytes, box 128 B x 128 rows, 128-byte swizzle
+  // [slot | staging][matrix]: code bytes, box 128 B x 128 rows, 128-byte
+  // swizzle; matrix 0 is gate and up together (2I rows interleaved per 64,
+  // blob layout tiled = 2), 1 is unused, 2 is down
+  CUtensorMap w[2][3];
   CUtensorMap act[2];        // [x | h]: quantised activation rows, box 128 B x 128 rows, 128-byte swizzle
 };
 
@@ -260,9 +269,13 @@ struct A4GemmArgs {
   const int *prow_pair;
   const float *gates;
   int *err;
+  int *work_ctr;             // item counter of this pass, zero at launch
+  int grid;                  // persistent CTAs
   DevBounds db;           // device bounds checks (checked build)
 };
-void launch_gemm_a4(int wf, int mode, const A4GemmArgs &a, int grid_tiles, cudaStream_t s);
+// rows: h width I (gate/up; items cover 64 h columns each, n_rowblocks = I / 64)
+// or H (down; n_rowblocks = H / 128).
+void launch_gemm_a4(int wf, int mode, const A4GemmArgs &a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // EXACT numerics on the tensor core (MXFP4 experts): the weights stay E2M1
