@@ -39,9 +39,8 @@
 //                G_d * gate * acc -> O' (fp32, pair order);
 //   warps 6..13  decoders: raw stage -> bf16 weight rows in TMEM, warp w the
 //                rows of TMEM lane quadrant w % 4 of the first (w < 10) or
-//                second 128 rows (NVFP4: one hardware E2M1 -> f16x2
-//                conversion per two codes, then integer bit moves and one
-//                bf16 multiply by the scale);
+//                second 128 rows (NVFP4: hardware E2M1 -> f16x2, an f16
+//                multiply by the scale, widening to bf16);
 //   warps 14..15 activation loaders: the tile's bf16 rows of this K slab by
 //                16-byte cp.async (x rows gathered through the padded-row ->
 //                token map for gate/up; h rows for down), 128-byte swizzled
@@ -153,40 +152,30 @@ __device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t 
   return r;
 }
 
-// f16x2 -> bf16x2 of the same two values times 2^-112, for values whose f16
-// significand has its low three bits zero (E2M1 values, E4M3 values): the
-// 5-bit exponent and the top 7 mantissa bits move down by three bit positions
-// into the bf16 fields, so the bf16 exponent field equals the f16 one (a bias
-// difference of 127 - 15 = 112); zeros and f16 subnormals map the same way.
-// Integer operations only, where a conversion through fp32 would take three
-// conversions per pair.
-__device__ __forceinline__ uint32_t f16x2_to_bf16x2_m112(uint32_t h) {
-  return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
-}
-
-constexpr uint32_t kBf16x2Pow112 = 0x77807780u;   // 2^112 in both halves
-constexpr uint32_t kBf16x2NegZero = 0x80008000u;
-
-// Two E4M3 block scales (low byte first) -> bf16x2 of scale * 2^112, exact
-// (scales lie in [2^-9, 448]; the result in [2^103, 2^121]).
-__device__ __forceinline__ uint32_t nv_scale2_p112(uint16_t two_codes) {
-  const uint32_t t = f16x2_to_bf16x2_m112(e4m3x2_to_f16x2(two_codes));   // scale * 2^-112
-  return bf16x2_fma(bf16x2_fma(t, kBf16x2Pow112, kBf16x2NegZero), kBf16x2Pow112, kBf16x2NegZero);
+// f16x2 -> bf16x2 for values exactly representable in bf16 (no rounding
+// happens): the two halves widen to fp32 on the FMA pipe and one conversion
+// packs them, so the decode spends two integer-pipe instructions per pair
+// (this one and the E2M1 conversion) and three on the otherwise idle FMA pipe.
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
+  const float lo = __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
+  const float hi = __half2float(__ushort_as_half((unsigned short)(h >> 16)));
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Eight E2M1 codes (one 32-bit word, element 2i in the low nibble of byte i)
-// times one E4M3 scale -> eight bf16.  sc2: bf16x2 of scale * 2^112 in both
-// halves.  Each code becomes v * 2^-112 in bf16 and one bf16 multiply by
-// scale * 2^112 gives v * scale exactly (at most 6 significant bits, in
-// [2^-10, 2688]).
+// times one E4M3 scale (f16x2 with the scale in both halves) -> eight bf16:
+// the f16 product is exact (at most 6 significant bits, in [2^-10, 2688]) and
+// so is its bf16.
 __device__ __forceinline__ uint4 decode8(uint32_t w, uint32_t sc2) {
   uint32_t f[4];
   e2m1x8_to_f16x2(w, f);
   uint4 o;
-  o.x = bf16x2_fma(f16x2_to_bf16x2_m112(f[0]), sc2, kBf16x2NegZero);
-  o.y = bf16x2_fma(f16x2_to_bf16x2_m112(f[1]), sc2, kBf16x2NegZero);
-  o.z = bf16x2_fma(f16x2_to_bf16x2_m112(f[2]), sc2, kBf16x2NegZero);
-  o.w = bf16x2_fma(f16x2_to_bf16x2_m112(f[3]), sc2, kBf16x2NegZero);
+  o.x = f16x2_to_bf16x2(hmul2_u32(f[0], sc2));
+  o.y = f16x2_to_bf16x2(hmul2_u32(f[1], sc2));
+  o.z = f16x2_to_bf16x2(hmul2_u32(f[2], sc2));
+  o.w = f16x2_to_bf16x2(hmul2_u32(f[3], sc2));
   return o;
 }
 
@@ -492,8 +481,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
           if constexpr (F == DQ_NV) {
             const uint32_t sf4 =
                 *reinterpret_cast<const uint32_t *>(raw + 8192 + hh * 512 + 16 * (rr & 31) + 4 * (rr >> 5));
-            const uint32_t s01 = nv_scale2_p112((uint16_t)(sf4 & 0xFFFFu));
-            const uint32_t s23 = nv_scale2_p112((uint16_t)(sf4 >> 16));
+            const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(sf4 & 0xFFFFu));
+            const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(sf4 >> 16));
             const uint32_t sc[4] = {dup_lo16(s01), dup_hi16(s01), dup_lo16(s23), dup_hi16(s23)};
 #pragma unroll
             for (int c = 0; c < 8; ++c) {

@@ -21,9 +21,10 @@
 //
 // Persistent, one CTA per SM, work items taken from a counter in index order.
 // Warp roles: warp 0 takes the items and issues the copies (one lane), warp 1
-// allocates TMEM and one lane issues every MMA, warps 2..5 (one per TMEM lane
-// quadrant) read the accumulators back with tcgen05.ld.  All mbarrier waits
-// are bounded.
+// allocates TMEM and one lane issues every MMA, warps 2..9 read the
+// accumulators back with tcgen05.ld (warp w the lanes of quadrant w % 4; warps
+// 2..5 tokens 0..63 of an item, warps 6..9 tokens 64..127).  All mbarrier
+// waits are bounded.
 //
 // TMEM columns: accumulators at 0 and 128; the A and B scale blocks of stage
 // s at 256 + s * SF_COLS (16 columns per stage for MXFP4, 32 for NVFP4).
@@ -55,9 +56,10 @@ __device__ __forceinline__ TileInfo load_tile_a4(const TileInfo *p) {
 }
 
 constexpr int kTileBytes = 128 * 128;   // 128 rows x 128 bytes (256 FP4 per row)
-constexpr int kGThreads = 192;          // warp 0 copies, warp 1 MMA, warps 2..5 epilogue
+constexpr int kGThreads = 320;          // warp 0 copies, warp 1 MMA, warps 2..9 epilogue
+constexpr int kGEpi = 256;              // epilogue threads
 constexpr int kGSched = 4;
-constexpr int kGSchedReaders = 5;       // MMA lane + 4 epilogue warps
+constexpr int kGSchedReaders = 9;       // MMA lane + 8 epilogue warps
 
 }  // namespace
 
@@ -75,7 +77,7 @@ struct GemmGeom {
   static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024;
   static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static_assert(SF_TMEM + STAGES * SF_COLS <= 512, "TMEM budget");
-  static_assert(SMEM + 12 * 1024 <= 227 * 1024, "shared-memory budget");
+  static_assert(SMEM + 22 * 1024 <= 227 * 1024, "shared-memory budget");
 };
 
 template <int WF, int MODE>
@@ -100,12 +102,15 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
   __shared__ float col_bs[128];
   __shared__ int col_pair[128];
   __shared__ float col_gate[128];
-  // gate/up: the up rows' values of 32 tokens, handed to the gate rows' warps
-  __shared__ float xchg[64][33];
-  // MXFP4 gate/up with h quantised in the epilogue: per gate warp, the codes
-  // and block scales of 32 tokens before they go out
-  __shared__ __align__(16) uint8_t hq_stage[2][32][16];
-  __shared__ uint8_t sf_stage[2][32];
+  // gate/up, per epilogue group: gate values of the second 16 tokens of a
+  // 32-token chunk (for the up warps) and up values of the first 16 (for the
+  // gate warps), 64 rows each
+  __shared__ float xg[2][64][17];
+  __shared__ float xu[2][64][17];
+  // MXFP4 gate/up with h quantised in the epilogue: per epilogue warp, the
+  // codes and block scales of its 16 tokens before they go out
+  __shared__ __align__(16) uint8_t hq_stage[8][16][16];
+  __shared__ uint8_t sf_stage[8][16];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -122,7 +127,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(smem_u32(&accf_bar[b]), 1);
-      mbar_init(smem_u32(&acce_bar[b]), 4);
+      mbar_init(smem_u32(&acce_bar[b]), kGEpi / 32);
     }
     for (int q = 0; q < kGSched; ++q) {
       mbar_init(smem_u32(&sched_full[q]), 1);
@@ -257,9 +262,13 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
       mbar_drain(smem_u32(&quiesce_bar), 0);
     }
   } else {
-    // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+    // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31; the
+    // warps 2..5 (group 0) take tokens 0..63 of an item, warps 6..9 (group 1)
+    // tokens 64..127
     const int quad = warp & 3;
-    const int et = threadIdx.x - 64;                                 // 0..127 over warps 2..5
+    const int grp = (warp - 2) >> 2;
+    const int wslot = warp - 2;
+    const int et = threadIdx.x - 64;                                 // 0..255 over warps 2..9
     int n = 0;
     bool ok = true;
     int q = 0;
@@ -275,14 +284,14 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
       __syncwarp();
       if (okw && lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
       if (++q == kGSched) { q = 0; qph ^= 1u; }
-      // the four warps stop together (each takes every named barrier below)
-      if (!named_bar_and(1, 128, okw != 0 && item >= 0)) break;
+      // the eight warps stop together (each takes every named barrier below)
+      if (!named_bar_and(1, kGEpi, okw != 0 && item >= 0)) break;
       if (loc == kLocAbsent) continue;
       const int rb = item % ipt;
       const int prow0 = ti.prow0, nrows = ti.nrows;
       const int buf = n % NBUF;
       const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
-      if (et < nrows) {
+      if (et < nrows && et < 128) {
         col_bs[et] = (WF == WF_NV) ? __ldg(a.bG + prow0 + et) : 1.0f;
         if constexpr (MODE == MODE_DOWN) {
           const int p = checked_index(__ldg(a.prow_pair + prow0 + et), 0, a.db.n_pairs, 0, a.db.err, kChkPair);
@@ -291,79 +300,91 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
         }
       }
       ok = mbar_wait(smem_u32(&accf_bar[buf]), (n / NBUF) & 1, a.err, 13);
-      ok = named_bar_and(1, 128, ok);                                 // also publishes col_*
+      ok = named_bar_and(1, kGEpi, ok);                               // also publishes col_*
       tc_fence_after();
       const uint32_t acc = tmem + (uint32_t)(buf * 128) + ((uint32_t)(32 * quad) << 16);
       if constexpr (MODE == MODE_GATEUP) {
-        // lanes 0..63: gate rows, 64..127: up rows of h columns rb*64 .. +63
+        // lanes 0..63: gate rows, 64..127: up rows of h columns rb*64 .. +63.
+        // A gate warp and the up warp of the same 32 columns split each
+        // 32-token chunk: the gate warp computes tokens 0..15, the up warp
+        // 16..31, each handing the other the values it needs
         const bool is_up = quad >= 2;
         const int half = quad & 1;
         const int I = a.rows;
-        const int hcol = rb * 64 + 32 * half + lane;
+        const int hrow = 32 * half + lane;                           // h column within the item's 64
+        const int hcol = rb * 64 + hrow;
         const float wsc = (WF == WF_NV) ? reinterpret_cast<const float *>(blob + a.L.glob)[is_up ? 1 : 0] : 1.0f;
         const bool quantise = (WF == WF_MX) && a.hq_out != nullptr;
-        for (int cb = 0; cb < 4; ++cb) {
-          if (32 * cb >= nrows) break;                               // uniform over the four warps
+        const int j0 = is_up ? 16 : 0;                               // this warp's tokens in a chunk
+        for (int cc = 0; cc < 2; ++cc) {
+          const int cb = 2 * grp + cc;
+          if (32 * cb >= nrows) break;                               // uniform over the group
           uint32_t d[32];
           tmem_ld32(acc + (uint32_t)(32 * cb), d);
           tmem_ld_wait();
-          if (is_up && ok) {
+          float v[32];
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-              xchg[32 * half + lane][jj] = __uint_as_float(d[jj]) * (wsc * col_bs[32 * cb + jj]);
+          for (int jj = 0; jj < 32; ++jj) v[jj] = __uint_as_float(d[jj]) * (wsc * col_bs[32 * cb + jj]);
+          if (ok) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              if (is_up) xu[grp][hrow][jj] = v[jj];                  // up of tokens 0..15 for the gate warp
+              else xg[grp][hrow][jj] = v[16 + jj];                   // gate of tokens 16..31 for the up warp
+            }
           }
-          named_bar_sync(1, 128);
-          if (!is_up && ok) {
+          named_bar_sync(2 + grp, 128);
+          if (ok) {
+            float h[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              h[jj] = is_up ? silu_f(xg[grp][hrow][jj]) * v[16 + jj] : silu_f(v[jj]) * xu[grp][hrow][jj];
             if (quantise) {
               // h quantised for the down pass (MXFP4 rule of the activation
               // quantiser: per 32 consecutive h columns of a token, E8M0
               // exponent clamp(floor(log2 amax) - 2 + 127, 1, 254), codes RNE
               // E2M1 of h * 2^(127 - e), saturating).  The warp's 32 lanes are
               // one block of 32 h columns of each token.
-              uint8_t(*qs)[16] = hq_stage[half];
+              uint8_t(*qs)[16] = hq_stage[wslot];
 #pragma unroll
-              for (int jj = 0; jj < 32; ++jj) {
-                const float gv = __uint_as_float(d[jj]) * (wsc * col_bs[32 * cb + jj]);
-                const float h = silu_f(gv) * xchg[32 * half + lane][jj];
+              for (int jj = 0; jj < 16; ++jj) {
                 // block maximum of |h| (non-negative floats order like their bit patterns)
-                const uint32_t am = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h)));
+                const uint32_t am = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h[jj])));
                 int code = 1;
                 if (am != 0u) {
                   const int ex = (int)((am >> 23) & 0xFF);
                   code = min(254, max(1, (ex == 0 ? -127 : ex - 127) - 2 + 127));
                 }
-                const float v = h * __int_as_float((254 - code) << 23);   // h * 2^(127 - code)
-                const float vn = __shfl_down_sync(0xffffffffu, v, 1);
-                if ((lane & 1) == 0) qs[jj][lane >> 1] = (uint8_t)(e2m1x2_pack(v, vn) & 0xFFu);
-                if (lane == 0) sf_stage[half][jj] = (uint8_t)code;
+                const float qv = h[jj] * __int_as_float((254 - code) << 23);   // h * 2^(127 - code)
+                const float qn = __shfl_down_sync(0xffffffffu, qv, 1);
+                if ((lane & 1) == 0) qs[jj][lane >> 1] = (uint8_t)(e2m1x2_pack(qv, qn) & 0xFFu);
+                if (lane == 0) sf_stage[wslot][jj] = (uint8_t)code;
               }
               __syncwarp();
-              // lane j writes token j of the chunk: 16 code bytes and one scale
-              const int col = 32 * cb + lane;
-              if (col < nrows) {
+              // lane t < 16 writes token j0 + t of the chunk: 16 code bytes and one scale
+              const int col = 32 * cb + j0 + lane;
+              if (lane < 16 && col < nrows) {
                 const size_t prow = (size_t)(prow0 + col);
                 const int c0 = rb * 64 + 32 * half;
                 *reinterpret_cast<uint4 *>(a.hq_out + prow * (I / 2) + c0 / 2) =
                     *reinterpret_cast<const uint4 *>(qs[lane]);
-                a.hsf_out[sf_offset(I / 32, (int)prow, c0 / 32)] = sf_stage[half][lane];
+                a.hsf_out[sf_offset(I / 32, (int)prow, c0 / 32)] = sf_stage[wslot][lane];
               }
               __syncwarp();
             } else {
 #pragma unroll
-              for (int jj = 0; jj < 32; ++jj) {
-                const int col = 32 * cb + jj;
-                if (col >= nrows) continue;                            // warp-uniform
-                const float gv = __uint_as_float(d[jj]) * (wsc * col_bs[col]);
-                a.h_out[(size_t)(prow0 + col) * I + hcol] = silu_f(gv) * xchg[32 * half + lane][jj];
+              for (int jj = 0; jj < 16; ++jj) {
+                const int col = 32 * cb + j0 + jj;
+                if (col < nrows) a.h_out[(size_t)(prow0 + col) * I + hcol] = h[jj];   // warp-uniform test
               }
             }
           }
-          named_bar_sync(1, 128);                                      // xchg is rewritten by the next chunk
+          named_bar_sync(2 + grp, 128);                                // xg / xu are rewritten by the next chunk
         }
       } else {
         const float wsc = (WF == WF_NV) ? reinterpret_cast<const float *>(blob + a.L.glob)[2] : 1.0f;
         const int row = rb * 128 + 32 * quad + lane;                   // output row (H index)
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int cb = 2 * grp + cc;
           if (32 * cb >= nrows) break;
           uint32_t d[32];
           tmem_ld32(acc + (uint32_t)(32 * cb), d);
@@ -381,7 +402,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&acce_bar[buf]));
-      named_bar_sync(1, 128);                                          // col_* are rewritten by the next item
+      named_bar_sync(1, kGEpi);                                        // col_* are rewritten by the next item
       ++n;
     }
   }
