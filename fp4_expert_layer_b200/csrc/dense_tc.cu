@@ -263,10 +263,12 @@ void launch_dense_tc(int mode, const DenseTcArgs &a, cudaStream_t s) {
 // thread-block cluster of S CTAs.  CTA ks of the cluster for row block rb
 // accumulates its 128 gate + 128 up rows (or 256 down rows) over the K slabs
 // [ks * nslab / S, (ks + 1) * nslab / S) for all T tokens at once (N = T
-// rounded up to 16; TMA zero-fills the rows past T), copies the partial
-// accumulators to its shared memory, and the cluster sums them in rank order
-// through distributed shared memory (the same order every run, so the result
-// does not depend on timing), each CTA finishing 128 / S of the rows.
+// rounded up to 16; TMA zero-fills the rows past T).  Once every CTA of the
+// cluster is done with its stages, each pushes its partial accumulators into
+// the shared memory of the CTA that finishes those rows (distributed shared
+// memory stores, one slot per source rank, over the stage memory), and each
+// CTA sums the slots of its 128 / S rows in rank order (the same order every
+// run, so the result does not depend on timing).
 // Roles: warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 epilogue.
 // ---------------------------------------------------------------------------
 namespace {
@@ -279,7 +281,7 @@ struct SplitGeom {
   static constexpr int STAGE = (A_BYTES + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int COLS = 2 * NP;
   static constexpr int TMEM_COLS = COLS <= 32 ? 32 : (COLS <= 64 ? 64 : (COLS <= 128 ? 128 : 256));
-  static constexpr int RED_BYTES = 2 * 128 * NP * 4;   // partial accumulators, fp32
+  static constexpr int RED_BYTES = 2 * 128 * NP * 4;   // received partial accumulators, fp32
   static constexpr size_t SMEM = (size_t)(STAGES * STAGE > RED_BYTES ? STAGES * STAGE : RED_BYTES) + 1024;
   static_assert(SMEM <= 227 * 1024, "shared-memory budget");
 };
@@ -297,7 +299,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
   __shared__ int ok_s;
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sk_smem_raw) + 1023) & ~uintptr_t(1023));
-  float *red = reinterpret_cast<float *>(smem);       // [2][128][NP], over the stages once they are consumed
+  // partials received from the cluster's ranks: [source rank][half][128 / S rows][NP],
+  // over the stages once every CTA of the cluster is done with them
+  float *recv = reinterpret_cast<float *>(smem);
   cg::cluster_group cluster = cg::this_cluster();
   const int S = (int)cluster.num_blocks();
   const int ks = (int)cluster.block_rank();
@@ -387,37 +391,49 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
       mbar_drain(smem_u32(&accf_bar), 0);
       if (failed) ok_s = 0;
     }
-  } else {
-    // epilogue warps: partial accumulators -> shared memory (rows 32*quad + lane)
-    const int quad = warp & 3;
-    const bool ok = mbar_wait(smem_u32(&accf_bar), 0, a.err, 48);
+  }
+  bool ok = true;
+  if (warp >= 2) {
+    ok = mbar_wait(smem_u32(&accf_bar), 0, a.err, 48);
+    if (!ok) ok_s = 0;
+  }
+  tc_fence_before();
+  cluster.sync();                                      // every rank is done with its stage memory
+  const int rows = 128 / S, r0 = ks * rows;
+  if (warp >= 2) {
+    // push this rank's partials (rows 32*quad + lane) into the receive slot
+    // [ks] of the rank that finishes them
     tc_fence_after();
+    const int quad = warp & 3;
+    const int row = 32 * quad + lane;
+    const int owner = row / rows, rl = row % rows;
+    float *dst = cluster.map_shared_rank(recv, owner);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int row = 32 * quad + lane;
 #pragma unroll
       for (int c0 = 0; c0 < NP; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem + (uint32_t)(h * NP + c0) + ((uint32_t)(32 * quad) << 16), v);
         tmem_ld_wait();
+        float4 *d4 = reinterpret_cast<float4 *>(dst + (((size_t)ks * 2 + h) * rows + rl) * NP + c0);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) red[(h * 128 + row) * NP + c0 + j] = ok ? __uint_as_float(v[j]) : 0.0f;
+        for (int j = 0; j < 4; ++j)
+          d4[j] = ok ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                     : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       }
     }
-    if (!ok) ok_s = 0;
   }
-  tc_fence_before();
-  cluster.sync();                                      // every rank's partials are in its shared memory
+  cluster.sync();                                      // every partial is in its owner's shared memory
   // this rank finishes rows [ks * 128 / S, (ks + 1) * 128 / S) of both halves,
-  // summing the ranks' partials in rank order
-  const int rows = 128 / S, r0 = ks * rows;
+  // summing the slots in rank order (local shared memory only)
   for (int i = threadIdx.x; i < rows * NP; i += blockDim.x) {
-    const int r = r0 + i / NP, c = i % NP;
+    const int rl = i / NP, c = i % NP;
+    const int r = r0 + rl;
     float v0 = 0.0f, v1 = 0.0f;
     for (int q = 0; q < S; ++q) {
-      const float *rr = cluster.map_shared_rank(red, q);
-      v0 += rr[(0 * 128 + r) * NP + c];
-      v1 += rr[(1 * 128 + r) * NP + c];
+      v0 += recv[(((size_t)q * 2 + 0) * rows + rl) * NP + c];
+      v1 += recv[(((size_t)q * 2 + 1) * rows + rl) * NP + c];
     }
     if (c >= a.T) continue;
     if constexpr (MODE == MODE_GATEUP) {
@@ -427,7 +443,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
       a.s_out[(size_t)c * a.rows + rb * 256 + 128 + r] = v1;
     }
   }
-  cluster.sync();                                      // no rank leaves while others read its partials
+  tc_fence_before();
+  __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Geo::TMEM_COLS);
