@@ -1141,7 +1141,11 @@ static moe_status_t run_experts_dq(moe_layer *L, const int *locs, const void *x,
   a.K = c.hidden;
   a.rows = c.inter;
   a.n_rowblocks = c.inter / 128;
-  a.act = reinterpret_cast<const uint16_t *>(x);
+  // NVFP4: x as f16 rows with a power-of-two scale per token (written into
+  // the f16 activation buffer by the conversion before the first pass)
+  const bool f16x = c.fmt == MOE_FMT_NVFP4;
+  a.act = f16x ? L->xf16 : reinterpret_cast<const uint16_t *>(x);
+  a.act_scale = f16x ? L->xs : nullptr;
   a.h_out = L->hbuf;
   a.work_ctr = L->dq_work;
   a.wfmt = c.fmt == MOE_FMT_INT4G128 ? DQ_I4 : (c.fmt == MOE_FMT_FP8B128 ? DQ_F8 : DQ_NV);
@@ -1155,6 +1159,7 @@ static moe_status_t run_experts_dq(moe_layer *L, const int *locs, const void *x,
   a.rows = c.hidden;
   a.n_rowblocks = c.hidden / 256;
   a.act = L->hbuf;
+  a.act_scale = nullptr;
   a.o_out = L->oprime;
   a.work_ctr = L->dq_work + 1;
   a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
@@ -1446,6 +1451,15 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     q.xsf = L->txsf;
     StageTimer tq(L, 8, s);
     launch_tc_quant_x(q, s);
+    CUDA_TRY(cudaGetLastError());
+    tq.launched(1);
+    tq.end();
+  }
+  if (dq && c.fmt == MOE_FMT_NVFP4) {
+    // NVFP4 on the tensor core multiplies gate/up in f16: x rows as f16 with a
+    // power-of-two scale per token
+    StageTimer tq(L, 8, s);
+    launch_x_rows_f16(reinterpret_cast<const uint16_t *>(x), T, H, L->xf16, L->xs, s);
     CUDA_TRY(cudaGetLastError());
     tq.launched(1);
     tq.end();

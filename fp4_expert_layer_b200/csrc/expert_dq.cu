@@ -110,12 +110,13 @@ struct DqGeom {
   static_assert(SMEM <= 227 * 1024, "shared-memory budget");
 };
 
-// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, K-major.
-__device__ __forceinline__ uint32_t idesc_bf16_dq(int M, int N) {
+// kind::f16 instruction descriptor: fp32 accumulator, A and B both f16 or
+// both bf16, K-major.
+__device__ __forceinline__ uint32_t idesc_16_dq(int M, int N, bool f16) {
   uint32_t d = 0;
-  d |= 1u << 4;    // C: F32
-  d |= 1u << 7;    // A: BF16
-  d |= 1u << 10;   // B: BF16
+  d |= 1u << 4;                     // C: F32
+  d |= (f16 ? 0u : 1u) << 7;        // A: F16 / BF16
+  d |= (f16 ? 0u : 1u) << 10;       // B: F16 / BF16
   d |= (uint32_t)(N >> 3) << 17;
   d |= (uint32_t)(M >> 4) << 24;
   return d;
@@ -165,17 +166,25 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
 }
 
 // Eight E2M1 codes (one 32-bit word, element 2i in the low nibble of byte i)
-// times one E4M3 scale (f16x2 with the scale in both halves) -> eight bf16:
-// the f16 product is exact (at most 6 significant bits, in [2^-10, 2688]) and
-// so is its bf16.
+// times one E4M3 scale (f16x2 with the scale in both halves) -> eight f16, or
+// eight bf16 (F16 = false): the f16 product is exact (at most 6 significant
+// bits, in [2^-10, 2688]) and so is its bf16.
+template <bool F16>
 __device__ __forceinline__ uint4 decode8(uint32_t w, uint32_t sc2) {
   uint32_t f[4];
   e2m1x8_to_f16x2(w, f);
   uint4 o;
-  o.x = f16x2_to_bf16x2(hmul2_u32(f[0], sc2));
-  o.y = f16x2_to_bf16x2(hmul2_u32(f[1], sc2));
-  o.z = f16x2_to_bf16x2(hmul2_u32(f[2], sc2));
-  o.w = f16x2_to_bf16x2(hmul2_u32(f[3], sc2));
+  if constexpr (F16) {
+    o.x = hmul2_u32(f[0], sc2);
+    o.y = hmul2_u32(f[1], sc2);
+    o.z = hmul2_u32(f[2], sc2);
+    o.w = hmul2_u32(f[3], sc2);
+  } else {
+    o.x = f16x2_to_bf16x2(hmul2_u32(f[0], sc2));
+    o.y = f16x2_to_bf16x2(hmul2_u32(f[1], sc2));
+    o.z = f16x2_to_bf16x2(hmul2_u32(f[2], sc2));
+    o.w = f16x2_to_bf16x2(hmul2_u32(f[3], sc2));
+  }
   return o;
 }
 
@@ -220,6 +229,10 @@ __device__ __forceinline__ uint4 decode8_fp8(uint32_t w0, uint32_t w1, float s) 
 template <int MODE, int NB, int F>
 __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_constant__ DqArgs a) {
   using Geo = DqGeom<NB, F>;
+  // NVFP4 gate/up multiplies in f16: the weights need no widening to bf16
+  // (one conversion and one f16 multiply per pair of codes) and x comes as
+  // f16 rows with a power-of-two scale per token (act_scale)
+  constexpr bool kF16 = F == DQ_NV && MODE == MODE_GATEUP;
   constexpr int kRawBytes = Geo::RAW_BYTES;
   constexpr int SO = Geo::OP_STAGES;
   constexpr int SR = Geo::RAW_STAGES;
@@ -374,7 +387,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 54)) break;
         tc_fence_after();
         const uint32_t acc = tmem + (uint32_t)(buf * Geo::ACC_COLS);
-        const uint32_t idesc = idesc_bf16_dq(128, N);
+        const uint32_t idesc = idesc_16_dq(128, N, kF16);
         bool failed = false;
         for (int slab = 0; slab < nslab; ++slab) {
           if (!mbar_wait(smem_u32(&op_full[s]), ph, a.err, 51)) { failed = true; break; }
@@ -486,7 +499,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
             const uint32_t sc[4] = {dup_lo16(s01), dup_hi16(s01), dup_lo16(s23), dup_hi16(s23)};
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const uint4 o = decode8(w[c], sc[c >> 1]);
+              const uint4 o = decode8<kF16>(w[c], sc[c >> 1]);
               v[4 * c + 0] = o.x; v[4 * c + 1] = o.y; v[4 * c + 2] = o.z; v[4 * c + 3] = o.w;
             }
           } else {
@@ -600,14 +613,19 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       // NVFP4: the per-tensor fp32 scales of gate, up and down; other formats carry none
       const float one3[3] = {1.0f, 1.0f, 1.0f};
       const float *gsc = F == DQ_NV ? reinterpret_cast<const float *>(blob + a.L.glob) : one3;
+      // down: each token's pair and gate; f16 gate/up: each token's x scale
       int my_pair = 0;
       float my_gate = 0.0f;
       if (MODE == MODE_DOWN && et < ntok) {
         my_pair = checked_index(__ldg(a.prow_pair + ti.prow0 + et), 0, a.db.n_pairs, 0, a.db.err, kChkPair);
         my_gate = __ldg(a.gates + my_pair);
       }
+      if (kF16 && et < ntok) {
+        const int tok = checked_index(__ldg(a.prow_token + ti.prow0 + et), 0, a.db.n_tokens, 0, a.db.err, kChkToken);
+        my_gate = __ldg(a.act_scale + tok);
+      }
       ok = mbar_wait(smem_u32(&accf_bar[buf]), (n / NBUF) & 1, a.err, 57);
-      if (MODE == MODE_DOWN && et < ntok) {
+      if ((MODE == MODE_DOWN || kF16) && et < ntok) {
         tok_pair[et] = my_pair;
         tok_gate[et] = my_gate;
       }
@@ -628,8 +646,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
           for (int jj = 0; jj < 32; ++jj) {
             const int j = c0 + jj;
             if (j >= ntok) continue;                         // warp-uniform
-            const float av = __uint_as_float(g[jj]) * gg;
-            const float uv = __uint_as_float(u[jj]) * gu;
+            const float ts = kF16 ? tok_gate[j] : 1.0f;   // f16 x rows: their power-of-two scale
+            const float av = __uint_as_float(g[jj]) * (gg * ts);
+            const float uv = __uint_as_float(u[jj]) * (gu * ts);
             a.h_out[(size_t)(ti.prow0 + j) * I + rcol] = bf16_bits(silu_f(av) * uv);
           }
         }
@@ -666,6 +685,49 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem, Geo::TMEM_COLS);
   }
+}
+
+// x rows (bf16) -> f16 rows, each multiplied by a power of two 2^p that puts
+// its largest magnitude in [2^14, 2^15): every element within 2^31 of the
+// row's maximum converts exactly (f16 keeps 11 significant bits, bf16 has 8;
+// smaller ones land on the f16 subnormal grid, off by less than 2^-25 of the
+// row maximum).  xs[row] = 2^-p, applied to the row's accumulators.  One warp
+// per row, 16-byte loads and stores (H a multiple of 256, rows 16-byte aligned).
+__global__ void __launch_bounds__(256) x_rows_f16_kernel(const uint16_t *x, int T, int H, uint16_t *xh, float *xs) {
+  wait_prior_grid();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= T) return;
+  const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)row * H);
+  uint4 *dst = reinterpret_cast<uint4 *>(xh + (size_t)row * H);
+  const int n8 = H / 8;
+  uint32_t am = 0;                                    // largest |bf16| bit pattern (orders like the magnitude)
+  for (int i = lane; i < n8; i += 32) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) am = max(am, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+  }
+  am = __reduce_max_sync(0xffffffffu, am);
+  const int e = am >= 0x80u ? (int)(am >> 7) - 127 : -127;   // floor(log2 max), bf16 exponent field
+  const int p = min(127, max(-126, 14 - e));
+  const float sc = __int_as_float((p + 127) << 23);
+  for (int i = lane; i < n8; i += 32) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = __uint_as_float(w[k] << 16) * sc, hi = __uint_as_float(w[k] & 0xFFFF0000u) * sc;
+      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(o[k]) : "f"(hi), "f"(lo));
+    }
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (lane == 0) xs[row] = __int_as_float((127 - p) << 23);
+}
+
+void launch_x_rows_f16(const uint16_t *x, int T, int H, uint16_t *xh, float *xs, cudaStream_t s) {
+  if (T <= 0) return;
+  launch_dependent(x_rows_f16_kernel, (T + 7) / 8, 256, 0, s, x, T, H, xh, xs);
 }
 
 template <int MODE, int NB, int F>

@@ -394,7 +394,8 @@ struct DqArgs {
   const int *prow_token;     // gate/up: padded row -> token
   const int *prow_pair;      // down: padded row -> pair
   const float *gates;
-  const uint16_t *act;       // gate/up: x bf16 [T, H]; down: h bf16 [padded rows, I]
+  const uint16_t *act;       // gate/up: x bf16 [T, H] (NVFP4: f16 rows, see act_scale); down: h bf16 [padded rows, I]
+  const float *act_scale;    // gate/up of NVFP4 layers: per-token scale of the f16 x rows (x = row * scale)
   uint16_t *h_out;           // gate/up: h bf16 [padded rows, I]
   float *o_out;              // down: O' [pairs, H]
   int *work_ctr;             // item counter of this pass, zero at launch
@@ -404,5 +405,8 @@ struct DqArgs {
 };
 // nb: tokens per tile (64 or 128)
 void launch_expert_dq(int mode, int nb, const DqArgs &a, cudaStream_t s);
+// x rows (bf16) -> f16 rows with a power-of-two scale per row (xs = the
+// inverse), the gate/up activations of NVFP4 layers on the tensor core
+void launch_x_rows_f16(const uint16_t *x, int T, int H, uint16_t *xh, float *xs, cudaStream_t s);
 
 }  // namespace moe
