@@ -37,10 +37,11 @@
 //                (gate and up, or the two 128-row halves of down) per item;
 //   warps 2..5   epilogue: TMEM -> SwiGLU -> h (bf16, padded-row order), or
 //                G_d * gate * acc -> O' (fp32, pair order);
-//   warps 6..13  decoders: raw stage -> bf16 weight rows in TMEM, warp w the
-//                rows of TMEM lane quadrant w % 4 of the first (w < 10) or
-//                second 128 rows (NVFP4: hardware E2M1 -> f16x2, an f16
-//                multiply by the scale, widening to bf16);
+//   warps 6..13  decoders: raw stage -> weight rows in TMEM, in two groups
+//                of four warps taking alternate slabs (warp w the rows of TMEM
+//                lane quadrant w % 4 of both 128-row halves; NVFP4: hardware
+//                E2M1 -> f16x2 and an f16 multiply by the scale, widened to
+//                bf16 for the down pass);
 //   warps 14..15 activation loaders: the tile's bf16 rows of this K slab by
 //                16-byte cp.async (x rows gathered through the padded-row ->
 //                token map for gate/up; h rows for down), 128-byte swizzled
@@ -264,10 +265,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int s = 0; s < SR; ++s) {
       mbar_init(smem_u32(&raw_full[s]), 1);
-      mbar_init(smem_u32(&raw_empty[s]), kDqDecoders / 32);
+      mbar_init(smem_u32(&raw_empty[s]), kDqDecoders / 64);     // one slab group
     }
     for (int s = 0; s < SO; ++s) {
-      mbar_init(smem_u32(&op_full[s]), kDqLoaders + kDqDecoders / 32);
+      mbar_init(smem_u32(&op_full[s]), kDqLoaders + kDqDecoders / 64);
       mbar_init(smem_u32(&op_empty[s]), 1);
     }
     for (int b = 0; b < NBUF; ++b) {
@@ -416,11 +417,14 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       mbar_drain(smem_u32(&quiesce_bar), 0);
     }
   } else if (warp >= 6 && warp < 14) {
-    // ---------------- decoders: raw codes + scales -> bf16 weight rows in TMEM
+    // ---------------- decoders: raw codes + scales -> weight rows in TMEM.
+    // Two groups of four warps take alternate slabs (group g the slabs n of
+    // the CTA's sequence with n % 2 == g), so that one group's TMEM stores
+    // drain while the other decodes; a thread decodes rows rr and 128 + rr.
     const int quad = warp & 3;                               // TMEM lane quadrant of this warp
-    const int hh = warp >= 10 ? 1 : 0;                       // first or second 128 rows of the 256
-    const int rr = 32 * quad + lane;                         // row within the 128-row half
-    const int row = 128 * hh + rr;                           // row of the 256 in the raw stage
+    const int grp = warp >= 10 ? 1 : 0;
+    const int rr = 32 * quad + lane;                         // row within each 128-row half
+    const uint32_t tlane = (uint32_t)(32 * quad) << 16;
     int r = 0, s = 0, n_slabs = 0;
     uint32_t rph = 0, sph = 0;
     int q = 0;
@@ -439,13 +443,19 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       if (++q == kDqSched) { q = 0; qph ^= 1u; }
       if (item < 0) break;
       if (loc == kLocAbsent) continue;
+      // FP8: base of each half's fp32 block scales (one per 128 K) in the blob
+      const float *bsp[2] = {nullptr, nullptr};
       if constexpr (F == DQ_F8) {
-        // base of this row's fp32 block scales (one per 128 K) in the blob
-        const int m = MODE == MODE_GATEUP ? hh : 2;
-        const int rbk = MODE == MODE_GATEUP ? item % ipt : 2 * (item % ipt) + hh;
         const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
-        const float *bsp = reinterpret_cast<const float *>(blob + a.L.scales[m]) + (size_t)rbk * (K / 128);
-        for (int slab = 0; slab < nslab; ++slab) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int m = MODE == MODE_GATEUP ? hh : 2;
+          const int rbk = MODE == MODE_GATEUP ? item % ipt : 2 * (item % ipt) + hh;
+          bsp[hh] = reinterpret_cast<const float *>(blob + a.L.scales[m]) + (size_t)rbk * (K / 128);
+        }
+      }
+      for (int slab = 0; slab < nslab; ++slab) {
+        if ((n_slabs & 1) == grp) {
           int ok = 1;
           if (lane == 0) {
             ok = mbar_wait(smem_u32(&raw_full[r]), rph, a.err, 53) ? 1 : 0;
@@ -455,16 +465,46 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
           if (!ok) { failed = true; break; }
           tc_fence_after();
           const uint8_t *raw = smem + Geo::RAW_OFF + (size_t)r * kRawBytes;
-          const float sblk = __ldg(bsp + slab / 2);
-          uint32_t v[32];
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const uint4 cv = *reinterpret_cast<const uint4 *>(raw + row * 64 + c4 * 16);
-            const uint4 o0 = decode8_fp8(cv.x, cv.y, sblk), o1 = decode8_fp8(cv.z, cv.w, sblk);
-            v[8 * c4 + 0] = o0.x; v[8 * c4 + 1] = o0.y; v[8 * c4 + 2] = o0.z; v[8 * c4 + 3] = o0.w;
-            v[8 * c4 + 4] = o1.x; v[8 * c4 + 5] = o1.y; v[8 * c4 + 6] = o1.z; v[8 * c4 + 7] = o1.w;
+          for (int hh = 0; hh < 2; ++hh) {
+            const int row = 128 * hh + rr;                   // row of the 256 in the raw stage
+            uint32_t v[32];
+            if constexpr (F == DQ_F8) {
+              const float sblk = __ldg(bsp[hh] + slab / 2);
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4) {
+                const uint4 cv = *reinterpret_cast<const uint4 *>(raw + row * 64 + c4 * 16);
+                const uint4 o0 = decode8_fp8(cv.x, cv.y, sblk), o1 = decode8_fp8(cv.z, cv.w, sblk);
+                v[8 * c4 + 0] = o0.x; v[8 * c4 + 1] = o0.y; v[8 * c4 + 2] = o0.z; v[8 * c4 + 3] = o0.w;
+                v[8 * c4 + 4] = o1.x; v[8 * c4 + 5] = o1.y; v[8 * c4 + 6] = o1.z; v[8 * c4 + 7] = o1.w;
+              }
+            } else {
+              const uint4 c0 = *reinterpret_cast<const uint4 *>(raw + row * 32);
+              const uint4 c1 = *reinterpret_cast<const uint4 *>(raw + row * 32 + 16);
+              const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+              if constexpr (F == DQ_NV) {
+                const uint32_t sf4 =
+                    *reinterpret_cast<const uint32_t *>(raw + 8192 + hh * 512 + 16 * (rr & 31) + 4 * (rr >> 5));
+                const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(sf4 & 0xFFFFu));
+                const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(sf4 >> 16));
+                const uint32_t sc[4] = {dup_lo16(s01), dup_hi16(s01), dup_lo16(s23), dup_hi16(s23)};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const uint4 o = decode8<kF16>(w[c], sc[c >> 1]);
+                  v[4 * c + 0] = o.x; v[4 * c + 1] = o.y; v[4 * c + 2] = o.z; v[4 * c + 3] = o.w;
+                }
+              } else {
+                const uint32_t sb = *reinterpret_cast<const uint16_t *>(raw + 8192 + hh * 256 + rr * 2);
+                const uint32_t sc2 = sb | (sb << 16);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const uint4 o = decode8_int4(w[c], sc2);
+                  v[4 * c + 0] = o.x; v[4 * c + 1] = o.y; v[4 * c + 2] = o.z; v[4 * c + 3] = o.w;
+                }
+              }
+            }
+            tmem_st32(tmem + tlane + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS + 32 * hh), v);
           }
-          tmem_st32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS + 32 * hh), v);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
@@ -472,57 +512,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
             mbar_arrive(smem_u32(&raw_empty[r]));
             mbar_arrive(smem_u32(&op_full[s]));
           }
-          ++n_slabs;
-          if (++r == SR) { r = 0; rph ^= 1u; }
-          if (++s == SO) { s = 0; sph ^= 1u; }
         }
-      } else {
-        for (int slab = 0; slab < nslab; ++slab) {
-          int ok = 1;
-          if (lane == 0) {
-            ok = mbar_wait(smem_u32(&raw_full[r]), rph, a.err, 53) ? 1 : 0;
-            if (ok && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 55) ? 1 : 0;
-          }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) { failed = true; break; }
-          tc_fence_after();
-          const uint8_t *raw = smem + Geo::RAW_OFF + (size_t)r * kRawBytes;
-          const uint4 c0 = *reinterpret_cast<const uint4 *>(raw + row * 32);
-          const uint4 c1 = *reinterpret_cast<const uint4 *>(raw + row * 32 + 16);
-          const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          uint32_t v[32];
-          if constexpr (F == DQ_NV) {
-            const uint32_t sf4 =
-                *reinterpret_cast<const uint32_t *>(raw + 8192 + hh * 512 + 16 * (rr & 31) + 4 * (rr >> 5));
-            const uint32_t s01 = e4m3x2_to_f16x2((uint16_t)(sf4 & 0xFFFFu));
-            const uint32_t s23 = e4m3x2_to_f16x2((uint16_t)(sf4 >> 16));
-            const uint32_t sc[4] = {dup_lo16(s01), dup_hi16(s01), dup_lo16(s23), dup_hi16(s23)};
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint4 o = decode8<kF16>(w[c], sc[c >> 1]);
-              v[4 * c + 0] = o.x; v[4 * c + 1] = o.y; v[4 * c + 2] = o.z; v[4 * c + 3] = o.w;
-            }
-          } else {
-            const uint32_t sb = *reinterpret_cast<const uint16_t *>(raw + 8192 + hh * 256 + rr * 2);
-            const uint32_t sc2 = sb | (sb << 16);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint4 o = decode8_int4(w[c], sc2);
-              v[4 * c + 0] = o.x; v[4 * c + 1] = o.y; v[4 * c + 2] = o.z; v[4 * c + 3] = o.w;
-            }
-          }
-          tmem_st32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS + 32 * hh), v);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(smem_u32(&raw_empty[r]));
-            mbar_arrive(smem_u32(&op_full[s]));
-          }
-          ++n_slabs;
-          if (++r == SR) { r = 0; rph ^= 1u; }
-          if (++s == SO) { s = 0; sph ^= 1u; }
-        }
+        ++n_slabs;
+        if (++r == SR) { r = 0; rph ^= 1u; }
+        if (++s == SO) { s = 0; sph ^= 1u; }
       }
     }
   } else if (warp >= 14) {
