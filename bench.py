@@ -372,7 +372,7 @@ def gateup_roofline(wl, T, n_active, prof, hbm_peak, bf16_sus, numerics, peak_sr
         ach = flops / (g_ms / 1e3) / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": bf16_sus, "unit": "TFLOP/s", "frac": ach / bf16_sus,
                 "traffic": traffic,
-                "kernel": "expert_dq_kernel gate/up+SwiGLU (tcgen05 kind::f16, NVFP4 decoded to bf16 in shared memory)",
+                "kernel": "expert_dq_kernel gate/up+SwiGLU (tcgen05 kind::f16, NVFP4 decoded to f16 into TMEM as the A operand)",
                 "peak_source": f"{peak_src} bf16_tflops_sustained (the MMA kind this path runs)",
                 "algorithmic_flops_per_step": flops, "kernel_ms_per_step": g_ms, "launches_per_step": launches,
                 "hbm_gbs_of_same_pass": gateup_bytes(wl, n_active, T) / (g_ms / 1e3) / 1e9}
@@ -405,10 +405,17 @@ def short_leg(torch, F, dev, flush, stream, name, T, numerics, K, W, peaks_t, sl
         n_active = int((r["counts"] > 0).sum().item())
         ms = time_steps(torch, layer, x, y, T, K, W, flush, stream) / K
         prof = stage_profile(torch, layer, x, y, T, min(K, 50), flush, stream)
+        # DRAM bytes per gate/up launch from a committed ncu summary of the same
+        # kernel source on the same workload (all resident: one launch per step)
+        csrc = os.path.join(ROOT, "fp4_expert_layer_b200", "csrc")
         traffic = None
-        if name == "olmoe_like" and T == 32:
-            traffic = traffic_record("expert_tc_gateup_olmoe_like_T32.md",
-                                     os.path.join(ROOT, "fp4_expert_layer_b200", "csrc", "expert_tc.cu"))
+        if slots == "all" and numerics == "exact" and name == "olmoe_like" and T == 32:
+            traffic = traffic_record("expert_tc_gateup_olmoe_like_T32.md", os.path.join(csrc, "expert_tc.cu"))
+        elif slots == "all" and numerics == "exact" and name == "qwen3_8_flash_next_like" and T == 8192:
+            traffic = traffic_record("expert_dq_gateup_qwen3_8_flash_next_like_T8192.md",
+                                     os.path.join(csrc, "expert_dq.cu"))
+        elif slots == "all" and numerics == "a4" and name == "fp4_peak_probe" and T == 8192:
+            traffic = traffic_record("gemm_a4_gateup_fp4_peak_probe_T8192.md", os.path.join(csrc, "gemm_a4.cu"))
         roof = gateup_roofline(wl, T, n_active, prof, hbm_peak, bf16_sus, numerics, src, traffic)
         return {"workload": name, "tokens": T, "numerics": numerics, "resident_slots": S,
                 "value": T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": K,
