@@ -1396,12 +1396,12 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     if (T <= 128) {
       const int np = dense_splitk_rows(T);
       ST_TRY(make_bf16_map(&d.xmap, xs, H, T, np));
-      launch_dense_splitk(MODE_GATEUP, d, dense_splitk_ways(d.n_rowblocks, H, L->n_sms), s);
+      launch_dense_splitk(MODE_GATEUP, d, s);
       CUDA_TRY(cudaGetLastError());
       d.wmap[0] = L->sh_map[2];
       ST_TRY(make_bf16_map(&d.xmap, L->sh_h, Is, T, np));
       d.K = Is; d.rows = H; d.n_rowblocks = H / 256;
-      launch_dense_splitk(MODE_DOWN, d, dense_splitk_ways(d.n_rowblocks, Is, L->n_sms), s);
+      launch_dense_splitk(MODE_DOWN, d, s);
       CUDA_TRY(cudaGetLastError());
     } else {
       ST_TRY(make_bf16_map(&d.xmap, xs, H, T));

@@ -281,7 +281,8 @@ struct SplitGeom {
   static constexpr int STAGE = (A_BYTES + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int COLS = 2 * NP;
   static constexpr int TMEM_COLS = COLS <= 32 ? 32 : (COLS <= 64 ? 64 : (COLS <= 128 ? 128 : 256));
-  static constexpr int RED_BYTES = 2 * 128 * NP * 4;   // received partial accumulators, fp32
+  // received partial accumulators, fp32: S slots x 2 halves x ceil(128 / S) rows, at most S = 7
+  static constexpr int RED_BYTES = 7 * 2 * 19 * NP * 4;
   static constexpr size_t SMEM = (size_t)(STAGES * STAGE > RED_BYTES ? STAGES * STAGE : RED_BYTES) + 1024;
   static_assert(SMEM <= 227 * 1024, "shared-memory budget");
 };
@@ -399,14 +400,17 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
   }
   tc_fence_before();
   cluster.sync();                                      // every rank is done with its stage memory
-  const int rows = 128 / S, r0 = ks * rows;
+  // rank q finishes rows [q * 128 / S, (q + 1) * 128 / S) of both halves
+  const int rmax = (128 + S - 1) / S;                  // rows of the largest range (receive slot size)
+  const int r0 = ks * 128 / S, r1 = (ks + 1) * 128 / S;
   if (warp >= 2) {
     // push this rank's partials (rows 32*quad + lane) into the receive slot
     // [ks] of the rank that finishes them
     tc_fence_after();
     const int quad = warp & 3;
     const int row = 32 * quad + lane;
-    const int owner = row / rows, rl = row % rows;
+    const int owner = ((row + 1) * S + 127) / 128 - 1;   // the q whose range holds row
+    const int rl = row - owner * 128 / S;
     float *dst = cluster.map_shared_rank(recv, owner);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -415,7 +419,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
         uint32_t v[16];
         tmem_ld16(tmem + (uint32_t)(h * NP + c0) + ((uint32_t)(32 * quad) << 16), v);
         tmem_ld_wait();
-        float4 *d4 = reinterpret_cast<float4 *>(dst + (((size_t)ks * 2 + h) * rows + rl) * NP + c0);
+        float4 *d4 = reinterpret_cast<float4 *>(dst + (((size_t)ks * 2 + h) * rmax + rl) * NP + c0);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           d4[j] = ok ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
@@ -427,13 +431,13 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
   cluster.sync();                                      // every partial is in its owner's shared memory
   // this rank finishes rows [ks * 128 / S, (ks + 1) * 128 / S) of both halves,
   // summing the slots in rank order (local shared memory only)
-  for (int i = threadIdx.x; i < rows * NP; i += blockDim.x) {
+  for (int i = threadIdx.x; i < (r1 - r0) * NP; i += blockDim.x) {
     const int rl = i / NP, c = i % NP;
     const int r = r0 + rl;
     float v0 = 0.0f, v1 = 0.0f;
     for (int q = 0; q < S; ++q) {
-      v0 += recv[(((size_t)q * 2 + 0) * rows + rl) * NP + c];
-      v1 += recv[(((size_t)q * 2 + 1) * rows + rl) * NP + c];
+      v0 += recv[(((size_t)q * 2 + 0) * rmax + rl) * NP + c];
+      v1 += recv[(((size_t)q * 2 + 1) * rmax + rl) * NP + c];
     }
     if (c >= a.T) continue;
     if constexpr (MODE == MODE_GATEUP) {
@@ -451,10 +455,50 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
   }
 }
 
+// Clusters of S CTAs of this kernel that the device runs at once (0 if the
+// query fails); cached per kernel and S.
 template <int MODE, int NP>
-static void launch_splitk_one(const DenseTcArgs &a, int S, cudaStream_t s) {
+static int splitk_max_clusters(int S) {
+  static int cache[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};   // by S = 1..8
+  if (cache[S] >= 0) return cache[S];
   using Geo = SplitGeom<NP>;
   auto fn = dense_splitk_kernel<MODE, NP>;
+  cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::SMEM);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)S);
+  cfg.blockDim = dim3(kDenseThreads);
+  cfg.dynamicSmemBytes = Geo::SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cache[S] = n;
+  return n;
+}
+
+// Cluster size for n_rowblocks row blocks: the largest S in 8..2 that leaves
+// each CTA at least 4 K slabs and lets all n_rowblocks clusters run at once
+// (a cluster left for a second round would double the pass), else 1.
+template <int MODE, int NP>
+static int splitk_ways(int n_rowblocks, int K) {
+  for (int S = 8; S > 1; --S)
+    if ((K / 64) >= 4 * S && splitk_max_clusters<MODE, NP>(S) >= n_rowblocks) return S;
+  return 1;
+}
+
+template <int MODE, int NP>
+static void launch_splitk_one(const DenseTcArgs &a, cudaStream_t s) {
+  using Geo = SplitGeom<NP>;
+  auto fn = dense_splitk_kernel<MODE, NP>;
+  const int S = splitk_ways<MODE, NP>(a.n_rowblocks, a.K);
   cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Geo::SMEM);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.n_rowblocks * S));
@@ -473,17 +517,11 @@ static void launch_splitk_one(const DenseTcArgs &a, int S, cudaStream_t s) {
   cudaLaunchKernelEx(&cfg, fn, a);
 }
 
-int dense_splitk_ways(int n_rowblocks, int K, int n_sms) {
-  int S = 1;
-  while (S < 8 && n_rowblocks * S * 2 <= n_sms && (K / 64) >= S * 2 * 2) S *= 2;
-  return S;
-}
-
-void launch_dense_splitk(int mode, const DenseTcArgs &a, int S, cudaStream_t s) {
+void launch_dense_splitk(int mode, const DenseTcArgs &a, cudaStream_t s) {
   const int np = dense_splitk_rows(a.T);
 #define MOE_SPLITK(NP)                                              \
-  if (mode == MODE_GATEUP) launch_splitk_one<MODE_GATEUP, NP>(a, S, s); \
-  else launch_splitk_one<MODE_DOWN, NP>(a, S, s);
+  if (mode == MODE_GATEUP) launch_splitk_one<MODE_GATEUP, NP>(a, s); \
+  else launch_splitk_one<MODE_DOWN, NP>(a, s);
   if (np == 16) { MOE_SPLITK(16) }
   else if (np == 32) { MOE_SPLITK(32) }
   else if (np == 64) { MOE_SPLITK(64) }

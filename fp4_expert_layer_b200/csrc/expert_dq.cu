@@ -90,21 +90,21 @@ struct DqRaw<DQ_F8> {
 
 template <int NB, int F>
 struct DqGeom {
-  static constexpr int B_BYTES = NB * 128;                 // NB token rows x 64 16-bit values
-  static constexpr int B_STAGES = NB >= 128 ? 6 : 8;       // activation ring (shared memory)
-  static constexpr int OP_STAGES = 4;                      // decoded-weight ring (TMEM A stages)
+  static constexpr int B_BYTES = NB * 128;                 // NB token rows x 64 bf16
+  static constexpr int OP_STAGE = B_BYTES;                 // multiple of 1024
+  static constexpr int OP_STAGES = 4;
   static constexpr int A_COLS = 64;                        // TMEM columns of one stage's A (2 halves x 32)
   static constexpr int ACC_COLS = 2 * NB;                  // gate + up (or the two down halves)
   static constexpr int NBUF = (512 - OP_STAGES * A_COLS) / ACC_COLS >= 2 ? 2 : 1;
   static constexpr int A_TMEM = NBUF * ACC_COLS;           // first A column
   static constexpr int TMEM_COLS = 512;
-  static constexpr int RAW_OFF = B_STAGES * B_BYTES;
+  static constexpr int RAW_OFF = OP_STAGES * OP_STAGE;
   static constexpr int RAW_BYTES = DqRaw<F>::BYTES;
   // raw stages in what is left of 227 KB (1 KB alignment slack, 4 KB for the static part)
   static constexpr int RAW_FIT = (227 * 1024 - 1024 - 4096 - RAW_OFF) / RAW_BYTES;
   static constexpr int RAW_STAGES = RAW_FIT < 12 ? RAW_FIT : 12;
   static constexpr size_t SMEM = (size_t)RAW_OFF + (size_t)RAW_STAGES * RAW_BYTES + 1024;
-  static_assert(B_BYTES % 1024 == 0, "activation stages must keep the 1024-byte swizzle alignment");
+  static_assert(OP_STAGE % 1024 == 0, "operand stages must keep the 1024-byte swizzle alignment");
   static_assert(RAW_BYTES % 512 == 0, "raw stages keep 128-byte TMA destinations");
   static_assert(RAW_STAGES >= 3, "raw ring depth");
   static_assert(A_TMEM + OP_STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
@@ -236,16 +236,13 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
   constexpr bool kF16 = F == DQ_NV && MODE == MODE_GATEUP;
   constexpr int kRawBytes = Geo::RAW_BYTES;
   constexpr int SO = Geo::OP_STAGES;
-  constexpr int SB = Geo::B_STAGES;
   constexpr int SR = Geo::RAW_STAGES;
   constexpr int NBUF = Geo::NBUF;
   extern __shared__ __align__(1024) uint8_t dq_smem_raw[];
   __shared__ __align__(8) uint64_t raw_full[SR];    // packed codes + scales landed (TMA / bulk)
   __shared__ __align__(8) uint64_t raw_empty[SR];   // decoders done with a raw stage
-  __shared__ __align__(8) uint64_t op_full[SO];     // weights of a slab decoded into a TMEM A stage
-  __shared__ __align__(8) uint64_t op_empty[SO];    // MMAs done with a TMEM A stage
-  __shared__ __align__(8) uint64_t b_full[SB];      // activation rows of a slab landed
-  __shared__ __align__(8) uint64_t b_empty[SB];     // MMAs done with an activation stage
+  __shared__ __align__(8) uint64_t op_full[SO];     // bf16 weights decoded + activation rows landed
+  __shared__ __align__(8) uint64_t op_empty[SO];    // MMAs done with an operand stage
   __shared__ __align__(8) uint64_t accf_bar[NBUF];
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
   __shared__ __align__(8) uint64_t quiesce_bar;     // all MMAs of the CTA done (before TMEM is freed)
@@ -271,12 +268,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       mbar_init(smem_u32(&raw_empty[s]), kDqDecoders / 64);     // one slab group
     }
     for (int s = 0; s < SO; ++s) {
-      mbar_init(smem_u32(&op_full[s]), kDqDecoders / 64);
+      mbar_init(smem_u32(&op_full[s]), kDqLoaders + kDqDecoders / 64);
       mbar_init(smem_u32(&op_empty[s]), 1);
-    }
-    for (int s = 0; s < SB; ++s) {
-      mbar_init(smem_u32(&b_full[s]), kDqLoaders);
-      mbar_init(smem_u32(&b_empty[s]), 1);
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(smem_u32(&accf_bar[b]), 1);
@@ -377,8 +370,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
   } else if (warp == 1) {
     // ---------------- MMA issuer (one lane)
     if (lane == 0) {
-      int s = 0, n = 0, sb = 0;
-      uint32_t ph = 0, bph = 0;
+      int s = 0, n = 0;
+      uint32_t ph = 0;
       int q = 0;
       uint32_t qph = 0;
       while (true) {
@@ -398,13 +391,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         const uint32_t idesc = idesc_16_dq(128, N, kF16);
         bool failed = false;
         for (int slab = 0; slab < nslab; ++slab) {
-          if (!mbar_wait(smem_u32(&op_full[s]), ph, a.err, 51) || !mbar_wait(smem_u32(&b_full[sb]), bph, a.err, 50)) {
-            failed = true;
-            break;
-          }
+          if (!mbar_wait(smem_u32(&op_full[s]), ph, a.err, 51)) { failed = true; break; }
           fence_proxy_async_dq();
           tc_fence_after();
-          const uint32_t st = smem_u32(smem + (size_t)sb * Geo::B_BYTES);
+          const uint32_t st = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
           const uint32_t at = tmem + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {                   // K = 16 per MMA (8 TMEM columns of A)
@@ -414,10 +404,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
               umma_bf16_ts(acc + (uint32_t)(h * NB), at + (uint32_t)(h * 32 + 8 * kk), bdesc, idesc,
                            (slab > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(smem_u32(&op_empty[s]));                 // stages free once these MMAs finish
-          tc_commit(smem_u32(&b_empty[sb]));
+          tc_commit(smem_u32(&op_empty[s]));                 // stage free once these MMAs finish
           if (++s == SO) { s = 0; ph ^= 1u; }
-          if (++sb == SB) { sb = 0; bph ^= 1u; }
         }
         if (failed) break;
         tc_commit(smem_u32(&accf_bar[buf]));
@@ -574,19 +562,19 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       }
       for (int slab = 0; slab < nslab; ++slab) {
         int ok = 1;
-        if (lane == 0 && n_slabs >= SB) ok = mbar_wait(smem_u32(&b_empty[s]), sph ^ 1u, a.err, 56) ? 1 : 0;
+        if (lane == 0 && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 56) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { failed = true; break; }
-        const uint32_t bst = smem_u32(smem + (size_t)s * Geo::B_BYTES);
+        const uint32_t bst = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
 #pragma unroll
         for (int i = 0; i < RPT; ++i) {
           const int j = (lt >> 3) + (kDqLoaders / 8) * i;
           if (roff[i] != 0xFFFFFFFFu)
             cp_async16_dq(bst + j * 128 + ((cq ^ (j & 7)) << 4), a.act + roff[i] + slab * 64 + cq * 8);
         }
-        cp_async_arrive_dq(smem_u32(&b_full[s]));
+        cp_async_arrive_dq(smem_u32(&op_full[s]));
         ++n_slabs;
-        if (++s == SB) { s = 0; sph ^= 1u; }
+        if (++s == SO) { s = 0; sph ^= 1u; }
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");

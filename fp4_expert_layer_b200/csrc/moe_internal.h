@@ -321,8 +321,10 @@ struct DenseTcArgs {
 void launch_dense_tc(int mode, const DenseTcArgs &a, cudaStream_t s);
 // Decode-sized batches (T <= 128): K split over a cluster of S CTAs per row
 // block (xmap's box is 64 x NP rows, NP = T rounded up to 16, 32, 64 or 128).
-int dense_splitk_ways(int n_rowblocks, int K, int n_sms);
-void launch_dense_splitk(int mode, const DenseTcArgs &a, int S, cudaStream_t s);
+// The cluster size S is chosen per launch: the largest (8, 4, 2) that keeps
+// at least 4 K slabs per CTA and fits every row block's cluster on the device
+// at once (cudaOccupancyMaxActiveClusters), else 1.
+void launch_dense_splitk(int mode, const DenseTcArgs &a, cudaStream_t s);
 inline int dense_splitk_rows(int T) { return T <= 16 ? 16 : (T <= 32 ? 32 : (T <= 64 ? 64 : 128)); }
 
 struct TcArgs {
