@@ -21,6 +21,7 @@
 #include <vector>
 
 #include "moe_internal.h"
+#include "tma.cuh"
 
 using namespace moe;
 
@@ -100,7 +101,8 @@ struct moe_layer {
   uint8_t *slots = nullptr, *staging = nullptr;
   int *loc_resident = nullptr, *loc_pass = nullptr;
   CodeMaps maps{};
-  int *h_err = nullptr, *d_err = nullptr;   // mapped pinned error word (bounded device waits)
+  int *h_err = nullptr;                      // mapped pinned error word, read by the host
+  int *d_err = nullptr;                      // device error word (ErrWord) the kernels poll and write
   float *logits = nullptr, *gates = nullptr;
   int *ids = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr;
   TileInfo *tiles = nullptr;
@@ -536,6 +538,21 @@ static moe_status_t push_table(moe_layer *L, cudaStream_t s) {
   return MOE_OK;
 }
 
+// An earlier forward's kernels recorded an error: report it and clear both
+// words (the device word on the caller's stream, finished before returning,
+// so that the next forward starts clean on any stream).
+static moe_status_t report_device_error(moe_layer *L, void *stream) {
+  char buf[128];
+  snprintf(buf, sizeof buf, "a device-side wait or check of an earlier forward gave up (code %d); outputs of that "
+           "forward are invalid", *(volatile int *)L->h_err);
+  *(volatile int *)L->h_err = 0;
+  cudaSetDevice(L->cfg.device);
+  if (cudaMemsetAsync(L->d_err, 0, sizeof(int), (cudaStream_t)stream) != cudaSuccess ||
+      cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+    (void)cudaGetLastError();
+  return fail(MOE_ERR_CUDA, buf);
+}
+
 // ------------------------------------------------------------------ C ABI
 extern "C" {
 
@@ -888,7 +905,13 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   C_CUDA(cudaMemsetAsync(L->loc_resident, 0xFF, sizeof(int) * E, s));   // -1: absent
   C_CUDA(cudaMemsetAsync(L->loc_pass, 0xFF, sizeof(int) * E, s));
   *L->h_err = 0;
-  C_CUDA(cudaHostGetDevicePointer((void **)&L->d_err, L->h_err, 0));
+  {
+    ErrWord ew{};
+    C_CUDA(cudaHostGetDevicePointer((void **)&ew.host, L->h_err, 0));
+    C_TRY(dalloc(L, &L->d_err, sizeof(ErrWord)));
+    C_CUDA(cudaMemcpyAsync(L->d_err, &ew, sizeof ew, cudaMemcpyHostToDevice, s));
+    C_CUDA(cudaStreamSynchronize(s));                  // ew lives on this stack frame
+  }
   for (int m = 0; m < 3; ++m) {
     const int box_rows = m < 2 ? 128 : 256;
     if (cfg->n_slots) C_TRY(make_code_map(&L->maps.slot[m], L->slots, cfg->n_slots, L->L, m, box_rows));
@@ -1254,19 +1277,14 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   if (T < 0 || T > c.max_tokens) return fail(MOE_ERR_INVALID_ARG, "T out of range [0, max_tokens]");
   if (T == 0) return MOE_OK;
   if (!x || !y) return fail(MOE_ERR_INVALID_ARG, "x or y is NULL");
-  if (*(volatile int *)L->h_err != 0) {
-    char buf[128];
-    snprintf(buf, sizeof buf, "a device-side wait of an earlier forward gave up (code %d); outputs of that "
-             "forward are invalid", *(volatile int *)L->h_err);
-    *(volatile int *)L->h_err = 0;
-    return fail(MOE_ERR_CUDA, buf);
-  }
+  if (*(volatile int *)L->h_err != 0) return report_device_error(L, stream);
   if (L->inject == 3) {
     // test hook: the device error word is set before this forward's kernels
     // run, so that every bounded wait of theirs that has to wait gives up
     // at once (the path a wait takes when its time limit passes)
     L->inject = 0;
     *(volatile int *)L->h_err = 99;
+    CUDA_TRY(cudaMemsetAsync(L->d_err, 0x63, sizeof(int), (cudaStream_t)stream));
   }
   CUDA_TRY(cudaSetDevice(c.device));
   cudaStream_t s = (cudaStream_t)stream;
@@ -1686,13 +1704,7 @@ moe_status_t moe_graph_launch(moe_graph_t G, void *stream) {
   moe_layer *L = G->L;
   if (L->table_version != G->table_version)
     return fail(MOE_ERR_INVALID_ARG, "the slot table changed since the graph was captured");
-  if (*(volatile int *)L->h_err != 0) {
-    char buf[128];
-    snprintf(buf, sizeof buf, "a device-side wait of an earlier forward gave up (code %d); outputs of that "
-             "forward are invalid", *(volatile int *)L->h_err);
-    *(volatile int *)L->h_err = 0;
-    return fail(MOE_ERR_CUDA, buf);
-  }
+  if (*(volatile int *)L->h_err != 0) return report_device_error(L, stream);
   CUDA_TRY(cudaSetDevice(L->cfg.device));
   CUDA_TRY(cudaGraphLaunch(G->exec, (cudaStream_t)stream));
   L->st.forwards += 1;

@@ -12,6 +12,7 @@
 #pragma once
 
 #include "moe_internal.h"
+#include "tma.cuh"
 
 namespace moe {
 
@@ -32,7 +33,7 @@ enum CheckCode {
 // `ok`, recording `code` when it is false (checked build); true otherwise.
 __device__ __forceinline__ bool dcheck(bool ok, int *err, int code) {
   if constexpr (kCheckedBuild) {
-    if (!ok && err) atomicCAS(err, 0, code);
+    if (!ok && err) record_first_error(err, code);
     return ok;
   } else {
     return true;

@@ -10,6 +10,27 @@ namespace moe {
 // to completion, so that no wait can run forever.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+// The error word the kernels share: a device-memory int that the bounded
+// waits poll (a read of mapped host memory would cross PCIe at every check),
+// followed by the address of the mapped host word that the host reads without
+// synchronising.  A failure is recorded in both.
+struct ErrWord {
+  int code;
+  int pad;
+  int *host;
+};
+__device__ __forceinline__ void record_error(int *err, int code) {
+  atomicExch(err, code);
+  int *host = reinterpret_cast<ErrWord *>(err)->host;
+  if (host) atomicExch(host, code);
+}
+// The same, keeping the first code recorded.
+__device__ __forceinline__ void record_first_error(int *err, int code) {
+  if (atomicCAS(err, 0, code) != 0) return;
+  int *host = reinterpret_cast<ErrWord *>(err)->host;
+  if (host) atomicCAS(host, 0, code);
+}
+
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -58,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *er
     if ((i & 255u) == 0) {
       if (err && *(volatile int *)err != 0) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
-        if (err) atomicExch(err, code);
+        if (err) record_error(err, code);
         return false;
       }
     }
@@ -82,7 +103,7 @@ __device__ __forceinline__ bool flag_wait(const int *f, int v, int *err, int cod
     if ((i & 63u) == 0) {
       if (err && *(volatile int *)err != 0) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
-        if (err) atomicExch(err, code);
+        if (err) record_error(err, code);
         return false;
       }
     }
