@@ -1169,6 +1169,8 @@ static moe_status_t run_experts_dq(moe_layer *L, const int *locs, const void *x,
   const bool f16x = c.fmt == MOE_FMT_NVFP4;
   a.act = f16x ? L->xf16 : reinterpret_cast<const uint16_t *>(x);
   a.act_scale = f16x ? L->xs : nullptr;
+  // x rows for the loader's four-row gathers (box one row high)
+  ST_TRY(make_bf16_map(&a.maps.act, a.act, c.hidden, L->cur_T, 1));
   a.h_out = L->hbuf;
   a.work_ctr = L->dq_work;
   a.wfmt = c.fmt == MOE_FMT_INT4G128 ? DQ_I4 : (c.fmt == MOE_FMT_FP8B128 ? DQ_F8 : DQ_NV);
@@ -1183,6 +1185,7 @@ static moe_status_t run_experts_dq(moe_layer *L, const int *locs, const void *x,
   a.n_rowblocks = c.hidden / 256;
   a.act = L->hbuf;
   a.act_scale = nullptr;
+  ST_TRY(make_bf16_map(&a.maps.act, L->hbuf, c.inter, L->max_prows, 64));
   a.o_out = L->oprime;
   a.work_ctr = L->dq_work + 1;
   a.grid = std::min(grid_tiles * a.n_rowblocks, L->n_sms);
@@ -1306,7 +1309,9 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   const bool x16 = (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
   if (dq_only(&c) && !x16) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned for INT4 / FP8 experts");
   const bool dq = L->nv && (dq_only(&c) || P > 12 * act_est) && x16;
-  const int nb_dq = avg >= 96 ? 128 : 64;
+  // 128-token tiles once experts average more than 64 tokens: an MMA issue
+  // costs about as much as an N = 128 MMA runs, so N = 64 tiles halve the rate
+  const int nb_dq = avg > 64 ? 128 : 64;
   const int ts = a4 ? 128 : (tc ? nbox / 2 : (dq ? nb_dq : 8 * nt));
   const int grid_tiles = P / ts + act_est + 1;
   // routing targets (experts, then sinks) and logit rows (+ the shared-expert gate)

@@ -42,10 +42,10 @@
 //                lane quadrant w % 4 of both 128-row halves; NVFP4: hardware
 //                E2M1 -> f16x2 and an f16 multiply by the scale, widened to
 //                bf16 for the down pass);
-//   warps 14..15 activation loaders: the tile's bf16 rows of this K slab by
-//                16-byte cp.async (x rows gathered through the padded-row ->
-//                token map for gate/up; h rows for down), 128-byte swizzled
-//                K-major as the B descriptor reads them.
+//   warp 14      activation loader: the tile's 16-bit rows of this K slab by
+//                TMA (x rows gathered four at a time through the padded-row
+//                -> token map for gate/up; 64-row boxes of h for down),
+//                128-byte swizzled K-major as the B descriptor reads them.
 // TMEM: accumulators (2 x NB columns per buffer; two buffers when NB = 64),
 // then 4 A stages of 64 columns (32 per 128-row half: 64 bf16 of a row).
 // Every mbarrier wait is bounded (error word, then the kernel runs out).
@@ -60,12 +60,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kDqThreads = 512;
-constexpr int kDqDecoders = 256;   // warps 6..13
-constexpr int kDqLoaders = 64;     // warps 14..15
+constexpr int kDqThreads = 480;
+constexpr int kDqDecoders = 256;   // warps 6..13 (warp 14 loads the activations)
 constexpr int kDqSched = 8;
-// arrivals that free a hand-over slot: MMA lane, 4 epilogue warps, 8 decoder warps, 2 loader warps
-constexpr int kDqSchedReaders = 15;
+// arrivals that free a hand-over slot: MMA lane, 4 epilogue warps, 8 decoder warps, the loader warp
+constexpr int kDqSchedReaders = 14;
 // Raw stage of one 64-element K slab of 256 weight rows, per weight format:
 //   DQ_NV  NVFP4: codes 256 rows x 32 bytes, then two 512-byte E4M3 scale blocks
 //          (rows 0..127, 128..255; 4 scales per row);
@@ -135,13 +134,6 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
-__device__ __forceinline__ void cp_async16_dq(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive_dq(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_dq() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ TileInfo load_tile_dq(const TileInfo *p) {
   const int4 v = __ldcg(reinterpret_cast<const int4 *>(p));
@@ -241,7 +233,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
   extern __shared__ __align__(1024) uint8_t dq_smem_raw[];
   __shared__ __align__(8) uint64_t raw_full[SR];    // packed codes + scales landed (TMA / bulk)
   __shared__ __align__(8) uint64_t raw_empty[SR];   // decoders done with a raw stage
-  __shared__ __align__(8) uint64_t op_full[SO];     // bf16 weights decoded + activation rows landed
+  __shared__ __align__(8) uint64_t op_full[SO];     // weights of a slab decoded into a TMEM A stage
+  __shared__ __align__(8) uint64_t b_full[SO];      // activation rows of the slab landed (TMA)
   __shared__ __align__(8) uint64_t op_empty[SO];    // MMAs done with an operand stage
   __shared__ __align__(8) uint64_t accf_bar[NBUF];
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
@@ -268,8 +261,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       mbar_init(smem_u32(&raw_empty[s]), kDqDecoders / 64);     // one slab group
     }
     for (int s = 0; s < SO; ++s) {
-      mbar_init(smem_u32(&op_full[s]), kDqLoaders + kDqDecoders / 64);
+      mbar_init(smem_u32(&op_full[s]), kDqDecoders / 64);
       mbar_init(smem_u32(&op_empty[s]), 1);
+      mbar_init(smem_u32(&b_full[s]), 1);
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(smem_u32(&accf_bar[b]), 1);
@@ -391,8 +385,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         const uint32_t idesc = idesc_16_dq(128, N, kF16);
         bool failed = false;
         for (int slab = 0; slab < nslab; ++slab) {
-          if (!mbar_wait(smem_u32(&op_full[s]), ph, a.err, 51)) { failed = true; break; }
-          fence_proxy_async_dq();
+          if (!mbar_wait(smem_u32(&op_full[s]), ph, a.err, 51) || !mbar_wait(smem_u32(&b_full[s]), ph, a.err, 50)) {
+            failed = true;
+            break;
+          }
           tc_fence_after();
           const uint32_t st = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
           const uint32_t at = tmem + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS);
@@ -518,10 +514,13 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         if (++s == SO) { s = 0; sph ^= 1u; }
       }
     }
-  } else if (warp >= 14) {
-    // ---------------- activation loaders: the tile's bf16 rows of this K slab
-    const int lt = threadIdx.x - 448;                        // 0..63
-    int s = 0, n_slabs = 0;
+  } else if (warp == 14) {
+    // ---------------- activation loader: the tile's 16-bit rows of each K
+    // slab by TMA into the 128-byte swizzled K-major layout of the B
+    // descriptor: x rows gathered four at a time by token index (lane l the
+    // rows 4l .. 4l + 3; pad rows read token 0, never stored), or 64-row
+    // boxes of h (down)
+    int s = 0, n_slabs = 0, issued = 0;
     uint32_t sph = 0;
     int q = 0;
     uint32_t qph = 0;
@@ -540,24 +539,13 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       if (++q == kDqSched) { q = 0; qph ^= 1u; }
       if (item < 0) break;
       if (loc == kLocAbsent) continue;
-      // this thread's rows: j = lt / 8 + 8 i, 16-byte chunk lt % 8 of each;
-      // their element offsets are looked up once per item (one round of
-      // independent loads), not per slab; rows past the tile's tokens are
-      // pad columns the epilogue never stores and are not copied
-      constexpr int RPT = NB / (kDqLoaders / 8);
-      const int cq = lt & 7;
-      uint32_t roff[RPT];
+      int rows[4] = {0, 0, 0, 0};
+      if constexpr (MODE == MODE_GATEUP) {
 #pragma unroll
-      for (int i = 0; i < RPT; ++i) {
-        const int j = (lt >> 3) + (kDqLoaders / 8) * i;
-        roff[i] = 0xFFFFFFFFu;
-        if (j < ti.nrows) {
-          if constexpr (MODE == MODE_GATEUP) {
-            const int tok = checked_index(__ldg(a.prow_token + ti.prow0 + j), 0, a.db.n_tokens, 0, a.db.err, kChkToken);
-            roff[i] = (uint32_t)tok * (uint32_t)K;
-          } else {
-            roff[i] = (uint32_t)(ti.prow0 + j) * (uint32_t)K;
-          }
+        for (int u = 0; u < 4; ++u) {
+          const int j = 4 * lane + u;
+          if (j < NB && j < ti.nrows)
+            rows[u] = checked_index(__ldg(a.prow_token + ti.prow0 + j), 0, a.db.n_tokens, 0, a.db.err, kChkToken);
         }
       }
       for (int slab = 0; slab < nslab; ++slab) {
@@ -566,18 +554,29 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { failed = true; break; }
         const uint32_t bst = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-          const int j = (lt >> 3) + (kDqLoaders / 8) * i;
-          if (roff[i] != 0xFFFFFFFFu)
-            cp_async16_dq(bst + j * 128 + ((cq ^ (j & 7)) << 4), a.act + roff[i] + slab * 64 + cq * 8);
+        const uint32_t bar = smem_u32(&b_full[s]);
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)Geo::B_BYTES);
+        __syncwarp();
+        if constexpr (MODE == MODE_GATEUP) {
+          if (4 * lane < NB) tma_gather4(bst + 512 * lane, &a.maps.act, bar, slab * 64, rows[0], rows[1], rows[2], rows[3]);
+        } else {
+          if (lane < NB / 64) tma_load_2d(bst + 8192 * lane, &a.maps.act, bar, slab * 64, ti.prow0 + 64 * lane);
         }
-        cp_async_arrive_dq(smem_u32(&op_full[s]));
+        ++issued;
         ++n_slabs;
         if (++s == SO) { s = 0; sph ^= 1u; }
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // the last copies issued have landed before the CTA exits (also when a
+    // wait gave up)
+    if (lane == 0) {
+      int s2 = 0;
+      uint32_t ph2 = 0;
+      for (int i = 0; i < issued; ++i) {
+        if (i >= issued - SO) mbar_drain(smem_u32(&b_full[s2]), ph2);
+        if (++s2 == SO) { s2 = 0; ph2 ^= 1u; }
+      }
+    }
   } else {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
     const int quad = warp & 3;

@@ -377,6 +377,10 @@ struct DqMaps {
   // blob), box 32 bytes x (128 rows: gate / up | 256 rows: down) x 1
   CUtensorMap slot[3];
   CUtensorMap stage[3];
+  // the pass's 16-bit activation rows, 128-byte swizzle: gate/up x [T, H] with
+  // a box one row high (rows gathered four at a time by token index), down h
+  // [padded rows, I] with a box of 64 rows
+  CUtensorMap act;
 };
 
 // weight formats of the dequantise-to-shared kernels
