@@ -120,6 +120,8 @@ struct moe_layer {
   uint8_t *xq = nullptr, *xsf = nullptr, *hq = nullptr, *hsf = nullptr;
   float *xG = nullptr, *hG = nullptr, *h32 = nullptr;
   int *n_prows = nullptr;
+  uint16_t *xg = nullptr;            // dequantising path: x rows in padded expert order
+  float *xgs = nullptr;              // their f16 scales (NVFP4)
   int *a4_work = nullptr;            // [kWorkCtrs] item counters of the two A4 passes
   // EXACT numerics of MXFP4 experts on the tensor core (E4M3 activation pieces)
   bool tc = false;
@@ -298,7 +300,11 @@ static bool uses_dq(const moe_config_t *c) {
 static bool dq_only(const moe_config_t *c) { return c->fmt == MOE_FMT_INT4G128 || c->fmt == MOE_FMT_FP8B128; }
 
 static size_t tc_scratch_bytes(const moe_config_t *c) {
-  if (uses_dq(c)) return align256(kWorkCtrs * sizeof(int));
+  if (uses_dq(c)) {
+    const Sizes z = sizes_of(c);
+    return align256(kWorkCtrs * sizeof(int)) + align256(z.max_prows * c->hidden * 2) + align256(z.max_prows * 4) +
+           align256(4);
+  }
   if (!uses_tc(c)) return 0;
   const Sizes z = sizes_of(c);
   const size_t R = z.tc_tiles * kTcSlotRows, H = c->hidden, I = c->inter;
@@ -896,6 +902,10 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   if (L->nv) {
     C_TRY(dalloc(L, &L->dq_work, kWorkCtrs * sizeof(int)));
     C_CUDA(cudaMemsetAsync(L->dq_work, 0, kWorkCtrs * sizeof(int), s));
+    // x rows gathered into the padded expert order (and their f16 scales)
+    C_TRY(dalloc(L, &L->xg, z.max_prows * H * 2));
+    C_TRY(dalloc(L, &L->xgs, z.max_prows * 4));
+    if (!L->n_prows) C_TRY(dalloc(L, &L->n_prows, 4));
   }
   C_TRY(dalloc(L, &L->yout, T * H * 4));
 
@@ -1167,10 +1177,10 @@ static moe_status_t run_experts_dq(moe_layer *L, const int *locs, const void *x,
   // NVFP4: x as f16 rows with a power-of-two scale per token (written into
   // the f16 activation buffer by the conversion before the first pass)
   const bool f16x = c.fmt == MOE_FMT_NVFP4;
-  a.act = f16x ? L->xf16 : reinterpret_cast<const uint16_t *>(x);
-  a.act_scale = f16x ? L->xs : nullptr;
-  // x rows for the loader's four-row gathers (box one row high)
-  ST_TRY(make_bf16_map(&a.maps.act, a.act, c.hidden, L->cur_T, 1));
+  (void)x;
+  a.act = L->xg;                                   // x rows gathered into the padded expert order
+  a.act_scale = f16x ? L->xgs : nullptr;
+  ST_TRY(make_bf16_map(&a.maps.act, L->xg, c.hidden, L->max_prows, 64));
   a.h_out = L->hbuf;
   a.work_ctr = L->dq_work;
   a.wfmt = c.fmt == MOE_FMT_INT4G128 ? DQ_I4 : (c.fmt == MOE_FMT_FP8B128 ? DQ_F8 : DQ_NV);
@@ -1337,7 +1347,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   pa.tiles = L->tiles; pa.n_tiles = L->n_tiles; pa.prow_token = L->prow_token;
   pa.prow_pair = L->prow_pair; pa.active = L->active;
   pa.pad = a4 ? 128 : 8;
-  pa.n_prows = a4 ? L->n_prows : nullptr;
+  pa.n_prows = (a4 || dq) ? L->n_prows : nullptr;
   pa.work_ctr = tc ? L->tc_work : (dq ? L->dq_work : (a4 ? L->a4_work : nullptr));
   pa.tile_done = tc ? L->tile_done : nullptr;
   // decode-sized batches: the router's last CTA also runs the permutation
@@ -1478,11 +1488,12 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     tq.launched(1);
     tq.end();
   }
-  if (dq && c.fmt == MOE_FMT_NVFP4) {
-    // NVFP4 on the tensor core multiplies gate/up in f16: x rows as f16 with a
-    // power-of-two scale per token
+  if (dq) {
+    // the dequantising pass reads x in the padded expert order, one box per
+    // slab; NVFP4 multiplies gate/up in f16 (rows with a power-of-two scale)
     StageTimer tq(L, 8, s);
-    launch_x_rows_f16(reinterpret_cast<const uint16_t *>(x), T, H, L->xf16, L->xs, s);
+    launch_gather_rows(reinterpret_cast<const uint16_t *>(x), H, L->prow_token, L->n_prows, (int)L->max_prows,
+                       c.fmt == MOE_FMT_NVFP4 ? 1 : 0, L->xg, L->xgs, dev_bounds(L), s);
     CUDA_TRY(cudaGetLastError());
     tq.launched(1);
     tq.end();

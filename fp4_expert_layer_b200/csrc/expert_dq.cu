@@ -42,10 +42,10 @@
 //                lane quadrant w % 4 of both 128-row halves; NVFP4: hardware
 //                E2M1 -> f16x2 and an f16 multiply by the scale, widened to
 //                bf16 for the down pass);
-//   warp 14      activation loader: the tile's 16-bit rows of this K slab by
-//                TMA (x rows gathered four at a time through the padded-row
-//                -> token map for gate/up; 64-row boxes of h for down),
-//                128-byte swizzled K-major as the B descriptor reads them.
+//   warp 14      activation loader: the tile's 16-bit rows of this K slab
+//                (x rows gathered into the padded expert order beforehand,
+//                or h) by TMA in 64-row boxes, 128-byte swizzled K-major as
+//                the B descriptor reads them.
 // TMEM: accumulators (2 x NB columns per buffer; two buffers when NB = 64),
 // then 4 A stages of 64 columns (32 per 128-row half: 64 bf16 of a row).
 // Every mbarrier wait is bounded (error word, then the kernel runs out).
@@ -516,10 +516,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
     }
   } else if (warp == 14) {
     // ---------------- activation loader: the tile's 16-bit rows of each K
-    // slab by TMA into the 128-byte swizzled K-major layout of the B
-    // descriptor: x rows gathered four at a time by token index (lane l the
-    // rows 4l .. 4l + 3; pad rows read token 0, never stored), or 64-row
-    // boxes of h (down)
+    // slab (x or h in padded-row order) by TMA, 64-row boxes, into the
+    // 128-byte swizzled K-major layout of the B descriptor
     int s = 0, n_slabs = 0, issued = 0;
     uint32_t sph = 0;
     int q = 0;
@@ -539,15 +537,6 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       if (++q == kDqSched) { q = 0; qph ^= 1u; }
       if (item < 0) break;
       if (loc == kLocAbsent) continue;
-      int rows[4] = {0, 0, 0, 0};
-      if constexpr (MODE == MODE_GATEUP) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = 4 * lane + u;
-          if (j < NB && j < ti.nrows)
-            rows[u] = checked_index(__ldg(a.prow_token + ti.prow0 + j), 0, a.db.n_tokens, 0, a.db.err, kChkToken);
-        }
-      }
       for (int slab = 0; slab < nslab; ++slab) {
         int ok = 1;
         if (lane == 0 && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 56) ? 1 : 0;
@@ -557,11 +546,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         const uint32_t bar = smem_u32(&b_full[s]);
         if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)Geo::B_BYTES);
         __syncwarp();
-        if constexpr (MODE == MODE_GATEUP) {
-          if (4 * lane < NB) tma_gather4(bst + 512 * lane, &a.maps.act, bar, slab * 64, rows[0], rows[1], rows[2], rows[3]);
-        } else {
-          if (lane < NB / 64) tma_load_2d(bst + 8192 * lane, &a.maps.act, bar, slab * 64, ti.prow0 + 64 * lane);
-        }
+        if (lane < NB / 64) tma_load_2d(bst + 8192 * lane, &a.maps.act, bar, slab * 64, ti.prow0 + 64 * lane);
         ++issued;
         ++n_slabs;
         if (++s == SO) { s = 0; sph ^= 1u; }
@@ -612,10 +597,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         my_pair = checked_index(__ldg(a.prow_pair + ti.prow0 + et), 0, a.db.n_pairs, 0, a.db.err, kChkPair);
         my_gate = __ldg(a.gates + my_pair);
       }
-      if (kF16 && et < ntok) {
-        const int tok = checked_index(__ldg(a.prow_token + ti.prow0 + et), 0, a.db.n_tokens, 0, a.db.err, kChkToken);
-        my_gate = __ldg(a.act_scale + tok);
-      }
+      if (kF16 && et < ntok) my_gate = __ldg(a.act_scale + ti.prow0 + et);
       ok = mbar_wait(smem_u32(&accf_bar[buf]), (n / NBUF) & 1, a.err, 57);
       if ((MODE == MODE_DOWN || kF16) && et < ntok) {
         tok_pair[et] = my_pair;
@@ -679,19 +661,30 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
   }
 }
 
-// x rows (bf16) -> f16 rows, each multiplied by a power of two 2^p that puts
-// its largest magnitude in [2^14, 2^15): every element within 2^31 of the
-// row's maximum converts exactly (f16 keeps 11 significant bits, bf16 has 8;
-// smaller ones land on the f16 subnormal grid, off by less than 2^-25 of the
-// row maximum).  xs[row] = 2^-p, applied to the row's accumulators.  One warp
-// per row, 16-byte loads and stores (H a multiple of 256, rows 16-byte aligned).
-__global__ void __launch_bounds__(256) x_rows_f16_kernel(const uint16_t *x, int T, int H, uint16_t *xh, float *xs) {
+// The gate/up activations in the padded expert order: padded row r is token
+// prow_token[r]'s x row (pad rows, token -1, are left as they are: their
+// columns are never stored), as bf16 (to_f16 = 0) or as f16 multiplied by a
+// power of two 2^p that puts the token's largest magnitude in [2^14, 2^15)
+// (every element within 2^31 of the row's maximum converts exactly: f16 keeps
+// 11 significant bits, bf16 has 8; smaller ones land on the f16 subnormal
+// grid, off by less than 2^-25 of the maximum), xs[r] = 2^-p.  The expert
+// pass then reads each tile's rows as one contiguous box per K slab.  One warp
+// per padded row, 16-byte loads and stores (H a multiple of 256).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t *x, int H, const int *prow_token,
+                                                          const int *n_rows, int max_rows, int to_f16,
+                                                          uint16_t *xg, float *xs, DevBounds db) {
   wait_prior_grid();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (row >= T) return;
-  const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)row * H);
-  uint4 *dst = reinterpret_cast<uint4 *>(xh + (size_t)row * H);
+  if (row >= max_rows || row >= __ldcg(n_rows)) return;
+  const int tok = checked_index(__ldcg(prow_token + row), -1, db.n_tokens, -1, db.err, kChkToken);
+  if (tok < 0) return;
+  const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)tok * H);
+  uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)row * H);
   const int n8 = H / 8;
+  if (!to_f16) {
+    for (int i = lane; i < n8; i += 32) dst[i] = src[i];
+    return;
+  }
   uint32_t am = 0;                                    // largest |bf16| bit pattern (orders like the magnitude)
   for (int i = lane; i < n8; i += 32) {
     const uint4 v = src[i];
@@ -717,9 +710,11 @@ __global__ void __launch_bounds__(256) x_rows_f16_kernel(const uint16_t *x, int 
   if (lane == 0) xs[row] = __int_as_float((127 - p) << 23);
 }
 
-void launch_x_rows_f16(const uint16_t *x, int T, int H, uint16_t *xh, float *xs, cudaStream_t s) {
-  if (T <= 0) return;
-  launch_dependent(x_rows_f16_kernel, (T + 7) / 8, 256, 0, s, x, T, H, xh, xs);
+void launch_gather_rows(const uint16_t *x, int H, const int *prow_token, const int *n_rows, int max_rows,
+                        int to_f16, uint16_t *xg, float *xs, const DevBounds &db, cudaStream_t s) {
+  if (max_rows <= 0) return;
+  launch_dependent(gather_rows_kernel, (max_rows + 7) / 8, 256, 0, s, x, H, prow_token, n_rows, max_rows, to_f16,
+                   xg, xs, db);
 }
 
 template <int MODE, int NB, int F>

@@ -377,9 +377,8 @@ struct DqMaps {
   // blob), box 32 bytes x (128 rows: gate / up | 256 rows: down) x 1
   CUtensorMap slot[3];
   CUtensorMap stage[3];
-  // the pass's 16-bit activation rows, 128-byte swizzle: gate/up x [T, H] with
-  // a box one row high (rows gathered four at a time by token index), down h
-  // [padded rows, I] with a box of 64 rows
+  // the pass's 16-bit activation rows in padded-row order (gate/up: x rows
+  // gathered beforehand; down: h), 128-byte swizzle, box 64 x 64 rows
   CUtensorMap act;
 };
 
@@ -400,8 +399,9 @@ struct DqArgs {
   const int *prow_token;     // gate/up: padded row -> token
   const int *prow_pair;      // down: padded row -> pair
   const float *gates;
-  const uint16_t *act;       // gate/up: x bf16 [T, H] (NVFP4: f16 rows, see act_scale); down: h bf16 [padded rows, I]
-  const float *act_scale;    // gate/up of NVFP4 layers: per-token scale of the f16 x rows (x = row * scale)
+  const uint16_t *act;       // gate/up: x rows in padded-row order [padded rows, H], bf16 (NVFP4: f16, see
+                             // act_scale); down: h bf16 [padded rows, I]
+  const float *act_scale;    // gate/up of NVFP4 layers: per padded row, the scale of its f16 x row (x = row * scale)
   uint16_t *h_out;           // gate/up: h bf16 [padded rows, I]
   float *o_out;              // down: O' [pairs, H]
   int *work_ctr;             // item counter of this pass, zero at launch
@@ -411,8 +411,10 @@ struct DqArgs {
 };
 // nb: tokens per tile (64 or 128)
 void launch_expert_dq(int mode, int nb, const DqArgs &a, cudaStream_t s);
-// x rows (bf16) -> f16 rows with a power-of-two scale per row (xs = the
-// inverse), the gate/up activations of NVFP4 layers on the tensor core
-void launch_x_rows_f16(const uint16_t *x, int T, int H, uint16_t *xh, float *xs, cudaStream_t s);
+// x rows into the padded expert order for the dequantising expert pass:
+// bf16 copies, or (to_f16) f16 rows with a power-of-two scale per row (xs =
+// its inverse); rows up to *n_rows, pad rows (token -1) left as they are
+void launch_gather_rows(const uint16_t *x, int H, const int *prow_token, const int *n_rows, int max_rows,
+                        int to_f16, uint16_t *xg, float *xs, const DevBounds &db, cudaStream_t s);
 
 }  // namespace moe

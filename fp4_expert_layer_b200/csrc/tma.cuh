@@ -130,17 +130,6 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *tmap, uint
       : "memory");
 }
 
-// Four rows of a 2-D tensor (row indices r0..r3; the map's box is one row
-// high) into four consecutive box rows of shared memory (tile::gather4).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, uint32_t bar, int c0, int r0, int r1,
-                                            int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-      "%4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // Fetch a tensor map into the descriptor cache ahead of its first use.
 __device__ __forceinline__ void tmap_prefetch(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
