@@ -131,6 +131,7 @@ struct moe_layer {
   uint8_t *txq = nullptr, *txsf = nullptr, *thq = nullptr, *thsf = nullptr;
   int *tc_work = nullptr;            // [kWorkCtrs] item counters of the expert passes
   int *tile_done = nullptr;          // [tc tiles] gate/up items finished per tile (decode hand-over)
+  CUtensorMap tc_act[2];             // activation-piece maps of the two passes (x pieces, h pieces)
   // EXACT numerics of NVFP4 experts at prefill sizes on the tensor core
   // (weights decoded to bf16 in shared memory)
   bool nv = false;
@@ -465,6 +466,21 @@ static moe_status_t make_tc_weight_map(CUtensorMap *map, const uint8_t *region, 
     snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (%d) for a tiled weight map", (int)r);
     return fail(MOE_ERR_CUDA, buf);
   }
+  return MOE_OK;
+}
+
+// Activation-piece rows [rows, row_bytes] E4M3: box 128 bytes x 16 rows, 128-byte swizzle.
+static moe_status_t make_piece_map(CUtensorMap *map, const void *base, size_t row_bytes, size_t rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {128, 16};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation-piece map");
   return MOE_OK;
 }
 
@@ -897,6 +913,8 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
     C_CUDA(cudaMemsetAsync(L->tc_work, 0, kWorkCtrs * sizeof(int), s));
     C_TRY(dalloc(L, &L->tile_done, z.tc_tiles * sizeof(int)));
     C_CUDA(cudaMemsetAsync(L->tile_done, 0, z.tc_tiles * sizeof(int), s));
+    C_TRY(make_piece_map(&L->tc_act[0], L->txq, H, R));
+    C_TRY(make_piece_map(&L->tc_act[1], L->thq, I, R));
   }
   L->nv = uses_dq(cfg);
   if (L->nv) {
@@ -1116,6 +1134,7 @@ static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int 
   a.hsf = L->thsf;
   a.o_out = L->oprime;
   a.act = L->txq;
+  a.maps.act = L->tc_act[0];
   a.K = c.hidden;
   a.rows = c.inter;
   a.n_rowblocks = c.inter / 128;
@@ -1133,6 +1152,7 @@ static moe_status_t run_experts_tc(moe_layer *L, const int *locs, int nbox, int 
   t3.launched(1);
   t3.end();
   a.act = L->thq;
+  a.maps.act = L->tc_act[1];
   a.K = c.inter;
   a.rows = c.hidden;
   a.n_rowblocks = c.hidden / 256;

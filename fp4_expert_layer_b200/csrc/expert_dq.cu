@@ -32,9 +32,9 @@
 //                codes (32 bytes x 128 or 256 rows) per matrix and the
 //                512-byte E4M3 scale-factor blocks by bulk copy, into a ring
 //                of raw stages;
-//   warp 1       MMA issuer (one lane): M = 128, N = tokens rounded up to 16,
-//                K = 16, A from TMEM, B from shared memory, two accumulators
-//                (gate and up, or the two 128-row halves of down) per item;
+//   warps 1, 15  MMA issuers (one lane each, one accumulator each: gate and
+//                up, or the two 128-row halves of down): M = 128, N = tokens
+//                rounded up to 16, K = 16, A from TMEM, B from shared memory;
 //   warps 2..5   epilogue: TMEM -> SwiGLU -> h (bf16, padded-row order), or
 //                G_d * gate * acc -> O' (fp32, pair order);
 //   warps 6..13  decoders: raw stage -> weight rows in TMEM, in two groups
@@ -60,11 +60,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kDqThreads = 480;
+constexpr int kDqThreads = 512;
 constexpr int kDqDecoders = 256;   // warps 6..13 (warp 14 loads the activations)
 constexpr int kDqSched = 8;
-// arrivals that free a hand-over slot: MMA lane, 4 epilogue warps, 8 decoder warps, the loader warp
-constexpr int kDqSchedReaders = 14;
+// arrivals that free a hand-over slot: 2 MMA lanes, 4 epilogue warps, 8 decoder warps, the loader warp
+constexpr int kDqSchedReaders = 15;
 // Raw stage of one 64-element K slab of 256 weight rows, per weight format:
 //   DQ_NV  NVFP4: codes 256 rows x 32 bytes, then two 512-byte E4M3 scale blocks
 //          (rows 0..127, 128..255; 4 scales per row);
@@ -262,18 +262,18 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
     }
     for (int s = 0; s < SO; ++s) {
       mbar_init(smem_u32(&op_full[s]), kDqDecoders / 64);
-      mbar_init(smem_u32(&op_empty[s]), 1);
+      mbar_init(smem_u32(&op_empty[s]), 2);               // both MMA issuers
       mbar_init(smem_u32(&b_full[s]), 1);
     }
     for (int b = 0; b < NBUF; ++b) {
-      mbar_init(smem_u32(&accf_bar[b]), 1);
+      mbar_init(smem_u32(&accf_bar[b]), 2);
       mbar_init(smem_u32(&acce_bar[b]), 4);
     }
     for (int q = 0; q < kDqSched; ++q) {
       mbar_init(smem_u32(&sched_full[q]), 1);
       mbar_init(smem_u32(&sched_empty[q]), kDqSchedReaders);
     }
-    mbar_init(smem_u32(&quiesce_bar), 1);
+    mbar_init(smem_u32(&quiesce_bar), 2);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -361,13 +361,20 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         }
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (one lane)
+  } else if (warp == 1 || warp == 15) {
+    // ---------------- MMA issuers: lane 0 of warp 1 issues the MMAs of the
+    // first accumulator (gate, or the first 128 down rows), lane 0 of warp 15
+    // those of the second; each K slab is 4 MMAs of K = 16 per issuer (a
+    // single issuer spent about as long issuing the 8 MMAs of a slab as the
+    // tensor core took to run them).  Descriptors advance from one computed
+    // up front.
     if (lane == 0) {
+      const int h = warp == 1 ? 0 : 1;
       int s = 0, n = 0;
       uint32_t ph = 0;
       int q = 0;
       uint32_t qph = 0;
+      const uint64_t bdesc0 = umma_desc(smem_u32(smem), 16, 1024, 2);
       while (true) {
         if (!mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 59)) break;
         const int item = sched_item[q];
@@ -381,7 +388,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         const int buf = n % NBUF;
         if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 54)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * Geo::ACC_COLS);
+        const uint32_t acc = tmem + (uint32_t)(buf * Geo::ACC_COLS + h * NB);
         const uint32_t idesc = idesc_16_dq(128, N, kF16);
         bool failed = false;
         for (int slab = 0; slab < nslab; ++slab) {
@@ -390,17 +397,12 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
             break;
           }
           tc_fence_after();
-          const uint32_t st = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
-          const uint32_t at = tmem + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS);
+          const uint64_t bd = bdesc0 + (uint64_t)(((uint32_t)s * (uint32_t)Geo::OP_STAGE) >> 4);
+          const uint32_t at = tmem + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS + h * 32);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {                   // K = 16 per MMA (8 TMEM columns of A)
-            const uint64_t bdesc = umma_desc(st + 32 * kk, 16, 1024, 2);
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              umma_bf16_ts(acc + (uint32_t)(h * NB), at + (uint32_t)(h * 32 + 8 * kk), bdesc, idesc,
-                           (slab > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(smem_u32(&op_empty[s]));                 // stage free once these MMAs finish
+          for (int kk = 0; kk < 4; ++kk)                     // K = 16 per MMA (8 TMEM columns of A, 32 B of B)
+            umma_bf16_ts(acc, at + (uint32_t)(8 * kk), bd + (uint64_t)(2 * kk), idesc, (slab > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(smem_u32(&op_empty[s]));                 // stage free once both issuers' MMAs finish
           if (++s == SO) { s = 0; ph ^= 1u; }
         }
         if (failed) break;

@@ -48,22 +48,13 @@ namespace moe {
 namespace {
 
 // warp 0: weight TMA; warp 1: TMEM allocation and MMA issue; warps 2..5:
-// epilogue; warps 6..7: activation pieces and scale factors by cp.async (the
-// LSU path), so that the per-SM TMA unit carries only the weight stream
+// epilogue; warp 6: activation pieces (16-row TMA boxes) and scale factors
+// (bulk copies), one lane; a per-lane cp.async copy of the pieces cost about
+// a thousand cycles of issue per slab at prefill tile sizes
 constexpr int kTcThreads = 256;
-constexpr int kTcLoaders = 64;
 constexpr int kSched = 8;         // work items handed from the producer to the other roles in flight
-constexpr int kSchedReaders = 7;  // arrivals that free a hand-over slot: MMA lane, 2 loader warps, 4 epilogue warps
+constexpr int kSchedReaders = 6;  // arrivals that free a hand-over slot: MMA lane, the loader warp, 4 epilogue warps
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-// Arrive on `bar` once every cp.async this thread issued so far has landed
-// (the barrier's expected count includes these arrivals).
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // tile descriptor read from L2 (written by another kernel)
 __device__ __forceinline__ TileInfo load_tile(const TileInfo *p) {
@@ -132,7 +123,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   constexpr int NBUF = Geo::NBUF;
   extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[S];    // weights landed (TMA)
-  __shared__ __align__(8) uint64_t bfull_bar[S];   // activation pieces + scale factors landed (cp.async)
+  __shared__ __align__(8) uint64_t bfull_bar[S];   // activation pieces + scale factors landed (TMA, bulk)
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ __align__(8) uint64_t accf_bar[NBUF];
   __shared__ __align__(8) uint64_t acce_bar[NBUF];
@@ -162,7 +153,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
-      mbar_init(smem_u32(&bfull_bar[s]), kTcLoaders);
+      mbar_init(smem_u32(&bfull_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     for (int b = 0; b < NBUF; ++b) {
@@ -341,64 +332,78 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       mbar_drain(smem_u32(&quiesce_bar), 0);
     }
   } else if (warp >= 6) {
-    // ---------------- loaders: the tile's activation-piece rows of this K slab
-    // (written with the 128-byte swizzle the MMA descriptor expects) and the
-    // three scale-factor blocks, by 16-byte cp.async
-    const int lt = threadIdx.x - 192;
-    int s = 0, issued = 0;
-    uint32_t ph = 0;
-    int q = 0;
-    uint32_t qph = 0;
-    bool failed = false;
-    while (!failed) {
-      int okw = 1;
-      if (lane == 0) okw = mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 40) ? 1 : 0;
-      okw = __shfl_sync(0xffffffffu, okw, 0);
-      if (!okw) break;                                       // warp-uniform
-      __syncwarp();
-      const int item = sched_item[q];
-      const TileInfo ti = sched_ti[q];
-      const int loc = sched_loc[q];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
-      if (++q == kSched) { q = 0; qph ^= 1u; }
-      if (item < 0) break;
-      if (loc == kLocAbsent) continue;
-      const int tile = item / ipt, rb = item % ipt;
-      const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
-      const int act_row0 = tile * kTcSlotRows;
-      // scale blocks of the chunk's two halves (1 KB per chunk), and of the activation rows
-      const uint8_t *sfa = blob + a.L.scales[MODE == MODE_GATEUP ? 0 : 2] + (size_t)rb * nslab * kTcSfChunk;
-      const uint8_t *sfb = a.bsf + sf_offset(nsf, act_row0, 0);
-      const uint8_t *act = a.act + (size_t)act_row0 * K;
-      const int nb = 8 * max(16, (2 * ti.nrows + 15) & ~15);   // 16-byte chunks of the piece rows read
-      if (per_tile) {
-        // this tile's h pieces are complete once every gate/up item of it is
-        int okt = 1;
-        if (lane == 0) okt = flag_wait(a.tile_done + tile, a.tile_target, a.err, 42) ? 1 : 0;
-        okt = __shfl_sync(0xffffffffu, okt, 0);
-        if (!okt) { failed = true; break; }                  // warp-uniform
-      }
-      for (int slab = 0; slab < nslab; ++slab) {
-        if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 35)) { failed = true; break; }
-        const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
-        for (int c = lt; c < nb + 96; c += kTcLoaders) {
-          if (c < nb) {
-            const int r = c >> 3, q = c & 7;
-            cp_async16(st + Geo::B_OFF + r * 128 + ((q ^ (r & 7)) << 4), act + (size_t)r * K + slab * 128 + q * 16);
-          } else {
-            const int cc = c - nb;
-            const uint8_t *src = cc < 64 ? sfa + (size_t)slab * kTcSfChunk + cc * 16
-                                         : sfb + (size_t)slab * 512 + (cc - 64) * 16;
-            cp_async16(st + Geo::SF_OFF + cc * 16, src);
+    // ---------------- loader (warp 6, one lane): per K slab, the tile's
+    // activation-piece rows by TMA (16-row boxes, 128-byte swizzle as the MMA
+    // descriptor reads them) and the three scale-factor blocks (the weight
+    // chunk's two halves, the activation rows) by bulk copy
+    if (warp == 6) {
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      int q = 0;
+      uint32_t qph = 0;
+      bool failed = false;
+      while (!failed) {
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 40) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) break;                                     // warp-uniform
+        __syncwarp();
+        const int item = sched_item[q];
+        const TileInfo ti = sched_ti[q];
+        const int loc = sched_loc[q];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+        if (++q == kSched) { q = 0; qph ^= 1u; }
+        if (item < 0) break;
+        if (loc == kLocAbsent) continue;
+        const int tile = item / ipt, rb = item % ipt;
+        const uint8_t *blob = (loc >= 0 ? a.slots : a.staging) + (size_t)(loc >= 0 ? loc : (-2 - loc)) * a.blob_bytes;
+        const int act_row0 = tile * kTcSlotRows;
+        // scale blocks of the chunk's two halves (1 KB per chunk), and of the activation rows
+        const uint8_t *sfa = blob + a.L.scales[MODE == MODE_GATEUP ? 0 : 2] + (size_t)rb * nslab * kTcSfChunk;
+        const uint8_t *sfb = a.bsf + sf_offset(nsf, act_row0, 0);
+        const int nbox = max(16, (2 * ti.nrows + 15) & ~15) / 16;   // 16-row boxes of piece rows read
+        const uint32_t tx = (uint32_t)(nbox * 16 * 128 + kTcSfChunk + 512);
+        if (per_tile) {
+          // this tile's h pieces are complete once every gate/up item of it is
+          int okt = 1;
+          if (lane == 0) okt = flag_wait(a.tile_done + tile, a.tile_target, a.err, 42) ? 1 : 0;
+          okt = __shfl_sync(0xffffffffu, okt, 0);
+          if (!okt) { failed = true; break; }                // warp-uniform
+          // the h pieces were written by other CTAs' ordinary stores; the TMA
+          // reads them through the async proxy
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        if (lane == 0) {
+          for (int slab = 0; slab < nslab; ++slab) {
+            if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 35)) { failed = true; break; }
+            const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+            const uint32_t bar = smem_u32(&bfull_bar[s]);
+            mbar_arrive_expect_tx(bar, tx);
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d(st + Geo::B_OFF + b * 2048, &a.maps.act, bar, slab * 128, act_row0 + 16 * b);
+            bulk_load(st + Geo::SF_OFF, sfa + (size_t)slab * kTcSfChunk, kTcSfChunk, bar);
+            bulk_load(st + Geo::SF_OFF + kTcSfChunk, sfb + (size_t)slab * 512, 512, bar);
+            ++issued;
+            if (++s == S) { s = 0; ph ^= 1u; }
           }
         }
-        cp_async_arrive(smem_u32(&bfull_bar[s]));
-        ++issued;
-        if (++s == S) { s = 0; ph ^= 1u; }
+        failed = __shfl_sync(0xffffffffu, failed ? 1 : 0, 0) != 0;
+        issued = __shfl_sync(0xffffffffu, issued, 0);
+        s = __shfl_sync(0xffffffffu, s, 0);
+        ph = __shfl_sync(0xffffffffu, ph, 0);
+      }
+      // the last copies issued have landed before the CTA exits (also when a
+      // wait gave up)
+      if (lane == 0) {
+        int s2 = 0;
+        uint32_t ph2 = 0;
+        for (int i = 0; i < issued; ++i) {
+          if (i >= issued - S) mbar_drain(smem_u32(&bfull_bar[s2]), ph2);
+          if (++s2 == S) { s2 = 0; ph2 ^= 1u; }
+        }
       }
     }
-    cp_async_wait_all();
   } else {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
     const int quad = warp & 3;

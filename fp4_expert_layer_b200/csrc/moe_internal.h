@@ -294,6 +294,9 @@ struct TcMaps {
   //                  1 = down (3-D: K, rows, blob; box 128 x 256 x 1)]: E2M1 codes unpacked by the
   // TMA to one byte per element, 128-byte swizzle
   CUtensorMap w[2][2];
+  // the pass's activation pieces [slot rows, K] E4M3 (x pieces for gate/up,
+  // h pieces for down), box 128 bytes x 16 rows, 128-byte swizzle
+  CUtensorMap act;
 };
 
 struct TcQuantArgs {
