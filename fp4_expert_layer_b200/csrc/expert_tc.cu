@@ -47,15 +47,15 @@ namespace moe {
 
 namespace {
 
-// warp 0: weight TMA; warp 1: TMEM allocation and MMA issue; warps 2..5:
-// epilogue; warp 6: activation pieces (16-row TMA boxes) and scale factors
-// (bulk copies), one lane; a per-lane cp.async copy of the pieces cost about
+// warp 0: weight TMA; warp 1: TMEM allocation and MMA issue (first
+// accumulator); warps 2..5: epilogue; warp 6: activation pieces (16-row TMA
+// boxes) and scale factors (bulk copies), one lane; warp 7: MMA issue (second
+// accumulator); a per-lane cp.async copy of the pieces cost about
 // a thousand cycles of issue per slab at prefill tile sizes
 constexpr int kTcThreads = 256;
 constexpr int kSched = 8;         // work items handed from the producer to the other roles in flight
-constexpr int kSchedReaders = 6;  // arrivals that free a hand-over slot: MMA lane, the loader warp, 4 epilogue warps
+constexpr int kSchedReaders = 7;  // arrivals that free a hand-over slot: 2 MMA lanes, the loader warp, 4 epilogue warps
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // tile descriptor read from L2 (written by another kernel)
 __device__ __forceinline__ TileInfo load_tile(const TileInfo *p) {
   const int4 v = __ldcg(reinterpret_cast<const int4 *>(p));
@@ -107,9 +107,12 @@ struct TcGeom {
   static constexpr int SF_OFF = B_OFF + B_BYTES;     // SFA half 0, SFA half 1, SFB: 512 B each
   static constexpr int STAGE = ((SF_OFF + 3 * 512) + 1023) / 1024 * 1024;
   // accumulator buffers: two whenever they fit in TMEM beside the scale columns
-  static constexpr int NBUF = (2 * 2 * NBOX + 12 * STAGES <= 512) ? 2 : 1;
+  // TMEM scale columns per stage: per MMA issuer its weight half's block and
+  // its own copy of the activation block (4 columns each)
+  static constexpr int SF_PER_STAGE = 16;
+  static constexpr int NBUF = (2 * 2 * NBOX + SF_PER_STAGE * STAGES <= 512) ? 2 : 1;
   static constexpr int SF_COL0 = NBUF * 2 * NBOX;    // TMEM: accumulators first
-  static constexpr int COLS_NEEDED = SF_COL0 + 12 * STAGES;
+  static constexpr int COLS_NEEDED = SF_COL0 + SF_PER_STAGE * STAGES;
   static constexpr int TMEM_COLS = COLS_NEEDED <= 128 ? 128 : (COLS_NEEDED <= 256 ? 256 : 512);
   static_assert(COLS_NEEDED <= 512, "TMEM budget");
   static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024;
@@ -154,17 +157,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&bfull_bar[s]), 1);
-      mbar_init(smem_u32(&empty_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 2);           // both MMA issuers commit
     }
     for (int b = 0; b < NBUF; ++b) {
-      mbar_init(smem_u32(&accf_bar[b]), 1);
+      mbar_init(smem_u32(&accf_bar[b]), 2);
       mbar_init(smem_u32(&acce_bar[b]), 4);           // one arrival per epilogue warp
     }
     for (int q = 0; q < kSched; ++q) {
       mbar_init(smem_u32(&sched_full[q]), 1);
       mbar_init(smem_u32(&sched_empty[q]), kSchedReaders);
     }
-    mbar_init(smem_u32(&quiesce_bar), 1);
+    mbar_init(smem_u32(&quiesce_bar), 2);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -272,14 +275,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
         }
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (one lane)
+  } else if (warp == 1 || warp == 7) {
+    // ---------------- MMA issuers: lane 0 of warp 1 the MMAs of the first
+    // accumulator (gate, or the first 128 down rows), lane 0 of warp 7 those
+    // of the second.  Each copies the scale blocks its MMAs read (its weight
+    // half, and its own copy of the activation block: a tcgen05.cp is ordered
+    // only before the MMAs of the thread that issued it).  Descriptors
+    // advance from ones computed up front.
     if (lane == 0) {
+      const int h = warp == 1 ? 0 : 1;
       int s = 0, n = 0;
       uint32_t ph = 0;
       int q = 0;
       uint32_t qph = 0;
       bool failed = false;
+      const uint32_t sbase = smem_u32(smem);
+      const uint64_t adesc0 = umma_desc(sbase + h * 16384, 16, 1024, 2);
+      const uint64_t bdesc0 = umma_desc(sbase + Geo::B_OFF, 16, 1024, 2);
       while (!failed) {
         if (!mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 39)) break;
         const int item = sched_item[q];
@@ -294,33 +306,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
         // the epilogue must have drained this accumulator buffer
         if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 34)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX);
+        const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX + h * NBOX);
+        uint32_t idesc[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          idesc[kk] = idesc_f8f6f4_block(128, N, kFmtE2M1_f8f6f4, kFmtE4M3, (uint32_t)kk, (uint32_t)kk);
         for (int slab = 0; slab < nslab; ++slab) {
           if (!mbar_wait(smem_u32(&full_bar[s]), ph, a.err, 31) ||
               !mbar_wait(smem_u32(&bfull_bar[s]), ph, a.err, 36)) {
             failed = true;
             break;
           }
-          fence_proxy_async();                               // cp.async data -> tensor-core reads
           tc_fence_after();
-          const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
-          const uint32_t sf = tmem + (uint32_t)(Geo::SF_COL0 + 12 * s);
-          tc_cp_sf_block(sf, st + Geo::SF_OFF);
-          tc_cp_sf_block(sf + 4, st + Geo::SF_OFF + 512);
-          tc_cp_sf_block(sf + 8, st + Geo::SF_OFF + 1024);
+          const uint32_t soff = (uint32_t)s * (uint32_t)Geo::STAGE;
+          const uint32_t sf = tmem + (uint32_t)(Geo::SF_COL0 + Geo::SF_PER_STAGE * s + 8 * h);
+          tc_cp_sf_block(sf, sbase + soff + Geo::SF_OFF + 512 * h);       // this half's weight scales
+          tc_cp_sf_block(sf + 4, sbase + soff + Geo::SF_OFF + 1024);      // the activation rows' scales
+          const uint64_t ad = adesc0 + (uint64_t)(soff >> 4), bd = bdesc0 + (uint64_t)(soff >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {                  // K = 32 per MMA
-            const uint64_t bdesc = umma_desc(st + Geo::B_OFF + 32 * kk, 16, 1024, 2);
-            const uint32_t idesc = idesc_f8f6f4_block(128, N, kFmtE2M1_f8f6f4, kFmtE4M3, (uint32_t)kk, (uint32_t)kk);
-            const uint32_t sfb = (sf + 8) | ((uint32_t)kk << 30);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint64_t adesc = umma_desc(st + h * 16384 + 32 * kk, 16, 1024, 2);
-              umma_mxf8f6f4(acc + (uint32_t)(h * NBOX), adesc, bdesc, idesc, (sf + 4 * h) | ((uint32_t)kk << 30),
-                            sfb, (slab > 0 || kk > 0) ? 1u : 0u);
-            }
-          }
-          tc_commit(smem_u32(&empty_bar[s]));                // stage free once these MMAs finish
+          for (int kk = 0; kk < 4; ++kk)                    // K = 32 per MMA
+            umma_mxf8f6f4(acc, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc[kk], sf | ((uint32_t)kk << 30),
+                          (sf + 4) | ((uint32_t)kk << 30), (slab > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(smem_u32(&empty_bar[s]));                // stage free once both issuers' MMAs finish
           if (++s == S) { s = 0; ph ^= 1u; }
         }
         tc_commit(smem_u32(&accf_bar[buf]));                 // this item's accumulators complete
@@ -331,7 +338,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       tc_commit(smem_u32(&quiesce_bar));
       mbar_drain(smem_u32(&quiesce_bar), 0);
     }
-  } else if (warp >= 6) {
+  } else if (warp == 6) {
     // ---------------- loader (warp 6, one lane): per K slab, the tile's
     // activation-piece rows by TMA (16-row boxes, 128-byte swizzle as the MMA
     // descriptor reads them) and the three scale-factor blocks (the weight
