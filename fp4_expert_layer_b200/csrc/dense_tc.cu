@@ -143,24 +143,26 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_tc_kernel(const __grid
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
-      int s = 0, n = 0;
-      uint32_t ph = 0;
-      bool failed = false;
-      for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
-        const int tile = item / ipt;
-        const int ntok = min(NBOX, a.T - tile * NBOX);
-        const int N = max(16, (ntok + 15) & ~15);
-        const int buf = n % NBUF;
-        if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 44)) break;
+    // ---------------- MMA issuer: the whole warp runs the loop (every wait
+    // warp-uniform) and one elected lane issues, so that the MMA operands stay
+    // in uniform registers
+    int s = 0, n = 0;
+    uint32_t ph = 0;
+    bool failed = false;
+    for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
+      const int tile = item / ipt;
+      const int ntok = min(NBOX, a.T - tile * NBOX);
+      const int N = max(16, (ntok + 15) & ~15);
+      const int buf = n % NBUF;
+      if (n >= NBUF && !mbar_wait_warp(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 44)) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX);
+      const uint32_t idesc = idesc_bf16(128, N);
+      for (int slab = 0; slab < nslab; ++slab) {
+        if (!mbar_wait_warp(smem_u32(&full_bar[s]), ph, a.err, 41)) { failed = true; break; }
         tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX);
-        const uint32_t idesc = idesc_bf16(128, N);
-        for (int slab = 0; slab < nslab; ++slab) {
-          if (!mbar_wait(smem_u32(&full_bar[s]), ph, a.err, 41)) { failed = true; break; }
-          tc_fence_after();
-          const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+        const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {                 // K = 16 per MMA
             const uint64_t bdesc = umma_desc(st + Geo::B_OFF + 32 * kk, 16, 1024, 2);
@@ -171,16 +173,21 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_tc_kernel(const __grid
             }
           }
           tc_commit(smem_u32(&empty_bar[s]));
-          if (++s == S) { s = 0; ph ^= 1u; }
         }
-        tc_commit(smem_u32(&accf_bar[buf]));
-        ++n;
+        __syncwarp();
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
-      // every MMA issued above has completed before the CTA frees TMEM and
-      // leaves (also after a wait gave up and the loop was left early)
-      tc_commit(smem_u32(&quiesce_bar));
-      mbar_drain(smem_u32(&quiesce_bar), 0);
+      if (failed) break;
+      if (elect_one()) tc_commit(smem_u32(&accf_bar[buf]));
+      __syncwarp();
+      ++n;
     }
+    // every MMA issued above has completed before the CTA frees TMEM and
+    // leaves (also after a wait gave up and the loop was left early)
+    __syncwarp();
+    if (elect_one()) tc_commit(smem_u32(&quiesce_bar));
+    __syncwarp();
+    mbar_drain(smem_u32(&quiesce_bar), 0);
   } else {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
     const int quad = warp & 3;
@@ -204,12 +211,16 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_tc_kernel(const __grid
           tmem_ld32(acc + (uint32_t)(NBOX + c0), u);
           tmem_ld_wait();
           if (!ok) continue;
+          // all 32 columns without a branch (columns past the tile's tokens
+          // are not stored), so that different tokens' exp / reciprocal
+          // chains overlap
+          uint16_t hv[32];
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            if (c0 + jj >= ntok) continue;
-            const float h = silu_f(__uint_as_float(g[jj])) * __uint_as_float(u[jj]);
-            a.h_out[(size_t)(t0 + c0 + jj) * Is + r] = bf16_bits(h);
-          }
+          for (int jj = 0; jj < 32; ++jj) hv[jj] = bf16_bits(silu_f(__uint_as_float(g[jj])) * __uint_as_float(u[jj]));
+          const int nj = min(32, ntok - c0);
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (jj < nj) a.h_out[(size_t)(t0 + c0 + jj) * Is + r] = hv[jj];
         }
       } else {
         const int H = a.rows;
@@ -364,15 +375,17 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      bool failed = false;
-      const uint32_t idesc = idesc_bf16(128, NP);
-      for (int slab = s0; slab < s1; ++slab) {
-        if (!mbar_wait(smem_u32(&full_bar[s]), ph, a.err, 47)) { failed = true; break; }
-        tc_fence_after();
-        const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+    // MMA issuer: the whole warp runs the loop (every wait warp-uniform) and
+    // one elected lane issues
+    int s = 0;
+    uint32_t ph = 0;
+    bool failed = false;
+    const uint32_t idesc = idesc_bf16(128, NP);
+    for (int slab = s0; slab < s1; ++slab) {
+      if (!mbar_wait_warp(smem_u32(&full_bar[s]), ph, a.err, 47)) { failed = true; break; }
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bdesc = umma_desc(st + Geo::B_OFF + 32 * kk, 16, 1024, 2);
@@ -383,15 +396,18 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
           }
         }
         tc_commit(smem_u32(&empty_bar[s]));
-        if (++s == SN) { s = 0; ph ^= 1u; }
       }
-      // completes once every MMA above has (or at once, with none issued);
-      // this lane also waits for it, so that no MMA is still running when the
-      // cluster's final barrier lets the CTA free TMEM and leave
-      tc_commit(smem_u32(&accf_bar));
-      mbar_drain(smem_u32(&accf_bar), 0);
-      if (failed) ok_s = 0;
+      __syncwarp();
+      if (++s == SN) { s = 0; ph ^= 1u; }
     }
+    // completes once every MMA above has (or at once, with none issued); the
+    // warp also waits for it, so that no MMA is still running when the
+    // cluster's final barrier lets the CTA free TMEM and leave
+    __syncwarp();
+    if (elect_one()) tc_commit(smem_u32(&accf_bar));
+    __syncwarp();
+    mbar_drain(smem_u32(&accf_bar), 0);
+    if (failed && lane == 0) ok_s = 0;
   }
   bool ok = true;
   if (warp >= 2) {

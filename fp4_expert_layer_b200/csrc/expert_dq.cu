@@ -362,58 +362,64 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       }
     }
   } else if (warp == 1 || warp == 15) {
-    // ---------------- MMA issuers: lane 0 of warp 1 issues the MMAs of the
-    // first accumulator (gate, or the first 128 down rows), lane 0 of warp 15
-    // those of the second; each K slab is 4 MMAs of K = 16 per issuer (a
-    // single issuer spent about as long issuing the 8 MMAs of a slab as the
-    // tensor core took to run them).  Descriptors advance from one computed
-    // up front.
-    if (lane == 0) {
-      const int h = warp == 1 ? 0 : 1;
-      int s = 0, n = 0;
-      uint32_t ph = 0;
-      int q = 0;
-      uint32_t qph = 0;
-      const uint64_t bdesc0 = umma_desc(smem_u32(smem), 16, 1024, 2);
-      while (true) {
-        if (!mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 59)) break;
-        const int item = sched_item[q];
-        const TileInfo ti = sched_ti[q];
-        const int loc = sched_loc[q];
-        mbar_arrive(smem_u32(&sched_empty[q]));
-        if (++q == kDqSched) { q = 0; qph ^= 1u; }
-        if (item < 0) break;
-        if (loc == kLocAbsent) continue;
-        const int N = max(16, (ti.nrows + 15) & ~15);
-        const int buf = n % NBUF;
-        if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 54)) break;
+    // ---------------- MMA issuers: warp 1 issues the MMAs of the first
+    // accumulator (gate, or the first 128 down rows), warp 15 those of the
+    // second; each K slab is 4 MMAs of K = 16 per issuer.  The whole warp runs
+    // the loop (every wait warp-uniform) and one elected lane issues, so that
+    // the descriptors, advanced from ones computed up front, stay in uniform
+    // registers.
+    const int h = warp == 1 ? 0 : 1;
+    int s = 0, n = 0;
+    uint32_t ph = 0;
+    int q = 0;
+    uint32_t qph = 0;
+    const uint64_t bdesc0 = umma_desc(smem_u32(smem), 16, 1024, 2);
+    while (true) {
+      if (!mbar_wait_warp(smem_u32(&sched_full[q]), qph, a.err, 59)) break;
+      // broadcast from lane 0: values the compiler knows to be warp-uniform
+      const int item = __shfl_sync(0xffffffffu, sched_item[q], 0);
+      const int nrows = __shfl_sync(0xffffffffu, sched_ti[q].nrows, 0);
+      const int loc = __shfl_sync(0xffffffffu, sched_loc[q], 0);
+      if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+      if (++q == kDqSched) { q = 0; qph ^= 1u; }
+      if (item < 0) break;
+      if (loc == kLocAbsent) continue;
+      const int N = max(16, (nrows + 15) & ~15);
+      const int buf = n % NBUF;
+      if (n >= NBUF && !mbar_wait_warp(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 54)) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(buf * Geo::ACC_COLS + h * NB);
+      const uint32_t idesc = idesc_16_dq(128, N, kF16);
+      bool failed = false;
+      for (int slab = 0; slab < nslab; ++slab) {
+        if (!mbar_wait_warp(smem_u32(&op_full[s]), ph, a.err, 51) ||
+            !mbar_wait_warp(smem_u32(&b_full[s]), ph, a.err, 50)) {
+          failed = true;
+          break;
+        }
         tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * Geo::ACC_COLS + h * NB);
-        const uint32_t idesc = idesc_16_dq(128, N, kF16);
-        bool failed = false;
-        for (int slab = 0; slab < nslab; ++slab) {
-          if (!mbar_wait(smem_u32(&op_full[s]), ph, a.err, 51) || !mbar_wait(smem_u32(&b_full[s]), ph, a.err, 50)) {
-            failed = true;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t bd = bdesc0 + (uint64_t)(((uint32_t)s * (uint32_t)Geo::OP_STAGE) >> 4);
-          const uint32_t at = tmem + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS + h * 32);
+        const uint64_t bd = bdesc0 + (uint64_t)(((uint32_t)s * (uint32_t)Geo::OP_STAGE) >> 4);
+        const uint32_t at = tmem + (uint32_t)(Geo::A_TMEM + s * Geo::A_COLS + h * 32);
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)                     // K = 16 per MMA (8 TMEM columns of A, 32 B of B)
             umma_bf16_ts(acc, at + (uint32_t)(8 * kk), bd + (uint64_t)(2 * kk), idesc, (slab > 0 || kk > 0) ? 1u : 0u);
           tc_commit(smem_u32(&op_empty[s]));                 // stage free once both issuers' MMAs finish
-          if (++s == SO) { s = 0; ph ^= 1u; }
         }
-        if (failed) break;
-        tc_commit(smem_u32(&accf_bar[buf]));
-        ++n;
+        __syncwarp();
+        if (++s == SO) { s = 0; ph ^= 1u; }
       }
-      // every MMA issued above has completed before the CTA frees TMEM and
-      // leaves (also after a wait gave up and the loop was left early)
-      tc_commit(smem_u32(&quiesce_bar));
-      mbar_drain(smem_u32(&quiesce_bar), 0);
+      if (failed) break;
+      if (elect_one()) tc_commit(smem_u32(&accf_bar[buf]));
+      __syncwarp();
+      ++n;
     }
+    // every MMA issued above has completed before the CTA frees TMEM and
+    // leaves (also after a wait gave up and the loop was left early)
+    __syncwarp();
+    if (elect_one()) tc_commit(smem_u32(&quiesce_bar));
+    __syncwarp();
+    mbar_drain(smem_u32(&quiesce_bar), 0);
   } else if (warp >= 6 && warp < 14) {
     // ---------------- decoders: raw codes + scales -> weight rows in TMEM.
     // Two groups of four warps take alternate slabs (group g the slabs n of
@@ -612,21 +618,33 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
         const float gg = gsc[0], gu = gsc[1];
         const int I = a.rows;
         const int rcol = rb * 128 + 32 * quad + lane;        // h column
+        uint16_t *hcol = a.h_out + (size_t)ti.prow0 * I + rcol;
         for (int c0 = 0; c0 < ntok; c0 += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(acc + (uint32_t)c0, g);
           tmem_ld32(acc + (uint32_t)(NB + c0), u);
           tmem_ld_wait();
           if (!ok) continue;
+          // all 32 columns without a branch (columns past the tile's tokens
+          // hold values of no one and are not stored), so that the dependent
+          // exp / reciprocal chains of different tokens overlap
+          uint32_t hv[16];
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            const int j = c0 + jj;
-            if (j >= ntok) continue;                         // warp-uniform
-            const float ts = kF16 ? tok_gate[j] : 1.0f;   // f16 x rows: their power-of-two scale
-            const float av = __uint_as_float(g[jj]) * (gg * ts);
-            const float uv = __uint_as_float(u[jj]) * (gu * ts);
-            a.h_out[(size_t)(ti.prow0 + j) * I + rcol] = bf16_bits(silu_f(av) * uv);
+          for (int jj = 0; jj < 32; jj += 2) {
+            float hh[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float ts = kF16 ? tok_gate[c0 + jj + e] : 1.0f;   // f16 x rows: their power-of-two scale
+              const float av = __uint_as_float(g[jj + e]) * (gg * ts);
+              const float uv = __uint_as_float(u[jj + e]) * (gu * ts);
+              hh[e] = silu_f(av) * uv;
+            }
+            hv[jj / 2] = (uint32_t)bf16_bits(hh[0]) | ((uint32_t)bf16_bits(hh[1]) << 16);
           }
+          const int nj = min(32, ntok - c0);
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (jj < nj) hcol[(size_t)(c0 + jj) * I] = (uint16_t)(hv[jj / 2] >> (16 * (jj & 1)));
         }
       } else {
         const float gd = gsc[2];
@@ -638,12 +656,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
             tmem_ld32(acc + (uint32_t)(hh * NB + c0), dv);
             tmem_ld_wait();
             if (!ok) continue;
+            const int nj = min(32, ntok - c0);
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
-              const int j = c0 + jj;
-              if (j >= ntok) continue;
-              a.o_out[(size_t)tok_pair[j] * H + orow] = __uint_as_float(dv[jj]) * gd * tok_gate[j];
-            }
+            for (int jj = 0; jj < 32; ++jj)
+              if (jj < nj) a.o_out[(size_t)tok_pair[c0 + jj] * H + orow] = __uint_as_float(dv[jj]) * gd * tok_gate[c0 + jj];
           }
         }
       }

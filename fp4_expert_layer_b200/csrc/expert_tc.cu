@@ -276,68 +276,75 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
       }
     }
   } else if (warp == 1 || warp == 7) {
-    // ---------------- MMA issuers: lane 0 of warp 1 the MMAs of the first
-    // accumulator (gate, or the first 128 down rows), lane 0 of warp 7 those
-    // of the second.  Each copies the scale blocks its MMAs read (its weight
-    // half, and its own copy of the activation block: a tcgen05.cp is ordered
-    // only before the MMAs of the thread that issued it).  Descriptors
-    // advance from ones computed up front.
-    if (lane == 0) {
-      const int h = warp == 1 ? 0 : 1;
-      int s = 0, n = 0;
-      uint32_t ph = 0;
-      int q = 0;
-      uint32_t qph = 0;
-      bool failed = false;
-      const uint32_t sbase = smem_u32(smem);
-      const uint64_t adesc0 = umma_desc(sbase + h * 16384, 16, 1024, 2);
-      const uint64_t bdesc0 = umma_desc(sbase + Geo::B_OFF, 16, 1024, 2);
-      while (!failed) {
-        if (!mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 39)) break;
-        const int item = sched_item[q];
-        const TileInfo ti = sched_ti[q];
-        const int loc = sched_loc[q];
-        mbar_arrive(smem_u32(&sched_empty[q]));
-        if (++q == kSched) { q = 0; qph ^= 1u; }
-        if (item < 0) break;
-        if (loc == kLocAbsent) continue;
-        const int N = max(16, (2 * ti.nrows + 15) & ~15);    // piece rows rounded up to 16
-        const int buf = n % NBUF;
-        // the epilogue must have drained this accumulator buffer
-        if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 34)) break;
-        tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX + h * NBOX);
-        uint32_t idesc[4];
+    // ---------------- MMA issuers: warp 1 the MMAs of the first accumulator
+    // (gate, or the first 128 down rows), warp 7 those of the second.  Each
+    // copies the scale blocks its MMAs read (its weight half, and its own copy
+    // of the activation block: a tcgen05.cp is ordered only before the MMAs of
+    // the thread that issued it).  The whole warp runs the loop (every wait
+    // warp-uniform) and one elected lane issues, so that the descriptors,
+    // advanced from ones computed up front, stay in uniform registers.
+    const int h = warp == 1 ? 0 : 1;
+    int s = 0, n = 0;
+    uint32_t ph = 0;
+    int q = 0;
+    uint32_t qph = 0;
+    bool failed = false;
+    const uint32_t sbase = smem_u32(smem);
+    const uint64_t adesc0 = umma_desc(sbase + h * 16384, 16, 1024, 2);
+    const uint64_t bdesc0 = umma_desc(sbase + Geo::B_OFF, 16, 1024, 2);
+    while (!failed) {
+      if (!mbar_wait_warp(smem_u32(&sched_full[q]), qph, a.err, 39)) break;
+      // broadcast from lane 0: values the compiler knows to be warp-uniform
+      const int item = __shfl_sync(0xffffffffu, sched_item[q], 0);
+      const int nrows = __shfl_sync(0xffffffffu, sched_ti[q].nrows, 0);
+      const int loc = __shfl_sync(0xffffffffu, sched_loc[q], 0);
+      if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+      if (++q == kSched) { q = 0; qph ^= 1u; }
+      if (item < 0) break;
+      if (loc == kLocAbsent) continue;
+      const int N = max(16, (2 * nrows + 15) & ~15);         // piece rows rounded up to 16
+      const int buf = n % NBUF;
+      // the epilogue must have drained this accumulator buffer
+      if (n >= NBUF && !mbar_wait_warp(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 34)) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(buf * 2 * NBOX + h * NBOX);
+      uint32_t idesc[4];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          idesc[kk] = idesc_f8f6f4_block(128, N, kFmtE2M1_f8f6f4, kFmtE4M3, (uint32_t)kk, (uint32_t)kk);
-        for (int slab = 0; slab < nslab; ++slab) {
-          if (!mbar_wait(smem_u32(&full_bar[s]), ph, a.err, 31) ||
-              !mbar_wait(smem_u32(&bfull_bar[s]), ph, a.err, 36)) {
-            failed = true;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t soff = (uint32_t)s * (uint32_t)Geo::STAGE;
-          const uint32_t sf = tmem + (uint32_t)(Geo::SF_COL0 + Geo::SF_PER_STAGE * s + 8 * h);
+      for (int kk = 0; kk < 4; ++kk)
+        idesc[kk] = idesc_f8f6f4_block(128, N, kFmtE2M1_f8f6f4, kFmtE4M3, (uint32_t)kk, (uint32_t)kk);
+      for (int slab = 0; slab < nslab; ++slab) {
+        if (!mbar_wait_warp(smem_u32(&full_bar[s]), ph, a.err, 31) ||
+            !mbar_wait_warp(smem_u32(&bfull_bar[s]), ph, a.err, 36)) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t soff = (uint32_t)s * (uint32_t)Geo::STAGE;
+        const uint32_t sf = tmem + (uint32_t)(Geo::SF_COL0 + Geo::SF_PER_STAGE * s + 8 * h);
+        const uint64_t ad = adesc0 + (uint64_t)(soff >> 4), bd = bdesc0 + (uint64_t)(soff >> 4);
+        if (elect_one()) {
           tc_cp_sf_block(sf, sbase + soff + Geo::SF_OFF + 512 * h);       // this half's weight scales
           tc_cp_sf_block(sf + 4, sbase + soff + Geo::SF_OFF + 1024);      // the activation rows' scales
-          const uint64_t ad = adesc0 + (uint64_t)(soff >> 4), bd = bdesc0 + (uint64_t)(soff >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)                    // K = 32 per MMA
+          for (int kk = 0; kk < 4; ++kk)                  // K = 32 per MMA
             umma_mxf8f6f4(acc, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc[kk], sf | ((uint32_t)kk << 30),
                           (sf + 4) | ((uint32_t)kk << 30), (slab > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(smem_u32(&empty_bar[s]));                // stage free once both issuers' MMAs finish
-          if (++s == S) { s = 0; ph ^= 1u; }
+          tc_commit(smem_u32(&empty_bar[s]));              // stage free once both issuers' MMAs finish
         }
-        tc_commit(smem_u32(&accf_bar[buf]));                 // this item's accumulators complete
-        ++n;
+        __syncwarp();
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
-      // every MMA issued above has completed before the CTA frees TMEM and
-      // leaves (also after a wait gave up and the loop was left early)
-      tc_commit(smem_u32(&quiesce_bar));
-      mbar_drain(smem_u32(&quiesce_bar), 0);
+      if (failed) break;
+      if (elect_one()) tc_commit(smem_u32(&accf_bar[buf]));   // this item's accumulators complete
+      __syncwarp();
+      ++n;
     }
+    // every MMA issued above has completed before the CTA frees TMEM and
+    // leaves (also after a wait gave up and the loop was left early)
+    __syncwarp();
+    if (elect_one()) tc_commit(smem_u32(&quiesce_bar));
+    __syncwarp();
+    mbar_drain(smem_u32(&quiesce_bar), 0);
   } else if (warp == 6) {
     // ---------------- loader (warp 6, one lane): per K slab, the tile's
     // activation-piece rows by TMA (16-row boxes, 128-byte swizzle as the MMA
@@ -490,18 +497,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
           for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) am[jj] = fmaxf(am[jj], __shfl_xor_sync(0xffffffffu, am[jj], o));
+          int e2r[16];
+          uint32_t c2[16];
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
-            const int j = c0 / 2 + jj;
-            if (j >= ntok) continue;                         // warp-uniform
-            const int e2r = split_e2rel(am[jj], e1[jj]);
-            const uint32_t c2 = e4m3x2(w[jj] * exp2_int(-e2r), 0.0f) & 0xFFu;
-            const size_t row = (size_t)act_row0 + 2 * j;
+            e2r[jj] = split_e2rel(am[jj], e1[jj]);
+            c2[jj] = e4m3x2(w[jj] * exp2_int(-e2r[jj]), 0.0f) & 0xFFu;
+          }
+          const int nj = min(16, ntok - c0 / 2);             // warp-uniform
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            if (jj >= nj) break;
+            const size_t row = (size_t)act_row0 + 2 * (c0 / 2 + jj);
             a.hq[row * I + r] = (uint8_t)c1[jj];
-            a.hq[(row + 1) * I + r] = (uint8_t)c2;
+            a.hq[(row + 1) * I + r] = (uint8_t)c2[jj];
             if (lane == 0) {
               a.hsf[sf_offset(nsf_h, (int)row, r / 32)] = (uint8_t)(e1[jj] + 127);
-              a.hsf[sf_offset(nsf_h, (int)row + 1, r / 32)] = (uint8_t)(e1[jj] + e2r + 127);
+              a.hsf[sf_offset(nsf_h, (int)row + 1, r / 32)] = (uint8_t)(e1[jj] + e2r[jj] + 127);
             }
           }
         }
@@ -522,10 +534,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
             tmem_ld32(acc + (uint32_t)(hh * NBOX + c0), d);
             tmem_ld_wait();
             if (!ok) continue;
+            const int nj = min(16, ntok - c0 / 2);
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
+              if (jj >= nj) break;
               const int j = c0 / 2 + jj;
-              if (j >= ntok) continue;
               a.o_out[(size_t)tok_pair[j] * H + r] =
                   (__uint_as_float(d[2 * jj]) + __uint_as_float(d[2 * jj + 1])) * tok_gate[j];
             }

@@ -205,32 +205,35 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer (one lane)
-    if (lane == 0) {
-      int s = 0, n = 0;
-      uint32_t ph = 0;
-      int q = 0;
-      uint32_t qph = 0;
-      while (true) {
-        if (!mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 15)) break;
-        const int item = sched_item[q];
-        const int loc = sched_loc[q];
-        mbar_arrive(smem_u32(&sched_empty[q]));
-        if (++q == kGSched) { q = 0; qph ^= 1u; }
-        if (item < 0) break;
-        if (loc == kLocAbsent) continue;
-        const int buf = n % NBUF;
-        if (n >= NBUF && !mbar_wait(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 16)) break;
+    // ---------------- MMA issuer: the whole warp runs the loop (every wait
+    // warp-uniform) and one elected lane issues the scale copies, the MMAs and
+    // the commits, so that their operands stay in uniform registers
+    int s = 0, n = 0;
+    uint32_t ph = 0;
+    int q = 0;
+    uint32_t qph = 0;
+    while (true) {
+      if (!mbar_wait_warp(smem_u32(&sched_full[q]), qph, a.err, 15)) break;
+      // broadcast from lane 0: values the compiler knows to be warp-uniform
+      const int item = __shfl_sync(0xffffffffu, sched_item[q], 0);
+      const int loc = __shfl_sync(0xffffffffu, sched_loc[q], 0);
+      if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
+      if (++q == kGSched) { q = 0; qph ^= 1u; }
+      if (item < 0) break;
+      if (loc == kLocAbsent) continue;
+      const int buf = n % NBUF;
+      if (n >= NBUF && !mbar_wait_warp(smem_u32(&acce_bar[buf]), ((n / NBUF) - 1) & 1, a.err, 16)) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(buf * 128);
+      bool failed = false;
+      for (int it = 0; it < nk; ++it) {
+        if (!mbar_wait_warp(smem_u32(&full_bar[s]), ph, a.err, 11)) { failed = true; break; }
         tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * 128);
-        bool failed = false;
-        for (int it = 0; it < nk; ++it) {
-          if (!mbar_wait(smem_u32(&full_bar[s]), ph, a.err, 11)) { failed = true; break; }
-          tc_fence_after();
-          const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
-          const uint32_t sf_t = tmem + (uint32_t)(Geo::SF_TMEM + s * Geo::SF_COLS);
-          const int kmma = min(256, K - it * 256) / 64;              // 4, or 2 in a half stage
-          const int nblk = (WF == WF_MX) ? kmma / 2 : kmma;          // valid scale blocks per operand
+        const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+        const uint32_t sf_t = tmem + (uint32_t)(Geo::SF_TMEM + s * Geo::SF_COLS);
+        const int kmma = min(256, K - it * 256) / 64;                // 4, or 2 in a half stage
+        const int nblk = (WF == WF_MX) ? kmma / 2 : kmma;            // valid scale blocks per operand
+        if (elect_one()) {
 #pragma unroll
           for (int mat = 0; mat < 2; ++mat)
             for (int b = 0; b < nblk; ++b)
@@ -250,17 +253,21 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
             else umma_nvf4(acc, adesc, bdesc, idesc, sfa, sfb, accum);
           }
           tc_commit(smem_u32(&empty_bar[s]));                        // stage free once these MMAs finish
-          if (++s == S) { s = 0; ph ^= 1u; }
         }
-        if (failed) break;
-        tc_commit(smem_u32(&accf_bar[buf]));                         // this item's accumulator complete
-        ++n;
+        __syncwarp();
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
-      // every MMA issued above has completed before the CTA frees TMEM and
-      // leaves (also after a wait gave up and the loop was left early)
-      tc_commit(smem_u32(&quiesce_bar));
-      mbar_drain(smem_u32(&quiesce_bar), 0);
+      if (failed) break;
+      if (elect_one()) tc_commit(smem_u32(&accf_bar[buf]));         // this item's accumulator complete
+      __syncwarp();
+      ++n;
     }
+    // every MMA issued above has completed before the CTA frees TMEM and
+    // leaves (also after a wait gave up and the loop was left early)
+    __syncwarp();
+    if (elect_one()) tc_commit(smem_u32(&quiesce_bar));
+    __syncwarp();
+    mbar_drain(smem_u32(&quiesce_bar), 0);
   } else {
     // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31; the
     // warps 2..5 (group 0) take tokens 0..63 of an item, warps 6..9 (group 1)
