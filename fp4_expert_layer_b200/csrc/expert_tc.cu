@@ -144,6 +144,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
   // down epilogue: pair index and gate of each token of the current item
   __shared__ int tok_pair[NBOX / 2];
   __shared__ float tok_gate[NBOX / 2];
+  // per epilogue warp: one chunk of its 32 rows (16 tokens), turned from one
+  // row per lane into token rows so that the stores go out 16 bytes a lane
+  // (gate/up: 32 piece rows x 32 bytes; down: 16 pairs x 32 fp32)
+  __shared__ __align__(16) uint32_t epi_tile[4][16 * 32];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -504,18 +508,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
             e2r[jj] = split_e2rel(am[jj], e1[jj]);
             c2[jj] = e4m3x2(w[jj] * exp2_int(-e2r[jj]), 0.0f) & 0xFFu;
           }
-          const int nj = min(16, ntok - c0 / 2);             // warp-uniform
+          // piece row 2 jj + p of the tile holds this warp's 32 columns
+          uint8_t *tile8 = reinterpret_cast<uint8_t *>(epi_tile[quad]);
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
-            if (jj >= nj) break;
-            const size_t row = (size_t)act_row0 + 2 * (c0 / 2 + jj);
-            a.hq[row * I + r] = (uint8_t)c1[jj];
-            a.hq[(row + 1) * I + r] = (uint8_t)c2[jj];
-            if (lane == 0) {
-              a.hsf[sf_offset(nsf_h, (int)row, r / 32)] = (uint8_t)(e1[jj] + 127);
-              a.hsf[sf_offset(nsf_h, (int)row + 1, r / 32)] = (uint8_t)(e1[jj] + e2r[jj] + 127);
+            tile8[(2 * jj) * 32 + lane] = (uint8_t)c1[jj];
+            tile8[(2 * jj + 1) * 32 + lane] = (uint8_t)c2[jj];
+          }
+          __syncwarp();
+          const int nj = min(16, ntok - c0 / 2);             // warp-uniform
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {                      // 16 piece rows per pass, 2 lanes a row
+            const int pr = (lane >> 1) + 16 * i;
+            if (pr < 2 * nj)
+              *reinterpret_cast<uint4 *>(a.hq + ((size_t)act_row0 + c0 + pr) * I + (r - lane) + 16 * (lane & 1)) =
+                  *reinterpret_cast<const uint4 *>(tile8 + pr * 32 + 16 * (lane & 1));
+          }
+          if (lane == 0) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              if (jj >= nj) break;
+              const int row = act_row0 + c0 + 2 * jj;
+              a.hsf[sf_offset(nsf_h, row, r / 32)] = (uint8_t)(e1[jj] + 127);
+              a.hsf[sf_offset(nsf_h, row + 1, r / 32)] = (uint8_t)(e1[jj] + e2r[jj] + 127);
             }
           }
+          __syncwarp();                                      // the tile is rewritten by the next chunk
         }
         tc_fence_before();
         __syncwarp();
@@ -534,14 +552,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
             tmem_ld32(acc + (uint32_t)(hh * NBOX + c0), d);
             tmem_ld_wait();
             if (!ok) continue;
+            // pair row jj of the tile holds this warp's 32 output values of
+            // that pair (column index rotated by the row against bank conflicts)
+            uint32_t *tile = epi_tile[quad];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              tile[jj * 32 + ((lane + jj) & 31)] = __float_as_uint(
+                  (__uint_as_float(d[2 * jj]) + __uint_as_float(d[2 * jj + 1])) * tok_gate[c0 / 2 + jj]);
+            __syncwarp();
             const int nj = min(16, ntok - c0 / 2);
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              if (jj >= nj) break;
-              const int j = c0 / 2 + jj;
-              a.o_out[(size_t)tok_pair[j] * H + r] =
-                  (__uint_as_float(d[2 * jj]) + __uint_as_float(d[2 * jj + 1])) * tok_gate[j];
+            for (int i = 0; i < 4; ++i) {                    // 4 pair rows per pass, 8 lanes a row
+              const int pr = (lane >> 3) + 4 * i;
+              if (pr < nj) {
+                const int c = 4 * (lane & 7);
+                float4 v;
+                v.x = __uint_as_float(tile[pr * 32 + ((c + 0 + pr) & 31)]);
+                v.y = __uint_as_float(tile[pr * 32 + ((c + 1 + pr) & 31)]);
+                v.z = __uint_as_float(tile[pr * 32 + ((c + 2 + pr) & 31)]);
+                v.w = __uint_as_float(tile[pr * 32 + ((c + 3 + pr) & 31)]);
+                *reinterpret_cast<float4 *>(a.o_out + (size_t)tok_pair[c0 / 2 + pr] * H + (r - lane) + c) = v;
+              }
             }
+            __syncwarp();                                    // the tile is rewritten by the next chunk
           }
         }
         tc_fence_before();
