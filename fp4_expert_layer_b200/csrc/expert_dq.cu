@@ -6,8 +6,8 @@
 // block-scaled MMA kinds cannot take an NVFP4 weight against a 16-bit
 // activation: kind::mxf4nvf4 (the one that reads E4M3 block scales) wants
 // FP4 on both sides, and kind::mxf8f6f4 takes only UE8M0 per-32 scales.  So
-// each weight tile is decoded ONCE per token tile into shared memory as bf16
-// and multiplied with tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM):
+// each weight tile is decoded ONCE per token tile into TMEM as bf16 (f16 for
+// the gate/up pass) and multiplied with tcgen05.mma kind::f16 (fp32 in TMEM):
 //   * an E2M1 value (at most 2 significant bits) times its E4M3 block scale
 //     (4 significant bits, 2^-9 .. 448) has at most 6 significant bits and lies
 //     in [2^-10, 2688]: exact in f16 and in bf16;
@@ -32,16 +32,20 @@
 //                codes (32 bytes x 128 or 256 rows) per matrix and the
 //                512-byte E4M3 scale-factor blocks by bulk copy, into a ring
 //                of raw stages;
-//   warps 1, 15  MMA issuers (one lane each, one accumulator each: gate and
-//                up, or the two 128-row halves of down): M = 128, N = tokens
-//                rounded up to 16, K = 16, A from TMEM, B from shared memory;
+//   warps 1, 15  MMA issuers (whole warps, one elected lane issuing; one
+//                accumulator each: gate and up, or the two 128-row halves of
+//                down): M = 128, N = tokens rounded up to 16, K = 16, A from
+//                TMEM, B from shared memory;
 //   warps 2..5   epilogue: TMEM -> SwiGLU -> h (bf16, padded-row order), or
-//                G_d * gate * acc -> O' (fp32, pair order);
+//                G_d * gate * acc -> O' (fp32, pair order), each warp's
+//                32 x 32 chunk turned into token rows in shared memory and
+//                stored 16 bytes a lane;
 //   warps 6..13  decoders: raw stage -> weight rows in TMEM, in two groups
 //                of four warps taking alternate slabs (warp w the rows of TMEM
 //                lane quadrant w % 4 of both 128-row halves; NVFP4: hardware
 //                E2M1 -> f16x2 and an f16 multiply by the scale, widened to
-//                bf16 for the down pass);
+//                bf16 for the down pass); every warp on every slab, one row a
+//                thread, was slower (all eight then wait on the same stages);
 //   warp 14      activation loader: the tile's 16-bit rows of this K slab
 //                (x rows gathered into the padded expert order beforehand,
 //                or h) by TMA in 64-row boxes, 128-byte swizzled K-major as
@@ -99,15 +103,16 @@ struct DqGeom {
   static constexpr int TMEM_COLS = 512;
   static constexpr int RAW_OFF = OP_STAGES * OP_STAGE;
   static constexpr int RAW_BYTES = DqRaw<F>::BYTES;
-  // raw stages in what is left of 227 KB (1 KB alignment slack, 4 KB for the static part)
-  static constexpr int RAW_FIT = (227 * 1024 - 1024 - 4096 - RAW_OFF) / RAW_BYTES;
+  // raw stages in what is left of 227 KB (1 KB alignment slack, 20 KB for the
+  // static part: the epilogue's transpose tiles and the hand-over slots)
+  static constexpr int RAW_FIT = (227 * 1024 - 1024 - 20 * 1024 - RAW_OFF) / RAW_BYTES;
   static constexpr int RAW_STAGES = RAW_FIT < 12 ? RAW_FIT : 12;
   static constexpr size_t SMEM = (size_t)RAW_OFF + (size_t)RAW_STAGES * RAW_BYTES + 1024;
   static_assert(OP_STAGE % 1024 == 0, "operand stages must keep the 1024-byte swizzle alignment");
   static_assert(RAW_BYTES % 512 == 0, "raw stages keep 128-byte TMA destinations");
   static_assert(RAW_STAGES >= 3, "raw ring depth");
   static_assert(A_TMEM + OP_STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
-  static_assert(SMEM <= 227 * 1024, "shared-memory budget");
+  static_assert(SMEM + 20 * 1024 <= 227 * 1024, "shared-memory budget");
 };
 
 // kind::f16 instruction descriptor: fp32 accumulator, A and B both f16 or
@@ -247,6 +252,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
   __shared__ int sched_loc[kDqSched];
   __shared__ int tok_pair[NB];
   __shared__ float tok_gate[NB];
+  // per epilogue warp: its 32 rows x 32 tokens of a chunk, turned from one
+  // row per lane into token rows so that the stores go out 16 bytes a lane
+  __shared__ __align__(16) uint32_t epi_tile[4][32 * 32];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dq_smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -617,8 +625,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
       if constexpr (MODE == MODE_GATEUP) {
         const float gg = gsc[0], gu = gsc[1];
         const int I = a.rows;
-        const int rcol = rb * 128 + 32 * quad + lane;        // h column
-        uint16_t *hcol = a.h_out + (size_t)ti.prow0 * I + rcol;
+        uint32_t *tile = epi_tile[quad];
+        uint16_t *tile16 = reinterpret_cast<uint16_t *>(tile);
+        const int hcol0 = rb * 128 + 32 * quad;              // first h column of this warp
         for (int c0 = 0; c0 < ntok; c0 += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(acc + (uint32_t)c0, g);
@@ -641,25 +650,56 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
             }
             hv[jj / 2] = (uint32_t)bf16_bits(hh[0]) | ((uint32_t)bf16_bits(hh[1]) << 16);
           }
+          // token row jj of the tile holds this warp's 32 h columns (64 bytes)
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) tile16[jj * 32 + lane] = (uint16_t)(hv[jj / 2] >> (16 * (jj & 1)));
+          __syncwarp();
           const int nj = min(32, ntok - c0);
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj)
-            if (jj < nj) hcol[(size_t)(c0 + jj) * I] = (uint16_t)(hv[jj / 2] >> (16 * (jj & 1)));
+          for (int i = 0; i < 4; ++i) {                      // 8 token rows per pass, 4 lanes a row
+            const int r = (lane >> 2) + 8 * i;
+            if (r < nj)
+              *reinterpret_cast<uint4 *>(a.h_out + (size_t)(ti.prow0 + c0 + r) * I + hcol0 + 8 * (lane & 3)) =
+                  *reinterpret_cast<const uint4 *>(tile16 + r * 32 + 8 * (lane & 3));
+          }
+          __syncwarp();                                      // the tile is rewritten by the next chunk
         }
       } else {
         const float gd = gsc[2];
         const int H = a.rows;
+        uint32_t *tile = epi_tile[quad];
         for (int hh = 0; hh < 2; ++hh) {
-          const int orow = rb * 256 + hh * 128 + 32 * quad + lane;
+          const int orow0 = rb * 256 + hh * 128 + 32 * quad;  // first output row of this warp
           for (int c0 = 0; c0 < ntok; c0 += 32) {
             uint32_t dv[32];
             tmem_ld32(acc + (uint32_t)(hh * NB + c0), dv);
             tmem_ld_wait();
             if (!ok) continue;
-            const int nj = min(32, ntok - c0);
+            // token row jj of the tile holds this warp's 32 output values of
+            // that pair (the column index is rotated by the row against bank
+            // conflicts)
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
-              if (jj < nj) a.o_out[(size_t)tok_pair[c0 + jj] * H + orow] = __uint_as_float(dv[jj]) * gd * tok_gate[c0 + jj];
+              tile[jj * 32 + ((lane + jj) & 31)] = __float_as_uint(__uint_as_float(dv[jj]) * gd * tok_gate[c0 + jj]);
+            __syncwarp();
+            const int nj = min(32, ntok - c0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {                    // 4 pair rows per pass, 8 lanes a row
+#pragma unroll
+              for (int i2 = 0; i2 < 2; ++i2) {
+                const int r = (lane >> 3) + 4 * (2 * i + i2);
+                if (r < nj) {
+                  const int c = 4 * (lane & 7);
+                  float4 v;
+                  v.x = __uint_as_float(tile[r * 32 + ((c + 0 + r) & 31)]);
+                  v.y = __uint_as_float(tile[r * 32 + ((c + 1 + r) & 31)]);
+                  v.z = __uint_as_float(tile[r * 32 + ((c + 2 + r) & 31)]);
+                  v.w = __uint_as_float(tile[r * 32 + ((c + 3 + r) & 31)]);
+                  *reinterpret_cast<float4 *>(a.o_out + (size_t)tok_pair[c0 + r] * H + orow0 + c) = v;
+                }
+              }
+            }
+            __syncwarp();                                    // the tile is rewritten by the next chunk
           }
         }
       }
