@@ -1339,9 +1339,13 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   const bool x16 = (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
   if (dq_only(&c) && !x16) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned for INT4 / FP8 experts");
   const bool dq = L->nv && (dq_only(&c) || P > 12 * act_est) && x16;
-  // 128-token tiles once experts average more than 64 tokens: an MMA issue
-  // costs about as much as an N = 128 MMA runs, so N = 64 tiles halve the rate
-  const int nb_dq = avg > 64 ? 128 : 64;
+  // 128-token tiles once experts average more than 16 tokens: a weight slab
+  // decoded into TMEM then serves twice the tokens, and the pass is bound by
+  // the bytes each SM pulls through L2 per MMA (measured on the
+  // Qwen3.8-Flash-Next-like layer: at 40 tokens per expert, gate/up 0.98 ms
+  // with 64-token tiles, 0.74 ms with 128); 64-token tiles (two accumulator
+  // buffers) for decode-sized batches, where an expert's rows fit one tile
+  const int nb_dq = avg > 16 ? 128 : 64;
   const int ts = a4 ? 128 : (tc ? nbox / 2 : (dq ? nb_dq : 8 * nt));
   const int grid_tiles = P / ts + act_est + 1;
   // routing targets (experts, then sinks) and logit rows (+ the shared-expert gate)
