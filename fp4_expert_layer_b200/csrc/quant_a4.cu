@@ -45,9 +45,41 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
-__device__ __forceinline__ float load_elem(const QuantArgs &q, int token, int row, int k) {
-  if (q.src_bf16) return bf16_bits_to_float(q.src_bf16[(size_t)token * q.K + k]);
-  return q.src_f32[(size_t)row * q.K + k];
+// The N source values k0 .. k0 + N - 1 of a row (token `src` of x, or row `row`
+// of h; zeros for a pad row): 16-byte loads when the source allows them (h
+// always, x when its base is 16-byte aligned), else one element at a time.
+template <int N>
+__device__ __forceinline__ void load_block(const QuantArgs &q, int src, int row, int k0, bool vec, float (&v)[N]) {
+  if (src < 0) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = 0.0f;
+    return;
+  }
+  if (q.src_bf16) {
+    const uint16_t *p = q.src_bf16 + (size_t)src * q.K + k0;
+    if (vec) {
+#pragma unroll
+      for (int c = 0; c < N / 8; ++c) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p) + c);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[8 * c + 2 * j] = __uint_as_float(w[j] << 16);
+          v[8 * c + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < N; ++i) v[i] = bf16_bits_to_float(p[i]);
+    }
+  } else {
+    const float4 *p = reinterpret_cast<const float4 *>(q.src_f32 + (size_t)row * q.K + k0);
+#pragma unroll
+    for (int c = 0; c < N / 4; ++c) {
+      const float4 f = __ldg(p + c);
+      v[4 * c] = f.x; v[4 * c + 1] = f.y; v[4 * c + 2] = f.z; v[4 * c + 3] = f.w;
+    }
+  }
 }
 
 }  // namespace
@@ -69,17 +101,16 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const QuantArgs q) {
     }
   }
   uint8_t *codes = q.codes + (size_t)row * (K / 2);
+  const bool vec = q.src_f32 != nullptr || (reinterpret_cast<uintptr_t>(q.src_bf16) & 15u) == 0;
 
   if (q.fmt == MOE_FMT_MXFP4) {
     const int nsf = K / 32;
     for (int b = lane; b < nsf; b += 32) {
       float v[32];
+      load_block<32>(q, src, row, b * 32, vec, v);
       float amax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        v[i] = src >= 0 ? load_elem(q, src, row, b * 32 + i) : 0.0f;
-        amax = fmaxf(amax, fabsf(v[i]));
-      }
+      for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
       int code = 1;
       if (amax > 0.0f) {
         const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF);
@@ -101,9 +132,29 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const QuantArgs q) {
     }
   } else {
     const int nsf = K / 16;
+    // row maximum: 16-byte loads spread over the lanes (the block pass below
+    // reads the same bytes again, from L1)
     float amax = 0.0f;
-    if (src >= 0)
-      for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(load_elem(q, src, row, k)));
+    if (src >= 0) {
+      if (q.src_f32) {
+        const float4 *p = reinterpret_cast<const float4 *>(q.src_f32 + (size_t)row * K);
+        for (int i = lane; i < K / 4; i += 32) {
+          const float4 f = __ldg(p + i);
+          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
+        }
+      } else if (vec) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(q.src_bf16 + (size_t)src * K);
+        for (int i = lane; i < K / 8; i += 32) {
+          const uint4 u = __ldg(p + i);
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[j] << 16)), fabsf(__uint_as_float(w[j] & 0xFFFF0000u))));
+        }
+      } else {
+        for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(bf16_bits_to_float(q.src_bf16[(size_t)src * K + k])));
+      }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     float G = 1.0f;
@@ -117,12 +168,10 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const QuantArgs q) {
     if (lane == 0) q.G[row] = G;
     for (int b = lane; b < nsf; b += 32) {
       float v[16];
+      load_block<16>(q, src, row, b * 16, vec, v);
       float bmax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        v[i] = src >= 0 ? load_elem(q, src, row, b * 16 + i) : 0.0f;
-        bmax = fmaxf(bmax, fabsf(v[i]));
-      }
+      for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
       const float t = __fdiv_rn(__fdiv_rn(bmax, 6.0f), G);
       const uint32_t sc = e4m3_from_f32(t);
       uint32_t w[2] = {0u, 0u};
