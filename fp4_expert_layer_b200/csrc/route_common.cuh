@@ -85,12 +85,14 @@ __device__ __forceinline__ void topk_warp(const float (&lv)[KPER], int E, int k,
 // ---------------------------------------------------------------------------
 // Permutation: stable counting sort of pair index p = t*k + j by expert, as a
 // block-level routine (NTH threads, `sm` = shared scratch of
-// (5E + 3 + (NTH/32)*E) ints).  Counts by shared-memory atomics, offsets /
-// padded offsets / tile offsets by one block scan, then pairs are placed in
-// chunks of NTH: ranks inside a chunk come from warp match plus per-warp counts
-// scanned in warp order, so equal experts keep ascending p (stable).  The
-// expert ids are read from global memory (IDS_GLOBAL, another CTA wrote them)
-// or from this CTA's shared memory.
+// (5E + 3 + (NTH/32)*E) ints).  Each warp owns one contiguous range of pairs:
+// per-warp counts by shared-memory atomics, then per target the start of each
+// warp's run (warp order), offsets / padded offsets / tile offsets by one
+// block scan, and each warp places its range in order, 32 pairs at a time
+// (ranks inside a group from warp match, a per-warp cursor per target across
+// groups), so equal experts keep ascending p (stable).  The expert ids are
+// read from global memory (IDS_GLOBAL, another CTA wrote them) or from this
+// CTA's shared memory.
 // ---------------------------------------------------------------------------
 template <int NTH, bool IDS_GLOBAL>
 __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
@@ -105,13 +107,28 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
   int *wcnt = toff + E + 1;       // [W][E]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  for (int i = tid; i < E; i += NTH) { cnt[i] = 0; cursor[i] = 0; }
+  (void)cursor;
   if (a.work_ctr && tid < kWorkCtrs) a.work_ctr[tid] = 0;
   for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;
   __syncthreads();
-  for (int p = tid; p < a.n_pairs; p += NTH) {
+  // warp w owns pairs [p0, p1): its own count per target
+  const int span = (a.n_pairs + W - 1) / W;
+  const int p0 = min(a.n_pairs, warp * span), p1 = min(a.n_pairs, p0 + span);
+  for (int p = p0 + lane; p < p1; p += 32) {
     const int e = load_id<IDS_GLOBAL>(ids, p);
-    if (dcheck(e >= 0 && e < E, a.db.err, kChkTarget)) atomicAdd(&cnt[e], 1);
+    if (dcheck(e >= 0 && e < E, a.db.err, kChkTarget)) atomicAdd(&wcnt[warp * E + e], 1);
+  }
+  __syncthreads();
+  // per target: its count, and each warp's count replaced by the start of
+  // its run among the target's pairs (exclusive, in warp order)
+  for (int e = tid; e < E; e += NTH) {
+    int run = 0;
+    for (int w = 0; w < W; ++w) {
+      const int c = wcnt[w * E + e];
+      wcnt[w * E + e] = run;
+      run += c;
+    }
+    cnt[e] = run;
   }
   __syncthreads();
 
@@ -194,27 +211,18 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
   }
 
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < a.n_pairs; base += NTH) {
-    const int p = base + tid;
-    int e = p < a.n_pairs ? load_id<IDS_GLOBAL>(ids, p) : -1;
+  for (int base = p0; base < p1; base += 32) {
+    const int p = base + lane;
+    int e = p < p1 ? load_id<IDS_GLOBAL>(ids, p) : -1;
     if (kCheckedBuild && (e < 0 || e >= E)) e = -1;   // recorded by the count above
     const bool valid = e >= 0;
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & lt_mask);
-    if (valid && rank == 0) wcnt[warp * E + e] = __popc(peers);
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += NTH) {
-      int run = cursor[ee];
-      for (int w = 0; w < W; ++w) {
-        const int c = wcnt[w * E + ee];
-        wcnt[w * E + ee] = run;
-        run += c;
-      }
-      cursor[ee] = run;
-    }
-    __syncthreads();
+    const int local = valid ? wcnt[warp * E + e] + rank : 0;   // index among the target's pairs
+    __syncwarp();
+    if (valid && rank == 0) wcnt[warp * E + e] += __popc(peers);
+    __syncwarp();
     if (valid) {
-      const int local = wcnt[warp * E + e] + rank;
       const int pos = off[e] + local;
       a.perm[pos] = p;
       a.inv[p] = pos;
@@ -224,9 +232,6 @@ __device__ void permute_block(const PermArgs &a, const int *ids, int *sm) {
         a.prow_pair[prow] = p;
       }
     }
-    __syncthreads();
-    for (int i = tid; i < W * E; i += NTH) wcnt[i] = 0;
-    __syncthreads();
   }
 }
 
