@@ -221,39 +221,51 @@ __global__ void combine_kernel(const CombineArgs a) {
 
 // ---------------------------------------------------------------------------
 // Router logits for prefill-sized batches: a register-tiled fp32 GEMM on the
-// CUDA cores.  CTA tile 128 tokens x 64 experts, K in chunks of 32 staged in
-// shared memory (x converted from bf16, both operands transposed to [k][.]),
-// each thread 8 tokens x 4 experts.  Each chunk's 32 products are summed into
-// a chunk partial that is then added to the running sum (two-level summation:
-// the fp32 rounding of H = 4096 sequential additions would otherwise approach
-// the 1e-5 the logits are held to).  With few tiles (small T or E) the K range
-// is split over gridDim.z CTAs that write partial logits to a workspace; the
-// top-k kernel adds the parts in split order (deterministic, no atomics).
+// CUDA cores.  CTA tile 128 tokens x 16 JN experts, K in chunks of 32 staged
+// in shared memory (x converted from bf16, both operands transposed to
+// [k][.], double-buffered, the next chunk's global loads in flight during this
+// one's 32 k steps), each thread 8 tokens x JN experts (tokens 4 ty .. +3 and
+// 64 + 4 ty .. +3, experts 4 tx .. +3 and, for JN = 8, 64 + 4 tx .. +3, so that
+// the 16-byte shared loads of a quarter warp fall in distinct banks).  Each
+// chunk's 32 products are summed into a chunk partial that is then added to
+// the running sum (two-level summation: the fp32 rounding of H = 4096
+// sequential additions would otherwise approach the 1e-5 the logits are held
+// to).  With few tiles (small T or E) the K range is split over gridDim.z
+// CTAs that write partial logits to a workspace; the top-k kernel adds the
+// parts in split order (deterministic, no atomics).
 // ---------------------------------------------------------------------------
 namespace {
-constexpr int kRgT = 128, kRgE = 64, kRgK = 32;
+constexpr int kRgT = 128, kRgK = 32;
+template <int JN>
+constexpr size_t router_gemm_smem() { return (size_t)2 * kRgK * (kRgT + 16 * JN) * sizeof(float); }
 }
 
-__global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__restrict__ x, const float *__restrict__ w,
-                                                          const float *__restrict__ bias, int T, int H, int E,
-                                                          float *__restrict__ logits, float *__restrict__ parts) {
-  __shared__ __align__(16) float xs[2][kRgK][kRgT];
-  __shared__ __align__(16) float ws[2][kRgK][kRgE];
+template <int JN>
+__global__ void __launch_bounds__(256, 1) router_gemm_kernel(const uint16_t *__restrict__ x,
+                                                             const float *__restrict__ w,
+                                                             const float *__restrict__ bias, int T, int H, int E,
+                                                             float *__restrict__ logits, float *__restrict__ parts) {
+  constexpr int TE = 16 * JN;                           // experts per CTA
+  constexpr int WPR = 256 / TE;                         // loader threads per expert row
+  constexpr int WF4 = kRgK / WPR / 4;                   // float4 per loader thread
+  extern __shared__ __align__(16) float rg_smem[];
+  float (*xs)[kRgK][kRgT] = reinterpret_cast<float (*)[kRgK][kRgT]>(rg_smem);
+  float (*ws)[kRgK][TE] = reinterpret_cast<float (*)[kRgK][TE]>(rg_smem + 2 * kRgK * kRgT);
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;               // experts 4*tx.., tokens 8*ty..
-  const int t0 = blockIdx.x * kRgT, e0 = blockIdx.y * kRgE;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int t0 = blockIdx.x * kRgT, e0 = blockIdx.y * TE;
   const int nsplit = gridDim.z;
   const int ck0 = (int)((long)(H / kRgK) * blockIdx.z / nsplit);
   const int ck1 = (int)((long)(H / kRgK) * (blockIdx.z + 1) / nsplit);
   const int nck = ck1 - ck0;
-  // loader roles: x: token tid/2, 16 elements from (tid%2)*16; w: expert tid/4, 8 from (tid%4)*8
+  // loader roles: x token tid/2, 16 elements from (tid%2)*16; w expert tid/WPR, 4 WF4 from (tid%WPR)*4 WF4
   const int lt = tid >> 1, lk = (tid & 1) * 16;
-  const int le = tid >> 2, lkw = (tid & 3) * 8;
+  const int le = tid / WPR, lkw = (tid % WPR) * 4 * WF4;
   const bool xok = t0 + lt < T, wok = e0 + le < E;
   const uint16_t *xrow = x + (size_t)(t0 + lt) * H + lk;
   const float *wrow = w + (size_t)(e0 + le) * H + lkw;
   uint4 xr0, xr1;
-  float4 wr0, wr1;
+  float4 wr[WF4];
   auto fetch = [&](int c) {
     const int k0 = (ck0 + c) * kRgK;
     if (xok) {
@@ -262,12 +274,9 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
     } else {
       xr0 = xr1 = make_uint4(0u, 0u, 0u, 0u);
     }
-    if (wok) {
-      wr0 = __ldg(reinterpret_cast<const float4 *>(wrow + k0));
-      wr1 = __ldg(reinterpret_cast<const float4 *>(wrow + k0 + 4));
-    } else {
-      wr0 = wr1 = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+#pragma unroll
+    for (int q = 0; q < WF4; ++q)
+      wr[q] = wok ? __ldg(reinterpret_cast<const float4 *>(wrow + k0) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
   };
   auto stash = [&](int b) {
     const uint32_t xv[8] = {xr0.x, xr0.y, xr0.z, xr0.w, xr1.x, xr1.y, xr1.z, xr1.w};
@@ -276,52 +285,61 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
       xs[b][lk + 2 * i][lt] = __uint_as_float(xv[i] << 16);
       xs[b][lk + 2 * i + 1][lt] = __uint_as_float(xv[i] & 0xFFFF0000u);
     }
-    const float wv[8] = {wr0.x, wr0.y, wr0.z, wr0.w, wr1.x, wr1.y, wr1.z, wr1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) ws[b][lkw + i][le] = wv[i];
+    for (int q = 0; q < WF4; ++q) {
+      ws[b][lkw + 4 * q + 0][le] = wr[q].x;
+      ws[b][lkw + 4 * q + 1][le] = wr[q].y;
+      ws[b][lkw + 4 * q + 2][le] = wr[q].z;
+      ws[b][lkw + 4 * q + 3][le] = wr[q].w;
+    }
   };
-  float acc[8][4];
+  float acc[8][JN];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < JN; ++j) acc[i][j] = 0.0f;
   fetch(0);
   stash(0);
   __syncthreads();
   for (int c = 0; c < nck; ++c) {
     const int b = c & 1;
     if (c + 1 < nck) fetch(c + 1);
-    float part[8][4];
+    float part[8][JN];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) part[i][j] = 0.0f;
-#pragma unroll 8
+      for (int j = 0; j < JN; ++j) part[i][j] = 0.0f;
+#pragma unroll 4
     for (int k = 0; k < kRgK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4 *>(&xs[b][k][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4 *>(&xs[b][k][ty * 8 + 4]);
-      const float4 bw = *reinterpret_cast<const float4 *>(&ws[b][k][tx * 4]);
+      const float4 a0 = *reinterpret_cast<const float4 *>(&xs[b][k][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&xs[b][k][64 + ty * 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[4] = {bw.x, bw.y, bw.z, bw.w};
+      float bv[JN];
+      const float4 b0 = *reinterpret_cast<const float4 *>(&ws[b][k][tx * 4]);
+      bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w;
+      if constexpr (JN == 8) {
+        const float4 b1 = *reinterpret_cast<const float4 *>(&ws[b][k][64 + tx * 4]);
+        bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
+        for (int j = 0; j < JN; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
+      for (int j = 0; j < JN; ++j) acc[i][j] += part[i][j];
     if (c + 1 < nck) stash(b ^ 1);
     __syncthreads();
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int t = t0 + ty * 8 + i;
+    const int t = t0 + ty * 4 + (i & 3) + 64 * (i >> 2);
     if (t >= T) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
+    for (int j = 0; j < JN; ++j) {
+      const int e = e0 + tx * 4 + (j & 3) + 64 * (j >> 2);
       if (e >= E) continue;
       if (nsplit == 1) logits[(size_t)t * E + e] = acc[i][j] + (bias ? bias[e] : 0.0f);
       else parts[((size_t)blockIdx.z * T + t) * E + e] = acc[i][j];
@@ -329,8 +347,11 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *__rest
   }
 }
 
+static int router_gemm_te(int E) { return E <= 64 ? 64 : 128; }
+
 int router_gemm_splits(int T, int H, int E, size_t part_floats) {
-  const int tiles = ((T + kRgT - 1) / kRgT) * ((E + kRgE - 1) / kRgE);
+  const int te = router_gemm_te(E);
+  const int tiles = ((T + kRgT - 1) / kRgT) * ((E + te - 1) / te);
   int sp = 1;
   while (sp < 8 && tiles * sp < 2 * 148 && (H / kRgK) / (sp * 2) >= 4 &&
          (size_t)(sp * 2) * T * E <= part_floats)
@@ -338,10 +359,19 @@ int router_gemm_splits(int T, int H, int E, size_t part_floats) {
   return sp;
 }
 
+template <int JN>
+static void launch_router_gemm_jn(const uint16_t *x, const float *w, const float *bias, int T, int H, int E,
+                                  float *logits, float *parts, int splits, cudaStream_t s) {
+  constexpr size_t smem = router_gemm_smem<JN>();
+  cudaFuncSetAttribute(router_gemm_kernel<JN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid((T + kRgT - 1) / kRgT, (E + 16 * JN - 1) / (16 * JN), splits);
+  router_gemm_kernel<JN><<<grid, 256, smem, s>>>(x, w, bias, T, H, E, logits, parts);
+}
+
 void launch_router_gemm(const uint16_t *x, const float *w, const float *bias, int T, int H, int E, float *logits,
                         float *parts, int splits, cudaStream_t s) {
-  dim3 grid((T + kRgT - 1) / kRgT, (E + kRgE - 1) / kRgE, splits);
-  router_gemm_kernel<<<grid, 256, 0, s>>>(x, w, bias, T, H, E, logits, parts);
+  if (router_gemm_te(E) == 64) launch_router_gemm_jn<4>(x, w, bias, T, H, E, logits, parts, splits, s);
+  else launch_router_gemm_jn<8>(x, w, bias, T, H, E, logits, parts, splits, s);
 }
 
 // Top-k of tokens whose logits are in memory: warp per token.
