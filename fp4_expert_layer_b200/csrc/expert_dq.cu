@@ -296,39 +296,47 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
   const uint32_t tmem = tmem_base_s;
 
   if (warp == 0) {
-    // ---------------- producer (one lane): work items and the raw weight stream
-    if (lane == 0) {
-      int r = 0, issued = 0;
-      uint32_t ph = 0;
-      int q = 0;
-      uint32_t qph = 0;
-      bool failed = false;
-      for (int j = 0; !failed; ++j) {
-        const int item = atomicAdd(a.work_ctr, 1);
-        TileInfo ti{};
-        int loc = kLocAbsent;
-        if (item < n_items) {
-          ti = load_tile_dq(a.tiles + item / ipt);
-          loc = load_loc(a.loc, ti.expert, a.db);
-        }
-        if (j >= kDqSched && !mbar_wait(smem_u32(&sched_empty[q]), qph ^ 1u, a.err, 58)) { failed = true; break; }
-        const bool done = item >= n_items;
+    // ---------------- producer: work items and the raw weight stream.  The
+    // whole warp runs the loop (warp-uniform waits, values broadcast from lane
+    // 0) and one elected lane issues the copies: a copy issued from a one-lane
+    // loop behind a lane test costs about twice as much.
+    int r = 0, issued = 0;
+    uint32_t ph = 0;
+    int q = 0;
+    uint32_t qph = 0;
+    bool failed = false;
+    for (int j = 0; !failed; ++j) {
+      int item = 0;
+      if (lane == 0) item = atomicAdd(a.work_ctr, 1);
+      item = __shfl_sync(0xffffffffu, item, 0);
+      TileInfo ti{};
+      int loc = kLocAbsent;
+      if (item < n_items) {
+        ti = load_tile_dq(a.tiles + item / ipt);
+        loc = load_loc(a.loc, ti.expert, a.db);
+      }
+      if (j >= kDqSched && !mbar_wait_warp(smem_u32(&sched_empty[q]), qph ^ 1u, a.err, 58)) { failed = true; break; }
+      const bool done = item >= n_items;
+      if (lane == 0) {
         sched_item[q] = done ? -1 : item;
         sched_ti[q] = ti;
         sched_loc[q] = loc;
         mbar_arrive(smem_u32(&sched_full[q]));
-        if (++q == kDqSched) { q = 0; qph ^= 1u; }
-        if (done) break;
-        if (loc == kLocAbsent) continue;
-        const int rb = item % ipt;
-        const bool in_slot = loc >= 0;
-        const int bidx = in_slot ? loc : (-2 - loc);
-        const uint8_t *blob = (in_slot ? a.slots : a.staging) + (size_t)bidx * a.blob_bytes;
-        const CUtensorMap *maps = in_slot ? a.maps.slot : a.maps.stage;
-        for (int slab = 0; slab < nslab; ++slab) {
-          if (issued >= SR && !mbar_wait(smem_u32(&raw_empty[r]), ph ^ 1u, a.err, 52)) { failed = true; break; }
-          const uint32_t bar = smem_u32(&raw_full[r]);
-          const uint32_t st = smem_u32(smem + Geo::RAW_OFF + (size_t)r * kRawBytes);
+      }
+      __syncwarp();
+      if (++q == kDqSched) { q = 0; qph ^= 1u; }
+      if (done) break;
+      if (loc == kLocAbsent) continue;
+      const int rb = item % ipt;
+      const bool in_slot = loc >= 0;
+      const int bidx = in_slot ? loc : (-2 - loc);
+      const uint8_t *blob = (in_slot ? a.slots : a.staging) + (size_t)bidx * a.blob_bytes;
+      const CUtensorMap *maps = in_slot ? a.maps.slot : a.maps.stage;
+      for (int slab = 0; slab < nslab; ++slab) {
+        if (issued >= SR && !mbar_wait_warp(smem_u32(&raw_empty[r]), ph ^ 1u, a.err, 52)) { failed = true; break; }
+        const uint32_t bar = smem_u32(&raw_full[r]);
+        const uint32_t st = smem_u32(smem + Geo::RAW_OFF + (size_t)r * kRawBytes);
+        if (elect_one()) {
           mbar_arrive_expect_tx(bar, (uint32_t)kRawBytes);
           // codes of the slab (TMA boxes of 32 bytes = 64 nibbles, or 64
           // bytes = 64 E4M3), then the scales the decoders need
@@ -353,20 +361,21 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
             bulk_load(st + 8192, blob + a.L.scales[m0] + ((size_t)b0 * ng + slab / 2) * 256, 256, bar);
             bulk_load(st + 8448, blob + a.L.scales[m1] + ((size_t)b1 * ng + slab / 2) * 256, 256, bar);
           }
-          ++issued;
-          if (++r == SR) { r = 0; ph ^= 1u; }
         }
+        __syncwarp();
+        ++issued;
+        if (++r == SR) { r = 0; ph ^= 1u; }
       }
-      {
-        // the last copies issued have landed before the CTA exits: at once on
-        // a normal run (their consumers waited for them), and also when a
-        // consumer gave up waiting
-        int r2 = 0;
-        uint32_t ph2 = 0;
-        for (int i = 0; i < issued; ++i) {
-          if (i >= issued - SR) mbar_drain(smem_u32(&raw_full[r2]), ph2);
-          if (++r2 == SR) { r2 = 0; ph2 ^= 1u; }
-        }
+    }
+    // the last copies issued have landed before the CTA exits: at once on a
+    // normal run (their consumers waited for them), and also when a consumer
+    // gave up waiting
+    if (lane == 0) {
+      int r2 = 0;
+      uint32_t ph2 = 0;
+      for (int i = 0; i < issued; ++i) {
+        if (i >= issued - SR) mbar_drain(smem_u32(&raw_full[r2]), ph2);
+        if (++r2 == SR) { r2 = 0; ph2 ^= 1u; }
       }
     }
   } else if (warp == 1 || warp == 15) {
@@ -540,29 +549,26 @@ __global__ void __launch_bounds__(kDqThreads, 1) expert_dq_kernel(const __grid_c
     uint32_t qph = 0;
     bool failed = false;
     while (!failed) {
-      int okw = 1;
-      if (lane == 0) okw = mbar_wait(smem_u32(&sched_full[q]), qph, a.err, 61) ? 1 : 0;
-      okw = __shfl_sync(0xffffffffu, okw, 0);
-      if (!okw) break;
-      __syncwarp();
-      const int item = sched_item[q];
-      const TileInfo ti = sched_ti[q];
-      const int loc = sched_loc[q];
-      __syncwarp();
+      // the whole warp runs the loop (warp-uniform waits, values broadcast
+      // from lane 0) and one elected lane issues the copies
+      if (!mbar_wait_warp(smem_u32(&sched_full[q]), qph, a.err, 61)) break;
+      const int item = __shfl_sync(0xffffffffu, sched_item[q], 0);
+      const int prow0 = __shfl_sync(0xffffffffu, sched_ti[q].prow0, 0);
+      const int loc = __shfl_sync(0xffffffffu, sched_loc[q], 0);
       if (lane == 0) mbar_arrive(smem_u32(&sched_empty[q]));
       if (++q == kDqSched) { q = 0; qph ^= 1u; }
       if (item < 0) break;
       if (loc == kLocAbsent) continue;
       for (int slab = 0; slab < nslab; ++slab) {
-        int ok = 1;
-        if (lane == 0 && n_slabs >= SO) ok = mbar_wait(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 56) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) { failed = true; break; }
+        if (n_slabs >= SO && !mbar_wait_warp(smem_u32(&op_empty[s]), sph ^ 1u, a.err, 56)) { failed = true; break; }
         const uint32_t bst = smem_u32(smem + (size_t)s * Geo::OP_STAGE);
         const uint32_t bar = smem_u32(&b_full[s]);
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)Geo::B_BYTES);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar, (uint32_t)Geo::B_BYTES);
+#pragma unroll
+          for (int bx = 0; bx < NB / 64; ++bx) tma_load_2d(bst + 8192 * bx, &a.maps.act, bar, slab * 64, prow0 + 64 * bx);
+        }
         __syncwarp();
-        if (lane < NB / 64) tma_load_2d(bst + 8192 * lane, &a.maps.act, bar, slab * 64, ti.prow0 + 64 * lane);
         ++issued;
         ++n_slabs;
         if (++s == SO) { s = 0; sph ^= 1u; }

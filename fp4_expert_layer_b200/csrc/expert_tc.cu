@@ -392,24 +392,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
           // reads them through the async proxy
           asm volatile("fence.proxy.async.global;" ::: "memory");
         }
-        if (lane == 0) {
-          for (int slab = 0; slab < nslab; ++slab) {
-            if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 35)) { failed = true; break; }
-            const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
-            const uint32_t bar = smem_u32(&bfull_bar[s]);
+        // the whole warp runs the slab loop (warp-uniform waits) and one
+        // elected lane issues the copies
+        for (int slab = 0; slab < nslab; ++slab) {
+          if (issued >= S && !mbar_wait_warp(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 35)) { failed = true; break; }
+          const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+          const uint32_t bar = smem_u32(&bfull_bar[s]);
+          if (elect_one()) {
             mbar_arrive_expect_tx(bar, tx);
             for (int b = 0; b < nbox; ++b)
               tma_load_2d(st + Geo::B_OFF + b * 2048, &a.maps.act, bar, slab * 128, act_row0 + 16 * b);
             bulk_load(st + Geo::SF_OFF, sfa + (size_t)slab * kTcSfChunk, kTcSfChunk, bar);
             bulk_load(st + Geo::SF_OFF + kTcSfChunk, sfb + (size_t)slab * 512, 512, bar);
-            ++issued;
-            if (++s == S) { s = 0; ph ^= 1u; }
           }
+          __syncwarp();
+          ++issued;
+          if (++s == S) { s = 0; ph ^= 1u; }
         }
-        failed = __shfl_sync(0xffffffffu, failed ? 1 : 0, 0) != 0;
-        issued = __shfl_sync(0xffffffffu, issued, 0);
-        s = __shfl_sync(0xffffffffu, s, 0);
-        ph = __shfl_sync(0xffffffffu, ph, 0);
       }
       // the last copies issued have landed before the CTA exits (also when a
       // wait gave up)

@@ -148,55 +148,66 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_a4_kernel(const __grid_cons
   const uint32_t tmem = tmem_base_s;
 
   if (warp == 0) {
-    // ---------------- copies (one lane): work items, weight + activation tiles and their scales
-    if (lane == 0) {
-      int s = 0, issued = 0;
-      uint32_t ph = 0;
-      int q = 0;
-      uint32_t qph = 0;
-      bool failed = false;
-      const int m = (MODE == MODE_GATEUP) ? 0 : 2;
-      for (int j = 0; !failed; ++j) {
-        const int item = atomicAdd(a.work_ctr, 1);
-        TileInfo ti{};
-        int loc = kLocAbsent;
-        if (item < n_items) {
-          ti = load_tile_a4(a.tiles + item / ipt);
-          loc = load_loc(a.loc, ti.expert, a.db);
-        }
-        if (j >= kGSched && !mbar_wait(smem_u32(&sched_empty[q]), qph ^ 1u, a.err, 14)) { failed = true; break; }
-        const bool done = item >= n_items;
+    // ---------------- copies: work items, weight + activation tiles and their
+    // scales.  The whole warp runs the loop (warp-uniform waits, values
+    // broadcast from lane 0) and one elected lane issues the copies: a copy
+    // issued from a one-lane loop behind a lane test costs about twice as much.
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    int q = 0;
+    uint32_t qph = 0;
+    bool failed = false;
+    const int m = (MODE == MODE_GATEUP) ? 0 : 2;
+    for (int j = 0; !failed; ++j) {
+      int item = 0;
+      if (lane == 0) item = atomicAdd(a.work_ctr, 1);
+      item = __shfl_sync(0xffffffffu, item, 0);
+      TileInfo ti{};
+      int loc = kLocAbsent;
+      if (item < n_items) {
+        ti = load_tile_a4(a.tiles + item / ipt);
+        loc = load_loc(a.loc, ti.expert, a.db);
+      }
+      if (j >= kGSched && !mbar_wait_warp(smem_u32(&sched_empty[q]), qph ^ 1u, a.err, 14)) { failed = true; break; }
+      const bool done = item >= n_items;
+      if (lane == 0) {
         sched_item[q] = done ? -1 : item;
         sched_ti[q] = ti;
         sched_loc[q] = loc;
         mbar_arrive(smem_u32(&sched_full[q]));
-        if (++q == kGSched) { q = 0; qph ^= 1u; }
-        if (done) break;
-        if (loc == kLocAbsent) continue;
-        const int rb = item % ipt;
-        const bool in_slot = loc >= 0;
-        const int bidx = in_slot ? loc : (-2 - loc);
-        const int region = in_slot ? 0 : 1;
-        const uint8_t *blob = (in_slot ? a.slots : a.staging) + (size_t)bidx * a.blob_bytes;
-        for (int it = 0; it < nk; ++it) {
-          if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 12)) { failed = true; break; }
-          const uint32_t bar = smem_u32(&full_bar[s]);
-          const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
-          // a half stage (last 128 K elements) carries half the scale blocks; the
-          // code tiles are full boxes whose out-of-range half TMA fills with zeros
-          const int sfb = (min(256, K - it * 256) / G) / 4 * 512;
+      }
+      __syncwarp();
+      if (++q == kGSched) { q = 0; qph ^= 1u; }
+      if (done) break;
+      if (loc == kLocAbsent) continue;
+      const int rb = item % ipt;
+      const bool in_slot = loc >= 0;
+      const int bidx = in_slot ? loc : (-2 - loc);
+      const int region = in_slot ? 0 : 1;
+      const uint8_t *blob = (in_slot ? a.slots : a.staging) + (size_t)bidx * a.blob_bytes;
+      for (int it = 0; it < nk; ++it) {
+        if (issued >= S && !mbar_wait_warp(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 12)) { failed = true; break; }
+        const uint32_t bar = smem_u32(&full_bar[s]);
+        const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
+        // a half stage (last 128 K elements) carries half the scale blocks; the
+        // code tiles are full boxes whose out-of-range half TMA fills with zeros
+        const int sfb = (min(256, K - it * 256) / G) / 4 * 512;
+        const int col0 = it * (256 / G);                         // first scale column of this stage
+        if (elect_one()) {
           mbar_arrive_expect_tx(bar, (uint32_t)(2 * kTileBytes + 2 * sfb));
-          const int col0 = it * (256 / G);                         // first scale column of this stage
           tma_load_3d(st, &a.maps.w[region][m], bar, it * 128, rb * 128, bidx);
           bulk_load(st + Geo::SF_OFF, blob + a.L.scales[m] + sf_offset(nsf, rb * 128, col0), (uint32_t)sfb, bar);
           tma_load_2d(st + Geo::B_OFF, &a.maps.act[a.act_map], bar, it * 128, ti.prow0);
           bulk_load(st + Geo::SF_OFF + Geo::SF_BYTES, a.bsf + sf_offset(nsf, ti.prow0, col0), (uint32_t)sfb, bar);
-          ++issued;
-          if (++s == S) { s = 0; ph ^= 1u; }
         }
+        __syncwarp();
+        ++issued;
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
-      // the last copies issued have landed before the CTA exits: at once on a
-      // normal run (the MMA lane waited for them), and also when a wait gave up
+    }
+    // the last copies issued have landed before the CTA exits: at once on a
+    // normal run (the MMA warp waited for them), and also when a wait gave up
+    if (lane == 0) {
       int s2 = 0;
       uint32_t ph2 = 0;
       for (int i = 0; i < issued; ++i) {
