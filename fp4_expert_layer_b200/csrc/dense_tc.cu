@@ -106,26 +106,30 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_tc_kernel(const __grid
   wait_prior_grid();                                   // x / h come from earlier kernels
 
   if (warp == 0) {
-    // ---------------- producer
-    if (lane == 0) {
+    // ---------------- producer: the whole warp runs the loop (warp-uniform
+    // waits) and one elected lane issues the copies
+    {
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool failed = false;
       for (int item = blockIdx.x; item < n_items && !failed; item += gridDim.x) {
         const int tile = item / ipt, rb = item % ipt;
         for (int slab = 0; slab < nslab; ++slab) {
-          if (issued >= S && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 42)) { failed = true; break; }
+          if (issued >= S && !mbar_wait_warp(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 42)) { failed = true; break; }
           const uint32_t bar = smem_u32(&full_bar[s]);
           const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
-          mbar_arrive_expect_tx(bar, (uint32_t)(Geo::A_BYTES + Geo::B_BYTES));
-          if constexpr (MODE == MODE_GATEUP) {
-            tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 128);
-            tma_load_2d(st + 16384, &a.wmap[1], bar, slab * 64, rb * 128);
-          } else {
-            tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 256);
-            tma_load_2d(st + 16384, &a.wmap[0], bar, slab * 64, rb * 256 + 128);
+          if (elect_one()) {
+            mbar_arrive_expect_tx(bar, (uint32_t)(Geo::A_BYTES + Geo::B_BYTES));
+            if constexpr (MODE == MODE_GATEUP) {
+              tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 128);
+              tma_load_2d(st + 16384, &a.wmap[1], bar, slab * 64, rb * 128);
+            } else {
+              tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 256);
+              tma_load_2d(st + 16384, &a.wmap[0], bar, slab * 64, rb * 256 + 128);
+            }
+            tma_load_2d(st + Geo::B_OFF, &a.xmap, bar, slab * 64, tile * NBOX);
           }
-          tma_load_2d(st + Geo::B_OFF, &a.xmap, bar, slab * 64, tile * NBOX);
+          __syncwarp();
           ++issued;
           if (++s == S) { s = 0; ph ^= 1u; }
         }
@@ -342,23 +346,28 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_splitk_kernel(const __
   wait_prior_grid();                                   // x / h come from earlier kernels
 
   if (warp == 0) {
-    if (lane == 0) {
+    // producer: the whole warp runs the loop (warp-uniform waits) and one
+    // elected lane issues the copies
+    {
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool failed = false;
       for (int slab = s0; slab < s1; ++slab) {
-        if (issued >= SN && !mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 46)) { failed = true; break; }
+        if (issued >= SN && !mbar_wait_warp(smem_u32(&empty_bar[s]), ph ^ 1u, a.err, 46)) { failed = true; break; }
         const uint32_t bar = smem_u32(&full_bar[s]);
         const uint32_t st = smem_u32(smem + (size_t)s * Geo::STAGE);
-        mbar_arrive_expect_tx(bar, (uint32_t)(Geo::A_BYTES + Geo::B_BYTES));
-        if constexpr (MODE == MODE_GATEUP) {
-          tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 128);
-          tma_load_2d(st + 16384, &a.wmap[1], bar, slab * 64, rb * 128);
-        } else {
-          tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 256);
-          tma_load_2d(st + 16384, &a.wmap[0], bar, slab * 64, rb * 256 + 128);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar, (uint32_t)(Geo::A_BYTES + Geo::B_BYTES));
+          if constexpr (MODE == MODE_GATEUP) {
+            tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 128);
+            tma_load_2d(st + 16384, &a.wmap[1], bar, slab * 64, rb * 128);
+          } else {
+            tma_load_2d(st, &a.wmap[0], bar, slab * 64, rb * 256);
+            tma_load_2d(st + 16384, &a.wmap[0], bar, slab * 64, rb * 256 + 128);
+          }
+          tma_load_2d(st + Geo::B_OFF, &a.xmap, bar, slab * 64, 0);
         }
-        tma_load_2d(st + Geo::B_OFF, &a.xmap, bar, slab * 64, 0);
+        __syncwarp();
         ++issued;
         if (++s == SN) { s = 0; ph ^= 1u; }
       }
