@@ -304,32 +304,41 @@ __global__ void __launch_bounds__(256, 1) router_gemm_kernel(const uint16_t *__r
   for (int c = 0; c < nck; ++c) {
     const int b = c & 1;
     if (c + 1 < nck) fetch(c + 1);
-    float part[8][JN];
+    // chunk partials as pairs of adjacent experts: one packed fp32 FMA
+    // (two IEEE fmaf, the same per-element sequence) per pair
+    float2 part[8][JN / 2];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < JN; ++j) part[i][j] = 0.0f;
+      for (int j = 0; j < JN / 2; ++j) part[i][j] = make_float2(0.0f, 0.0f);
 #pragma unroll 4
     for (int k = 0; k < kRgK; ++k) {
       const float4 a0 = *reinterpret_cast<const float4 *>(&xs[b][k][ty * 4]);
       const float4 a1 = *reinterpret_cast<const float4 *>(&xs[b][k][64 + ty * 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      float bv[JN];
+      float2 bv[JN / 2];
       const float4 b0 = *reinterpret_cast<const float4 *>(&ws[b][k][tx * 4]);
-      bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w;
+      bv[0] = make_float2(b0.x, b0.y);
+      bv[1] = make_float2(b0.z, b0.w);
       if constexpr (JN == 8) {
         const float4 b1 = *reinterpret_cast<const float4 *>(&ws[b][k][64 + tx * 4]);
-        bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
+        bv[2] = make_float2(b1.x, b1.y);
+        bv[3] = make_float2(b1.z, b1.w);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 8; ++i) {
+        const float2 ai = make_float2(av[i], av[i]);
 #pragma unroll
-        for (int j = 0; j < JN; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
+        for (int j = 0; j < JN / 2; ++j) part[i][j] = __ffma2_rn(ai, bv[j], part[i][j]);
+      }
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < JN; ++j) acc[i][j] += part[i][j];
+      for (int j = 0; j < JN / 2; ++j) {
+        acc[i][2 * j] += part[i][j].x;
+        acc[i][2 * j + 1] += part[i][j].y;
+      }
     if (c + 1 < nck) stash(b ^ 1);
     __syncthreads();
   }
