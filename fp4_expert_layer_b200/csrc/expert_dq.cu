@@ -31,7 +31,7 @@
 //   warp 0       producer: per 64-element K slab, one TMA box of the packed
 //                codes (32 bytes x 128 or 256 rows) per matrix and the
 //                512-byte E4M3 scale-factor blocks by bulk copy, into a ring
-//                of raw stages;
+//                of raw stages (whole warp, one elected lane issuing);
 //   warps 1, 15  MMA issuers (whole warps, one elected lane issuing; one
 //                accumulator each: gate and up, or the two 128-row halves of
 //                down): M = 128, N = tokens rounded up to 16, K = 16, A from
@@ -49,7 +49,7 @@
 //   warp 14      activation loader: the tile's 16-bit rows of this K slab
 //                (x rows gathered into the padded expert order beforehand,
 //                or h) by TMA in 64-row boxes, 128-byte swizzled K-major as
-//                the B descriptor reads them.
+//                the B descriptor reads them (whole warp, one elected lane).
 // TMEM: accumulators (2 x NB columns per buffer; two buffers when NB = 64),
 // then 4 A stages of 64 columns (32 per 128-row half: 64 bf16 of a row).
 // Every mbarrier wait is bounded (error word, then the kernel runs out).

@@ -29,8 +29,9 @@
 //    a producer warp streams 128x128 weight tiles (TMA unpacks the E2M1 codes
 //    to one byte per element), the matching 128-element slab of the tile's
 //    activation pieces and both scale-factor blocks into a ring of stages;
-//    one thread issues the MMAs (M = 128, N = 2 x tokens, K = 32 each) into
-//    TMEM; four warps read the accumulators back.  Gate/up stages alternate
+//    two warps issue the MMAs (M = 128, N = 2 x tokens, K = 32 each) into
+//    their own TMEM accumulator, one elected lane each; four warps read the
+//    accumulators back.  Gate/up stages alternate
 //    gate and up tiles of the same K slab (two accumulators) and the epilogue
 //    computes SwiGLU and the pieces of h; down scales by the gate and writes
 //    O' (the ordered combine into y is a separate kernel).
@@ -47,11 +48,13 @@ namespace moe {
 
 namespace {
 
-// warp 0: weight TMA; warp 1: TMEM allocation and MMA issue (first
-// accumulator); warps 2..5: epilogue; warp 6: activation pieces (16-row TMA
-// boxes) and scale factors (bulk copies), one lane; warp 7: MMA issue (second
-// accumulator); a per-lane cp.async copy of the pieces cost about
-// a thousand cycles of issue per slab at prefill tile sizes
+// warp 0: weight TMA (one lane: one 16 KB box per stage); warp 1: TMEM
+// allocation and MMA issue (first accumulator); warps 2..5: epilogue; warp 6:
+// activation pieces (16-row TMA boxes) and scale factors (bulk copies); warp
+// 7: MMA issue (second accumulator).  The MMA and piece-copy loops run on
+// whole warps with one elected lane issuing (from a one-lane loop behind a
+// lane test each issue cost about twice as much); a per-lane cp.async copy of
+// the pieces cost about a thousand cycles of issue per slab at prefill sizes
 constexpr int kTcThreads = 256;
 constexpr int kSched = 8;         // work items handed from the producer to the other roles in flight
 constexpr int kSchedReaders = 7;  // arrivals that free a hand-over slot: 2 MMA lanes, the loader warp, 4 epilogue warps
@@ -350,7 +353,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) expert_tc_kernel(const __grid_c
     __syncwarp();
     mbar_drain(smem_u32(&quiesce_bar), 0);
   } else if (warp == 6) {
-    // ---------------- loader (warp 6, one lane): per K slab, the tile's
+    // ---------------- loader (warp 6): per K slab, the tile's
     // activation-piece rows by TMA (16-row boxes, 128-byte swizzle as the MMA
     // descriptor reads them) and the three scale-factor blocks (the weight
     // chunk's two halves, the activation rows) by bulk copy

@@ -20,8 +20,9 @@
 // TMEM, so an item's epilogue overlaps the next item's main loop.
 //
 // Persistent, one CTA per SM, work items taken from a counter in index order.
-// Warp roles: warp 0 takes the items and issues the copies (one lane), warp 1
-// allocates TMEM and one lane issues every MMA, warps 2..9 read the
+// Warp roles: warp 0 takes the items and issues the copies, warp 1 allocates
+// TMEM and issues every MMA (both whole warps with one elected lane issuing),
+// warps 2..9 read the
 // accumulators back with tcgen05.ld (warp w the lanes of quadrant w % 4; warps
 // 2..5 tokens 0..63 of an item, warps 6..9 tokens 64..127).  All mbarrier
 // waits are bounded.
