@@ -233,6 +233,35 @@ def cpu_baseline(lw, x_bits, budget_s, numerics="exact"):
             "sample": f"{what} ({n} tokens, {el:.1f} s, {numerics} numerics)"}
 
 
+def gpu_local_cpus(torch, dev_index, nvml=None):
+    """The host CPUs NVML reports as local to this process's GPU (its NUMA
+    node), intersected with the CPUs the process may run on; None when NVML
+    cannot tell.  With one replica per GPU, each rank's pinned expert store
+    and staging copies then sit on the socket its GPU hangs off."""
+    try:
+        if nvml is None:
+            import pynvml as nvml
+        nvml.nvmlInit()
+        h = None
+        props = torch.cuda.get_device_properties(dev_index) if torch is not None else None
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            devn = getattr(props, "pci_device_id", 0)
+            try:
+                h = nvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{devn:02x}.0")
+            except Exception:
+                h = None
+        if h is None:
+            h = nvml.nvmlDeviceGetHandleByIndex(dev_index)
+        words = nvml.nvmlDeviceGetCpuAffinity(h, ((os.cpu_count() or 64) + 63) // 64)
+        cpus = {64 * w + b for w, m in enumerate(words) for b in range(64) if (int(m) >> b) & 1}
+    except Exception:
+        return None
+    local = cpus & os.sched_getaffinity(0)
+    return local or None
+
+
 def max_over_ranks(vals, world):
     """Element-wise maximum of this rank's timings over all ranks, returned on
     every rank: the job is as slow as its slowest replica."""
@@ -451,6 +480,13 @@ def main():
         fbuild.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    host_binding = "unchanged"
+    if world > 1:
+        # replicas: keep each rank's host memory and copy threads on its GPU's socket
+        cpus = gpu_local_cpus(torch, local)
+        if cpus:
+            os.sched_setaffinity(0, cpus)
+            host_binding = f"gpu-local cpus ({len(cpus)})"
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
@@ -603,6 +639,7 @@ def main():
                        "n_experts": wl.n_experts, "top_k": wl.top_k, "fmt": wl.fmt,
                        "shared_inter": wl.shared_inter, "resident_slots": S, "numerics": args.numerics,
                        "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before every step",
+                       "host_binding": host_binding,
                        "active_experts": n_active},
             "roofline": roof,
             "layer_roofline": {"bytes_per_step": layer_bytes(wl, n_active, T),

@@ -101,3 +101,40 @@ def test_default_workload_is_the_largest_single_gpu_layer():
     assert a.slots == "workload" and a.numerics == "exact" and a.warmup >= 3
     sizes = {n: w.n_experts * w.expert_bytes() for n, w in synth.WORKLOADS.items()}
     assert max(sizes, key=sizes.get) == a.workload
+
+
+class _FakeNvml:
+    """Stands in for pynvml: two 64-bit affinity words for the GPU."""
+
+    def __init__(self, words, fail=False):
+        self.words, self.fail = words, fail
+
+    def nvmlInit(self):
+        if self.fail:
+            raise RuntimeError("no driver")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("index", i)
+
+    def nvmlDeviceGetCpuAffinity(self, h, n):
+        return self.words[:n] + [0] * max(0, n - len(self.words))
+
+
+def test_gpu_local_cpus_intersects_nvml_affinity_with_allowed_cpus():
+    allowed = os.sched_getaffinity(0)
+    # every allowed CPU below 128 marked local, plus one that is not allowed
+    words = [0, 0]
+    for c in allowed:
+        if c < 128:
+            words[c // 64] |= 1 << (c % 64)
+    extra = next((c for c in range(128) if c not in allowed), None)
+    if extra is not None:
+        words[extra // 64] |= 1 << (extra % 64)
+    got = bench.gpu_local_cpus(None, 0, nvml=_FakeNvml(words))
+    want = {c for c in allowed if c < 128}
+    assert got == (want or None)
+
+
+def test_gpu_local_cpus_gives_none_without_nvml_or_overlap():
+    assert bench.gpu_local_cpus(None, 0, nvml=_FakeNvml([0, 0], fail=True)) is None
+    assert bench.gpu_local_cpus(None, 0, nvml=_FakeNvml([0, 0])) is None
