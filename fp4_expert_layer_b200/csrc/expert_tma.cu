@@ -23,6 +23,7 @@
 #include "checks.cuh"
 #include "device_utils.cuh"
 #include "moe_internal.h"
+#include "tcgen05.cuh"
 #include "tma.cuh"
 
 namespace cg = cooperative_groups;
@@ -111,37 +112,42 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) expert_tma_kernel(c
   int mrow[2][2] = {{0, 0}, {0, 0}};        // matrix row of (m-tile j, half i)
 
   if (warp == kConsumers) {
-    // ================= producer: one lane issues every copy
-    if (lane == 0) {
+    // ================= producer: the whole warp runs the loop (warp-uniform
+    // waits) and one elected lane issues the copies
+    {
       const int nsf = K / 16;
       int issued = 0;
       for (int it = 0; it < n_iter; ++it) {
         const int s = it % kStages;
-        if (it >= kStages && !mbar_wait(smem_u32(&empty_bar[s]), ((it / kStages) - 1) & 1, a.err, 2)) break;
+        if (it >= kStages && !mbar_wait_warp(smem_u32(&empty_bar[s]), ((it / kStages) - 1) & 1, a.err, 2)) break;
         issued = it + 1;
         const int c = c_begin + it;
         const uint32_t bar = smem_u32(&full_bar[s]);
         const uint32_t dst = smem_u32(smem + (size_t)s * Geo::kStageBytes);
-        mbar_arrive_expect_tx(bar, Geo::kStageBytes);
-        // scale columns covered by this chunk: 8 (two 512-byte blocks)
-        const int col0 = 8 * c;
-        if constexpr (MODE == MODE_GATEUP) {
-          tma_load_3d(dst, &maps[0], bar, c * 64, rb * 128, bidx);
-          tma_load_3d(dst + 8192, &maps[1], bar, c * 64, rb * 128, bidx);
-          for (int j = 0; j < 2; ++j)
-            bulk_load(dst + kABytes + j * Geo::kSfPerGroup, blob + a.L.scales[j] + sf_offset(nsf, rb * 128, col0),
-                      Geo::kSfPerGroup, bar);
-        } else {
-          tma_load_3d(dst, &maps[2], bar, c * 64, rb * 256, bidx);
-          for (int j = 0; j < 2; ++j)
-            bulk_load(dst + kABytes + j * Geo::kSfPerGroup,
-                      blob + a.L.scales[2] + sf_offset(nsf, rb * 256 + 128 * j, col0), Geo::kSfPerGroup, bar);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar, Geo::kStageBytes);
+          // scale columns covered by this chunk: 8 (two 512-byte blocks)
+          const int col0 = 8 * c;
+          if constexpr (MODE == MODE_GATEUP) {
+            tma_load_3d(dst, &maps[0], bar, c * 64, rb * 128, bidx);
+            tma_load_3d(dst + 8192, &maps[1], bar, c * 64, rb * 128, bidx);
+            for (int j = 0; j < 2; ++j)
+              bulk_load(dst + kABytes + j * Geo::kSfPerGroup, blob + a.L.scales[j] + sf_offset(nsf, rb * 128, col0),
+                        Geo::kSfPerGroup, bar);
+          } else {
+            tma_load_3d(dst, &maps[2], bar, c * 64, rb * 256, bidx);
+            for (int j = 0; j < 2; ++j)
+              bulk_load(dst + kABytes + j * Geo::kSfPerGroup,
+                        blob + a.L.scales[2] + sf_offset(nsf, rb * 256 + 128 * j, col0), Geo::kSfPerGroup, bar);
+          }
         }
+        __syncwarp();
       }
       // the last copies issued have landed before the CTA exits: at once on a
       // normal run (the consumers waited for them), and also when a wait gave up
-      for (int i = max(0, issued - kStages); i < issued; ++i)
-        mbar_drain(smem_u32(&full_bar[i % kStages]), (i / kStages) & 1);
+      if (lane == 0)
+        for (int i = max(0, issued - kStages); i < issued; ++i)
+          mbar_drain(smem_u32(&full_bar[i % kStages]), (i / kStages) & 1);
     }
   } else {
     // ================= consumers
