@@ -165,8 +165,8 @@ typedef struct {
   int32_t last_path;       /* 0 = register-decode kernels (EXACT), 1 = A4      */
                            /* tcgen05 FP4 x FP4, 2 = EXACT on tcgen05 (MXFP4    */
                            /* weights x E4M3 activation pieces), 3 = EXACT on   */
-                           /* tcgen05 (NVFP4 weights decoded to bf16 in shared  */
-                           /* memory x bf16 activations)                        */
+                           /* tcgen05 (NVFP4 / INT4 / FP8 weights decoded into  */
+                           /* TMEM x 16-bit activations)                        */
   uint64_t launches;       /* kernels this library launched, cumulative         */
   uint64_t expert_bytes;   /* device-layout bytes of one routed expert          */
   uint64_t device_bytes;   /* HBM held by the layer                             */
