@@ -28,30 +28,36 @@ template <int KPER>
 __device__ __forceinline__ void topk_warp(const float (&lv)[KPER], int E, int k, int *ids, float *gates,
                                           int *ids_s, int scoring = 0, int renorm = 1) {
   const int lane = threadIdx.x & 31;
-  uint32_t taken = 0;   // bit i: lane's i-th expert already chosen
   float lmax = 0.0f, den = 0.0f;
   float my_l = 0.0f;    // lane j keeps the logit of choice j
   int my_id = 0;
+  // Each logit as an order-preserving 32-bit key (-0 taken as +0, so that
+  // equal values tie as they compare), 0 for targets that are out of range or
+  // taken: a round is one warp max of the keys and one warp min of the
+  // indices that hold it (the lower index wins a tie).
+  uint32_t key[KPER];
+#pragma unroll
+  for (int i = 0; i < KPER; ++i) {
+    const float v = lv[i] == 0.0f ? 0.0f : lv[i];
+    const uint32_t b = __float_as_uint(v);
+    key[i] = (lane + 32 * i < E) ? ((b & 0x80000000u) ? ~b : (b | 0x80000000u)) : 0u;
+  }
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+    uint32_t kb = 0u;
 #pragma unroll
-    for (int i = 0; i < KPER; ++i) {
-      const int ee = lane + 32 * i;
-      if (ee < E && !((taken >> i) & 1u)) {
-        if (bi == 0x7fffffff || lv[i] > bv) { bv = lv[i]; bi = ee; }
-      }
-    }
+    for (int i = 0; i < KPER; ++i) kb = max(kb, key[i]);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, kb);
+    uint32_t ib = 0xffffffffu;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-        bv = ov;
-        bi = oi;
-      }
+    for (int i = 0; i < KPER; ++i)
+      if (key[i] == kmax && ib == 0xffffffffu) ib = (uint32_t)(lane + 32 * i);
+    const int bi = (int)__reduce_min_sync(0xffffffffu, ib);
+    const float bv = __uint_as_float((kmax & 0x80000000u) ? (kmax & 0x7fffffffu) : ~kmax);   // the winning logit
+    if ((bi & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < KPER; ++i)
+        if (i == (bi >> 5)) key[i] = 0u;                 // taken
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     if (j == 0) lmax = bv;
     if (lane == j) { my_l = bv; my_id = bi; }
   }
