@@ -143,14 +143,19 @@ __global__ void __launch_bounds__(256) router_kernel(const RouterArgs a) {
   }
   if (!a.fuse_perm) return;
 
-  // the last token tile to finish top-k runs the permutation
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) is_last = (atomicAdd(a.tiles_done, 1) == (int)gridDim.x - 1);
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  if (threadIdx.x == 0) *a.tiles_done = 0;
+  // the last token tile to finish top-k runs the permutation (with a single
+  // token tile this CTA wrote every id itself: a block barrier suffices)
+  if (gridDim.x > 1) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = (atomicAdd(a.tiles_done, 1) == (int)gridDim.x - 1);
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (threadIdx.x == 0) *a.tiles_done = 0;
+  } else {
+    __syncthreads();
+  }
   permute_block<256, true>(a.perm, a.perm.ids, reinterpret_cast<int *>(xs_smem));
 }
 
