@@ -93,6 +93,11 @@ struct moe_layer {
   int n_staging = 0;
   cudaStream_t side = nullptr;
   cudaEvent_t ev_copied[2] = {}, ev_done[2] = {}, ev_counts = nullptr, ev_fwd_done = nullptr;
+  // decode-sized batches run the shared expert on its own stream, forked
+  // before the router and joined before the first kernel that reads its output
+  cudaStream_t sh_stream = nullptr;
+  cudaEvent_t ev_sh_fork = nullptr, ev_sh_join = nullptr;
+  bool sh_join_pending = false;
   // device memory
   std::vector<void *> dev;
   float *router_w = nullptr, *router_b = nullptr;
@@ -371,7 +376,10 @@ static void free_layer(moe_layer *L) {
   if (L->ev_prefetch) cudaEventDestroy(L->ev_prefetch);
   for (auto &p : L->pend) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
   for (auto e : L->evpool) cudaEventDestroy(e);
+  if (L->ev_sh_fork) cudaEventDestroy(L->ev_sh_fork);
+  if (L->ev_sh_join) cudaEventDestroy(L->ev_sh_join);
   if (L->side) cudaStreamDestroy(L->side);
+  if (L->sh_stream) cudaStreamDestroy(L->sh_stream);
   delete L;
 }
 
@@ -975,6 +983,11 @@ moe_status_t moe_layer_create(const moe_config_t *cfg, const moe_weights_t *w, v
   C_CUDA(cudaStreamSynchronize(s));
 
   C_CUDA(cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking));
+  if (Is) {
+    C_CUDA(cudaStreamCreateWithFlags(&L->sh_stream, cudaStreamNonBlocking));
+    C_CUDA(cudaEventCreateWithFlags(&L->ev_sh_fork, cudaEventDisableTiming));
+    C_CUDA(cudaEventCreateWithFlags(&L->ev_sh_join, cudaEventDisableTiming));
+  }
   for (int i = 0; i < 2; ++i) {
     C_CUDA(cudaEventCreateWithFlags(&L->ev_copied[i], cudaEventDisableTiming));
     C_CUDA(cudaEventCreateWithFlags(&L->ev_done[i], cudaEventDisableTiming));
@@ -1061,6 +1074,15 @@ static int pick_split(int est_ctas, int nck) {
   return cs;
 }
 
+// The stream waits for the shared expert forked onto its own stream (once per
+// forward, before the first kernel that reads the shared expert's output).
+static moe_status_t join_shared(moe_layer *L, cudaStream_t s) {
+  if (!L->sh_join_pending) return MOE_OK;
+  L->sh_join_pending = false;
+  CUDA_TRY(cudaStreamWaitEvent(s, L->ev_sh_join, 0));
+  return MOE_OK;
+}
+
 static moe_status_t run_experts(moe_layer *L, const int *locs, int nt, int grid_tiles, int cs_gu, int cs_dn,
                                 float *y, cudaStream_t s) {
   const moe_config_t &c = L->cfg;
@@ -1105,6 +1127,8 @@ static moe_status_t run_experts(moe_layer *L, const int *locs, int nt, int grid_
   a.act = L->hbuf;
   a.act_scale = L->hscale;
   a.o_out = L->oprime;
+  // the down pass adds the shared expert's output when it runs the combine
+  if (y) ST_TRY(join_shared(L, s));
   StageTimer t4(L, 4, s);
   launch_expert_tma(L->wf, MODE_DOWN, nt, a, grid_tiles, s);
   CUDA_TRY(cudaGetLastError());
@@ -1357,6 +1381,12 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   float *y_fused = sep_combine ? nullptr : static_cast<float *>(y);
 
   StageTimer t7(L, 7, s);
+  // decode-sized batches: the shared expert reads only x, so it runs on its
+  // own stream beside the routing and the routed passes (its split-K clusters
+  // and the routed kernels are each too short to keep HBM busy alone)
+  const bool sh_fork = Is && T <= 128;
+  L->sh_join_pending = false;
+  if (sh_fork) CUDA_TRY(cudaEventRecord(L->ev_sh_fork, s));
   RouterArgs ra{};
   ra.x = reinterpret_cast<const uint16_t *>(x);
   ra.T = T; ra.H = H; ra.E = NR; ra.k = k;
@@ -1437,10 +1467,12 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   // 128 tokens.  Its operands are read by TMA, which needs x 16-byte aligned:
   // an unaligned x is first copied to the layer's own buffer.
   if (Is) {
-    StageTimer t2(L, 2, s);
+    const cudaStream_t ss = sh_fork ? L->sh_stream : s;
+    if (sh_fork) CUDA_TRY(cudaStreamWaitEvent(ss, L->ev_sh_fork, 0));
+    StageTimer t2(L, 2, ss);
     const void *xs = x;
     if (!x16) {
-      CUDA_TRY(cudaMemcpyAsync(L->xin, x, (size_t)T * H * 2, cudaMemcpyDeviceToDevice, s));
+      CUDA_TRY(cudaMemcpyAsync(L->xin, x, (size_t)T * H * 2, cudaMemcpyDeviceToDevice, ss));
       xs = L->xin;
     }
     DenseTcArgs d{};
@@ -1453,12 +1485,12 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     if (T <= 128) {
       const int np = dense_splitk_rows(T);
       ST_TRY(make_bf16_map(&d.xmap, xs, H, T, np));
-      launch_dense_splitk(MODE_GATEUP, d, s);
+      launch_dense_splitk(MODE_GATEUP, d, ss);
       CUDA_TRY(cudaGetLastError());
       d.wmap[0] = L->sh_map[2];
       ST_TRY(make_bf16_map(&d.xmap, L->sh_h, Is, T, np));
       d.K = Is; d.rows = H; d.n_rowblocks = H / 256;
-      launch_dense_splitk(MODE_DOWN, d, s);
+      launch_dense_splitk(MODE_DOWN, d, ss);
       CUDA_TRY(cudaGetLastError());
     } else {
       ST_TRY(make_bf16_map(&d.xmap, xs, H, T));
@@ -1474,6 +1506,10 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     }
     t2.launched(2);
     t2.end();
+    if (sh_fork) {
+      CUDA_TRY(cudaEventRecord(L->ev_sh_join, ss));
+      L->sh_join_pending = true;
+    }
   }
 
   if (a4) {
@@ -1641,12 +1677,16 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     ca.sg_logits = c.shared_gate ? L->logits : nullptr;
     ca.ld = NR;
     ca.sg_col = NT;
+    ST_TRY(join_shared(L, s));
     StageTimer t5(L, 5, s);
     launch_combine(ca, s);
     CUDA_TRY(cudaGetLastError());
     t5.launched(1);
     t5.end();
   }
+  // every path has read the shared output by now; a forward whose passes all
+  // fused the combine without one still ends behind the shared stream
+  ST_TRY(join_shared(L, s));
   if (admit_table_pending) ST_TRY(push_table(L, s));
   t7.end();
   if (L->prof) L->prof_acc.forwards += 1;
