@@ -33,7 +33,11 @@
  *  - Nothing throws across this ABI.  Every call returns a moe_status_t; on
  *    failure moe_last_error() returns a thread-local description.
  *  - "stream" is a cudaStream_t passed as void* (NULL = the legacy default
- *    stream).  All device work of a call is ordered on that stream.
+ *    stream).  All device work of a call is ordered on that stream: work the
+ *    layer runs on a stream of its own (staging copies, the shared expert of
+ *    a decode-sized forward) starts after the work queued on `stream` before
+ *    the call and is joined back into `stream` before the call returns, so
+ *    work queued on `stream` after the call follows all of it.
  *  - Device pointers are CUDA device memory of the layer's device; host
  *    pointers are ordinary (pageable or pinned) host memory.
  */
@@ -260,7 +264,10 @@ moe_status_t moe_prefetch(moe_layer_t layer, const int32_t *experts, int32_t n, 
  * work on `stream` and returns.  Otherwise it waits for the routing counts
  * (one small device-to-host copy), then copies the missing experts from the
  * pinned store on the layer's side stream, overlapped with compute in waves
- * of at most n_staging experts; it returns once all work is enqueued.
+ * of at most n_staging experts; it returns once all work is enqueued.  With
+ * T <= 128 a layer with a shared expert runs it on a stream of the layer's
+ * own, forked from `stream` before the router and joined back before the
+ * first kernel that reads its output.
  * dbg (may be NULL) receives the routing tensors of this forward. */
 moe_status_t moe_forward(moe_layer_t layer, const void *x, int32_t T, void *y, void *stream,
                          const moe_routing_t *dbg);
@@ -290,7 +297,9 @@ moe_status_t moe_graph_destroy(moe_graph_t graph);
 moe_status_t moe_get_stats(moe_layer_t layer, moe_stats_t *out);
 
 /* Per-stage device timing (tracing).  While enabled, every forward records a
- * CUDA event pair around each stage on the forward's stream; moe_profile_read
+ * CUDA event pair around each stage on the stream the stage runs on (the
+ * forward's stream, or the layer's own for a forked shared expert, whose
+ * time then overlaps the other stages); moe_profile_read
  * waits for those events and returns the accumulated milliseconds and launch
  * counts since the last enable.  Stages: 0 router + top-k, 1 permutation,
  * 2 shared expert, 3 routed gate/up + SwiGLU, 4 routed down + gate scale,
