@@ -1400,6 +1400,18 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   const bool sh_fork = Is && T <= 128;
   L->sh_join_pending = false;
   if (sh_fork) CUDA_TRY(cudaEventRecord(L->ev_sh_fork, s));
+  // every return from here on, an error return included, leaves `s` ordered
+  // after the work this forward queued on the shared expert's stream
+  struct SharedJoinGuard {
+    moe_layer *L;
+    cudaStream_t s;
+    ~SharedJoinGuard() {
+      if (!L->sh_join_pending) return;
+      L->sh_join_pending = false;
+      cudaEventRecord(L->ev_sh_join, L->sh_stream);
+      cudaStreamWaitEvent(s, L->ev_sh_join, 0);
+    }
+  } sh_guard{L, s};
   RouterArgs ra{};
   ra.x = reinterpret_cast<const uint16_t *>(x);
   ra.T = T; ra.H = H; ra.E = NR; ra.k = k;
@@ -1481,7 +1493,10 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
   // an unaligned x is first copied to the layer's own buffer.
   if (Is) {
     const cudaStream_t ss = sh_fork ? L->sh_stream : s;
-    if (sh_fork) CUDA_TRY(cudaStreamWaitEvent(ss, L->ev_sh_fork, 0));
+    if (sh_fork) {
+      CUDA_TRY(cudaStreamWaitEvent(ss, L->ev_sh_fork, 0));
+      L->sh_join_pending = true;
+    }
     StageTimer t2(L, 2, ss);
     const void *xs = x;
     if (!x16) {
@@ -1519,10 +1534,7 @@ moe_status_t moe_forward(moe_layer_t L, const void *x, int32_t T, void *y, void 
     }
     t2.launched(2);
     t2.end();
-    if (sh_fork) {
-      CUDA_TRY(cudaEventRecord(L->ev_sh_join, ss));
-      L->sh_join_pending = true;
-    }
+    if (sh_fork) CUDA_TRY(cudaEventRecord(L->ev_sh_join, ss));
   }
 
   if (a4) {
